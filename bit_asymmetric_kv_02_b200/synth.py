@@ -1,0 +1,138 @@
+"""Seeded synthetic KV-cache workloads (inputs only: no quantization or attention arithmetic).
+
+Every array is drawn per (batch, head[, step]) from its own numpy PCG64 stream keyed by
+(seed, stream id, indices), so any subset of heads can be regenerated on its own and a prefix of a
+prompt equals the shorter prompt.  Distributions follow the KV-cache statistics the KIVI explainer
+page describes (section KVキャッシュの分布特性): keys have a few outlier channels with large
+magnitude across all tokens, values have a large early "sink" token.
+
+  K: N(0,1) fp32, 4 outlier channels per (batch, KV head) (drawn without replacement) scaled x10,
+     cast to fp16 (round to nearest even).
+  V: N(0,1) fp32, token 0 of every sequence scaled x5, cast to fp16.
+  q: N(0,1) fp32 per (batch, query head, step), cast to fp16.
+  new decode tokens: K with the head's outlier channels x10, V plain N(0,1).
+"""
+from __future__ import annotations
+
+import os
+from concurrent.futures import ThreadPoolExecutor
+from dataclasses import dataclass, replace
+
+import numpy as np
+
+STREAM_K, STREAM_V, STREAM_OUTLIER, STREAM_Q, STREAM_KNEW, STREAM_VNEW = range(6)
+N_OUTLIER_CHANNELS = 4
+OUTLIER_GAIN = 10.0
+SINK_GAIN = 5.0
+
+
+@dataclass(frozen=True)
+class Workload:
+    """Shape of one decode workload.  T = cached tokens per head at the attention step."""
+    name: str
+    batch: int
+    q_heads: int
+    kv_heads: int
+    tokens: int
+    head_dim: int = 128
+    bits: int = 2
+    group: int = 32          # G_k = G_v
+    residual: int = 128      # R
+    seed: int = 1000
+    steps: int = 0           # streaming decode steps after the prefill (0: single attention)
+
+    @property
+    def gqa(self) -> int:
+        return self.q_heads // self.kv_heads
+
+    def with_(self, **kw) -> "Workload":
+        return replace(self, **kw)
+
+
+# The five workloads, named by what they are.
+TINY = Workload("tiny_b1_h4_t1024", 1, 4, 4, 1024, seed=1000)
+LLAMA2_7B = Workload("llama2_7b_layer_b8_h32_t4096", 8, 32, 32, 4096, seed=1001)
+LARGE_BATCH = Workload("large_batch_b64_h32_t8192", 64, 32, 32, 8192, seed=1002)
+GQA_LLAMA3_8B = Workload("gqa_llama31_8b_b16_hq32_hkv8_t32768", 16, 32, 8, 32768, seed=1003)
+STREAMING = Workload("streaming_b4_h32_prefill32768_steps256", 4, 32, 32, 32768, seed=1004, steps=256)
+WORKLOADS = {w.name: w for w in (TINY, LLAMA2_7B, LARGE_BATCH, GQA_LLAMA3_8B, STREAMING)}
+
+
+def _rng(seed: int, *key: int) -> np.random.Generator:
+    return np.random.Generator(np.random.PCG64(np.random.SeedSequence([seed, *key])))
+
+
+def outlier_channels(w: Workload, b: int, h: int) -> np.ndarray:
+    """The N_OUTLIER_CHANNELS distinct outlier channels of KV head (b, h)."""
+    return np.sort(_rng(w.seed, STREAM_OUTLIER, b, h).choice(w.head_dim, N_OUTLIER_CHANNELS,
+                                                             replace=False))
+
+
+def prompt_k(w: Workload, b: int, h: int, n: int) -> np.ndarray:
+    """fp16 [n][d] prompt keys of KV head (b, h)."""
+    x = _rng(w.seed, STREAM_K, b, h).standard_normal((n, w.head_dim), dtype=np.float32)
+    x[:, outlier_channels(w, b, h)] *= np.float32(OUTLIER_GAIN)
+    return x.astype(np.float16)
+
+
+def prompt_v(w: Workload, b: int, h: int, n: int) -> np.ndarray:
+    """fp16 [n][d] prompt values of KV head (b, h); token 0 is the x5 sink."""
+    x = _rng(w.seed, STREAM_V, b, h).standard_normal((n, w.head_dim), dtype=np.float32)
+    if n > 0:
+        x[0] *= np.float32(SINK_GAIN)
+    return x.astype(np.float16)
+
+
+def query(w: Workload, b: int, hq: int, step: int = 0) -> np.ndarray:
+    """fp16 [d] query of query head (b, hq) at decode step `step`."""
+    return _rng(w.seed, STREAM_Q, b, hq, step).standard_normal(w.head_dim, dtype=np.float32) \
+        .astype(np.float16)
+
+
+def new_k(w: Workload, b: int, h: int, step: int) -> np.ndarray:
+    """fp16 [d] key appended to KV head (b, h) at decode step `step` (outlier channels x10)."""
+    x = _rng(w.seed, STREAM_KNEW, b, h, step).standard_normal(w.head_dim, dtype=np.float32)
+    x[outlier_channels(w, b, h)] *= np.float32(OUTLIER_GAIN)
+    return x.astype(np.float16)
+
+
+def new_v(w: Workload, b: int, h: int, step: int) -> np.ndarray:
+    """fp16 [d] value appended to KV head (b, h) at decode step `step`."""
+    return _rng(w.seed, STREAM_VNEW, b, h, step).standard_normal(w.head_dim, dtype=np.float32) \
+        .astype(np.float16)
+
+
+def _threads() -> int:
+    return max(1, min(32, os.cpu_count() or 1))
+
+
+def prompt_kv(w: Workload, n: int, out_k: np.ndarray | None = None,
+              out_v: np.ndarray | None = None):
+    """fp16 [B][H][n][d] prompt keys and values of every KV head (threads over heads)."""
+    shape = (w.batch, w.kv_heads, n, w.head_dim)
+    k = np.empty(shape, np.float16) if out_k is None else out_k
+    v = np.empty(shape, np.float16) if out_v is None else out_v
+
+    def one(bh):
+        b, h = divmod(bh, w.kv_heads)
+        k[b, h] = prompt_k(w, b, h, n)
+        v[b, h] = prompt_v(w, b, h, n)
+
+    with ThreadPoolExecutor(_threads()) as ex:
+        list(ex.map(one, range(w.batch * w.kv_heads)))
+    return k, v
+
+
+def queries(w: Workload, step: int = 0) -> np.ndarray:
+    """fp16 [B][Hq][d] queries of one decode step."""
+    return np.stack([np.stack([query(w, b, hq, step) for hq in range(w.q_heads)])
+                     for b in range(w.batch)])
+
+
+def new_kv(w: Workload, step: int):
+    """fp16 [B][H][d] key and value appended at one decode step."""
+    k = np.stack([np.stack([new_k(w, b, h, step) for h in range(w.kv_heads)])
+                  for b in range(w.batch)])
+    v = np.stack([np.stack([new_v(w, b, h, step) for h in range(w.kv_heads)])
+                  for b in range(w.batch)])
+    return k, v

@@ -1,0 +1,172 @@
+/*
+ * kivi.h - C ABI of the B200 (sm_100a) KIVI-style asymmetric low-bit KV-cache library.
+ *
+ * Method source: the KIVI explainer page "ICML 2024論文解説: KIVI — チューニング不要のKVキャッシュ2bit
+ * 非対称量子化" (arXiv 2402.02750). Section and equation names below refer to that page.
+ *
+ *   Q(X) = clamp(round((X - z) / s), 0, 2^b - 1)         section 量子化アルゴリズム, Q equation
+ *   D(X^) = s * X^ + z                                   section 量子化アルゴリズム, D equation
+ *   s = (max X_g - min X_g) / (2^b - 1),  z = min X_g    section 量子化アルゴリズム, s/z equation
+ *   K: groups of g_k consecutive channels                section Per-Channel量子化（Key Cache）
+ *   V: groups of g_v consecutive tokens                  section Per-Token量子化（Value Cache）
+ *   newest tokens stay fp16 in a residual buffer;        section 残差バッファ（Residual Buffer）,
+ *   attention = softmax(q [D(Kq); Kres]^T / sqrt(d)) [D(Vq); Vres]   Attention equation
+ *
+ * Readings this library fixes where the page leaves a step open:
+ *   - A K group is one R-token block x g_k consecutive channels (every R-token block gets its own
+ *     scale/zero per channel group); a V group is g_v consecutive tokens x all d channels.
+ *   - s is stored as fp16, rounded to nearest-even from the exact real (max-min)/(2^b-1);
+ *     z = min is stored as fp16 (exact).
+ *   - A code is round-half-to-even of the EXACT rational (x - z)/s computed with the stored fp16
+ *     s and z, then clamped to [0, 2^b-1].  s == 0 gives code 0 (D reproduces z).
+ *   - The residual always holds the newest 1..R tokens once anything is cached; a full residual
+ *     is flushed (quantized as one R-token block) before the next append.
+ *
+ * Every pointer argument named *_dev is DEVICE memory owned by the caller; the library never
+ * allocates, frees or retains memory.
+ * fp16 values are passed as their IEEE binary16 bit patterns (uint16_t).  Every call is
+ * asynchronous on `stream` (a cudaStream_t passed as void*; NULL = legacy default stream) and
+ * returns a status code synchronously.  On any error return nothing has been enqueued and the
+ * cache counters are unchanged.
+ *
+ * DEVICE LAYOUT (B batch, H = num_kv_heads, d = head_dim, b = bits, P = 32/b codes per uint32,
+ * R = residual, C = capacity, G_k = group_k, G_v = group_v; all arrays dense, row-major):
+ *   k_codes  uint32 [B][H][C][d/P]   token-major.  Word i of token t holds the codes of channels
+ *                                     P*i + j (j = 0..P-1) at bits [b*j, b*j + b).
+ *   v_codes  uint32 [B][H][C/P][d]   channel-major within P-token rows.  Word (r, c) holds the
+ *                                     codes of tokens P*r + j of channel c at bits [b*j, b*j + b).
+ *   k_scale, k_zero  fp16 [B][H][C/R][d/G_k]   one pair per (R-token block, channel group).
+ *   v_scale, v_zero  fp16 [B][H][C/G_v]        one pair per G_v-token group.
+ *   k_res, v_res     fp16 [B][H][R][d]         residual slots 0..n_res-1 hold the newest tokens.
+ *   Token order of a head: quantized tokens 0..n_quant-1, then residual slots 0..n_res-1.
+ * Host inputs: k, v fp16 [B][H][T][d]; k_new, v_new fp16 [B][H][d]; q, out fp16 [B][Hq][d].
+ * Query head h attends with KV head h / (Hq/H) (contiguous grouped-query mapping).
+ *
+ * Every device pointer must be 16-byte aligned.
+ */
+#ifndef KIVI_H
+#define KIVI_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define KIVI_ABI_VERSION 1
+
+/* Status codes. */
+#define KIVI_OK 0
+#define KIVI_ERR_INVALID_ARG 1       /* NULL/misaligned pointer or a shape rule below violated */
+#define KIVI_ERR_UNSUPPORTED 2       /* bits not in {2,4}, head_dim not 128, or a size limit */
+#define KIVI_ERR_CAPACITY 3          /* the call would exceed `capacity` quantized tokens */
+#define KIVI_ERR_RESIDUAL_FULL 4     /* append with n_res == R: flush first */
+#define KIVI_ERR_RESIDUAL_NOT_FULL 5 /* flush with n_res < R */
+#define KIVI_ERR_EMPTY 6             /* attention over an empty cache */
+#define KIVI_ERR_WORKSPACE 7         /* workspace NULL, misaligned or too small */
+#define KIVI_ERR_CUDA 8              /* a CUDA runtime call or kernel launch failed */
+#define KIVI_ERR_DEVICE_TIMEOUT 9    /* a bounded device-side wait expired (reported via status) */
+#define KIVI_ERR_STATE 10            /* cache counters inconsistent with the call */
+
+/*
+ * Quantization configuration; mirrors the page's QuantConfig (section アルゴリズム: bits,
+ * group_size_k, group_size_v, residual_length) plus the shape and capacity of the cache.
+ * Rules: batch >= 1, num_kv_heads >= 1, capacity >= 0, capacity % residual == 0,
+ * group_k in {32, 64, 128}, group_v % 32 == 0 and group_v divides residual,
+ * residual % 128 == 0 and 128 <= residual <= 1024 (KIVI_ERR_INVALID_ARG otherwise);
+ * head_dim == 128, bits in {2, 4} (KIVI_ERR_UNSUPPORTED otherwise).
+ */
+typedef struct kivi_config {
+  int32_t batch;        /* B */
+  int32_t num_kv_heads; /* H */
+  int32_t head_dim;     /* d: 128 */
+  int32_t bits;         /* b: 2 or 4 */
+  int32_t group_k;      /* G_k: channels per K group */
+  int32_t group_v;      /* G_v: tokens per V group */
+  int32_t residual;     /* R: residual (fp16) capacity in tokens, also the K block length */
+  int32_t capacity;     /* C: maximum number of quantized tokens per head */
+} kivi_config;
+
+/* Device buffers of one cache (caller-owned) plus the two host-side counters the calls advance.
+ * n_quant is always a multiple of R; 0 <= n_res <= R.  Counters are uniform over (batch, head). */
+typedef struct kivi_cache {
+  uint32_t *k_codes, *v_codes;
+  uint16_t *k_scale, *k_zero, *v_scale, *v_zero;
+  uint16_t *k_res, *v_res;
+  int32_t n_quant;
+  int32_t n_res;
+} kivi_cache;
+
+/* Index of each buffer in kivi_cache_sizes' output. */
+enum {
+  KIVI_BUF_K_CODES = 0, KIVI_BUF_V_CODES, KIVI_BUF_K_SCALE, KIVI_BUF_K_ZERO,
+  KIVI_BUF_V_SCALE, KIVI_BUF_V_ZERO, KIVI_BUF_K_RES, KIVI_BUF_V_RES, KIVI_NUM_BUFS
+};
+
+/* Writes the byte size of each cache buffer (layout above) into out_bytes[KIVI_NUM_BUFS].
+ * Host-only; no CUDA call.  Returns KIVI_OK or KIVI_ERR_INVALID_ARG / KIVI_ERR_UNSUPPORTED. */
+int kivi_cache_sizes(const kivi_config* cfg, size_t* out_bytes);
+
+/* Checks cfg against the rules above without touching the device. */
+int kivi_check_config(const kivi_config* cfg);
+
+/*
+ * Prefill: quantizes a prompt of T tokens per head and resets the cache.
+ * Sections 量子化アルゴリズム, Per-Channel量子化, Per-Token量子化 and 残差バッファ.
+ * k_dev, v_dev: fp16 [B][H][T][d].  Afterwards n_res = ((T-1) mod R) + 1 and
+ * n_quant = T - n_res (so T <= R keeps everything in fp16); tokens [0, n_quant) are quantized
+ * as n_quant/R blocks and tokens [n_quant, T) are copied into residual slots 0..n_res-1.
+ * Errors: T < 1 (INVALID_ARG), n_quant > capacity (CAPACITY).  One kernel launch.
+ */
+int kivi_quantize_prefill(const kivi_config* cfg, kivi_cache* cache, const uint16_t* k_dev,
+                          const uint16_t* v_dev, int32_t num_tokens, void* stream);
+
+/*
+ * Append: writes one new token's K and V (fp16 [B][H][d]) into residual slot n_res and
+ * increments n_res.  Section 残差バッファ.  Errors: n_res == R (RESIDUAL_FULL).  One launch.
+ */
+int kivi_append_token(const kivi_config* cfg, kivi_cache* cache, const uint16_t* k_new_dev,
+                      const uint16_t* v_new_dev, void* stream);
+
+/*
+ * Flush: quantizes the full residual (R tokens) as quantized block n_quant/R, then
+ * n_quant += R, n_res = 0.  Sections Per-Token量子化 (flush once the group fills) and 残差バッファ.
+ * Errors: n_res < R (RESIDUAL_NOT_FULL), n_quant + R > capacity (CAPACITY).  One launch.
+ */
+int kivi_flush_residual(const kivi_config* cfg, kivi_cache* cache, void* stream);
+
+/* Bytes of scratch workspace kivi_decode_attention needs for this config and query-head count.
+ * Returns 0 if the arguments are invalid.  The size does not depend on the cache counters. */
+size_t kivi_decode_workspace_bytes(const kivi_config* cfg, int32_t num_q_heads);
+
+/*
+ * Decode attention for one query token per query head over the whole cache:
+ *   out[b][h] = softmax(scale * q[b][h] . [D(Kq); Kres]^T) [D(Vq); Vres]
+ * Section 残差バッファ, Attention equation (scale = 1/sqrt(d_k) there; any finite scale accepted).
+ * q_dev, out_dev: fp16 [B][Hq][d]; Hq must be a multiple of H.
+ * workspace_dev: kivi_decode_workspace_bytes(cfg, Hq) bytes, 256-byte aligned; it must be ZERO
+ * before its first use and is left zero by every call that completes without a device error
+ * (after a device error, zero it again).  Calls sharing one workspace must not overlap.
+ * dev_status: optional (may be NULL) device int32 that receives KIVI_ERR_DEVICE_TIMEOUT if a
+ * bounded wait inside the kernel expires; the caller zeroes it and reads it with kivi_read_status.
+ * Errors: empty cache (EMPTY), workspace too small (WORKSPACE).  One kernel launch.
+ */
+int kivi_decode_attention(const kivi_config* cfg, const kivi_cache* cache, const uint16_t* q_dev,
+                          int32_t num_q_heads, float scale, uint16_t* out_dev, void* workspace_dev,
+                          size_t workspace_bytes, int32_t* dev_status, void* stream);
+
+/* Synchronizes `stream` and returns the device-side status word (KIVI_OK if it is 0). */
+int kivi_read_status(const int32_t* dev_status, void* stream);
+
+/* Human-readable name of a status code (static string). */
+const char* kivi_strerror(int status);
+
+/* KIVI_ABI_VERSION of the loaded library. */
+int kivi_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KIVI_H */

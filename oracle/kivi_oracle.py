@@ -1,0 +1,354 @@
+"""CPU oracle: KIVI-style asymmetric low-bit KV-cache quantization and decode attention.
+
+TEST INFRASTRUCTURE, NOT PRODUCT CODE.  Only the tests, ``__graft_entry__.smoke()`` and the
+``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` may import or run this module.  The
+CUDA library never calls it and shares no code, table or helper with it.
+
+Plain numpy, float64 arithmetic, written for reading rather than speed.  Method source: the KIVI
+explainer page "ICML 2024論文解説: KIVI — チューニング不要のKVキャッシュ2bit非対称量子化"
+(arXiv 2402.02750).  Each function names the section / equation of that page it follows.
+
+Readings taken where the page leaves a step open (each is pinned by tests/test_oracle_pins.py):
+  * K group = one R-token block x G_k consecutive channels; V group = G_v consecutive tokens x
+    all d channels (sections Per-Channel量子化 / Per-Token量子化, their K_quant / V_quant equations).
+  * s is stored in fp16: the exact real (max-min)/(2^b-1) rounded to nearest, ties to even.
+    The subtraction of two fp16 values is exact in fp64 and the quotient by 3 or 15 cannot
+    fall onto an fp16 rounding midpoint unless it is exactly one, so "fp64 divide, then round to
+    fp16" is the correctly rounded value.
+  * A code is round-half-to-even of the exact rational (x - z)/s with the STORED fp16 s and z,
+    clamped to [0, 2^b-1]; s == 0 gives code 0.  (x - z) is exact in fp64; the fp64 quotient is
+    within 2^-50 of the exact value, far closer than any non-tie can be to a half-integer, so
+    np.rint of it gives the exact decision.  This is checked against exact rationals.
+  * The residual holds the newest 1..R tokens; prefill of T tokens keeps ((T-1) mod R)+1 of them
+    in fp16 and quantizes the rest as R-token blocks; a full residual is flushed before an append.
+  * Decode attention follows the Attention equation of section 残差バッファ: logits over the
+    dequantized quantized tokens followed by the fp16 residual tokens, softmax, weighted sum of
+    the matching V rows.  No mask; the query-head -> KV-head map is contiguous (h // (Hq/H)).
+
+Parity pinned: every public function below is pinned by at least one test that does not reuse
+its code (exact rationals, nearest-grid-point brute force, hand-derived fixtures, closed forms,
+textbook attention).
+"""
+from __future__ import annotations
+
+import numpy as np
+
+__all__ = [
+    "OracleError", "levels", "codes_per_word", "fp16_round", "scale_zero", "quantize_values",
+    "quantize_k_block", "quantize_v_block", "pack_k", "pack_v", "unpack_k", "unpack_v",
+    "dequantize_k", "dequantize_v", "attention", "HeadCache", "OracleCache",
+]
+
+
+class OracleError(Exception):
+    """Raised for a call the cache contract forbids; ``.code`` names the matching C status."""
+
+    def __init__(self, code: str, msg: str = ""):
+        super().__init__(f"{code}: {msg}")
+        self.code = code
+
+
+def levels(bits: int) -> int:
+    """Largest code 2^b - 1 (section 量子化アルゴリズム, clamp bound of the Q equation)."""
+    return (1 << bits) - 1
+
+
+def codes_per_word(bits: int) -> int:
+    """Codes packed into one uint32 word of the cache layout."""
+    return 32 // bits
+
+
+def fp16_round(x) -> np.ndarray:
+    """Round float64 values to binary16, nearest with ties to even (numpy's direct conversion)."""
+    return np.asarray(x, dtype=np.float64).astype(np.float16)
+
+
+def scale_zero(lo, hi, bits: int):
+    """s = (max X_g - min X_g)/(2^b - 1) stored as fp16, z = min X_g (section 量子化アルゴリズム,
+    s/z equation).  lo, hi: fp16 group minima and maxima (arrays of equal shape)."""
+    lo64 = np.asarray(lo, dtype=np.float16).astype(np.float64)
+    hi64 = np.asarray(hi, dtype=np.float16).astype(np.float64)
+    s = fp16_round((hi64 - lo64) / levels(bits))
+    z = np.asarray(lo, dtype=np.float16).copy()
+    return s, z
+
+
+def quantize_values(x, s, z, bits: int) -> np.ndarray:
+    """Q(X) = clamp(round((X - z)/s), 0, 2^b - 1) with round-half-to-even (section 量子化アルゴリズム,
+    Q equation).  x, s, z are fp16 and broadcast together; s == 0 yields code 0."""
+    x64 = np.asarray(x, dtype=np.float16).astype(np.float64)
+    s64 = np.asarray(s, dtype=np.float16).astype(np.float64)
+    z64 = np.asarray(z, dtype=np.float16).astype(np.float64)
+    safe = np.where(s64 == 0.0, 1.0, s64)
+    r = np.rint((x64 - z64) / safe)
+    q = np.clip(r, 0, levels(bits))
+    q = np.where(s64 == 0.0, 0.0, q)
+    return q.astype(np.uint8)
+
+
+def quantize_k_block(block, group_k: int, bits: int):
+    """Per-channel K quantization of one R-token block (section Per-Channel量子化（Key Cache）,
+    K_quant[:, j:j+g_k] = Q(K[:, j:j+g_k])): one (s, z) per g_k consecutive channels, taken over
+    every token of the block.  block: fp16 [R][d].  Returns codes uint8 [R][d], s and z fp16
+    [d/g_k]."""
+    block = np.asarray(block, dtype=np.float16)
+    n, d = block.shape
+    ng = d // group_k
+    lo = np.empty(ng, dtype=np.float16)
+    hi = np.empty(ng, dtype=np.float16)
+    for g in range(ng):
+        cols = block[:, g * group_k:(g + 1) * group_k]
+        lo[g] = cols.min()
+        hi[g] = cols.max()
+    s, z = scale_zero(lo, hi, bits)
+    s_per_col = np.repeat(s, group_k)[None, :]
+    z_per_col = np.repeat(z, group_k)[None, :]
+    codes = quantize_values(block, s_per_col, z_per_col, bits)
+    return codes, s, z
+
+
+def quantize_v_block(block, group_v: int, bits: int):
+    """Per-token V quantization (section Per-Token量子化（Value Cache）,
+    V_quant[i:i+g_v, :] = Q(V[i:i+g_v, :])): one (s, z) per g_v consecutive tokens, taken over
+    every channel.  block: fp16 [n][d] with n a multiple of g_v.  Returns codes uint8 [n][d],
+    s and z fp16 [n/g_v]."""
+    block = np.asarray(block, dtype=np.float16)
+    n, d = block.shape
+    ng = n // group_v
+    lo = np.empty(ng, dtype=np.float16)
+    hi = np.empty(ng, dtype=np.float16)
+    for u in range(ng):
+        rows = block[u * group_v:(u + 1) * group_v, :]
+        lo[u] = rows.min()
+        hi[u] = rows.max()
+    s, z = scale_zero(lo, hi, bits)
+    s_per_row = np.repeat(s, group_v)[:, None]
+    z_per_row = np.repeat(z, group_v)[:, None]
+    codes = quantize_values(block, s_per_row, z_per_row, bits)
+    return codes, s, z
+
+
+def pack_k(codes, bits: int) -> np.ndarray:
+    """Token-major K packing of the cache layout: word i of token t holds the codes of channels
+    P*i + j at bits [b*j, b*j+b), P = 32/b.  codes: uint8 [n][d] -> uint32 [n][d/P]."""
+    codes = np.asarray(codes, dtype=np.uint64)
+    n, d = codes.shape
+    per = codes_per_word(bits)
+    out = np.zeros((n, d // per), dtype=np.uint64)
+    for j in range(per):
+        out |= codes[:, j::per] << np.uint64(bits * j)
+    return out.astype(np.uint32)
+
+
+def pack_v(codes, bits: int) -> np.ndarray:
+    """V packing of the cache layout: word (r, c) holds the codes of tokens P*r + j of channel c at
+    bits [b*j, b*j+b).  codes: uint8 [n][d], n a multiple of P -> uint32 [n/P][d]."""
+    codes = np.asarray(codes, dtype=np.uint64)
+    n, d = codes.shape
+    per = codes_per_word(bits)
+    out = np.zeros((n // per, d), dtype=np.uint64)
+    for j in range(per):
+        out |= codes[j::per, :] << np.uint64(bits * j)
+    return out.astype(np.uint32)
+
+
+def unpack_k(words, bits: int) -> np.ndarray:
+    """Inverse of pack_k: uint32 [n][d/P] -> uint8 [n][d]."""
+    words = np.asarray(words, dtype=np.uint32)
+    n, nw = words.shape
+    per = codes_per_word(bits)
+    mask = np.uint32(levels(bits))
+    out = np.zeros((n, nw * per), dtype=np.uint8)
+    for j in range(per):
+        out[:, j::per] = (words >> np.uint32(bits * j)) & mask
+    return out
+
+
+def unpack_v(words, bits: int) -> np.ndarray:
+    """Inverse of pack_v: uint32 [n/P][d] -> uint8 [n][d]."""
+    words = np.asarray(words, dtype=np.uint32)
+    nr, d = words.shape
+    per = codes_per_word(bits)
+    mask = np.uint32(levels(bits))
+    out = np.zeros((nr * per, d), dtype=np.uint8)
+    for j in range(per):
+        out[j::per, :] = (words >> np.uint32(bits * j)) & mask
+    return out
+
+
+def dequantize_k(codes, s, z, block: int, group_k: int) -> np.ndarray:
+    """D(K^) = s*K^ + z in float64 with the (block, channel group) scale of each element (section
+    量子化アルゴリズム, D equation).  codes uint8 [n][d]; s, z fp16 [n/block][d/group_k]."""
+    codes = np.asarray(codes, dtype=np.float64)
+    s64 = np.asarray(s, dtype=np.float16).astype(np.float64)
+    z64 = np.asarray(z, dtype=np.float16).astype(np.float64)
+    s_full = np.repeat(np.repeat(s64, block, axis=0), group_k, axis=1)
+    z_full = np.repeat(np.repeat(z64, block, axis=0), group_k, axis=1)
+    return s_full * codes + z_full
+
+
+def dequantize_v(codes, s, z, group_v: int) -> np.ndarray:
+    """D(V^) = s*V^ + z in float64 with the token-group scale of each row (D equation).
+    codes uint8 [n][d]; s, z fp16 [n/group_v]."""
+    codes = np.asarray(codes, dtype=np.float64)
+    s64 = np.repeat(np.asarray(s, dtype=np.float16).astype(np.float64), group_v)[:, None]
+    z64 = np.repeat(np.asarray(z, dtype=np.float16).astype(np.float64), group_v)[:, None]
+    return s64 * codes + z64
+
+
+def attention(q, keys, values, scale: float) -> np.ndarray:
+    """softmax(scale * q K^T) V for each query row, in float64 (section 残差バッファ, Attention
+    equation).  q: [G][d]; keys, values: [T][d] float64 (dequantized then residual rows).
+    Returns float64 [G][d]."""
+    q64 = np.asarray(q, dtype=np.float16).astype(np.float64)
+    logits = (q64 @ np.asarray(keys, dtype=np.float64).T) * float(scale)   # [G][T]
+    logits = logits - logits.max(axis=1, keepdims=True)
+    w = np.exp(logits)
+    w = w / w.sum(axis=1, keepdims=True)
+    return w @ np.asarray(values, dtype=np.float64)
+
+
+class HeadCache:
+    """Quantized cache of one (batch, KV head): quantized blocks plus the fp16 residual.
+
+    Mirrors the library's counters: n_quant (a multiple of R) and n_res in [0, R]."""
+
+    def __init__(self, head_dim: int, bits: int, group_k: int, group_v: int, residual: int,
+                 capacity: int):
+        self.d, self.bits, self.gk, self.gv = head_dim, bits, group_k, group_v
+        self.R, self.capacity = residual, capacity
+        self.k_codes = np.zeros((0, head_dim), np.uint8)
+        self.v_codes = np.zeros((0, head_dim), np.uint8)
+        self.k_s = np.zeros((0, head_dim // group_k), np.float16)
+        self.k_z = np.zeros((0, head_dim // group_k), np.float16)
+        self.v_s = np.zeros((0,), np.float16)
+        self.v_z = np.zeros((0,), np.float16)
+        self.k_res = np.zeros((0, head_dim), np.float16)
+        self.v_res = np.zeros((0, head_dim), np.float16)
+
+    @property
+    def n_quant(self) -> int:
+        return self.k_codes.shape[0]
+
+    @property
+    def n_res(self) -> int:
+        return self.k_res.shape[0]
+
+    def _quantize_block(self, kblk, vblk):
+        kc, ks, kz = quantize_k_block(kblk, self.gk, self.bits)
+        vc, vs, vz = quantize_v_block(vblk, self.gv, self.bits)
+        self.k_codes = np.concatenate([self.k_codes, kc])
+        self.v_codes = np.concatenate([self.v_codes, vc])
+        self.k_s = np.concatenate([self.k_s, ks[None, :]])
+        self.k_z = np.concatenate([self.k_z, kz[None, :]])
+        self.v_s = np.concatenate([self.v_s, vs])
+        self.v_z = np.concatenate([self.v_z, vz])
+
+    def prefill(self, k, v):
+        """Resets the head and caches a prompt: the newest ((T-1) mod R)+1 tokens stay fp16, the
+        older ones are quantized block by block (sections Per-Channel量子化, Per-Token量子化,
+        残差バッファ)."""
+        k = np.asarray(k, np.float16)
+        v = np.asarray(v, np.float16)
+        T = k.shape[0]
+        if T < 1:
+            raise OracleError("INVALID_ARG", "empty prompt")
+        n_res = (T - 1) % self.R + 1
+        n_quant = T - n_res
+        if n_quant > self.capacity:
+            raise OracleError("CAPACITY", f"{n_quant} > {self.capacity}")
+        self.__init__(self.d, self.bits, self.gk, self.gv, self.R, self.capacity)
+        for j in range(n_quant // self.R):
+            sl = slice(j * self.R, (j + 1) * self.R)
+            self._quantize_block(k[sl], v[sl])
+        self.k_res = k[n_quant:].copy()
+        self.v_res = v[n_quant:].copy()
+
+    def append(self, k_new, v_new):
+        """Writes the newest token into the fp16 residual (section 残差バッファ)."""
+        if self.n_res == self.R:
+            raise OracleError("RESIDUAL_FULL")
+        self.k_res = np.concatenate([self.k_res, np.asarray(k_new, np.float16)[None, :]])
+        self.v_res = np.concatenate([self.v_res, np.asarray(v_new, np.float16)[None, :]])
+
+    def flush(self):
+        """Quantizes a full residual as the next block (section Per-Token量子化: tokens are
+        quantized together once a group has accumulated; section 残差バッファ)."""
+        if self.n_res < self.R:
+            raise OracleError("RESIDUAL_NOT_FULL")
+        if self.n_quant + self.R > self.capacity:
+            raise OracleError("CAPACITY")
+        self._quantize_block(self.k_res, self.v_res)
+        self.k_res = np.zeros((0, self.d), np.float16)
+        self.v_res = np.zeros((0, self.d), np.float16)
+
+    def keys(self) -> np.ndarray:
+        """[D(K_quant); K_res] as float64 [n_quant + n_res][d]."""
+        kd = dequantize_k(self.k_codes, self.k_s, self.k_z, self.R, self.gk)
+        return np.concatenate([kd, self.k_res.astype(np.float64)])
+
+    def values(self) -> np.ndarray:
+        """[D(V_quant); V_res] as float64 [n_quant + n_res][d]."""
+        vd = dequantize_v(self.v_codes, self.v_s, self.v_z, self.gv)
+        return np.concatenate([vd, self.v_res.astype(np.float64)])
+
+    def attend(self, q, scale: float) -> np.ndarray:
+        """Decode attention of the query rows q [G][d] over this head (Attention equation)."""
+        if self.n_quant + self.n_res == 0:
+            raise OracleError("EMPTY")
+        return attention(q, self.keys(), self.values(), scale)
+
+    def packed(self):
+        """The head's filled cache in the library's device layout (tokens [0, n_quant))."""
+        return {
+            "k_codes": pack_k(self.k_codes, self.bits),
+            "v_codes": pack_v(self.v_codes, self.bits),
+            "k_scale": self.k_s, "k_zero": self.k_z, "v_scale": self.v_s, "v_zero": self.v_z,
+            "k_res": self.k_res, "v_res": self.v_res,
+        }
+
+
+class OracleCache:
+    """A [batch][kv head] grid of HeadCache objects with the library's calls.  ``heads`` limits the
+    work to a subset of (b, h) pairs (the other heads stay empty)."""
+
+    def __init__(self, batch: int, num_kv_heads: int, head_dim: int = 128, bits: int = 2,
+                 group_k: int = 32, group_v: int = 32, residual: int = 128, capacity: int = 0,
+                 heads=None):
+        self.B, self.H = batch, num_kv_heads
+        self.heads = sorted(heads) if heads is not None else [
+            (b, h) for b in range(batch) for h in range(num_kv_heads)]
+        self.cache = {bh: HeadCache(head_dim, bits, group_k, group_v, residual, capacity)
+                      for bh in self.heads}
+
+    def _counters(self):
+        c = next(iter(self.cache.values()))
+        return c.n_quant, c.n_res
+
+    @property
+    def n_quant(self) -> int:
+        return self._counters()[0]
+
+    @property
+    def n_res(self) -> int:
+        return self._counters()[1]
+
+    def prefill(self, k_of, v_of):
+        """k_of(b, h) / v_of(b, h) return the fp16 [T][d] prompt of one head."""
+        for (b, h), c in self.cache.items():
+            c.prefill(k_of(b, h), v_of(b, h))
+
+    def append(self, k_new_of, v_new_of):
+        if self.n_res == next(iter(self.cache.values())).R:
+            raise OracleError("RESIDUAL_FULL")
+        for (b, h), c in self.cache.items():
+            c.append(k_new_of(b, h), v_new_of(b, h))
+
+    def flush(self):
+        for c in self.cache.values():
+            c.flush()
+
+    def attend(self, q_of, group: int, scale: float):
+        """q_of(b, h) returns the fp16 [group][d] query rows of KV head h (query heads
+        h*group .. h*group+group-1).  Returns {(b, h): float64 [group][d]}."""
+        return {(b, h): c.attend(q_of(b, h), scale) for (b, h), c in self.cache.items()}

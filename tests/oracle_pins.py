@@ -1,0 +1,376 @@
+"""Checks that pin the CPU oracle to facts other than its own code.
+
+Each ``check_*`` takes the oracle module and raises AssertionError on a mismatch, so the same
+checks run against the real oracle (test_oracle_pins.py) and against planted mistakes
+(test_oracle_mutants.py).  Sources of truth: exact rational arithmetic (tests/exact.py), search
+for the nearest grid point, hand-derived fixtures in tests/golden/, closed forms of attention
+special cases, PyTorch's scaled_dot_product_attention in float64, and pure-Python brute force
+that reads the packed words bit by bit.
+"""
+from __future__ import annotations
+
+import json
+import math
+import os
+from fractions import Fraction
+
+import numpy as np
+import torch
+
+from exact import code_exact, code_nearest_grid, fp16_round_exact
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+def _fr(x) -> Fraction:
+    return Fraction(float(x))
+
+
+def _hex16(x) -> str:
+    return "0x%04x" % int(np.asarray(x, np.float16).view(np.uint16))
+
+
+def _rand_fp16(rng, n, lo_exp=-24, hi_exp=15):
+    """fp16 values with log-uniform magnitudes and random signs (includes subnormals)."""
+    e = rng.uniform(lo_exp, hi_exp, n)
+    x = np.sign(rng.standard_normal(n)) * np.exp2(e)
+    return np.clip(x, -65504, 65504).astype(np.float16)
+
+
+# --------------------------------------------------------------------------------------------
+# fp16 rounding and s / z
+# --------------------------------------------------------------------------------------------
+def check_fp16_round(O):
+    rng = np.random.default_rng(11)
+    xs = [1 + 2 ** -11, 1 + 3 * 2 ** -11, 1 + 2 ** -11 + 2 ** -40, 2 ** -25, 3 * 2 ** -25,
+          2 ** -25 + 2 ** -60, 65504.0, 65519.0, 0.2, 1 / 3, 2 / 3, 1e-7, 43669.0]
+    xs += list(rng.standard_normal(200) * np.exp2(rng.uniform(-26, 15, 200)))
+    got = O.fp16_round(np.array(xs))
+    for x, g in zip(xs, got):
+        want = fp16_round_exact(Fraction(x))
+        assert Fraction(float(g)) == want, (x, float(g), want)
+
+
+def check_scale_zero_exact(O, bits):
+    rng = np.random.default_rng(12 + bits)
+    L = 2 ** bits - 1
+    a = _rand_fp16(rng, 3000)
+    b = _rand_fp16(rng, 3000)
+    lo = np.minimum(a, b)
+    hi = np.maximum(a, b)
+    # every positive finite fp16 as a range starting at 0 and at -hi: all quotients near midpoints
+    allpos = np.arange(1, 0x7C00, dtype=np.uint16).view(np.float16)
+    lo = np.concatenate([lo, np.zeros_like(allpos), -allpos[::7]])
+    hi = np.concatenate([hi, allpos, allpos[::7]])
+    s, z = O.scale_zero(lo, hi, bits)
+    assert s.dtype == np.float16 and z.dtype == np.float16
+    assert np.array_equal(z.view(np.uint16), lo.view(np.uint16))
+    for l_, h_, s_ in zip(lo[::3], hi[::3], s[::3]):
+        want = fp16_round_exact((_fr(h_) - _fr(l_)) / L)
+        assert Fraction(float(s_)) == want, (float(l_), float(h_), float(s_), want)
+    # the all-pos sweep in full (these are the cases where a double rounding would show)
+    n0 = 3000
+    for l_, h_, s_ in zip(lo[n0:n0 + len(allpos)], hi[n0:n0 + len(allpos)], s[n0:n0 + len(allpos)]):
+        want = fp16_round_exact((_fr(h_) - _fr(l_)) / L)
+        assert Fraction(float(s_)) == want, (float(l_), float(h_), float(s_), want)
+
+
+# --------------------------------------------------------------------------------------------
+# codes
+# --------------------------------------------------------------------------------------------
+def _tie_cases(rng, bits, n):
+    """(x, s, z) triples where (x - z)/s lands exactly on half-integers or a hair away."""
+    L = 2 ** bits - 1
+    xs, ss, zs = [], [], []
+    while len(xs) < n:
+        e = int(rng.integers(-12, 6))
+        s = np.float16(float(rng.integers(1, 64)) * 2.0 ** (e - 5))
+        z = np.float16(float(rng.integers(-512, 512)) * 2.0 ** (e - 6))
+        k = int(rng.integers(0, L + 1))
+        for off in (0.5, -0.5):
+            x = np.float16(float(z) + (k + off) * float(s))
+            # the (usually exact) tie and one fp16 ulp either side of it
+            for xv in (x, np.nextafter(x, np.float16(np.inf)), np.nextafter(x, np.float16(-np.inf))):
+                if np.isfinite(xv) and float(xv) >= float(z):
+                    xs.append(xv)
+                    ss.append(s)
+                    zs.append(z)
+    return (np.array(xs, np.float16), np.array(ss, np.float16), np.array(zs, np.float16))
+
+
+def check_codes_exact(O, bits):
+    rng = np.random.default_rng(21 + bits)
+    x, s, z = _tie_cases(rng, bits, 1500)
+    # plus ordinary groups with their own (s, z)
+    for _ in range(60):
+        g = _rand_fp16(rng, 40, -10, 4)
+        ss, zz = O.scale_zero(np.array([g.min()]), np.array([g.max()]), bits)
+        x = np.concatenate([x, g])
+        s = np.concatenate([s, np.repeat(ss, len(g))])
+        z = np.concatenate([z, np.repeat(zz, len(g))])
+    codes = O.quantize_values(x, s, z, bits)
+    assert codes.dtype == np.uint8
+    for xi, si, zi, ci in zip(x, s, z, codes):
+        want = code_exact(_fr(xi), _fr(si), _fr(zi), bits)
+        assert int(ci) == want, (float(xi), float(si), float(zi), int(ci), want)
+        if si != 0 and float(xi) <= float(zi) + (2 ** bits - 1 + 0.5) * float(si):
+            assert want == code_nearest_grid(_fr(xi), _fr(si), _fr(zi), bits)
+
+
+def check_hand_examples(O):
+    with open(os.path.join(GOLDEN, "quantize_hand_examples.json")) as f:
+        cases = json.load(f)["cases"]
+    for c in cases:
+        g = np.array(c["group"], np.float16)
+        s, z = O.scale_zero(np.array([g.min()]), np.array([g.max()]), c["bits"])
+        assert _hex16(s[0]) == c["s_fp16_bits"], (c["name"], _hex16(s[0]))
+        assert _hex16(z[0]) == c["z_fp16_bits"], (c["name"], _hex16(z[0]))
+        codes = O.quantize_values(g, s[0], z[0], c["bits"])
+        assert codes.tolist() == c["codes"], (c["name"], codes.tolist())
+
+
+def check_invariants(O, bits):
+    """codes in [0, L]; min -> 0; max -> L and |x - D(Q(x))| <= s/2 when s is a normal fp16;
+    all 2^b levels reachable; zero range reconstructs exactly."""
+    rng = np.random.default_rng(31 + bits)
+    L = 2 ** bits - 1
+    for trial in range(200):
+        n = int(rng.integers(2, 300))
+        g = (rng.standard_normal(n) * np.exp2(rng.uniform(-8, 8))).astype(np.float16)
+        s, z = O.scale_zero(np.array([g.min()]), np.array([g.max()]), bits)
+        c = O.quantize_values(g, s[0], z[0], bits)
+        assert c.min() >= 0 and c.max() <= L
+        assert c[np.argmin(g)] == 0
+        s64, z64 = float(s[0]), float(z[0])
+        if s64 >= 2 ** -14:
+            assert c[np.argmax(g)] == L
+            err = np.abs(g.astype(np.float64) - (s64 * c + z64))
+            assert err.max() <= s64 / 2, (err.max(), s64)
+    lin = np.linspace(-1, 1, 64).astype(np.float16)
+    s, z = O.scale_zero(np.array([lin.min()]), np.array([lin.max()]), bits)
+    assert sorted(set(O.quantize_values(lin, s[0], z[0], bits).tolist())) == list(range(L + 1))
+    const = np.full(17, -3.375, np.float16)
+    s, z = O.scale_zero(np.array([const.min()]), np.array([const.max()]), bits)
+    c = O.quantize_values(const, s[0], z[0], bits)
+    assert float(s[0]) == 0.0 and not c.any()
+    assert np.array_equal(float(s[0]) * c + float(z[0]), const.astype(np.float64))
+
+
+# --------------------------------------------------------------------------------------------
+# group axes of K and V blocks
+# --------------------------------------------------------------------------------------------
+def check_block_groups(O, bits, group):
+    """Per-channel K groups span every token of the block and `group` consecutive channels;
+    per-token V groups span `group` consecutive tokens and every channel.  Brute force with
+    explicit index loops and exact rationals."""
+    rng = np.random.default_rng(41 + bits + group)
+    n, d = 2 * group, 128
+    blk = (rng.standard_normal((n, d)) * np.exp2(rng.integers(-3, 4, (1, d)))).astype(np.float16)
+    blk[:, 5] *= np.float16(9)
+    blk[3, :] *= np.float16(7)
+    L = 2 ** bits - 1
+    kc, ks, kz = O.quantize_k_block(blk, group, bits)
+    assert ks.shape == (d // group,) and kc.shape == (n, d)
+    for g in range(d // group):
+        vals = [_fr(blk[t, c]) for t in range(n) for c in range(g * group, (g + 1) * group)]
+        lo, hi = min(vals), max(vals)
+        s = fp16_round_exact((hi - lo) / L)
+        assert Fraction(float(ks[g])) == s and Fraction(float(kz[g])) == lo
+        for t in range(0, n, 7):
+            for c in range(g * group, (g + 1) * group, 3):
+                assert kc[t, c] == code_exact(_fr(blk[t, c]), s, lo, bits)
+    vc, vs, vz = O.quantize_v_block(blk, group, bits)
+    assert vs.shape == (n // group,) and vc.shape == (n, d)
+    for u in range(n // group):
+        vals = [_fr(blk[t, c]) for t in range(u * group, (u + 1) * group) for c in range(d)]
+        lo, hi = min(vals), max(vals)
+        s = fp16_round_exact((hi - lo) / L)
+        assert Fraction(float(vs[u])) == s and Fraction(float(vz[u])) == lo
+        for t in range(u * group, (u + 1) * group, 5):
+            for c in range(0, d, 9):
+                assert vc[t, c] == code_exact(_fr(blk[t, c]), s, lo, bits)
+
+
+# --------------------------------------------------------------------------------------------
+# packing
+# --------------------------------------------------------------------------------------------
+def check_pack_golden(O):
+    with open(os.path.join(GOLDEN, "pack_hand_examples.json")) as f:
+        cases = json.load(f)["cases"]
+    for c in cases:
+        t, ch, bits = c["tokens"], c["channels"], c["bits"]
+        codes = np.zeros((t, ch), np.uint8)
+        for i in range(t):
+            for j in range(ch):
+                codes[i, j] = {"code(t, c) = c mod 4": j % 4, "code(t, c) = c mod 8": j % 8,
+                               "code(t, c) = (t + c) mod 4": (i + j) % 4,
+                               "code(t, c) = t": i}[c["codes_rule"]]
+        want = np.array([int(w, 16) for w in np.ravel(c["words"])], np.uint32)
+        got = (O.pack_k(codes, bits) if c["layout"] == "k" else O.pack_v(codes, bits)).ravel()
+        assert np.array_equal(got, want), (c["name"], [hex(w) for w in got])
+
+
+def check_pack_roundtrip(O, bits):
+    rng = np.random.default_rng(51 + bits)
+    P = 32 // bits
+    codes = rng.integers(0, 2 ** bits, (4 * P, 128)).astype(np.uint8)
+    wk = O.pack_k(codes, bits)
+    wv = O.pack_v(codes, bits)
+    assert wk.shape == (4 * P, 128 // P) and wv.shape == (4, 128)
+    assert np.array_equal(O.unpack_k(wk, bits), codes)
+    assert np.array_equal(O.unpack_v(wv, bits), codes)
+    # bit-level brute force of a few words
+    for t, i in [(0, 0), (3, 5), (4 * P - 1, 128 // P - 1)]:
+        w = int(wk[t, i])
+        for j in range(P):
+            assert (w >> (bits * j)) & (2 ** bits - 1) == codes[t, P * i + j]
+    for r, c in [(0, 0), (2, 77), (3, 127)]:
+        w = int(wv[r, c])
+        for j in range(P):
+            assert (w >> (bits * j)) & (2 ** bits - 1) == codes[P * r + j, c]
+
+
+# --------------------------------------------------------------------------------------------
+# cache semantics
+# --------------------------------------------------------------------------------------------
+def _head(O, bits=2, group=32, R=128, cap=4096):
+    return O.HeadCache(128, bits, group, group, R, cap)
+
+
+def check_prefill_split(O):
+    rng = np.random.default_rng(61)
+    R = 128
+    for T in (1, 2, 127, 128, 129, 255, 256, 257, 1024, 1025):
+        k = rng.standard_normal((T, 128)).astype(np.float16)
+        h = _head(O)
+        h.prefill(k, k)
+        assert h.n_res == (T - 1) % R + 1 and h.n_quant == T - h.n_res, (T, h.n_quant, h.n_res)
+        assert h.n_quant % R == 0 and 1 <= h.n_res <= R
+        assert np.array_equal(h.k_res, k[h.n_quant:])
+
+
+def check_prefill_equals_streaming(O, bits, group):
+    """prefill(T0) followed by appends (flushing whenever the residual is full) equals prefill of
+    all tokens at once, for every counter and every stored value."""
+    rng = np.random.default_rng(71 + bits)
+    T0, extra = 200, 190
+    k = (rng.standard_normal((T0 + extra, 128)) * 3).astype(np.float16)
+    v = rng.standard_normal((T0 + extra, 128)).astype(np.float16)
+    a = _head(O, bits, group)
+    a.prefill(k[:T0], v[:T0])
+    for t in range(T0, T0 + extra):
+        if a.n_res == a.R:
+            a.flush()
+        a.append(k[t], v[t])
+    b = _head(O, bits, group)
+    b.prefill(k, v)
+    assert (a.n_quant, a.n_res) == (b.n_quant, b.n_res)
+    pa, pb = a.packed(), b.packed()
+    for key in pa:
+        assert np.array_equal(np.asarray(pa[key]).view(np.uint8), np.asarray(pb[key]).view(np.uint8)), key
+
+
+def check_errors(O):
+    h = _head(O, cap=128)
+    k = np.zeros((128, 128), np.float16)
+    h.prefill(k, k)
+    for fn, code in ((lambda: h.append(k[0], k[0]), "RESIDUAL_FULL"),):
+        try:
+            fn()
+            raise AssertionError("expected " + code)
+        except O.OracleError as e:
+            assert e.code == code
+    h.flush()
+    try:
+        h.flush()
+        raise AssertionError("expected RESIDUAL_NOT_FULL")
+    except O.OracleError as e:
+        assert e.code == "RESIDUAL_NOT_FULL"
+    for _ in range(128):
+        h.append(k[0], k[0])
+    try:
+        h.flush()
+        raise AssertionError("expected CAPACITY")
+    except O.OracleError as e:
+        assert e.code == "CAPACITY"
+
+
+# --------------------------------------------------------------------------------------------
+# attention
+# --------------------------------------------------------------------------------------------
+def check_attention_sdpa(O):
+    """All-residual cache (T <= R): the oracle equals PyTorch SDPA in float64, GQA included."""
+    rng = np.random.default_rng(81)
+    for T, G in ((1, 1), (7, 1), (128, 4), (100, 2)):
+        k = rng.standard_normal((T, 128)).astype(np.float16)
+        v = rng.standard_normal((T, 128)).astype(np.float16)
+        q = rng.standard_normal((G, 128)).astype(np.float16)
+        h = _head(O)
+        h.prefill(k, v)
+        assert h.n_quant == 0
+        scale = 1 / math.sqrt(128)
+        got = h.attend(q, scale)
+        ref = torch.nn.functional.scaled_dot_product_attention(
+            torch.from_numpy(q.astype(np.float64))[None, :, None, :],
+            torch.from_numpy(k.astype(np.float64))[None, None].expand(1, G, T, 128),
+            torch.from_numpy(v.astype(np.float64))[None, None].expand(1, G, T, 128),
+            scale=scale)[0, :, 0, :].numpy()
+        assert np.allclose(got, ref, rtol=1e-12, atol=1e-13), np.abs(got - ref).max()
+
+
+def check_attention_closed_forms(O):
+    rng = np.random.default_rng(91)
+    k = rng.standard_normal((640, 128)).astype(np.float16)
+    v = (rng.standard_normal((640, 128)) * 2).astype(np.float16)
+    h = _head(O)
+    h.prefill(k, v)
+    assert h.n_quant == 512
+    # q = 0: uniform weights -> mean of the dequantized values (D of every quantized row + residual)
+    vd = np.concatenate([
+        np.array([[float(h.v_s[t // h.gv]) * h.v_codes[t, c] + float(h.v_z[t // h.gv])
+                   for c in range(128)] for t in range(h.n_quant)]),
+        h.v_res.astype(np.float64)])
+    got = h.attend(np.zeros((1, 128), np.float16), 0.0884)
+    assert np.allclose(got[0], vd.mean(axis=0), rtol=0, atol=1e-12)
+    # one token: the output is that token's value
+    h1 = _head(O)
+    h1.prefill(k[:1], v[:1])
+    assert np.array_equal(h1.attend(k[:1], 1.0)[0], v[0].astype(np.float64))
+
+
+def check_attention_bruteforce(O, bits, group):
+    """Tiny cache with quantized blocks and residual; pure-Python attention that reads the packed
+    words bit by bit and applies D = s*code + z with the block / group scale of each element."""
+    rng = np.random.default_rng(101 + bits)
+    R = 128
+    T = 2 * R + 37
+    k = (rng.standard_normal((T, 128)) * np.where(np.arange(128) % 29 == 0, 8, 1)).astype(np.float16)
+    v = rng.standard_normal((T, 128)).astype(np.float16)
+    v[0] *= np.float16(5)
+    q = rng.standard_normal((2, 128)).astype(np.float16)
+    h = _head(O, bits, group)
+    h.prefill(k, v)
+    pk = h.packed()
+    P, mask = 32 // bits, 2 ** bits - 1
+    keys, vals = [], []
+    for t in range(h.n_quant):
+        kr, vr = [], []
+        for c in range(128):
+            code = (int(pk["k_codes"][t, c // P]) >> (bits * (c % P))) & mask
+            kr.append(float(pk["k_scale"][t // R, c // group]) * code + float(pk["k_zero"][t // R, c // group]))
+            code = (int(pk["v_codes"][t // P, c]) >> (bits * (t % P))) & mask
+            vr.append(float(pk["v_scale"][t // group]) * code + float(pk["v_zero"][t // group]))
+        keys.append(kr)
+        vals.append(vr)
+    for t in range(h.n_res):
+        keys.append([float(x) for x in pk["k_res"][t]])
+        vals.append([float(x) for x in pk["v_res"][t]])
+    scale = 1 / math.sqrt(128)
+    got = h.attend(q, scale)
+    for gq in range(2):
+        logits = [scale * sum(float(q[gq, c]) * kr[c] for c in range(128)) for kr in keys]
+        m = max(logits)
+        w = [math.exp(x - m) for x in logits]
+        tot = sum(w)
+        out = [sum(w[t] * vals[t][c] for t in range(len(w))) / tot for c in range(128)]
+        assert np.allclose(got[gq], out, rtol=1e-11, atol=1e-12), np.abs(got[gq] - out).max()
