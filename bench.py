@@ -1,0 +1,459 @@
+#!/usr/bin/env python
+"""Benchmark: 2-bit KIVI decode over a quantized KV cache on B200, one JSON line on stdout.
+
+A step is one streaming decode step of the large-batch workload (B=64, H=32, d=128, 2-bit, G=32,
+R=128): flush the residual when it is full (once every 128 steps), append one new K/V token per
+(batch, KV head), and run decode attention for every query head over the whole cache.  After each
+128-step cycle the host moves n_quant back by one block, so the cache cycles between 8193 and 8320
+cached tokens instead of growing; every step does its full work.  Inputs live in HBM (1.2 GB of codes
+and scales per step, ten times the 126 MB L2, so no L2 flush is needed).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+N > 1 runs under torch.distributed.run, one rank per GPU, each rank its own batch (weak scaling,
+no collective on the data path); the time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from bit_asymmetric_kv_02_b200 import synth  # noqa: E402
+
+METRIC = "2-bit KV decode-attention cached tokens/s/head and HBM GB/s vs 8 TB/s peak (1 B200)"
+UNIT = "cached tokens/s/head"
+SPEC_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+WORKLOAD = synth.LARGE_BATCH
+DECODE_SOURCES = ["decode.cu", "common.cuh", "kernels.h"]
+
+
+# ------------------------------------------------------------------------------------------------
+# helpers
+# ------------------------------------------------------------------------------------------------
+def decode_kernel_sha() -> str:
+    h = hashlib.sha256()
+    for f in DECODE_SOURCES:
+        with open(os.path.join(ROOT, "bit_asymmetric_kv_02_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def hbm_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def profiled_traffic(w: synth.Workload):
+    """DRAM bytes per decode launch from the committed ncu summary, if it was taken on the current
+    kernel sources; else None."""
+    path = os.path.join(ROOT, "profiles", "decode_traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+    except Exception:
+        return None
+    if rec.get("kernel_sha") != decode_kernel_sha() or rec.get("workload") != w.name:
+        return None
+    return rec.get("bytes_per_launch")
+
+
+def decode_alg_bytes(w: synth.Workload, n_quant: int, n_res: int) -> int:
+    """Bytes decode attention must move at least once: codes, scales/zeros, residual rows, q, out."""
+    bh = w.batch * w.kv_heads
+    per_head = (2 * n_quant * w.head_dim * w.bits // 8                 # K and V codes
+                + (n_quant // w.residual) * (w.head_dim // w.group) * 4  # K scale + zero (fp16)
+                + (n_quant // w.group) * 4                               # V scale + zero
+                + n_res * w.head_dim * 4                                 # fp16 K and V residual rows
+                + 2 * w.gqa * w.head_dim * 2)                            # q in, out
+    return bh * per_head
+
+
+class ClockSampler:
+    """Samples SM clock, max clock and throttle reasons with NVML every 20 ms (falls back to
+    nvidia-smi) while the timed region runs."""
+
+    REASONS = {  # NVML clocks-event reason bits
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+        0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+        0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting",
+    }
+
+    def __init__(self, device_index: int):
+        self.samples = []
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._handle = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            import torch
+            bus = torch.cuda.get_device_properties(device_index).pci_bus_id
+            self._handle = pynvml.nvmlDeviceGetHandleByPciBusId(bus.encode() if isinstance(bus, str) else bus)
+            self._nv = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._handle, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self._handle = None
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self._handle, nv.NVML_CLOCK_SM)
+                reasons = nv.nvmlDeviceGetCurrentClocksEventReasons(self._handle)
+                util = nv.nvmlDeviceGetUtilizationRates(self._handle).gpu
+                self.samples.append((mhz, reasons, util))
+            except Exception:
+                pass
+            self._stop.wait(0.02)
+
+    def __enter__(self):
+        if self._handle is not None:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._handle is not None:
+            self._t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        loaded = [s for s in self.samples if not (s[1] & 0x1)] or self.samples
+        reasons = set()
+        for _, r, _ in loaded:
+            for bit, name in self.REASONS.items():
+                if r & bit and name != "gpu_idle":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(s[0] for s in loaded), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(reasons), "samples": len(loaded)}
+
+
+BAD_REASONS = {"hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown"}
+
+
+class Ranks:
+    """The plumbing bench.py needs from torch.distributed: barrier and max over ranks.  Works with
+    any backend (NCCL on GPUs, gloo in the CPU tests); world == 1 needs no process group."""
+
+    def __init__(self, dist=None, device=None):
+        self.dist = dist
+        self.device = device
+        self.world = dist.get_world_size() if dist is not None else 1
+        self.rank = dist.get_rank() if dist is not None else 0
+
+    def barrier(self):
+        if self.dist is not None:
+            if self.device is not None and self.device.type == "cuda":
+                self.dist.barrier(device_ids=[self.device.index])
+            else:
+                self.dist.barrier()
+
+    def max(self, *values: float):
+        if self.dist is None:
+            return values if len(values) > 1 else values[0]
+        import torch
+        t = torch.tensor(values, dtype=torch.float64, device=self.device)
+        self.dist.all_reduce(t, op=self.dist.ReduceOp.MAX)
+        out = tuple(float(x) for x in t.cpu())
+        return out if len(out) > 1 else out[0]
+
+
+def weak_scaling_value(world: int, tokens_per_rank: int, batch: int, t_max_ms: float) -> float:
+    """Whole-job cached tokens/s/head: every rank attends its own B sequences; a step counts B*T
+    tokens per head; the job time is the slowest rank's."""
+    return world * tokens_per_rank * batch / (t_max_ms / 1e3)
+
+
+# ------------------------------------------------------------------------------------------------
+# the GPU arm
+# ------------------------------------------------------------------------------------------------
+def make_state(w: synth.Workload, torch, kivi, device):
+    n_quant0 = (w.tokens - 1) // w.residual * w.residual      # 8064: the prompt leaves a full residual
+    capacity = n_quant0 + w.residual
+    k, v = synth.prompt_kv(w, w.tokens)
+    cache = kivi.KiviCache(w.batch, w.kv_heads, capacity, bits=w.bits, group_k=w.group, group_v=w.group,
+                           residual=w.residual, num_q_heads=w.q_heads, device=device)
+    kd = torch.from_numpy(k).to(device)
+    vd = torch.from_numpy(v).to(device)
+    cache.prefill(kd, vd)
+    torch.cuda.synchronize(device)
+    del kd, vd, k, v
+    torch.cuda.empty_cache()   # hand the 8.6 GB of prompt back: the decode loop holds ~1.3 GB
+    # per-step inputs for a cycle of 128 steps (new K/V rows and queries), resident in HBM
+    steps_in = []
+    for s in range(w.residual):
+        kn, vn = synth.new_kv(w, s + 1)
+        q = synth.queries(w, s + 1)
+        steps_in.append((kn, vn, q))
+    dev_in = [tuple(torch.from_numpy(a).to(device) for a in x) for x in steps_in]
+    torch.cuda.synchronize(device)
+    assert (cache.n_quant, cache.n_res) == (n_quant0, w.residual)
+    return cache, n_quant0, steps_in, dev_in
+
+
+def gpu_step(cache, n_quant0, w, inputs, out, stream, decode_events=None):
+    """One streaming decode step on device-resident inputs; returns (launches, cached tokens)."""
+    launches = 0
+    if cache.c.n_res == w.residual:
+        if cache.c.n_quant == n_quant0 + w.residual:
+            cache.c.n_quant = n_quant0     # end of a 128-step cycle: drop the newest block again
+        cache.flush(stream)
+        launches += 1
+    kn, vn, q = inputs
+    cache.append(kn, vn, stream)
+    launches += 1
+    if decode_events is not None:
+        decode_events[0].record(stream)
+    cache.attend(q, out=out, stream=stream, status=False)
+    if decode_events is not None:
+        decode_events[1].record(stream)
+    launches += 1
+    return launches, cache.c.n_quant + cache.c.n_res
+
+
+def run_gpu(args, rank, world, local_rank):
+    import torch
+    from bit_asymmetric_kv_02_b200 import kivi
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    kivi.load_library()
+    w = WORKLOAD
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=device)
+    ranks = Ranks(dist, device)
+
+    cache, n_quant0, host_in, dev_in = make_state(w, torch, kivi, device)
+    stream = torch.cuda.Stream(device)
+    out = torch.empty(w.batch, w.q_heads, w.head_dim, dtype=torch.float16, device=device)
+    R = w.residual
+
+    barrier = ranks.barrier
+
+    # ---- device-resident timing -------------------------------------------------------------
+    def timed_loop(K, W):
+        with torch.cuda.stream(stream):
+            for i in range(W):
+                gpu_step(cache, n_quant0, w, dev_in[i % R], out, stream)
+        stream.synchronize()
+        barrier()
+        torch.cuda.synchronize(device)
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        launches, tokens = 0, 0
+        bytes_decode = 0
+        with ClockSampler(local_rank) as clocks, torch.cuda.stream(stream):
+            e0.record(stream)
+            for i in range(K):
+                n_q, n_r = cache.c.n_quant, cache.c.n_res
+                lz, t = gpu_step(cache, n_quant0, w, dev_in[(W + i) % R], out, stream, ev[i])
+                launches += lz
+                tokens += t
+                n_q2 = cache.c.n_quant
+                bytes_decode += decode_alg_bytes(w, n_q2, t - n_q2)
+            e1.record(stream)
+            stream.synchronize()
+        torch.cuda.synchronize(device)
+        barrier()
+        ms = e0.elapsed_time(e1)
+        dec_ms = sum(a.elapsed_time(b) for a, b in ev)
+        return ms, dec_ms, launches, tokens, bytes_decode, clocks.summary()
+
+    ms, dec_ms, launches, tokens, bytes_decode, clk = timed_loop(args.steps, args.warmup)
+    if BAD_REASONS & set(clk["reasons"]):
+        ms, dec_ms, launches, tokens, bytes_decode, clk = timed_loop(args.steps, args.warmup)
+        clk["remeasured"] = True
+    t_max, dec_ms = ranks.max(ms, dec_ms)
+
+    # ---- end to end through the public API with host buffers ---------------------------------
+    pinned = [tuple(torch.from_numpy(a).pin_memory() for a in x) for x in host_in]
+    out_host = torch.empty(w.batch, w.q_heads, w.head_dim, dtype=torch.float16).pin_memory()
+    stage = [torch.empty_like(t) for t in dev_in[0]]
+    h2d = sum(t.numel() * t.element_size() for t in pinned[0])
+    d2h = out_host.numel() * out_host.element_size()
+
+    def e2e_loop(K):
+        barrier()
+        torch.cuda.synchronize(device)
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        toks = 0
+        with torch.cuda.stream(stream):
+            f0.record(stream)
+            for i in range(K):
+                src = pinned[i % R]
+                for d_, s_ in zip(stage, src):
+                    d_.copy_(s_, non_blocking=True)
+                _, t = gpu_step(cache, n_quant0, w, stage, out, stream)
+                toks += t
+                out_host.copy_(out, non_blocking=True)
+                stream.synchronize()      # the caller consumes the step's result
+            f1.record(stream)
+            stream.synchronize()
+        return f0.elapsed_time(f1), toks
+
+    e2e_steps = 0 if args.no_e2e else min(args.steps, 4 * R)
+    e2e_ms, e2e_tokens = e2e_loop(e2e_steps) if e2e_steps else (float("nan"), 0)
+    e2e_ms = ranks.max(e2e_ms)
+
+    result = None
+    if rank == 0:
+        K = args.steps
+        value = weak_scaling_value(world, tokens, w.batch, t_max)
+        peak, peak_kind = hbm_peak()
+        dec_avg_ms = dec_ms / K
+        achieved = (bytes_decode / K) / (dec_avg_ms / 1e3) / 1e9
+        traffic = profiled_traffic(w)
+        e2e_value = weak_scaling_value(world, e2e_tokens, w.batch, e2e_ms)
+        result = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
+            "ms_per_step": t_max / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "u2 codes x i8 limbs (dp4a, i32 acc), f32 softmax", "data": "synthetic",
+            "config": {
+                "workload": w.name, "batch": w.batch, "q_heads": w.q_heads, "kv_heads": w.kv_heads,
+                "head_dim": w.head_dim, "bits": w.bits, "group_k": w.group, "group_v": w.group,
+                "residual": w.residual, "cached_tokens": f"{n_quant0 + 1}-{n_quant0 + 2 * R} (128-step cycles)",
+                "step": "flush when full + append + decode attention",
+                "l2": "not flushed: inputs (1.2 GB per step) exceed the 126 MB L2",
+                "parallelism": f"weak: one independent batch per GPU x {world}",
+            },
+            "hbm_gbs_decode": achieved, "hbm_frac_of_8tbs": achieved / SPEC_HBM_GBS,
+            "decode_ms_avg": dec_avg_ms,
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "peak_kind": peak_kind, "traffic": traffic,
+                         "kernel": "decode_kernel<2,1>", "alg_bytes_per_launch": bytes_decode / K},
+            "clocks": clk,
+            "gpu_launches": launches,
+            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "steps": e2e_steps, "ms_per_step": e2e_ms / max(1, e2e_steps)},
+        }
+    if dist is not None:
+        ranks.barrier()
+        dist.destroy_process_group()
+    return result
+
+
+# ------------------------------------------------------------------------------------------------
+# the CPU oracle (cpu_baseline leg and --impl reference)
+# ------------------------------------------------------------------------------------------------
+def oracle_sample(w: synth.Workload, n_heads: int, n_steps: int, budget_s: float):
+    """Times the oracle as it stands on `n_heads` KV heads for up to `n_steps` decode steps each
+    (threads over heads).  Returns (value in tokens/s/head, cores, sample description, seconds)."""
+    import oracle.kivi_oracle as O
+    from concurrent.futures import ThreadPoolExecutor
+    R = w.residual
+    n_quant0 = (w.tokens - 1) // R * R
+    cap = n_quant0 + R
+    heads = [(b, h) for b in range(w.batch) for h in range(w.kv_heads)][:: max(1, (w.batch * w.kv_heads) // n_heads)]
+    heads = heads[:n_heads]
+    caches = {}
+    for (b, h) in heads:
+        hc = O.HeadCache(w.head_dim, w.bits, w.group, w.group, R, cap)
+        hc.prefill(synth.prompt_k(w, b, h, w.tokens), synth.prompt_v(w, b, h, w.tokens))
+        caches[(b, h)] = hc
+    scale = 1.0 / math.sqrt(w.head_dim)
+    cores = os.cpu_count() or 1
+    deadline = time.perf_counter() + budget_s
+
+    def run_head(bh):
+        b, h = bh
+        hc = caches[bh]
+        done, toks = 0, 0
+        for s in range(1, n_steps + 1):
+            if time.perf_counter() > deadline and done > 0:
+                break
+            if hc.n_res == R:
+                if hc.n_quant == n_quant0 + R:   # same 128-step cycle as the GPU arm
+                    hc.k_codes, hc.v_codes = hc.k_codes[:n_quant0], hc.v_codes[:n_quant0]
+                    hc.k_s, hc.k_z = hc.k_s[:n_quant0 // R], hc.k_z[:n_quant0 // R]
+                    hc.v_s, hc.v_z = hc.v_s[:n_quant0 // w.group], hc.v_z[:n_quant0 // w.group]
+                hc.flush()
+            hc.append(synth.new_k(w, b, h, s), synth.new_v(w, b, h, s))
+            q = np.stack([synth.query(w, b, h * w.gqa + g, s) for g in range(w.gqa)])
+            hc.attend(q, scale)
+            done += 1
+            toks += hc.n_quant + hc.n_res
+        return done, toks
+
+    t0 = time.perf_counter()
+    with ThreadPoolExecutor(cores) as ex:
+        res = list(ex.map(run_head, heads))
+    dt = time.perf_counter() - t0
+    head_steps = sum(r[0] for r in res)
+    tok = sum(r[1] for r in res)
+    sample = (f"oracle (numpy fp64) decode steps of {len(heads)} of {w.batch * w.kv_heads} KV heads of "
+              f"{w.name}: {head_steps} head-steps (flush when full + append + attention), "
+              f"{cores} threads over heads, {dt:.1f} s")
+    # A full step is B*H head-steps and counts B*T tokens per head, so a sample of head-steps with
+    # `tok` cached tokens in total gives tok / dt / H cached tokens/s/head.
+    return tok / dt / w.kv_heads, cores, sample, dt, head_steps
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    w = WORKLOAD
+    budget = max(5.0, min(60.0, 0.6 * args.steps + 5.0))
+    value, cores, sample, dt, hs = oracle_sample(w, n_heads=min(64, 2 * (os.cpu_count() or 1)),
+                                                 n_steps=max(1, args.steps), budget_s=budget)
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": None, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "batch": w.batch, "q_heads": w.q_heads, "kv_heads": w.kv_heads,
+                   "head_dim": w.head_dim, "bits": w.bits, "group_k": w.group, "group_v": w.group,
+                   "residual": w.residual, "step": "flush when full + append + decode attention"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2048)
+    ap.add_argument("--warmup", type=int, default=128)
+    ap.add_argument("--impl", choices=["kivi", "reference"], default="kivi")
+    ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing (profiling runs)")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end loop (profiling runs)")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", str(args.gpus if args.gpus == 1 else 1)))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        res = run_reference(args, rank, world)
+    else:
+        res = run_gpu(args, rank, world, local_rank)
+        if rank == 0 and world == 1 and not args.no_cpu_baseline:
+            value, cores, sample, dt, hs = oracle_sample(WORKLOAD, n_heads=min(64, 2 * (os.cpu_count() or 1)),
+                                                         n_steps=16, budget_s=25.0)
+            res["cpu_baseline"] = {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                                   "sample": sample}
+    if rank == 0 and res is not None:
+        print(json.dumps(res), flush=True)
+
+
+if __name__ == "__main__":
+    main()

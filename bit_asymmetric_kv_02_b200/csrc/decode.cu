@@ -1,0 +1,639 @@
+// Fused decode attention over the quantized KV cache plus its fp16 residual (sm_100a).
+//
+// Method: KIVI explainer page "ICML 2024論文解説: KIVI — チューニング不要のKVキャッシュ2bit非対称量子化",
+//   section 残差バッファ（Residual Buffer）, Attention equation:
+//     out = softmax(scale * q [D(K_quant); K_res]^T) [D(V_quant); V_res],  D(x^) = s x^ + z.
+//
+// Work decomposition (stream-K over warps).  Every (batch, KV head) is a sequence of equal-size
+// "units": quantized units of UT tokens (UT = 128 at 2 bits, 64 at 4 bits; 4 KB of K codes +
+// 4 KB of V codes) followed by residual units of 16 fp16 tokens (4 KB K + 4 KB V).  The global
+// unit sequence is cut into one contiguous range per warp, so the load is balanced to one unit
+// whatever the batch, head count or context length.  Each warp streams its range through two
+// 8 KB shared-memory stages filled by 1-D TMA bulk copies (cp.async.bulk, no multicast) and
+// completed on an mbarrier; every wait is bounded and reports KIVI_ERR_DEVICE_TIMEOUT.
+// A warp whose range covers a whole head writes the output directly; a head split over several
+// warps is merged (log-sum-exp) by the warp that arrives last on the head's atomic ticket, which
+// then resets the ticket to zero.  No warp ever waits for another.
+//
+// Arithmetic (CUDA cores, no tensor cores: one query row per head is a matrix-vector product).
+//   A6  logit_t = sum_c q_c (s_g code + z_g) = sum_c (q_c s_g) code_tc + sum_g z_g sum_{c in g} q_c.
+//       (q_c s_g) for one R-token block is turned into a 24-bit signed fixed-point integer split in
+//       three byte limbs; the codes are unpacked to bytes with one shift and masks, and dp4a forms
+//       byte dot products exactly in int32.  The block constant sum_g z_g q_g is added in fp32.
+//   A8  online softmax in base 2 (q pre-scaled by scale*log2 e), warp-shuffle max, lane-local sums.
+//   A9  o_c = sum_t (p_t s_g(t)) code_tc + sum_t p_t z_g(t): (p_t s_g(t)) is turned into 24-bit
+//       unsigned fixed point relative to the unit's largest value and dotted with the V codes by
+//       dp4a; the z term is the same for every channel and is kept as one scalar.
+//   A7/A9 residual rows: fp32 FMAs on the fp16 values.
+//   A10 merge of (m, l, Z, o) states: o / l with o += Z.
+// 24-bit limbs keep every product relative error below 2^-21, the integer sums are exact, and the
+// remaining error is fp32 rounding.
+#include <cstdint>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace kivi {
+
+namespace {
+
+constexpr int kWarps = 4;           // stream-K workers per CTA
+constexpr int kStageBytes = 8192;   // one unit: 4 KB K + 4 KB V
+constexpr int kHalfStage = 4096;
+constexpr int kResTokens = 16;      // tokens per residual unit
+constexpr unsigned kFull = 0xffffffffu;
+
+template <int G>
+struct __align__(128) WarpSmem {
+  uint8_t stage[2][kStageBytes];
+  uint4 qw[24];   // Q limbs: 96 words
+  uint4 pw[24];   // P limbs: 96 words
+  float qf[G][kHeadDim];
+  uint64_t bar[2];
+};
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(kFull, v, o));
+  return v;
+}
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(kFull, v, o);
+  return v;
+}
+__device__ __forceinline__ uint32_t comp(const uint4& v, int i) {
+  return i == 0 ? v.x : (i == 1 ? v.y : (i == 2 ? v.z : v.w));
+}
+__device__ __forceinline__ float combine_limbs(int hi, int mid, int lo) {
+  return fmaf(static_cast<float>(hi), 65536.f, fmaf(static_cast<float>(mid), 256.f, static_cast<float>(lo)));
+}
+
+// Largest worker whose range starts at or before unit u: start(x) = floor(U x / W).
+__device__ __forceinline__ long long worker_of(long long u, long long U, long long W) {
+  return ((u + 1) * W + U - 1) / U - 1;
+}
+
+template <int BITS, int G>
+struct Decoder {
+  static constexpr int P = 32 / BITS;            // codes per word
+  static constexpr int UT = BITS == 2 ? 128 : 64; // tokens per quantized unit
+  static constexpr int TPL = UT / 32;             // tokens per lane (K side)
+  static constexpr int WPT = kHeadDim / P;        // K words per token
+  static constexpr int ROWS = UT / P;             // V word rows per unit (8)
+
+  const DecodeArgs& a;
+  WarpSmem<G>& S;
+  const int lane;
+  const long long worker, ub, ue;
+  const int ngk;  // K groups per head (d / G_k)
+
+  // per-head state
+  float qreg[G][4];
+  float qsum[G][4];
+  float m[G], l[G], Z[G], o[G][4];
+
+  __device__ Decoder(const DecodeArgs& args, WarpSmem<G>& smem, int ln, long long w, long long b, long long e)
+      : a(args), S(smem), lane(ln), worker(w), ub(b), ue(e), ngk(kHeadDim / args.group_k) {}
+
+  // ---- unit addressing ------------------------------------------------------------------
+  __device__ void issue(long long u, int stage) {  // lane 0 only
+    const long long head = u / a.units;
+    const int local = static_cast<int>(u % a.units);
+    uint8_t* dst = S.stage[stage];
+    const void *ks, *vs;
+    if (local < a.units_q) {
+      const size_t tok0 = static_cast<size_t>(local) * UT;
+      ks = a.k_codes + (static_cast<size_t>(head) * a.capacity + tok0) * WPT;
+      vs = a.v_codes + (static_cast<size_t>(head) * (a.capacity / P) + tok0 / P) * kHeadDim;
+    } else {
+      const size_t t0 = static_cast<size_t>(local - a.units_q) * kResTokens;
+      ks = a.k_res + (static_cast<size_t>(head) * a.residual + t0) * kHeadDim;
+      vs = a.v_res + (static_cast<size_t>(head) * a.residual + t0) * kHeadDim;
+    }
+    mbar_arrive_expect_tx(&S.bar[stage], kStageBytes + a.debug_extra_tx);
+    bulk_g2s(dst, ks, kHalfStage, &S.bar[stage]);
+    bulk_g2s(dst + kHalfStage, vs, kHalfStage, &S.bar[stage]);
+  }
+
+  // (s, z) pairs of a quantized unit: lanes [0, ngk) hold K groups, lanes [8, 8 + nvg) V groups.
+  __device__ uint32_t load_pairs(long long u) const {
+    const long long head = u / a.units;
+    const int local = static_cast<int>(u % a.units);
+    if (local >= a.units_q) return 0u;
+    const int tok0 = local * UT;
+    if (lane < ngk) {
+      const size_t i = (static_cast<size_t>(head) * (a.capacity / a.residual) + tok0 / a.residual) * ngk + lane;
+      return static_cast<uint32_t>(__ldg(a.k_scale + i)) | (static_cast<uint32_t>(__ldg(a.k_zero + i)) << 16);
+    }
+    const int nvg = UT >= a.group_v ? UT / a.group_v : 1;
+    if (lane >= 8 && lane < 8 + nvg) {
+      const size_t i = static_cast<size_t>(head) * (a.capacity / a.group_v) + tok0 / a.group_v + (lane - 8);
+      return static_cast<uint32_t>(__ldg(a.v_scale + i)) | (static_cast<uint32_t>(__ldg(a.v_zero + i)) << 16);
+    }
+    return 0u;
+  }
+
+  // ---- per-head state ---------------------------------------------------------------------
+  __device__ void start_head(long long head) {
+    __syncwarp();
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      const uint16_t* qp = a.q + (static_cast<size_t>(head) * G + g) * kHeadDim;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float v = h2f(__ldg(qp + lane + 32 * j)) * a.qscale;
+        qreg[g][j] = v;
+        S.qf[g][lane + 32 * j] = v;
+      }
+#pragma unroll
+      for (int gi = 0; gi < 4; ++gi) {
+        float part = 0.f;
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          if ((32 * j) / a.group_k == gi) part += qreg[g][j];
+        qsum[g][gi] = gi < ngk ? warp_sum(part) : 0.f;
+      }
+      m[g] = -INFINITY;
+      l[g] = 0.f;
+      Z[g] = 0.f;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) o[g][e] = 0.f;
+    }
+    __syncwarp();
+  }
+
+  // ---- one quantized unit -------------------------------------------------------------------
+  __device__ void quantized_unit(int stage, int tok0, uint32_t pairs) {
+    const uint8_t* kt = S.stage[stage];
+    const uint8_t* vt = S.stage[stage] + kHalfStage;
+    uint8_t* qwb = reinterpret_cast<uint8_t*>(S.qw);
+    uint8_t* pwb = reinterpret_cast<uint8_t*>(S.pw);
+    (void)tok0;
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      // -- A6: fixed-point limbs of q_c * s_g(c) for this block
+      float qv[4], mabs = 0.f;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int gi = (32 * j) / a.group_k;
+        const float s = h2f(static_cast<uint16_t>(__shfl_sync(kFull, pairs, gi) & 0xFFFFu));
+        qv[j] = qreg[g][j] * s;
+        mabs = fmaxf(mabs, fabsf(qv[j]));
+      }
+      mabs = warp_max(mabs);
+      const float scq = mabs > 0.f ? 8388607.f / mabs : 0.f;
+      const float invq = mabs > 0.f ? mabs / 8388607.f : 0.f;
+      float cblk = 0.f;
+#pragma unroll
+      for (int gi = 0; gi < 4; ++gi) {
+        if (gi < ngk) {
+          const float z = h2f(static_cast<uint16_t>(__shfl_sync(kFull, pairs, gi) >> 16));
+          cblk = fmaf(z, qsum[g][gi], cblk);
+        }
+      }
+      __syncwarp();
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int c = lane + 32 * j;
+        int word, k;
+        float f = qv[j] * scq;
+        if (BITS == 2) {  // word i = c/16, set k = c%4 (odd sets read as 4*code), byte m = (c%16)/4
+          k = c & 3;
+          word = c >> 4;
+          if (k & 1) f *= 0.25f;
+        } else {          // word i = c/8, set k = c%2, byte m = (c%8)/2
+          k = c & 1;
+          word = c >> 3;
+        }
+        const int mb = BITS == 2 ? ((c >> 2) & 3) : ((c >> 1) & 3);
+        const int Q = __float2int_rn(f);
+        const int nset = BITS == 2 ? 4 : 2;
+        uint8_t* base = qwb + ((word * 3) * nset + k) * 4 + mb;
+        base[0] = static_cast<uint8_t>(Q & 255);
+        base[nset * 4] = static_cast<uint8_t>((Q >> 8) & 255);
+        base[2 * nset * 4] = static_cast<uint8_t>((Q >> 16) & 255);
+      }
+      __syncwarp();
+
+      int al[TPL], am[TPL], ah[TPL];
+#pragma unroll
+      for (int j = 0; j < TPL; ++j) al[j] = am[j] = ah[j] = 0;
+      if (BITS == 2) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int hh = h ^ ((lane >> 2) & 1);  // bank-conflict-free order of the two 16-byte halves
+          uint4 kw[TPL];
+#pragma unroll
+          for (int j = 0; j < TPL; ++j)
+            kw[j] = *reinterpret_cast<const uint4*>(kt + (lane + 32 * j) * 32 + 16 * hh);
+#pragma unroll
+          for (int ii = 0; ii < 4; ++ii) {
+            const int i = 4 * hh + ii;
+            const uint4 QL = S.qw[i * 3 + 0], QM = S.qw[i * 3 + 1], QH = S.qw[i * 3 + 2];
+#pragma unroll
+            for (int j = 0; j < TPL; ++j) {
+              const uint32_t w = comp(kw[j], ii);
+              const uint32_t w4 = w >> 4;
+              const uint32_t m0 = w & 0x03030303u, m1 = w & 0x0C0C0C0Cu;
+              const uint32_t m2 = w4 & 0x03030303u, m3 = w4 & 0x0C0C0C0Cu;
+              al[j] = dp4a_uu(m0, QL.x, al[j]);
+              am[j] = dp4a_uu(m0, QM.x, am[j]);
+              ah[j] = dp4a_us(m0, QH.x, ah[j]);
+              al[j] = dp4a_uu(m1, QL.y, al[j]);
+              am[j] = dp4a_uu(m1, QM.y, am[j]);
+              ah[j] = dp4a_us(m1, QH.y, ah[j]);
+              al[j] = dp4a_uu(m2, QL.z, al[j]);
+              am[j] = dp4a_uu(m2, QM.z, am[j]);
+              ah[j] = dp4a_us(m2, QH.z, ah[j]);
+              al[j] = dp4a_uu(m3, QL.w, al[j]);
+              am[j] = dp4a_uu(m3, QM.w, am[j]);
+              ah[j] = dp4a_us(m3, QH.w, ah[j]);
+            }
+          }
+        }
+      } else {
+        const uint2* qw2 = reinterpret_cast<const uint2*>(S.qw);
+#pragma unroll
+        for (int qq = 0; qq < 4; ++qq) {
+          const int cq = (qq + (lane >> 1)) & 3;  // bank-conflict-free chunk order
+          uint4 kw[TPL];
+#pragma unroll
+          for (int j = 0; j < TPL; ++j)
+            kw[j] = *reinterpret_cast<const uint4*>(kt + (lane + 32 * j) * 64 + 16 * cq);
+#pragma unroll
+          for (int ii = 0; ii < 4; ++ii) {
+            const int i = 4 * cq + ii;
+            const uint2 QL = qw2[i * 3 + 0], QM = qw2[i * 3 + 1], QH = qw2[i * 3 + 2];
+#pragma unroll
+            for (int j = 0; j < TPL; ++j) {
+              const uint32_t w = comp(kw[j], ii);
+              const uint32_t n0 = w & 0x0F0F0F0Fu, n1 = (w >> 4) & 0x0F0F0F0Fu;
+              al[j] = dp4a_uu(n0, QL.x, al[j]);
+              am[j] = dp4a_uu(n0, QM.x, am[j]);
+              ah[j] = dp4a_us(n0, QH.x, ah[j]);
+              al[j] = dp4a_uu(n1, QL.y, al[j]);
+              am[j] = dp4a_uu(n1, QM.y, am[j]);
+              ah[j] = dp4a_us(n1, QH.y, ah[j]);
+            }
+          }
+        }
+      }
+
+      // -- A8: online softmax over the unit's UT tokens
+      float lg[TPL], mu = -INFINITY;
+#pragma unroll
+      for (int j = 0; j < TPL; ++j) {
+        lg[j] = fmaf(combine_limbs(ah[j], am[j], al[j]), invq, cblk);
+        mu = fmaxf(mu, lg[j]);
+      }
+      mu = warp_max(mu);
+      const float m_new = fmaxf(m[g], mu);
+      const float alpha = exp2f(m[g] - m_new);
+      float psum = 0.f, zsum = 0.f, mv = 0.f, pp[TPL];
+#pragma unroll
+      for (int j = 0; j < TPL; ++j) {
+        const int vg = (32 * j) / a.group_v;  // V group of token lane + 32 j within the unit
+        const uint32_t vp = __shfl_sync(kFull, pairs, 8 + (UT >= a.group_v ? vg : 0));
+        const float p = exp2f(lg[j] - m_new);
+        psum += p;
+        zsum = fmaf(p, h2f(static_cast<uint16_t>(vp >> 16)), zsum);
+        pp[j] = p * h2f(static_cast<uint16_t>(vp & 0xFFFFu));
+        mv = fmaxf(mv, pp[j]);
+      }
+      mv = warp_max(mv);
+      m[g] = m_new;
+      l[g] = fmaf(l[g], alpha, psum);
+      Z[g] = fmaf(Z[g], alpha, zsum);
+
+      // -- A9: fixed-point limbs of p_t * s_g(t), then the V codes
+      if (mv > 0.f) {
+        const float scv = 16777215.f / mv;
+        const float invv = mv / 16777215.f;
+#pragma unroll
+        for (int j = 0; j < TPL; ++j) {
+          const int t = lane + 32 * j;
+          int row, k, mb;
+          float f = pp[j] * scv;
+          if (BITS == 2) {
+            row = t >> 4;
+            k = t & 3;
+            mb = (t >> 2) & 3;
+            if (k & 1) f *= 0.25f;
+          } else {
+            row = t >> 3;
+            k = t & 1;
+            mb = (t >> 1) & 3;
+          }
+          const uint32_t Pq = __float2uint_rn(f);
+          const int nset = BITS == 2 ? 4 : 2;
+          uint8_t* base = pwb + ((row * 3) * nset + k) * 4 + mb;
+          base[0] = static_cast<uint8_t>(Pq & 255u);
+          base[nset * 4] = static_cast<uint8_t>((Pq >> 8) & 255u);
+          base[2 * nset * 4] = static_cast<uint8_t>((Pq >> 16) & 255u);
+        }
+        __syncwarp();
+        int vl[4] = {0, 0, 0, 0}, vm[4] = {0, 0, 0, 0}, vh[4] = {0, 0, 0, 0};
+#pragma unroll
+        for (int r = 0; r < ROWS; ++r) {
+          const uint4 vw = *reinterpret_cast<const uint4*>(vt + r * 512 + 16 * lane);
+          if (BITS == 2) {
+            const uint4 PL = S.pw[r * 3 + 0], PM = S.pw[r * 3 + 1], PH = S.pw[r * 3 + 2];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const uint32_t w = comp(vw, e);
+              const uint32_t w4 = w >> 4;
+              const uint32_t m0 = w & 0x03030303u, m1 = w & 0x0C0C0C0Cu;
+              const uint32_t m2 = w4 & 0x03030303u, m3 = w4 & 0x0C0C0C0Cu;
+              vl[e] = dp4a_uu(m0, PL.x, vl[e]);
+              vm[e] = dp4a_uu(m0, PM.x, vm[e]);
+              vh[e] = dp4a_uu(m0, PH.x, vh[e]);
+              vl[e] = dp4a_uu(m1, PL.y, vl[e]);
+              vm[e] = dp4a_uu(m1, PM.y, vm[e]);
+              vh[e] = dp4a_uu(m1, PH.y, vh[e]);
+              vl[e] = dp4a_uu(m2, PL.z, vl[e]);
+              vm[e] = dp4a_uu(m2, PM.z, vm[e]);
+              vh[e] = dp4a_uu(m2, PH.z, vh[e]);
+              vl[e] = dp4a_uu(m3, PL.w, vl[e]);
+              vm[e] = dp4a_uu(m3, PM.w, vm[e]);
+              vh[e] = dp4a_uu(m3, PH.w, vh[e]);
+            }
+          } else {
+            const uint2* pw2 = reinterpret_cast<const uint2*>(S.pw);
+            const uint2 PL = pw2[r * 3 + 0], PM = pw2[r * 3 + 1], PH = pw2[r * 3 + 2];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const uint32_t w = comp(vw, e);
+              const uint32_t n0 = w & 0x0F0F0F0Fu, n1 = (w >> 4) & 0x0F0F0F0Fu;
+              vl[e] = dp4a_uu(n0, PL.x, vl[e]);
+              vm[e] = dp4a_uu(n0, PM.x, vm[e]);
+              vh[e] = dp4a_uu(n0, PH.x, vh[e]);
+              vl[e] = dp4a_uu(n1, PL.y, vl[e]);
+              vm[e] = dp4a_uu(n1, PM.y, vm[e]);
+              vh[e] = dp4a_uu(n1, PH.y, vh[e]);
+            }
+          }
+        }
+#pragma unroll
+        for (int e = 0; e < 4; ++e) o[g][e] = fmaf(o[g][e], alpha, combine_limbs(vh[e], vm[e], vl[e]) * invv);
+      } else {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) o[g][e] *= alpha;
+      }
+      __syncwarp();  // qw / pw are rewritten by the next query or unit
+    }
+  }
+
+  // ---- one residual unit (fp16 rows) --------------------------------------------------------
+  __device__ void residual_unit(int stage, int nvalid) {
+    const uint8_t* kt = S.stage[stage];
+    const uint8_t* vt = S.stage[stage] + kHalfStage;
+    const int t = lane >> 1, hf = lane & 1;
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      float dot = 0.f;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const int cc = (k + lane) & 7;  // bank-conflict-free chunk order
+        const uint4 kv = *reinterpret_cast<const uint4*>(kt + t * 256 + hf * 128 + 16 * cc);
+        const float4 q0 = *reinterpret_cast<const float4*>(&S.qf[g][64 * hf + 8 * cc]);
+        const float4 q1 = *reinterpret_cast<const float4*>(&S.qf[g][64 * hf + 8 * cc + 4]);
+        const float2 k0 = __half22float2(*reinterpret_cast<const __half2*>(&kv.x));
+        const float2 k1 = __half22float2(*reinterpret_cast<const __half2*>(&kv.y));
+        const float2 k2 = __half22float2(*reinterpret_cast<const __half2*>(&kv.z));
+        const float2 k3 = __half22float2(*reinterpret_cast<const __half2*>(&kv.w));
+        dot = fmaf(q0.x, k0.x, dot);
+        dot = fmaf(q0.y, k0.y, dot);
+        dot = fmaf(q0.z, k1.x, dot);
+        dot = fmaf(q0.w, k1.y, dot);
+        dot = fmaf(q1.x, k2.x, dot);
+        dot = fmaf(q1.y, k2.y, dot);
+        dot = fmaf(q1.z, k3.x, dot);
+        dot = fmaf(q1.w, k3.y, dot);
+      }
+      dot += __shfl_xor_sync(kFull, dot, 1);
+      const bool valid = t < nvalid;
+      const float lg = valid ? dot : -INFINITY;
+      const float m_new = fmaxf(m[g], warp_max(lg));
+      const float alpha = exp2f(m[g] - m_new);
+      const float p = valid ? exp2f(lg - m_new) : 0.f;
+      m[g] = m_new;
+      l[g] = fmaf(l[g], alpha, hf == 0 ? p : 0.f);
+      Z[g] *= alpha;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) o[g][e] *= alpha;
+#pragma unroll 4
+      for (int tt = 0; tt < nvalid; ++tt) {
+        const float pt = __shfl_sync(kFull, p, 2 * tt);
+        const uint2 vv = *reinterpret_cast<const uint2*>(vt + tt * 256 + 8 * lane);
+        const float2 v0 = __half22float2(*reinterpret_cast<const __half2*>(&vv.x));
+        const float2 v1 = __half22float2(*reinterpret_cast<const __half2*>(&vv.y));
+        o[g][0] = fmaf(pt, v0.x, o[g][0]);
+        o[g][1] = fmaf(pt, v0.y, o[g][1]);
+        o[g][2] = fmaf(pt, v1.x, o[g][2]);
+        o[g][3] = fmaf(pt, v1.y, o[g][3]);
+      }
+    }
+  }
+
+  // ---- end of a head segment: write the output, or a partial and maybe merge ----------------
+  __device__ void finish_segment(long long head, long long seg_a, long long seg_b) {
+    const long long h0 = head * a.units, h1 = h0 + a.units;
+    float lsum[G], zsum[G];
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      lsum[g] = warp_sum(l[g]);
+      zsum[g] = warp_sum(Z[g]);
+    }
+    if (seg_a == h0 && seg_b == h1) {
+#pragma unroll
+      for (int g = 0; g < G; ++g) store_out(head, g, o[g], zsum[g], 1.f / lsum[g]);
+      return;
+    }
+    const int slot = seg_a == ub ? 0 : 1;
+    float* mine = a.partials + ((worker * 2 + slot) * G) * kPartialStride;
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      float* p = mine + g * kPartialStride;
+      if (lane == 0) {
+        p[0] = m[g];
+        p[1] = lsum[g];
+        p[2] = zsum[g];
+      }
+      *reinterpret_cast<float4*>(p + 4 + 4 * lane) = make_float4(o[g][0], o[g][1], o[g][2], o[g][3]);
+    }
+    __threadfence();  // every lane publishes its own slice of the partial before the ticket
+    __syncwarp();
+    const long long W = a.workers, U = a.total_units;
+    const long long wfirst = worker_of(h0, U, W), wlast = worker_of(h1 - 1, U, W);
+    int last = 0;
+    if (lane == 0) {
+      const int ticket = atomicAdd(a.tickets + head, 1);
+      last = ticket == static_cast<int>(wlast - wfirst);
+    }
+    last = __shfl_sync(kFull, last, 0);
+    if (!last) return;
+    __threadfence();
+#pragma unroll 1
+    for (int g = 0; g < G; ++g) {
+      float mm = -INFINITY;
+      for (long long x = wfirst; x <= wlast; ++x) {
+        const int sx = (U * x / W) >= h0 ? 0 : 1;
+        mm = fmaxf(mm, __ldcg(a.partials + ((x * 2 + sx) * G + g) * kPartialStride));
+      }
+      float ls = 0.f, zs = 0.f, acc[4] = {0.f, 0.f, 0.f, 0.f};
+      for (long long x = wfirst; x <= wlast; ++x) {
+        const int sx = (U * x / W) >= h0 ? 0 : 1;
+        const float* p = a.partials + ((x * 2 + sx) * G + g) * kPartialStride;
+        const float w = exp2f(__ldcg(p) - mm);
+        ls = fmaf(w, __ldcg(p + 1), ls);
+        zs = fmaf(w, __ldcg(p + 2), zs);
+        const float4 ov = __ldcg(reinterpret_cast<const float4*>(p + 4 + 4 * lane));
+        acc[0] = fmaf(w, ov.x, acc[0]);
+        acc[1] = fmaf(w, ov.y, acc[1]);
+        acc[2] = fmaf(w, ov.z, acc[2]);
+        acc[3] = fmaf(w, ov.w, acc[3]);
+      }
+      store_out(head, g, acc, zs, 1.f / ls);
+    }
+    if (lane == 0) a.tickets[head] = 0;
+  }
+
+  __device__ void store_out(long long head, int g, const float* acc, float z, float inv_l) const {
+    __half2 h01 = __floats2half2_rn((acc[0] + z) * inv_l, (acc[1] + z) * inv_l);
+    __half2 h23 = __floats2half2_rn((acc[2] + z) * inv_l, (acc[3] + z) * inv_l);
+    uint2 v;
+    v.x = *reinterpret_cast<uint32_t*>(&h01);
+    v.y = *reinterpret_cast<uint32_t*>(&h23);
+    *reinterpret_cast<uint2*>(a.out + (static_cast<size_t>(head) * G + g) * kHeadDim + 4 * lane) = v;
+  }
+
+  // all lanes wait; the decision is made warp-uniform
+  __device__ bool wait_stage(int stage, uint32_t parity) {
+    const bool ok = mbar_wait_bounded(&S.bar[stage], parity, a.timeout_ns);
+    return __all_sync(kFull, ok);
+  }
+
+  // After a timeout: wait (bounded by max(timeout, 1 s)) until the bytes of a copy have landed.
+  __device__ void drain(int stage, uint32_t parity) {
+    const unsigned long long lim = a.timeout_ns > 1000000000ull ? a.timeout_ns : 1000000000ull;
+    (void)mbar_wait_bounded(&S.bar[stage], parity, lim);
+    __syncwarp();
+  }
+
+  __device__ void run() {
+    if (lane == 0) {
+      mbar_init(&S.bar[0], 1);
+      mbar_init(&S.bar[1], 1);
+      asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncwarp();
+    if (lane == 0) {
+      issue(ub, 0);
+      if (ub + 1 < ue) issue(ub + 1, 1);
+    }
+    uint32_t pairs = load_pairs(ub);
+    long long cur_head = -1, seg_a = ub;
+    int it = 0;
+    for (long long u = ub; u < ue; ++u, ++it) {
+      const int stage = it & 1;
+      const uint32_t parity = (it >> 1) & 1;
+      const long long head = u / a.units;
+      const int local = static_cast<int>(u % a.units);
+      if (head != cur_head) {
+        if (cur_head >= 0) finish_segment(cur_head, seg_a, u);
+        start_head(head);
+        cur_head = head;
+        seg_a = u;
+      }
+      const uint32_t pairs_next = (u + 1 < ue) ? load_pairs(u + 1) : 0u;
+      if (!wait_stage(stage, parity)) {
+        // Give up: record the error, let this warp's copies in flight land, and leave.
+        if (lane == 0) report_status(a.status, KIVI_ERR_DEVICE_TIMEOUT);
+        drain(stage, parity);
+        if (u + 1 < ue) drain(stage ^ 1, ((it + 1) >> 1) & 1);
+        return;
+      }
+      if (local < a.units_q) {
+        quantized_unit(stage, local * UT, pairs);
+      } else {
+        const int t0 = (local - a.units_q) * kResTokens;
+        residual_unit(stage, min(kResTokens, a.n_res - t0));
+      }
+      __syncwarp();
+      fence_proxy_async_smem();
+      if (lane == 0 && u + 2 < ue) issue(u + 2, stage);
+      pairs = pairs_next;
+    }
+    finish_segment(cur_head, seg_a, ue);
+  }
+};
+
+template <int BITS, int G>
+__global__ void __launch_bounds__(kWarps * 32) decode_kernel(const __grid_constant__ DecodeArgs a) {
+  extern __shared__ __align__(128) uint8_t smem_raw[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  WarpSmem<G>& S = reinterpret_cast<WarpSmem<G>*>(smem_raw)[warp];
+  const long long W = a.workers, U = a.total_units;
+  const long long worker = static_cast<long long>(blockIdx.x) * kWarps + warp;
+  if (worker >= W) return;  // the last CTA may hold fewer workers
+  const long long ub = U * worker / W, ue = U * (worker + 1) / W;  // non-empty because W <= U
+  Decoder<BITS, G> d(a, S, lane, worker, ub, ue);
+  d.run();
+}
+
+template <int BITS, int G>
+cudaError_t plan_for(DecodePlan* plan) {
+  const int smem = kWarps * static_cast<int>(sizeof(WarpSmem<G>));
+  cudaError_t e = cudaFuncSetAttribute(decode_kernel<BITS, G>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  int dev = 0, sms = 0, occ = 0;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+  if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+  if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, decode_kernel<BITS, G>, kWarps * 32, smem)) !=
+      cudaSuccess)
+    return e;
+  if (occ < 1) return cudaErrorInvalidConfiguration;
+  plan->warps_per_cta = kWarps;
+  plan->ctas = sms * occ;
+  plan->smem_bytes = smem;
+  return cudaSuccess;
+}
+
+template <int BITS, int G>
+cudaError_t launch_for(const DecodeArgs& a, const DecodePlan& plan, cudaStream_t stream) {
+  if (a.workers < 1 || a.workers > plan.workers() || a.total_units < a.workers) return cudaErrorInvalidValue;
+  const int ctas = (a.workers + plan.warps_per_cta - 1) / plan.warps_per_cta;
+  decode_kernel<BITS, G><<<ctas, plan.warps_per_cta * 32, plan.smem_bytes, stream>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+#define KIVI_DISPATCH(BITS_, GQA_, FN, ...)                              \
+  do {                                                                   \
+    if ((BITS_) == 2) {                                                  \
+      switch (GQA_) {                                                    \
+        case 1: return FN<2, 1>(__VA_ARGS__);                            \
+        case 2: return FN<2, 2>(__VA_ARGS__);                            \
+        case 4: return FN<2, 4>(__VA_ARGS__);                            \
+        case 8: return FN<2, 8>(__VA_ARGS__);                            \
+      }                                                                  \
+    } else if ((BITS_) == 4) {                                           \
+      switch (GQA_) {                                                    \
+        case 1: return FN<4, 1>(__VA_ARGS__);                            \
+        case 2: return FN<4, 2>(__VA_ARGS__);                            \
+        case 4: return FN<4, 4>(__VA_ARGS__);                            \
+        case 8: return FN<4, 8>(__VA_ARGS__);                            \
+      }                                                                  \
+    }                                                                    \
+    return cudaErrorInvalidValue;                                        \
+  } while (0)
+
+cudaError_t decode_plan(int bits, int gqa, DecodePlan* plan) { KIVI_DISPATCH(bits, gqa, plan_for, plan); }
+
+cudaError_t launch_decode(const DecodeArgs& a, int bits, const DecodePlan& plan, cudaStream_t stream) {
+  KIVI_DISPATCH(bits, a.gqa, launch_for, a, plan, stream);
+}
+
+}  // namespace kivi

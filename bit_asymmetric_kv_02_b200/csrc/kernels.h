@@ -1,0 +1,72 @@
+// Launch arguments of the library's kernels (host <-> device, plain data).
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace kivi {
+
+// Quantize `nblocks` R-token blocks of K and V per (batch, KV head) and optionally copy a tail
+// into the residual.  Source tensors are fp16 [bh][src_tokens][128]; block j reads tokens
+// src_tok0 + j*R .. and is written as quantized block dst_blk0 + j.
+struct QuantizeArgs {
+  const uint16_t* k_src;
+  const uint16_t* v_src;
+  uint32_t* k_codes;
+  uint32_t* v_codes;
+  uint16_t *k_scale, *k_zero, *v_scale, *v_zero;
+  uint16_t *k_res, *v_res;
+  int bh;          // batch * kv_heads
+  int src_tokens;  // tokens per head in the source tensors
+  int src_tok0;    // first source token of block 0
+  int nblocks;     // blocks to quantize per head
+  int dst_blk0;    // destination block index of block 0
+  int res_tok0;    // first source token copied into residual slot 0
+  int res_tokens;  // tokens copied into the residual (0: none)
+  int residual, capacity, group_k, group_v;
+};
+
+struct AppendArgs {
+  const uint16_t* k_new;
+  const uint16_t* v_new;
+  uint16_t *k_res, *v_res;
+  int bh, residual, slot;
+};
+
+struct DecodeArgs {
+  const uint32_t* k_codes;
+  const uint32_t* v_codes;
+  const uint16_t *k_scale, *k_zero, *v_scale, *v_zero;
+  const uint16_t *k_res, *v_res;
+  const uint16_t* q;
+  uint16_t* out;
+  float* partials;    // [workers][2][gqa][kPartialStride]
+  int32_t* tickets;   // [bh], zero between calls
+  int32_t* status;    // optional device status word
+  int bh, gqa, capacity, residual, group_k, group_v;
+  int n_quant, n_res;
+  int units_q;        // quantized units per head
+  int units;          // units per head (quantized + residual)
+  long long total_units;
+  int workers;
+  float qscale;       // softmax scale * log2(e)
+  unsigned long long timeout_ns;
+  uint32_t debug_extra_tx;  // test hook: bytes a barrier expects beyond the copy (0 normally)
+};
+
+constexpr int kPartialStride = 132;  // m, l, Z, pad, o[128]
+
+cudaError_t launch_quantize_blocks(const QuantizeArgs& a, int bits, cudaStream_t stream);
+cudaError_t launch_append(const AppendArgs& a, cudaStream_t stream);
+
+// Decode launch plan: warps per CTA, CTAs, dynamic shared memory.
+struct DecodePlan {
+  int warps_per_cta;
+  int ctas;
+  int smem_bytes;
+  int workers() const { return warps_per_cta * ctas; }
+};
+cudaError_t decode_plan(int bits, int gqa, DecodePlan* plan);
+cudaError_t launch_decode(const DecodeArgs& a, int bits, const DecodePlan& plan, cudaStream_t stream);
+
+}  // namespace kivi

@@ -1,0 +1,325 @@
+// C ABI of the library (include/kivi.h): argument checks, cache counters, launch plans.
+// Host code only; every computation runs in the kernels of quantize.cu and decode.cu.
+#include <cstdint>
+#include <cstdlib>
+#include <mutex>
+
+#include <cuda_runtime.h>
+
+#include "kernels.h"
+#include "kivi.h"
+
+namespace {
+
+using kivi::DecodeArgs;
+using kivi::DecodePlan;
+
+constexpr int kHeadDim = 128;
+constexpr unsigned long long kDefaultTimeoutNs = 2000000000ull;  // 2 s per bounded device wait
+
+struct DebugState {
+  std::mutex mu;
+  int mode = 0;
+  unsigned long long timeout_ns = kDefaultTimeoutNs;
+};
+DebugState& debug_state() {
+  static DebugState s;
+  return s;
+}
+
+bool aligned16(const void* p) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+int unit_tokens(int bits) { return bits == 2 ? 128 : 64; }
+
+int check_cfg(const kivi_config* c) {
+  if (c == nullptr) return KIVI_ERR_INVALID_ARG;
+  if (c->head_dim != kHeadDim) return KIVI_ERR_UNSUPPORTED;
+  if (c->bits != 2 && c->bits != 4) return KIVI_ERR_UNSUPPORTED;
+  if (c->batch < 1 || c->num_kv_heads < 1 || c->capacity < 0) return KIVI_ERR_INVALID_ARG;
+  if (c->residual < 128 || c->residual > 1024 || c->residual % 128 != 0) return KIVI_ERR_INVALID_ARG;
+  if (c->capacity % c->residual != 0) return KIVI_ERR_INVALID_ARG;
+  if (c->group_k != 32 && c->group_k != 64 && c->group_k != 128) return KIVI_ERR_INVALID_ARG;
+  if (c->group_v < 32 || c->group_v % 32 != 0 || c->residual % c->group_v != 0) return KIVI_ERR_INVALID_ARG;
+  if (static_cast<long long>(c->batch) * c->num_kv_heads > (1ll << 30)) return KIVI_ERR_UNSUPPORTED;
+  if (c->capacity / c->residual > 32767) return KIVI_ERR_UNSUPPORTED;  // grid.y limit of a prefill
+  return KIVI_OK;
+}
+
+int check_state(const kivi_config* c, const kivi_cache* k) {
+  if (k == nullptr) return KIVI_ERR_INVALID_ARG;
+  if (k->n_quant < 0 || k->n_quant % c->residual != 0 || k->n_quant > c->capacity) return KIVI_ERR_STATE;
+  if (k->n_res < 0 || k->n_res > c->residual) return KIVI_ERR_STATE;
+  return KIVI_OK;
+}
+
+bool cache_ptrs_ok(const kivi_cache* k, bool need_codes) {
+  if (!aligned16(k->k_res) || !aligned16(k->v_res)) return false;
+  if (!need_codes) return true;
+  return aligned16(k->k_codes) && aligned16(k->v_codes) && aligned16(k->k_scale) && aligned16(k->k_zero) &&
+         aligned16(k->v_scale) && aligned16(k->v_zero);
+}
+
+// Decode plans are cached per (device, bits, gqa).
+struct PlanCache {
+  std::mutex mu;
+  struct Entry {
+    int dev, bits, gqa;
+    DecodePlan plan;
+  };
+  Entry entries[64];
+  int n = 0;
+};
+PlanCache& plan_cache() {
+  static PlanCache c;
+  return c;
+}
+
+cudaError_t get_plan(int bits, int gqa, DecodePlan* out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  PlanCache& pc = plan_cache();
+  std::lock_guard<std::mutex> lock(pc.mu);
+  for (int i = 0; i < pc.n; ++i) {
+    if (pc.entries[i].dev == dev && pc.entries[i].bits == bits && pc.entries[i].gqa == gqa) {
+      *out = pc.entries[i].plan;
+      return cudaSuccess;
+    }
+  }
+  DecodePlan p{};
+  if ((e = kivi::decode_plan(bits, gqa, &p)) != cudaSuccess) return e;
+  if (pc.n < 64) pc.entries[pc.n++] = {dev, bits, gqa, p};
+  *out = p;
+  return cudaSuccess;
+}
+
+bool gqa_supported(int g) { return g == 1 || g == 2 || g == 4 || g == 8; }
+
+}  // namespace
+
+extern "C" {
+
+int kivi_abi_version(void) { return KIVI_ABI_VERSION; }
+
+const char* kivi_strerror(int s) {
+  switch (s) {
+    case KIVI_OK: return "ok";
+    case KIVI_ERR_INVALID_ARG: return "invalid argument";
+    case KIVI_ERR_UNSUPPORTED: return "unsupported configuration";
+    case KIVI_ERR_CAPACITY: return "cache capacity exceeded";
+    case KIVI_ERR_RESIDUAL_FULL: return "residual buffer full: flush first";
+    case KIVI_ERR_RESIDUAL_NOT_FULL: return "residual buffer not full";
+    case KIVI_ERR_EMPTY: return "attention over an empty cache";
+    case KIVI_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case KIVI_ERR_CUDA: return "CUDA runtime error";
+    case KIVI_ERR_DEVICE_TIMEOUT: return "bounded device wait expired";
+    case KIVI_ERR_STATE: return "cache counters inconsistent";
+    default: return "unknown status";
+  }
+}
+
+int kivi_check_config(const kivi_config* cfg) { return check_cfg(cfg); }
+
+int kivi_cache_sizes(const kivi_config* cfg, size_t* out) {
+  const int st = check_cfg(cfg);
+  if (st != KIVI_OK) return st;
+  if (out == nullptr) return KIVI_ERR_INVALID_ARG;
+  const size_t bh = static_cast<size_t>(cfg->batch) * cfg->num_kv_heads;
+  const size_t C = static_cast<size_t>(cfg->capacity), d = kHeadDim;
+  const size_t code_bytes = bh * C * d * cfg->bits / 8;
+  out[KIVI_BUF_K_CODES] = code_bytes;
+  out[KIVI_BUF_V_CODES] = code_bytes;
+  out[KIVI_BUF_K_SCALE] = out[KIVI_BUF_K_ZERO] = bh * (C / cfg->residual) * (d / cfg->group_k) * 2;
+  out[KIVI_BUF_V_SCALE] = out[KIVI_BUF_V_ZERO] = bh * (C / cfg->group_v) * 2;
+  out[KIVI_BUF_K_RES] = out[KIVI_BUF_V_RES] = bh * cfg->residual * d * 2;
+  return KIVI_OK;
+}
+
+int kivi_quantize_prefill(const kivi_config* cfg, kivi_cache* cache, const uint16_t* k_dev, const uint16_t* v_dev,
+                          int32_t num_tokens, void* stream) {
+  int st = check_cfg(cfg);
+  if (st != KIVI_OK) return st;
+  if (cache == nullptr || num_tokens < 1 || !aligned16(k_dev) || !aligned16(v_dev)) return KIVI_ERR_INVALID_ARG;
+  const int R = cfg->residual;
+  const int n_res = (num_tokens - 1) % R + 1;
+  const int n_quant = num_tokens - n_res;
+  if (n_quant > cfg->capacity) return KIVI_ERR_CAPACITY;
+  if (!cache_ptrs_ok(cache, n_quant > 0)) return KIVI_ERR_INVALID_ARG;
+  kivi::QuantizeArgs a{};
+  a.k_src = k_dev;
+  a.v_src = v_dev;
+  a.k_codes = cache->k_codes;
+  a.v_codes = cache->v_codes;
+  a.k_scale = cache->k_scale;
+  a.k_zero = cache->k_zero;
+  a.v_scale = cache->v_scale;
+  a.v_zero = cache->v_zero;
+  a.k_res = cache->k_res;
+  a.v_res = cache->v_res;
+  a.bh = cfg->batch * cfg->num_kv_heads;
+  a.src_tokens = num_tokens;
+  a.src_tok0 = 0;
+  a.nblocks = n_quant / R;
+  a.dst_blk0 = 0;
+  a.res_tok0 = n_quant;
+  a.res_tokens = n_res;
+  a.residual = R;
+  a.capacity = cfg->capacity;
+  a.group_k = cfg->group_k;
+  a.group_v = cfg->group_v;
+  if (kivi::launch_quantize_blocks(a, cfg->bits, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return KIVI_ERR_CUDA;
+  cache->n_quant = n_quant;
+  cache->n_res = n_res;
+  return KIVI_OK;
+}
+
+int kivi_append_token(const kivi_config* cfg, kivi_cache* cache, const uint16_t* k_new_dev,
+                      const uint16_t* v_new_dev, void* stream) {
+  int st = check_cfg(cfg);
+  if (st != KIVI_OK) return st;
+  if ((st = check_state(cfg, cache)) != KIVI_OK) return st;
+  if (!aligned16(k_new_dev) || !aligned16(v_new_dev) || !cache_ptrs_ok(cache, false)) return KIVI_ERR_INVALID_ARG;
+  if (cache->n_res == cfg->residual) return KIVI_ERR_RESIDUAL_FULL;
+  kivi::AppendArgs a{};
+  a.k_new = k_new_dev;
+  a.v_new = v_new_dev;
+  a.k_res = cache->k_res;
+  a.v_res = cache->v_res;
+  a.bh = cfg->batch * cfg->num_kv_heads;
+  a.residual = cfg->residual;
+  a.slot = cache->n_res;
+  if (kivi::launch_append(a, static_cast<cudaStream_t>(stream)) != cudaSuccess) return KIVI_ERR_CUDA;
+  cache->n_res += 1;
+  return KIVI_OK;
+}
+
+int kivi_flush_residual(const kivi_config* cfg, kivi_cache* cache, void* stream) {
+  int st = check_cfg(cfg);
+  if (st != KIVI_OK) return st;
+  if ((st = check_state(cfg, cache)) != KIVI_OK) return st;
+  if (cache->n_res < cfg->residual) return KIVI_ERR_RESIDUAL_NOT_FULL;
+  if (cache->n_quant + cfg->residual > cfg->capacity) return KIVI_ERR_CAPACITY;
+  if (!cache_ptrs_ok(cache, true)) return KIVI_ERR_INVALID_ARG;
+  const int R = cfg->residual;
+  kivi::QuantizeArgs a{};
+  a.k_src = cache->k_res;
+  a.v_src = cache->v_res;
+  a.k_codes = cache->k_codes;
+  a.v_codes = cache->v_codes;
+  a.k_scale = cache->k_scale;
+  a.k_zero = cache->k_zero;
+  a.v_scale = cache->v_scale;
+  a.v_zero = cache->v_zero;
+  a.k_res = cache->k_res;
+  a.v_res = cache->v_res;
+  a.bh = cfg->batch * cfg->num_kv_heads;
+  a.src_tokens = R;
+  a.src_tok0 = 0;
+  a.nblocks = 1;
+  a.dst_blk0 = cache->n_quant / R;
+  a.res_tokens = 0;
+  a.residual = R;
+  a.capacity = cfg->capacity;
+  a.group_k = cfg->group_k;
+  a.group_v = cfg->group_v;
+  if (kivi::launch_quantize_blocks(a, cfg->bits, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return KIVI_ERR_CUDA;
+  cache->n_quant += R;
+  cache->n_res = 0;
+  return KIVI_OK;
+}
+
+size_t kivi_decode_workspace_bytes(const kivi_config* cfg, int32_t num_q_heads) {
+  if (check_cfg(cfg) != KIVI_OK || num_q_heads < 1 || num_q_heads % cfg->num_kv_heads != 0) return 0;
+  const int gqa = num_q_heads / cfg->num_kv_heads;
+  if (!gqa_supported(gqa)) return 0;
+  DecodePlan p{};
+  if (get_plan(cfg->bits, gqa, &p) != cudaSuccess) return 0;
+  const size_t bh = static_cast<size_t>(cfg->batch) * cfg->num_kv_heads;
+  return align256(static_cast<size_t>(p.workers()) * 2 * gqa * kivi::kPartialStride * sizeof(float)) +
+         align256(bh * sizeof(int32_t));
+}
+
+int kivi_decode_attention(const kivi_config* cfg, const kivi_cache* cache, const uint16_t* q_dev,
+                          int32_t num_q_heads, float scale, uint16_t* out_dev, void* workspace_dev,
+                          size_t workspace_bytes, int32_t* dev_status, void* stream) {
+  int st = check_cfg(cfg);
+  if (st != KIVI_OK) return st;
+  if ((st = check_state(cfg, cache)) != KIVI_OK) return st;
+  if (num_q_heads < 1 || num_q_heads % cfg->num_kv_heads != 0) return KIVI_ERR_INVALID_ARG;
+  const int gqa = num_q_heads / cfg->num_kv_heads;
+  if (!gqa_supported(gqa)) return KIVI_ERR_UNSUPPORTED;
+  if (!aligned16(q_dev) || !aligned16(out_dev) || !(scale == scale) || scale > 3.0e38f || scale < -3.0e38f)
+    return KIVI_ERR_INVALID_ARG;
+  if (cache->n_quant + cache->n_res == 0) return KIVI_ERR_EMPTY;
+  if (!cache_ptrs_ok(cache, cache->n_quant > 0)) return KIVI_ERR_INVALID_ARG;
+  if (dev_status != nullptr && (reinterpret_cast<uintptr_t>(dev_status) & 3u) != 0) return KIVI_ERR_INVALID_ARG;
+  DecodePlan plan{};
+  if (get_plan(cfg->bits, gqa, &plan) != cudaSuccess) return KIVI_ERR_CUDA;
+  const size_t bh = static_cast<size_t>(cfg->batch) * cfg->num_kv_heads;
+  const size_t part_bytes = align256(static_cast<size_t>(plan.workers()) * 2 * gqa * kivi::kPartialStride * 4);
+  if (workspace_dev == nullptr || (reinterpret_cast<uintptr_t>(workspace_dev) & 255u) != 0 ||
+      workspace_bytes < part_bytes + align256(bh * 4))
+    return KIVI_ERR_WORKSPACE;
+
+  const int ut = unit_tokens(cfg->bits);
+  DecodeArgs a{};
+  a.k_codes = cache->k_codes;
+  a.v_codes = cache->v_codes;
+  a.k_scale = cache->k_scale;
+  a.k_zero = cache->k_zero;
+  a.v_scale = cache->v_scale;
+  a.v_zero = cache->v_zero;
+  a.k_res = cache->k_res;
+  a.v_res = cache->v_res;
+  a.q = q_dev;
+  a.out = out_dev;
+  a.partials = static_cast<float*>(workspace_dev);
+  a.tickets = reinterpret_cast<int32_t*>(static_cast<char*>(workspace_dev) + part_bytes);
+  a.status = dev_status;
+  a.bh = static_cast<int>(bh);
+  a.gqa = gqa;
+  a.capacity = cfg->capacity;
+  a.residual = cfg->residual;
+  a.group_k = cfg->group_k;
+  a.group_v = cfg->group_v;
+  a.n_quant = cache->n_quant;
+  a.n_res = cache->n_res;
+  a.units_q = cache->n_quant / ut;
+  a.units = a.units_q + (cache->n_res + 15) / 16;
+  a.total_units = static_cast<long long>(bh) * a.units;
+  // every worker must own at least one unit: the merge counts all workers that touch a head
+  a.workers = static_cast<int>(a.total_units < plan.workers() ? a.total_units : plan.workers());
+  a.qscale = scale * 1.4426950408889634f;
+  {
+    DebugState& d = debug_state();
+    std::lock_guard<std::mutex> lock(d.mu);
+    a.timeout_ns = d.timeout_ns;
+    a.debug_extra_tx = d.mode == 1 ? 16u : 0u;
+  }
+  if (kivi::launch_decode(a, cfg->bits, plan, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return KIVI_ERR_CUDA;
+  return KIVI_OK;
+}
+
+int kivi_read_status(const int32_t* dev_status, void* stream) {
+  if (dev_status == nullptr) return KIVI_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return KIVI_ERR_CUDA;
+  int32_t v = 0;
+  if (cudaMemcpy(&v, dev_status, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) return KIVI_ERR_CUDA;
+  return v;
+}
+
+int kivi_debug_inject(int32_t mode, uint64_t timeout_ns) {
+  if (mode != 0 && mode != 1) return KIVI_ERR_INVALID_ARG;
+  DebugState& d = debug_state();
+  std::lock_guard<std::mutex> lock(d.mu);
+  d.mode = mode;
+  d.timeout_ns = timeout_ns == 0 ? kDefaultTimeoutNs : timeout_ns;
+  return KIVI_OK;
+}
+
+}  // extern "C"

@@ -1,8 +1,8 @@
 """Seeded synthetic KV-cache workloads (inputs only: no quantization or attention arithmetic).
 
-Every array is drawn per (batch, head[, step]) from its own numpy PCG64 stream keyed by
-(seed, stream id, indices), so any subset of heads can be regenerated on its own and a prefix of a
-prompt equals the shorter prompt.  Distributions follow the KV-cache statistics the KIVI explainer
+Prompts are drawn per (batch, KV head) and decode-step rows per (batch, step), each from its own
+numpy PCG64 stream keyed by (seed, stream id, indices), so any subset of heads can be regenerated
+on its own and a prefix of a prompt equals the shorter prompt.  Distributions follow the KV-cache statistics the KIVI explainer
 page describes (section KVキャッシュの分布特性): keys have a few outlier channels with large
 magnitude across all tokens, values have a large early "sink" token.
 
@@ -14,6 +14,7 @@ magnitude across all tokens, values have a large early "sink" token.
 """
 from __future__ import annotations
 
+import functools
 import os
 from concurrent.futures import ThreadPoolExecutor
 from dataclasses import dataclass, replace
@@ -62,10 +63,14 @@ def _rng(seed: int, *key: int) -> np.random.Generator:
     return np.random.Generator(np.random.PCG64(np.random.SeedSequence([seed, *key])))
 
 
+@functools.lru_cache(maxsize=1 << 16)
+def _outliers(seed: int, d: int, b: int, h: int) -> tuple:
+    return tuple(np.sort(_rng(seed, STREAM_OUTLIER, b, h).choice(d, N_OUTLIER_CHANNELS, replace=False)))
+
+
 def outlier_channels(w: Workload, b: int, h: int) -> np.ndarray:
     """The N_OUTLIER_CHANNELS distinct outlier channels of KV head (b, h)."""
-    return np.sort(_rng(w.seed, STREAM_OUTLIER, b, h).choice(w.head_dim, N_OUTLIER_CHANNELS,
-                                                             replace=False))
+    return np.array(_outliers(w.seed, w.head_dim, b, h), dtype=np.int64)
 
 
 def prompt_k(w: Workload, b: int, h: int, n: int) -> np.ndarray:
@@ -83,23 +88,31 @@ def prompt_v(w: Workload, b: int, h: int, n: int) -> np.ndarray:
     return x.astype(np.float16)
 
 
+def _step_rows(w: Workload, stream: int, b: int, step: int, n: int) -> np.ndarray:
+    """fp32 N(0,1) [n][d]: one row per head of sequence b at decode step `step`."""
+    return _rng(w.seed, stream, b, step).standard_normal((n, w.head_dim), dtype=np.float32)
+
+
+def _keys_of_step(w: Workload, b: int, step: int) -> np.ndarray:
+    x = _step_rows(w, STREAM_KNEW, b, step, w.kv_heads)
+    for h in range(w.kv_heads):
+        x[h, outlier_channels(w, b, h)] *= np.float32(OUTLIER_GAIN)
+    return x.astype(np.float16)
+
+
 def query(w: Workload, b: int, hq: int, step: int = 0) -> np.ndarray:
     """fp16 [d] query of query head (b, hq) at decode step `step`."""
-    return _rng(w.seed, STREAM_Q, b, hq, step).standard_normal(w.head_dim, dtype=np.float32) \
-        .astype(np.float16)
+    return _step_rows(w, STREAM_Q, b, step, w.q_heads)[hq].astype(np.float16)
 
 
 def new_k(w: Workload, b: int, h: int, step: int) -> np.ndarray:
     """fp16 [d] key appended to KV head (b, h) at decode step `step` (outlier channels x10)."""
-    x = _rng(w.seed, STREAM_KNEW, b, h, step).standard_normal(w.head_dim, dtype=np.float32)
-    x[outlier_channels(w, b, h)] *= np.float32(OUTLIER_GAIN)
-    return x.astype(np.float16)
+    return _keys_of_step(w, b, step)[h]
 
 
 def new_v(w: Workload, b: int, h: int, step: int) -> np.ndarray:
     """fp16 [d] value appended to KV head (b, h) at decode step `step`."""
-    return _rng(w.seed, STREAM_VNEW, b, h, step).standard_normal(w.head_dim, dtype=np.float32) \
-        .astype(np.float16)
+    return _step_rows(w, STREAM_VNEW, b, step, w.kv_heads)[h].astype(np.float16)
 
 
 def _threads() -> int:
@@ -125,14 +138,13 @@ def prompt_kv(w: Workload, n: int, out_k: np.ndarray | None = None,
 
 def queries(w: Workload, step: int = 0) -> np.ndarray:
     """fp16 [B][Hq][d] queries of one decode step."""
-    return np.stack([np.stack([query(w, b, hq, step) for hq in range(w.q_heads)])
+    return np.stack([_step_rows(w, STREAM_Q, b, step, w.q_heads).astype(np.float16)
                      for b in range(w.batch)])
 
 
 def new_kv(w: Workload, step: int):
     """fp16 [B][H][d] key and value appended at one decode step."""
-    k = np.stack([np.stack([new_k(w, b, h, step) for h in range(w.kv_heads)])
-                  for b in range(w.batch)])
-    v = np.stack([np.stack([new_v(w, b, h, step) for h in range(w.kv_heads)])
+    k = np.stack([_keys_of_step(w, b, step) for b in range(w.batch)])
+    v = np.stack([_step_rows(w, STREAM_VNEW, b, step, w.kv_heads).astype(np.float16)
                   for b in range(w.batch)])
     return k, v

@@ -165,6 +165,15 @@ const char* kivi_strerror(int status);
 /* KIVI_ABI_VERSION of the loaded library. */
 int kivi_abi_version(void);
 
+/*
+ * Test hook for the failure path (no counterpart on the page).  mode 1: every later
+ * kivi_decode_attention makes its bulk-copy barriers expect 16 bytes more than are copied, so each
+ * bounded wait runs out after `timeout_ns` and the kernel reports KIVI_ERR_DEVICE_TIMEOUT through
+ * dev_status and returns (the output is then undefined).  mode 0 restores normal operation;
+ * timeout_ns == 0 restores the default bound (2 s).  Process-wide; not for production use.
+ */
+int kivi_debug_inject(int32_t mode, uint64_t timeout_ns);
+
 #ifdef __cplusplus
 }
 #endif

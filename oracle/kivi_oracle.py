@@ -11,6 +11,7 @@ explainer page "ICML 2024論文解説: KIVI — チューニング不要のKVキ
 Readings taken where the page leaves a step open (each is pinned by tests/test_oracle_pins.py):
   * K group = one R-token block x G_k consecutive channels; V group = G_v consecutive tokens x
     all d channels (sections Per-Channel量子化 / Per-Token量子化, their K_quant / V_quant equations).
+  * z is the group minimum itself (exact in fp16); a minimum of -0 is stored as +0.
   * s is stored in fp16: the exact real (max-min)/(2^b-1) rounded to nearest, ties to even.
     The subtraction of two fp16 values is exact in fp64 and the quotient by 3 or 15 cannot
     fall onto an fp16 rounding midpoint unless it is exactly one, so "fp64 divide, then round to
@@ -69,7 +70,7 @@ def scale_zero(lo, hi, bits: int):
     lo64 = np.asarray(lo, dtype=np.float16).astype(np.float64)
     hi64 = np.asarray(hi, dtype=np.float16).astype(np.float64)
     s = fp16_round((hi64 - lo64) / levels(bits))
-    z = np.asarray(lo, dtype=np.float16).copy()
+    z = fp16_round(lo64 + 0.0)          # exact; a zero minimum is stored as +0
     return s, z
 
 

@@ -1,0 +1,76 @@
+"""Helpers shared by the GPU parity tests: run the CUDA path and the oracle on the same inputs."""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+import oracle.kivi_oracle as O
+from bit_asymmetric_kv_02_b200 import synth
+
+ATOL = 2e-3        # max-abs bound on decode outputs
+RTOL = 1e-2        # max-rel bound, relative to max(|o*|, REL_FLOOR)
+REL_FLOOR = 1e-2
+
+
+def attention_errors(got, want):
+    """(max abs error, max rel error with floor) of fp16 outputs vs fp64 oracle outputs."""
+    got = np.asarray(got, np.float64)
+    want = np.asarray(want, np.float64)
+    err = np.abs(got - want)
+    return float(err.max()), float((err / np.maximum(np.abs(want), REL_FLOOR)).max())
+
+
+def assert_attention_close(got, want, what=""):
+    ea, er = attention_errors(got, want)
+    assert ea <= ATOL and er <= RTOL, f"{what}: max abs {ea:.3e} (bar {ATOL}), max rel {er:.3e} (bar {RTOL})"
+    return ea, er
+
+
+def oracle_head(w: synth.Workload, b: int, h: int, capacity: int, prompt_tokens: int):
+    """HeadCache of KV head (b, h) after prefill of `prompt_tokens` synthetic tokens."""
+    hc = O.HeadCache(w.head_dim, w.bits, w.group, w.group, w.residual, capacity)
+    hc.prefill(synth.prompt_k(w, b, h, prompt_tokens), synth.prompt_v(w, b, h, prompt_tokens))
+    return hc
+
+
+def sample_heads(w: synth.Workload, n: int, seed: int = 0):
+    """First, last and n-2 seeded random (b, h) KV heads."""
+    rng = np.random.default_rng(seed)
+    heads = {(0, 0), (w.batch - 1, w.kv_heads - 1)}
+    while len(heads) < min(n, w.batch * w.kv_heads):
+        heads.add((int(rng.integers(w.batch)), int(rng.integers(w.kv_heads))))
+    return sorted(heads)
+
+
+def gpu_buffers_of_head(cache, b: int, h: int, n_quant: int, n_res: int):
+    """Host copies of one head's filled cache in the library layout (tokens [0, n_quant))."""
+    cfg = cache.cfg
+    P = 32 // cfg.bits
+    out = {
+        "k_codes": cache.view("k_codes")[b, h, :n_quant].cpu().numpy().view(np.uint32),
+        "v_codes": cache.view("v_codes")[b, h, :n_quant // P].cpu().numpy().view(np.uint32),
+        "k_scale": cache.view("k_scale")[b, h, :n_quant // cfg.residual].cpu().numpy(),
+        "k_zero": cache.view("k_zero")[b, h, :n_quant // cfg.residual].cpu().numpy(),
+        "v_scale": cache.view("v_scale")[b, h, :n_quant // cfg.group_v].cpu().numpy(),
+        "v_zero": cache.view("v_zero")[b, h, :n_quant // cfg.group_v].cpu().numpy(),
+        "k_res": cache.view("k_res")[b, h, :n_res].cpu().numpy(),
+        "v_res": cache.view("v_res")[b, h, :n_res].cpu().numpy(),
+    }
+    return out
+
+
+def assert_head_bitexact(gpu: dict, ref: dict, what=""):
+    for key, want in ref.items():
+        got = gpu[key]
+        want = np.asarray(want)
+        assert got.shape == want.shape, f"{what} {key}: shape {got.shape} vs {want.shape}"
+        gb = np.ascontiguousarray(got).view(np.uint8)
+        wb = np.ascontiguousarray(want).view(np.uint8)
+        if not np.array_equal(gb, wb):
+            bad = np.argwhere(np.ascontiguousarray(got) != np.ascontiguousarray(want))
+            raise AssertionError(f"{what} {key}: {len(bad)} mismatches, first at {bad[:3].tolist()}")
+
+
+def default_scale(d: int = 128) -> float:
+    return 1.0 / math.sqrt(d)

@@ -1,0 +1,122 @@
+"""The C-ABI library loads, exports every function include/kivi.h declares, and its host-side
+checks work without a GPU (no compute call is made here)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "kivi.h")
+
+
+@pytest.fixture(scope="module")
+def kivi():
+    from bit_asymmetric_kv_02_b200 import build, kivi as k
+    build.build()
+    k.load_library()
+    return k
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(kivi_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported(kivi):
+    names = declared_functions()
+    assert len(names) >= 11
+    lib = ctypes.CDLL(kivi.LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_version_and_strerror(kivi):
+    assert kivi.kivi_abi_version() == 1
+    assert kivi.kivi_strerror(0) == "ok"
+    assert "flush" in kivi.kivi_strerror(4)
+    assert kivi.kivi_strerror(12345) == "unknown status"
+
+
+def _cfg(kivi, **kw):
+    base = dict(batch=2, num_kv_heads=3, head_dim=128, bits=2, group_k=32, group_v=32, residual=128, capacity=1024)
+    base.update(kw)
+    return kivi.kivi_config(**base)
+
+
+def test_config_rules(kivi):
+    assert kivi.kivi_check_config(_cfg(kivi)) == 0
+    assert kivi.kivi_check_config(_cfg(kivi, bits=3)) == 2
+    assert kivi.kivi_check_config(_cfg(kivi, head_dim=64)) == 2
+    assert kivi.kivi_check_config(_cfg(kivi, group_k=48)) == 1
+    assert kivi.kivi_check_config(_cfg(kivi, group_v=48)) == 1
+    assert kivi.kivi_check_config(_cfg(kivi, residual=100)) == 1
+    assert kivi.kivi_check_config(_cfg(kivi, capacity=1000)) == 1
+    assert kivi.kivi_check_config(_cfg(kivi, batch=0)) == 1
+    assert kivi.kivi_check_config(_cfg(kivi, bits=4, group_k=128, group_v=128)) == 0
+
+
+def test_cache_sizes(kivi):
+    sizes = kivi.kivi_cache_sizes(_cfg(kivi))
+    bh, C, d = 6, 1024, 128
+    assert sizes[0] == sizes[1] == bh * C * d * 2 // 8
+    assert sizes[2] == sizes[3] == bh * (C // 128) * (d // 32) * 2
+    assert sizes[4] == sizes[5] == bh * (C // 32) * 2
+    assert sizes[6] == sizes[7] == bh * 128 * d * 2
+    s4 = kivi.kivi_cache_sizes(_cfg(kivi, bits=4, group_k=128, group_v=128))
+    assert s4[0] == bh * C * d // 2 and s4[2] == bh * (C // 128) * 2 and s4[4] == bh * (C // 128) * 2
+
+
+def test_state_errors_before_any_device_work(kivi):
+    """Errors detected on the host return before anything is enqueued; fake (aligned, never
+    dereferenced) pointers are enough to reach them."""
+    cfg = _cfg(kivi)
+    fake = 1 << 20
+    cache = kivi.kivi_cache(*([fake] * 8), 0, 128)
+    with pytest.raises(kivi.KiviError) as e:
+        kivi.kivi_append_token(cfg, cache, fake, fake, 0)
+    assert e.value.code == "RESIDUAL_FULL"
+    cache.n_res = 5
+    with pytest.raises(kivi.KiviError) as e:
+        kivi.kivi_flush_residual(cfg, cache, 0)
+    assert e.value.code == "RESIDUAL_NOT_FULL"
+    cache.n_quant, cache.n_res = 1024, 128
+    with pytest.raises(kivi.KiviError) as e:
+        kivi.kivi_flush_residual(cfg, cache, 0)
+    assert e.value.code == "CAPACITY"
+    cache.n_quant = 100
+    with pytest.raises(kivi.KiviError) as e:
+        kivi.kivi_flush_residual(cfg, cache, 0)
+    assert e.value.code == "STATE"
+    cache.n_quant, cache.n_res = 0, 0
+    with pytest.raises(kivi.KiviError) as e:
+        kivi.kivi_decode_attention(cfg, cache, fake, 3, 0.1, fake, fake, 1 << 30, None, 0)
+    assert e.value.code == "EMPTY"
+    with pytest.raises(kivi.KiviError) as e:
+        kivi.kivi_decode_attention(cfg, cache, fake, 4, 0.1, fake, fake, 1 << 30, None, 0)
+    assert e.value.code == "INVALID_ARG"
+    cache.n_res = 1
+    with pytest.raises(kivi.KiviError) as e:
+        kivi.kivi_decode_attention(cfg, cache, fake, 3 * 16, 0.1, fake, fake, 1 << 30, None, 0)
+    assert e.value.code == "UNSUPPORTED"
+    with pytest.raises(kivi.KiviError) as e:
+        kivi.kivi_quantize_prefill(cfg, cache, fake, fake, 0, 0)
+    assert e.value.code == "INVALID_ARG"
+    with pytest.raises(kivi.KiviError) as e:
+        kivi.kivi_quantize_prefill(cfg, cache, fake + 8, fake, 10, 0)
+    assert e.value.code == "INVALID_ARG"
+    with pytest.raises(kivi.KiviError) as e:
+        kivi.kivi_quantize_prefill(cfg, cache, fake, fake, 1024 + 129, 0)
+    assert e.value.code == "CAPACITY"
+
+
+def test_binding_fails_loudly_without_library(tmp_path):
+    from bit_asymmetric_kv_02_b200 import kivi as k
+    saved = k._lib
+    k._lib = None
+    try:
+        with pytest.raises(RuntimeError):
+            k.load_library(str(tmp_path / "missing.so"))
+    finally:
+        k._lib = saved

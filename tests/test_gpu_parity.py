@@ -1,0 +1,281 @@
+"""CUDA path (through the C ABI) vs the CPU oracle on the same seeded inputs.
+
+Codes, scales, zero points and residual rows must match bit for bit; decode outputs must be within
+max-abs 2e-3 and max-rel 1e-2 (relative to max(|o*|, 1e-2)) of the fp64 oracle run on the same
+quantized cache.
+"""
+import numpy as np
+import pytest
+
+import gpu_common as gc
+import oracle.kivi_oracle as O
+from bit_asymmetric_kv_02_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+
+
+@pytest.fixture(scope="module", autouse=True)
+def cuda_lib():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    from bit_asymmetric_kv_02_b200 import build, kivi
+    build.build()
+    kivi.load_library()
+    torch.cuda.set_device(0)
+
+
+def _kivi():
+    from bit_asymmetric_kv_02_b200 import kivi
+    return kivi
+
+
+def run_prefill_case(w: synth.Workload, heads=None, capacity=None, check_attention=True):
+    """GPU prefill + decode of workload w; oracle on `heads` (all if None)."""
+    kivi = _kivi()
+    T = w.tokens
+    cap = capacity if capacity is not None else ((T + w.residual - 1) // w.residual) * w.residual
+    k, v = synth.prompt_kv(w, T)
+    q = synth.queries(w, 0)
+    cache = kivi.KiviCache(w.batch, w.kv_heads, cap, bits=w.bits, group_k=w.group, group_v=w.group,
+                           residual=w.residual, num_q_heads=w.q_heads)
+    kd = torch.from_numpy(k).cuda()
+    vd = torch.from_numpy(v).cuda()
+    qd = torch.from_numpy(q).cuda()
+    cache.status.zero_()
+    cache.prefill(kd, vd)
+    out = cache.attend(qd).cpu().numpy()
+    assert cache.read_status() == 0
+    n_quant, n_res = cache.n_quant, cache.n_res
+    assert n_res == (T - 1) % w.residual + 1 and n_quant == T - n_res
+    heads = heads if heads is not None else [(b, h) for b in range(w.batch) for h in range(w.kv_heads)]
+    worst = (0.0, 0.0)
+    for (b, h) in heads:
+        hc = O.HeadCache(w.head_dim, w.bits, w.group, w.group, w.residual, cap)
+        hc.prefill(k[b, h], v[b, h])
+        gc.assert_head_bitexact(gc.gpu_buffers_of_head(cache, b, h, n_quant, n_res), hc.packed(),
+                                f"{w.name} head {(b, h)}")
+        if check_attention:
+            g = w.gqa
+            want = hc.attend(q[b, h * g:(h + 1) * g], gc.default_scale())
+            ea, er = gc.assert_attention_close(out[b, h * g:(h + 1) * g], want, f"{w.name} head {(b, h)}")
+            worst = (max(worst[0], ea), max(worst[1], er))
+    return worst
+
+
+SMALL = [
+    synth.TINY,
+    synth.TINY.with_(name="ragged_2bit_g32", batch=2, q_heads=3, kv_heads=3, tokens=3 * 128 + 37, seed=7),
+    synth.TINY.with_(name="ragged_4bit_g32", batch=1, q_heads=2, kv_heads=2, tokens=1024 + 5, bits=4, seed=8),
+    synth.TINY.with_(name="2bit_g128", batch=2, q_heads=2, kv_heads=2, tokens=700, group=128, seed=9),
+    synth.TINY.with_(name="4bit_g128", batch=1, q_heads=2, kv_heads=2, tokens=513, bits=4, group=128, seed=10),
+    synth.TINY.with_(name="one_token", batch=2, q_heads=2, kv_heads=2, tokens=1, seed=11),
+    synth.TINY.with_(name="exactly_R", batch=1, q_heads=2, kv_heads=2, tokens=128, seed=12),
+    synth.TINY.with_(name="R_plus_1", batch=1, q_heads=2, kv_heads=2, tokens=129, seed=13),
+    synth.TINY.with_(name="gqa4", batch=2, q_heads=8, kv_heads=2, tokens=900, seed=14),
+    synth.TINY.with_(name="gqa2_4bit", batch=1, q_heads=4, kv_heads=2, tokens=300, bits=4, seed=15),
+    synth.TINY.with_(name="gqa8", batch=1, q_heads=8, kv_heads=1, tokens=500, seed=16),
+    synth.TINY.with_(name="many_heads_short", batch=16, q_heads=8, kv_heads=8, tokens=200, seed=17),
+]
+
+
+@pytest.mark.parametrize("w", SMALL, ids=[w.name for w in SMALL])
+def test_prefill_and_decode_small(w):
+    run_prefill_case(w)
+
+
+def test_capacity_larger_than_used():
+    w = synth.TINY.with_(name="spare_capacity", tokens=600, seed=21)
+    run_prefill_case(w, capacity=2048)
+
+
+@pytest.mark.parametrize("bits,group", [(2, 32), (4, 32), (2, 128), (4, 128)])
+def test_streaming_append_flush(bits, group):
+    """prefill, then decode steps that flush when the residual is full, append one token and
+    attend; codes after every flush and outputs at chosen steps must match the oracle."""
+    kivi = _kivi()
+    w = synth.TINY.with_(name=f"stream_{bits}_{group}", batch=2, q_heads=4, kv_heads=2, tokens=250,
+                         bits=bits, group=group, seed=30 + bits + group)
+    steps = 300
+    cap = 1024
+    k, v = synth.prompt_kv(w, w.tokens)
+    cache = kivi.KiviCache(w.batch, w.kv_heads, cap, bits=bits, group_k=group, group_v=group,
+                           residual=w.residual, num_q_heads=w.q_heads)
+    cache.prefill(torch.from_numpy(k).cuda(), torch.from_numpy(v).cuda())
+    ref = {(b, h): O.HeadCache(128, bits, group, group, w.residual, cap)
+           for b in range(w.batch) for h in range(w.kv_heads)}
+    for (b, h), hc in ref.items():
+        hc.prefill(k[b, h], v[b, h])
+    check_at = {1, 2, 5, 6, 7, 133, 134, 135, 261, 262, 299, 300}
+    for s in range(1, steps + 1):
+        flushed = False
+        if cache.n_res == w.residual:
+            cache.flush()
+            for hc in ref.values():
+                hc.flush()
+            flushed = True
+        kn, vn = synth.new_kv(w, s)
+        cache.append(torch.from_numpy(kn).cuda(), torch.from_numpy(vn).cuda())
+        for (b, h), hc in ref.items():
+            hc.append(kn[b, h], vn[b, h])
+        if s in check_at or flushed:
+            q = synth.queries(w, s)
+            out = cache.attend(torch.from_numpy(q).cuda()).cpu().numpy()
+            for (b, h), hc in ref.items():
+                g = w.gqa
+                gc.assert_attention_close(out[b, h * g:(h + 1) * g], hc.attend(q[b, h * g:(h + 1) * g], gc.default_scale()),
+                                          f"step {s} head {(b, h)}")
+                gc.assert_head_bitexact(gc.gpu_buffers_of_head(cache, b, h, cache.n_quant, cache.n_res), hc.packed(),
+                                        f"step {s} head {(b, h)}")
+    assert cache.read_status() == 0
+
+
+def test_prefill_equals_streaming_on_gpu():
+    """The GPU cache after prefill(T) equals the GPU cache after prefill(T0) + appends/flushes."""
+    kivi = _kivi()
+    w = synth.TINY.with_(batch=1, q_heads=2, kv_heads=2, tokens=700, seed=40)
+    k, v = synth.prompt_kv(w, w.tokens)
+    a = kivi.KiviCache(1, 2, 1024, num_q_heads=2)
+    a.prefill(torch.from_numpy(k).cuda(), torch.from_numpy(v).cuda())
+    b = kivi.KiviCache(1, 2, 1024, num_q_heads=2)
+    b.prefill(torch.from_numpy(k[:, :, :100]).contiguous().cuda(), torch.from_numpy(v[:, :, :100]).contiguous().cuda())
+    for t in range(100, 700):
+        if b.n_res == 128:
+            b.flush()
+        b.append(torch.from_numpy(k[:, :, t]).contiguous().cuda(), torch.from_numpy(v[:, :, t]).contiguous().cuda())
+    assert (a.n_quant, a.n_res) == (b.n_quant, b.n_res)
+    for h in range(2):
+        ga = gc.gpu_buffers_of_head(a, 0, h, a.n_quant, a.n_res)
+        gb = gc.gpu_buffers_of_head(b, 0, h, b.n_quant, b.n_res)
+        gc.assert_head_bitexact(ga, gb, f"head {h}")
+
+
+def test_repeated_calls_are_identical():
+    """The workspace tickets are left at zero, so back-to-back calls give identical outputs."""
+    kivi = _kivi()
+    w = synth.TINY.with_(batch=4, q_heads=8, kv_heads=8, tokens=3000, seed=50)
+    k, v = synth.prompt_kv(w, w.tokens)
+    cache = kivi.KiviCache(w.batch, w.kv_heads, 3072, num_q_heads=w.q_heads)
+    cache.prefill(torch.from_numpy(k).cuda(), torch.from_numpy(v).cuda())
+    q = torch.from_numpy(synth.queries(w)).cuda()
+    o1 = cache.attend(q).clone()
+    o2 = cache.attend(q).clone()
+    assert torch.equal(o1, o2)
+    tickets = cache.workspace[cache.ws_ptr - cache.workspace.data_ptr():][: cache.ws_bytes]
+    assert int(tickets[-w.batch * w.kv_heads * 4:].view(torch.int32).abs().sum()) == 0
+
+
+def test_errors_through_the_abi():
+    kivi = _kivi()
+    cache = kivi.KiviCache(1, 2, 128, num_q_heads=2)
+    q = torch.zeros(1, 2, 128, dtype=torch.float16, device="cuda")
+    with pytest.raises(kivi.KiviError) as e:
+        cache.attend(q)
+    assert e.value.code == "EMPTY"
+    with pytest.raises(kivi.KiviError) as e:
+        cache.flush()
+    assert e.value.code == "RESIDUAL_NOT_FULL"
+    x = torch.zeros(1, 2, 128, 128, dtype=torch.float16, device="cuda")
+    cache.prefill(x, x)
+    assert (cache.n_quant, cache.n_res) == (0, 128)
+    row = torch.zeros(1, 2, 128, dtype=torch.float16, device="cuda")
+    with pytest.raises(kivi.KiviError) as e:
+        cache.append(row, row)
+    assert e.value.code == "RESIDUAL_FULL"
+    cache.flush()
+    for _ in range(128):
+        cache.append(row, row)
+    with pytest.raises(kivi.KiviError) as e:
+        cache.flush()
+    assert e.value.code == "CAPACITY"
+    with pytest.raises(kivi.KiviError) as e:
+        kivi.kivi_decode_attention(cache.cfg, cache.c, q.data_ptr(), 2, 0.1, q.data_ptr(), cache.ws_ptr, 16,
+                                   None, torch.cuda.current_stream().cuda_stream)
+    assert e.value.code == "WORKSPACE"
+
+
+def test_device_timeout_is_reported_and_context_survives():
+    """A barrier that can never complete (the test hook asks for 16 bytes more than are copied)
+    makes every bounded wait run out: the kernel reports DEVICE_TIMEOUT and returns; afterwards
+    normal calls work on the same context."""
+    kivi = _kivi()
+    w = synth.TINY.with_(batch=1, q_heads=2, kv_heads=2, tokens=600, seed=60)
+    k, v = synth.prompt_kv(w, w.tokens)
+    cache = kivi.KiviCache(1, 2, 1024, num_q_heads=2)
+    cache.prefill(torch.from_numpy(k).cuda(), torch.from_numpy(v).cuda())
+    q = torch.from_numpy(synth.queries(w)).cuda()
+    ref = cache.attend(q).clone()
+    assert cache.read_status() == 0
+    try:
+        kivi.kivi_debug_inject(1, 5_000_000)   # 5 ms bound per wait
+        cache.status.zero_()
+        cache.attend(q)
+        assert cache.read_status() == 9   # KIVI_ERR_DEVICE_TIMEOUT
+    finally:
+        kivi.kivi_debug_inject(0, 0)
+    cache.workspace.zero_()
+    cache.status.zero_()
+    again = cache.attend(q)
+    assert cache.read_status() == 0
+    assert torch.equal(again, ref)
+
+
+FULL = [synth.LLAMA2_7B, synth.LARGE_BATCH, synth.GQA_LLAMA3_8B]
+
+
+@pytest.mark.parametrize("w", FULL, ids=[w.name for w in FULL])
+def test_full_size_sampled_heads(w):
+    """Full-size workloads in the bench's launch configuration; the oracle checks 12 sampled KV
+    heads (codes bit-exact, outputs within tolerance)."""
+    gc_heads = gc.sample_heads(w, 12, seed=w.seed)
+    run_prefill_case(w, heads=gc_heads)
+
+
+@pytest.mark.parametrize("bits,group", [(2, 32), (2, 128), (4, 32), (4, 128)])
+def test_full_size_streaming(bits, group):
+    """Prefill 32768 tokens, then 256 decode steps (append, flush when full, attend).  The oracle
+    follows 4 sampled heads through every step and checks steps around both flushes."""
+    kivi = _kivi()
+    w = synth.STREAMING.with_(bits=bits, group=group)
+    cap = 33024
+    k, v = _streaming_prompt()
+    heads = gc.sample_heads(w, 4, seed=bits * 1000 + group)
+    ref = {bh: O.HeadCache(128, bits, group, group, w.residual, cap) for bh in heads}
+    for (b, h), hc in ref.items():
+        hc.prefill(k[b, h], v[b, h])
+    cache = kivi.KiviCache(w.batch, w.kv_heads, cap, bits=bits, group_k=group, group_v=group,
+                           residual=w.residual, num_q_heads=w.q_heads)
+    cache.prefill(torch.from_numpy(k).cuda(), torch.from_numpy(v).cuda())
+    for (b, h), hc in ref.items():
+        gc.assert_head_bitexact(gc.gpu_buffers_of_head(cache, b, h, cache.n_quant, cache.n_res), hc.packed(),
+                                f"prefill head {(b, h)}")
+    check_at = {1, 2, 127, 128, 129, 256}
+    for s in range(1, w.steps + 1):
+        if cache.n_res == w.residual:
+            cache.flush()
+            for hc in ref.values():
+                hc.flush()
+        kn, vn = synth.new_kv(w, s)
+        cache.append(torch.from_numpy(kn).cuda(), torch.from_numpy(vn).cuda())
+        for (b, h), hc in ref.items():
+            hc.append(kn[b, h], vn[b, h])
+        q = synth.queries(w, s)
+        out = cache.attend(torch.from_numpy(q).cuda())
+        if s in check_at:
+            out = out.cpu().numpy()
+            for (b, h), hc in ref.items():
+                gc.assert_attention_close(out[b, h:h + 1], hc.attend(q[b, h:h + 1], gc.default_scale()),
+                                          f"step {s} head {(b, h)}")
+                gc.assert_head_bitexact(gc.gpu_buffers_of_head(cache, b, h, cache.n_quant, cache.n_res),
+                                        hc.packed(), f"step {s} head {(b, h)}")
+    assert cache.read_status() == 0
+    assert (cache.n_quant, cache.n_res) == (32896, 128)
+
+
+_PROMPT = {}
+
+
+def _streaming_prompt():
+    if "kv" not in _PROMPT:
+        _PROMPT["kv"] = synth.prompt_kv(synth.STREAMING, synth.STREAMING.tokens)
+    return _PROMPT["kv"]
