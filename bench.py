@@ -16,13 +16,13 @@ no collective on the data path); the time is the max over ranks.
 from __future__ import annotations
 
 import argparse
+import faulthandler
 import hashlib
 import json
 import math
 import os
 import statistics
 import sys
-import threading
 import time
 
 import numpy as np
@@ -86,65 +86,66 @@ def decode_alg_bytes(w: synth.Workload, n_quant: int, n_res: int) -> int:
 
 
 class ClockSampler:
-    """Samples SM clock, max clock and throttle reasons with NVML every 20 ms (falls back to
-    nvidia-smi) while the timed region runs."""
+    """Samples SM clock, max clock and throttle reasons of one GPU with nvidia-smi every 50 ms while
+    the timed region runs (the clocks line of the profiling recipe)."""
 
-    REASONS = {  # NVML clocks-event reason bits
-        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
-        0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
-        0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting",
-    }
+    FIELDS = ("index,pci.bus_id,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
 
     def __init__(self, device_index: int):
-        self.samples = []
-        self.max_mhz = None
-        self._stop = threading.Event()
-        self._handle = None
+        self.bus = None
         try:
-            import pynvml
-            pynvml.nvmlInit()
             import torch
-            bus = torch.cuda.get_device_properties(device_index).pci_bus_id
-            self._handle = pynvml.nvmlDeviceGetHandleByPciBusId(bus.encode() if isinstance(bus, str) else bus)
-            self._nv = pynvml
-            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._handle, pynvml.NVML_CLOCK_SM)
+            self.bus = str(torch.cuda.get_device_properties(device_index).pci_bus_id).lower()
         except Exception:
-            self._handle = None
-
-    def _run(self):
-        nv = self._nv
-        while not self._stop.is_set():
-            try:
-                mhz = nv.nvmlDeviceGetClockInfo(self._handle, nv.NVML_CLOCK_SM)
-                reasons = nv.nvmlDeviceGetCurrentClocksEventReasons(self._handle)
-                util = nv.nvmlDeviceGetUtilizationRates(self._handle).gpu
-                self.samples.append((mhz, reasons, util))
-            except Exception:
-                pass
-            self._stop.wait(0.02)
+            pass
+        self.proc = None
+        self.lines = []
 
     def __enter__(self):
-        if self._handle is not None:
-            self._t = threading.Thread(target=self._run, daemon=True)
-            self._t.start()
+        import shutil
+        import subprocess
+        exe = shutil.which("nvidia-smi")
+        if exe:
+            self.proc = subprocess.Popen([exe, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                                         text=True)
         return self
 
     def __exit__(self, *exc):
-        self._stop.set()
-        if self._handle is not None:
-            self._t.join()
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=10)
+            except Exception:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
 
     def summary(self):
-        if not self.samples:
-            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
-        loaded = [s for s in self.samples if not (s[1] & 0x1)] or self.samples
+        rows = []
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 10:
+                continue
+            if self.bus and not self.bus.endswith(f[1].lower()[-12:]) and not f[1].lower().endswith(self.bus[-12:]):
+                continue
+            try:
+                rows.append((float(f[2]), float(f[3]), float(f[4]), f[6:10]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        loaded = [r for r in rows if r[2] > 300.0] or rows   # power draw separates load from idle
         reasons = set()
-        for _, r, _ in loaded:
-            for bit, name in self.REASONS.items():
-                if r & bit and name != "gpu_idle":
+        for r in loaded:
+            for name, flag in zip(self.NAMES, r[3]):
+                if flag.lower() == "active":
                     reasons.add(name)
-        return {"sm_mhz": statistics.median(s[0] for s in loaded), "sm_max_mhz": self.max_mhz,
-                "reasons": sorted(reasons), "samples": len(loaded)}
+        return {"sm_mhz": statistics.median(r[0] for r in loaded), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": sorted(reasons), "samples": len(loaded), "samples_total": len(rows)}
 
 
 BAD_REASONS = {"hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown"}
@@ -244,7 +245,9 @@ def run_gpu(args, rank, world, local_rank):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=device)
     ranks = Ranks(dist, device)
 
+    log("generating inputs and prefilling the cache")
     cache, n_quant0, host_in, dev_in = make_state(w, torch, kivi, device)
+    log("cache ready")
     stream = torch.cuda.Stream(device)
     out = torch.empty(w.batch, w.q_heads, w.head_dim, dtype=torch.float16, device=device)
     R = w.residual
@@ -281,9 +284,11 @@ def run_gpu(args, rank, world, local_rank):
         return ms, dec_ms, launches, tokens, bytes_decode, clocks.summary()
 
     ms, dec_ms, launches, tokens, bytes_decode, clk = timed_loop(args.steps, args.warmup)
+    log(f"timed loop done: {ms:.3f} ms for {args.steps} steps")
     if BAD_REASONS & set(clk["reasons"]):
         ms, dec_ms, launches, tokens, bytes_decode, clk = timed_loop(args.steps, args.warmup)
         clk["remeasured"] = True
+        log(f"re-measured (throttle reasons seen): {ms:.3f} ms")
     t_max, dec_ms = ranks.max(ms, dec_ms)
 
     # ---- end to end through the public API with host buffers ---------------------------------
@@ -312,6 +317,7 @@ def run_gpu(args, rank, world, local_rank):
             stream.synchronize()
         return f0.elapsed_time(f1), toks
 
+    log("end-to-end loop")
     e2e_steps = 0 if args.no_e2e else min(args.steps, 4 * R)
     e2e_ms, e2e_tokens = e2e_loop(e2e_steps) if e2e_steps else (float("nan"), 0)
     e2e_ms = ranks.max(e2e_ms)
@@ -428,7 +434,13 @@ def run_reference(args, rank, world):
     }
 
 
+def log(msg: str) -> None:
+    sys.stderr.write(f"[bench {time.strftime('%H:%M:%S')}] {msg}\n")
+    sys.stderr.flush()
+
+
 def main():
+    faulthandler.enable()
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=2048)
@@ -447,6 +459,7 @@ def main():
     else:
         res = run_gpu(args, rank, world, local_rank)
         if rank == 0 and world == 1 and not args.no_cpu_baseline:
+            log("cpu baseline (oracle)")
             value, cores, sample, dt, hs = oracle_sample(WORKLOAD, n_heads=min(64, 2 * (os.cpu_count() or 1)),
                                                          n_steps=16, budget_s=25.0)
             res["cpu_baseline"] = {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",

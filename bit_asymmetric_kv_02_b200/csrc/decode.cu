@@ -42,6 +42,8 @@ constexpr int kStageBytes = 8192;   // one unit: 4 KB K + 4 KB V
 constexpr int kHalfStage = 4096;
 constexpr int kResTokens = 16;      // tokens per residual unit
 constexpr unsigned kFull = 0xffffffffu;
+constexpr float kQRange = 8388544.f;   // 2^23 - 64: largest |Q| before rounding (signed 24-bit limbs)
+constexpr float kPRange = 16777088.f;  // 2^24 - 128: largest P before rounding (unsigned 24-bit limbs)
 
 template <int G>
 struct __align__(128) WarpSmem {
@@ -182,8 +184,10 @@ struct Decoder {
         mabs = fmaxf(mabs, fabsf(qv[j]));
       }
       mabs = warp_max(mabs);
-      const float scq = mabs > 0.f ? 8388607.f / mabs : 0.f;
-      const float invq = mabs > 0.f ? mabs / 8388607.f : 0.f;
+      // Q = rint(q s * scq) with |Q| <= 2^23 - 63: the margin keeps the rounded product of the
+      // largest element below 2^23 (it would wrap the signed top limb)
+      const float scq = mabs > 0.f ? kQRange / mabs : 0.f;
+      const float invq = mabs > 0.f ? mabs / kQRange : 0.f;
       float cblk = 0.f;
 #pragma unroll
       for (int gi = 0; gi < 4; ++gi) {
@@ -308,8 +312,9 @@ struct Decoder {
 
       // -- A9: fixed-point limbs of p_t * s_g(t), then the V codes
       if (mv > 0.f) {
-        const float scv = 16777215.f / mv;
-        const float invv = mv / 16777215.f;
+        // P = rint(p s * scv) <= 2^24 - 127: the top token must not round to 2^24 (it would wrap to 0)
+        const float scv = kPRange / mv;
+        const float invv = mv / kPRange;
 #pragma unroll
         for (int j = 0; j < TPL; ++j) {
           const int t = lane + 32 * j;
@@ -470,7 +475,9 @@ struct Decoder {
     if (lane == 0) {
       const int ticket = atomicAdd(a.tickets + head, 1);
       last = ticket == static_cast<int>(wlast - wfirst);
+      __threadfence();  // acquire side: the partials published before the other tickets
     }
+    __syncwarp();
     last = __shfl_sync(kFull, last, 0);
     if (!last) return;
     __threadfence();
@@ -486,7 +493,9 @@ struct Decoder {
         const int sx = (U * x / W) >= h0 ? 0 : 1;
         const float* p = a.partials + ((x * 2 + sx) * G + g) * kPartialStride;
         const float w = exp2f(__ldcg(p) - mm);
-        ls = fmaf(w, __ldcg(p + 1), ls);
+        const float lx = __ldcg(p + 1);
+        if (!(lx > 0.f) && lane == 0) report_status(a.status, KIVI_ERR_INTERNAL);  // never written
+        ls = fmaf(w, lx, ls);
         zs = fmaf(w, __ldcg(p + 2), zs);
         const float4 ov = __ldcg(reinterpret_cast<const float4*>(p + 4 + 4 * lane));
         acc[0] = fmaf(w, ov.x, acc[0]);

@@ -21,6 +21,7 @@ struct DebugState {
   std::mutex mu;
   int mode = 0;
   unsigned long long timeout_ns = kDefaultTimeoutNs;
+  long long max_workers = 0;  // 0: no cap
 };
 DebugState& debug_state() {
   static DebugState s;
@@ -115,6 +116,7 @@ const char* kivi_strerror(int s) {
     case KIVI_ERR_CUDA: return "CUDA runtime error";
     case KIVI_ERR_DEVICE_TIMEOUT: return "bounded device wait expired";
     case KIVI_ERR_STATE: return "cache counters inconsistent";
+    case KIVI_ERR_INTERNAL: return "internal consistency check failed on the device";
     default: return "unknown status";
   }
 }
@@ -291,7 +293,13 @@ int kivi_decode_attention(const kivi_config* cfg, const kivi_cache* cache, const
   a.units = a.units_q + (cache->n_res + 15) / 16;
   a.total_units = static_cast<long long>(bh) * a.units;
   // every worker must own at least one unit: the merge counts all workers that touch a head
-  a.workers = static_cast<int>(a.total_units < plan.workers() ? a.total_units : plan.workers());
+  long long workers = a.total_units < plan.workers() ? a.total_units : plan.workers();
+  {
+    DebugState& d = debug_state();
+    std::lock_guard<std::mutex> lock(d.mu);
+    if (d.max_workers > 0 && d.max_workers < workers) workers = d.max_workers;
+  }
+  a.workers = static_cast<int>(workers);
   a.qscale = scale * 1.4426950408889634f;
   {
     DebugState& d = debug_state();
@@ -313,13 +321,25 @@ int kivi_read_status(const int32_t* dev_status, void* stream) {
   return v;
 }
 
-int kivi_debug_inject(int32_t mode, uint64_t timeout_ns) {
-  if (mode != 0 && mode != 1) return KIVI_ERR_INVALID_ARG;
+int kivi_debug_inject(int32_t mode, uint64_t value) {
   DebugState& d = debug_state();
   std::lock_guard<std::mutex> lock(d.mu);
-  d.mode = mode;
-  d.timeout_ns = timeout_ns == 0 ? kDefaultTimeoutNs : timeout_ns;
-  return KIVI_OK;
+  switch (mode) {
+    case 0:
+      d.mode = 0;
+      d.timeout_ns = kDefaultTimeoutNs;
+      d.max_workers = 0;
+      return KIVI_OK;
+    case 1:
+      d.mode = 1;
+      d.timeout_ns = value == 0 ? kDefaultTimeoutNs : value;
+      return KIVI_OK;
+    case 2:
+      d.max_workers = static_cast<long long>(value);
+      return KIVI_OK;
+    default:
+      return KIVI_ERR_INVALID_ARG;
+  }
 }
 
 }  // extern "C"

@@ -18,6 +18,7 @@ KIVI_OK = 0
 STATUS_NAMES = {
     0: "OK", 1: "INVALID_ARG", 2: "UNSUPPORTED", 3: "CAPACITY", 4: "RESIDUAL_FULL",
     5: "RESIDUAL_NOT_FULL", 6: "EMPTY", 7: "WORKSPACE", 8: "CUDA", 9: "DEVICE_TIMEOUT", 10: "STATE",
+    11: "INTERNAL",
 }
 BUFFERS = ("k_codes", "v_codes", "k_scale", "k_zero", "v_scale", "v_zero", "k_res", "v_res")
 
@@ -129,8 +130,8 @@ def kivi_read_status(status_ptr: int, stream: int) -> int:
     return load_library().kivi_read_status(status_ptr, stream)
 
 
-def kivi_debug_inject(mode: int, timeout_ns: int = 0) -> None:
-    _check(load_library().kivi_debug_inject(mode, timeout_ns), "kivi_debug_inject")
+def kivi_debug_inject(mode: int, value: int = 0) -> None:
+    _check(load_library().kivi_debug_inject(mode, value), "kivi_debug_inject")
 
 
 # ---- torch-owned cache --------------------------------------------------------------------------

@@ -68,6 +68,7 @@ extern "C" {
 #define KIVI_ERR_CUDA 8              /* a CUDA runtime call or kernel launch failed */
 #define KIVI_ERR_DEVICE_TIMEOUT 9    /* a bounded device-side wait expired (reported via status) */
 #define KIVI_ERR_STATE 10            /* cache counters inconsistent with the call */
+#define KIVI_ERR_INTERNAL 11         /* a device-side consistency check failed (reported via status) */
 
 /*
  * Quantization configuration; mirrors the page's QuantConfig (section アルゴリズム: bits,
@@ -166,13 +167,16 @@ const char* kivi_strerror(int status);
 int kivi_abi_version(void);
 
 /*
- * Test hook for the failure path (no counterpart on the page).  mode 1: every later
- * kivi_decode_attention makes its bulk-copy barriers expect 16 bytes more than are copied, so each
- * bounded wait runs out after `timeout_ns` and the kernel reports KIVI_ERR_DEVICE_TIMEOUT through
- * dev_status and returns (the output is then undefined).  mode 0 restores normal operation;
- * timeout_ns == 0 restores the default bound (2 s).  Process-wide; not for production use.
+ * Test hooks (no counterpart on the page); process-wide, not for production use.
+ *   mode 0: restore normal operation.
+ *   mode 1: every later kivi_decode_attention makes its bulk-copy barriers expect 16 bytes more
+ *           than are copied, so each bounded wait runs out after `value` ns (0: the 2 s default)
+ *           and the kernel reports KIVI_ERR_DEVICE_TIMEOUT through dev_status and returns (the
+ *           output is then undefined).
+ *   mode 2: cap the number of decode workers (warps) at `value` (0: no cap), to exercise the
+ *           split-and-merge path with chosen splits.
  */
-int kivi_debug_inject(int32_t mode, uint64_t timeout_ns);
+int kivi_debug_inject(int32_t mode, uint64_t value);
 
 #ifdef __cplusplus
 }
