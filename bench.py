@@ -60,9 +60,11 @@ def hbm_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def profiled_traffic(w: synth.Workload):
-    """DRAM bytes per decode launch from the committed ncu summary, if it was taken on the current
-    kernel sources; else None."""
+def profiled_traffic(w: synth.Workload, alg_bytes_per_launch: float):
+    """DRAM bytes per decode launch from the committed ncu record, if it was taken on the current
+    kernel sources; else None.  The record holds one captured launch (its DRAM bytes and its
+    algorithmic bytes); the bench's average launch moves slightly different algorithmic bytes (the
+    residual fill cycles), so the captured traffic is scaled by that ratio."""
     path = os.path.join(ROOT, "profiles", "decode_traffic.json")
     try:
         with open(path) as f:
@@ -71,7 +73,7 @@ def profiled_traffic(w: synth.Workload):
         return None
     if rec.get("kernel_sha") != decode_kernel_sha() or rec.get("workload") != w.name:
         return None
-    return rec.get("bytes_per_launch")
+    return rec["dram_bytes"] / rec["alg_bytes"] * alg_bytes_per_launch
 
 
 def decode_alg_bytes(w: synth.Workload, n_quant: int, n_res: int) -> int:
@@ -95,14 +97,24 @@ class ClockSampler:
     NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
 
     def __init__(self, device_index: int):
-        self.bus = None
+        self.bus = None   # (bus, device) numbers of the CUDA device, as torch reports them
         try:
             import torch
-            self.bus = str(torch.cuda.get_device_properties(device_index).pci_bus_id).lower()
+            p = torch.cuda.get_device_properties(device_index)
+            self.bus = (int(p.pci_bus_id), int(p.pci_device_id))
         except Exception:
             pass
         self.proc = None
         self.lines = []
+
+    @staticmethod
+    def _bus_of(field: str):
+        """(bus, device) of an nvidia-smi pci.bus_id such as 00000000:1B:00.0."""
+        try:
+            parts = field.strip().split(":")
+            return int(parts[-2], 16), int(parts[-1].split(".")[0], 16)
+        except (ValueError, IndexError):
+            return None
 
     def __enter__(self):
         import shutil
@@ -130,7 +142,7 @@ class ClockSampler:
             f = [x.strip() for x in ln.split(",")]
             if len(f) < 10:
                 continue
-            if self.bus and not self.bus.endswith(f[1].lower()[-12:]) and not f[1].lower().endswith(self.bus[-12:]):
+            if self.bus is not None and self._bus_of(f[1]) not in (None, self.bus):
                 continue
             try:
                 rows.append((float(f[2]), float(f[3]), float(f[4]), f[6:10]))
@@ -329,7 +341,7 @@ def run_gpu(args, rank, world, local_rank):
         peak, peak_kind = hbm_peak()
         dec_avg_ms = dec_ms / K
         achieved = (bytes_decode / K) / (dec_avg_ms / 1e3) / 1e9
-        traffic = profiled_traffic(w)
+        traffic = profiled_traffic(w, bytes_decode / K)
         e2e_value = weak_scaling_value(world, e2e_tokens, w.batch, e2e_ms)
         result = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,

@@ -5,12 +5,13 @@
 //     out = softmax(scale * q [D(K_quant); K_res]^T) [D(V_quant); V_res],  D(x^) = s x^ + z.
 //
 // Work decomposition (stream-K over warps).  Every (batch, KV head) is a sequence of equal-size
-// "units": quantized units of UT tokens (UT = 128 at 2 bits, 64 at 4 bits; 4 KB of K codes +
-// 4 KB of V codes) followed by residual units of 16 fp16 tokens (4 KB K + 4 KB V).  The global
+// 4 KB "units": quantized units of UT tokens (UT = 64 at 2 bits, 32 at 4 bits; 2 KB of K codes +
+// 2 KB of V codes) followed by residual units of 8 fp16 tokens (2 KB K + 2 KB V).  The global
 // unit sequence is cut into one contiguous range per warp, so the load is balanced to one unit
 // whatever the batch, head count or context length.  Each warp streams its range through two
-// 8 KB shared-memory stages filled by 1-D TMA bulk copies (cp.async.bulk, no multicast) and
-// completed on an mbarrier; every wait is bounded and reports KIVI_ERR_DEVICE_TIMEOUT.
+// 4 KB shared-memory stages filled by 1-D TMA bulk copies (cp.async.bulk, no multicast) and
+// completed on an mbarrier; small stages leave room for ~20 resident warps per SM.  Every wait is
+// bounded and reports KIVI_ERR_DEVICE_TIMEOUT.
 // A warp whose range covers a whole head writes the output directly; a head split over several
 // warps is merged (log-sum-exp) by the warp that arrives last on the head's atomic ticket, which
 // then resets the ticket to zero.  No warp ever waits for another.
@@ -18,8 +19,9 @@
 // Arithmetic (CUDA cores, no tensor cores: one query row per head is a matrix-vector product).
 //   A6  logit_t = sum_c q_c (s_g code + z_g) = sum_c (q_c s_g) code_tc + sum_g z_g sum_{c in g} q_c.
 //       (q_c s_g) for one R-token block is turned into a 24-bit signed fixed-point integer split in
-//       three byte limbs; the codes are unpacked to bytes with one shift and masks, and dp4a forms
-//       byte dot products exactly in int32.  The block constant sum_g z_g q_g is added in fp32.
+//       three byte limbs (kept while the warp stays in the same block); the codes are unpacked to
+//       bytes with one shift and masks, and dp4a forms the byte dot products exactly in int32.
+//       The block constant sum_g z_g q_g is added in fp32.
 //   A8  online softmax in base 2 (q pre-scaled by scale*log2 e), warp-shuffle max, lane-local sums.
 //   A9  o_c = sum_t (p_t s_g(t)) code_tc + sum_t p_t z_g(t): (p_t s_g(t)) is turned into 24-bit
 //       unsigned fixed point relative to the unit's largest value and dotted with the V codes by
@@ -38,9 +40,9 @@ namespace kivi {
 namespace {
 
 constexpr int kWarps = 4;           // stream-K workers per CTA
-constexpr int kStageBytes = 8192;   // one unit: 4 KB K + 4 KB V
-constexpr int kHalfStage = 4096;
-constexpr int kResTokens = 16;      // tokens per residual unit
+constexpr int kStageBytes = 4096;   // one unit: 2 KB K + 2 KB V
+constexpr int kHalfStage = 2048;
+constexpr int kResTokens = 8;       // tokens per residual unit
 constexpr unsigned kFull = 0xffffffffu;
 constexpr float kQRange = 8388544.f;   // 2^23 - 64: largest |Q| before rounding (signed 24-bit limbs)
 constexpr float kPRange = 16777088.f;  // 2^24 - 128: largest P before rounding (unsigned 24-bit limbs)
@@ -48,8 +50,8 @@ constexpr float kPRange = 16777088.f;  // 2^24 - 128: largest P before rounding 
 template <int G>
 struct __align__(128) WarpSmem {
   uint8_t stage[2][kStageBytes];
-  uint4 qw[24];   // Q limbs: 96 words
-  uint4 pw[24];   // P limbs: 96 words
+  uint4 qw[G][24];  // Q limbs of each query: 96 words
+  uint4 pw[12];     // P limbs: 48 words
   float qf[G][kHeadDim];
   uint64_t bar[2];
 };
@@ -67,6 +69,18 @@ __device__ __forceinline__ float warp_sum(float v) {
 __device__ __forceinline__ uint32_t comp(const uint4& v, int i) {
   return i == 0 ? v.x : (i == 1 ? v.y : (i == 2 ? v.z : v.w));
 }
+// 1/x with the MUFU approximation (relative error < 2^-22).
+__device__ __forceinline__ float fast_rcp(float x) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+// 2^x with the MUFU approximation (relative error ~2^-22); exp2(-inf) = +0.
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 __device__ __forceinline__ float combine_limbs(int hi, int mid, int lo) {
   return fmaf(static_cast<float>(hi), 65536.f, fmaf(static_cast<float>(mid), 256.f, static_cast<float>(lo)));
 }
@@ -76,13 +90,47 @@ __device__ __forceinline__ long long worker_of(long long u, long long U, long lo
   return ((u + 1) * W + U - 1) / U - 1;
 }
 
+// dp4a of one packed 2-bit word against 4 sets x 3 limbs: sets 0/2 hold codes, sets 1/3 four times
+// the codes (the matching operand limbs are pre-divided by 4).
+__device__ __forceinline__ void dot2(uint32_t w, const uint4& L, const uint4& M, const uint4& H, int& al, int& am,
+                                     int& ah, bool signed_hi) {
+  const uint32_t w4 = w >> 4;
+  const uint32_t m0 = w & 0x03030303u, m1 = w & 0x0C0C0C0Cu;
+  const uint32_t m2 = w4 & 0x03030303u, m3 = w4 & 0x0C0C0C0Cu;
+  al = dp4a_uu(m0, L.x, al);
+  am = dp4a_uu(m0, M.x, am);
+  ah = signed_hi ? dp4a_us(m0, H.x, ah) : dp4a_uu(m0, H.x, ah);
+  al = dp4a_uu(m1, L.y, al);
+  am = dp4a_uu(m1, M.y, am);
+  ah = signed_hi ? dp4a_us(m1, H.y, ah) : dp4a_uu(m1, H.y, ah);
+  al = dp4a_uu(m2, L.z, al);
+  am = dp4a_uu(m2, M.z, am);
+  ah = signed_hi ? dp4a_us(m2, H.z, ah) : dp4a_uu(m2, H.z, ah);
+  al = dp4a_uu(m3, L.w, al);
+  am = dp4a_uu(m3, M.w, am);
+  ah = signed_hi ? dp4a_us(m3, H.w, ah) : dp4a_uu(m3, H.w, ah);
+}
+
+// The same for one packed 4-bit word against 2 sets x 3 limbs (low and high nibbles).
+__device__ __forceinline__ void dot4(uint32_t w, const uint2& L, const uint2& M, const uint2& H, int& al, int& am,
+                                     int& ah, bool signed_hi) {
+  const uint32_t n0 = w & 0x0F0F0F0Fu, n1 = (w >> 4) & 0x0F0F0F0Fu;
+  al = dp4a_uu(n0, L.x, al);
+  am = dp4a_uu(n0, M.x, am);
+  ah = signed_hi ? dp4a_us(n0, H.x, ah) : dp4a_uu(n0, H.x, ah);
+  al = dp4a_uu(n1, L.y, al);
+  am = dp4a_uu(n1, M.y, am);
+  ah = signed_hi ? dp4a_us(n1, H.y, ah) : dp4a_uu(n1, H.y, ah);
+}
+
 template <int BITS, int G>
 struct Decoder {
-  static constexpr int P = 32 / BITS;            // codes per word
-  static constexpr int UT = BITS == 2 ? 128 : 64; // tokens per quantized unit
+  static constexpr int P = 32 / BITS;             // codes per word
+  static constexpr int UT = BITS == 2 ? 64 : 32;  // tokens per quantized unit
   static constexpr int TPL = UT / 32;             // tokens per lane (K side)
   static constexpr int WPT = kHeadDim / P;        // K words per token
-  static constexpr int ROWS = UT / P;             // V word rows per unit (8)
+  static constexpr int ROWS = UT / P;             // V word rows per unit (4)
+  static constexpr int NSET = BITS == 2 ? 4 : 2;  // byte sets per word
 
   const DecodeArgs& a;
   WarpSmem<G>& S;
@@ -94,14 +142,15 @@ struct Decoder {
   float qreg[G][4];
   float qsum[G][4];
   float m[G], l[G], Z[G], o[G][4];
+  // per-block state: the Q limbs in S.qw belong to (head, block) == qkey
+  long long qkey;
+  float invq[G], cblk[G];
 
   __device__ Decoder(const DecodeArgs& args, WarpSmem<G>& smem, int ln, long long w, long long b, long long e)
-      : a(args), S(smem), lane(ln), worker(w), ub(b), ue(e), ngk(kHeadDim / args.group_k) {}
+      : a(args), S(smem), lane(ln), worker(w), ub(b), ue(e), ngk(kHeadDim >> args.lg_gk), qkey(-1) {}
 
   // ---- unit addressing ------------------------------------------------------------------
-  __device__ void issue(long long u, int stage) {  // lane 0 only
-    const long long head = u / a.units;
-    const int local = static_cast<int>(u % a.units);
+  __device__ void issue(long long head, int local, int stage) {  // lane 0 only
     uint8_t* dst = S.stage[stage];
     const void *ks, *vs;
     if (local < a.units_q) {
@@ -119,18 +168,17 @@ struct Decoder {
   }
 
   // (s, z) pairs of a quantized unit: lanes [0, ngk) hold K groups, lanes [8, 8 + nvg) V groups.
-  __device__ uint32_t load_pairs(long long u) const {
-    const long long head = u / a.units;
-    const int local = static_cast<int>(u % a.units);
+  __device__ uint32_t load_pairs(long long head, int local) const {
     if (local >= a.units_q) return 0u;
     const int tok0 = local * UT;
     if (lane < ngk) {
-      const size_t i = (static_cast<size_t>(head) * (a.capacity / a.residual) + tok0 / a.residual) * ngk + lane;
+      const size_t i =
+          (static_cast<size_t>(head) * a.blocks_per_head + (local >> a.lg_units_per_blk)) * ngk + lane;
       return static_cast<uint32_t>(__ldg(a.k_scale + i)) | (static_cast<uint32_t>(__ldg(a.k_zero + i)) << 16);
     }
-    const int nvg = UT >= a.group_v ? UT / a.group_v : 1;
+    const int nvg = (UT >> a.lg_gv) > 0 ? (UT >> a.lg_gv) : 1;
     if (lane >= 8 && lane < 8 + nvg) {
-      const size_t i = static_cast<size_t>(head) * (a.capacity / a.group_v) + tok0 / a.group_v + (lane - 8);
+      const size_t i = static_cast<size_t>(head) * a.vgroups_per_head + (tok0 >> a.lg_gv) + (lane - 8);
       return static_cast<uint32_t>(__ldg(a.v_scale + i)) | (static_cast<uint32_t>(__ldg(a.v_zero + i)) << 16);
     }
     return 0u;
@@ -153,7 +201,7 @@ struct Decoder {
         float part = 0.f;
 #pragma unroll
         for (int j = 0; j < 4; ++j)
-          if ((32 * j) / a.group_k == gi) part += qreg[g][j];
+          if (((32 * j) >> a.lg_gk) == gi) part += qreg[g][j];
         qsum[g][gi] = gi < ngk ? warp_sum(part) : 0.f;
       }
       m[g] = -INFINITY;
@@ -162,144 +210,127 @@ struct Decoder {
 #pragma unroll
       for (int e = 0; e < 4; ++e) o[g][e] = 0.f;
     }
+    qkey = -1;
     __syncwarp();
   }
 
-  // ---- one quantized unit -------------------------------------------------------------------
-  __device__ void quantized_unit(int stage, int tok0, uint32_t pairs) {
-    const uint8_t* kt = S.stage[stage];
-    const uint8_t* vt = S.stage[stage] + kHalfStage;
-    uint8_t* qwb = reinterpret_cast<uint8_t*>(S.qw);
-    uint8_t* pwb = reinterpret_cast<uint8_t*>(S.pw);
-    (void)tok0;
+  // ---- A6 set-up for one K block: fixed-point limbs of q_c * s_g(c) -------------------------
+  __device__ void build_q(uint32_t pairs) {
+    __syncwarp();  // the previous block's limbs are no longer read
 #pragma unroll
     for (int g = 0; g < G; ++g) {
-      // -- A6: fixed-point limbs of q_c * s_g(c) for this block
       float qv[4], mabs = 0.f;
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        const int gi = (32 * j) / a.group_k;
+        const int gi = (32 * j) >> a.lg_gk;
         const float s = h2f(static_cast<uint16_t>(__shfl_sync(kFull, pairs, gi) & 0xFFFFu));
         qv[j] = qreg[g][j] * s;
         mabs = fmaxf(mabs, fabsf(qv[j]));
       }
       mabs = warp_max(mabs);
-      // Q = rint(q s * scq) with |Q| <= 2^23 - 63: the margin keeps the rounded product of the
-      // largest element below 2^23 (it would wrap the signed top limb)
-      const float scq = mabs > 0.f ? kQRange / mabs : 0.f;
-      const float invq = mabs > 0.f ? mabs / kQRange : 0.f;
-      float cblk = 0.f;
+      // |Q| <= 2^23 - 61: the margin keeps the rounded largest element below 2^23, where the
+      // signed top limb would wrap (rcp and the product add at most 3 * 2^-22 relative)
+      const float scq = mabs > 0.f ? kQRange * fast_rcp(mabs) : 0.f;
+      invq[g] = mabs * (1.0f / kQRange);
+      float c = 0.f;
 #pragma unroll
       for (int gi = 0; gi < 4; ++gi) {
         if (gi < ngk) {
           const float z = h2f(static_cast<uint16_t>(__shfl_sync(kFull, pairs, gi) >> 16));
-          cblk = fmaf(z, qsum[g][gi], cblk);
+          c = fmaf(z, qsum[g][gi], c);
         }
       }
-      __syncwarp();
+      cblk[g] = c;
+      uint8_t* qwb = reinterpret_cast<uint8_t*>(S.qw[g]);
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        const int c = lane + 32 * j;
-        int word, k;
+        const int ch = lane + 32 * j;
         float f = qv[j] * scq;
+        int word, k, mb;
         if (BITS == 2) {  // word i = c/16, set k = c%4 (odd sets read as 4*code), byte m = (c%16)/4
-          k = c & 3;
-          word = c >> 4;
+          word = ch >> 4;
+          k = ch & 3;
+          mb = (ch >> 2) & 3;
           if (k & 1) f *= 0.25f;
         } else {          // word i = c/8, set k = c%2, byte m = (c%8)/2
-          k = c & 1;
-          word = c >> 3;
+          word = ch >> 3;
+          k = ch & 1;
+          mb = (ch >> 1) & 3;
         }
-        const int mb = BITS == 2 ? ((c >> 2) & 3) : ((c >> 1) & 3);
         const int Q = __float2int_rn(f);
-        const int nset = BITS == 2 ? 4 : 2;
-        uint8_t* base = qwb + ((word * 3) * nset + k) * 4 + mb;
+        uint8_t* base = qwb + ((word * 3) * NSET + k) * 4 + mb;
         base[0] = static_cast<uint8_t>(Q & 255);
-        base[nset * 4] = static_cast<uint8_t>((Q >> 8) & 255);
-        base[2 * nset * 4] = static_cast<uint8_t>((Q >> 16) & 255);
+        base[NSET * 4] = static_cast<uint8_t>((Q >> 8) & 255);
+        base[2 * NSET * 4] = static_cast<uint8_t>((Q >> 16) & 255);
       }
-      __syncwarp();
+    }
+    __syncwarp();
+  }
 
-      int al[TPL], am[TPL], ah[TPL];
+  // ---- A6 over the K codes of the unit: integer dot products of TPL tokens ----------------------
+  __device__ void k_dot(const uint8_t* kt, int g, int (&al)[TPL], int (&am)[TPL], int (&ah)[TPL]) const {
 #pragma unroll
-      for (int j = 0; j < TPL; ++j) al[j] = am[j] = ah[j] = 0;
-      if (BITS == 2) {
+    for (int j = 0; j < TPL; ++j) al[j] = am[j] = ah[j] = 0;
+    if (BITS == 2) {
+#pragma unroll 1
+      for (int h = 0; h < 2; ++h) {
+        const int hh = h ^ ((lane >> 2) & 1);  // bank-conflict-free order of the two 16-byte halves
+        uint4 kw[TPL];
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const int hh = h ^ ((lane >> 2) & 1);  // bank-conflict-free order of the two 16-byte halves
-          uint4 kw[TPL];
+        for (int j = 0; j < TPL; ++j) kw[j] = *reinterpret_cast<const uint4*>(kt + (lane + 32 * j) * 32 + 16 * hh);
+        const uint4* qrow = S.qw[g] + 12 * hh;
 #pragma unroll
-          for (int j = 0; j < TPL; ++j)
-            kw[j] = *reinterpret_cast<const uint4*>(kt + (lane + 32 * j) * 32 + 16 * hh);
+        for (int ii = 0; ii < 4; ++ii) {
+          const uint4 QL = qrow[ii * 3 + 0], QM = qrow[ii * 3 + 1], QH = qrow[ii * 3 + 2];
 #pragma unroll
-          for (int ii = 0; ii < 4; ++ii) {
-            const int i = 4 * hh + ii;
-            const uint4 QL = S.qw[i * 3 + 0], QM = S.qw[i * 3 + 1], QH = S.qw[i * 3 + 2];
-#pragma unroll
-            for (int j = 0; j < TPL; ++j) {
-              const uint32_t w = comp(kw[j], ii);
-              const uint32_t w4 = w >> 4;
-              const uint32_t m0 = w & 0x03030303u, m1 = w & 0x0C0C0C0Cu;
-              const uint32_t m2 = w4 & 0x03030303u, m3 = w4 & 0x0C0C0C0Cu;
-              al[j] = dp4a_uu(m0, QL.x, al[j]);
-              am[j] = dp4a_uu(m0, QM.x, am[j]);
-              ah[j] = dp4a_us(m0, QH.x, ah[j]);
-              al[j] = dp4a_uu(m1, QL.y, al[j]);
-              am[j] = dp4a_uu(m1, QM.y, am[j]);
-              ah[j] = dp4a_us(m1, QH.y, ah[j]);
-              al[j] = dp4a_uu(m2, QL.z, al[j]);
-              am[j] = dp4a_uu(m2, QM.z, am[j]);
-              ah[j] = dp4a_us(m2, QH.z, ah[j]);
-              al[j] = dp4a_uu(m3, QL.w, al[j]);
-              am[j] = dp4a_uu(m3, QM.w, am[j]);
-              ah[j] = dp4a_us(m3, QH.w, ah[j]);
-            }
-          }
-        }
-      } else {
-        const uint2* qw2 = reinterpret_cast<const uint2*>(S.qw);
-#pragma unroll
-        for (int qq = 0; qq < 4; ++qq) {
-          const int cq = (qq + (lane >> 1)) & 3;  // bank-conflict-free chunk order
-          uint4 kw[TPL];
-#pragma unroll
-          for (int j = 0; j < TPL; ++j)
-            kw[j] = *reinterpret_cast<const uint4*>(kt + (lane + 32 * j) * 64 + 16 * cq);
-#pragma unroll
-          for (int ii = 0; ii < 4; ++ii) {
-            const int i = 4 * cq + ii;
-            const uint2 QL = qw2[i * 3 + 0], QM = qw2[i * 3 + 1], QH = qw2[i * 3 + 2];
-#pragma unroll
-            for (int j = 0; j < TPL; ++j) {
-              const uint32_t w = comp(kw[j], ii);
-              const uint32_t n0 = w & 0x0F0F0F0Fu, n1 = (w >> 4) & 0x0F0F0F0Fu;
-              al[j] = dp4a_uu(n0, QL.x, al[j]);
-              am[j] = dp4a_uu(n0, QM.x, am[j]);
-              ah[j] = dp4a_us(n0, QH.x, ah[j]);
-              al[j] = dp4a_uu(n1, QL.y, al[j]);
-              am[j] = dp4a_uu(n1, QM.y, am[j]);
-              ah[j] = dp4a_us(n1, QH.y, ah[j]);
-            }
-          }
+          for (int j = 0; j < TPL; ++j) dot2(comp(kw[j], ii), QL, QM, QH, al[j], am[j], ah[j], true);
         }
       }
+    } else {
+      const uint2* qw2 = reinterpret_cast<const uint2*>(S.qw[g]);
+#pragma unroll 1
+      for (int qq = 0; qq < 4; ++qq) {
+        const int cq = (qq + (lane >> 1)) & 3;  // bank-conflict-free chunk order
+        const uint4 kw = *reinterpret_cast<const uint4*>(kt + lane * 64 + 16 * cq);
+        const uint2* qrow = qw2 + 12 * cq;
+#pragma unroll
+        for (int ii = 0; ii < 4; ++ii)
+          dot4(comp(kw, ii), qrow[ii * 3 + 0], qrow[ii * 3 + 1], qrow[ii * 3 + 2], al[0], am[0], ah[0], true);
+      }
+    }
+  }
+
+  // ---- one quantized unit -------------------------------------------------------------------
+  __device__ void quantized_unit(int stage, long long head, int local, uint32_t pairs) {
+    const uint8_t* kt = S.stage[stage];
+    const uint8_t* vt = S.stage[stage] + kHalfStage;
+    const long long key = head * a.blocks_per_head + (local >> a.lg_units_per_blk);
+    if (key != qkey) {
+      build_q(pairs);
+      qkey = key;
+    }
+    uint8_t* pwb = reinterpret_cast<uint8_t*>(S.pw);
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      int al[TPL], am[TPL], ah[TPL];
+      k_dot(kt, g, al, am, ah);
 
       // -- A8: online softmax over the unit's UT tokens
       float lg[TPL], mu = -INFINITY;
 #pragma unroll
       for (int j = 0; j < TPL; ++j) {
-        lg[j] = fmaf(combine_limbs(ah[j], am[j], al[j]), invq, cblk);
+        lg[j] = fmaf(combine_limbs(ah[j], am[j], al[j]), invq[g], cblk[g]);
         mu = fmaxf(mu, lg[j]);
       }
       mu = warp_max(mu);
       const float m_new = fmaxf(m[g], mu);
-      const float alpha = exp2f(m[g] - m_new);
+      const float alpha = fast_exp2(m[g] - m_new);
       float psum = 0.f, zsum = 0.f, mv = 0.f, pp[TPL];
 #pragma unroll
       for (int j = 0; j < TPL; ++j) {
-        const int vg = (32 * j) / a.group_v;  // V group of token lane + 32 j within the unit
-        const uint32_t vp = __shfl_sync(kFull, pairs, 8 + (UT >= a.group_v ? vg : 0));
-        const float p = exp2f(lg[j] - m_new);
+        const int vg = (32 * j) >> a.lg_gv;  // V group of token lane + 32 j within the unit
+        const uint32_t vp = __shfl_sync(kFull, pairs, 8 + vg);
+        const float p = fast_exp2(lg[j] - m_new);
         psum += p;
         zsum = fmaf(p, h2f(static_cast<uint16_t>(vp >> 16)), zsum);
         pp[j] = p * h2f(static_cast<uint16_t>(vp & 0xFFFFu));
@@ -312,9 +343,9 @@ struct Decoder {
 
       // -- A9: fixed-point limbs of p_t * s_g(t), then the V codes
       if (mv > 0.f) {
-        // P = rint(p s * scv) <= 2^24 - 127: the top token must not round to 2^24 (it would wrap to 0)
-        const float scv = kPRange / mv;
-        const float invv = mv / kPRange;
+        // P <= 2^24 - 124: the top token must not round to 2^24, where it would wrap to 0
+        const float scv = kPRange * fast_rcp(mv);
+        const float invv = mv * (1.0f / kPRange);
 #pragma unroll
         for (int j = 0; j < TPL; ++j) {
           const int t = lane + 32 * j;
@@ -331,78 +362,52 @@ struct Decoder {
             mb = (t >> 1) & 3;
           }
           const uint32_t Pq = __float2uint_rn(f);
-          const int nset = BITS == 2 ? 4 : 2;
-          uint8_t* base = pwb + ((row * 3) * nset + k) * 4 + mb;
+          uint8_t* base = pwb + ((row * 3) * NSET + k) * 4 + mb;
           base[0] = static_cast<uint8_t>(Pq & 255u);
-          base[nset * 4] = static_cast<uint8_t>((Pq >> 8) & 255u);
-          base[2 * nset * 4] = static_cast<uint8_t>((Pq >> 16) & 255u);
+          base[NSET * 4] = static_cast<uint8_t>((Pq >> 8) & 255u);
+          base[2 * NSET * 4] = static_cast<uint8_t>((Pq >> 16) & 255u);
         }
         __syncwarp();
         int vl[4] = {0, 0, 0, 0}, vm[4] = {0, 0, 0, 0}, vh[4] = {0, 0, 0, 0};
-#pragma unroll
+#pragma unroll 2
         for (int r = 0; r < ROWS; ++r) {
           const uint4 vw = *reinterpret_cast<const uint4*>(vt + r * 512 + 16 * lane);
           if (BITS == 2) {
             const uint4 PL = S.pw[r * 3 + 0], PM = S.pw[r * 3 + 1], PH = S.pw[r * 3 + 2];
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const uint32_t w = comp(vw, e);
-              const uint32_t w4 = w >> 4;
-              const uint32_t m0 = w & 0x03030303u, m1 = w & 0x0C0C0C0Cu;
-              const uint32_t m2 = w4 & 0x03030303u, m3 = w4 & 0x0C0C0C0Cu;
-              vl[e] = dp4a_uu(m0, PL.x, vl[e]);
-              vm[e] = dp4a_uu(m0, PM.x, vm[e]);
-              vh[e] = dp4a_uu(m0, PH.x, vh[e]);
-              vl[e] = dp4a_uu(m1, PL.y, vl[e]);
-              vm[e] = dp4a_uu(m1, PM.y, vm[e]);
-              vh[e] = dp4a_uu(m1, PH.y, vh[e]);
-              vl[e] = dp4a_uu(m2, PL.z, vl[e]);
-              vm[e] = dp4a_uu(m2, PM.z, vm[e]);
-              vh[e] = dp4a_uu(m2, PH.z, vh[e]);
-              vl[e] = dp4a_uu(m3, PL.w, vl[e]);
-              vm[e] = dp4a_uu(m3, PM.w, vm[e]);
-              vh[e] = dp4a_uu(m3, PH.w, vh[e]);
-            }
+            for (int e = 0; e < 4; ++e) dot2(comp(vw, e), PL, PM, PH, vl[e], vm[e], vh[e], false);
           } else {
             const uint2* pw2 = reinterpret_cast<const uint2*>(S.pw);
             const uint2 PL = pw2[r * 3 + 0], PM = pw2[r * 3 + 1], PH = pw2[r * 3 + 2];
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const uint32_t w = comp(vw, e);
-              const uint32_t n0 = w & 0x0F0F0F0Fu, n1 = (w >> 4) & 0x0F0F0F0Fu;
-              vl[e] = dp4a_uu(n0, PL.x, vl[e]);
-              vm[e] = dp4a_uu(n0, PM.x, vm[e]);
-              vh[e] = dp4a_uu(n0, PH.x, vh[e]);
-              vl[e] = dp4a_uu(n1, PL.y, vl[e]);
-              vm[e] = dp4a_uu(n1, PM.y, vm[e]);
-              vh[e] = dp4a_uu(n1, PH.y, vh[e]);
-            }
+            for (int e = 0; e < 4; ++e) dot4(comp(vw, e), PL, PM, PH, vl[e], vm[e], vh[e], false);
           }
         }
 #pragma unroll
         for (int e = 0; e < 4; ++e) o[g][e] = fmaf(o[g][e], alpha, combine_limbs(vh[e], vm[e], vl[e]) * invv);
+        __syncwarp();  // pw is rewritten by the next query or unit
       } else {
 #pragma unroll
         for (int e = 0; e < 4; ++e) o[g][e] *= alpha;
       }
-      __syncwarp();  // qw / pw are rewritten by the next query or unit
     }
   }
 
-  // ---- one residual unit (fp16 rows) --------------------------------------------------------
+  // ---- one residual unit (8 fp16 rows) -------------------------------------------------------
   __device__ void residual_unit(int stage, int nvalid) {
     const uint8_t* kt = S.stage[stage];
     const uint8_t* vt = S.stage[stage] + kHalfStage;
-    const int t = lane >> 1, hf = lane & 1;
+    const int t = lane >> 2, quarter = lane & 3;  // 4 lanes per token, 32 channels each
 #pragma unroll
     for (int g = 0; g < G; ++g) {
       float dot = 0.f;
 #pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        const int cc = (k + lane) & 7;  // bank-conflict-free chunk order
-        const uint4 kv = *reinterpret_cast<const uint4*>(kt + t * 256 + hf * 128 + 16 * cc);
-        const float4 q0 = *reinterpret_cast<const float4*>(&S.qf[g][64 * hf + 8 * cc]);
-        const float4 q1 = *reinterpret_cast<const float4*>(&S.qf[g][64 * hf + 8 * cc + 4]);
+      for (int k = 0; k < 4; ++k) {
+        const int cc = (k + (lane >> 1)) & 3;  // bank-conflict-free chunk order
+        const int c0 = 32 * quarter + 8 * cc;
+        const uint4 kv = *reinterpret_cast<const uint4*>(kt + t * 256 + 2 * c0);
+        const float4 q0 = *reinterpret_cast<const float4*>(&S.qf[g][c0]);
+        const float4 q1 = *reinterpret_cast<const float4*>(&S.qf[g][c0 + 4]);
         const float2 k0 = __half22float2(*reinterpret_cast<const __half2*>(&kv.x));
         const float2 k1 = __half22float2(*reinterpret_cast<const __half2*>(&kv.y));
         const float2 k2 = __half22float2(*reinterpret_cast<const __half2*>(&kv.z));
@@ -417,19 +422,19 @@ struct Decoder {
         dot = fmaf(q1.w, k3.y, dot);
       }
       dot += __shfl_xor_sync(kFull, dot, 1);
+      dot += __shfl_xor_sync(kFull, dot, 2);
       const bool valid = t < nvalid;
       const float lg = valid ? dot : -INFINITY;
       const float m_new = fmaxf(m[g], warp_max(lg));
-      const float alpha = exp2f(m[g] - m_new);
-      const float p = valid ? exp2f(lg - m_new) : 0.f;
+      const float alpha = fast_exp2(m[g] - m_new);
+      const float p = valid ? fast_exp2(lg - m_new) : 0.f;
       m[g] = m_new;
-      l[g] = fmaf(l[g], alpha, hf == 0 ? p : 0.f);
+      l[g] = fmaf(l[g], alpha, quarter == 0 ? p : 0.f);
       Z[g] *= alpha;
 #pragma unroll
       for (int e = 0; e < 4; ++e) o[g][e] *= alpha;
-#pragma unroll 4
       for (int tt = 0; tt < nvalid; ++tt) {
-        const float pt = __shfl_sync(kFull, p, 2 * tt);
+        const float pt = __shfl_sync(kFull, p, 4 * tt);
         const uint2 vv = *reinterpret_cast<const uint2*>(vt + tt * 256 + 8 * lane);
         const float2 v0 = __half22float2(*reinterpret_cast<const __half2*>(&vv.x));
         const float2 v1 = __half22float2(*reinterpret_cast<const __half2*>(&vv.y));
@@ -492,7 +497,7 @@ struct Decoder {
       for (long long x = wfirst; x <= wlast; ++x) {
         const int sx = (U * x / W) >= h0 ? 0 : 1;
         const float* p = a.partials + ((x * 2 + sx) * G + g) * kPartialStride;
-        const float w = exp2f(__ldcg(p) - mm);
+        const float w = fast_exp2(__ldcg(p) - mm);
         const float lx = __ldcg(p + 1);
         if (!(lx > 0.f) && lane == 0) report_status(a.status, KIVI_ERR_INTERNAL);  // never written
         ls = fmaf(w, lx, ls);
@@ -537,25 +542,33 @@ struct Decoder {
       asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     __syncwarp();
+    // (head, local unit) cursors for the current unit, the next one (scales) and the one after
+    // (bulk copies); advanced by increments, no division on the per-unit path
+    long long head = ub / a.units;
+    int local = static_cast<int>(ub - head * a.units);
+    long long h1 = head, h2;
+    int l1 = local, l2;
+    advance(h1, l1);
+    h2 = h1;
+    l2 = l1;
+    advance(h2, l2);
     if (lane == 0) {
-      issue(ub, 0);
-      if (ub + 1 < ue) issue(ub + 1, 1);
+      issue(head, local, 0);
+      if (ub + 1 < ue) issue(h1, l1, 1);
     }
-    uint32_t pairs = load_pairs(ub);
+    uint32_t pairs = load_pairs(head, local);
     long long cur_head = -1, seg_a = ub;
     int it = 0;
     for (long long u = ub; u < ue; ++u, ++it) {
       const int stage = it & 1;
       const uint32_t parity = (it >> 1) & 1;
-      const long long head = u / a.units;
-      const int local = static_cast<int>(u % a.units);
       if (head != cur_head) {
         if (cur_head >= 0) finish_segment(cur_head, seg_a, u);
         start_head(head);
         cur_head = head;
         seg_a = u;
       }
-      const uint32_t pairs_next = (u + 1 < ue) ? load_pairs(u + 1) : 0u;
+      const uint32_t pairs_next = (u + 1 < ue) ? load_pairs(h1, l1) : 0u;
       if (!wait_stage(stage, parity)) {
         // Give up: record the error, let this warp's copies in flight land, and leave.
         if (lane == 0) report_status(a.status, KIVI_ERR_DEVICE_TIMEOUT);
@@ -564,22 +577,34 @@ struct Decoder {
         return;
       }
       if (local < a.units_q) {
-        quantized_unit(stage, local * UT, pairs);
+        quantized_unit(stage, head, local, pairs);
       } else {
         const int t0 = (local - a.units_q) * kResTokens;
         residual_unit(stage, min(kResTokens, a.n_res - t0));
       }
       __syncwarp();
       fence_proxy_async_smem();
-      if (lane == 0 && u + 2 < ue) issue(u + 2, stage);
+      if (lane == 0 && u + 2 < ue) issue(h2, l2, stage);
       pairs = pairs_next;
+      head = h1;
+      local = l1;
+      h1 = h2;
+      l1 = l2;
+      advance(h2, l2);
     }
     finish_segment(cur_head, seg_a, ue);
+  }
+
+  __device__ __forceinline__ void advance(long long& h, int& l) const {
+    if (++l == a.units) {
+      l = 0;
+      ++h;
+    }
   }
 };
 
 template <int BITS, int G>
-__global__ void __launch_bounds__(kWarps * 32) decode_kernel(const __grid_constant__ DecodeArgs a) {
+__global__ void __launch_bounds__(kWarps * 32, G == 1 ? 5 : 1) decode_kernel(const __grid_constant__ DecodeArgs a) {
   extern __shared__ __align__(128) uint8_t smem_raw[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   WarpSmem<G>& S = reinterpret_cast<WarpSmem<G>*>(smem_raw)[warp];
@@ -606,6 +631,8 @@ cudaError_t plan_for(DecodePlan* plan) {
   plan->warps_per_cta = kWarps;
   plan->ctas = sms * occ;
   plan->smem_bytes = smem;
+  plan->unit_tokens = Decoder<BITS, G>::UT;
+  plan->res_unit_tokens = kResTokens;
   return cudaSuccess;
 }
 

@@ -48,6 +48,10 @@ struct DecodeArgs {
   int units_q;        // quantized units per head
   int units;          // units per head (quantized + residual)
   long long total_units;
+  int blocks_per_head;   // capacity / residual (K scale rows per head)
+  int vgroups_per_head;  // capacity / group_v (V scales per head)
+  int lg_gk, lg_gv;      // log2(group_k), log2(group_v)
+  int lg_units_per_blk;  // log2(residual / tokens per quantized unit)
   int workers;
   float qscale;       // softmax scale * log2(e)
   unsigned long long timeout_ns;
@@ -64,6 +68,8 @@ struct DecodePlan {
   int warps_per_cta;
   int ctas;
   int smem_bytes;
+  int unit_tokens;      // tokens per quantized unit
+  int res_unit_tokens;  // tokens per residual unit
   int workers() const { return warps_per_cta * ctas; }
 };
 cudaError_t decode_plan(int bits, int gqa, DecodePlan* plan);

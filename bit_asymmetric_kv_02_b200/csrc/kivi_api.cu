@@ -28,20 +28,25 @@ DebugState& debug_state() {
   return s;
 }
 
+bool pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
+int log2i(int x) {
+  int r = 0;
+  while ((1 << r) < x) ++r;
+  return r;
+}
+
 bool aligned16(const void* p) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
-
-int unit_tokens(int bits) { return bits == 2 ? 128 : 64; }
 
 int check_cfg(const kivi_config* c) {
   if (c == nullptr) return KIVI_ERR_INVALID_ARG;
   if (c->head_dim != kHeadDim) return KIVI_ERR_UNSUPPORTED;
   if (c->bits != 2 && c->bits != 4) return KIVI_ERR_UNSUPPORTED;
   if (c->batch < 1 || c->num_kv_heads < 1 || c->capacity < 0) return KIVI_ERR_INVALID_ARG;
-  if (c->residual < 128 || c->residual > 1024 || c->residual % 128 != 0) return KIVI_ERR_INVALID_ARG;
+  if (c->residual < 128 || c->residual > 1024 || !pow2(c->residual)) return KIVI_ERR_INVALID_ARG;
   if (c->capacity % c->residual != 0) return KIVI_ERR_INVALID_ARG;
   if (c->group_k != 32 && c->group_k != 64 && c->group_k != 128) return KIVI_ERR_INVALID_ARG;
-  if (c->group_v < 32 || c->group_v % 32 != 0 || c->residual % c->group_v != 0) return KIVI_ERR_INVALID_ARG;
+  if (c->group_v < 32 || !pow2(c->group_v) || c->group_v > c->residual) return KIVI_ERR_INVALID_ARG;
   if (static_cast<long long>(c->batch) * c->num_kv_heads > (1ll << 30)) return KIVI_ERR_UNSUPPORTED;
   if (c->capacity / c->residual > 32767) return KIVI_ERR_UNSUPPORTED;  // grid.y limit of a prefill
   return KIVI_OK;
@@ -266,7 +271,6 @@ int kivi_decode_attention(const kivi_config* cfg, const kivi_cache* cache, const
       workspace_bytes < part_bytes + align256(bh * 4))
     return KIVI_ERR_WORKSPACE;
 
-  const int ut = unit_tokens(cfg->bits);
   DecodeArgs a{};
   a.k_codes = cache->k_codes;
   a.v_codes = cache->v_codes;
@@ -289,9 +293,14 @@ int kivi_decode_attention(const kivi_config* cfg, const kivi_cache* cache, const
   a.group_v = cfg->group_v;
   a.n_quant = cache->n_quant;
   a.n_res = cache->n_res;
-  a.units_q = cache->n_quant / ut;
-  a.units = a.units_q + (cache->n_res + 15) / 16;
+  a.units_q = cache->n_quant / plan.unit_tokens;
+  a.units = a.units_q + (cache->n_res + plan.res_unit_tokens - 1) / plan.res_unit_tokens;
   a.total_units = static_cast<long long>(bh) * a.units;
+  a.blocks_per_head = cfg->capacity / cfg->residual;
+  a.vgroups_per_head = cfg->capacity / cfg->group_v;
+  a.lg_gk = log2i(cfg->group_k);
+  a.lg_gv = log2i(cfg->group_v);
+  a.lg_units_per_blk = log2i(cfg->residual / plan.unit_tokens);
   // every worker must own at least one unit: the merge counts all workers that touch a head
   long long workers = a.total_units < plan.workers() ? a.total_units : plan.workers();
   {

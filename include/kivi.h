@@ -74,8 +74,8 @@ extern "C" {
  * Quantization configuration; mirrors the page's QuantConfig (section アルゴリズム: bits,
  * group_size_k, group_size_v, residual_length) plus the shape and capacity of the cache.
  * Rules: batch >= 1, num_kv_heads >= 1, capacity >= 0, capacity % residual == 0,
- * group_k in {32, 64, 128}, group_v % 32 == 0 and group_v divides residual,
- * residual % 128 == 0 and 128 <= residual <= 1024 (KIVI_ERR_INVALID_ARG otherwise);
+ * residual in {128, 256, 512, 1024}, group_k in {32, 64, 128}, group_v a power of two with
+ * 32 <= group_v <= residual (KIVI_ERR_INVALID_ARG otherwise);
  * head_dim == 128, bits in {2, 4} (KIVI_ERR_UNSUPPORTED otherwise).
  */
 typedef struct kivi_config {

@@ -52,6 +52,10 @@ def test_config_rules(kivi):
     assert kivi.kivi_check_config(_cfg(kivi, group_k=48)) == 1
     assert kivi.kivi_check_config(_cfg(kivi, group_v=48)) == 1
     assert kivi.kivi_check_config(_cfg(kivi, residual=100)) == 1
+    assert kivi.kivi_check_config(_cfg(kivi, residual=384, capacity=768)) == 1
+    assert kivi.kivi_check_config(_cfg(kivi, group_v=96)) == 1
+    assert kivi.kivi_check_config(_cfg(kivi, group_v=256)) == 1
+    assert kivi.kivi_check_config(_cfg(kivi, residual=256, group_v=256, capacity=1024)) == 0
     assert kivi.kivi_check_config(_cfg(kivi, capacity=1000)) == 1
     assert kivi.kivi_check_config(_cfg(kivi, batch=0)) == 1
     assert kivi.kivi_check_config(_cfg(kivi, bits=4, group_k=128, group_v=128)) == 0

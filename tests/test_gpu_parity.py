@@ -130,6 +130,33 @@ def test_streaming_append_flush(bits, group):
     assert cache.read_status() == 0
 
 
+@pytest.mark.parametrize("workers", [1, 2, 3, 5, 13, 0])
+def test_forced_splits_match_oracle(workers):
+    """The same cache decoded with 1, 2, 3, 5, 13 or the default number of workers: every split of
+    heads across warps (direct writes, merges of 2..N partials, several heads per warp) matches."""
+    kivi = _kivi()
+    w = synth.TINY.with_(name="splits", batch=3, q_heads=4, kv_heads=2, tokens=5 * 128 + 77, seed=70)
+    k, v = synth.prompt_kv(w, w.tokens)
+    q = synth.queries(w)
+    cap = 768
+    cache = kivi.KiviCache(w.batch, w.kv_heads, cap, num_q_heads=w.q_heads)
+    cache.prefill(torch.from_numpy(k).cuda(), torch.from_numpy(v).cuda())
+    try:
+        kivi.kivi_debug_inject(2, workers)
+        cache.status.zero_()
+        out = cache.attend(torch.from_numpy(q).cuda()).cpu().numpy()
+        assert cache.read_status() == 0
+    finally:
+        kivi.kivi_debug_inject(0, 0)
+    for b in range(w.batch):
+        for h in range(w.kv_heads):
+            hc = O.HeadCache(128, 2, 32, 32, 128, cap)
+            hc.prefill(k[b, h], v[b, h])
+            g = w.gqa
+            gc.assert_attention_close(out[b, h * g:(h + 1) * g], hc.attend(q[b, h * g:(h + 1) * g], gc.default_scale()),
+                                      f"workers={workers} head {(b, h)}")
+
+
 def test_prefill_equals_streaming_on_gpu():
     """The GPU cache after prefill(T) equals the GPU cache after prefill(T0) + appends/flushes."""
     kivi = _kivi()
