@@ -14,7 +14,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libkivi.so")
-SOURCES = ["kivi_api.cu", "quantize.cu", "decode.cu"]
+SOURCES = ["kivi_api.cu", "quantize.cu", "decode.cu", "noalloc.cu"]
 HEADERS = ["common.cuh", "kernels.h"]
 
 

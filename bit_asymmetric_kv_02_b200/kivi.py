@@ -66,6 +66,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "kivi_flush_residual": (I32, [cfgp, cachep, P]),
         "kivi_decode_workspace_bytes": (SZ, [cfgp, I32]),
         "kivi_decode_attention": (I32, [cfgp, cachep, P, I32, ctypes.c_float, P, P, SZ, P, P]),
+        "kivi_decode_attention_noalloc": (I32, [cfgp, cachep, P, I32, ctypes.c_float, P, P, P]),
         "kivi_read_status": (I32, [P, P]),
         "kivi_debug_inject": (I32, [I32, U64]),
     }
@@ -124,6 +125,15 @@ def kivi_decode_attention(cfg, cache, q_ptr: int, num_q_heads: int, scale: float
     _check(load_library().kivi_decode_attention(ctypes.byref(cfg), ctypes.byref(cache), q_ptr, num_q_heads,
                                                 scale, out_ptr, ws_ptr, ws_bytes, status_ptr, stream),
            "kivi_decode_attention")
+
+
+def kivi_decode_attention_noalloc(cfg, cache, q_ptr: int, num_q_heads: int, scale: float, out_ptr: int,
+                                  status_ptr: int | None, stream: int) -> None:
+    """Decode attention with the library's fixed scratch array instead of a caller workspace, for
+    callers that cannot allocate device memory at decode time (see include/kivi.h)."""
+    _check(load_library().kivi_decode_attention_noalloc(ctypes.byref(cfg), ctypes.byref(cache), q_ptr, num_q_heads,
+                                                        scale, out_ptr, status_ptr, stream),
+           "kivi_decode_attention_noalloc")
 
 
 def kivi_read_status(status_ptr: int, stream: int) -> int:

@@ -23,7 +23,8 @@
  *     is flushed (quantized as one R-token block) before the next append.
  *
  * Every pointer argument named *_dev is DEVICE memory owned by the caller; the library never
- * allocates, frees or retains memory.
+ * allocates, frees or retains memory (kivi_decode_attention_noalloc's fixed scratch array is
+ * part of the library image, not an allocation).
  * fp16 values are passed as their IEEE binary16 bit patterns (uint16_t).  Every call is
  * asynchronous on `stream` (a cudaStream_t passed as void*; NULL = legacy default stream) and
  * returns a status code synchronously.  On any error return nothing has been enqueued and the
@@ -156,6 +157,34 @@ size_t kivi_decode_workspace_bytes(const kivi_config* cfg, int32_t num_q_heads);
 int kivi_decode_attention(const kivi_config* cfg, const kivi_cache* cache, const uint16_t* q_dev,
                           int32_t num_q_heads, float scale, uint16_t* out_dev, void* workspace_dev,
                           size_t workspace_bytes, int32_t* dev_status, void* stream);
+
+/*
+ * Largest scratch kivi_decode_attention_noalloc can use, in bytes (see below).
+ */
+#define KIVI_NOALLOC_SCRATCH_BYTES (16u << 20)
+
+/*
+ * Decode attention that allocates nothing.  The paper has no counterpart: this is a variant of
+ * kivi_decode_attention for callers that cannot allocate device memory when they decode, for
+ * example a serving process that hands all free device memory to its own pool at start-up (a
+ * cudaMalloc later would fail or stall the step), or a host that gives this library only the
+ * input and output buffers of each call.  Arguments, results and errors are those of
+ * kivi_decode_attention without the workspace: the scratch (split partials and per-head tickets)
+ * lives in a fixed array of KIVI_NOALLOC_SCRATCH_BYTES inside the library, which every GPU that
+ * loads the library holds until the process exits.  The caller still passes q and out.
+ *   - Limit: if kivi_decode_workspace_bytes(cfg, num_q_heads) exceeds KIVI_NOALLOC_SCRATCH_BYTES
+ *     (very many heads), the call returns KIVI_ERR_WORKSPACE and enqueues nothing; use
+ *     kivi_decode_attention with a caller workspace instead.
+ *   - Set-up: the first call on each device looks up the array's device address on that device
+ *     (cudaGetSymbolAddress); make that first call before any stream capture.
+ *   - Sharing: every call uses the same array.  Each call first clears the tickets (an async
+ *     memset on `stream`), so the contents left by an earlier call, even a failed one, do not
+ *     matter; but calls whose work overlaps on the GPU (different streams, or several host threads
+ *     on one device) race on the array and must be serialized by the caller.
+ */
+int kivi_decode_attention_noalloc(const kivi_config* cfg, const kivi_cache* cache, const uint16_t* q_dev,
+                                  int32_t num_q_heads, float scale, uint16_t* out_dev, int32_t* dev_status,
+                                  void* stream);
 
 /* Synchronizes `stream` and returns the device-side status word (KIVI_OK if it is 0). */
 int kivi_read_status(const int32_t* dev_status, void* stream);
