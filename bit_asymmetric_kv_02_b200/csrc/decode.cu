@@ -5,13 +5,14 @@
 //     out = softmax(scale * q [D(K_quant); K_res]^T) [D(V_quant); V_res],  D(x^) = s x^ + z.
 //
 // Work decomposition (stream-K over warps).  Every (batch, KV head) is a sequence of equal-size
-// 4 KB "units": quantized units of UT tokens (UT = 64 at 2 bits, 32 at 4 bits; 2 KB of K codes +
-// 2 KB of V codes) followed by residual units of 8 fp16 tokens (2 KB K + 2 KB V).  The global
+// 8 KB "units": quantized units of UT tokens (UT = 128 at 2 bits, 64 at 4 bits; 4 KB of K codes +
+// 4 KB of V codes) followed by residual units of 16 fp16 tokens (4 KB K + 4 KB V).  The global
 // unit sequence is cut into one contiguous range per warp, so the load is balanced to one unit
-// whatever the batch, head count or context length.  Each warp streams its range through two
-// 4 KB shared-memory stages filled by 1-D TMA bulk copies (cp.async.bulk, no multicast) and
-// completed on an mbarrier; small stages leave room for ~20 resident warps per SM.  Every wait is
-// bounded and reports KIVI_ERR_DEVICE_TIMEOUT.
+// whatever the batch, head count or context length.  Each warp streams its range as half units
+// K0 V0 K1 V1 ... through a ring of three 4 KB shared-memory buffers filled by 1-D TMA bulk copies
+// (cp.async.bulk, no multicast) and completed on mbarriers: half h uses buffer h % 3 and is
+// reissued as soon as half h - 3 is consumed, which keeps one unit in flight with 12 KB per warp
+// (16 resident warps per SM).  Every wait is bounded and reports KIVI_ERR_DEVICE_TIMEOUT.
 // A warp whose range covers a whole head writes the output directly; a head split over several
 // warps is merged (log-sum-exp) by the warp that arrives last on the head's atomic ticket, which
 // then resets the ticket to zero.  No warp ever waits for another.
@@ -40,20 +41,20 @@ namespace kivi {
 namespace {
 
 constexpr int kWarps = 4;           // stream-K workers per CTA
-constexpr int kStageBytes = 4096;   // one unit: 2 KB K + 2 KB V
-constexpr int kHalfStage = 2048;
-constexpr int kResTokens = 8;       // tokens per residual unit
+constexpr int kHalfBytes = 4096;    // one half unit: the K part or the V part of a unit
+constexpr int kBuffers = 3;         // half-unit buffers per warp (ring K0 V0 K1 | V1 K2 V2 | ...)
+constexpr int kResTokens = 16;      // tokens per residual unit
 constexpr unsigned kFull = 0xffffffffu;
 constexpr float kQRange = 8388544.f;   // 2^23 - 64: largest |Q| before rounding (signed 24-bit limbs)
 constexpr float kPRange = 16777088.f;  // 2^24 - 128: largest P before rounding (unsigned 24-bit limbs)
 
 template <int G>
 struct __align__(128) WarpSmem {
-  uint8_t stage[2][kStageBytes];
+  uint8_t buf[kBuffers][kHalfBytes];
   uint4 qw[G][24];  // Q limbs of each query: 96 words
-  uint4 pw[12];     // P limbs: 48 words
+  uint4 pw[G][24];  // P limbs of each query: up to 96 words
   float qf[G][kHeadDim];
-  uint64_t bar[2];
+  uint64_t bar[kBuffers];
 };
 
 __device__ __forceinline__ float warp_max(float v) {
@@ -125,12 +126,12 @@ __device__ __forceinline__ void dot4(uint32_t w, const uint2& L, const uint2& M,
 
 template <int BITS, int G>
 struct Decoder {
-  static constexpr int P = 32 / BITS;             // codes per word
-  static constexpr int UT = BITS == 2 ? 64 : 32;  // tokens per quantized unit
-  static constexpr int TPL = UT / 32;             // tokens per lane (K side)
-  static constexpr int WPT = kHeadDim / P;        // K words per token
-  static constexpr int ROWS = UT / P;             // V word rows per unit (4)
-  static constexpr int NSET = BITS == 2 ? 4 : 2;  // byte sets per word
+  static constexpr int P = 32 / BITS;              // codes per word
+  static constexpr int UT = BITS == 2 ? 128 : 64;  // tokens per quantized unit (8 KB of codes)
+  static constexpr int TPL = UT / 32;              // tokens per lane (K side)
+  static constexpr int WPT = kHeadDim / P;         // K words per token
+  static constexpr int ROWS = UT / P;              // V word rows per unit (8)
+  static constexpr int NSET = BITS == 2 ? 4 : 2;   // byte sets per word
 
   const DecodeArgs& a;
   WarpSmem<G>& S;
@@ -145,26 +146,30 @@ struct Decoder {
   // per-block state: the Q limbs in S.qw belong to (head, block) == qkey
   long long qkey;
   float invq[G], cblk[G];
+  // state handed from the K half to the V half of a unit
+  float alpha_[G], invv_[G], pres_[G];
+  bool hasv_[G];
 
   __device__ Decoder(const DecodeArgs& args, WarpSmem<G>& smem, int ln, long long w, long long b, long long e)
       : a(args), S(smem), lane(ln), worker(w), ub(b), ue(e), ngk(kHeadDim >> args.lg_gk), qkey(-1) {}
 
-  // ---- unit addressing ------------------------------------------------------------------
-  __device__ void issue(long long head, int local, int stage) {  // lane 0 only
-    uint8_t* dst = S.stage[stage];
-    const void *ks, *vs;
+  // ---- half-unit addressing: half h of the warp's range is the K (h even) or V (h odd) part -----
+  __device__ void issue_half(int h, long long head, int local) {  // lane 0 only
+    const int b = h % kBuffers;
+    const bool is_v = h & 1;
+    const void* src;
     if (local < a.units_q) {
       const size_t tok0 = static_cast<size_t>(local) * UT;
-      ks = a.k_codes + (static_cast<size_t>(head) * a.capacity + tok0) * WPT;
-      vs = a.v_codes + (static_cast<size_t>(head) * (a.capacity / P) + tok0 / P) * kHeadDim;
+      src = is_v ? static_cast<const void*>(a.v_codes + (static_cast<size_t>(head) * (a.capacity / P) + tok0 / P) *
+                                                            kHeadDim)
+                 : static_cast<const void*>(a.k_codes + (static_cast<size_t>(head) * a.capacity + tok0) * WPT);
     } else {
       const size_t t0 = static_cast<size_t>(local - a.units_q) * kResTokens;
-      ks = a.k_res + (static_cast<size_t>(head) * a.residual + t0) * kHeadDim;
-      vs = a.v_res + (static_cast<size_t>(head) * a.residual + t0) * kHeadDim;
+      const uint16_t* base = is_v ? a.v_res : a.k_res;
+      src = base + (static_cast<size_t>(head) * a.residual + t0) * kHeadDim;
     }
-    mbar_arrive_expect_tx(&S.bar[stage], kStageBytes + a.debug_extra_tx);
-    bulk_g2s(dst, ks, kHalfStage, &S.bar[stage]);
-    bulk_g2s(dst + kHalfStage, vs, kHalfStage, &S.bar[stage]);
+    mbar_arrive_expect_tx(&S.bar[b], kHalfBytes + a.debug_extra_tx);
+    bulk_g2s(S.buf[b], src, kHalfBytes, &S.bar[b]);
   }
 
   // (s, z) pairs of a quantized unit: lanes [0, ngk) hold K groups, lanes [8, 8 + nvg) V groups.
@@ -267,7 +272,7 @@ struct Decoder {
     __syncwarp();
   }
 
-  // ---- A6 over the K codes of the unit: integer dot products of TPL tokens ----------------------
+  // ---- A6 over the K codes of a unit: integer dot products of TPL tokens per lane --------------
   __device__ void k_dot(const uint8_t* kt, int g, int (&al)[TPL], int (&am)[TPL], int (&ah)[TPL]) const {
 #pragma unroll
     for (int j = 0; j < TPL; ++j) al[j] = am[j] = ah[j] = 0;
@@ -291,31 +296,31 @@ struct Decoder {
 #pragma unroll 1
       for (int qq = 0; qq < 4; ++qq) {
         const int cq = (qq + (lane >> 1)) & 3;  // bank-conflict-free chunk order
-        const uint4 kw = *reinterpret_cast<const uint4*>(kt + lane * 64 + 16 * cq);
+        uint4 kw[TPL];
+#pragma unroll
+        for (int j = 0; j < TPL; ++j) kw[j] = *reinterpret_cast<const uint4*>(kt + (lane + 32 * j) * 64 + 16 * cq);
         const uint2* qrow = qw2 + 12 * cq;
 #pragma unroll
-        for (int ii = 0; ii < 4; ++ii)
-          dot4(comp(kw, ii), qrow[ii * 3 + 0], qrow[ii * 3 + 1], qrow[ii * 3 + 2], al[0], am[0], ah[0], true);
+        for (int ii = 0; ii < 4; ++ii) {
+          const uint2 QL = qrow[ii * 3 + 0], QM = qrow[ii * 3 + 1], QH = qrow[ii * 3 + 2];
+#pragma unroll
+          for (int j = 0; j < TPL; ++j) dot4(comp(kw[j], ii), QL, QM, QH, al[j], am[j], ah[j], true);
+        }
       }
     }
   }
 
-  // ---- one quantized unit -------------------------------------------------------------------
-  __device__ void quantized_unit(int stage, long long head, int local, uint32_t pairs) {
-    const uint8_t* kt = S.stage[stage];
-    const uint8_t* vt = S.stage[stage] + kHalfStage;
+  // ---- K half of a quantized unit: logits, online softmax, P limbs (A6, A8, A9 set-up) ---------
+  __device__ void quantized_k(const uint8_t* kt, long long head, int local, uint32_t pairs) {
     const long long key = head * a.blocks_per_head + (local >> a.lg_units_per_blk);
     if (key != qkey) {
       build_q(pairs);
       qkey = key;
     }
-    uint8_t* pwb = reinterpret_cast<uint8_t*>(S.pw);
 #pragma unroll
     for (int g = 0; g < G; ++g) {
       int al[TPL], am[TPL], ah[TPL];
       k_dot(kt, g, al, am, ah);
-
-      // -- A8: online softmax over the unit's UT tokens
       float lg[TPL], mu = -INFINITY;
 #pragma unroll
       for (int j = 0; j < TPL; ++j) {
@@ -340,71 +345,78 @@ struct Decoder {
       m[g] = m_new;
       l[g] = fmaf(l[g], alpha, psum);
       Z[g] = fmaf(Z[g], alpha, zsum);
-
-      // -- A9: fixed-point limbs of p_t * s_g(t), then the V codes
-      if (mv > 0.f) {
-        // P <= 2^24 - 124: the top token must not round to 2^24, where it would wrap to 0
-        const float scv = kPRange * fast_rcp(mv);
-        const float invv = mv * (1.0f / kPRange);
+      alpha_[g] = alpha;
+      hasv_[g] = mv > 0.f;
+      // P <= 2^24 - 124: the top token must not round to 2^24, where it would wrap to 0
+      const float scv = mv > 0.f ? kPRange * fast_rcp(mv) : 0.f;
+      invv_[g] = mv * (1.0f / kPRange);
+      uint8_t* pwb = reinterpret_cast<uint8_t*>(S.pw[g]);
 #pragma unroll
-        for (int j = 0; j < TPL; ++j) {
-          const int t = lane + 32 * j;
-          int row, k, mb;
-          float f = pp[j] * scv;
-          if (BITS == 2) {
-            row = t >> 4;
-            k = t & 3;
-            mb = (t >> 2) & 3;
-            if (k & 1) f *= 0.25f;
-          } else {
-            row = t >> 3;
-            k = t & 1;
-            mb = (t >> 1) & 3;
-          }
-          const uint32_t Pq = __float2uint_rn(f);
-          uint8_t* base = pwb + ((row * 3) * NSET + k) * 4 + mb;
-          base[0] = static_cast<uint8_t>(Pq & 255u);
-          base[NSET * 4] = static_cast<uint8_t>((Pq >> 8) & 255u);
-          base[2 * NSET * 4] = static_cast<uint8_t>((Pq >> 16) & 255u);
+      for (int j = 0; j < TPL; ++j) {
+        const int t = lane + 32 * j;
+        int row, k, mb;
+        float f = pp[j] * scv;
+        if (BITS == 2) {
+          row = t >> 4;
+          k = t & 3;
+          mb = (t >> 2) & 3;
+          if (k & 1) f *= 0.25f;
+        } else {
+          row = t >> 3;
+          k = t & 1;
+          mb = (t >> 1) & 3;
         }
-        __syncwarp();
+        const uint32_t Pq = __float2uint_rn(f);
+        uint8_t* base = pwb + ((row * 3) * NSET + k) * 4 + mb;
+        base[0] = static_cast<uint8_t>(Pq & 255u);
+        base[NSET * 4] = static_cast<uint8_t>((Pq >> 8) & 255u);
+        base[2 * NSET * 4] = static_cast<uint8_t>((Pq >> 16) & 255u);
+      }
+    }
+  }
+
+  // ---- V half of a quantized unit: P . codes (A9) --------------------------------------------
+  __device__ void quantized_v(const uint8_t* vt) {
+    __syncwarp();  // P limbs of every query are in shared memory
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      if (hasv_[g]) {
         int vl[4] = {0, 0, 0, 0}, vm[4] = {0, 0, 0, 0}, vh[4] = {0, 0, 0, 0};
 #pragma unroll 2
         for (int r = 0; r < ROWS; ++r) {
           const uint4 vw = *reinterpret_cast<const uint4*>(vt + r * 512 + 16 * lane);
           if (BITS == 2) {
-            const uint4 PL = S.pw[r * 3 + 0], PM = S.pw[r * 3 + 1], PH = S.pw[r * 3 + 2];
+            const uint4 PL = S.pw[g][r * 3 + 0], PM = S.pw[g][r * 3 + 1], PH = S.pw[g][r * 3 + 2];
 #pragma unroll
             for (int e = 0; e < 4; ++e) dot2(comp(vw, e), PL, PM, PH, vl[e], vm[e], vh[e], false);
           } else {
-            const uint2* pw2 = reinterpret_cast<const uint2*>(S.pw);
+            const uint2* pw2 = reinterpret_cast<const uint2*>(S.pw[g]);
             const uint2 PL = pw2[r * 3 + 0], PM = pw2[r * 3 + 1], PH = pw2[r * 3 + 2];
 #pragma unroll
             for (int e = 0; e < 4; ++e) dot4(comp(vw, e), PL, PM, PH, vl[e], vm[e], vh[e], false);
           }
         }
 #pragma unroll
-        for (int e = 0; e < 4; ++e) o[g][e] = fmaf(o[g][e], alpha, combine_limbs(vh[e], vm[e], vl[e]) * invv);
-        __syncwarp();  // pw is rewritten by the next query or unit
+        for (int e = 0; e < 4; ++e)
+          o[g][e] = fmaf(o[g][e], alpha_[g], combine_limbs(vh[e], vm[e], vl[e]) * invv_[g]);
       } else {
 #pragma unroll
-        for (int e = 0; e < 4; ++e) o[g][e] *= alpha;
+        for (int e = 0; e < 4; ++e) o[g][e] *= alpha_[g];
       }
     }
+    __syncwarp();  // P limbs are rewritten by the next unit
   }
 
-  // ---- one residual unit (8 fp16 rows) -------------------------------------------------------
-  __device__ void residual_unit(int stage, int nvalid) {
-    const uint8_t* kt = S.stage[stage];
-    const uint8_t* vt = S.stage[stage] + kHalfStage;
-    const int t = lane >> 2, quarter = lane & 3;  // 4 lanes per token, 32 channels each
+  // ---- K half of a residual unit (16 fp16 rows): logits and softmax weights --------------------
+  __device__ void residual_k(const uint8_t* kt, int nvalid) {
+    const int t = lane >> 1, hf = lane & 1;  // 2 lanes per token, 64 channels each
 #pragma unroll
     for (int g = 0; g < G; ++g) {
       float dot = 0.f;
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const int cc = (k + (lane >> 1)) & 3;  // bank-conflict-free chunk order
-        const int c0 = 32 * quarter + 8 * cc;
+      for (int k = 0; k < 8; ++k) {
+        const int cc = (k + lane) & 7;  // bank-conflict-free chunk order
+        const int c0 = 64 * hf + 8 * cc;
         const uint4 kv = *reinterpret_cast<const uint4*>(kt + t * 256 + 2 * c0);
         const float4 q0 = *reinterpret_cast<const float4*>(&S.qf[g][c0]);
         const float4 q1 = *reinterpret_cast<const float4*>(&S.qf[g][c0 + 4]);
@@ -422,19 +434,27 @@ struct Decoder {
         dot = fmaf(q1.w, k3.y, dot);
       }
       dot += __shfl_xor_sync(kFull, dot, 1);
-      dot += __shfl_xor_sync(kFull, dot, 2);
       const bool valid = t < nvalid;
       const float lg = valid ? dot : -INFINITY;
       const float m_new = fmaxf(m[g], warp_max(lg));
       const float alpha = fast_exp2(m[g] - m_new);
       const float p = valid ? fast_exp2(lg - m_new) : 0.f;
       m[g] = m_new;
-      l[g] = fmaf(l[g], alpha, quarter == 0 ? p : 0.f);
+      l[g] = fmaf(l[g], alpha, hf == 0 ? p : 0.f);
       Z[g] *= alpha;
+      alpha_[g] = alpha;
+      pres_[g] = p;
+    }
+  }
+
+  // ---- V half of a residual unit: p . rows -----------------------------------------------------
+  __device__ void residual_v(const uint8_t* vt, int nvalid) {
 #pragma unroll
-      for (int e = 0; e < 4; ++e) o[g][e] *= alpha;
+    for (int g = 0; g < G; ++g) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) o[g][e] *= alpha_[g];
       for (int tt = 0; tt < nvalid; ++tt) {
-        const float pt = __shfl_sync(kFull, p, 4 * tt);
+        const float pt = __shfl_sync(kFull, pres_[g], 2 * tt);
         const uint2 vv = *reinterpret_cast<const uint2*>(vt + tt * 256 + 8 * lane);
         const float2 v0 = __half22float2(*reinterpret_cast<const __half2*>(&vv.x));
         const float2 v1 = __half22float2(*reinterpret_cast<const __half2*>(&vv.y));
@@ -523,27 +543,35 @@ struct Decoder {
   }
 
   // all lanes wait; the decision is made warp-uniform
-  __device__ bool wait_stage(int stage, uint32_t parity) {
-    const bool ok = mbar_wait_bounded(&S.bar[stage], parity, a.timeout_ns);
+  __device__ bool wait_half(int h) {
+    const bool ok = mbar_wait_bounded(&S.bar[h % kBuffers], (h / kBuffers) & 1, a.timeout_ns);
     return __all_sync(kFull, ok);
   }
 
-  // After a timeout: wait (bounded by max(timeout, 1 s)) until the bytes of a copy have landed.
-  __device__ void drain(int stage, uint32_t parity) {
+  // After a timeout: wait (bounded by max(timeout, 1 s)) until the halves in flight have landed.
+  __device__ void drain_from(int h, int nhalves) {
     const unsigned long long lim = a.timeout_ns > 1000000000ull ? a.timeout_ns : 1000000000ull;
-    (void)mbar_wait_bounded(&S.bar[stage], parity, lim);
+    for (int x = h; x < h + kBuffers && x < nhalves; ++x)
+      (void)mbar_wait_bounded(&S.bar[x % kBuffers], (x / kBuffers) & 1, lim);
     __syncwarp();
+  }
+
+  __device__ __forceinline__ void advance(long long& h, int& l) const {
+    if (++l == a.units) {
+      l = 0;
+      ++h;
+    }
   }
 
   __device__ void run() {
     if (lane == 0) {
-      mbar_init(&S.bar[0], 1);
-      mbar_init(&S.bar[1], 1);
+#pragma unroll
+      for (int b = 0; b < kBuffers; ++b) mbar_init(&S.bar[b], 1);
       asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     __syncwarp();
-    // (head, local unit) cursors for the current unit, the next one (scales) and the one after
-    // (bulk copies); advanced by increments, no division on the per-unit path
+    const int nhalves = static_cast<int>(2 * (ue - ub));
+    // (head, local unit) cursors for the current unit and the next two; advanced by increments
     long long head = ub / a.units;
     int local = static_cast<int>(ub - head * a.units);
     long long h1 = head, h2;
@@ -552,16 +580,15 @@ struct Decoder {
     h2 = h1;
     l2 = l1;
     advance(h2, l2);
-    if (lane == 0) {
-      issue(head, local, 0);
-      if (ub + 1 < ue) issue(h1, l1, 1);
+    if (lane == 0) {  // halves 0, 1, 2 = K0, V0, K1
+      issue_half(0, head, local);
+      issue_half(1, head, local);
+      if (nhalves > 2) issue_half(2, h1, l1);
     }
     uint32_t pairs = load_pairs(head, local);
     long long cur_head = -1, seg_a = ub;
-    int it = 0;
-    for (long long u = ub; u < ue; ++u, ++it) {
-      const int stage = it & 1;
-      const uint32_t parity = (it >> 1) & 1;
+    int hk = 0;
+    for (long long u = ub; u < ue; ++u, hk += 2) {
       if (head != cur_head) {
         if (cur_head >= 0) finish_segment(cur_head, seg_a, u);
         start_head(head);
@@ -569,22 +596,34 @@ struct Decoder {
         seg_a = u;
       }
       const uint32_t pairs_next = (u + 1 < ue) ? load_pairs(h1, l1) : 0u;
-      if (!wait_stage(stage, parity)) {
-        // Give up: record the error, let this warp's copies in flight land, and leave.
+      const bool quant = local < a.units_q;
+      const int nvalid = quant ? 0 : min(kResTokens, a.n_res - (local - a.units_q) * kResTokens);
+      // K half
+      if (!wait_half(hk)) {
         if (lane == 0) report_status(a.status, KIVI_ERR_DEVICE_TIMEOUT);
-        drain(stage, parity);
-        if (u + 1 < ue) drain(stage ^ 1, ((it + 1) >> 1) & 1);
+        drain_from(hk, nhalves);
         return;
       }
-      if (local < a.units_q) {
-        quantized_unit(stage, head, local, pairs);
-      } else {
-        const int t0 = (local - a.units_q) * kResTokens;
-        residual_unit(stage, min(kResTokens, a.n_res - t0));
-      }
+      if (quant)
+        quantized_k(S.buf[hk % kBuffers], head, local, pairs);
+      else
+        residual_k(S.buf[hk % kBuffers], nvalid);
       __syncwarp();
       fence_proxy_async_smem();
-      if (lane == 0 && u + 2 < ue) issue(h2, l2, stage);
+      if (lane == 0 && hk + 3 < nhalves) issue_half(hk + 3, h1, l1);  // V half of the next unit
+      // V half
+      if (!wait_half(hk + 1)) {
+        if (lane == 0) report_status(a.status, KIVI_ERR_DEVICE_TIMEOUT);
+        drain_from(hk + 1, nhalves);
+        return;
+      }
+      if (quant)
+        quantized_v(S.buf[(hk + 1) % kBuffers]);
+      else
+        residual_v(S.buf[(hk + 1) % kBuffers], nvalid);
+      __syncwarp();
+      fence_proxy_async_smem();
+      if (lane == 0 && hk + 4 < nhalves) issue_half(hk + 4, h2, l2);  // K half of the unit after
       pairs = pairs_next;
       head = h1;
       local = l1;
@@ -594,17 +633,10 @@ struct Decoder {
     }
     finish_segment(cur_head, seg_a, ue);
   }
-
-  __device__ __forceinline__ void advance(long long& h, int& l) const {
-    if (++l == a.units) {
-      l = 0;
-      ++h;
-    }
-  }
 };
 
 template <int BITS, int G>
-__global__ void __launch_bounds__(kWarps * 32, G == 1 ? 5 : 1) decode_kernel(const __grid_constant__ DecodeArgs a) {
+__global__ void __launch_bounds__(kWarps * 32, G == 1 ? 4 : 1) decode_kernel(const __grid_constant__ DecodeArgs a) {
   extern __shared__ __align__(128) uint8_t smem_raw[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   WarpSmem<G>& S = reinterpret_cast<WarpSmem<G>*>(smem_raw)[warp];
