@@ -76,6 +76,13 @@ def profiled_traffic(w: synth.Workload, alg_bytes_per_launch: float):
     return rec["dram_bytes"] / rec["alg_bytes"] * alg_bytes_per_launch
 
 
+def l2_note(w: synth.Workload, n_quant: int) -> str:
+    gb = decode_alg_bytes(w, n_quant, w.residual) / 1e9
+    if gb * 1e3 > 2 * 126:
+        return f"not flushed: inputs ({gb:.2f} GB per step) exceed the 126 MB L2"
+    return f"WARNING: inputs ({gb * 1e3:.0f} MB per step) fit in the 126 MB L2; not flushed"
+
+
 def decode_alg_bytes(w: synth.Workload, n_quant: int, n_res: int) -> int:
     """Bytes decode attention must move at least once: codes, scales/zeros, residual rows, q, out."""
     bh = w.batch * w.kv_heads
@@ -207,8 +214,13 @@ def make_state(w: synth.Workload, torch, kivi, device):
                            residual=w.residual, num_q_heads=w.q_heads, device=device)
     kd = torch.from_numpy(k).to(device)
     vd = torch.from_numpy(v).to(device)
+    cache.prefill(kd, vd)            # first run loads the module; the second one is timed
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
     cache.prefill(kd, vd)
+    e1.record()
     torch.cuda.synchronize(device)
+    prefill_ms = e0.elapsed_time(e1)
     del kd, vd, k, v
     torch.cuda.empty_cache()   # hand the 8.6 GB of prompt back: the decode loop holds ~1.3 GB
     # per-step inputs for a cycle of 128 steps (new K/V rows and queries), resident in HBM
@@ -220,19 +232,33 @@ def make_state(w: synth.Workload, torch, kivi, device):
     dev_in = [tuple(torch.from_numpy(a).to(device) for a in x) for x in steps_in]
     torch.cuda.synchronize(device)
     assert (cache.n_quant, cache.n_res) == (n_quant0, w.residual)
-    return cache, n_quant0, steps_in, dev_in
+    return cache, n_quant0, steps_in, dev_in, prefill_ms
 
 
-def gpu_step(cache, n_quant0, w, inputs, out, stream, decode_events=None):
-    """One streaming decode step on device-resident inputs; returns (launches, cached tokens)."""
+def gpu_step(cache, n_quant0, w, inputs, out, stream, decode_events=None, stage_events=None):
+    """One streaming decode step on device-resident inputs; returns (launches, cached tokens).
+    stage_events (optional): {"flush": [...], "append": [...]} lists that receive event pairs."""
+    import torch
     launches = 0
     if cache.c.n_res == w.residual:
         if cache.c.n_quant == n_quant0 + w.residual:
             cache.c.n_quant = n_quant0     # end of a 128-step cycle: drop the newest block again
+        if stage_events is not None:
+            ev = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            ev[0].record(stream)
         cache.flush(stream)
+        if stage_events is not None:
+            ev[1].record(stream)
+            stage_events["flush"].append(ev)
         launches += 1
     kn, vn, q = inputs
+    if stage_events is not None:
+        ev = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+        ev[0].record(stream)
     cache.append(kn, vn, stream)
+    if stage_events is not None:
+        ev[1].record(stream)
+        stage_events["append"].append(ev)
     launches += 1
     if decode_events is not None:
         decode_events[0].record(stream)
@@ -243,13 +269,12 @@ def gpu_step(cache, n_quant0, w, inputs, out, stream, decode_events=None):
     return launches, cache.c.n_quant + cache.c.n_res
 
 
-def run_gpu(args, rank, world, local_rank):
+def run_gpu(args, rank, world, local_rank, w: synth.Workload):
     import torch
     from bit_asymmetric_kv_02_b200 import kivi
     device = torch.device("cuda", local_rank)
     torch.cuda.set_device(device)
     kivi.load_library()
-    w = WORKLOAD
     dist = None
     if world > 1:
         import torch.distributed as dist
@@ -258,7 +283,7 @@ def run_gpu(args, rank, world, local_rank):
     ranks = Ranks(dist, device)
 
     log("generating inputs and prefilling the cache")
-    cache, n_quant0, host_in, dev_in = make_state(w, torch, kivi, device)
+    cache, n_quant0, host_in, dev_in, prefill_ms = make_state(w, torch, kivi, device)
     log("cache ready")
     stream = torch.cuda.Stream(device)
     out = torch.empty(w.batch, w.q_heads, w.head_dim, dtype=torch.float16, device=device)
@@ -278,11 +303,12 @@ def run_gpu(args, rank, world, local_rank):
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         launches, tokens = 0, 0
         bytes_decode = 0
+        stage_ev = {"flush": [], "append": []}
         with ClockSampler(local_rank) as clocks, torch.cuda.stream(stream):
             e0.record(stream)
             for i in range(K):
                 n_q, n_r = cache.c.n_quant, cache.c.n_res
-                lz, t = gpu_step(cache, n_quant0, w, dev_in[(W + i) % R], out, stream, ev[i])
+                lz, t = gpu_step(cache, n_quant0, w, dev_in[(W + i) % R], out, stream, ev[i], stage_ev)
                 launches += lz
                 tokens += t
                 n_q2 = cache.c.n_quant
@@ -293,7 +319,10 @@ def run_gpu(args, rank, world, local_rank):
         barrier()
         ms = e0.elapsed_time(e1)
         dec_ms = sum(a.elapsed_time(b) for a, b in ev)
-        return ms, dec_ms, launches, tokens, bytes_decode, clocks.summary()
+        stage_ms = {k: (sum(a.elapsed_time(b) for a, b in v) / len(v) if v else None) for k, v in stage_ev.items()}
+        clk = clocks.summary()
+        clk["stage_ms"] = stage_ms
+        return ms, dec_ms, launches, tokens, bytes_decode, clk
 
     ms, dec_ms, launches, tokens, bytes_decode, clk = timed_loop(args.steps, args.warmup)
     log(f"timed loop done: {ms:.3f} ms for {args.steps} steps")
@@ -346,21 +375,28 @@ def run_gpu(args, rank, world, local_rank):
         result = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
             "ms_per_step": t_max / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "u2 codes x i8 limbs (dp4a, i32 acc), f32 softmax", "data": "synthetic",
+            "dtype": f"u{w.bits} codes x i8 limbs (dp4a, i32 acc), f32 softmax", "data": "synthetic",
             "config": {
                 "workload": w.name, "batch": w.batch, "q_heads": w.q_heads, "kv_heads": w.kv_heads,
                 "head_dim": w.head_dim, "bits": w.bits, "group_k": w.group, "group_v": w.group,
                 "residual": w.residual, "cached_tokens": f"{n_quant0 + 1}-{n_quant0 + 2 * R} (128-step cycles)",
                 "step": "flush when full + append + decode attention",
-                "l2": "not flushed: inputs (1.2 GB per step) exceed the 126 MB L2",
+                "l2": l2_note(w, n_quant0),
                 "parallelism": f"weak: one independent batch per GPU x {world}",
             },
             "hbm_gbs_decode": achieved, "hbm_frac_of_8tbs": achieved / SPEC_HBM_GBS,
             "decode_ms_avg": dec_avg_ms,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "peak_kind": peak_kind, "traffic": traffic,
-                         "kernel": "decode_kernel<2,1>", "alg_bytes_per_launch": bytes_decode / K},
-            "clocks": clk,
+                         "kernel": f"decode_kernel<{w.bits},{w.gqa}>", "alg_bytes_per_launch": bytes_decode / K},
+            "clocks": {k: v for k, v in clk.items() if k != "stage_ms"},
+            "stages": {
+                "decode_ms": dec_avg_ms,
+                "append_ms": clk["stage_ms"]["append"], "flush_ms": clk["stage_ms"]["flush"],
+                "prefill_ms": prefill_ms, "prefill_tokens": w.tokens,
+                "prefill_gbs": (w.batch * w.kv_heads * w.tokens * w.head_dim * 2 * 2
+                                + decode_alg_bytes(w, n_quant0, 0)) / (prefill_ms / 1e3) / 1e9,
+            },
             "gpu_launches": launches,
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "steps": e2e_steps, "ms_per_step": e2e_ms / max(1, e2e_steps)},
@@ -427,16 +463,16 @@ def oracle_sample(w: synth.Workload, n_heads: int, n_steps: int, budget_s: float
     return tok / dt / w.kv_heads, cores, sample, dt, head_steps
 
 
-def run_reference(args, rank, world):
+def run_reference(args, rank, world, w: synth.Workload):
     if rank != 0:
         return None
-    w = WORKLOAD
     budget = max(5.0, min(60.0, 0.6 * args.steps + 5.0))
     value, cores, sample, dt, hs = oracle_sample(w, n_heads=min(64, 2 * (os.cpu_count() or 1)),
                                                  n_steps=max(1, args.steps), budget_s=budget)
+    ms_full_step = dt * 1e3 * (w.batch * w.kv_heads) / max(1, hs)   # one step covers every KV head
     return {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": None, "higher_is_better": True,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_full_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": w.name, "batch": w.batch, "q_heads": w.q_heads, "kv_heads": w.kv_heads,
                    "head_dim": w.head_dim, "bits": w.bits, "group_k": w.group, "group_v": w.group,
@@ -458,21 +494,30 @@ def main():
     ap.add_argument("--steps", type=int, default=2048)
     ap.add_argument("--warmup", type=int, default=128)
     ap.add_argument("--impl", choices=["kivi", "reference"], default="kivi")
+    ap.add_argument("--workload", choices=sorted(synth.WORKLOADS), default=WORKLOAD.name,
+                    help="workload to time (default: the large-batch workload the metric is quoted on)")
+    ap.add_argument("--bits", type=int, choices=[2, 4], default=None, help="override the workload's bits")
+    ap.add_argument("--group", type=int, choices=[32, 64, 128], default=None, help="override G_k = G_v")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing (profiling runs)")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end loop (profiling runs)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    w = synth.WORKLOADS[args.workload]
+    if args.bits is not None:
+        w = w.with_(bits=args.bits)
+    if args.group is not None:
+        w = w.with_(group=args.group)
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", str(args.gpus if args.gpus == 1 else 1)))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
-        res = run_reference(args, rank, world)
+        res = run_reference(args, rank, world, w)
     else:
-        res = run_gpu(args, rank, world, local_rank)
+        res = run_gpu(args, rank, world, local_rank, w)
         if rank == 0 and world == 1 and not args.no_cpu_baseline:
             log("cpu baseline (oracle)")
-            value, cores, sample, dt, hs = oracle_sample(WORKLOAD, n_heads=min(64, 2 * (os.cpu_count() or 1)),
+            value, cores, sample, dt, hs = oracle_sample(w, n_heads=min(64, 2 * (os.cpu_count() or 1)),
                                                          n_steps=16, budget_s=25.0)
             res["cpu_baseline"] = {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
                                    "sample": sample}

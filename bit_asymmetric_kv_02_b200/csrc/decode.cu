@@ -91,37 +91,25 @@ __device__ __forceinline__ long long worker_of(long long u, long long U, long lo
   return ((u + 1) * W + U - 1) / U - 1;
 }
 
-// dp4a of one packed 2-bit word against 4 sets x 3 limbs: sets 0/2 hold codes, sets 1/3 four times
-// the codes (the matching operand limbs are pre-divided by 4).
-__device__ __forceinline__ void dot2(uint32_t w, const uint4& L, const uint4& M, const uint4& H, int& al, int& am,
-                                     int& ah, bool signed_hi) {
+// Byte vectors of the 4 sets of a packed 2-bit word (sets 1 and 3 hold four times the codes).
+__device__ __forceinline__ void masks2(uint32_t w, uint32_t (&m)[4]) {
   const uint32_t w4 = w >> 4;
-  const uint32_t m0 = w & 0x03030303u, m1 = w & 0x0C0C0C0Cu;
-  const uint32_t m2 = w4 & 0x03030303u, m3 = w4 & 0x0C0C0C0Cu;
-  al = dp4a_uu(m0, L.x, al);
-  am = dp4a_uu(m0, M.x, am);
-  ah = signed_hi ? dp4a_us(m0, H.x, ah) : dp4a_uu(m0, H.x, ah);
-  al = dp4a_uu(m1, L.y, al);
-  am = dp4a_uu(m1, M.y, am);
-  ah = signed_hi ? dp4a_us(m1, H.y, ah) : dp4a_uu(m1, H.y, ah);
-  al = dp4a_uu(m2, L.z, al);
-  am = dp4a_uu(m2, M.z, am);
-  ah = signed_hi ? dp4a_us(m2, H.z, ah) : dp4a_uu(m2, H.z, ah);
-  al = dp4a_uu(m3, L.w, al);
-  am = dp4a_uu(m3, M.w, am);
-  ah = signed_hi ? dp4a_us(m3, H.w, ah) : dp4a_uu(m3, H.w, ah);
+  m[0] = w & 0x03030303u;
+  m[1] = w & 0x0C0C0C0Cu;
+  m[2] = w4 & 0x03030303u;
+  m[3] = w4 & 0x0C0C0C0Cu;
 }
-
-// The same for one packed 4-bit word against 2 sets x 3 limbs (low and high nibbles).
-__device__ __forceinline__ void dot4(uint32_t w, const uint2& L, const uint2& M, const uint2& H, int& al, int& am,
-                                     int& ah, bool signed_hi) {
-  const uint32_t n0 = w & 0x0F0F0F0Fu, n1 = (w >> 4) & 0x0F0F0F0Fu;
-  al = dp4a_uu(n0, L.x, al);
-  am = dp4a_uu(n0, M.x, am);
-  ah = signed_hi ? dp4a_us(n0, H.x, ah) : dp4a_uu(n0, H.x, ah);
-  al = dp4a_uu(n1, L.y, al);
-  am = dp4a_uu(n1, M.y, am);
-  ah = signed_hi ? dp4a_us(n1, H.y, ah) : dp4a_uu(n1, H.y, ah);
+// Byte vectors of the 2 sets (low and high nibbles) of a packed 4-bit word.
+__device__ __forceinline__ void masks4(uint32_t w, uint32_t (&m)[2]) {
+  m[0] = w & 0x0F0F0F0Fu;
+  m[1] = (w >> 4) & 0x0F0F0F0Fu;
+}
+// One set of one word against the three limbs of the matching operand bytes.
+__device__ __forceinline__ void dot_set(uint32_t m, uint32_t L, uint32_t M, uint32_t H, int& al, int& am, int& ah,
+                                        bool signed_hi) {
+  al = dp4a_uu(m, L, al);
+  am = dp4a_uu(m, M, am);
+  ah = signed_hi ? dp4a_us(m, H, ah) : dp4a_uu(m, H, ah);
 }
 
 template <int BITS, int G>
@@ -149,44 +137,47 @@ struct Decoder {
   // state handed from the K half to the V half of a unit
   float alpha_[G], invv_[G], pres_[G];
   bool hasv_[G];
+  // bytes per head of the code arrays and of a residual array; this lane's scale role
+  const size_t code_head_bytes, res_head_bytes;
+  const bool k_lane, v_lane;
 
   __device__ Decoder(const DecodeArgs& args, WarpSmem<G>& smem, int ln, long long w, long long b, long long e)
-      : a(args), S(smem), lane(ln), worker(w), ub(b), ue(e), ngk(kHeadDim >> args.lg_gk), qkey(-1) {}
+      : a(args), S(smem), lane(ln), worker(w), ub(b), ue(e), ngk(kHeadDim >> args.lg_gk), qkey(-1),
+        code_head_bytes(static_cast<size_t>(args.capacity) * (kHeadDim * BITS / 8)),
+        res_head_bytes(static_cast<size_t>(args.residual) * kHeadDim * 2),
+        k_lane(ln < (kHeadDim >> args.lg_gk)),
+        v_lane(ln >= 8 && ln < 8 + ((UT >> args.lg_gv) > 0 ? (UT >> args.lg_gv) : 1)) {}
 
   // ---- half-unit addressing: half h of the warp's range is the K (h even) or V (h odd) part -----
+  // A unit's K half and V half are each 4 KB and contiguous: quantized unit `local` of a head
+  // starts at byte local * 4 KB of that head's code arrays, residual unit r at byte r * 4 KB of
+  // its residual arrays.
   __device__ void issue_half(int h, long long head, int local) {  // lane 0 only
     const int b = h % kBuffers;
     const bool is_v = h & 1;
-    const void* src;
-    if (local < a.units_q) {
-      const size_t tok0 = static_cast<size_t>(local) * UT;
-      src = is_v ? static_cast<const void*>(a.v_codes + (static_cast<size_t>(head) * (a.capacity / P) + tok0 / P) *
-                                                            kHeadDim)
-                 : static_cast<const void*>(a.k_codes + (static_cast<size_t>(head) * a.capacity + tok0) * WPT);
-    } else {
-      const size_t t0 = static_cast<size_t>(local - a.units_q) * kResTokens;
-      const uint16_t* base = is_v ? a.v_res : a.k_res;
-      src = base + (static_cast<size_t>(head) * a.residual + t0) * kHeadDim;
-    }
+    const bool quant = local < a.units_q;
+    const char* base = quant ? reinterpret_cast<const char*>(is_v ? a.v_codes : a.k_codes)
+                             : reinterpret_cast<const char*>(is_v ? a.v_res : a.k_res);
+    const size_t stride = quant ? code_head_bytes : res_head_bytes;
+    const int unit = quant ? local : local - a.units_q;
+    const char* src = base + static_cast<size_t>(head) * stride + static_cast<size_t>(unit) * kHalfBytes;
     mbar_arrive_expect_tx(&S.bar[b], kHalfBytes + a.debug_extra_tx);
     bulk_g2s(S.buf[b], src, kHalfBytes, &S.bar[b]);
   }
 
   // (s, z) pairs of a quantized unit: lanes [0, ngk) hold K groups, lanes [8, 8 + nvg) V groups.
+  // Branch-free: every lane forms both candidate indices and at most one lane group loads.
   __device__ uint32_t load_pairs(long long head, int local) const {
-    if (local >= a.units_q) return 0u;
-    const int tok0 = local * UT;
-    if (lane < ngk) {
-      const size_t i =
-          (static_cast<size_t>(head) * a.blocks_per_head + (local >> a.lg_units_per_blk)) * ngk + lane;
-      return static_cast<uint32_t>(__ldg(a.k_scale + i)) | (static_cast<uint32_t>(__ldg(a.k_zero + i)) << 16);
-    }
-    const int nvg = (UT >> a.lg_gv) > 0 ? (UT >> a.lg_gv) : 1;
-    if (lane >= 8 && lane < 8 + nvg) {
-      const size_t i = static_cast<size_t>(head) * a.vgroups_per_head + (tok0 >> a.lg_gv) + (lane - 8);
-      return static_cast<uint32_t>(__ldg(a.v_scale + i)) | (static_cast<uint32_t>(__ldg(a.v_zero + i)) << 16);
-    }
-    return 0u;
+    const size_t ik = (static_cast<size_t>(head) * a.blocks_per_head + (local >> a.lg_units_per_blk)) * ngk +
+                      (k_lane ? lane : 0);
+    const size_t iv = static_cast<size_t>(head) * a.vgroups_per_head + ((local * UT) >> a.lg_gv) +
+                      (v_lane ? lane - 8 : 0);
+    const uint16_t* ps = k_lane ? a.k_scale + ik : a.v_scale + iv;
+    const uint16_t* pz = k_lane ? a.k_zero + ik : a.v_zero + iv;
+    uint32_t r = 0u;
+    if ((k_lane || v_lane) && local < a.units_q)
+      r = static_cast<uint32_t>(__ldg(ps)) | (static_cast<uint32_t>(__ldg(pz)) << 16);
+    return r;
   }
 
   // ---- per-head state ---------------------------------------------------------------------
@@ -272,10 +263,13 @@ struct Decoder {
     __syncwarp();
   }
 
-  // ---- A6 over the K codes of a unit: integer dot products of TPL tokens per lane --------------
-  __device__ void k_dot(const uint8_t* kt, int g, int (&al)[TPL], int (&am)[TPL], int (&ah)[TPL]) const {
+  // ---- A6 over the K codes of a unit: integer dot products of TPL tokens per lane, for every
+  // query of the KV head (each code word is unpacked once) -----------------------------------------
+  __device__ void k_dot(const uint8_t* kt, int (&al)[G][TPL], int (&am)[G][TPL], int (&ah)[G][TPL]) const {
 #pragma unroll
-    for (int j = 0; j < TPL; ++j) al[j] = am[j] = ah[j] = 0;
+    for (int g = 0; g < G; ++g)
+#pragma unroll
+      for (int j = 0; j < TPL; ++j) al[g][j] = am[g][j] = ah[g][j] = 0;
     if (BITS == 2) {
 #pragma unroll 1
       for (int h = 0; h < 2; ++h) {
@@ -283,28 +277,44 @@ struct Decoder {
         uint4 kw[TPL];
 #pragma unroll
         for (int j = 0; j < TPL; ++j) kw[j] = *reinterpret_cast<const uint4*>(kt + (lane + 32 * j) * 32 + 16 * hh);
-        const uint4* qrow = S.qw[g] + 12 * hh;
 #pragma unroll
         for (int ii = 0; ii < 4; ++ii) {
-          const uint4 QL = qrow[ii * 3 + 0], QM = qrow[ii * 3 + 1], QH = qrow[ii * 3 + 2];
+          uint32_t mk[TPL][4];
 #pragma unroll
-          for (int j = 0; j < TPL; ++j) dot2(comp(kw[j], ii), QL, QM, QH, al[j], am[j], ah[j], true);
+          for (int j = 0; j < TPL; ++j) masks2(comp(kw[j], ii), mk[j]);
+#pragma unroll
+          for (int g = 0; g < G; ++g) {
+            const uint4* qrow = S.qw[g] + 12 * hh + ii * 3;
+            const uint4 QL = qrow[0], QM = qrow[1], QH = qrow[2];
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+#pragma unroll
+              for (int j = 0; j < TPL; ++j)
+                dot_set(mk[j][k], comp(QL, k), comp(QM, k), comp(QH, k), al[g][j], am[g][j], ah[g][j], true);
+          }
         }
       }
     } else {
-      const uint2* qw2 = reinterpret_cast<const uint2*>(S.qw[g]);
 #pragma unroll 1
       for (int qq = 0; qq < 4; ++qq) {
         const int cq = (qq + (lane >> 1)) & 3;  // bank-conflict-free chunk order
         uint4 kw[TPL];
 #pragma unroll
         for (int j = 0; j < TPL; ++j) kw[j] = *reinterpret_cast<const uint4*>(kt + (lane + 32 * j) * 64 + 16 * cq);
-        const uint2* qrow = qw2 + 12 * cq;
 #pragma unroll
         for (int ii = 0; ii < 4; ++ii) {
-          const uint2 QL = qrow[ii * 3 + 0], QM = qrow[ii * 3 + 1], QH = qrow[ii * 3 + 2];
+          uint32_t mk[TPL][2];
 #pragma unroll
-          for (int j = 0; j < TPL; ++j) dot4(comp(kw[j], ii), QL, QM, QH, al[j], am[j], ah[j], true);
+          for (int j = 0; j < TPL; ++j) masks4(comp(kw[j], ii), mk[j]);
+#pragma unroll
+          for (int g = 0; g < G; ++g) {
+            const uint2* qrow = reinterpret_cast<const uint2*>(S.qw[g]) + 12 * cq + ii * 3;
+            const uint2 QL = qrow[0], QM = qrow[1], QH = qrow[2];
+#pragma unroll
+            for (int j = 0; j < TPL; ++j) dot_set(mk[j][0], QL.x, QM.x, QH.x, al[g][j], am[g][j], ah[g][j], true);
+#pragma unroll
+            for (int j = 0; j < TPL; ++j) dot_set(mk[j][1], QL.y, QM.y, QH.y, al[g][j], am[g][j], ah[g][j], true);
+          }
         }
       }
     }
@@ -317,14 +327,14 @@ struct Decoder {
       build_q(pairs);
       qkey = key;
     }
+    int al[G][TPL], am[G][TPL], ah[G][TPL];
+    k_dot(kt, al, am, ah);
 #pragma unroll
     for (int g = 0; g < G; ++g) {
-      int al[TPL], am[TPL], ah[TPL];
-      k_dot(kt, g, al, am, ah);
       float lg[TPL], mu = -INFINITY;
 #pragma unroll
       for (int j = 0; j < TPL; ++j) {
-        lg[j] = fmaf(combine_limbs(ah[j], am[j], al[j]), invq[g], cblk[g]);
+        lg[j] = fmaf(combine_limbs(ah[g][j], am[g][j], al[g][j]), invq[g], cblk[g]);
         mu = fmaxf(mu, lg[j]);
       }
       mu = warp_max(mu);
@@ -375,30 +385,59 @@ struct Decoder {
     }
   }
 
-  // ---- V half of a quantized unit: P . codes (A9) --------------------------------------------
+  // ---- V half of a quantized unit: P . codes for every query (A9) ------------------------------
   __device__ void quantized_v(const uint8_t* vt) {
     __syncwarp();  // P limbs of every query are in shared memory
+    if (G == 1 && !hasv_[0]) {  // every weight of the unit is zero: only rescale
+#pragma unroll
+      for (int e = 0; e < 4; ++e) o[0][e] *= alpha_[0];
+      __syncwarp();
+      return;
+    }
+    int vl[G][4], vm[G][4], vh[G][4];
+#pragma unroll
+    for (int g = 0; g < G; ++g)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) vl[g][e] = vm[g][e] = vh[g][e] = 0;
+#pragma unroll 2
+    for (int r = 0; r < ROWS; ++r) {
+      const uint4 vw = *reinterpret_cast<const uint4*>(vt + r * 512 + 16 * lane);
+      if (BITS == 2) {
+        uint32_t mv4[4][4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) masks2(comp(vw, e), mv4[e]);
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+          if (G > 1 && !hasv_[g]) continue;
+          const uint4 PL = S.pw[g][r * 3 + 0], PM = S.pw[g][r * 3 + 1], PH = S.pw[g][r * 3 + 2];
+#pragma unroll
+          for (int k = 0; k < 4; ++k)  // set-major: 12 independent accumulators between reuses
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              dot_set(mv4[e][k], comp(PL, k), comp(PM, k), comp(PH, k), vl[g][e], vm[g][e], vh[g][e], false);
+        }
+      } else {
+        uint32_t mv4[4][2];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) masks4(comp(vw, e), mv4[e]);
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+          if (G > 1 && !hasv_[g]) continue;
+          const uint2* pw2 = reinterpret_cast<const uint2*>(S.pw[g]);
+          const uint2 PL = pw2[r * 3 + 0], PM = pw2[r * 3 + 1], PH = pw2[r * 3 + 2];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) dot_set(mv4[e][0], PL.x, PM.x, PH.x, vl[g][e], vm[g][e], vh[g][e], false);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) dot_set(mv4[e][1], PL.y, PM.y, PH.y, vl[g][e], vm[g][e], vh[g][e], false);
+        }
+      }
+    }
 #pragma unroll
     for (int g = 0; g < G; ++g) {
       if (hasv_[g]) {
-        int vl[4] = {0, 0, 0, 0}, vm[4] = {0, 0, 0, 0}, vh[4] = {0, 0, 0, 0};
-#pragma unroll 2
-        for (int r = 0; r < ROWS; ++r) {
-          const uint4 vw = *reinterpret_cast<const uint4*>(vt + r * 512 + 16 * lane);
-          if (BITS == 2) {
-            const uint4 PL = S.pw[g][r * 3 + 0], PM = S.pw[g][r * 3 + 1], PH = S.pw[g][r * 3 + 2];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) dot2(comp(vw, e), PL, PM, PH, vl[e], vm[e], vh[e], false);
-          } else {
-            const uint2* pw2 = reinterpret_cast<const uint2*>(S.pw[g]);
-            const uint2 PL = pw2[r * 3 + 0], PM = pw2[r * 3 + 1], PH = pw2[r * 3 + 2];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) dot4(comp(vw, e), PL, PM, PH, vl[e], vm[e], vh[e], false);
-          }
-        }
 #pragma unroll
         for (int e = 0; e < 4; ++e)
-          o[g][e] = fmaf(o[g][e], alpha_[g], combine_limbs(vh[e], vm[e], vl[e]) * invv_[g]);
+          o[g][e] = fmaf(o[g][e], alpha_[g], combine_limbs(vh[g][e], vm[g][e], vl[g][e]) * invv_[g]);
       } else {
 #pragma unroll
         for (int e = 0; e < 4; ++e) o[g][e] *= alpha_[g];
@@ -506,29 +545,60 @@ struct Decoder {
     last = __shfl_sync(kFull, last, 0);
     if (!last) return;
     __threadfence();
+    // Workers wfirst..wlast each left one partial of this head.  Only wfirst can have started
+    // before the head (its partial is then in its slot 1); every later one starts inside it.
+    const int nparts = static_cast<int>(wlast - wfirst + 1);
+    const int first_slot = (U * wfirst / W) >= h0 ? 0 : 1;
 #pragma unroll 1
     for (int g = 0; g < G; ++g) {
+      auto part = [&](int k) -> const float* {
+        const long long x = wfirst + k;
+        return a.partials + ((x * 2 + (k == 0 ? first_slot : 0)) * G + g) * kPartialStride;
+      };
+      // (m, l, Z) of up to 32 partials per pass, one per lane
       float mm = -INFINITY;
-      for (long long x = wfirst; x <= wlast; ++x) {
-        const int sx = (U * x / W) >= h0 ? 0 : 1;
-        mm = fmaxf(mm, __ldcg(a.partials + ((x * 2 + sx) * G + g) * kPartialStride));
+      for (int base = 0; base < nparts; base += 32) {
+        const int k = base + lane;
+        if (k < nparts) mm = fmaxf(mm, __ldcg(part(k)));
       }
+      mm = warp_max(mm);
       float ls = 0.f, zs = 0.f, acc[4] = {0.f, 0.f, 0.f, 0.f};
-      for (long long x = wfirst; x <= wlast; ++x) {
-        const int sx = (U * x / W) >= h0 ? 0 : 1;
-        const float* p = a.partials + ((x * 2 + sx) * G + g) * kPartialStride;
-        const float w = fast_exp2(__ldcg(p) - mm);
-        const float lx = __ldcg(p + 1);
-        if (!(lx > 0.f) && lane == 0) report_status(a.status, KIVI_ERR_INTERNAL);  // never written
-        ls = fmaf(w, lx, ls);
-        zs = fmaf(w, __ldcg(p + 2), zs);
-        const float4 ov = __ldcg(reinterpret_cast<const float4*>(p + 4 + 4 * lane));
-        acc[0] = fmaf(w, ov.x, acc[0]);
-        acc[1] = fmaf(w, ov.y, acc[1]);
-        acc[2] = fmaf(w, ov.z, acc[2]);
-        acc[3] = fmaf(w, ov.w, acc[3]);
+      for (int base = 0; base < nparts; base += 32) {
+        const int k = base + lane;
+        float wk = 0.f;
+        if (k < nparts) {
+          const float* p = part(k);
+          const float lx = __ldcg(p + 1);
+          if (!(lx > 0.f)) report_status(a.status, KIVI_ERR_INTERNAL);  // never written
+          wk = fast_exp2(__ldcg(p) - mm);
+          ls = fmaf(wk, lx, ls);
+          zs = fmaf(wk, __ldcg(p + 2), zs);
+        }
+        const int n = min(32, nparts - base);
+        int i = 0;
+        for (; i + 4 <= n; i += 4) {  // four partial rows in flight
+          float4 ov[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) ov[u] = __ldcg(reinterpret_cast<const float4*>(part(base + i + u) + 4) + lane);
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const float w = __shfl_sync(kFull, wk, i + u);
+            acc[0] = fmaf(w, ov[u].x, acc[0]);
+            acc[1] = fmaf(w, ov[u].y, acc[1]);
+            acc[2] = fmaf(w, ov[u].z, acc[2]);
+            acc[3] = fmaf(w, ov[u].w, acc[3]);
+          }
+        }
+        for (; i < n; ++i) {
+          const float4 ov = __ldcg(reinterpret_cast<const float4*>(part(base + i) + 4) + lane);
+          const float w = __shfl_sync(kFull, wk, i);
+          acc[0] = fmaf(w, ov.x, acc[0]);
+          acc[1] = fmaf(w, ov.y, acc[1]);
+          acc[2] = fmaf(w, ov.z, acc[2]);
+          acc[3] = fmaf(w, ov.w, acc[3]);
+        }
       }
-      store_out(head, g, acc, zs, 1.f / ls);
+      store_out(head, g, acc, warp_sum(zs), 1.f / warp_sum(ls));
     }
     if (lane == 0) a.tickets[head] = 0;
   }

@@ -54,20 +54,29 @@ __device__ __forceinline__ GroupParams make_group(float lo, float hi, int levels
   return g;
 }
 
-// Q of one element (section 量子化アルゴリズム, Q equation) with the stored fp16 s and z.
-__device__ __forceinline__ uint32_t quantize_one(float x, const GroupParams& g, int levels) {
-  if (g.inv_s == 0.f) return 0u;
-  const float r = (x - g.zf) * g.inv_s;
-  const float fl = floorf(r);
-  float q;
-  if (fabsf(r - fl - 0.5f) < 0.000244140625f) {  // within 2^-12 of a tie: decide exactly
-    const double r64 = (static_cast<double>(x) - static_cast<double>(g.zf)) / static_cast<double>(h2f(g.s_bits));
-    q = static_cast<float>(rint(r64));
-  } else {
-    q = rintf(r);
-  }
-  q = fminf(fmaxf(q, 0.f), static_cast<float>(levels));
-  return static_cast<uint32_t>(q);
+// Q of one element (section 量子化アルゴリズム, Q equation) with the stored fp16 s and z, taken
+// exactly: the fp64 quotient decides (used near ties only).
+__device__ __forceinline__ uint32_t quantize_exact(float x, const GroupParams& g, int levels) {
+  const double r64 = (static_cast<double>(x) - static_cast<double>(g.zf)) / static_cast<double>(h2f(g.s_bits));
+  return min(static_cast<uint32_t>(rint(r64)), static_cast<uint32_t>(levels));
+}
+
+// Q of two elements at once with packed fp32 pairs.  r = (x - z) * (1/s) has absolute error below
+// 2^-18 for every reachable r (< 24); adding 1.5 * 2^23 rounds it to the nearest integer, ties to
+// even, exactly like rint.  An element whose r lies within 2^-12 of a half-integer is decided
+// again by quantize_exact.
+__device__ __forceinline__ void quantize_pair(uint32_t hx2, const GroupParams& g, int levels, uint32_t& qa,
+                                              uint32_t& qb) {
+  constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
+  const float2 x = __half22float2(*reinterpret_cast<const __half2*>(&hx2));
+  const float2 r = __fmul2_rn(__fadd2_rn(x, make_float2(-g.zf, -g.zf)), make_float2(g.inv_s, g.inv_s));
+  const float2 t = __fadd2_rn(r, make_float2(kMagic, kMagic));
+  const float2 d = __fadd2_rn(r, __fadd2_rn(make_float2(kMagic, kMagic), make_float2(-t.x, -t.y)));
+  qa = min(__float_as_uint(t.x) - 0x4B400000u, static_cast<uint32_t>(levels));
+  qb = min(__float_as_uint(t.y) - 0x4B400000u, static_cast<uint32_t>(levels));
+  if (fabsf(d.x) > 0.499755859375f) qa = quantize_exact(x.x, g, levels);  // within 2^-12 of a tie
+  if (fabsf(d.y) > 0.499755859375f) qb = quantize_exact(x.y, g, levels);
+  if (g.inv_s == 0.f) qa = qb = 0u;
 }
 
 // ---------------------------------------------------------------------------------------------
@@ -118,23 +127,25 @@ __device__ void quantize_k_block(const uint16_t* __restrict__ src, int R, int gk
   }
   __syncthreads();
 
-  // pass 2: word (t, i) holds channels P*i + j at bits BITS*j
+  // pass 2: word (t, i) holds channels P*i + j at bits BITS*j; a word never straddles a group
+  // (P <= 16 <= group_k)
   constexpr int WPT = kHeadDim / P;  // words per token
+#pragma unroll 4
   for (int w = tid; w < R * WPT; w += kThreads) {
     const int t = w / WPT, i = w % WPT;
     const uint4* p = s4 + t * kChunks + (i * P) / 8;
+    const GroupParams g = grp[(i * P) / gk];
     uint32_t word = 0;
 #pragma unroll
     for (int c8 = 0; c8 < P / 8; ++c8) {
       const uint4 v = __ldg(p + c8);
       const uint32_t hw[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const int j = c8 * 8 + e;
-        const int ch = i * P + j;
-        const GroupParams& g = grp[ch / gk];
-        const uint16_t xb = static_cast<uint16_t>((e & 1) ? (hw[e >> 1] >> 16) : (hw[e >> 1] & 0xFFFFu));
-        word |= quantize_one(h2f(xb), g, L) << (BITS * j);
+      for (int e = 0; e < 4; ++e) {  // channels j, j + 1 of the word
+        const int j = c8 * 8 + 2 * e;
+        uint32_t qa, qb;
+        quantize_pair(hw[e], g, L, qa, qb);
+        word += (qa << (BITS * j)) + (qb << (BITS * (j + 1)));  // disjoint bit fields
       }
     }
     codes[w] = word;
@@ -192,15 +203,18 @@ __device__ void quantize_v_block(const uint16_t* __restrict__ src, int R, int gv
   // pass 2: word (r, c) holds tokens P*r + j of channel c at bits BITS*j; a thread does two
   // adjacent channels with 32-bit loads.
   const uint32_t* s2 = reinterpret_cast<const uint32_t*>(src);
+#pragma unroll 2
   for (int w2 = tid; w2 < (R / P) * (kHeadDim / 2); w2 += kThreads) {
     const int r = w2 / (kHeadDim / 2), cp = w2 % (kHeadDim / 2);
-    const GroupParams& g = grp[(r * P) / gv];
+    const GroupParams g = grp[(r * P) / gv];
     uint32_t wa = 0, wb = 0;
 #pragma unroll
-    for (int j = 0; j < P; ++j) {
+    for (int j = 0; j < P; ++j) {  // channels 2 cp, 2 cp + 1 of token P r + j
       const uint32_t pair = __ldg(s2 + (r * P + j) * (kHeadDim / 2) + cp);
-      wa |= quantize_one(h2f(static_cast<uint16_t>(pair & 0xFFFFu)), g, L) << (BITS * j);
-      wb |= quantize_one(h2f(static_cast<uint16_t>(pair >> 16)), g, L) << (BITS * j);
+      uint32_t qa, qb;
+      quantize_pair(pair, g, L, qa, qb);
+      wa += qa << (BITS * j);
+      wb += qb << (BITS * j);
     }
     codes[r * kHeadDim + 2 * cp] = wa;
     codes[r * kHeadDim + 2 * cp + 1] = wb;
