@@ -42,25 +42,33 @@ namespace {
 
 constexpr int kWarps = 4;           // stream-K workers per CTA
 constexpr int kHalfBytes = 4096;    // one half unit: the K part or the V part of a unit
-constexpr int kBuffers = 3;         // half-unit buffers per warp (ring K0 V0 K1 | V1 K2 V2 | ...)
+#ifndef KIVI_DECODE_BUFFERS
+#define KIVI_DECODE_BUFFERS 3
+#endif
+#ifndef KIVI_DECODE_MIN_CTAS
+#define KIVI_DECODE_MIN_CTAS 4
+#endif
+// Half-unit buffers per warp: 3 gives the ring K0 V0 K1 | V1 K2 V2 | ..., 2 gives K | V.
+constexpr int kBuffers = KIVI_DECODE_BUFFERS;
+static_assert(kBuffers == 2 || kBuffers == 3, "the ring holds 2 or 3 half units");
 constexpr int kResTokens = 16;      // tokens per residual unit
 constexpr unsigned kFull = 0xffffffffu;
 constexpr float kQRange = 8388544.f;   // 2^23 - 64: largest |Q| before rounding (signed 24-bit limbs)
 constexpr float kPRange = 16777088.f;  // 2^24 - 128: largest P before rounding (unsigned 24-bit limbs)
 
 template <int G>
-struct __align__(128) WarpSmem {
+struct __align__(16) WarpSmem {
   uint8_t buf[kBuffers][kHalfBytes];
   uint4 qw[G][24];  // Q limbs of each query: 96 words
   uint4 pw[G][24];  // P limbs of each query: up to 96 words
-  float qf[G][kHeadDim];
   uint64_t bar[kBuffers];
 };
 
+// Maximum over the warp in one instruction (sm_100a redux.sync on f32; NaN inputs are ignored).
 __device__ __forceinline__ float warp_max(float v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(kFull, v, o));
-  return v;
+  float r;
+  asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(v));
+  return r;
 }
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
@@ -82,8 +90,10 @@ __device__ __forceinline__ float fast_exp2(float x) {
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
+// hi * 2^16 + mid * 2^8 + lo.  mid * 2^8 + lo stays below 2^27 for every sum formed here (at most
+// 128 products of a byte with a code of at most 15), so it is formed exactly in int32.
 __device__ __forceinline__ float combine_limbs(int hi, int mid, int lo) {
-  return fmaf(static_cast<float>(hi), 65536.f, fmaf(static_cast<float>(mid), 256.f, static_cast<float>(lo)));
+  return fmaf(static_cast<float>(hi), 65536.f, static_cast<float>((mid << 8) + lo));
 }
 
 // Largest worker whose range starts at or before unit u: start(x) = floor(U x / W).
@@ -117,9 +127,7 @@ struct Decoder {
   static constexpr int P = 32 / BITS;              // codes per word
   static constexpr int UT = BITS == 2 ? 128 : 64;  // tokens per quantized unit (8 KB of codes)
   static constexpr int TPL = UT / 32;              // tokens per lane (K side)
-  static constexpr int WPT = kHeadDim / P;         // K words per token
   static constexpr int ROWS = UT / P;              // V word rows per unit (8)
-  static constexpr int NSET = BITS == 2 ? 4 : 2;   // byte sets per word
 
   const DecodeArgs& a;
   WarpSmem<G>& S;
@@ -127,7 +135,9 @@ struct Decoder {
   const long long worker, ub, ue;
   const int ngk;  // K groups per head (d / G_k)
 
-  // per-head state
+  // per-head state.  At 2 bits lane (i, k) = (lane / 4, lane % 4) holds channels 16 i + 4 m + k
+  // (m = 0..3: byte m of set k of K word i) and lane j < d / G_k holds the q sum of K group j in
+  // qsum[g][0]; at 4 bits lane holds channels lane + 32 j and every lane holds all group sums.
   float qreg[G][4];
   float qsum[G][4];
   float m[G], l[G], Z[G], o[G][4];
@@ -186,11 +196,24 @@ struct Decoder {
 #pragma unroll
     for (int g = 0; g < G; ++g) {
       const uint16_t* qp = a.q + (static_cast<size_t>(head) * G + g) * kHeadDim;
+      if constexpr (BITS == 2) {
+        float part = 0.f;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int c = 16 * (lane >> 2) + 4 * j + (lane & 3);
+          const float v = h2f(__ldg(qp + c)) * a.qscale;
+          qreg[g][j] = v;
+          part += v;
+        }
+        // the 2^(lg_gk - 2) consecutive lanes of a K group reduce its sum; lane j takes group j's
+        const int span = 1 << (a.lg_gk - 2);
+        for (int off = 1; off < span; off <<= 1) part += __shfl_xor_sync(kFull, part, off);
+        qsum[g][0] = __shfl_sync(kFull, part, (lane & (ngk - 1)) * span);
+      } else {
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const float v = h2f(__ldg(qp + lane + 32 * j)) * a.qscale;
         qreg[g][j] = v;
-        S.qf[g][lane + 32 * j] = v;
       }
 #pragma unroll
       for (int gi = 0; gi < 4; ++gi) {
@@ -199,6 +222,7 @@ struct Decoder {
         for (int j = 0; j < 4; ++j)
           if (((32 * j) >> a.lg_gk) == gi) part += qreg[g][j];
         qsum[g][gi] = gi < ngk ? warp_sum(part) : 0.f;
+      }
       }
       m[g] = -INFINITY;
       l[g] = 0.f;
@@ -210,9 +234,61 @@ struct Decoder {
     __syncwarp();
   }
 
+  // Bytes 0, 1 and 2 of four integers as three words: word b holds byte b of x_m in byte m.
+  static __device__ __forceinline__ void limb_words(int x0, int x1, int x2, int x3, uint32_t& L, uint32_t& M,
+                                                   uint32_t& H) {
+    const uint32_t t01 = __byte_perm(x0, x1, 0x5140), t23 = __byte_perm(x2, x3, 0x5140);
+    L = __byte_perm(t01, t23, 0x5410);
+    M = __byte_perm(t01, t23, 0x7632);
+    H = __byte_perm(__byte_perm(x0, x1, 0x0062), __byte_perm(x2, x3, 0x0062), 0x5410);
+  }
+
+  // 2 bits: lane (i, k) owns byte m of set k of K word i for m = 0..3 (channels 16 i + 4 m + k), so
+  // it forms that set's three limb words itself.  Odd sets read as 4 * code: their limbs are / 4.
+  __device__ void build_q2(uint32_t pairs) {
+    const int gi = (16 * (lane >> 2)) >> a.lg_gk;  // the K group of all four channels
+    const float s = h2f(static_cast<uint16_t>(__shfl_sync(kFull, pairs, gi) & 0xFFFFu));
+    const float z_own = k_lane ? h2f(static_cast<uint16_t>(pairs >> 16)) : 0.f;
+    const float set_scale = (lane & 1) ? 0.25f : 1.f;
+    uint32_t* qw = reinterpret_cast<uint32_t*>(S.qw);
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      float qv[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) qv[j] = qreg[g][j] * s;
+      const float mabs = warp_max(fmaxf(fmaxf(fabsf(qv[0]), fabsf(qv[1])), fmaxf(fabsf(qv[2]), fabsf(qv[3]))));
+      // |Q| <= 2^23 - 61: the margin keeps the rounded largest element below 2^23, where the
+      // signed top limb would wrap (rcp and the product add at most 3 * 2^-22 relative)
+      const float scq = mabs > 0.f ? kQRange * fast_rcp(mabs) : 0.f;
+      invq[g] = mabs * (1.0f / kQRange);
+      // sum over K groups of z_g * (sum of q over group g): lanes 0..3 hold one group each
+      float c = z_own * qsum[g][0];
+      c += __shfl_xor_sync(kFull, c, 1);
+      c += __shfl_xor_sync(kFull, c, 2);
+      cblk[g] = __shfl_sync(kFull, c, 0);
+      const float f = scq * set_scale;
+      uint32_t L, M, H;
+      limb_words(__float2int_rn(qv[0] * f), __float2int_rn(qv[1] * f), __float2int_rn(qv[2] * f),
+                 __float2int_rn(qv[3] * f), L, M, H);
+      uint32_t* row = qw + g * 96 + (lane >> 2) * 12 + (lane & 3);  // word i, limb b, set k
+      row[0] = L;
+      row[4] = M;
+      row[8] = H;
+    }
+  }
+
   // ---- A6 set-up for one K block: fixed-point limbs of q_c * s_g(c) -------------------------
   __device__ void build_q(uint32_t pairs) {
     __syncwarp();  // the previous block's limbs are no longer read
+    if constexpr (BITS == 2)
+      build_q2(pairs);
+    else
+      build_q4(pairs);
+    __syncwarp();
+  }
+
+  // 4 bits: lane holds channels lane + 32 j; each byte of a limb word is stored on its own.
+  __device__ void build_q4(uint32_t pairs) {
 #pragma unroll
     for (int g = 0; g < G; ++g) {
       float qv[4], mabs = 0.f;
@@ -241,26 +317,14 @@ struct Decoder {
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const int ch = lane + 32 * j;
-        float f = qv[j] * scq;
-        int word, k, mb;
-        if (BITS == 2) {  // word i = c/16, set k = c%4 (odd sets read as 4*code), byte m = (c%16)/4
-          word = ch >> 4;
-          k = ch & 3;
-          mb = (ch >> 2) & 3;
-          if (k & 1) f *= 0.25f;
-        } else {          // word i = c/8, set k = c%2, byte m = (c%8)/2
-          word = ch >> 3;
-          k = ch & 1;
-          mb = (ch >> 1) & 3;
-        }
-        const int Q = __float2int_rn(f);
-        uint8_t* base = qwb + ((word * 3) * NSET + k) * 4 + mb;
+        const int word = ch >> 3, k = ch & 1, mb = (ch >> 1) & 3;  // word c/8, set c%2, byte (c%8)/2
+        const int Q = __float2int_rn(qv[j] * scq);
+        uint8_t* base = qwb + ((word * 3) * 2 + k) * 4 + mb;  // limb b of word i: 8 bytes at (3 i + b) * 8
         base[0] = static_cast<uint8_t>(Q & 255);
-        base[NSET * 4] = static_cast<uint8_t>((Q >> 8) & 255);
-        base[2 * NSET * 4] = static_cast<uint8_t>((Q >> 16) & 255);
+        base[8] = static_cast<uint8_t>((Q >> 8) & 255);
+        base[16] = static_cast<uint8_t>((Q >> 16) & 255);
       }
     }
-    __syncwarp();
   }
 
   // ---- A6 over the K codes of a unit: integer dot products of TPL tokens per lane, for every
@@ -276,7 +340,8 @@ struct Decoder {
         const int hh = h ^ ((lane >> 2) & 1);  // bank-conflict-free order of the two 16-byte halves
         uint4 kw[TPL];
 #pragma unroll
-        for (int j = 0; j < TPL; ++j) kw[j] = *reinterpret_cast<const uint4*>(kt + (lane + 32 * j) * 32 + 16 * hh);
+        for (int j = 0; j < TPL; ++j)  // token 16 (lane / 4) + 4 j + lane % 4
+          kw[j] = *reinterpret_cast<const uint4*>(kt + (16 * (lane >> 2) + 4 * j + (lane & 3)) * 32 + 16 * hh);
 #pragma unroll
         for (int ii = 0; ii < 4; ++ii) {
           uint32_t mk[TPL][4];
@@ -320,6 +385,48 @@ struct Decoder {
     }
   }
 
+  // 2 bits: lane (r, k) holds tokens 16 r + 4 j + k (j = 0..3), i.e. byte j of set k of V word row
+  // r, so it forms that set's three P limb words itself; its four tokens share one V group.
+  __device__ void softmax2(uint32_t pairs, const int (&al)[G][TPL], const int (&am)[G][TPL],
+                           const int (&ah)[G][TPL]) {
+    const uint32_t vp = __shfl_sync(kFull, pairs, 8 + ((16 * (lane >> 2)) >> a.lg_gv));
+    const float sv = h2f(static_cast<uint16_t>(vp & 0xFFFFu)), zv = h2f(static_cast<uint16_t>(vp >> 16));
+    const float set_scale = (lane & 1) ? 0.25f : 1.f;
+    uint32_t* pw = reinterpret_cast<uint32_t*>(S.pw);
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      float lg[TPL];
+#pragma unroll
+      for (int j = 0; j < TPL; ++j) lg[j] = fmaf(combine_limbs(ah[g][j], am[g][j], al[g][j]), invq[g], cblk[g]);
+      const float mu = warp_max(fmaxf(fmaxf(lg[0], lg[1]), fmaxf(lg[2], lg[3])));
+      const float m_new = fmaxf(m[g], mu);
+      const float alpha = fast_exp2(m[g] - m_new);
+      float p[TPL];
+#pragma unroll
+      for (int j = 0; j < TPL; ++j) p[j] = fast_exp2(lg[j] - m_new);
+      const float psum = (p[0] + p[1]) + (p[2] + p[3]);
+      // P is scaled by the unit's largest p * s; the four tokens of a lane share s
+      const float mv = warp_max(fmaxf(fmaxf(p[0], p[1]), fmaxf(p[2], p[3])) * sv);
+      m[g] = m_new;
+      l[g] = fmaf(l[g], alpha, psum);
+      Z[g] = fmaf(Z[g], alpha, psum * zv);
+      alpha_[g] = alpha;
+      hasv_[g] = mv > 0.f;
+      // P <= 2^24 - 124: the top token must not round to 2^24, where it would wrap to 0
+      const float scv = mv > 0.f ? kPRange * fast_rcp(mv) : 0.f;
+      invv_[g] = mv * (1.0f / kPRange);
+      const float f = scv * set_scale;
+      uint32_t L, M, H;
+      limb_words(static_cast<int>(__float2uint_rn(p[0] * sv * f)), static_cast<int>(__float2uint_rn(p[1] * sv * f)),
+                 static_cast<int>(__float2uint_rn(p[2] * sv * f)), static_cast<int>(__float2uint_rn(p[3] * sv * f)),
+                 L, M, H);
+      uint32_t* row = pw + g * 96 + (lane >> 2) * 12 + (lane & 3);  // row r, limb b, set k
+      row[0] = L;
+      row[4] = M;
+      row[8] = H;
+    }
+  }
+
   // ---- K half of a quantized unit: logits, online softmax, P limbs (A6, A8, A9 set-up) ---------
   __device__ void quantized_k(const uint8_t* kt, long long head, int local, uint32_t pairs) {
     const long long key = head * a.blocks_per_head + (local >> a.lg_units_per_blk);
@@ -329,6 +436,15 @@ struct Decoder {
     }
     int al[G][TPL], am[G][TPL], ah[G][TPL];
     k_dot(kt, al, am, ah);
+    if constexpr (BITS == 2)
+      softmax2(pairs, al, am, ah);
+    else
+      softmax4(pairs, al, am, ah);
+  }
+
+  // 4 bits: lane holds tokens lane + 32 j; each byte of a P limb word is stored on its own.
+  __device__ void softmax4(uint32_t pairs, const int (&al)[G][TPL], const int (&am)[G][TPL],
+                           const int (&ah)[G][TPL]) {
 #pragma unroll
     for (int g = 0; g < G; ++g) {
       float lg[TPL], mu = -INFINITY;
@@ -364,23 +480,12 @@ struct Decoder {
 #pragma unroll
       for (int j = 0; j < TPL; ++j) {
         const int t = lane + 32 * j;
-        int row, k, mb;
-        float f = pp[j] * scv;
-        if (BITS == 2) {
-          row = t >> 4;
-          k = t & 3;
-          mb = (t >> 2) & 3;
-          if (k & 1) f *= 0.25f;
-        } else {
-          row = t >> 3;
-          k = t & 1;
-          mb = (t >> 1) & 3;
-        }
-        const uint32_t Pq = __float2uint_rn(f);
-        uint8_t* base = pwb + ((row * 3) * NSET + k) * 4 + mb;
+        const int row = t >> 3, k = t & 1, mb = (t >> 1) & 3;  // row t/8, set t%2, byte (t%8)/2
+        const uint32_t Pq = __float2uint_rn(pp[j] * scv);
+        uint8_t* base = pwb + ((row * 3) * 2 + k) * 4 + mb;  // limb b of row r: 8 bytes at (3 r + b) * 8
         base[0] = static_cast<uint8_t>(Pq & 255u);
-        base[NSET * 4] = static_cast<uint8_t>((Pq >> 8) & 255u);
-        base[2 * NSET * 4] = static_cast<uint8_t>((Pq >> 16) & 255u);
+        base[8] = static_cast<uint8_t>((Pq >> 8) & 255u);
+        base[16] = static_cast<uint8_t>((Pq >> 16) & 255u);
       }
     }
   }
@@ -447,32 +552,30 @@ struct Decoder {
   }
 
   // ---- K half of a residual unit (16 fp16 rows): logits and softmax weights --------------------
-  __device__ void residual_k(const uint8_t* kt, int nvalid) {
+  // q is read in fp16 from global memory (L1-resident: every lane pair reads the same 256 bytes).
+  __device__ void residual_k(const uint8_t* kt, int nvalid, long long head) {
     const int t = lane >> 1, hf = lane & 1;  // 2 lanes per token, 64 channels each
 #pragma unroll
     for (int g = 0; g < G; ++g) {
+      const uint4* qp = reinterpret_cast<const uint4*>(a.q + (static_cast<size_t>(head) * G + g) * kHeadDim);
       float dot = 0.f;
 #pragma unroll
       for (int k = 0; k < 8; ++k) {
         const int cc = (k + lane) & 7;  // bank-conflict-free chunk order
         const int c0 = 64 * hf + 8 * cc;
         const uint4 kv = *reinterpret_cast<const uint4*>(kt + t * 256 + 2 * c0);
-        const float4 q0 = *reinterpret_cast<const float4*>(&S.qf[g][c0]);
-        const float4 q1 = *reinterpret_cast<const float4*>(&S.qf[g][c0 + 4]);
-        const float2 k0 = __half22float2(*reinterpret_cast<const __half2*>(&kv.x));
-        const float2 k1 = __half22float2(*reinterpret_cast<const __half2*>(&kv.y));
-        const float2 k2 = __half22float2(*reinterpret_cast<const __half2*>(&kv.z));
-        const float2 k3 = __half22float2(*reinterpret_cast<const __half2*>(&kv.w));
-        dot = fmaf(q0.x, k0.x, dot);
-        dot = fmaf(q0.y, k0.y, dot);
-        dot = fmaf(q0.z, k1.x, dot);
-        dot = fmaf(q0.w, k1.y, dot);
-        dot = fmaf(q1.x, k2.x, dot);
-        dot = fmaf(q1.y, k2.y, dot);
-        dot = fmaf(q1.z, k3.x, dot);
-        dot = fmaf(q1.w, k3.y, dot);
+        const uint4 qv = __ldg(qp + (c0 >> 3));
+        const uint32_t kw[4] = {kv.x, kv.y, kv.z, kv.w}, qw[4] = {qv.x, qv.y, qv.z, qv.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 kf = __half22float2(*reinterpret_cast<const __half2*>(&kw[e]));
+          const float2 qf = __half22float2(*reinterpret_cast<const __half2*>(&qw[e]));
+          dot = fmaf(qf.x, kf.x, dot);
+          dot = fmaf(qf.y, kf.y, dot);
+        }
       }
       dot += __shfl_xor_sync(kFull, dot, 1);
+      dot *= a.qscale;
       const bool valid = t < nvalid;
       const float lg = valid ? dot : -INFINITY;
       const float m_new = fmaxf(m[g], warp_max(lg));
@@ -653,7 +756,7 @@ struct Decoder {
     if (lane == 0) {  // halves 0, 1, 2 = K0, V0, K1
       issue_half(0, head, local);
       issue_half(1, head, local);
-      if (nhalves > 2) issue_half(2, h1, l1);
+      if (kBuffers == 3 && nhalves > 2) issue_half(2, h1, l1);
     }
     uint32_t pairs = load_pairs(head, local);
     long long cur_head = -1, seg_a = ub;
@@ -677,10 +780,11 @@ struct Decoder {
       if (quant)
         quantized_k(S.buf[hk % kBuffers], head, local, pairs);
       else
-        residual_k(S.buf[hk % kBuffers], nvalid);
+        residual_k(S.buf[hk % kBuffers], nvalid, head);
       __syncwarp();
       fence_proxy_async_smem();
-      if (lane == 0 && hk + 3 < nhalves) issue_half(hk + 3, h1, l1);  // V half of the next unit
+      // half hk + kBuffers reuses the buffer just consumed: the next unit's V (ring of 3) or K (2)
+      if (lane == 0 && hk + kBuffers < nhalves) issue_half(hk + kBuffers, h1, l1);
       // V half
       if (!wait_half(hk + 1)) {
         if (lane == 0) report_status(a.status, KIVI_ERR_DEVICE_TIMEOUT);
@@ -693,7 +797,13 @@ struct Decoder {
         residual_v(S.buf[(hk + 1) % kBuffers], nvalid);
       __syncwarp();
       fence_proxy_async_smem();
-      if (lane == 0 && hk + 4 < nhalves) issue_half(hk + 4, h2, l2);  // K half of the unit after
+      // the unit after next's K half (ring of 3) or the next unit's V half (2)
+      if (lane == 0 && hk + 1 + kBuffers < nhalves) {
+        if (kBuffers == 3)
+          issue_half(hk + 4, h2, l2);
+        else
+          issue_half(hk + 3, h1, l1);
+      }
       pairs = pairs_next;
       head = h1;
       local = l1;
@@ -706,7 +816,7 @@ struct Decoder {
 };
 
 template <int BITS, int G>
-__global__ void __launch_bounds__(kWarps * 32, G == 1 ? 4 : 1) decode_kernel(const __grid_constant__ DecodeArgs a) {
+__global__ void __launch_bounds__(kWarps * 32, G == 1 ? KIVI_DECODE_MIN_CTAS : 1) decode_kernel(const __grid_constant__ DecodeArgs a) {
   extern __shared__ __align__(128) uint8_t smem_raw[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   WarpSmem<G>& S = reinterpret_cast<WarpSmem<G>*>(smem_raw)[warp];
