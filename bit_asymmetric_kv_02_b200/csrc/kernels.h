@@ -24,6 +24,7 @@ struct QuantizeArgs {
   int res_tok0;    // first source token copied into residual slot 0
   int res_tokens;  // tokens copied into the residual (0: none)
   int residual, capacity, group_k, group_v;
+  int lg_gk, lg_gv;  // log2(group_k), log2(group_v): set by launch_quantize_blocks
 };
 
 struct AppendArgs {

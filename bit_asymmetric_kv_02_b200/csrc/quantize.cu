@@ -5,10 +5,13 @@
 //   consecutive channels), Per-Token量子化（Value Cache）(V groups: g_v consecutive tokens) and
 //   残差バッファ（Residual Buffer）(the newest tokens stay fp16 until a block is flushed).
 //
-// One CTA quantizes one R-token block of K or of V for one (batch, KV head):
-//   pass 1 reads the block once from HBM (128-bit loads) and reduces the group minima / maxima;
-//   s = fp16_rn((max - min)/(2^b - 1)) is formed in fp64 (exact range, one rounding), z = min;
-//   pass 2 re-reads the block (L2-resident) and emits codes, 32/b per uint32 word.
+// One CTA quantizes one R-token block of K or of V for one (batch, KV head).  Two kernels:
+//   R <= 512 (quantize_tiles_kernel): 2R threads hold the whole block in registers (one 128-bit
+//     load per thread and token row), reduce the group minima / maxima, and emit the codes from
+//     the same registers: the block is read from HBM exactly once.
+//   R = 1024 (quantize_blocks_kernel): 256 threads; pass 1 reduces the extremes, pass 2 re-reads
+//     the block from L2 and emits the codes.
+// s = fp16_rn((max - min)/(2^b - 1)) is formed in fp64 (exact range, one rounding), z = min.
 // A code is RNE of the exact rational (x - z)/s.  It is computed in fp32 as (x - z) * (1/s), whose
 // relative error is below 3*2^-24, i.e. below 2^-18 absolute for every reachable value; when the
 // fp32 value lies within 2^-12 of a half-integer the element is re-decided with an fp64 division,
@@ -56,7 +59,7 @@ __device__ __forceinline__ GroupParams make_group(float lo, float hi, int levels
 
 // Q of one element (section 量子化アルゴリズム, Q equation) with the stored fp16 s and z, taken
 // exactly: the fp64 quotient decides (used near ties only).
-__device__ __forceinline__ uint32_t quantize_exact(float x, const GroupParams& g, int levels) {
+__device__ __noinline__ uint32_t quantize_exact(float x, const GroupParams& g, int levels) {
   const double r64 = (static_cast<double>(x) - static_cast<double>(g.zf)) / static_cast<double>(h2f(g.s_bits));
   return min(static_cast<uint32_t>(rint(r64)), static_cast<uint32_t>(levels));
 }
@@ -221,6 +224,297 @@ __device__ void quantize_v_block(const uint16_t* __restrict__ src, int R, int gv
   }
 }
 
+// Residual copy: tokens [res_tok0, res_tok0 + res_tokens) of the source -> residual slots 0..
+__device__ void copy_residual(const QuantizeArgs& a, int bh) {
+  const size_t src_tok = static_cast<size_t>(bh) * a.src_tokens + a.res_tok0;
+  const uint4* ks = reinterpret_cast<const uint4*>(a.k_src + src_tok * kHeadDim);
+  const uint4* vs = reinterpret_cast<const uint4*>(a.v_src + src_tok * kHeadDim);
+  uint4* kd = reinterpret_cast<uint4*>(a.k_res + static_cast<size_t>(bh) * a.residual * kHeadDim);
+  uint4* vd = reinterpret_cast<uint4*>(a.v_res + static_cast<size_t>(bh) * a.residual * kHeadDim);
+  const int n = a.res_tokens * kChunks;
+  for (int i = threadIdx.x; i < n; i += blockDim.x) {
+    kd[i] = __ldg(ks + i);
+    vd[i] = __ldg(vs + i);
+  }
+}
+
+// ---------------------------------------------------------------------------------------------
+// Register-staged blocks (R <= 512): a CTA of 2R threads reads its block from HBM once.  Thread
+// (token group tg, chunk c) holds tokens 8 tg .. 8 tg + 7 x channels 8 c .. 8 c + 7 in registers.
+// Every K group (g_k >= 32 channels) and every V group (g_v >= 32 tokens) is a union of whole
+// thread tiles, so a thread quantizes its 64 values with one (s, z).  Group extremes travel as the
+// fp16 pair (min, -max), which one packed minimum reduces.
+// ---------------------------------------------------------------------------------------------
+constexpr int kTileTokens = 8;
+
+__device__ __forceinline__ __half2 tile_min_negmax(const uint4 (&x)[kTileTokens]) {
+  __half2 lo = *reinterpret_cast<const __half2*>(&x[0].x), hi = lo;
+#pragma unroll
+  for (int k = 0; k < kTileTokens; ++k) {
+    const uint32_t w[4] = {x[k].x, x[k].y, x[k].z, x[k].w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const __half2 v = *reinterpret_cast<const __half2*>(&w[i]);
+      lo = __hmin2(lo, v);
+      hi = __hmax2(hi, v);
+    }
+  }
+  return __halves2half2(__hmin(__low2half(lo), __high2half(lo)), __hneg(__hmax(__low2half(hi), __high2half(hi))));
+}
+
+__device__ __forceinline__ uint32_t comp4(const uint4& v, int i) {
+  return i == 0 ? v.x : (i == 1 ? v.y : (i == 2 ? v.z : v.w));
+}
+
+__device__ __forceinline__ __half2 shfl_xor_h2(__half2 v, int off) {
+  const uint32_t u = __shfl_xor_sync(0xffffffffu, *reinterpret_cast<uint32_t*>(&v), off);
+  return *reinterpret_cast<const __half2*>(&u);
+}
+
+__device__ __forceinline__ GroupParams group_from_pair(__half2 m, int levels) {
+  return make_group(__low2float(m), -__high2float(m), levels);
+}
+
+// ---- 2 bits: the code as a count of thresholds ----------------------------------------------
+// For s > 0, Q(x) = clamp(rint((x - z)/s), 0, 3) with ties to even is [r > 1/2] + [r >= 3/2] +
+// [r > 5/2], r = (x - z)/s, i.e. [x > T0] + [x >= T1] + [x > T2] with T_k = z + (k + 1/2) s.  T_k is
+// exact in fp64.  Over fp16 x, x > T equals x > (largest fp16 <= T) and x >= T equals
+// x > (largest fp16 < T), so three strict fp16 comparisons decide the code exactly; s = 0 (all
+// codes 0) uses +inf.
+struct Thresh2 {
+  uint32_t t[3];  // each threshold in both halves of a half2
+};
+
+__device__ __forceinline__ uint16_t f64_to_h_rd(double x) {
+  uint16_t r;
+  asm("cvt.rm.f16.f64 %0, %1;" : "=h"(r) : "d"(x));
+  return r;
+}
+// The largest fp16 below the finite fp16 h.
+__device__ __forceinline__ uint16_t h_below(uint16_t h) {
+  if ((h & 0x7FFFu) == 0) return 0x8001u;  // below +-0: the negative subnormal closest to 0
+  return (h & 0x8000u) ? static_cast<uint16_t>(h + 1) : static_cast<uint16_t>(h - 1);
+}
+
+__device__ Thresh2 make_thresh2(const GroupParams& g) {
+  Thresh2 t;
+  const double s = static_cast<double>(h2f(g.s_bits)), z = static_cast<double>(g.zf);
+#pragma unroll
+  for (int k = 0; k < 3; ++k) {
+    uint16_t h = 0x7C00u;  // +inf
+    if (s > 0.0) {
+      const double T = z + (k + 0.5) * s;  // exact
+      h = f64_to_h_rd(T);
+      if (k == 1 && static_cast<double>(h2f(h)) == T) h = h_below(h);
+    }
+    t.t[k] = static_cast<uint32_t>(h) * 0x00010001u;
+  }
+  return t;
+}
+
+// Codes of one half2 as the half2 (1024 + c0, 1024 + c1): byte 0 holds c0 and byte 2 holds c1.
+__device__ __forceinline__ uint32_t codes2_h2(uint32_t x2, const Thresh2& t) {
+  const __half2 x = *reinterpret_cast<const __half2*>(&x2);
+  const __half2 t0 = *reinterpret_cast<const __half2*>(&t.t[0]);
+  const __half2 t1 = *reinterpret_cast<const __half2*>(&t.t[1]);
+  const __half2 t2 = *reinterpret_cast<const __half2*>(&t.t[2]);
+  const __half2 c = __hadd2(__hadd2(__hgt2(x, t0), __hgt2(x, t1)), __hadd2(__hgt2(x, t2), __float2half2_rn(1024.f)));
+  return *reinterpret_cast<const uint32_t*>(&c);
+}
+
+// Four 2-bit codes held one per byte -> an 8-bit field (byte i at bits 2 i).  The product with
+// 2^24 + 2^18 + 2^12 + 2^6 moves byte i to bit 24 + 2 i; every other partial product lands below
+// bit 24 (their sum stays below 2^24) or above bit 31.
+__device__ __forceinline__ uint32_t gather4x2(uint32_t bytes) { return (bytes * 0x01041040u) >> 24; }
+
+// 16-bit codes of the 8 channels of one token row, channel 8 c + j at bits 2 j.
+__device__ __forceinline__ uint32_t row_codes2(const uint4& v, const Thresh2& t) {
+  const uint32_t h0 = codes2_h2(v.x, t), h1 = codes2_h2(v.y, t), h2 = codes2_h2(v.z, t), h3 = codes2_h2(v.w, t);
+  return gather4x2(__byte_perm(h0, h1, 0x6420)) | (gather4x2(__byte_perm(h2, h3, 0x6420)) << 8);
+}
+
+// Codes of the 8 channels of one token row of a tile (bits BITS * j for channel 8 c + j).
+template <int BITS>
+__device__ __forceinline__ uint32_t quantize_row8(const uint4& v, const GroupParams& g) {
+  constexpr int L = (1 << BITS) - 1;
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  uint32_t r = 0;
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    uint32_t qa, qb;
+    quantize_pair(w[e], g, L, qa, qb);
+    r += (qa << (BITS * 2 * e)) + (qb << (BITS * (2 * e + 1)));
+  }
+  return r;
+}
+
+template <int BITS>
+__device__ void quantize_k_tiles(const uint16_t* __restrict__ src, int R, int lg_gk, uint32_t* __restrict__ codes,
+                                 uint16_t* __restrict__ scale, uint16_t* __restrict__ zero) {
+  constexpr int L = (1 << BITS) - 1;
+  __shared__ __half2 red[1024 / 32][kHeadDim / 32];
+  __shared__ GroupParams grp[kHeadDim / 32];
+  __shared__ Thresh2 thr[kHeadDim / 32];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nwarps = blockDim.x >> 5;
+  const int c = tid & 15, tg = tid >> 4;
+  const uint4* s4 = reinterpret_cast<const uint4*>(src) + (tg * kTileTokens) * kChunks + c;
+  uint4 x[kTileTokens];
+#pragma unroll
+  for (int k = 0; k < kTileTokens; ++k) x[k] = __ldg(s4 + k * kChunks);
+
+  // K group of chunk c: chunks [cpg * g, cpg * (g + 1)), cpg = g_k / 8; the warp's two token
+  // groups (lanes < 16 and >= 16) hold the same chunks
+  const int lg_cpg = lg_gk - 3, ngk = kHeadDim >> lg_gk;
+  __half2 m = tile_min_negmax(x);
+  for (int off = 1; off < (1 << lg_cpg); off <<= 1) m = __hmin2(m, shfl_xor_h2(m, off));
+  m = __hmin2(m, shfl_xor_h2(m, 16));
+  if (lane < 16 && (c & ((1 << lg_cpg) - 1)) == 0) red[warp][c >> lg_cpg] = m;
+  __syncthreads();
+  if (tid < ngk) {
+    __half2 t = red[0][tid];
+    for (int w = 1; w < nwarps; ++w) t = __hmin2(t, red[w][tid]);
+    const GroupParams gp = group_from_pair(t, L);
+    if constexpr (BITS == 2)
+      thr[tid] = make_thresh2(gp);
+    else
+      grp[tid] = gp;
+    scale[tid] = gp.s_bits;
+    zero[tid] = gp.z_bits;
+  }
+  __syncthreads();
+  const int tok0 = tg * kTileTokens;
+  if constexpr (BITS == 4) {  // K word c of a token is exactly the tile's 8 channels
+    const GroupParams g = grp[c >> lg_cpg];
+#pragma unroll
+    for (int k = 0; k < kTileTokens; ++k) codes[(tok0 + k) * (kHeadDim / 8) + c] = quantize_row8<4>(x[k], g);
+  } else {  // K word c / 2 of a token: chunk 2i in bits 0..15, chunk 2i + 1 in bits 16..31
+    const Thresh2 t = thr[c >> lg_cpg];
+    uint32_t h[kTileTokens];
+#pragma unroll
+    for (int k = 0; k < kTileTokens; ++k) h[k] = row_codes2(x[k], t);
+    const bool odd = c & 1;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {  // the even chunk stores tokens 0..3 of the tile, the odd one 4..7
+      const uint32_t other = __shfl_xor_sync(0xffffffffu, odd ? h[j] : h[4 + j], 1);
+      const int k = odd ? 4 + j : j;
+      const uint32_t word = odd ? (other | (h[4 + j] << 16)) : (h[j] | (other << 16));
+      codes[(tok0 + k) * (kHeadDim / 16) + (c >> 1)] = word;
+    }
+  }
+}
+
+template <int BITS>
+__device__ void quantize_v_tiles(const uint16_t* __restrict__ src, int R, int lg_gv, uint32_t* __restrict__ codes,
+                                 uint16_t* __restrict__ scale, uint16_t* __restrict__ zero) {
+  constexpr int L = (1 << BITS) - 1;
+  __shared__ __half2 red[1024 / 32];
+  __shared__ GroupParams grp[512 / 32];
+  __shared__ Thresh2 thr[512 / 32];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int c = tid & 15, tg = tid >> 4;
+  const uint4* s4 = reinterpret_cast<const uint4*>(src) + (tg * kTileTokens) * kChunks + c;
+  uint4 x[kTileTokens];
+#pragma unroll
+  for (int k = 0; k < kTileTokens; ++k) x[k] = __ldg(s4 + k * kChunks);
+
+  // a warp's 16 tokens lie in one V group (g_v >= 32); group j spans warps [j g_v / 16, ...)
+  __half2 m = tile_min_negmax(x);
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) m = __hmin2(m, shfl_xor_h2(m, off));
+  if (lane == 0) red[warp] = m;
+  __syncthreads();
+  const int ngv = R >> lg_gv, wpg = 1 << (lg_gv - 4);
+  if (tid < ngv) {
+    __half2 t = red[tid * wpg];
+    for (int w = 1; w < wpg; ++w) t = __hmin2(t, red[tid * wpg + w]);
+    const GroupParams gp = group_from_pair(t, L);
+    if constexpr (BITS == 2)
+      thr[tid] = make_thresh2(gp);
+    else
+      grp[tid] = gp;
+    scale[tid] = gp.s_bits;
+    zero[tid] = gp.z_bits;
+  }
+  __syncthreads();
+  const int gv = (tg * kTileTokens) >> lg_gv;
+  // codes of channel 8 c + e for the tile's 8 tokens, token k at bits BITS * k
+  uint32_t col[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  if constexpr (BITS == 4) {
+    const GroupParams g = grp[gv];
+#pragma unroll
+    for (int k = 0; k < kTileTokens; ++k) {
+      const uint32_t w[4] = {x[k].x, x[k].y, x[k].z, x[k].w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        uint32_t qa, qb;
+        quantize_pair(w[e], g, L, qa, qb);
+        col[2 * e] += qa << (BITS * k);
+        col[2 * e + 1] += qb << (BITS * k);
+      }
+    }
+  } else {
+    // tokens 2a, 2a + 1 of channels 2e, 2e + 1 -> one word of four byte codes, then per channel
+    // the bytes of tokens 0..3 and 4..7 -> two 8-bit fields
+    const Thresh2 t = thr[gv];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      uint32_t A[4];
+#pragma unroll
+      for (int a2 = 0; a2 < 4; ++a2) {
+        const uint32_t w0 = comp4(x[2 * a2], e), w1 = comp4(x[2 * a2 + 1], e);
+        A[a2] = __byte_perm(codes2_h2(w0, t), codes2_h2(w1, t), 0x6240);
+      }
+      col[2 * e] = gather4x2(__byte_perm(A[0], A[1], 0x5410)) | (gather4x2(__byte_perm(A[2], A[3], 0x5410)) << 8);
+      col[2 * e + 1] = gather4x2(__byte_perm(A[0], A[1], 0x7632)) | (gather4x2(__byte_perm(A[2], A[3], 0x7632)) << 8);
+    }
+  }
+  if constexpr (BITS == 4) {  // V word (tg, 8 c + e) holds exactly the tile's 8 tokens
+    uint4* dst = reinterpret_cast<uint4*>(codes + tg * kHeadDim + 8 * c);
+    dst[0] = make_uint4(col[0], col[1], col[2], col[3]);
+    dst[1] = make_uint4(col[4], col[5], col[6], col[7]);
+  } else {  // V word (tg / 2, 8 c + e): the even token group in bits 0..15, the odd one in 16..31
+    const bool odd = tg & 1;
+    uint32_t word[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {  // the even token group stores channels 0..3, the odd one 4..7
+      const uint32_t other = __shfl_xor_sync(0xffffffffu, odd ? col[e] : col[4 + e], 16);
+      word[e] = odd ? (other | (col[4 + e] << 16)) : (col[e] | (other << 16));
+    }
+    *reinterpret_cast<uint4*>(codes + (tg >> 1) * kHeadDim + 8 * c + (odd ? 4 : 0)) =
+        make_uint4(word[0], word[1], word[2], word[3]);
+  }
+}
+
+// grid: x = batch * kv_heads, y = 2 * nblocks (+1 residual-copy job); block = 2R threads (R <= 512)
+template <int BITS>
+__global__ void __launch_bounds__(1024) quantize_tiles_kernel(QuantizeArgs a) {
+  constexpr int P = 32 / BITS;
+  const int bh = blockIdx.x;
+  const int job = blockIdx.y;
+  const int R = a.residual;
+  const size_t C = static_cast<size_t>(a.capacity);
+  if (job < 2 * a.nblocks) {
+    const int blk = job >> 1;
+    const bool is_v = job & 1;
+    const size_t src_tok = static_cast<size_t>(bh) * a.src_tokens + a.src_tok0 + static_cast<size_t>(blk) * R;
+    const int dst_blk = a.dst_blk0 + blk;
+    const size_t dst_tok = static_cast<size_t>(dst_blk) * R;
+    if (!is_v) {
+      quantize_k_tiles<BITS>(a.k_src + src_tok * kHeadDim, R, a.lg_gk,
+                             a.k_codes + (static_cast<size_t>(bh) * C + dst_tok) * (kHeadDim / P),
+                             a.k_scale + (static_cast<size_t>(bh) * (C / R) + dst_blk) * (kHeadDim >> a.lg_gk),
+                             a.k_zero + (static_cast<size_t>(bh) * (C / R) + dst_blk) * (kHeadDim >> a.lg_gk));
+    } else {
+      quantize_v_tiles<BITS>(a.v_src + src_tok * kHeadDim, R, a.lg_gv,
+                             a.v_codes + (static_cast<size_t>(bh) * (C / P) + dst_tok / P) * kHeadDim,
+                             a.v_scale + static_cast<size_t>(bh) * (C >> a.lg_gv) + (dst_tok >> a.lg_gv),
+                             a.v_zero + static_cast<size_t>(bh) * (C >> a.lg_gv) + (dst_tok >> a.lg_gv));
+    }
+  } else {
+    copy_residual(a, bh);
+  }
+}
+
 // grid: x = batch * kv_heads, y = 2 * nblocks (+1 residual-copy job when res_tokens > 0)
 template <int BITS>
 __global__ void __launch_bounds__(kThreads) quantize_blocks_kernel(QuantizeArgs a) {
@@ -247,17 +541,7 @@ __global__ void __launch_bounds__(kThreads) quantize_blocks_kernel(QuantizeArgs 
                              a.v_zero + static_cast<size_t>(bh) * (C / a.group_v) + dst_tok / a.group_v);
     }
   } else {
-    // residual copy: tokens [res_tok0, res_tok0 + res_tokens) of the source -> slots 0..
-    const size_t src_tok = static_cast<size_t>(bh) * a.src_tokens + a.res_tok0;
-    const uint4* ks = reinterpret_cast<const uint4*>(a.k_src + src_tok * kHeadDim);
-    const uint4* vs = reinterpret_cast<const uint4*>(a.v_src + src_tok * kHeadDim);
-    uint4* kd = reinterpret_cast<uint4*>(a.k_res + static_cast<size_t>(bh) * R * kHeadDim);
-    uint4* vd = reinterpret_cast<uint4*>(a.v_res + static_cast<size_t>(bh) * R * kHeadDim);
-    const int n = a.res_tokens * kChunks;
-    for (int i = threadIdx.x; i < n; i += kThreads) {
-      kd[i] = __ldg(ks + i);
-      vd[i] = __ldg(vs + i);
-    }
+    copy_residual(a, bh);
   }
 }
 
@@ -274,14 +558,23 @@ __global__ void __launch_bounds__(256) append_kernel(AppendArgs a) {
 
 }  // namespace
 
-cudaError_t launch_quantize_blocks(const QuantizeArgs& a, int bits, cudaStream_t stream) {
-  const int jobs = 2 * a.nblocks + (a.res_tokens > 0 ? 1 : 0);
+cudaError_t launch_quantize_blocks(const QuantizeArgs& args, int bits, cudaStream_t stream) {
+  const int jobs = 2 * args.nblocks + (args.res_tokens > 0 ? 1 : 0);
   if (jobs == 0) return cudaSuccess;
+  QuantizeArgs a = args;  // group sizes are powers of two (checked by the caller)
+  a.lg_gk = __builtin_ctz(static_cast<unsigned>(a.group_k));
+  a.lg_gv = __builtin_ctz(static_cast<unsigned>(a.group_v));
   dim3 grid(a.bh, jobs);
-  if (bits == 2)
+  if (a.residual <= 512) {  // one thread per 8 tokens x 8 channels of a block
+    if (bits == 2)
+      quantize_tiles_kernel<2><<<grid, 2 * a.residual, 0, stream>>>(a);
+    else
+      quantize_tiles_kernel<4><<<grid, 2 * a.residual, 0, stream>>>(a);
+  } else if (bits == 2) {
     quantize_blocks_kernel<2><<<grid, kThreads, 0, stream>>>(a);
-  else
+  } else {
     quantize_blocks_kernel<4><<<grid, kThreads, 0, stream>>>(a);
+  }
   return cudaGetLastError();
 }
 

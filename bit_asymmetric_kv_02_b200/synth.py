@@ -37,14 +37,19 @@ class Workload:
     tokens: int
     head_dim: int = 128
     bits: int = 2
-    group: int = 32          # G_k = G_v
+    group: int = 32          # G_k (and G_v unless group_v is set)
     residual: int = 128      # R
     seed: int = 1000
     steps: int = 0           # streaming decode steps after the prefill (0: single attention)
+    group_v: int = 0         # G_v when it differs from G_k (0: G_v = G_k)
 
     @property
     def gqa(self) -> int:
         return self.q_heads // self.kv_heads
+
+    @property
+    def gv(self) -> int:
+        return self.group_v or self.group
 
     def with_(self, **kw) -> "Workload":
         return replace(self, **kw)

@@ -37,7 +37,7 @@ def run_prefill_case(w: synth.Workload, heads=None, capacity=None, check_attenti
     cap = capacity if capacity is not None else ((T + w.residual - 1) // w.residual) * w.residual
     k, v = synth.prompt_kv(w, T)
     q = synth.queries(w, 0)
-    cache = kivi.KiviCache(w.batch, w.kv_heads, cap, bits=w.bits, group_k=w.group, group_v=w.group,
+    cache = kivi.KiviCache(w.batch, w.kv_heads, cap, bits=w.bits, group_k=w.group, group_v=w.gv,
                            residual=w.residual, num_q_heads=w.q_heads)
     kd = torch.from_numpy(k).cuda()
     vd = torch.from_numpy(v).cuda()
@@ -51,7 +51,7 @@ def run_prefill_case(w: synth.Workload, heads=None, capacity=None, check_attenti
     heads = heads if heads is not None else [(b, h) for b in range(w.batch) for h in range(w.kv_heads)]
     worst = (0.0, 0.0)
     for (b, h) in heads:
-        hc = O.HeadCache(w.head_dim, w.bits, w.group, w.group, w.residual, cap)
+        hc = O.HeadCache(w.head_dim, w.bits, w.group, w.gv, w.residual, cap)
         hc.prefill(k[b, h], v[b, h])
         gc.assert_head_bitexact(gc.gpu_buffers_of_head(cache, b, h, n_quant, n_res), hc.packed(),
                                 f"{w.name} head {(b, h)}")
@@ -76,6 +76,15 @@ SMALL = [
     synth.TINY.with_(name="gqa2_4bit", batch=1, q_heads=4, kv_heads=2, tokens=300, bits=4, seed=15),
     synth.TINY.with_(name="gqa8", batch=1, q_heads=8, kv_heads=1, tokens=500, seed=16),
     synth.TINY.with_(name="many_heads_short", batch=16, q_heads=8, kv_heads=8, tokens=200, seed=17),
+    # residual sizes and G_k != G_v: the register-tiled quantize path (R <= 512) and the two-pass one (R = 1024)
+    synth.TINY.with_(name="R128_gk32_gv128", batch=2, q_heads=2, kv_heads=2, tokens=3 * 128 + 9, group_v=128,
+                     seed=18),
+    synth.TINY.with_(name="R256_gk64_gv256", batch=2, q_heads=4, kv_heads=2, tokens=2 * 256 + 77, group=64,
+                     group_v=256, residual=256, seed=19),
+    synth.TINY.with_(name="R512_4bit_gk32_gv64", batch=1, q_heads=2, kv_heads=2, tokens=2 * 512 + 300, bits=4,
+                     group_v=64, residual=512, seed=20),
+    synth.TINY.with_(name="R1024_2bit_gk128_gv32", batch=1, q_heads=2, kv_heads=2, tokens=2 * 1024 + 5, group=128,
+                     group_v=32, residual=1024, seed=22),
 ]
 
 
