@@ -40,16 +40,16 @@ namespace kivi {
 
 namespace {
 
-constexpr int kWarps = 4;           // stream-K workers per CTA
+// Stream-K workers (warps) per CTA: one CTA per SM.  The warps of one CTA are scheduled fairly;
+// warps of separate CTAs on one SM are not (the oldest CTA's warps take precedence and finish
+// early, leaving the SM with fewer warps for the rest of the launch).
+template <int G>
+__host__ __device__ constexpr int warps_per_cta() {
+  return G == 1 ? 16 : 8;  // 16 x 128 registers or 8 x 255 registers
+}
 constexpr int kHalfBytes = 4096;    // one half unit: the K part or the V part of a unit
-#ifndef KIVI_DECODE_BUFFERS
-#define KIVI_DECODE_BUFFERS 3
-#endif
-#ifndef KIVI_DECODE_MIN_CTAS
-#define KIVI_DECODE_MIN_CTAS 4
-#endif
 // Half-unit buffers per warp: 3 gives the ring K0 V0 K1 | V1 K2 V2 | ..., 2 gives K | V.
-constexpr int kBuffers = KIVI_DECODE_BUFFERS;
+constexpr int kBuffers = 3;
 static_assert(kBuffers == 2 || kBuffers == 3, "the ring holds 2 or 3 half units");
 constexpr int kResTokens = 16;      // tokens per residual unit
 constexpr unsigned kFull = 0xffffffffu;
@@ -816,12 +816,12 @@ struct Decoder {
 };
 
 template <int BITS, int G>
-__global__ void __launch_bounds__(kWarps * 32, G == 1 ? KIVI_DECODE_MIN_CTAS : 1) decode_kernel(const __grid_constant__ DecodeArgs a) {
+__global__ void __launch_bounds__(warps_per_cta<G>() * 32, 1) decode_kernel(const __grid_constant__ DecodeArgs a) {
   extern __shared__ __align__(128) uint8_t smem_raw[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   WarpSmem<G>& S = reinterpret_cast<WarpSmem<G>*>(smem_raw)[warp];
   const long long W = a.workers, U = a.total_units;
-  const long long worker = static_cast<long long>(blockIdx.x) * kWarps + warp;
+  const long long worker = static_cast<long long>(blockIdx.x) * warps_per_cta<G>() + warp;
   if (worker >= W) return;  // the last CTA may hold fewer workers
   const long long ub = U * worker / W, ue = U * (worker + 1) / W;  // non-empty because W <= U
   Decoder<BITS, G> d(a, S, lane, worker, ub, ue);
@@ -830,6 +830,7 @@ __global__ void __launch_bounds__(kWarps * 32, G == 1 ? KIVI_DECODE_MIN_CTAS : 1
 
 template <int BITS, int G>
 cudaError_t plan_for(DecodePlan* plan) {
+  constexpr int kWarps = warps_per_cta<G>();
   const int smem = kWarps * static_cast<int>(sizeof(WarpSmem<G>));
   cudaError_t e = cudaFuncSetAttribute(decode_kernel<BITS, G>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
