@@ -48,9 +48,12 @@ __host__ __device__ constexpr int warps_per_cta() {
   return G == 1 ? 16 : 8;  // 16 x 128 registers or 8 x 255 registers
 }
 constexpr int kHalfBytes = 4096;    // one half unit: the K part or the V part of a unit
-// Half-unit buffers per warp: 3 gives the ring K0 V0 K1 | V1 K2 V2 | ..., 2 gives K | V.
-constexpr int kBuffers = 3;
-static_assert(kBuffers == 2 || kBuffers == 3, "the ring holds 2 or 3 half units");
+// Half-unit buffers per warp: 3 gives the ring K0 V0 K1 | V1 K2 V2 | ..., 2 gives K | V.  One query
+// per KV head uses 2 (measured 1.4% faster than 3 at 16 warps per SM), several queries use 3.
+template <int G>
+__host__ __device__ constexpr int ring_buffers() {
+  return G == 1 ? 2 : 3;
+}
 constexpr int kResTokens = 16;      // tokens per residual unit
 constexpr unsigned kFull = 0xffffffffu;
 constexpr float kQRange = 8388544.f;   // 2^23 - 64: largest |Q| before rounding (signed 24-bit limbs)
@@ -58,10 +61,10 @@ constexpr float kPRange = 16777088.f;  // 2^24 - 128: largest P before rounding 
 
 template <int G>
 struct __align__(16) WarpSmem {
-  uint8_t buf[kBuffers][kHalfBytes];
+  uint8_t buf[ring_buffers<G>()][kHalfBytes];
   uint4 qw[G][24];  // Q limbs of each query: 96 words
   uint4 pw[G][24];  // P limbs of each query: up to 96 words
-  uint64_t bar[kBuffers];
+  uint64_t bar[ring_buffers<G>()];
 };
 
 // Maximum over the warp in one instruction (sm_100a redux.sync on f32; NaN inputs are ignored).
@@ -128,6 +131,7 @@ struct Decoder {
   static constexpr int UT = BITS == 2 ? 128 : 64;  // tokens per quantized unit (8 KB of codes)
   static constexpr int TPL = UT / 32;              // tokens per lane (K side)
   static constexpr int ROWS = UT / P;              // V word rows per unit (8)
+  static constexpr int kBuffers = ring_buffers<G>();
 
   const DecodeArgs& a;
   WarpSmem<G>& S;
@@ -385,12 +389,29 @@ struct Decoder {
     }
   }
 
+  // V scale and zero of this lane's four tokens (one V group), and the unit's largest V scale.
+  struct VScales {
+    float sv, zv, smax, inv_smax;
+  };
+  __device__ __forceinline__ VScales v_scales2(uint32_t pairs) const {
+    VScales v;
+    const uint32_t vp = __shfl_sync(kFull, pairs, 8 + ((16 * (lane >> 2)) >> a.lg_gv));
+    v.sv = h2f(static_cast<uint16_t>(vp & 0xFFFFu));
+    v.zv = h2f(static_cast<uint16_t>(vp >> 16));
+    v.smax = warp_max(v_lane ? h2f(static_cast<uint16_t>(pairs & 0xFFFFu)) : 0.f);
+    v.inv_smax = v.smax > 0.f ? fast_rcp(v.smax) : 0.f;
+    return v;
+  }
+
   // 2 bits: lane (r, k) holds tokens 16 r + 4 j + k (j = 0..3), i.e. byte j of set k of V word row
   // r, so it forms that set's three P limb words itself; its four tokens share one V group.
-  __device__ void softmax2(uint32_t pairs, const int (&al)[G][TPL], const int (&am)[G][TPL],
+  // P is scaled by the bound (largest weight of the unit) x (largest V scale of the unit), which
+  // needs one warp reduction instead of two; the bound sums over the units to at most smax * l,
+  // the same error bound as the exact maximum.  A unit whose weights are all below 2^-64 of the
+  // running maximum contributes its z-terms only.
+  __device__ void softmax2(const VScales& vs, const int (&al)[G][TPL], const int (&am)[G][TPL],
                            const int (&ah)[G][TPL]) {
-    const uint32_t vp = __shfl_sync(kFull, pairs, 8 + ((16 * (lane >> 2)) >> a.lg_gv));
-    const float sv = h2f(static_cast<uint16_t>(vp & 0xFFFFu)), zv = h2f(static_cast<uint16_t>(vp >> 16));
+    const float sv = vs.sv, zv = vs.zv;
     const float set_scale = (lane & 1) ? 0.25f : 1.f;
     uint32_t* pw = reinterpret_cast<uint32_t*>(S.pw);
 #pragma unroll
@@ -405,20 +426,19 @@ struct Decoder {
 #pragma unroll
       for (int j = 0; j < TPL; ++j) p[j] = fast_exp2(lg[j] - m_new);
       const float psum = (p[0] + p[1]) + (p[2] + p[3]);
-      // P is scaled by the unit's largest p * s; the four tokens of a lane share s
-      const float mv = warp_max(fmaxf(fmaxf(p[0], p[1]), fmaxf(p[2], p[3])) * sv);
+      const float d = mu - m_new;  // <= 0: the unit's largest weight is 2^d
+      const bool hv = d > -64.f && vs.smax > 0.f;
       m[g] = m_new;
       l[g] = fmaf(l[g], alpha, psum);
       Z[g] = fmaf(Z[g], alpha, psum * zv);
       alpha_[g] = alpha;
-      hasv_[g] = mv > 0.f;
-      // P <= 2^24 - 124: the top token must not round to 2^24, where it would wrap to 0
-      const float scv = mv > 0.f ? kPRange * fast_rcp(mv) : 0.f;
-      invv_[g] = mv * (1.0f / kPRange);
-      const float f = scv * set_scale;
+      hasv_[g] = hv;
+      // P <= 2^24 - 128 (1 + 2^-20): the top token must not round to 2^24, where it would wrap to 0
+      invv_[g] = hv ? fast_exp2(d) * vs.smax * (1.0f / kPRange) : 0.f;
+      const float f = hv ? sv * (kPRange * vs.inv_smax) * fast_exp2(-d) * set_scale : 0.f;
       uint32_t L, M, H;
-      limb_words(static_cast<int>(__float2uint_rn(p[0] * sv * f)), static_cast<int>(__float2uint_rn(p[1] * sv * f)),
-                 static_cast<int>(__float2uint_rn(p[2] * sv * f)), static_cast<int>(__float2uint_rn(p[3] * sv * f)),
+      limb_words(static_cast<int>(__float2uint_rn(p[0] * f)), static_cast<int>(__float2uint_rn(p[1] * f)),
+                 static_cast<int>(__float2uint_rn(p[2] * f)), static_cast<int>(__float2uint_rn(p[3] * f)),
                  L, M, H);
       uint32_t* row = pw + g * 96 + (lane >> 2) * 12 + (lane & 3);  // row r, limb b, set k
       row[0] = L;
@@ -435,11 +455,14 @@ struct Decoder {
       qkey = key;
     }
     int al[G][TPL], am[G][TPL], ah[G][TPL];
-    k_dot(kt, al, am, ah);
-    if constexpr (BITS == 2)
-      softmax2(pairs, al, am, ah);
-    else
+    if constexpr (BITS == 2) {
+      const VScales vs = v_scales2(pairs);  // independent of the dot products: issued first
+      k_dot(kt, al, am, ah);
+      softmax2(vs, al, am, ah);
+    } else {
+      k_dot(kt, al, am, ah);
       softmax4(pairs, al, am, ah);
+    }
   }
 
   // 4 bits: lane holds tokens lane + 32 j; each byte of a P limb word is stored on its own.
