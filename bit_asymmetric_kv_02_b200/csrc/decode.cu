@@ -339,7 +339,7 @@ struct Decoder {
 #pragma unroll
       for (int j = 0; j < TPL; ++j) al[g][j] = am[g][j] = ah[g][j] = 0;
     if (BITS == 2) {
-#pragma unroll 1
+#pragma unroll  // both halves in one block: the second half's code words load during the first's dp4a
       for (int h = 0; h < 2; ++h) {
         const int hh = h ^ ((lane >> 2) & 1);  // bank-conflict-free order of the two 16-byte halves
         uint4 kw[TPL];
