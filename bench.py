@@ -37,6 +37,9 @@ UNIT = "cached tokens/s/head"
 SPEC_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
 WORKLOAD = synth.LARGE_BATCH
+FUSED = True   # append and decode in one launch (kivi_append_decode_attention); --separate-append: two
+STEP_NOTE = {True: "flush when full + append and decode attention in one launch",
+             False: "flush when full + append + decode attention"}
 DECODE_SOURCES = ["decode.cu", "common.cuh", "kernels.h"]
 
 
@@ -81,6 +84,11 @@ def l2_note(w: synth.Workload, n_quant: int) -> str:
     if gb * 1e3 > 2 * 126:
         return f"not flushed: inputs ({gb:.2f} GB per step) exceed the 126 MB L2"
     return f"WARNING: inputs ({gb * 1e3:.0f} MB per step) fit in the 126 MB L2; not flushed"
+
+
+def append_bytes(w: synth.Workload) -> int:
+    """Bytes a fused append adds to the decode launch: the new K and V rows read and written once."""
+    return w.batch * w.kv_heads * w.head_dim * 2 * 2 * 2
 
 
 def decode_alg_bytes(w: synth.Workload, n_quant: int, n_res: int) -> int:
@@ -252,6 +260,13 @@ def gpu_step(cache, n_quant0, w, inputs, out, stream, decode_events=None, stage_
             stage_events["flush"].append(ev)
         launches += 1
     kn, vn, q = inputs
+    if FUSED:
+        if decode_events is not None:
+            decode_events[0].record(stream)
+        cache.append_attend(kn, vn, q, out=out, stream=stream, status=False)
+        if decode_events is not None:
+            decode_events[1].record(stream)
+        return launches + 1, cache.c.n_quant + cache.c.n_res
     if stage_events is not None:
         ev = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
         ev[0].record(stream)
@@ -312,7 +327,7 @@ def run_gpu(args, rank, world, local_rank, w: synth.Workload):
                 launches += lz
                 tokens += t
                 n_q2 = cache.c.n_quant
-                bytes_decode += decode_alg_bytes(w, n_q2, t - n_q2)
+                bytes_decode += decode_alg_bytes(w, n_q2, t - n_q2) + (append_bytes(w) if FUSED else 0)
             e1.record(stream)
             stream.synchronize()
         torch.cuda.synchronize(device)
@@ -380,7 +395,7 @@ def run_gpu(args, rank, world, local_rank, w: synth.Workload):
                 "workload": w.name, "batch": w.batch, "q_heads": w.q_heads, "kv_heads": w.kv_heads,
                 "head_dim": w.head_dim, "bits": w.bits, "group_k": w.group, "group_v": w.group,
                 "residual": w.residual, "cached_tokens": f"{n_quant0 + 1}-{n_quant0 + 2 * R} (128-step cycles)",
-                "step": "flush when full + append + decode attention",
+                "step": STEP_NOTE[FUSED],
                 "l2": l2_note(w, n_quant0),
                 "parallelism": f"weak: one independent batch per GPU x {world}",
             },
@@ -476,7 +491,7 @@ def run_reference(args, rank, world, w: synth.Workload):
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": w.name, "batch": w.batch, "q_heads": w.q_heads, "kv_heads": w.kv_heads,
                    "head_dim": w.head_dim, "bits": w.bits, "group_k": w.group, "group_v": w.group,
-                   "residual": w.residual, "step": "flush when full + append + decode attention"},
+                   "residual": w.residual, "step": STEP_NOTE[FUSED]},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -500,9 +515,13 @@ def main():
     ap.add_argument("--group", type=int, choices=[32, 64, 128], default=None, help="override G_k = G_v")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing (profiling runs)")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end loop (profiling runs)")
+    ap.add_argument("--separate-append", action="store_true",
+                    help="append and decode as two launches (kivi_append_token + kivi_decode_attention)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    global FUSED
+    FUSED = not args.separate_append
     w = synth.WORKLOADS[args.workload]
     if args.bits is not None:
         w = w.with_(bits=args.bits)

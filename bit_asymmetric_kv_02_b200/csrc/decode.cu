@@ -576,7 +576,21 @@ struct Decoder {
 
   // ---- K half of a residual unit (16 fp16 rows): logits and softmax weights --------------------
   // q is read in fp16 from global memory (L1-resident: every lane pair reads the same 256 bytes).
-  __device__ void residual_k(const uint8_t* kt, int nvalid, long long head) {
+  // Fused append: if the new token's slot falls in residual unit r (rows 16 r .. 16 r + 15), copy its
+  // row from `src` into the unit's shared-memory copy (which the bulk copy filled from the cache)
+  // and into the cache itself.  Each residual unit belongs to one warp, so the row is written once.
+  __device__ void insert_new_row(uint8_t* buf, int r, long long head, const uint16_t* src, uint16_t* res) {
+    const int row = a.new_slot - r * kResTokens;
+    if (a.new_slot < 0 || row < 0 || row >= kResTokens) return;
+    const uint2 v = __ldg(reinterpret_cast<const uint2*>(src + static_cast<size_t>(head) * kHeadDim) + lane);
+    *reinterpret_cast<uint2*>(buf + row * 256 + 8 * lane) = v;
+    uint16_t* dst = res + (static_cast<size_t>(head) * a.residual + a.new_slot) * kHeadDim;
+    reinterpret_cast<uint2*>(dst)[lane] = v;
+    __syncwarp();
+  }
+
+  __device__ void residual_k(uint8_t* kt, int nvalid, long long head, int r) {
+    insert_new_row(kt, r, head, a.k_new, a.k_res);
     const int t = lane >> 1, hf = lane & 1;  // 2 lanes per token, 64 channels each
 #pragma unroll
     for (int g = 0; g < G; ++g) {
@@ -613,7 +627,8 @@ struct Decoder {
   }
 
   // ---- V half of a residual unit: p . rows -----------------------------------------------------
-  __device__ void residual_v(const uint8_t* vt, int nvalid) {
+  __device__ void residual_v(uint8_t* vt, int nvalid, long long head, int r) {
+    insert_new_row(vt, r, head, a.v_new, a.v_res);
 #pragma unroll
     for (int g = 0; g < G; ++g) {
 #pragma unroll
@@ -803,7 +818,7 @@ struct Decoder {
       if (quant)
         quantized_k(S.buf[hk % kBuffers], head, local, pairs);
       else
-        residual_k(S.buf[hk % kBuffers], nvalid, head);
+        residual_k(S.buf[hk % kBuffers], nvalid, head, local - a.units_q);
       __syncwarp();
       fence_proxy_async_smem();
       // half hk + kBuffers reuses the buffer just consumed: the next unit's V (ring of 3) or K (2)
@@ -817,7 +832,7 @@ struct Decoder {
       if (quant)
         quantized_v(S.buf[(hk + 1) % kBuffers]);
       else
-        residual_v(S.buf[(hk + 1) % kBuffers], nvalid);
+        residual_v(S.buf[(hk + 1) % kBuffers], nvalid, head, local - a.units_q);
       __syncwarp();
       fence_proxy_async_smem();
       // the unit after next's K half (ring of 3) or the next unit's V half (2)

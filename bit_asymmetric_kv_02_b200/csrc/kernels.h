@@ -38,7 +38,7 @@ struct DecodeArgs {
   const uint32_t* k_codes;
   const uint32_t* v_codes;
   const uint16_t *k_scale, *k_zero, *v_scale, *v_zero;
-  const uint16_t *k_res, *v_res;
+  uint16_t *k_res, *v_res;  // written only by a fused append
   const uint16_t* q;
   uint16_t* out;
   float* partials;    // [workers][2][gqa][kPartialStride]
@@ -57,6 +57,11 @@ struct DecodeArgs {
   float qscale;       // softmax scale * log2(e)
   unsigned long long timeout_ns;
   uint32_t debug_extra_tx;  // test hook: bytes a barrier expects beyond the copy (0 normally)
+  // fused append: the token in k_new / v_new ([bh][128] fp16) is residual slot new_slot (< n_res);
+  // new_slot < 0: no append
+  const uint16_t* k_new;
+  const uint16_t* v_new;
+  int new_slot;
 };
 
 constexpr int kPartialStride = 132;  // m, l, Z, pad, o[128]

@@ -249,9 +249,13 @@ size_t kivi_decode_workspace_bytes(const kivi_config* cfg, int32_t num_q_heads) 
          align256(bh * sizeof(int32_t));
 }
 
-int kivi_decode_attention(const kivi_config* cfg, const kivi_cache* cache, const uint16_t* q_dev,
-                          int32_t num_q_heads, float scale, uint16_t* out_dev, void* workspace_dev,
-                          size_t workspace_bytes, int32_t* dev_status, void* stream) {
+namespace {
+
+// Decode attention over `cache` (whose counters already include a fused append's token, which
+// k_new / v_new hold for residual slot new_slot; new_slot < 0: no append).
+int decode_impl(const kivi_config* cfg, const kivi_cache* cache, const uint16_t* q_dev, int32_t num_q_heads,
+                float scale, uint16_t* out_dev, void* workspace_dev, size_t workspace_bytes, int32_t* dev_status,
+                void* stream, const uint16_t* k_new_dev, const uint16_t* v_new_dev, int new_slot) {
   int st = check_cfg(cfg);
   if (st != KIVI_OK) return st;
   if ((st = check_state(cfg, cache)) != KIVI_OK) return st;
@@ -316,9 +320,38 @@ int kivi_decode_attention(const kivi_config* cfg, const kivi_cache* cache, const
     a.timeout_ns = d.timeout_ns;
     a.debug_extra_tx = d.mode == 1 ? 16u : 0u;
   }
+  a.k_new = k_new_dev;
+  a.v_new = v_new_dev;
+  a.new_slot = new_slot;
   if (kivi::launch_decode(a, cfg->bits, plan, static_cast<cudaStream_t>(stream)) != cudaSuccess)
     return KIVI_ERR_CUDA;
   return KIVI_OK;
+}
+
+}  // namespace
+
+int kivi_decode_attention(const kivi_config* cfg, const kivi_cache* cache, const uint16_t* q_dev,
+                          int32_t num_q_heads, float scale, uint16_t* out_dev, void* workspace_dev,
+                          size_t workspace_bytes, int32_t* dev_status, void* stream) {
+  return decode_impl(cfg, cache, q_dev, num_q_heads, scale, out_dev, workspace_dev, workspace_bytes, dev_status,
+                     stream, nullptr, nullptr, -1);
+}
+
+int kivi_append_decode_attention(const kivi_config* cfg, kivi_cache* cache, const uint16_t* k_new_dev,
+                                 const uint16_t* v_new_dev, const uint16_t* q_dev, int32_t num_q_heads, float scale,
+                                 uint16_t* out_dev, void* workspace_dev, size_t workspace_bytes, int32_t* dev_status,
+                                 void* stream) {
+  int st = check_cfg(cfg);
+  if (st != KIVI_OK) return st;
+  if ((st = check_state(cfg, cache)) != KIVI_OK) return st;
+  if (!aligned16(k_new_dev) || !aligned16(v_new_dev) || !cache_ptrs_ok(cache, false)) return KIVI_ERR_INVALID_ARG;
+  if (cache->n_res == cfg->residual) return KIVI_ERR_RESIDUAL_FULL;
+  kivi_cache after = *cache;
+  after.n_res += 1;
+  st = decode_impl(cfg, &after, q_dev, num_q_heads, scale, out_dev, workspace_dev, workspace_bytes, dev_status,
+                   stream, k_new_dev, v_new_dev, cache->n_res);
+  if (st == KIVI_OK) cache->n_res += 1;
+  return st;
 }
 
 int kivi_read_status(const int32_t* dev_status, void* stream) {

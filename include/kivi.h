@@ -159,6 +159,22 @@ int kivi_decode_attention(const kivi_config* cfg, const kivi_cache* cache, const
                           size_t workspace_bytes, int32_t* dev_status, void* stream);
 
 /*
+ * Append and decode attention in one launch: the same results and cache contents as
+ * kivi_append_token(k_new, v_new) followed by kivi_decode_attention(q).  Section 残差バッファ: the
+ * newest token joins the fp16 residual and is attended at once.
+ * The new token's K and V (fp16 [B][H][d], 16-byte aligned) are written into residual slot n_res
+ * by the decode kernel itself: the warp that attends the residual rows of that slot copies the
+ * row into its shared-memory tile and into the cache.  On success n_res is incremented; on any
+ * error the counters are unchanged (a device error may leave the slot written, as with a failed
+ * append).  Arguments and errors are those of the two calls; RESIDUAL_FULL when n_res == R
+ * (flush first).  One kernel launch.
+ */
+int kivi_append_decode_attention(const kivi_config* cfg, kivi_cache* cache, const uint16_t* k_new_dev,
+                                 const uint16_t* v_new_dev, const uint16_t* q_dev, int32_t num_q_heads,
+                                 float scale, uint16_t* out_dev, void* workspace_dev, size_t workspace_bytes,
+                                 int32_t* dev_status, void* stream);
+
+/*
  * Largest scratch kivi_decode_attention_noalloc can use, in bytes (see below).
  */
 #define KIVI_NOALLOC_SCRATCH_BYTES (16u << 20)

@@ -29,7 +29,7 @@ def assert_attention_close(got, want, what=""):
 
 def oracle_head(w: synth.Workload, b: int, h: int, capacity: int, prompt_tokens: int):
     """HeadCache of KV head (b, h) after prefill of `prompt_tokens` synthetic tokens."""
-    hc = O.HeadCache(w.head_dim, w.bits, w.group, w.group, w.residual, capacity)
+    hc = O.HeadCache(w.head_dim, w.bits, w.group, w.gv, w.residual, capacity)
     hc.prefill(synth.prompt_k(w, b, h, prompt_tokens), synth.prompt_v(w, b, h, prompt_tokens))
     return hc
 

@@ -104,6 +104,18 @@ def test_state_errors_before_any_device_work(kivi):
     with pytest.raises(kivi.KiviError) as e:
         kivi.kivi_decode_attention(cfg, cache, fake, 3 * 16, 0.1, fake, fake, 1 << 30, None, 0)
     assert e.value.code == "UNSUPPORTED"
+    cache.n_quant, cache.n_res = 0, 128
+    with pytest.raises(kivi.KiviError) as e:
+        kivi.kivi_append_decode_attention(cfg, cache, fake, fake, fake, 3, 0.1, fake, fake, 1 << 30, None, 0)
+    assert e.value.code == "RESIDUAL_FULL" and cache.n_res == 128
+    cache.n_res = 5
+    with pytest.raises(kivi.KiviError) as e:
+        kivi.kivi_append_decode_attention(cfg, cache, fake + 8, fake, fake, 3, 0.1, fake, fake, 1 << 30, None, 0)
+    assert e.value.code == "INVALID_ARG" and cache.n_res == 5
+    with pytest.raises(kivi.KiviError) as e:
+        kivi.kivi_append_decode_attention(cfg, cache, fake, fake, fake, 4, 0.1, fake, fake, 1 << 30, None, 0)
+    assert e.value.code == "INVALID_ARG" and cache.n_res == 5
+    cache.n_quant, cache.n_res = 0, 1
     with pytest.raises(kivi.KiviError) as e:
         kivi.kivi_quantize_prefill(cfg, cache, fake, fake, 0, 0)
     assert e.value.code == "INVALID_ARG"
