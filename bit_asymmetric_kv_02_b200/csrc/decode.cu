@@ -40,19 +40,22 @@ namespace kivi {
 
 namespace {
 
-// Stream-K workers (warps) per CTA: one CTA per SM.  The warps of one CTA are scheduled fairly;
+// Stream-K workers (warps) per CTA: one CTA per SM.  Two to four queries per KV head run their dot
+// products in passes of two queries, which fits 12 warps per SM (16 spill; 8 leave the FMA-heavy
+// pipe idle more often).  The warps of one CTA are scheduled fairly;
 // warps of separate CTAs on one SM are not (the oldest CTA's warps take precedence and finish
 // early, leaving the SM with fewer warps for the rest of the launch).
 template <int G>
 __host__ __device__ constexpr int warps_per_cta() {
-  return G == 1 ? 16 : 8;  // 16 x 128 registers or 8 x 255 registers
+  return G == 1 ? 16 : (G <= 4 ? 12 : 8);  // 128, 168 and 255 registers
 }
 constexpr int kHalfBytes = 4096;    // one half unit: the K part or the V part of a unit
-// Half-unit buffers per warp: 3 gives the ring K0 V0 K1 | V1 K2 V2 | ..., 2 gives K | V.  One query
-// per KV head uses 2 (measured 1.4% faster than 3 at 16 warps per SM), several queries use 3.
+// Half-unit buffers per warp: 3 gives the ring K0 V0 K1 | V1 K2 V2 | ..., 2 gives K | V.  Up to 4
+// queries per KV head use 2 (1.4% faster than 3 at 16 warps per SM, and 16 warps of 3 would not fit
+// in shared memory); 8 queries per KV head (8 warps per SM) use 3.
 template <int G>
 __host__ __device__ constexpr int ring_buffers() {
-  return G == 1 ? 2 : 3;
+  return G <= 4 ? 2 : 3;
 }
 constexpr int kResTokens = 16;      // tokens per residual unit
 constexpr unsigned kFull = 0xffffffffu;
@@ -132,6 +135,7 @@ struct Decoder {
   static constexpr int TPL = UT / 32;              // tokens per lane (K side)
   static constexpr int ROWS = UT / P;              // V word rows per unit (8)
   static constexpr int kBuffers = ring_buffers<G>();
+  static constexpr int GP = G == 1 ? 1 : 2;        // queries per pass over a unit's codes
 
   const DecodeArgs& a;
   WarpSmem<G>& S;
@@ -142,8 +146,9 @@ struct Decoder {
   // per-head state.  At 2 bits lane (i, k) = (lane / 4, lane % 4) holds channels 16 i + 4 m + k
   // (m = 0..3: byte m of set k of K word i) and lane j < d / G_k holds the q sum of K group j in
   // qsum[g][0]; at 4 bits lane holds channels lane + 32 j and every lane holds all group sums.
-  float qreg[G][4];
+  float qreg[4];        // one query per KV head: its channels of q; several: read from L1 (q_of)
   float qsum[G][4];
+  long long qhead;      // the KV head whose q is loaded
   float m[G], l[G], Z[G], o[G][4];
   // per-block state: the Q limbs in S.qw belong to (head, block) == qkey
   long long qkey;
@@ -206,7 +211,7 @@ struct Decoder {
         for (int j = 0; j < 4; ++j) {
           const int c = 16 * (lane >> 2) + 4 * j + (lane & 3);
           const float v = h2f(__ldg(qp + c)) * a.qscale;
-          qreg[g][j] = v;
+          if (G == 1) qreg[j] = v;
           part += v;
         }
         // the 2^(lg_gk - 2) consecutive lanes of a K group reduce its sum; lane j takes group j's
@@ -215,16 +220,17 @@ struct Decoder {
         qsum[g][0] = __shfl_sync(kFull, part, (lane & (ngk - 1)) * span);
       } else {
 #pragma unroll
+      float qv[4];
       for (int j = 0; j < 4; ++j) {
-        const float v = h2f(__ldg(qp + lane + 32 * j)) * a.qscale;
-        qreg[g][j] = v;
+        qv[j] = h2f(__ldg(qp + lane + 32 * j)) * a.qscale;
+        if (G == 1) qreg[j] = qv[j];
       }
 #pragma unroll
       for (int gi = 0; gi < 4; ++gi) {
         float part = 0.f;
 #pragma unroll
         for (int j = 0; j < 4; ++j)
-          if (((32 * j) >> a.lg_gk) == gi) part += qreg[g][j];
+          if (((32 * j) >> a.lg_gk) == gi) part += qv[j];
         qsum[g][gi] = gi < ngk ? warp_sum(part) : 0.f;
       }
       }
@@ -235,7 +241,18 @@ struct Decoder {
       for (int e = 0; e < 4; ++e) o[g][e] = 0.f;
     }
     qkey = -1;
+    qhead = head;
     __syncwarp();
+  }
+
+  // This lane's q channel j of query g (scaled by scale * log2 e): channel 16 (lane / 4) + 4 j +
+  // lane % 4 at 2 bits, lane + 32 j at 4 bits.  Several queries per KV head read it from L1 (the
+  // block set-up runs once per 128 tokens) to keep registers for a second resident warp per
+  // sub-partition.
+  __device__ __forceinline__ float q_of(int g, int j) const {
+    if (G == 1) return qreg[j];
+    const int c = BITS == 2 ? 16 * (lane >> 2) + 4 * j + (lane & 3) : lane + 32 * j;
+    return h2f(__ldg(a.q + (static_cast<size_t>(qhead) * G + g) * kHeadDim + c)) * a.qscale;
   }
 
   // Bytes 0, 1 and 2 of four integers as three words: word b holds byte b of x_m in byte m.
@@ -259,7 +276,7 @@ struct Decoder {
     for (int g = 0; g < G; ++g) {
       float qv[4];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) qv[j] = qreg[g][j] * s;
+      for (int j = 0; j < 4; ++j) qv[j] = q_of(g, j) * s;
       const float mabs = warp_max(fmaxf(fmaxf(fabsf(qv[0]), fabsf(qv[1])), fmaxf(fabsf(qv[2]), fabsf(qv[3]))));
       // |Q| <= 2^23 - 61: the margin keeps the rounded largest element below 2^23, where the
       // signed top limb would wrap (rcp and the product add at most 3 * 2^-22 relative)
@@ -300,7 +317,7 @@ struct Decoder {
       for (int j = 0; j < 4; ++j) {
         const int gi = (32 * j) >> a.lg_gk;
         const float s = h2f(static_cast<uint16_t>(__shfl_sync(kFull, pairs, gi) & 0xFFFFu));
-        qv[j] = qreg[g][j] * s;
+        qv[j] = q_of(g, j) * s;
         mabs = fmaxf(mabs, fabsf(qv[j]));
       }
       mabs = warp_max(mabs);
@@ -333,9 +350,10 @@ struct Decoder {
 
   // ---- A6 over the K codes of a unit: integer dot products of TPL tokens per lane, for every
   // query of the KV head (each code word is unpacked once) -----------------------------------------
-  __device__ void k_dot(const uint8_t* kt, int (&al)[G][TPL], int (&am)[G][TPL], int (&ah)[G][TPL]) const {
+  // Queries g0 .. g0 + GP - 1 (the accumulators of one pass).
+  __device__ void k_dot(const uint8_t* kt, int g0, int (&al)[GP][TPL], int (&am)[GP][TPL], int (&ah)[GP][TPL]) const {
 #pragma unroll
-    for (int g = 0; g < G; ++g)
+    for (int g = 0; g < GP; ++g)
 #pragma unroll
       for (int j = 0; j < TPL; ++j) al[g][j] = am[g][j] = ah[g][j] = 0;
     if (BITS == 2) {
@@ -352,8 +370,8 @@ struct Decoder {
 #pragma unroll
           for (int j = 0; j < TPL; ++j) masks2(comp(kw[j], ii), mk[j]);
 #pragma unroll
-          for (int g = 0; g < G; ++g) {
-            const uint4* qrow = S.qw[g] + 12 * hh + ii * 3;
+          for (int g = 0; g < GP; ++g) {
+            const uint4* qrow = S.qw[g0 + g] + 12 * hh + ii * 3;
             const uint4 QL = qrow[0], QM = qrow[1], QH = qrow[2];
 #pragma unroll
             for (int k = 0; k < 4; ++k)
@@ -376,8 +394,8 @@ struct Decoder {
 #pragma unroll
           for (int j = 0; j < TPL; ++j) masks4(comp(kw[j], ii), mk[j]);
 #pragma unroll
-          for (int g = 0; g < G; ++g) {
-            const uint2* qrow = reinterpret_cast<const uint2*>(S.qw[g]) + 12 * cq + ii * 3;
+          for (int g = 0; g < GP; ++g) {
+            const uint2* qrow = reinterpret_cast<const uint2*>(S.qw[g0 + g]) + 12 * cq + ii * 3;
             const uint2 QL = qrow[0], QM = qrow[1], QH = qrow[2];
 #pragma unroll
             for (int j = 0; j < TPL; ++j) dot_set(mk[j][0], QL.x, QM.x, QH.x, al[g][j], am[g][j], ah[g][j], true);
@@ -409,16 +427,17 @@ struct Decoder {
   // needs one warp reduction instead of two; the bound sums over the units to at most smax * l,
   // the same error bound as the exact maximum.  A unit whose weights are all below 2^-64 of the
   // running maximum contributes its z-terms only.
-  __device__ void softmax2(const VScales& vs, const int (&al)[G][TPL], const int (&am)[G][TPL],
-                           const int (&ah)[G][TPL]) {
+  __device__ void softmax2(const VScales& vs, int g0, const int (&al)[GP][TPL], const int (&am)[GP][TPL],
+                           const int (&ah)[GP][TPL]) {
     const float sv = vs.sv, zv = vs.zv;
     const float set_scale = (lane & 1) ? 0.25f : 1.f;
     uint32_t* pw = reinterpret_cast<uint32_t*>(S.pw);
 #pragma unroll
-    for (int g = 0; g < G; ++g) {
+    for (int gg = 0; gg < GP; ++gg) {
+      const int g = g0 + gg;
       float lg[TPL];
 #pragma unroll
-      for (int j = 0; j < TPL; ++j) lg[j] = fmaf(combine_limbs(ah[g][j], am[g][j], al[g][j]), invq[g], cblk[g]);
+      for (int j = 0; j < TPL; ++j) lg[j] = fmaf(combine_limbs(ah[gg][j], am[gg][j], al[gg][j]), invq[g], cblk[g]);
       const float mu = warp_max(fmaxf(fmaxf(lg[0], lg[1]), fmaxf(lg[2], lg[3])));
       const float m_new = fmaxf(m[g], mu);
       const float alpha = fast_exp2(m[g] - m_new);
@@ -454,26 +473,34 @@ struct Decoder {
       build_q(pairs);
       qkey = key;
     }
-    int al[G][TPL], am[G][TPL], ah[G][TPL];
     if constexpr (BITS == 2) {
       const VScales vs = v_scales2(pairs);  // independent of the dot products: issued first
-      k_dot(kt, al, am, ah);
-      softmax2(vs, al, am, ah);
+#pragma unroll
+      for (int g0 = 0; g0 < G; g0 += GP) {
+        int al[GP][TPL], am[GP][TPL], ah[GP][TPL];
+        k_dot(kt, g0, al, am, ah);
+        softmax2(vs, g0, al, am, ah);
+      }
     } else {
-      k_dot(kt, al, am, ah);
-      softmax4(pairs, al, am, ah);
+#pragma unroll
+      for (int g0 = 0; g0 < G; g0 += GP) {
+        int al[GP][TPL], am[GP][TPL], ah[GP][TPL];
+        k_dot(kt, g0, al, am, ah);
+        softmax4(pairs, g0, al, am, ah);
+      }
     }
   }
 
   // 4 bits: lane holds tokens lane + 32 j; each byte of a P limb word is stored on its own.
-  __device__ void softmax4(uint32_t pairs, const int (&al)[G][TPL], const int (&am)[G][TPL],
-                           const int (&ah)[G][TPL]) {
+  __device__ void softmax4(uint32_t pairs, int g0, const int (&al)[GP][TPL], const int (&am)[GP][TPL],
+                           const int (&ah)[GP][TPL]) {
 #pragma unroll
-    for (int g = 0; g < G; ++g) {
+    for (int gg = 0; gg < GP; ++gg) {
+      const int g = g0 + gg;
       float lg[TPL], mu = -INFINITY;
 #pragma unroll
       for (int j = 0; j < TPL; ++j) {
-        lg[j] = fmaf(combine_limbs(ah[g][j], am[g][j], al[g][j]), invq[g], cblk[g]);
+        lg[j] = fmaf(combine_limbs(ah[gg][j], am[gg][j], al[gg][j]), invq[g], cblk[g]);
         mu = fmaxf(mu, lg[j]);
       }
       mu = warp_max(mu);
@@ -522,53 +549,58 @@ struct Decoder {
       __syncwarp();
       return;
     }
-    int vl[G][4], vm[G][4], vh[G][4];
 #pragma unroll
-    for (int g = 0; g < G; ++g)
+    for (int g0 = 0; g0 < G; g0 += GP) {  // queries g0 .. g0 + GP - 1 per pass over the codes
+      int vl[GP][4], vm[GP][4], vh[GP][4];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) vl[g][e] = vm[g][e] = vh[g][e] = 0;
+      for (int g = 0; g < GP; ++g)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) vl[g][e] = vm[g][e] = vh[g][e] = 0;
 #pragma unroll 2
-    for (int r = 0; r < ROWS; ++r) {
-      const uint4 vw = *reinterpret_cast<const uint4*>(vt + r * 512 + 16 * lane);
-      if (BITS == 2) {
-        uint32_t mv4[4][4];
+      for (int r = 0; r < ROWS; ++r) {
+        const uint4 vw = *reinterpret_cast<const uint4*>(vt + r * 512 + 16 * lane);
+        if (BITS == 2) {
+          uint32_t mv4[4][4];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) masks2(comp(vw, e), mv4[e]);
+          for (int e = 0; e < 4; ++e) masks2(comp(vw, e), mv4[e]);
 #pragma unroll
-        for (int g = 0; g < G; ++g) {
-          if (G > 1 && !hasv_[g]) continue;
-          const uint4 PL = S.pw[g][r * 3 + 0], PM = S.pw[g][r * 3 + 1], PH = S.pw[g][r * 3 + 2];
+          for (int g = 0; g < GP; ++g) {
+            if (G > 1 && !hasv_[g0 + g]) continue;
+            const uint4* pr = S.pw[g0 + g] + r * 3;
+            const uint4 PL = pr[0], PM = pr[1], PH = pr[2];
 #pragma unroll
-          for (int k = 0; k < 4; ++k)  // set-major: 12 independent accumulators between reuses
+            for (int k = 0; k < 4; ++k)  // set-major: 12 independent accumulators between reuses
 #pragma unroll
-            for (int e = 0; e < 4; ++e)
-              dot_set(mv4[e][k], comp(PL, k), comp(PM, k), comp(PH, k), vl[g][e], vm[g][e], vh[g][e], false);
-        }
-      } else {
-        uint32_t mv4[4][2];
+              for (int e = 0; e < 4; ++e)
+                dot_set(mv4[e][k], comp(PL, k), comp(PM, k), comp(PH, k), vl[g][e], vm[g][e], vh[g][e], false);
+          }
+        } else {
+          uint32_t mv4[4][2];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) masks4(comp(vw, e), mv4[e]);
+          for (int e = 0; e < 4; ++e) masks4(comp(vw, e), mv4[e]);
 #pragma unroll
-        for (int g = 0; g < G; ++g) {
-          if (G > 1 && !hasv_[g]) continue;
-          const uint2* pw2 = reinterpret_cast<const uint2*>(S.pw[g]);
-          const uint2 PL = pw2[r * 3 + 0], PM = pw2[r * 3 + 1], PH = pw2[r * 3 + 2];
+          for (int g = 0; g < GP; ++g) {
+            if (G > 1 && !hasv_[g0 + g]) continue;
+            const uint2* pw2 = reinterpret_cast<const uint2*>(S.pw[g0 + g]);
+            const uint2 PL = pw2[r * 3 + 0], PM = pw2[r * 3 + 1], PH = pw2[r * 3 + 2];
 #pragma unroll
-          for (int e = 0; e < 4; ++e) dot_set(mv4[e][0], PL.x, PM.x, PH.x, vl[g][e], vm[g][e], vh[g][e], false);
+            for (int e = 0; e < 4; ++e) dot_set(mv4[e][0], PL.x, PM.x, PH.x, vl[g][e], vm[g][e], vh[g][e], false);
 #pragma unroll
-          for (int e = 0; e < 4; ++e) dot_set(mv4[e][1], PL.y, PM.y, PH.y, vl[g][e], vm[g][e], vh[g][e], false);
+            for (int e = 0; e < 4; ++e) dot_set(mv4[e][1], PL.y, PM.y, PH.y, vl[g][e], vm[g][e], vh[g][e], false);
+          }
         }
       }
-    }
 #pragma unroll
-    for (int g = 0; g < G; ++g) {
-      if (hasv_[g]) {
+      for (int gg = 0; gg < GP; ++gg) {
+        const int g = g0 + gg;
+        if (hasv_[g]) {
 #pragma unroll
-        for (int e = 0; e < 4; ++e)
-          o[g][e] = fmaf(o[g][e], alpha_[g], combine_limbs(vh[g][e], vm[g][e], vl[g][e]) * invv_[g]);
-      } else {
+          for (int e = 0; e < 4; ++e)
+            o[g][e] = fmaf(o[g][e], alpha_[g], combine_limbs(vh[gg][e], vm[gg][e], vl[gg][e]) * invv_[g]);
+        } else {
 #pragma unroll
-        for (int e = 0; e < 4; ++e) o[g][e] *= alpha_[g];
+          for (int e = 0; e < 4; ++e) o[g][e] *= alpha_[g];
+        }
       }
     }
     __syncwarp();  // P limbs are rewritten by the next unit
