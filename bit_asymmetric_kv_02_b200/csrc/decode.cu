@@ -8,14 +8,16 @@
 // 8 KB "units": quantized units of UT tokens (UT = 128 at 2 bits, 64 at 4 bits; 4 KB of K codes +
 // 4 KB of V codes) followed by residual units of 16 fp16 tokens (4 KB K + 4 KB V).  The global
 // unit sequence is cut into one contiguous range per warp, so the load is balanced to one unit
-// whatever the batch, head count or context length.  Each warp streams its range as half units
-// K0 V0 K1 V1 ... through a ring of three 4 KB shared-memory buffers filled by 1-D TMA bulk copies
-// (cp.async.bulk, no multicast) and completed on mbarriers: half h uses buffer h % 3 and is
-// reissued as soon as half h - 3 is consumed, which keeps one unit in flight with 12 KB per warp
-// (16 resident warps per SM).  Every wait is bounded and reports KIVI_ERR_DEVICE_TIMEOUT.
-// A warp whose range covers a whole head writes the output directly; a head split over several
-// warps is merged (log-sum-exp) by the warp that arrives last on the head's atomic ticket, which
-// then resets the ticket to zero.  No warp ever waits for another.
+// whatever the batch, head count or context length.  The grid is one CTA per SM (16, 12 or 8 warps
+// by queries per KV head).  Each warp streams its range as half units K0 V0 K1 V1 ... through a
+// ring of two (up to 4 queries per KV head) or three 4 KB shared-memory buffers filled by 1-D TMA
+// bulk copies (cp.async.bulk, no multicast) and completed on mbarriers: half h uses buffer h % n
+// and is reissued as soon as half h - n is consumed.  Every wait is bounded and reports
+// KIVI_ERR_DEVICE_TIMEOUT.  A warp whose range covers a whole head writes the output directly; a
+// head split over several warps is merged (log-sum-exp) by the warp that arrives last on the head's
+// atomic ticket, which then resets the ticket to zero.  No warp ever waits for another.
+// A fused append (kivi_append_decode_attention) hands the new token's rows to the warp that owns
+// the residual unit holding its slot; that warp patches its shared-memory copy and the cache.
 //
 // Arithmetic (CUDA cores, no tensor cores: one query row per head is a matrix-vector product).
 //   A6  logit_t = sum_c q_c (s_g code + z_g) = sum_c (q_c s_g) code_tc + sum_g z_g sum_{c in g} q_c.
@@ -23,10 +25,12 @@
 //       three byte limbs (kept while the warp stays in the same block); the codes are unpacked to
 //       bytes with one shift and masks, and dp4a forms the byte dot products exactly in int32.
 //       The block constant sum_g z_g q_g is added in fp32.
-//   A8  online softmax in base 2 (q pre-scaled by scale*log2 e), warp-shuffle max, lane-local sums.
+//   A8  online softmax in base 2 (q pre-scaled by scale*log2 e), redux.sync warp maxima, lane-local
+//       sums.
 //   A9  o_c = sum_t (p_t s_g(t)) code_tc + sum_t p_t z_g(t): (p_t s_g(t)) is turned into 24-bit
-//       unsigned fixed point relative to the unit's largest value and dotted with the V codes by
-//       dp4a; the z term is the same for every channel and is kept as one scalar.
+//       unsigned fixed point relative to a bound of the unit's largest value (at 2 bits: the
+//       unit's largest weight times its largest V scale; at 4 bits: the exact maximum) and dotted
+//       with the V codes by dp4a; the z term is the same for every channel and is one scalar.
 //   A7/A9 residual rows: fp32 FMAs on the fp16 values.
 //   A10 merge of (m, l, Z, o) states: o / l with o += Z.
 // 24-bit limbs keep every product relative error below 2^-21, the integer sums are exact, and the
@@ -219,8 +223,8 @@ struct Decoder {
         for (int off = 1; off < span; off <<= 1) part += __shfl_xor_sync(kFull, part, off);
         qsum[g][0] = __shfl_sync(kFull, part, (lane & (ngk - 1)) * span);
       } else {
-#pragma unroll
       float qv[4];
+#pragma unroll
       for (int j = 0; j < 4; ++j) {
         qv[j] = h2f(__ldg(qp + lane + 32 * j)) * a.qscale;
         if (G == 1) qreg[j] = qv[j];
