@@ -31,6 +31,10 @@ CASES = [
     synth.TINY.with_(name="fused_2bit", batch=2, q_heads=3, kv_heads=3, tokens=300, seed=31),
     synth.TINY.with_(name="fused_4bit_gqa2", batch=2, q_heads=4, kv_heads=2, tokens=250, bits=4, seed=32),
     synth.TINY.with_(name="fused_2bit_gqa4_g128", batch=1, q_heads=8, kv_heads=2, tokens=700, group=128, seed=33),
+    synth.TINY.with_(name="fused_2bit_R256_gv64", batch=1, q_heads=2, kv_heads=2, tokens=600, group_v=64, residual=256,
+                     seed=36),
+    synth.TINY.with_(name="fused_4bit_R512_gk64", batch=1, q_heads=2, kv_heads=1, tokens=900, bits=4, group=64,
+                     residual=512, seed=37),
 ]
 
 
@@ -72,7 +76,7 @@ def test_fused_equals_two_calls_and_oracle(w):
         assert (fused.n_quant, fused.n_res) == (two.n_quant, two.n_res)
         a, f = o_two.cpu().numpy(), o_fused.cpu().numpy()
         assert np.array_equal(a.view(np.uint16), f.view(np.uint16)), f"step {s}: fused output differs"
-        if s in (1, 2, 15, 16, 17, 84, 85, 128, 129, steps) or s % 37 == 0:
+        if s in (1, 2, 15, 16, 17, 84, 85, 128, 129, steps) or s % 37 == 0 or two.n_res in (1, w.residual):
             for (b, h), hc in ref.items():
                 gc.assert_attention_close(f[b, h * g:(h + 1) * g], hc.attend(q[b, h * g:(h + 1) * g], gc.default_scale()),
                                           f"{w.name} step {s} head {(b, h)}")
