@@ -265,6 +265,35 @@ class HeadCache:
         self.k_res = k[n_quant:].copy()
         self.v_res = v[n_quant:].copy()
 
+    def prefill_prefix_k(self, k, v):
+        """Prefill under the other reading of section Per-Channel量子化, in which one K group spans
+        every quantized token of the prompt (the channel group over tokens [0, n_quant)) instead of
+        one R-token block.  The residual split, the V groups (g_v consecutive tokens, section
+        Per-Token量子化) and the counters are those of prefill.  The shared K (s, z) is kept once per
+        R-token block, so dequantization and later flushes use the same layout as prefill."""
+        k = np.asarray(k, np.float16)
+        v = np.asarray(v, np.float16)
+        T = k.shape[0]
+        if T < 1:
+            raise OracleError("INVALID_ARG", "empty prompt")
+        n_res = (T - 1) % self.R + 1
+        n_quant = T - n_res
+        if n_quant > self.capacity:
+            raise OracleError("CAPACITY", f"{n_quant} > {self.capacity}")
+        self.__init__(self.d, self.bits, self.gk, self.gv, self.R, self.capacity)
+        if n_quant:
+            kc, ks, kz = quantize_k_block(k[:n_quant], self.gk, self.bits)
+            self.k_codes = kc
+            self.k_s = np.tile(ks[None, :], (n_quant // self.R, 1))
+            self.k_z = np.tile(kz[None, :], (n_quant // self.R, 1))
+            for j in range(n_quant // self.R):
+                vc, vs, vz = quantize_v_block(v[j * self.R:(j + 1) * self.R], self.gv, self.bits)
+                self.v_codes = np.concatenate([self.v_codes, vc])
+                self.v_s = np.concatenate([self.v_s, vs])
+                self.v_z = np.concatenate([self.v_z, vz])
+        self.k_res = k[n_quant:].copy()
+        self.v_res = v[n_quant:].copy()
+
     def append(self, k_new, v_new):
         """Writes the newest token into the fp16 residual (section 残差バッファ)."""
         if self.n_res == self.R:

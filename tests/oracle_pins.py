@@ -270,6 +270,51 @@ def check_prefill_equals_streaming(O, bits, group):
         assert np.array_equal(np.asarray(pa[key]).view(np.uint8), np.asarray(pb[key]).view(np.uint8)), key
 
 
+def check_prefix_k_groups(O, bits, group):
+    """The prefix-K prefill (section Per-Channel量子化 read with one K group over every quantized
+    token of the prompt): brute force over the whole prefix with exact rationals; V, residual and
+    counters equal those of prefill; a single quantized block equals prefill exactly; a flush after
+    it quantizes the next block on its own."""
+    rng = np.random.default_rng(91 + bits + group)
+    R, d, L = 128, 128, 2 ** bits - 1
+    T = 3 * R + 5
+    k = (rng.standard_normal((T, d)) * np.exp2(rng.integers(-2, 3, (1, d)))).astype(np.float16)
+    k[200:260, 7] *= np.float16(11)                 # an outlier run inside one block only
+    k[3 * R + 2, :] *= np.float16(20)               # a large residual row: outside every K group
+    v = rng.standard_normal((T, d)).astype(np.float16)
+    h = O.HeadCache(d, bits, group, group, R, 8 * R)
+    h.prefill_prefix_k(k, v)
+    n_q = 3 * R
+    assert (h.n_quant, h.n_res) == (n_q, 5) and h.k_s.shape == (3, d // group)
+    for g in range(d // group):
+        vals = [_fr(k[t, c]) for t in range(n_q) for c in range(g * group, (g + 1) * group)]
+        lo, hi = min(vals), max(vals)
+        s = fp16_round_exact((hi - lo) / L)
+        for blk in range(3):
+            assert Fraction(float(h.k_s[blk, g])) == s and Fraction(float(h.k_z[blk, g])) == lo, (g, blk)
+        for t in range(0, n_q, 11):
+            for c in range(g * group, (g + 1) * group, 5):
+                assert h.k_codes[t, c] == code_exact(_fr(k[t, c]), s, lo, bits), (t, c)
+    ref = O.HeadCache(d, bits, group, group, R, 8 * R)
+    ref.prefill(k, v)
+    for key in ("v_codes", "v_s", "v_z", "k_res", "v_res"):
+        assert np.array_equal(getattr(h, key), getattr(ref, key)), key
+    # the outlier run lies in block 1 only: block-local K scales differ, the prefix ones do not
+    g7 = 7 // group
+    assert ref.k_s[0, g7] != ref.k_s[1, g7] and h.k_s[0, g7] == h.k_s[1, g7]
+    one = O.HeadCache(d, bits, group, group, R, 8 * R)
+    one.prefill_prefix_k(k[:R + 9], v[:R + 9])
+    ref1 = O.HeadCache(d, bits, group, group, R, 8 * R)
+    ref1.prefill(k[:R + 9], v[:R + 9])
+    for key, want in ref1.packed().items():
+        assert np.array_equal(np.asarray(one.packed()[key]).view(np.uint8), np.asarray(want).view(np.uint8)), key
+    for t in range(T, T + R - 5):
+        h.append(k[t % T], v[t % T])
+    h.flush()
+    kc, ks, kz = O.quantize_k_block(np.concatenate([k[n_q:], k[: R - 5]]), group, bits)
+    assert np.array_equal(h.k_s[3], ks) and np.array_equal(h.k_codes[n_q:], kc)
+
+
 def check_errors(O):
     h = _head(O, cap=128)
     k = np.zeros((128, 128), np.float16)

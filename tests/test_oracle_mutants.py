@@ -138,3 +138,29 @@ def test_some_pin_catches_mutant(mutant, monkeypatch):
             caught.append(type(e).__name__)
             break
     assert caught, f"no pin catches the planted mistake {mutant}"
+
+
+def _prefix_k_per_block(self, k, v):                 # K groups per R-token block, as in prefill
+    return O.HeadCache.prefill(self, k, v)
+
+
+def _prefix_k_whole_prompt(self, k, v):              # K groups over the residual tokens too
+    k = np.asarray(k, np.float16)
+    T = k.shape[0]
+    n_q = T - ((T - 1) % self.R + 1)
+    _real_prefix(self, k, v)
+    if n_q:
+        kc, ks, kz = O.quantize_k_block(k, self.gk, self.bits)
+        self.k_codes = kc[:n_q]
+        self.k_s = np.tile(ks[None, :], (n_q // self.R, 1))
+        self.k_z = np.tile(kz[None, :], (n_q // self.R, 1))
+
+
+_real_prefix = O.HeadCache.prefill_prefix_k
+
+
+@pytest.mark.parametrize("mutant", [_prefix_k_per_block, _prefix_k_whole_prompt], ids=["per_block", "whole_prompt"])
+def test_prefix_pin_catches_mutant(mutant, monkeypatch):
+    monkeypatch.setattr(O.HeadCache, "prefill_prefix_k", mutant)
+    with pytest.raises(AssertionError):
+        pins.check_prefix_k_groups(O, 2, 32)

@@ -66,3 +66,8 @@ def test_attention_closed_forms():
 @pytest.mark.parametrize("bits,group", [(2, 32), (4, 128)])
 def test_attention_bruteforce_from_packed_words(bits, group):
     pins.check_attention_bruteforce(O, bits, group)
+
+
+@pytest.mark.parametrize("bits,group", [(2, 32), (4, 64), (2, 128)])
+def test_prefix_k_groups(bits, group):
+    pins.check_prefix_k_groups(O, bits, group)
