@@ -25,6 +25,7 @@ struct QuantizeArgs {
   int res_tokens;  // tokens copied into the residual (0: none)
   int residual, capacity, group_k, group_v;
   int lg_gk, lg_gv;  // log2(group_k), log2(group_v): set by launch_quantize_blocks
+  int k_given;       // 1: the K (s, z) of each block are already in k_scale / k_zero (prefix groups)
 };
 
 struct AppendArgs {
@@ -67,6 +68,9 @@ struct DecodeArgs {
 constexpr int kPartialStride = 132;  // m, l, Z, pad, o[128]
 
 cudaError_t launch_quantize_blocks(const QuantizeArgs& a, int bits, cudaStream_t stream);
+// K (s, z) of every channel group over all a.nblocks * R source tokens, stored in every
+// destination block's slot (the prefix-group prefill); then launch_quantize_blocks with k_given.
+cudaError_t launch_k_prefix_extremes(const QuantizeArgs& a, int bits, cudaStream_t stream);
 cudaError_t launch_append(const AppendArgs& a, cudaStream_t stream);
 
 // Decode launch plan: warps per CTA, CTAs, dynamic shared memory.

@@ -143,8 +143,10 @@ int kivi_cache_sizes(const kivi_config* cfg, size_t* out) {
   return KIVI_OK;
 }
 
-int kivi_quantize_prefill(const kivi_config* cfg, kivi_cache* cache, const uint16_t* k_dev, const uint16_t* v_dev,
-                          int32_t num_tokens, void* stream) {
+namespace {
+
+int prefill_impl(const kivi_config* cfg, kivi_cache* cache, const uint16_t* k_dev, const uint16_t* v_dev,
+                 int32_t num_tokens, void* stream, bool prefix_k) {
   int st = check_cfg(cfg);
   if (st != KIVI_OK) return st;
   if (cache == nullptr || num_tokens < 1 || !aligned16(k_dev) || !aligned16(v_dev)) return KIVI_ERR_INVALID_ARG;
@@ -175,11 +177,28 @@ int kivi_quantize_prefill(const kivi_config* cfg, kivi_cache* cache, const uint1
   a.capacity = cfg->capacity;
   a.group_k = cfg->group_k;
   a.group_v = cfg->group_v;
+  if (prefix_k && a.nblocks > 0) {
+    if (kivi::launch_k_prefix_extremes(a, cfg->bits, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+      return KIVI_ERR_CUDA;
+    a.k_given = 1;
+  }
   if (kivi::launch_quantize_blocks(a, cfg->bits, static_cast<cudaStream_t>(stream)) != cudaSuccess)
     return KIVI_ERR_CUDA;
   cache->n_quant = n_quant;
   cache->n_res = n_res;
   return KIVI_OK;
+}
+
+}  // namespace
+
+int kivi_quantize_prefill(const kivi_config* cfg, kivi_cache* cache, const uint16_t* k_dev, const uint16_t* v_dev,
+                          int32_t num_tokens, void* stream) {
+  return prefill_impl(cfg, cache, k_dev, v_dev, num_tokens, stream, false);
+}
+
+int kivi_quantize_prefill_prefix_k(const kivi_config* cfg, kivi_cache* cache, const uint16_t* k_dev,
+                                   const uint16_t* v_dev, int32_t num_tokens, void* stream) {
+  return prefill_impl(cfg, cache, k_dev, v_dev, num_tokens, stream, true);
 }
 
 int kivi_append_token(const kivi_config* cfg, kivi_cache* cache, const uint16_t* k_new_dev,

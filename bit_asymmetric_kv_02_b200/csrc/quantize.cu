@@ -57,6 +57,17 @@ __device__ __forceinline__ GroupParams make_group(float lo, float hi, int levels
   return g;
 }
 
+// Group parameters from a stored (s, z) pair (the prefix-group prefill stores them first).
+__device__ __forceinline__ GroupParams group_from_stored(uint16_t s_bits, uint16_t z_bits) {
+  GroupParams g;
+  g.s_bits = s_bits;
+  g.z_bits = z_bits;
+  g.zf = h2f(z_bits);
+  const float s = h2f(s_bits);
+  g.inv_s = s > 0.f ? 1.0f / s : 0.f;
+  return g;
+}
+
 // Q of one element (section 量子化アルゴリズム, Q equation) with the stored fp16 s and z, taken
 // exactly: the fp64 quotient decides (used near ties only).
 __device__ __noinline__ uint32_t quantize_exact(float x, const GroupParams& g, int levels) {
@@ -87,7 +98,7 @@ __device__ __forceinline__ void quantize_pair(uint32_t hx2, const GroupParams& g
 // ---------------------------------------------------------------------------------------------
 template <int BITS>
 __device__ void quantize_k_block(const uint16_t* __restrict__ src, int R, int gk, uint32_t* __restrict__ codes,
-                                 uint16_t* __restrict__ scale, uint16_t* __restrict__ zero) {
+                                 uint16_t* __restrict__ scale, uint16_t* __restrict__ zero, bool given) {
   constexpr int P = 32 / BITS;
   constexpr int L = (1 << BITS) - 1;
   __shared__ float red_lo[kThreads / 32][kChunks], red_hi[kThreads / 32][kChunks];
@@ -95,37 +106,40 @@ __device__ void quantize_k_block(const uint16_t* __restrict__ src, int R, int gk
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int chunk = tid % kChunks;
   const uint4* s4 = reinterpret_cast<const uint4*>(src);
-
-  float lo = INFINITY, hi = -INFINITY;
-  for (int t = tid / kChunks; t < R; t += kThreads / kChunks) minmax8(__ldg(s4 + t * kChunks + chunk), lo, hi);
-  lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, 16));
-  hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, 16));
-  if (lane < kChunks) {
-    red_lo[warp][lane] = lo;
-    red_hi[warp][lane] = hi;
-  }
-  __syncthreads();
-  if (warp == 0) {
-    // lanes 0..15: one chunk each, then combine the chunks of a group (gk/8 consecutive chunks)
-    float a = INFINITY, b = -INFINITY;
+  if (given) {  // prefix groups: (s, z) already stored for this block
+    if (tid < kHeadDim / gk) grp[tid] = group_from_stored(scale[tid], zero[tid]);
+  } else {
+    float lo = INFINITY, hi = -INFINITY;
+    for (int t = tid / kChunks; t < R; t += kThreads / kChunks) minmax8(__ldg(s4 + t * kChunks + chunk), lo, hi);
+    lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, 16));
+    hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, 16));
     if (lane < kChunks) {
+      red_lo[warp][lane] = lo;
+      red_hi[warp][lane] = hi;
+    }
+    __syncthreads();
+    if (warp == 0) {
+      // lanes 0..15: one chunk each, then combine the chunks of a group (gk/8 consecutive chunks)
+      float a = INFINITY, b = -INFINITY;
+      if (lane < kChunks) {
 #pragma unroll
-      for (int w = 0; w < kThreads / 32; ++w) {
-        a = fminf(a, red_lo[w][lane]);
-        b = fmaxf(b, red_hi[w][lane]);
+        for (int w = 0; w < kThreads / 32; ++w) {
+          a = fminf(a, red_lo[w][lane]);
+          b = fmaxf(b, red_hi[w][lane]);
+        }
       }
-    }
-    const int cpg = gk / 8;  // chunks per group: 4, 8 or 16
-    for (int off = 1; off < cpg; off <<= 1) {
-      a = fminf(a, __shfl_xor_sync(0xffffffffu, a, off));
-      b = fmaxf(b, __shfl_xor_sync(0xffffffffu, b, off));
-    }
-    if (lane < kChunks && lane % cpg == 0) {
-      const int g = lane / cpg;
-      GroupParams gp = make_group(a, b, L);
-      grp[g] = gp;
-      scale[g] = gp.s_bits;
-      zero[g] = gp.z_bits;
+      const int cpg = gk / 8;  // chunks per group: 4, 8 or 16
+      for (int off = 1; off < cpg; off <<= 1) {
+        a = fminf(a, __shfl_xor_sync(0xffffffffu, a, off));
+        b = fmaxf(b, __shfl_xor_sync(0xffffffffu, b, off));
+      }
+      if (lane < kChunks && lane % cpg == 0) {
+        const int g = lane / cpg;
+        GroupParams gp = make_group(a, b, L);
+        grp[g] = gp;
+        scale[g] = gp.s_bits;
+        zero[g] = gp.z_bits;
+      }
     }
   }
   __syncthreads();
@@ -350,7 +364,7 @@ __device__ __forceinline__ uint32_t quantize_row8(const uint4& v, const GroupPar
 
 template <int BITS>
 __device__ void quantize_k_tiles(const uint16_t* __restrict__ src, int R, int lg_gk, uint32_t* __restrict__ codes,
-                                 uint16_t* __restrict__ scale, uint16_t* __restrict__ zero) {
+                                 uint16_t* __restrict__ scale, uint16_t* __restrict__ zero, bool given) {
   constexpr int L = (1 << BITS) - 1;
   __shared__ __half2 red[1024 / 32][kHeadDim / 32];
   __shared__ GroupParams grp[kHeadDim / 32];
@@ -365,21 +379,28 @@ __device__ void quantize_k_tiles(const uint16_t* __restrict__ src, int R, int lg
   // K group of chunk c: chunks [cpg * g, cpg * (g + 1)), cpg = g_k / 8; the warp's two token
   // groups (lanes < 16 and >= 16) hold the same chunks
   const int lg_cpg = lg_gk - 3, ngk = kHeadDim >> lg_gk;
-  __half2 m = tile_min_negmax(x);
-  for (int off = 1; off < (1 << lg_cpg); off <<= 1) m = __hmin2(m, shfl_xor_h2(m, off));
-  m = __hmin2(m, shfl_xor_h2(m, 16));
-  if (lane < 16 && (c & ((1 << lg_cpg) - 1)) == 0) red[warp][c >> lg_cpg] = m;
-  __syncthreads();
+  if (!given) {
+    __half2 m = tile_min_negmax(x);
+    for (int off = 1; off < (1 << lg_cpg); off <<= 1) m = __hmin2(m, shfl_xor_h2(m, off));
+    m = __hmin2(m, shfl_xor_h2(m, 16));
+    if (lane < 16 && (c & ((1 << lg_cpg) - 1)) == 0) red[warp][c >> lg_cpg] = m;
+    __syncthreads();
+  }
   if (tid < ngk) {
-    __half2 t = red[0][tid];
-    for (int w = 1; w < nwarps; ++w) t = __hmin2(t, red[w][tid]);
-    const GroupParams gp = group_from_pair(t, L);
+    GroupParams gp;
+    if (given) {  // prefix groups: (s, z) already stored for this block
+      gp = group_from_stored(scale[tid], zero[tid]);
+    } else {
+      __half2 t = red[0][tid];
+      for (int w = 1; w < nwarps; ++w) t = __hmin2(t, red[w][tid]);
+      gp = group_from_pair(t, L);
+      scale[tid] = gp.s_bits;
+      zero[tid] = gp.z_bits;
+    }
     if constexpr (BITS == 2)
       thr[tid] = make_thresh2(gp);
     else
       grp[tid] = gp;
-    scale[tid] = gp.s_bits;
-    zero[tid] = gp.z_bits;
   }
   __syncthreads();
   const int tok0 = tg * kTileTokens;
@@ -503,7 +524,8 @@ __global__ void __launch_bounds__(1024) quantize_tiles_kernel(QuantizeArgs a) {
       quantize_k_tiles<BITS>(a.k_src + src_tok * kHeadDim, R, a.lg_gk,
                              a.k_codes + (static_cast<size_t>(bh) * C + dst_tok) * (kHeadDim / P),
                              a.k_scale + (static_cast<size_t>(bh) * (C / R) + dst_blk) * (kHeadDim >> a.lg_gk),
-                             a.k_zero + (static_cast<size_t>(bh) * (C / R) + dst_blk) * (kHeadDim >> a.lg_gk));
+                             a.k_zero + (static_cast<size_t>(bh) * (C / R) + dst_blk) * (kHeadDim >> a.lg_gk),
+                             a.k_given != 0);
     } else {
       quantize_v_tiles<BITS>(a.v_src + src_tok * kHeadDim, R, a.lg_gv,
                              a.v_codes + (static_cast<size_t>(bh) * (C / P) + dst_tok / P) * kHeadDim,
@@ -533,7 +555,8 @@ __global__ void __launch_bounds__(kThreads) quantize_blocks_kernel(QuantizeArgs 
       quantize_k_block<BITS>(a.k_src + src_tok * kHeadDim, R, a.group_k,
                              a.k_codes + (static_cast<size_t>(bh) * C + dst_tok) * (kHeadDim / P),
                              a.k_scale + (static_cast<size_t>(bh) * (C / R) + dst_blk) * (kHeadDim / a.group_k),
-                             a.k_zero + (static_cast<size_t>(bh) * (C / R) + dst_blk) * (kHeadDim / a.group_k));
+                             a.k_zero + (static_cast<size_t>(bh) * (C / R) + dst_blk) * (kHeadDim / a.group_k),
+                             a.k_given != 0);
     } else {
       quantize_v_block<BITS>(a.v_src + src_tok * kHeadDim, R, a.group_v,
                              a.v_codes + (static_cast<size_t>(bh) * (C / P) + dst_tok / P) * kHeadDim,
@@ -556,6 +579,53 @@ __global__ void __launch_bounds__(256) append_kernel(AppendArgs a) {
   reinterpret_cast<uint4*>(a.v_res)[dst] = __ldg(reinterpret_cast<const uint4*>(a.v_new) + i);
 }
 
+// K (s, z) of channel group blockIdx.y of head blockIdx.x over all nblocks * R source tokens
+// (section Per-Channel量子化 read with one group over every quantized token of the prompt), written
+// into the slot of every destination block.  256 threads; each warp reads 8 tokens x g_k channels
+// per step.
+template <int BITS>
+__global__ void __launch_bounds__(kThreads) k_prefix_extremes_kernel(QuantizeArgs a) {
+  constexpr int L = (1 << BITS) - 1;
+  __shared__ __half2 red[kThreads / 32];
+  __shared__ uint32_t sz;
+  const int bh = blockIdx.x, g = blockIdx.y, tid = threadIdx.x;
+  const int lg_cpg = a.lg_gk - 3, cpg = 1 << lg_cpg;  // 16-byte chunks per group
+  const long long ntok = static_cast<long long>(a.nblocks) * a.residual;
+  const uint4* src = reinterpret_cast<const uint4*>(a.k_src + (static_cast<size_t>(bh) * a.src_tokens + a.src_tok0) *
+                                                                  kHeadDim) + g * cpg;
+  const uint32_t kPosInf = 0x7C007C00u, kNegInf = 0xFC00FC00u;
+  __half2 lo = *reinterpret_cast<const __half2*>(&kPosInf), hi = *reinterpret_cast<const __half2*>(&kNegInf);
+  for (long long i = tid; i < (ntok << lg_cpg); i += kThreads) {
+    const uint4 v = __ldg(src + (i >> lg_cpg) * kChunks + (i & (cpg - 1)));
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const __half2 h = *reinterpret_cast<const __half2*>(&w[e]);
+      lo = __hmin2(lo, h);
+      hi = __hmax2(hi, h);
+    }
+  }
+  __half2 m = __halves2half2(__hmin(__low2half(lo), __high2half(lo)), __hneg(__hmax(__low2half(hi), __high2half(hi))));
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) m = __hmin2(m, shfl_xor_h2(m, off));
+  if ((tid & 31) == 0) red[tid >> 5] = m;
+  __syncthreads();
+  if (tid == 0) {
+    __half2 t = red[0];
+    for (int w = 1; w < kThreads / 32; ++w) t = __hmin2(t, red[w]);
+    const GroupParams gp = group_from_pair(t, L);
+    sz = static_cast<uint32_t>(gp.s_bits) | (static_cast<uint32_t>(gp.z_bits) << 16);
+  }
+  __syncthreads();
+  const int ngk = kHeadDim >> a.lg_gk;
+  const size_t C = static_cast<size_t>(a.capacity), R = static_cast<size_t>(a.residual);
+  for (int blk = tid; blk < a.nblocks; blk += kThreads) {
+    const size_t slot = (static_cast<size_t>(bh) * (C / R) + a.dst_blk0 + blk) * ngk + g;
+    a.k_scale[slot] = static_cast<uint16_t>(sz & 0xFFFFu);
+    a.k_zero[slot] = static_cast<uint16_t>(sz >> 16);
+  }
+}
+
 }  // namespace
 
 cudaError_t launch_quantize_blocks(const QuantizeArgs& args, int bits, cudaStream_t stream) {
@@ -575,6 +645,19 @@ cudaError_t launch_quantize_blocks(const QuantizeArgs& args, int bits, cudaStrea
   } else {
     quantize_blocks_kernel<4><<<grid, kThreads, 0, stream>>>(a);
   }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_k_prefix_extremes(const QuantizeArgs& args, int bits, cudaStream_t stream) {
+  if (args.nblocks == 0) return cudaSuccess;
+  QuantizeArgs a = args;
+  a.lg_gk = __builtin_ctz(static_cast<unsigned>(a.group_k));
+  a.lg_gv = __builtin_ctz(static_cast<unsigned>(a.group_v));
+  dim3 grid(a.bh, kHeadDim / a.group_k);
+  if (bits == 2)
+    k_prefix_extremes_kernel<2><<<grid, kThreads, 0, stream>>>(a);
+  else
+    k_prefix_extremes_kernel<4><<<grid, kThreads, 0, stream>>>(a);
   return cudaGetLastError();
 }
 

@@ -62,6 +62,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "kivi_check_config": (I32, [cfgp]),
         "kivi_cache_sizes": (I32, [cfgp, ctypes.POINTER(SZ)]),
         "kivi_quantize_prefill": (I32, [cfgp, cachep, P, P, I32, P]),
+        "kivi_quantize_prefill_prefix_k": (I32, [cfgp, cachep, P, P, I32, P]),
         "kivi_append_token": (I32, [cfgp, cachep, P, P, P]),
         "kivi_flush_residual": (I32, [cfgp, cachep, P]),
         "kivi_decode_workspace_bytes": (SZ, [cfgp, I32]),
@@ -105,6 +106,11 @@ def kivi_cache_sizes(cfg: kivi_config) -> list[int]:
 def kivi_quantize_prefill(cfg, cache, k_ptr: int, v_ptr: int, num_tokens: int, stream: int) -> None:
     _check(load_library().kivi_quantize_prefill(ctypes.byref(cfg), ctypes.byref(cache), k_ptr, v_ptr,
                                                 num_tokens, stream), "kivi_quantize_prefill")
+
+
+def kivi_quantize_prefill_prefix_k(cfg, cache, k_ptr: int, v_ptr: int, num_tokens: int, stream: int) -> None:
+    _check(load_library().kivi_quantize_prefill_prefix_k(ctypes.byref(cfg), ctypes.byref(cache), k_ptr, v_ptr,
+                                                         num_tokens, stream), "kivi_quantize_prefill_prefix_k")
 
 
 def kivi_append_token(cfg, cache, k_new_ptr: int, v_new_ptr: int, stream: int) -> None:
@@ -215,6 +221,11 @@ class KiviCache:
         """k, v: contiguous fp16 device tensors [B][H][T][d]."""
         assert k.dtype == self.torch.float16 and k.is_contiguous() and v.is_contiguous()
         kivi_quantize_prefill(self.cfg, self.c, k.data_ptr(), v.data_ptr(), k.shape[2], self._stream(stream))
+
+    def prefill_prefix_k(self, k, v, stream=None) -> None:
+        """prefill with one K group over the whole quantized prefix (kivi_quantize_prefill_prefix_k)."""
+        assert k.dtype == self.torch.float16 and k.is_contiguous() and v.is_contiguous()
+        kivi_quantize_prefill_prefix_k(self.cfg, self.c, k.data_ptr(), v.data_ptr(), k.shape[2], self._stream(stream))
 
     def append(self, k_new, v_new, stream=None) -> None:
         """k_new, v_new: contiguous fp16 device tensors [B][H][d]."""

@@ -125,6 +125,17 @@ int kivi_quantize_prefill(const kivi_config* cfg, kivi_cache* cache, const uint1
                           const uint16_t* v_dev, int32_t num_tokens, void* stream);
 
 /*
+ * Prefill under the other reading of section Per-Channel量子化, in which one K group spans every
+ * quantized token of the prompt instead of one R-token block: the K scale and zero of each
+ * channel group are taken over tokens [0, n_quant) and stored in every block's slot, so decode
+ * attention, appends and later flushes (which quantize their own R-token blocks) are unchanged.
+ * V groups, the residual split, arguments and errors are those of kivi_quantize_prefill.
+ * Two kernel launches (the K group extremes over the prefix, then the quantization).
+ */
+int kivi_quantize_prefill_prefix_k(const kivi_config* cfg, kivi_cache* cache, const uint16_t* k_dev,
+                                   const uint16_t* v_dev, int32_t num_tokens, void* stream);
+
+/*
  * Append: writes one new token's K and V (fp16 [B][H][d]) into residual slot n_res and
  * increments n_res.  Section 残差バッファ.  Errors: n_res == R (RESIDUAL_FULL).  One launch.
  */
