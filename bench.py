@@ -63,6 +63,11 @@ def hbm_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+def dot_engine(w):
+    """The instruction that forms the decode kernel's byte dot products for this workload."""
+    return "mma.sync m16n8k32" if w.bits == 2 and w.q_heads == w.kv_heads else "dp4a"
+
+
 def profiled_traffic(w: synth.Workload, alg_bytes_per_launch: float):
     """DRAM bytes per decode launch from the committed ncu record, if it was taken on the current
     kernel sources; else None.  The record holds one captured launch (its DRAM bytes and its
@@ -399,7 +404,7 @@ def run_gpu(args, rank, world, local_rank, w: synth.Workload):
         result = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
             "ms_per_step": t_max / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": f"u{w.bits} codes x i8 limbs (dp4a, i32 acc), f32 softmax", "data": "synthetic",
+            "dtype": f"u{w.bits} codes x i8 limbs ({dot_engine(w)}, i32 acc), f32 softmax", "data": "synthetic",
             "config": {
                 "workload": w.name, "batch": w.batch, "q_heads": w.q_heads, "kv_heads": w.kv_heads,
                 "head_dim": w.head_dim, "bits": w.bits, "group_k": w.group, "group_v": w.group,

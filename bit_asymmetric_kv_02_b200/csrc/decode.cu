@@ -19,18 +19,21 @@
 // A fused append (kivi_append_decode_attention) hands the new token's rows to the warp that owns
 // the residual unit holding its slot; that warp patches its shared-memory copy and the cache.
 //
-// Arithmetic (CUDA cores, no tensor cores: one query row per head is a matrix-vector product).
+// Arithmetic.  The byte dot products are exact int32 sums.  At 2 bits with one query per KV head
+// they run on the tensor cores (mma.sync m16n8k32, codes x limbs): dp4a would need 768 issues of
+// the half-rate FMA-heavy pipe per 8 KB, more than the HBM time of those bytes.  Elsewhere (4 bits,
+// several queries per KV head) dp4a on the CUDA cores forms them.
 //   A6  logit_t = sum_c q_c (s_g code + z_g) = sum_c (q_c s_g) code_tc + sum_g z_g sum_{c in g} q_c.
 //       (q_c s_g) for one R-token block is turned into a 24-bit signed fixed-point integer split in
 //       three byte limbs (kept while the warp stays in the same block); the codes are unpacked to
-//       bytes with one shift and masks, and dp4a forms the byte dot products exactly in int32.
+//       bytes with one shift and masks and multiplied with the limbs exactly in int32.
 //       The block constant sum_g z_g q_g is added in fp32.
 //   A8  online softmax in base 2 (q pre-scaled by scale*log2 e), redux.sync warp maxima, lane-local
 //       sums.
 //   A9  o_c = sum_t (p_t s_g(t)) code_tc + sum_t p_t z_g(t): (p_t s_g(t)) is turned into 24-bit
 //       unsigned fixed point relative to a bound of the unit's largest value (at 2 bits: the
 //       unit's largest weight times its largest V scale; at 4 bits: the exact maximum) and dotted
-//       with the V codes by dp4a; the z term is the same for every channel and is one scalar.
+//       with the V codes; the z term is the same for every channel and is one scalar.
 //   A7/A9 residual rows: fp32 FMAs on the fp16 values.
 //   A10 merge of (m, l, Z, o) states: o / l with o += Z.
 // 24-bit limbs keep every product relative error below 2^-21, the integer sums are exact, and the
@@ -65,12 +68,23 @@ constexpr int kResTokens = 16;      // tokens per residual unit
 constexpr unsigned kFull = 0xffffffffu;
 constexpr float kQRange = 8388544.f;   // 2^23 - 64: largest |Q| before rounding (signed 24-bit limbs)
 constexpr float kPRange = 16777088.f;  // 2^24 - 128: largest P before rounding (unsigned 24-bit limbs)
+// Largest |Q| before rounding for balanced signed limbs (every digit in [-128, 127], so the top
+// digit (Q + 32896) >> 16 must stay below 128): 2^23 - 2^16.
+constexpr float kQRangeBal = 8323072.f;
+
+// Limb words per query: 96 (three limbs) for the CUDA-core dot products; 128 for the tensor-core
+// path of one query per KV head, which keeps a fourth, all-zero limb slot (the B operand columns
+// that belong to no limb read it).
+template <int G>
+__host__ __device__ constexpr int limb_vecs() {
+  return G == 1 ? 32 : 24;
+}
 
 template <int G>
 struct __align__(16) WarpSmem {
   uint8_t buf[ring_buffers<G>()][kHalfBytes];
-  uint4 qw[G][24];  // Q limbs of each query: 96 words
-  uint4 pw[G][24];  // P limbs of each query: up to 96 words
+  uint4 qw[G][limb_vecs<G>()];  // Q limbs of each query
+  uint4 pw[G][limb_vecs<G>()];  // P limbs of each query
   uint64_t bar[ring_buffers<G>()];
 };
 
@@ -103,6 +117,38 @@ __device__ __forceinline__ float fast_exp2(float x) {
 // hi * 2^16 + mid * 2^8 + lo.  mid * 2^8 + lo stays below 2^27 for every sum formed here (at most
 // 128 products of a byte with a code of at most 15), so it is formed exactly in int32.
 __device__ __forceinline__ float combine_limbs(int hi, int mid, int lo) {
+  return fmaf(static_cast<float>(hi), 65536.f, static_cast<float>((mid << 8) + lo));
+}
+
+// Tensor-core byte dot products: D += A B with A a 16 x 32 tile of codes (unsigned bytes, row-major)
+// and B a 32 x 8 tile of limbs (signed or unsigned bytes), D 16 x 8 in int32.  Lane (g, t) =
+// (lane / 4, lane % 4) holds A rows g and g + 8, columns 4 t .. 4 t + 3 (a0, a1) and 16 + 4 t ..
+// 19 + 4 t (a2, a3); B column g, rows 4 t .. 4 t + 3 (b0) and 16 + 4 t .. (b1); D rows g and g + 8,
+// columns 2 t and 2 t + 1.
+__device__ __forceinline__ void mma_u8s8(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
+                                         uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ void mma_u8u8(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
+                                         uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k32.row.col.s32.u8.u8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+// Byte b of x0 .. x3 packed into one word (byte m from x_m).
+__device__ __forceinline__ uint32_t pick_bytes(uint32_t x0, uint32_t x1, uint32_t x2, uint32_t x3, int b) {
+  const uint32_t sel = static_cast<uint32_t>(b) | (static_cast<uint32_t>(b + 4) << 4);
+  return __byte_perm(__byte_perm(x0, x1, sel), __byte_perm(x2, x3, sel), 0x5410);
+}
+// Rows g and g + 8 of a tile pair's limb accumulators: lanes 2 t' and 2 t' + 1 (t' = 0, 1) hold
+// columns (H, M) and (L, 0) of tile t' of the pair (columns 4 t' .. 4 t' + 2).  After one exchange
+// with the partner lane, an even lane holds row g and an odd lane row g + 8, whole.
+__device__ __forceinline__ float gather_limbs(const int (&c)[4], bool odd) {
+  const int r1 = __shfl_xor_sync(0xffffffffu, odd ? c[0] : c[2], 1);
+  const int r2 = __shfl_xor_sync(0xffffffffu, c[3], 1);
+  const int hi = odd ? r1 : c[0], mid = odd ? r2 : c[1], lo = odd ? c[2] : r1;
   return fmaf(static_cast<float>(hi), 65536.f, static_cast<float>((mid << 8) + lo));
 }
 
@@ -140,6 +186,8 @@ struct Decoder {
   static constexpr int ROWS = UT / P;              // V word rows per unit (8)
   static constexpr int kBuffers = ring_buffers<G>();
   static constexpr int GP = G == 1 ? 1 : 2;        // queries per pass over a unit's codes
+  // 2 bits with one query per KV head: the byte dot products run on the tensor cores (mma.sync)
+  static constexpr bool kMma = BITS == 2 && G == 1;
 
   const DecodeArgs& a;
   WarpSmem<G>& S;
@@ -305,11 +353,162 @@ struct Decoder {
   // ---- A6 set-up for one K block: fixed-point limbs of q_c * s_g(c) -------------------------
   __device__ void build_q(uint32_t pairs) {
     __syncwarp();  // the previous block's limbs are no longer read
-    if constexpr (BITS == 2)
+    if constexpr (kMma)
+      build_q2_mma(pairs);
+    else if constexpr (BITS == 2)
       build_q2(pairs);
     else
       build_q4(pairs);
     __syncwarp();
+  }
+
+  // ---- tensor-core path (2 bits, one query per KV head) ---------------------------------------
+  // Limb layout in shared memory, Q and P alike: word (i, slot, set) at (16 i + 4 slot + set) for
+  // i = K code word (Q) or V word row (P); slots 0, 1, 2 hold the high, middle and low limbs and
+  // slot 3 stays zero.  Byte m of (i, slot, set) belongs to channel 16 i + 4 m + set (Q) or token
+  // 16 i + 4 m + set (P), the element that byte m of set `set` of a code word multiplies.
+  //
+  // An m16n8k32 tile contracts 32 channels (K) or 32 tokens (V) of 16 rows (tokens or channels)
+  // against the three limbs in B columns 0..2.  Two tiles share one accumulator: the second's limbs
+  // sit in columns 4..6, so lane (n, t) with n = lane / 4 reads B from slot n (n < 3) for the first
+  // tile and slot n - 4 (4 <= n < 7) for the second, slot 3 otherwise.
+
+  // Q limbs as balanced signed digits, Q = H 2^16 + M 2^8 + L with every digit in [-128, 127]
+  // (an s8 B operand): L = byte 0 of Q, M = byte 1 of Q + 128, H = byte 2 of Q + 32896.
+  // Lane (i, k) forms the words (i, slot, k) of channels 16 i + 4 m + k; odd sets read 4 * code.
+  __device__ void build_q2_mma(uint32_t pairs) {
+    const int gi = (16 * (lane >> 2)) >> a.lg_gk;  // the K group of all four channels
+    const float s = h2f(static_cast<uint16_t>(__shfl_sync(kFull, pairs, gi) & 0xFFFFu));
+    const float z_own = k_lane ? h2f(static_cast<uint16_t>(pairs >> 16)) : 0.f;
+    float qv[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) qv[j] = q_of(0, j) * s;
+    const float mabs = warp_max(fmaxf(fmaxf(fabsf(qv[0]), fabsf(qv[1])), fmaxf(fabsf(qv[2]), fabsf(qv[3]))));
+    const float scq = mabs > 0.f ? kQRangeBal * fast_rcp(mabs) : 0.f;
+    invq[0] = mabs * (1.0f / kQRangeBal);
+    float c = z_own * qsum[0][0];
+    c += __shfl_xor_sync(kFull, c, 1);
+    c += __shfl_xor_sync(kFull, c, 2);
+    cblk[0] = __shfl_sync(kFull, c, 0);
+    const float f = scq * ((lane & 1) ? 0.25f : 1.f);
+    uint32_t Q[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) Q[j] = static_cast<uint32_t>(__float2int_rn(qv[j] * f));
+    uint32_t* row = reinterpret_cast<uint32_t*>(S.qw[0]) + 16 * (lane >> 2) + (lane & 3);
+    row[0] = pick_bytes(Q[0] + 32896u, Q[1] + 32896u, Q[2] + 32896u, Q[3] + 32896u, 2);
+    row[4] = pick_bytes(Q[0] + 128u, Q[1] + 128u, Q[2] + 128u, Q[3] + 128u, 1);
+    row[8] = pick_bytes(Q[0], Q[1], Q[2], Q[3], 0);
+  }
+
+  // Logits of the unit's 128 tokens.  Tile 2 j + b holds tokens 32 j + 16 b + (0..15) as rows;
+  // lane (g, t) unpacks code words 2 t and 2 t + 1 of tokens 32 j + 16 b + g and + 8.  After the
+  // exchange, lg[j] is the logit of token 32 j + 16 (t / 2) + 8 (t % 2) + g.
+  __device__ void k_mma(const uint8_t* kt, float (&lg)[4]) const {
+    const int g = lane >> 2, t = lane & 3;
+    const int se = g < 4 ? g : 3, so = g >= 4 ? g - 4 : 3;
+    const uint4 be0 = S.qw[0][8 * t + se], be1 = S.qw[0][8 * t + 4 + se];
+    const uint4 bo0 = S.qw[0][8 * t + so], bo1 = S.qw[0][8 * t + 4 + so];
+    const bool odd = t & 1;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      int c[4] = {0, 0, 0, 0};
+#pragma unroll
+      for (int b = 0; b < 2; ++b) {
+        const uint8_t* r0 = kt + (32 * j + 16 * b + g) * 32 + 8 * t;
+        const uint2 wg = *reinterpret_cast<const uint2*>(r0);
+        const uint2 wh = *reinterpret_cast<const uint2*>(r0 + 8 * 32);
+        const uint4& B0 = b ? bo0 : be0;
+        const uint4& B1 = b ? bo1 : be1;
+        uint32_t mg[4], mh[4];
+        masks2(wg.x, mg);
+        masks2(wh.x, mh);
+        mma_u8s8(c, mg[0], mh[0], mg[1], mh[1], B0.x, B0.y);
+        mma_u8s8(c, mg[2], mh[2], mg[3], mh[3], B0.z, B0.w);
+        masks2(wg.y, mg);
+        masks2(wh.y, mh);
+        mma_u8s8(c, mg[0], mh[0], mg[1], mh[1], B1.x, B1.y);
+        mma_u8s8(c, mg[2], mh[2], mg[3], mh[3], B1.z, B1.w);
+      }
+      lg[j] = fmaf(gather_limbs(c, odd), invq[0], cblk[0]);
+    }
+  }
+
+  // Online softmax of the unit and its P limbs (unsigned bytes), scaled by the bound 2^(mu - m) *
+  // s_max as on the CUDA-core path.  Token 32 j + ... lies in V group (32 j) >> lg_gv of the unit
+  // (V groups span at least 32 tokens); its P goes to byte 2 (t % 2) + g / 4 of word
+  // (2 j + t / 2, slot, g % 4).
+  __device__ void softmax_mma(uint32_t pairs, const float (&lg)[4]) {
+    const int g = lane >> 2, t = lane & 3;
+    const float mu = warp_max(fmaxf(fmaxf(lg[0], lg[1]), fmaxf(lg[2], lg[3])));
+    const float smax = warp_max(v_lane ? h2f(static_cast<uint16_t>(pairs & 0xFFFFu)) : 0.f);
+    const float m_new = fmaxf(m[0], mu);
+    const float alpha = fast_exp2(m[0] - m_new);
+    const float d = mu - m_new;  // <= 0: the unit's largest weight is 2^d
+    const bool hv = d > -64.f && smax > 0.f;
+    const float fb = hv ? (kPRange * fast_rcp(smax)) * fast_exp2(-d) * ((g & 1) ? 0.25f : 1.f) : 0.f;
+    float p[4], sv[4], psum = 0.f, zsum = 0.f;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint32_t vp = __shfl_sync(kFull, pairs, 8 + ((32 * j) >> a.lg_gv));
+      sv[j] = h2f(static_cast<uint16_t>(vp & 0xFFFFu));
+      p[j] = fast_exp2(lg[j] - m_new);
+      psum += p[j];
+      zsum = fmaf(p[j], h2f(static_cast<uint16_t>(vp >> 16)), zsum);
+    }
+    m[0] = m_new;
+    l[0] = fmaf(l[0], alpha, psum);
+    Z[0] = fmaf(Z[0], alpha, zsum);
+    alpha_[0] = alpha;
+    hasv_[0] = hv;
+    invv_[0] = hv ? fast_exp2(d) * smax * (1.0f / kPRange) : 0.f;
+    uint8_t* pb = reinterpret_cast<uint8_t*>(S.pw[0]) + 64 * (t >> 1) + 4 * (g & 3) + 2 * (t & 1) + (g >> 2);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint32_t P = __float2uint_rn(p[j] * (sv[j] * fb));
+      pb[128 * j] = static_cast<uint8_t>(P >> 16);
+      pb[128 * j + 16] = static_cast<uint8_t>(P >> 8);
+      pb[128 * j + 32] = static_cast<uint8_t>(P);
+    }
+  }
+
+  // P . codes of the unit.  Tile pair v holds channels 16 g' + 8 b + 4 c + v (tile 2 v + b, row
+  // g' + 8 c) as rows; lane (g, t) unpacks V word rows 2 t and 2 t + 1 of channels 16 g .. 16 g + 15
+  // (four 16-byte loads per row).  After the exchange the lane holds channel 4 lane + v of tile
+  // pair v, the channel it accumulates in o[0][v].
+  __device__ void v_mma(const uint8_t* vt) {
+    static_assert(P == 16 && ROWS == 8, "2-bit units: 8 V word rows of 16 tokens");
+    const int g = lane >> 2, t = lane & 3;
+    const int se = g < 4 ? g : 3, so = g >= 4 ? g - 4 : 3;
+    uint4 be[2], bo[2];
+#pragma unroll
+    for (int x = 0; x < 2; ++x) {
+      be[x] = S.pw[0][8 * t + 4 * x + se];
+      bo[x] = S.pw[0][8 * t + 4 * x + so];
+    }
+    int cv[4][4];
+#pragma unroll
+    for (int v = 0; v < 4; ++v) cv[v][0] = cv[v][1] = cv[v][2] = cv[v][3] = 0;
+#pragma unroll
+    for (int x = 0; x < 2; ++x) {
+      const uint8_t* rowp = vt + (2 * t + x) * 512 + 64 * g;
+#pragma unroll
+      for (int b = 0; b < 2; ++b) {
+        const uint4 wlo = *reinterpret_cast<const uint4*>(rowp + 32 * b);
+        const uint4 whi = *reinterpret_cast<const uint4*>(rowp + 32 * b + 16);
+        const uint4& B = b ? bo[x] : be[x];
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+          uint32_t mg[4], mh[4];
+          masks2(comp(wlo, v), mg);
+          masks2(comp(whi, v), mh);
+          mma_u8u8(cv[v], mg[0], mh[0], mg[1], mh[1], B.x, B.y);
+          mma_u8u8(cv[v], mg[2], mh[2], mg[3], mh[3], B.z, B.w);
+        }
+      }
+    }
+    const bool odd = t & 1;
+#pragma unroll
+    for (int v = 0; v < 4; ++v) o[0][v] = fmaf(o[0][v], alpha_[0], gather_limbs(cv[v], odd) * invv_[0]);
   }
 
   // 4 bits: lane holds channels lane + 32 j; each byte of a limb word is stored on its own.
@@ -477,7 +676,11 @@ struct Decoder {
       build_q(pairs);
       qkey = key;
     }
-    if constexpr (BITS == 2) {
+    if constexpr (kMma) {
+      float lg[4];
+      k_mma(kt, lg);
+      softmax_mma(pairs, lg);
+    } else if constexpr (BITS == 2) {
       const VScales vs = v_scales2(pairs);  // independent of the dot products: issued first
 #pragma unroll
       for (int g0 = 0; g0 < G; g0 += GP) {
@@ -550,9 +753,16 @@ struct Decoder {
     if (G == 1 && !hasv_[0]) {  // every weight of the unit is zero: only rescale
 #pragma unroll
       for (int e = 0; e < 4; ++e) o[0][e] *= alpha_[0];
-      __syncwarp();
-      return;
+    } else if constexpr (kMma) {
+      v_mma(vt);
+    } else {
+      dot_v(vt);
     }
+    __syncwarp();  // P limbs are rewritten by the next unit
+  }
+
+  // CUDA-core P . codes: dp4a on the three limbs of every query's P.
+  __device__ void dot_v(const uint8_t* vt) {
 #pragma unroll
     for (int g0 = 0; g0 < G; g0 += GP) {  // queries g0 .. g0 + GP - 1 per pass over the codes
       int vl[GP][4], vm[GP][4], vh[GP][4];
@@ -607,7 +817,6 @@ struct Decoder {
         }
       }
     }
-    __syncwarp();  // P limbs are rewritten by the next unit
   }
 
   // ---- K half of a residual unit (16 fp16 rows): logits and softmax weights --------------------
@@ -815,6 +1024,12 @@ struct Decoder {
 #pragma unroll
       for (int b = 0; b < kBuffers; ++b) mbar_init(&S.bar[b], 1);
       asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if constexpr (kMma) {  // slot 3 of every limb row stays zero; slots 0..2 are written before use
+      for (int i = lane; i < 4 * limb_vecs<G>(); i += 32) {
+        reinterpret_cast<uint32_t*>(S.qw[0])[i] = 0u;
+        reinterpret_cast<uint32_t*>(S.pw[0])[i] = 0u;
+      }
     }
     __syncwarp();
     const int nhalves = static_cast<int>(2 * (ue - ub));
