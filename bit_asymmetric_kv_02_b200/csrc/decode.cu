@@ -57,6 +57,13 @@ __host__ __device__ constexpr int warps_per_cta() {
   return G == 1 ? 16 : (G <= 4 ? 12 : 8);  // 128, 168 and 255 registers
 }
 constexpr int kHalfBytes = 4096;    // one half unit: the K part or the V part of a unit
+// The tensor-core path lands a V half as four 1 KB pieces (two V word rows each) 1040 bytes apart,
+// so that the four lanes reading one channel from rows 2 t + x (t = 0..3) hit four bank groups.
+constexpr int kVPiece = 1024, kVPieceStride = 1040;
+template <int G>
+__host__ __device__ constexpr int buf_bytes() {
+  return G == 1 ? 4 * kVPieceStride : kHalfBytes;
+}
 // Half-unit buffers per warp: 3 gives the ring K0 V0 K1 | V1 K2 V2 | ..., 2 gives K | V.  Up to 4
 // queries per KV head use 2 (1.4% faster than 3 at 16 warps per SM, and 16 warps of 3 would not fit
 // in shared memory); 8 queries per KV head (8 warps per SM) use 3.
@@ -82,7 +89,7 @@ __host__ __device__ constexpr int limb_vecs() {
 
 template <int G>
 struct __align__(16) WarpSmem {
-  uint8_t buf[ring_buffers<G>()][kHalfBytes];
+  uint8_t buf[ring_buffers<G>()][buf_bytes<G>()];
   uint4 qw[G][limb_vecs<G>()];  // Q limbs of each query
   uint4 pw[G][limb_vecs<G>()];  // P limbs of each query
   uint64_t bar[ring_buffers<G>()];
@@ -233,7 +240,13 @@ struct Decoder {
     const int unit = quant ? local : local - a.units_q;
     const char* src = base + static_cast<size_t>(head) * stride + static_cast<size_t>(unit) * kHalfBytes;
     mbar_arrive_expect_tx(&S.bar[b], kHalfBytes + a.debug_extra_tx);
-    bulk_g2s(S.buf[b], src, kHalfBytes, &S.bar[b]);
+    if (kMma && is_v) {
+#pragma unroll
+      for (int c = 0; c < kHalfBytes / kVPiece; ++c)
+        bulk_g2s(S.buf[b] + c * kVPieceStride, src + c * kVPiece, kVPiece, &S.bar[b]);
+    } else {
+      bulk_g2s(S.buf[b], src, kHalfBytes, &S.bar[b]);
+    }
   }
 
   // (s, z) pairs of a quantized unit: lanes [0, ngk) hold K groups, lanes [8, 8 + nvg) V groups.
@@ -363,9 +376,10 @@ struct Decoder {
   }
 
   // ---- tensor-core path (2 bits, one query per KV head) ---------------------------------------
-  // Limb layout in shared memory, Q and P alike: word (i, slot, set) at (16 i + 4 slot + set) for
-  // i = K code word (Q) or V word row (P); slots 0, 1, 2 hold the high, middle and low limbs and
-  // slot 3 stays zero.  Byte m of (i, slot, set) belongs to channel 16 i + 4 m + set (Q) or token
+  // Limb layout in shared memory, Q and P alike: word (i, slot, set) at 16 i + 4 (slot ^ (i / 2 % 4))
+  // + set for i = K code word (Q) or V word row (P); slots 0, 1, 2 hold the high, middle and low
+  // limbs and slot 3 stays zero.  The XOR spreads the four lanes t that read rows 2 t + x of one
+  // slot over four bank groups.  Byte m of (i, slot, set) belongs to channel 16 i + 4 m + set (Q) or token
   // 16 i + 4 m + set (P), the element that byte m of set `set` of a code word multiplies.
   //
   // An m16n8k32 tile contracts 32 channels (K) or 32 tokens (V) of 16 rows (tokens or channels)
@@ -394,10 +408,11 @@ struct Decoder {
     uint32_t Q[4];
 #pragma unroll
     for (int j = 0; j < 4; ++j) Q[j] = static_cast<uint32_t>(__float2int_rn(qv[j] * f));
-    uint32_t* row = reinterpret_cast<uint32_t*>(S.qw[0]) + 16 * (lane >> 2) + (lane & 3);
-    row[0] = pick_bytes(Q[0] + 32896u, Q[1] + 32896u, Q[2] + 32896u, Q[3] + 32896u, 2);
-    row[4] = pick_bytes(Q[0] + 128u, Q[1] + 128u, Q[2] + 128u, Q[3] + 128u, 1);
-    row[8] = pick_bytes(Q[0], Q[1], Q[2], Q[3], 0);
+    const int i = lane >> 2, sw = (i >> 1) & 3;
+    uint32_t* row = reinterpret_cast<uint32_t*>(S.qw[0]) + 16 * i + (lane & 3);
+    row[4 * (0 ^ sw)] = pick_bytes(Q[0] + 32896u, Q[1] + 32896u, Q[2] + 32896u, Q[3] + 32896u, 2);
+    row[4 * (1 ^ sw)] = pick_bytes(Q[0] + 128u, Q[1] + 128u, Q[2] + 128u, Q[3] + 128u, 1);
+    row[4 * (2 ^ sw)] = pick_bytes(Q[0], Q[1], Q[2], Q[3], 0);
   }
 
   // Logits of the unit's 128 tokens.  Tile 2 j + b holds tokens 32 j + 16 b + (0..15) as rows;
@@ -406,8 +421,8 @@ struct Decoder {
   __device__ void k_mma(const uint8_t* kt, float (&lg)[4]) const {
     const int g = lane >> 2, t = lane & 3;
     const int se = g < 4 ? g : 3, so = g >= 4 ? g - 4 : 3;
-    const uint4 be0 = S.qw[0][8 * t + se], be1 = S.qw[0][8 * t + 4 + se];
-    const uint4 bo0 = S.qw[0][8 * t + so], bo1 = S.qw[0][8 * t + 4 + so];
+    const uint4 be0 = S.qw[0][8 * t + (se ^ t)], be1 = S.qw[0][8 * t + 4 + (se ^ t)];
+    const uint4 bo0 = S.qw[0][8 * t + (so ^ t)], bo1 = S.qw[0][8 * t + 4 + (so ^ t)];
     const bool odd = t & 1;
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
@@ -436,7 +451,7 @@ struct Decoder {
   // Online softmax of the unit and its P limbs (unsigned bytes), scaled by the bound 2^(mu - m) *
   // s_max as on the CUDA-core path.  Token 32 j + ... lies in V group (32 j) >> lg_gv of the unit
   // (V groups span at least 32 tokens); its P goes to byte 2 (t % 2) + g / 4 of word
-  // (2 j + t / 2, slot, g % 4).
+  // (2 j + t / 2, slot, g % 4), whose slot position is slot ^ j.
   __device__ void softmax_mma(uint32_t pairs, const float (&lg)[4]) {
     const int g = lane >> 2, t = lane & 3;
     const float mu = warp_max(fmaxf(fmaxf(lg[0], lg[1]), fmaxf(lg[2], lg[3])));
@@ -465,16 +480,16 @@ struct Decoder {
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const uint32_t P = __float2uint_rn(p[j] * (sv[j] * fb));
-      pb[128 * j] = static_cast<uint8_t>(P >> 16);
-      pb[128 * j + 16] = static_cast<uint8_t>(P >> 8);
-      pb[128 * j + 32] = static_cast<uint8_t>(P);
+      pb[128 * j + 16 * (0 ^ j)] = static_cast<uint8_t>(P >> 16);
+      pb[128 * j + 16 * (1 ^ j)] = static_cast<uint8_t>(P >> 8);
+      pb[128 * j + 16 * (2 ^ j)] = static_cast<uint8_t>(P);
     }
   }
 
   // P . codes of the unit.  Tile pair v holds channels 16 g' + 8 b + 4 c + v (tile 2 v + b, row
   // g' + 8 c) as rows; lane (g, t) unpacks V word rows 2 t and 2 t + 1 of channels 16 g .. 16 g + 15
   // (four 16-byte loads per row).  After the exchange the lane holds channel 4 lane + v of tile
-  // pair v, the channel it accumulates in o[0][v].
+  // pair v, the channel it accumulates in o[0][v].  Rows 2 t and 2 t + 1 are piece t of the buffer.
   __device__ void v_mma(const uint8_t* vt) {
     static_assert(P == 16 && ROWS == 8, "2-bit units: 8 V word rows of 16 tokens");
     const int g = lane >> 2, t = lane & 3;
@@ -482,15 +497,15 @@ struct Decoder {
     uint4 be[2], bo[2];
 #pragma unroll
     for (int x = 0; x < 2; ++x) {
-      be[x] = S.pw[0][8 * t + 4 * x + se];
-      bo[x] = S.pw[0][8 * t + 4 * x + so];
+      be[x] = S.pw[0][8 * t + 4 * x + (se ^ t)];
+      bo[x] = S.pw[0][8 * t + 4 * x + (so ^ t)];
     }
     int cv[4][4];
 #pragma unroll
     for (int v = 0; v < 4; ++v) cv[v][0] = cv[v][1] = cv[v][2] = cv[v][3] = 0;
 #pragma unroll
     for (int x = 0; x < 2; ++x) {
-      const uint8_t* rowp = vt + (2 * t + x) * 512 + 64 * g;
+      const uint8_t* rowp = vt + t * kVPieceStride + x * 512 + 64 * g;
 #pragma unroll
       for (int b = 0; b < 2; ++b) {
         const uint4 wlo = *reinterpret_cast<const uint4*>(rowp + 32 * b);
@@ -819,23 +834,26 @@ struct Decoder {
     }
   }
 
+  // Byte offset of fp16 row tt of a residual V half in its buffer (four rows per 1 KB piece).
+  static __device__ __forceinline__ int vrow(int tt) { return tt * 256 + (kMma ? (tt >> 2) * (kVPieceStride - kVPiece) : 0); }
+
   // ---- K half of a residual unit (16 fp16 rows): logits and softmax weights --------------------
   // q is read in fp16 from global memory (L1-resident: every lane pair reads the same 256 bytes).
   // Fused append: if the new token's slot falls in residual unit r (rows 16 r .. 16 r + 15), copy its
   // row from `src` into the unit's shared-memory copy (which the bulk copy filled from the cache)
   // and into the cache itself.  Each residual unit belongs to one warp, so the row is written once.
-  __device__ void insert_new_row(uint8_t* buf, int r, long long head, const uint16_t* src, uint16_t* res) {
+  __device__ void insert_new_row(uint8_t* buf, int r, long long head, const uint16_t* src, uint16_t* res, bool v_half) {
     const int row = a.new_slot - r * kResTokens;
     if (a.new_slot < 0 || row < 0 || row >= kResTokens) return;
     const uint2 v = __ldg(reinterpret_cast<const uint2*>(src + static_cast<size_t>(head) * kHeadDim) + lane);
-    *reinterpret_cast<uint2*>(buf + row * 256 + 8 * lane) = v;
+    *reinterpret_cast<uint2*>(buf + (v_half ? vrow(row) : row * 256) + 8 * lane) = v;
     uint16_t* dst = res + (static_cast<size_t>(head) * a.residual + a.new_slot) * kHeadDim;
     reinterpret_cast<uint2*>(dst)[lane] = v;
     __syncwarp();
   }
 
   __device__ void residual_k(uint8_t* kt, int nvalid, long long head, int r) {
-    insert_new_row(kt, r, head, a.k_new, a.k_res);
+    insert_new_row(kt, r, head, a.k_new, a.k_res, false);
     const int t = lane >> 1, hf = lane & 1;  // 2 lanes per token, 64 channels each
 #pragma unroll
     for (int g = 0; g < G; ++g) {
@@ -873,14 +891,14 @@ struct Decoder {
 
   // ---- V half of a residual unit: p . rows -----------------------------------------------------
   __device__ void residual_v(uint8_t* vt, int nvalid, long long head, int r) {
-    insert_new_row(vt, r, head, a.v_new, a.v_res);
+    insert_new_row(vt, r, head, a.v_new, a.v_res, true);
 #pragma unroll
     for (int g = 0; g < G; ++g) {
 #pragma unroll
       for (int e = 0; e < 4; ++e) o[g][e] *= alpha_[g];
       for (int tt = 0; tt < nvalid; ++tt) {
         const float pt = __shfl_sync(kFull, pres_[g], 2 * tt);
-        const uint2 vv = *reinterpret_cast<const uint2*>(vt + tt * 256 + 8 * lane);
+        const uint2 vv = *reinterpret_cast<const uint2*>(vt + vrow(tt) + 8 * lane);
         const float2 v0 = __half22float2(*reinterpret_cast<const __half2*>(&vv.x));
         const float2 v1 = __half22float2(*reinterpret_cast<const __half2*>(&vv.y));
         o[g][0] = fmaf(pt, v0.x, o[g][0]);
