@@ -65,7 +65,7 @@ def hbm_peak():
 
 def dot_engine(w):
     """The instruction that forms the decode kernel's byte dot products for this workload."""
-    return "mma.sync m16n8k32" if w.bits == 2 and w.q_heads == w.kv_heads else "dp4a"
+    return "mma.sync m16n8k32" if w.bits == 2 else "dp4a"
 
 
 def profiled_traffic(w: synth.Workload, alg_bytes_per_launch: float):

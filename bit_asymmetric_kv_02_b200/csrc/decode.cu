@@ -19,10 +19,10 @@
 // A fused append (kivi_append_decode_attention) hands the new token's rows to the warp that owns
 // the residual unit holding its slot; that warp patches its shared-memory copy and the cache.
 //
-// Arithmetic.  The byte dot products are exact int32 sums.  At 2 bits with one query per KV head
-// they run on the tensor cores (mma.sync m16n8k32, codes x limbs): dp4a would need 768 issues of
-// the half-rate FMA-heavy pipe per 8 KB, more than the HBM time of those bytes.  Elsewhere (4 bits,
-// several queries per KV head) dp4a on the CUDA cores forms them.
+// Arithmetic.  The byte dot products are exact int32 sums.  At 2 bits they run on the tensor cores
+// (mma.sync m16n8k32, codes x limbs): dp4a would need 768 issues of the half-rate FMA-heavy pipe per
+// 8 KB and query, more than the HBM time of those bytes.  At 4 bits dp4a on the CUDA cores forms
+// them (half the dp4a per byte).
 //   A6  logit_t = sum_c q_c (s_g code + z_g) = sum_c (q_c s_g) code_tc + sum_g z_g sum_{c in g} q_c.
 //       (q_c s_g) for one R-token block is turned into a 24-bit signed fixed-point integer split in
 //       three byte limbs (kept while the warp stays in the same block); the codes are unpacked to
@@ -62,7 +62,7 @@ constexpr int kHalfBytes = 4096;    // one half unit: the K part or the V part o
 constexpr int kVPiece = 1024, kVPieceStride = 1040;
 template <int G>
 __host__ __device__ constexpr int buf_bytes() {
-  return G == 1 ? 4 * kVPieceStride : kHalfBytes;
+  return 4 * kVPieceStride;
 }
 // Half-unit buffers per warp: 3 gives the ring K0 V0 K1 | V1 K2 V2 | ..., 2 gives K | V.  Up to 4
 // queries per KV head use 2 (1.4% faster than 3 at 16 warps per SM, and 16 warps of 3 would not fit
@@ -79,19 +79,15 @@ constexpr float kPRange = 16777088.f;  // 2^24 - 128: largest P before rounding 
 // digit (Q + 32896) >> 16 must stay below 128): 2^23 - 2^16.
 constexpr float kQRangeBal = 8323072.f;
 
-// Limb words per query: 96 (three limbs) for the CUDA-core dot products; 128 for the tensor-core
-// path of one query per KV head, which keeps a fourth, all-zero limb slot (the B operand columns
-// that belong to no limb read it).
-template <int G>
-__host__ __device__ constexpr int limb_vecs() {
-  return G == 1 ? 32 : 24;
-}
+// Limb words per query: 96 (three limbs) for the CUDA-core dot products, 128 for the tensor-core
+// path, which keeps a fourth, all-zero limb slot (the B operand columns of no limb read it).
+constexpr int kLimbVecs = 32;
 
 template <int G>
 struct __align__(16) WarpSmem {
   uint8_t buf[ring_buffers<G>()][buf_bytes<G>()];
-  uint4 qw[G][limb_vecs<G>()];  // Q limbs of each query
-  uint4 pw[G][limb_vecs<G>()];  // P limbs of each query
+  uint4 qw[G][kLimbVecs];  // Q limbs of each query
+  uint4 pw[G][kLimbVecs];  // P limbs of each query
   uint64_t bar[ring_buffers<G>()];
 };
 
@@ -193,8 +189,12 @@ struct Decoder {
   static constexpr int ROWS = UT / P;              // V word rows per unit (8)
   static constexpr int kBuffers = ring_buffers<G>();
   static constexpr int GP = G == 1 ? 1 : 2;        // queries per pass over a unit's codes
-  // 2 bits with one query per KV head: the byte dot products run on the tensor cores (mma.sync)
-  static constexpr bool kMma = BITS == 2 && G == 1;
+  // 2 bits: the byte dot products run on the tensor cores (mma.sync); one query per KV head pairs
+  // two token (channel) tiles per accumulator, several queries pair two queries per accumulator
+  static constexpr bool kMma = BITS == 2;
+  static constexpr bool kMma1 = kMma && G == 1;
+  static constexpr bool kMmaG = kMma && G > 1;
+  static constexpr int NBLK = G / 2;  // several queries: n8 blocks of queries (2 p, 2 p + 1)
 
   const DecodeArgs& a;
   WarpSmem<G>& S;
@@ -215,6 +215,7 @@ struct Decoder {
   // state handed from the K half to the V half of a unit
   float alpha_[G], invv_[G], pres_[G];
   bool hasv_[G];
+  bool omma_;  // o is in the tensor-core layout of several queries (see o_swap_layout)
   // bytes per head of the code arrays and of a residual array; this lane's scale role
   const size_t code_head_bytes, res_head_bytes;
   const bool k_lane, v_lane;
@@ -307,7 +308,18 @@ struct Decoder {
     }
     qkey = -1;
     qhead = head;
+    omma_ = kMmaG;  // o is zero: either layout
     __syncwarp();
+  }
+
+  // Residual units and the merge read o in the residual layout.
+  __device__ __forceinline__ void residual_layout() {
+    if constexpr (kMmaG) {
+      if (omma_) {
+        o_swap_layout();
+        omma_ = false;
+      }
+    }
   }
 
   // This lane's q channel j of query g (scaled by scale * log2 e): channel 16 (lane / 4) + 4 j +
@@ -394,25 +406,28 @@ struct Decoder {
     const int gi = (16 * (lane >> 2)) >> a.lg_gk;  // the K group of all four channels
     const float s = h2f(static_cast<uint16_t>(__shfl_sync(kFull, pairs, gi) & 0xFFFFu));
     const float z_own = k_lane ? h2f(static_cast<uint16_t>(pairs >> 16)) : 0.f;
-    float qv[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) qv[j] = q_of(0, j) * s;
-    const float mabs = warp_max(fmaxf(fmaxf(fabsf(qv[0]), fabsf(qv[1])), fmaxf(fabsf(qv[2]), fabsf(qv[3]))));
-    const float scq = mabs > 0.f ? kQRangeBal * fast_rcp(mabs) : 0.f;
-    invq[0] = mabs * (1.0f / kQRangeBal);
-    float c = z_own * qsum[0][0];
-    c += __shfl_xor_sync(kFull, c, 1);
-    c += __shfl_xor_sync(kFull, c, 2);
-    cblk[0] = __shfl_sync(kFull, c, 0);
-    const float f = scq * ((lane & 1) ? 0.25f : 1.f);
-    uint32_t Q[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) Q[j] = static_cast<uint32_t>(__float2int_rn(qv[j] * f));
     const int i = lane >> 2, sw = (i >> 1) & 3;
-    uint32_t* row = reinterpret_cast<uint32_t*>(S.qw[0]) + 16 * i + (lane & 3);
-    row[4 * (0 ^ sw)] = pick_bytes(Q[0] + 32896u, Q[1] + 32896u, Q[2] + 32896u, Q[3] + 32896u, 2);
-    row[4 * (1 ^ sw)] = pick_bytes(Q[0] + 128u, Q[1] + 128u, Q[2] + 128u, Q[3] + 128u, 1);
-    row[4 * (2 ^ sw)] = pick_bytes(Q[0], Q[1], Q[2], Q[3], 0);
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      float qv[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) qv[j] = q_of(g, j) * s;
+      const float mabs = warp_max(fmaxf(fmaxf(fabsf(qv[0]), fabsf(qv[1])), fmaxf(fabsf(qv[2]), fabsf(qv[3]))));
+      const float scq = mabs > 0.f ? kQRangeBal * fast_rcp(mabs) : 0.f;
+      invq[g] = mabs * (1.0f / kQRangeBal);
+      float c = z_own * qsum[g][0];
+      c += __shfl_xor_sync(kFull, c, 1);
+      c += __shfl_xor_sync(kFull, c, 2);
+      cblk[g] = __shfl_sync(kFull, c, 0);
+      const float f = scq * ((lane & 1) ? 0.25f : 1.f);
+      uint32_t Q[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) Q[j] = static_cast<uint32_t>(__float2int_rn(qv[j] * f));
+      uint32_t* row = reinterpret_cast<uint32_t*>(S.qw[g]) + 16 * i + (lane & 3);
+      row[4 * (0 ^ sw)] = pick_bytes(Q[0] + 32896u, Q[1] + 32896u, Q[2] + 32896u, Q[3] + 32896u, 2);
+      row[4 * (1 ^ sw)] = pick_bytes(Q[0] + 128u, Q[1] + 128u, Q[2] + 128u, Q[3] + 128u, 1);
+      row[4 * (2 ^ sw)] = pick_bytes(Q[0], Q[1], Q[2], Q[3], 0);
+    }
   }
 
   // Logits of the unit's 128 tokens.  Tile 2 j + b holds tokens 32 j + 16 b + (0..15) as rows;
@@ -566,6 +581,179 @@ struct Decoder {
     }
   }
 
+  // ---- tensor-core path, several queries per KV head ------------------------------------------
+  // B column n of n8 block p reads slot n % 4 of query 2 p + n / 4, so one accumulator holds the
+  // three limbs of queries 2 p (columns 0..2) and 2 p + 1 (columns 4..6) for one 16-row tile.  After
+  // the exchange a lane holds query 2 p + t / 2 of row g + 8 (t % 2).
+  //
+  // Output layout while quantized units run: o[2 p + b][v] of lane (g, t) holds query 2 p + t / 2,
+  // channel 16 g + 8 b + 4 (t % 2) + v.  o_swap_layout() turns it into the layout of the residual
+  // path and the merge (o[q][e]: query q, channel 4 lane + e) and back: it is an involution.
+
+  // Logits of the unit's 128 tokens for every query: tile tau holds tokens 16 tau + (0..15) as
+  // rows; lg[p][tau] is the logit of query 2 p + t / 2 for token 16 tau + 8 (t % 2) + g.
+  __device__ void k_mma_g(const uint8_t* kt, float (&lg)[NBLK][8]) const {
+    const int g = lane >> 2, t = lane & 3, qh = g >> 2, sl = (g & 3) ^ t;
+    const bool odd = t & 1;
+    uint4 B[NBLK][2];
+#pragma unroll
+    for (int p = 0; p < NBLK; ++p) {
+      B[p][0] = S.qw[2 * p + qh][8 * t + sl];
+      B[p][1] = S.qw[2 * p + qh][8 * t + 4 + sl];
+    }
+    float iq[NBLK], cb[NBLK];
+#pragma unroll
+    for (int p = 0; p < NBLK; ++p) {
+      iq[p] = (t >> 1) ? invq[2 * p + 1] : invq[2 * p];
+      cb[p] = (t >> 1) ? cblk[2 * p + 1] : cblk[2 * p];
+    }
+#pragma unroll
+    for (int tau = 0; tau < 8; ++tau) {
+      const uint8_t* r0 = kt + (16 * tau + g) * 32 + 8 * t;
+      const uint2 wg = *reinterpret_cast<const uint2*>(r0);
+      const uint2 wh = *reinterpret_cast<const uint2*>(r0 + 8 * 32);
+      int c[NBLK][4];
+#pragma unroll
+      for (int p = 0; p < NBLK; ++p) c[p][0] = c[p][1] = c[p][2] = c[p][3] = 0;
+#pragma unroll
+      for (int w = 0; w < 2; ++w) {
+        uint32_t mg[4], mh[4];
+        masks2(w ? wg.y : wg.x, mg);
+        masks2(w ? wh.y : wh.x, mh);
+#pragma unroll
+        for (int p = 0; p < NBLK; ++p) {
+          mma_u8s8(c[p], mg[0], mh[0], mg[1], mh[1], B[p][w].x, B[p][w].y);
+          mma_u8s8(c[p], mg[2], mh[2], mg[3], mh[3], B[p][w].z, B[p][w].w);
+        }
+      }
+#pragma unroll
+      for (int p = 0; p < NBLK; ++p) lg[p][tau] = fmaf(gather_limbs(c[p], odd), iq[p], cb[p]);
+    }
+  }
+
+  // Online softmax of every query over the unit and the P limbs of each query (bound scaling as on
+  // the other paths).  Token 16 tau + ... lies in V group (16 tau) >> lg_gv of the unit; its P goes
+  // to byte (g / 4) + 2 (t % 2) of word (tau, slot, g % 4) of its query.
+  __device__ void softmax_mma_g(uint32_t pairs, const float (&lg)[NBLK][8]) {
+    const int g = lane >> 2, t = lane & 3, h = t >> 1;
+    const float smax = warp_max(v_lane ? h2f(static_cast<uint16_t>(pairs & 0xFFFFu)) : 0.f);
+    const float kinv = smax > 0.f ? kPRange * fast_rcp(smax) : 0.f;
+    const float set_scale = (g & 1) ? 0.25f : 1.f;
+    float sv[8], zv[8];
+#pragma unroll
+    for (int tau = 0; tau < 8; ++tau) {
+      const uint32_t vp = __shfl_sync(kFull, pairs, 8 + ((16 * tau) >> a.lg_gv));
+      sv[tau] = h2f(static_cast<uint16_t>(vp & 0xFFFFu));
+      zv[tau] = h2f(static_cast<uint16_t>(vp >> 16));
+    }
+#pragma unroll
+    for (int p = 0; p < NBLK; ++p) {
+      float mloc = lg[p][0];
+#pragma unroll
+      for (int tau = 1; tau < 8; ++tau) mloc = fmaxf(mloc, lg[p][tau]);
+      float mn_l = 0.f, fb = 0.f;
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int q = 2 * p + e;
+        const float mu = warp_max(h == e ? mloc : -INFINITY);
+        const float m_new = fmaxf(m[q], mu);
+        const float d = mu - m_new;
+        const bool hv = d > -64.f && smax > 0.f;
+        alpha_[q] = fast_exp2(m[q] - m_new);
+        hasv_[q] = hv;
+        invv_[q] = hv ? fast_exp2(d) * smax * (1.0f / kPRange) : 0.f;
+        m[q] = m_new;
+        if (h == e) {
+          mn_l = m_new;
+          fb = hv ? kinv * fast_exp2(-d) * set_scale : 0.f;
+        }
+      }
+      uint8_t* pb = reinterpret_cast<uint8_t*>(S.pw[2 * p + h]) + 4 * (g & 3) + (g >> 2) + 2 * (t & 1);
+      float psum = 0.f, zsum = 0.f;
+#pragma unroll
+      for (int tau = 0; tau < 8; ++tau) {
+        const float pv = fast_exp2(lg[p][tau] - mn_l);
+        psum += pv;
+        zsum = fmaf(pv, zv[tau], zsum);
+        const uint32_t P = __float2uint_rn(pv * (sv[tau] * fb));
+        const int sw = (tau >> 1) & 3;
+        pb[64 * tau + 16 * (0 ^ sw)] = static_cast<uint8_t>(P >> 16);
+        pb[64 * tau + 16 * (1 ^ sw)] = static_cast<uint8_t>(P >> 8);
+        pb[64 * tau + 16 * (2 ^ sw)] = static_cast<uint8_t>(P);
+      }
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int q = 2 * p + e;
+        l[q] = fmaf(l[q], alpha_[q], h == e ? psum : 0.f);
+        Z[q] = fmaf(Z[q], alpha_[q], h == e ? zsum : 0.f);
+      }
+    }
+  }
+
+  // P . codes of the unit for every query.  Tile (v, b) holds channels 16 g' + 8 b + 4 c + v (row
+  // g' + 8 c); lane (g, t) unpacks V word rows 2 t + x of channels 16 g .. 16 g + 15.
+  __device__ void v_mma_g(const uint8_t* vt) {
+    const int g = lane >> 2, t = lane & 3, qh = g >> 2, sl = (g & 3) ^ t;
+    const bool odd = t & 1;
+    uint4 B[NBLK][2];
+#pragma unroll
+    for (int p = 0; p < NBLK; ++p) {
+      B[p][0] = S.pw[2 * p + qh][8 * t + sl];
+      B[p][1] = S.pw[2 * p + qh][8 * t + 4 + sl];
+    }
+    float al[NBLK], iv[NBLK];
+#pragma unroll
+    for (int p = 0; p < NBLK; ++p) {
+      al[p] = (t >> 1) ? alpha_[2 * p + 1] : alpha_[2 * p];
+      iv[p] = (t >> 1) ? invv_[2 * p + 1] : invv_[2 * p];
+    }
+#pragma unroll
+    for (int b = 0; b < 2; ++b) {
+      int acc[4][NBLK][4];
+#pragma unroll
+      for (int v = 0; v < 4; ++v)
+#pragma unroll
+        for (int p = 0; p < NBLK; ++p) acc[v][p][0] = acc[v][p][1] = acc[v][p][2] = acc[v][p][3] = 0;
+#pragma unroll
+      for (int x = 0; x < 2; ++x) {
+        const uint8_t* rowp = vt + t * kVPieceStride + x * 512 + 64 * g;
+        const uint4 wlo = *reinterpret_cast<const uint4*>(rowp + 32 * b);
+        const uint4 whi = *reinterpret_cast<const uint4*>(rowp + 32 * b + 16);
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+          uint32_t mg[4], mh[4];
+          masks2(comp(wlo, v), mg);
+          masks2(comp(whi, v), mh);
+#pragma unroll
+          for (int p = 0; p < NBLK; ++p) {
+            mma_u8u8(acc[v][p], mg[0], mh[0], mg[1], mh[1], B[p][x].x, B[p][x].y);
+            mma_u8u8(acc[v][p], mg[2], mh[2], mg[3], mh[3], B[p][x].z, B[p][x].w);
+          }
+        }
+      }
+#pragma unroll
+      for (int v = 0; v < 4; ++v)
+#pragma unroll
+        for (int p = 0; p < NBLK; ++p)
+          o[2 * p + b][v] = fmaf(o[2 * p + b][v], al[p], gather_limbs(acc[v][p], odd) * iv[p]);
+    }
+  }
+
+  // Swaps o[2 p + 1 - t / 2][v] with lane t ^ 2: the tensor-core layout <-> the residual layout.
+  __device__ void o_swap_layout() {
+    const bool h = (lane >> 1) & 1;
+#pragma unroll
+    for (int p = 0; p < NBLK; ++p)
+#pragma unroll
+      for (int v = 0; v < 4; ++v) {
+        const float y = __shfl_xor_sync(kFull, h ? o[2 * p][v] : o[2 * p + 1][v], 2);
+        if (h)
+          o[2 * p][v] = y;
+        else
+          o[2 * p + 1][v] = y;
+      }
+  }
+
   // ---- A6 over the K codes of a unit: integer dot products of TPL tokens per lane, for every
   // query of the KV head (each code word is unpacked once) -----------------------------------------
   // Queries g0 .. g0 + GP - 1 (the accumulators of one pass).
@@ -691,10 +879,14 @@ struct Decoder {
       build_q(pairs);
       qkey = key;
     }
-    if constexpr (kMma) {
+    if constexpr (kMma1) {
       float lg[4];
       k_mma(kt, lg);
       softmax_mma(pairs, lg);
+    } else if constexpr (kMmaG) {
+      float lg[NBLK][8];
+      k_mma_g(kt, lg);
+      softmax_mma_g(pairs, lg);
     } else if constexpr (BITS == 2) {
       const VScales vs = v_scales2(pairs);  // independent of the dot products: issued first
 #pragma unroll
@@ -768,8 +960,10 @@ struct Decoder {
     if (G == 1 && !hasv_[0]) {  // every weight of the unit is zero: only rescale
 #pragma unroll
       for (int e = 0; e < 4; ++e) o[0][e] *= alpha_[0];
-    } else if constexpr (kMma) {
+    } else if constexpr (kMma1) {
       v_mma(vt);
+    } else if constexpr (kMmaG) {
+      v_mma_g(vt);
     } else {
       dot_v(vt);
     }
@@ -911,6 +1105,7 @@ struct Decoder {
 
   // ---- end of a head segment: write the output, or a partial and maybe merge ----------------
   __device__ void finish_segment(long long head, long long seg_a, long long seg_b) {
+    residual_layout();
     const long long h0 = head * a.units, h1 = h0 + a.units;
     float lsum[G], zsum[G];
 #pragma unroll
@@ -1044,9 +1239,9 @@ struct Decoder {
       asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     if constexpr (kMma) {  // slot 3 of every limb row stays zero; slots 0..2 are written before use
-      for (int i = lane; i < 4 * limb_vecs<G>(); i += 32) {
-        reinterpret_cast<uint32_t*>(S.qw[0])[i] = 0u;
-        reinterpret_cast<uint32_t*>(S.pw[0])[i] = 0u;
+      for (int i = lane; i < 4 * kLimbVecs * G; i += 32) {
+        reinterpret_cast<uint32_t*>(S.qw)[i] = 0u;
+        reinterpret_cast<uint32_t*>(S.pw)[i] = 0u;
       }
     }
     __syncwarp();
@@ -1084,10 +1279,12 @@ struct Decoder {
         drain_from(hk, nhalves);
         return;
       }
-      if (quant)
+      if (quant) {
         quantized_k(S.buf[hk % kBuffers], head, local, pairs);
-      else
+      } else {
+        residual_layout();
         residual_k(S.buf[hk % kBuffers], nvalid, head, local - a.units_q);
+      }
       __syncwarp();
       fence_proxy_async_smem();
       // half hk + kBuffers reuses the buffer just consumed: the next unit's V (ring of 3) or K (2)
