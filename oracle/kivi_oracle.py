@@ -25,6 +25,12 @@ Readings taken where the page leaves a step open (each is pinned by tests/test_o
   * Decode attention follows the Attention equation of section 残差バッファ: logits over the
     dequantized quantized tokens followed by the fp16 residual tokens, softmax, weighted sum of
     the matching V rows.  No mask; the query-head -> KV-head map is contiguous (h // (Hq/H)).
+  * Online K (an opt-in variant, section Per-Channel量子化: a new token's K can be quantized at
+    once with the existing scale and zero point): once a quantized block exists, every new K row
+    is coded at append time with the (s, z) of the newest quantized block, clamped to [0, 2^b-1];
+    the block being filled keeps a copy of those (s, z).  No K row stays fp16; V keeps its fp16
+    residual and is quantized when the residual fills, as in the base scheme.  Before the first
+    block exists there are no scales to reuse and K stays in the fp16 residual.
 
 Parity pinned: every public function below is pinned by at least one test that does not reuse
 its code (exact rationals, nearest-grid-point brute force, hand-derived fixtures, closed forms,
@@ -179,12 +185,14 @@ def unpack_v(words, bits: int) -> np.ndarray:
 
 def dequantize_k(codes, s, z, block: int, group_k: int) -> np.ndarray:
     """D(K^) = s*K^ + z in float64 with the (block, channel group) scale of each element (section
-    量子化アルゴリズム, D equation).  codes uint8 [n][d]; s, z fp16 [n/block][d/group_k]."""
+    量子化アルゴリズム, D equation).  codes uint8 [n][d]; s, z fp16 [ceil(n/block)][d/group_k] (the
+    last block may be partly filled)."""
     codes = np.asarray(codes, dtype=np.float64)
+    n = codes.shape[0]
     s64 = np.asarray(s, dtype=np.float16).astype(np.float64)
     z64 = np.asarray(z, dtype=np.float16).astype(np.float64)
-    s_full = np.repeat(np.repeat(s64, block, axis=0), group_k, axis=1)
-    z_full = np.repeat(np.repeat(z64, block, axis=0), group_k, axis=1)
+    s_full = np.repeat(np.repeat(s64, block, axis=0), group_k, axis=1)[:n]
+    z_full = np.repeat(np.repeat(z64, block, axis=0), group_k, axis=1)[:n]
     return s_full * codes + z_full
 
 
@@ -212,12 +220,15 @@ def attention(q, keys, values, scale: float) -> np.ndarray:
 class HeadCache:
     """Quantized cache of one (batch, KV head): quantized blocks plus the fp16 residual.
 
-    Mirrors the library's counters: n_quant (a multiple of R) and n_res in [0, R]."""
+    Mirrors the library's counters: n_quant (a multiple of R) and n_res in [0, R].  With online_k,
+    k_codes also holds the n_res online-coded rows after the n_quant block rows and k_s / k_z
+    hold one row for the block being filled."""
 
     def __init__(self, head_dim: int, bits: int, group_k: int, group_v: int, residual: int,
-                 capacity: int):
+                 capacity: int, online_k: bool = False):
         self.d, self.bits, self.gk, self.gv = head_dim, bits, group_k, group_v
         self.R, self.capacity = residual, capacity
+        self.online_k = bool(online_k)
         self.k_codes = np.zeros((0, head_dim), np.uint8)
         self.v_codes = np.zeros((0, head_dim), np.uint8)
         self.k_s = np.zeros((0, head_dim // group_k), np.float16)
@@ -229,11 +240,29 @@ class HeadCache:
 
     @property
     def n_quant(self) -> int:
-        return self.k_codes.shape[0]
+        return self.v_codes.shape[0]
 
     @property
     def n_res(self) -> int:
-        return self.k_res.shape[0]
+        return self.v_res.shape[0]
+
+    @property
+    def k_online(self) -> bool:
+        """True when new K rows are coded at append time (online_k and a quantized block exists)."""
+        return self.online_k and self.n_quant > 0
+
+    def _code_online(self, rows):
+        """Codes K rows with the (s, z) of the newest quantized block (section Per-Channel量子化:
+        quantize a new token at once with the existing scale and zero point); the block being
+        filled gets a copy of that (s, z) row when its first row arrives."""
+        rows = np.asarray(rows, np.float16).reshape(-1, self.d)
+        last = self.n_quant // self.R - 1
+        s, z = self.k_s[last], self.k_z[last]
+        if self.k_s.shape[0] == self.n_quant // self.R:
+            self.k_s = np.concatenate([self.k_s, s[None, :]])
+            self.k_z = np.concatenate([self.k_z, z[None, :]])
+        codes = quantize_values(rows, np.repeat(s, self.gk)[None, :], np.repeat(z, self.gk)[None, :], self.bits)
+        self.k_codes = np.concatenate([self.k_codes, codes])
 
     def _quantize_block(self, kblk, vblk):
         kc, ks, kz = quantize_k_block(kblk, self.gk, self.bits)
@@ -258,12 +287,17 @@ class HeadCache:
         n_quant = T - n_res
         if n_quant > self.capacity:
             raise OracleError("CAPACITY", f"{n_quant} > {self.capacity}")
-        self.__init__(self.d, self.bits, self.gk, self.gv, self.R, self.capacity)
+        self.__init__(self.d, self.bits, self.gk, self.gv, self.R, self.capacity, self.online_k)
         for j in range(n_quant // self.R):
             sl = slice(j * self.R, (j + 1) * self.R)
             self._quantize_block(k[sl], v[sl])
-        self.k_res = k[n_quant:].copy()
         self.v_res = v[n_quant:].copy()
+        if self.k_online:
+            if n_quant + self.R > self.capacity:
+                raise OracleError("CAPACITY", "no block slot for the online K rows")
+            self._code_online(k[n_quant:])
+        else:
+            self.k_res = k[n_quant:].copy()
 
     def prefill_prefix_k(self, k, v):
         """Prefill under the other reading of section Per-Channel量子化, in which one K group spans
@@ -280,7 +314,7 @@ class HeadCache:
         n_quant = T - n_res
         if n_quant > self.capacity:
             raise OracleError("CAPACITY", f"{n_quant} > {self.capacity}")
-        self.__init__(self.d, self.bits, self.gk, self.gv, self.R, self.capacity)
+        self.__init__(self.d, self.bits, self.gk, self.gv, self.R, self.capacity, self.online_k)
         if n_quant:
             kc, ks, kz = quantize_k_block(k[:n_quant], self.gk, self.bits)
             self.k_codes = kc
@@ -295,10 +329,16 @@ class HeadCache:
         self.v_res = v[n_quant:].copy()
 
     def append(self, k_new, v_new):
-        """Writes the newest token into the fp16 residual (section 残差バッファ)."""
+        """Writes the newest token into the fp16 residual (section 残差バッファ); with online K its
+        K row is coded at once instead (section Per-Channel量子化)."""
         if self.n_res == self.R:
             raise OracleError("RESIDUAL_FULL")
-        self.k_res = np.concatenate([self.k_res, np.asarray(k_new, np.float16)[None, :]])
+        if self.k_online:
+            if self.n_quant + self.R > self.capacity:
+                raise OracleError("CAPACITY", "no block slot for the online K row")
+            self._code_online(k_new)
+        else:
+            self.k_res = np.concatenate([self.k_res, np.asarray(k_new, np.float16)[None, :]])
         self.v_res = np.concatenate([self.v_res, np.asarray(v_new, np.float16)[None, :]])
 
     def flush(self):
@@ -308,12 +348,19 @@ class HeadCache:
             raise OracleError("RESIDUAL_NOT_FULL")
         if self.n_quant + self.R > self.capacity:
             raise OracleError("CAPACITY")
-        self._quantize_block(self.k_res, self.v_res)
+        if self.k_online:  # K rows are coded already; the block keeps its copied (s, z)
+            vc, vs, vz = quantize_v_block(self.v_res, self.gv, self.bits)
+            self.v_codes = np.concatenate([self.v_codes, vc])
+            self.v_s = np.concatenate([self.v_s, vs])
+            self.v_z = np.concatenate([self.v_z, vz])
+        else:
+            self._quantize_block(self.k_res, self.v_res)
         self.k_res = np.zeros((0, self.d), np.float16)
         self.v_res = np.zeros((0, self.d), np.float16)
 
     def keys(self) -> np.ndarray:
-        """[D(K_quant); K_res] as float64 [n_quant + n_res][d]."""
+        """[D(K_quant); K_res] as float64 [n_quant + n_res][d] (with online K every row is
+        dequantized)."""
         kd = dequantize_k(self.k_codes, self.k_s, self.k_z, self.R, self.gk)
         return np.concatenate([kd, self.k_res.astype(np.float64)])
 
@@ -344,11 +391,11 @@ class OracleCache:
 
     def __init__(self, batch: int, num_kv_heads: int, head_dim: int = 128, bits: int = 2,
                  group_k: int = 32, group_v: int = 32, residual: int = 128, capacity: int = 0,
-                 heads=None):
+                 heads=None, online_k: bool = False):
         self.B, self.H = batch, num_kv_heads
         self.heads = sorted(heads) if heads is not None else [
             (b, h) for b in range(batch) for h in range(num_kv_heads)]
-        self.cache = {bh: HeadCache(head_dim, bits, group_k, group_v, residual, capacity)
+        self.cache = {bh: HeadCache(head_dim, bits, group_k, group_v, residual, capacity, online_k)
                       for bh in self.heads}
 
     def _counters(self):

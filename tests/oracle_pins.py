@@ -315,6 +315,85 @@ def check_prefix_k_groups(O, bits, group):
     assert np.array_equal(h.k_s[3], ks) and np.array_equal(h.k_codes[n_q:], kc)
 
 
+def check_online_k(O, bits, group):
+    """Online K (section Per-Channel量子化: a new token's K is quantized at once with the existing
+    scale and zero point).  Every online row is the nearest grid point of the newest quantized
+    block's stored (s, z), found by search over the 2^b levels with exact rationals (clamping
+    included); rows copied from that block get that block's codes; blocks, V and counters equal
+    the base scheme's; the copied (s, z) carries over flushes; before any block exists K stays in
+    fp16 and the first flush quantizes it as the base scheme does."""
+    rng = np.random.default_rng(131 + bits + group)
+    R, d = 128, 128
+    T = 2 * R + 37
+    k = (rng.standard_normal((T, d)) * np.exp2(rng.integers(-2, 3, (1, d)))).astype(np.float16)
+    k[R:2 * R, 3] *= np.float16(9)          # block 1's range differs from block 0's in group 3 // group
+    v = rng.standard_normal((T, d)).astype(np.float16)
+    h = O.HeadCache(d, bits, group, group, R, 8 * R, online_k=True)
+    h.prefill(k, v)
+    ref = O.HeadCache(d, bits, group, group, R, 8 * R)
+    ref.prefill(k, v)
+    assert (h.n_quant, h.n_res) == (ref.n_quant, ref.n_res) == (2 * R, 37)
+    assert h.k_res.shape[0] == 0 and h.k_codes.shape[0] == T and h.k_s.shape[0] == 3
+    assert np.array_equal(h.k_codes[:2 * R], ref.k_codes) and np.array_equal(h.k_s[:2], ref.k_s)
+    assert np.array_equal(h.k_s[2], ref.k_s[1]) and np.array_equal(h.k_z[2], ref.k_z[1])
+    assert ref.k_s[0, 3 // group] != ref.k_s[1, 3 // group]
+    for key in ("v_codes", "v_s", "v_z", "v_res"):
+        assert np.array_equal(getattr(h, key), getattr(ref, key)), key
+
+    def nearest(row_k, row_codes):
+        for c in range(0, d, 3):
+            g = c // group
+            want = code_nearest_grid(_fr(row_k[c]), _fr(ref.k_s[1, g]), _fr(ref.k_z[1, g]), bits)
+            assert row_codes[c] == want, (c, row_codes[c], want)
+
+    for i in range(2 * R, T, 5):
+        nearest(k[i], h.k_codes[i])
+    # appends: copies of block-1 rows, rows far outside its range (clamped), then fill and flush
+    n0 = h.k_codes.shape[0]
+    for j in range(10):
+        h.append(k[R + 7 * j], v[j])
+    assert np.array_equal(h.k_codes[n0:n0 + 10], ref.k_codes[R + 7 * np.arange(10)])
+    wide = (rng.standard_normal((6, d)) * 40).astype(np.float16)
+    for j in range(6):
+        h.append(wide[j], v[j])
+        nearest(wide[j], h.k_codes[-1])
+    assert set(np.unique(h.k_codes[-6:])) >= {0, 2 ** bits - 1}
+    while h.n_res < R:
+        h.append(k[h.n_res], v[h.n_res])
+    vres = h.v_res.copy()
+    h.flush()
+    vc, vs, vz = O.quantize_v_block(vres, group, bits)
+    assert (h.n_quant, h.n_res) == (3 * R, 0) and h.k_codes.shape[0] == 3 * R
+    assert np.array_equal(h.v_codes[2 * R:], vc) and np.array_equal(h.v_s[2 * R // group:], vs)
+    assert np.array_equal(h.k_s[2], ref.k_s[1])
+    h.append(wide[0], v[0])
+    assert h.k_s.shape[0] == 4 and np.array_equal(h.k_s[3], ref.k_s[1]) and np.array_equal(h.k_z[3], ref.k_z[1])
+    # dequantized keys of online rows: s * code + z with the carried (s, z), exactly
+    keys = h.keys()
+    for i in (2 * R + 1, 3 * R):
+        for c in (0, 3, 77):
+            g = c // group
+            assert Fraction(float(keys[i, c])) == _fr(ref.k_s[1, g]) * int(h.k_codes[i, c]) + _fr(ref.k_z[1, g])
+    # no block yet: K stays fp16, the first flush quantizes it as the base scheme does
+    e = O.HeadCache(d, bits, group, group, R, 8 * R, online_k=True)
+    b = O.HeadCache(d, bits, group, group, R, 8 * R)
+    e.prefill(k[:50], v[:50])
+    b.prefill(k[:50], v[:50])
+    assert e.k_res.shape[0] == 50 and e.k_codes.shape[0] == 0
+    for t in range(50, R):
+        e.append(k[t], v[t])
+        b.append(k[t], v[t])
+    e.flush()
+    b.flush()
+    for key, want in b.packed().items():
+        assert np.array_equal(np.asarray(e.packed()[key]).view(np.uint8), np.asarray(want).view(np.uint8)), key
+    e.append(k[R + 1], v[0])
+    kc0, ks0, kz0 = O.quantize_k_block(k[:R], group, bits)
+    nearest_codes = [code_nearest_grid(_fr(k[R + 1, c]), _fr(ks0[c // group]), _fr(kz0[c // group]), bits)
+                     for c in range(d)]
+    assert list(e.k_codes[R]) == nearest_codes and e.k_res.shape[0] == 0
+
+
 def check_errors(O):
     h = _head(O, cap=128)
     k = np.zeros((128, 128), np.float16)

@@ -164,3 +164,32 @@ def test_prefix_pin_catches_mutant(mutant, monkeypatch):
     monkeypatch.setattr(O.HeadCache, "prefill_prefix_k", mutant)
     with pytest.raises(AssertionError):
         pins.check_prefix_k_groups(O, 2, 32)
+
+
+def _online_first_block(self, rows):                  # reuses the oldest block's (s, z), not the newest
+    rows = np.asarray(rows, np.float16).reshape(-1, self.d)
+    s, z = self.k_s[0], self.k_z[0]
+    if self.k_s.shape[0] == self.n_quant // self.R:
+        self.k_s = np.concatenate([self.k_s, self.k_s[-1][None, :]])
+        self.k_z = np.concatenate([self.k_z, self.k_z[-1][None, :]])
+    codes = O.quantize_values(rows, np.repeat(s, self.gk)[None, :], np.repeat(z, self.gk)[None, :], self.bits)
+    self.k_codes = np.concatenate([self.k_codes, codes])
+
+
+def _online_no_clamp(self, rows):                     # rounds without clamping to [0, 2^b - 1]
+    rows = np.asarray(rows, np.float16).reshape(-1, self.d)
+    last = self.n_quant // self.R - 1
+    s, z = self.k_s[last], self.k_z[last]
+    if self.k_s.shape[0] == self.n_quant // self.R:
+        self.k_s = np.concatenate([self.k_s, s[None, :]])
+        self.k_z = np.concatenate([self.k_z, z[None, :]])
+    s64 = np.repeat(s, self.gk).astype(np.float64)
+    r = np.rint((rows.astype(np.float64) - np.repeat(z, self.gk).astype(np.float64)) / np.where(s64 == 0, 1, s64))
+    self.k_codes = np.concatenate([self.k_codes, (r.astype(np.int64) & 0xFF).astype(np.uint8)])
+
+
+@pytest.mark.parametrize("mutant", [_online_first_block, _online_no_clamp], ids=["first_block", "no_clamp"])
+def test_online_pin_catches_mutant(mutant, monkeypatch):
+    monkeypatch.setattr(O.HeadCache, "_code_online", mutant)
+    with pytest.raises(AssertionError):
+        pins.check_online_k(O, 2, 32)

@@ -71,3 +71,8 @@ def test_attention_bruteforce_from_packed_words(bits, group):
 @pytest.mark.parametrize("bits,group", [(2, 32), (4, 64), (2, 128)])
 def test_prefix_k_groups(bits, group):
     pins.check_prefix_k_groups(O, bits, group)
+
+
+@pytest.mark.parametrize("bits,group", [(2, 32), (4, 64), (2, 128)])
+def test_online_k(bits, group):
+    pins.check_online_k(O, bits, group)
