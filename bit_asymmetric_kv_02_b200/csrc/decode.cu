@@ -181,7 +181,9 @@ __device__ __forceinline__ void dot_set(uint32_t m, uint32_t L, uint32_t M, uint
   ah = signed_hi ? dp4a_us(m, H, ah) : dp4a_uu(m, H, ah);
 }
 
-template <int BITS, int G>
+// KC: the residual tokens' K rows are codes (online K); a separate instantiation keeps that path
+// out of the register allocation of the others.
+template <int BITS, int G, bool KC>
 struct Decoder {
   static constexpr int P = 32 / BITS;              // codes per word
   static constexpr int UT = BITS == 2 ? 128 : 64;  // tokens per quantized unit (8 KB of codes)
@@ -240,6 +242,14 @@ struct Decoder {
     const size_t stride = quant ? code_head_bytes : res_head_bytes;
     const int unit = quant ? local : local - a.units_q;
     const char* src = base + static_cast<size_t>(head) * stride + static_cast<size_t>(unit) * kHalfBytes;
+    if (KC && !quant && !is_v) {  // online K: 16 code rows from token n_quant + 16 unit
+      constexpr uint32_t kRowBytes = kHeadDim * BITS / 8;
+      src = reinterpret_cast<const char*>(a.k_codes) + static_cast<size_t>(head) * code_head_bytes +
+            (static_cast<size_t>(a.n_quant) + static_cast<size_t>(unit) * kResTokens) * kRowBytes;
+      mbar_arrive_expect_tx(&S.bar[b], kResTokens * kRowBytes + a.debug_extra_tx);
+      bulk_g2s(S.buf[b], src, kResTokens * kRowBytes, &S.bar[b]);
+      return;
+    }
     mbar_arrive_expect_tx(&S.bar[b], kHalfBytes + a.debug_extra_tx);
     if (kMma && is_v) {
 #pragma unroll
@@ -1046,7 +1056,67 @@ struct Decoder {
     __syncwarp();
   }
 
+  // K half of a residual unit under online K: 16 rows of codes, dequantized with block res_blk's
+  // (s, z) (section Per-Channel量子化: the block being filled carries the newest block's pair).
+  // Two lanes per token, 64 channels each; a code word lies in one K group (G_k >= 32 >= P).
+  __device__ void residual_k_coded(const uint8_t* kt, int nvalid, long long head) {
+    constexpr int kRowBytes = kHeadDim * BITS / 8, WPL = 64 / P;
+    constexpr uint32_t L = (1u << BITS) - 1u;
+    const int t = lane >> 1, hf = lane & 1;
+    const size_t sb = (static_cast<size_t>(head) * a.blocks_per_head + a.res_blk) * ngk;
+    uint32_t w[WPL];
+#pragma unroll
+    for (int i = 0; i < WPL; i += 4) {
+      const uint4 v4 = *reinterpret_cast<const uint4*>(kt + t * kRowBytes + hf * (kRowBytes / 2) + 4 * i);
+      w[i] = v4.x;
+      w[i + 1] = v4.y;
+      w[i + 2] = v4.z;
+      w[i + 3] = v4.w;
+    }
+#pragma unroll  // the per-query state must stay in registers: no runtime index into it
+    for (int g = 0; g < G; ++g) {
+      const uint4* qp = reinterpret_cast<const uint4*>(a.q + (static_cast<size_t>(head) * G + g) * kHeadDim + 64 * hf);
+      float dot = 0.f;
+#pragma unroll
+      for (int i = 0; i < WPL; ++i) {
+        const int gi = (64 * hf + P * i) >> a.lg_gk;
+        const float sk = h2f(__ldg(a.k_scale + sb + gi)), zk = h2f(__ldg(a.k_zero + sb + gi));
+        float acc = 0.f, qs = 0.f;
+#pragma unroll
+        for (int k8 = 0; k8 < P / 8; ++k8) {
+          const uint4 qv = __ldg(qp + (P * i) / 8 + k8);
+          const uint32_t qw4[4] = {qv.x, qv.y, qv.z, qv.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 qf = __half22float2(*reinterpret_cast<const __half2*>(&qw4[e]));
+            const int j = 8 * k8 + 2 * e;
+            acc = fmaf(qf.x, static_cast<float>((w[i] >> (BITS * j)) & L), acc);
+            acc = fmaf(qf.y, static_cast<float>((w[i] >> (BITS * (j + 1))) & L), acc);
+            qs += qf.x + qf.y;
+          }
+        }
+        dot = fmaf(sk, acc, fmaf(zk, qs, dot));
+      }
+      dot += __shfl_xor_sync(kFull, dot, 1);
+      dot *= a.qscale;
+      const bool valid = t < nvalid;
+      const float lg = valid ? dot : -INFINITY;
+      const float m_new = fmaxf(m[g], warp_max(lg));
+      const float alpha = fast_exp2(m[g] - m_new);
+      const float p = valid ? fast_exp2(lg - m_new) : 0.f;
+      m[g] = m_new;
+      l[g] = fmaf(l[g], alpha, hf == 0 ? p : 0.f);
+      Z[g] *= alpha;
+      alpha_[g] = alpha;
+      pres_[g] = p;
+    }
+  }
+
   __device__ void residual_k(uint8_t* kt, int nvalid, long long head, int r) {
+    if constexpr (KC) {
+      residual_k_coded(kt, nvalid, head);
+      return;
+    }
     insert_new_row(kt, r, head, a.k_new, a.k_res, false);
     const int t = lane >> 1, hf = lane & 1;  // 2 lanes per token, 64 channels each
 #pragma unroll
@@ -1319,7 +1389,7 @@ struct Decoder {
   }
 };
 
-template <int BITS, int G>
+template <int BITS, int G, bool KC>
 __global__ void __launch_bounds__(warps_per_cta<G>() * 32, 1) decode_kernel(const __grid_constant__ DecodeArgs a) {
   extern __shared__ __align__(128) uint8_t smem_raw[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -1328,7 +1398,7 @@ __global__ void __launch_bounds__(warps_per_cta<G>() * 32, 1) decode_kernel(cons
   const long long worker = static_cast<long long>(blockIdx.x) * warps_per_cta<G>() + warp;
   if (worker >= W) return;  // the last CTA may hold fewer workers
   const long long ub = U * worker / W, ue = U * (worker + 1) / W;  // non-empty because W <= U
-  Decoder<BITS, G> d(a, S, lane, worker, ub, ue);
+  Decoder<BITS, G, KC> d(a, S, lane, worker, ub, ue);
   d.run();
 }
 
@@ -1336,19 +1406,21 @@ template <int BITS, int G>
 cudaError_t plan_for(DecodePlan* plan) {
   constexpr int kWarps = warps_per_cta<G>();
   const int smem = kWarps * static_cast<int>(sizeof(WarpSmem<G>));
-  cudaError_t e = cudaFuncSetAttribute(decode_kernel<BITS, G>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  cudaError_t e = cudaFuncSetAttribute(decode_kernel<BITS, G, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(decode_kernel<BITS, G, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   int dev = 0, sms = 0, occ = 0;
   if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
   if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
-  if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, decode_kernel<BITS, G>, kWarps * 32, smem)) !=
+  if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, decode_kernel<BITS, G, false>, kWarps * 32, smem)) !=
       cudaSuccess)
     return e;
   if (occ < 1) return cudaErrorInvalidConfiguration;
   plan->warps_per_cta = kWarps;
   plan->ctas = sms * occ;
   plan->smem_bytes = smem;
-  plan->unit_tokens = Decoder<BITS, G>::UT;
+  plan->unit_tokens = Decoder<BITS, G, false>::UT;
   plan->res_unit_tokens = kResTokens;
   return cudaSuccess;
 }
@@ -1357,7 +1429,10 @@ template <int BITS, int G>
 cudaError_t launch_for(const DecodeArgs& a, const DecodePlan& plan, cudaStream_t stream) {
   if (a.workers < 1 || a.workers > plan.workers() || a.total_units < a.workers) return cudaErrorInvalidValue;
   const int ctas = (a.workers + plan.warps_per_cta - 1) / plan.warps_per_cta;
-  decode_kernel<BITS, G><<<ctas, plan.warps_per_cta * 32, plan.smem_bytes, stream>>>(a);
+  if (a.k_res_coded)
+    decode_kernel<BITS, G, true><<<ctas, plan.warps_per_cta * 32, plan.smem_bytes, stream>>>(a);
+  else
+    decode_kernel<BITS, G, false><<<ctas, plan.warps_per_cta * 32, plan.smem_bytes, stream>>>(a);
   return cudaGetLastError();
 }
 

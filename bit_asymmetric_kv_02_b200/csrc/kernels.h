@@ -26,6 +26,22 @@ struct QuantizeArgs {
   int residual, capacity, group_k, group_v;
   int lg_gk, lg_gv;  // log2(group_k), log2(group_v): set by launch_quantize_blocks
   int k_given;       // 1: the K (s, z) of each block are already in k_scale / k_zero (prefix groups)
+  int v_only;        // 1: quantize the V blocks only (online K: the K codes are in place)
+};
+
+// Online K: codes `rows` K rows per head (fp16 source rows src_tok0 .. of a [bh][src_tokens][128]
+// tensor) with the (s, z) of block blk_src into code rows dst_row0 .. of k_codes; copy_scales
+// also copies block blk_src's (s, z) into block blk_src + 1.  v_new != nullptr: also writes the
+// V row of each head into residual slot v_slot (an append).
+struct OnlineKArgs {
+  const uint16_t* k_src;
+  int src_tokens, src_tok0, rows;
+  uint32_t* k_codes;
+  uint16_t *k_scale, *k_zero;
+  const uint16_t* v_new;
+  uint16_t* v_res;
+  int bh, capacity, residual, group_k;
+  int blk_src, dst_row0, copy_scales, v_slot;
 };
 
 struct AppendArgs {
@@ -63,6 +79,9 @@ struct DecodeArgs {
   const uint16_t* k_new;
   const uint16_t* v_new;
   int new_slot;
+  // online K: the residual tokens' K rows are code rows n_quant .. of k_codes with the (s, z) of
+  // block res_blk (= n_quant / residual); 0: fp16 rows of k_res
+  int k_res_coded, res_blk;
 };
 
 constexpr int kPartialStride = 132;  // m, l, Z, pad, o[128]
@@ -72,6 +91,7 @@ cudaError_t launch_quantize_blocks(const QuantizeArgs& a, int bits, cudaStream_t
 // destination block's slot (the prefix-group prefill); then launch_quantize_blocks with k_given.
 cudaError_t launch_k_prefix_extremes(const QuantizeArgs& a, int bits, cudaStream_t stream);
 cudaError_t launch_append(const AppendArgs& a, cudaStream_t stream);
+cudaError_t launch_code_k_online(const OnlineKArgs& a, int bits, cudaStream_t stream);
 
 // Decode launch plan: warps per CTA, CTAs, dynamic shared memory.
 struct DecodePlan {

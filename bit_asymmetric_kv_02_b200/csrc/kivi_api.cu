@@ -47,6 +47,7 @@ int check_cfg(const kivi_config* c) {
   if (c->capacity % c->residual != 0) return KIVI_ERR_INVALID_ARG;
   if (c->group_k != 32 && c->group_k != 64 && c->group_k != 128) return KIVI_ERR_INVALID_ARG;
   if (c->group_v < 32 || !pow2(c->group_v) || c->group_v > c->residual) return KIVI_ERR_INVALID_ARG;
+  if (c->online_k != 0 && c->online_k != 1) return KIVI_ERR_INVALID_ARG;
   if (static_cast<long long>(c->batch) * c->num_kv_heads > (1ll << 30)) return KIVI_ERR_UNSUPPORTED;
   if (c->capacity / c->residual > 32767) return KIVI_ERR_UNSUPPORTED;  // grid.y limit of a prefill
   return KIVI_OK;
@@ -102,6 +103,35 @@ cudaError_t get_plan(int bits, int gqa, DecodePlan* out) {
 
 bool gqa_supported(int g) { return g == 1 || g == 2 || g == 4 || g == 8; }
 
+// Online K: the residual tokens' K rows are codes (a quantized block exists).
+bool k_online(const kivi_config* c, int n_quant) { return c->online_k == 1 && n_quant > 0; }
+
+// Online K coding of `rows` K rows per head from `src` (fp16 [bh][src_tokens][128], rows
+// src_tok0 ..) into code rows n_quant + slot0 .. with block n_quant/R - 1's (s, z); slot0 == 0
+// also copies that (s, z) into block n_quant/R.  v_new: the V row of an append (or nullptr).
+int code_k_online(const kivi_config* cfg, const kivi_cache* cache, const uint16_t* src, int src_tokens, int src_tok0,
+                  int rows, int slot0, const uint16_t* v_new, cudaStream_t stream) {
+  kivi::OnlineKArgs o{};
+  o.k_src = src;
+  o.src_tokens = src_tokens;
+  o.src_tok0 = src_tok0;
+  o.rows = rows;
+  o.k_codes = cache->k_codes;
+  o.k_scale = cache->k_scale;
+  o.k_zero = cache->k_zero;
+  o.v_new = v_new;
+  o.v_res = cache->v_res;
+  o.bh = cfg->batch * cfg->num_kv_heads;
+  o.capacity = cfg->capacity;
+  o.residual = cfg->residual;
+  o.group_k = cfg->group_k;
+  o.blk_src = cache->n_quant / cfg->residual - 1;
+  o.dst_row0 = cache->n_quant + slot0;
+  o.copy_scales = slot0 == 0 ? 1 : 0;
+  o.v_slot = slot0;
+  return kivi::launch_code_k_online(o, cfg->bits, stream) == cudaSuccess ? KIVI_OK : KIVI_ERR_CUDA;
+}
+
 }  // namespace
 
 extern "C" {
@@ -154,6 +184,8 @@ int prefill_impl(const kivi_config* cfg, kivi_cache* cache, const uint16_t* k_de
   const int n_res = (num_tokens - 1) % R + 1;
   const int n_quant = num_tokens - n_res;
   if (n_quant > cfg->capacity) return KIVI_ERR_CAPACITY;
+  if (prefix_k && cfg->online_k) return KIVI_ERR_UNSUPPORTED;
+  if (k_online(cfg, n_quant) && n_quant + R > cfg->capacity) return KIVI_ERR_CAPACITY;
   if (!cache_ptrs_ok(cache, n_quant > 0)) return KIVI_ERR_INVALID_ARG;
   kivi::QuantizeArgs a{};
   a.k_src = k_dev;
@@ -184,6 +216,13 @@ int prefill_impl(const kivi_config* cfg, kivi_cache* cache, const uint16_t* k_de
   }
   if (kivi::launch_quantize_blocks(a, cfg->bits, static_cast<cudaStream_t>(stream)) != cudaSuccess)
     return KIVI_ERR_CUDA;
+  if (k_online(cfg, n_quant)) {  // the tail's K rows become codes (the fp16 copy is left unused)
+    kivi_cache after = *cache;
+    after.n_quant = n_quant;
+    if (code_k_online(cfg, &after, k_dev, num_tokens, n_quant, n_res, 0, nullptr, static_cast<cudaStream_t>(stream)) !=
+        KIVI_OK)
+      return KIVI_ERR_CUDA;
+  }
   cache->n_quant = n_quant;
   cache->n_res = n_res;
   return KIVI_OK;
@@ -208,6 +247,13 @@ int kivi_append_token(const kivi_config* cfg, kivi_cache* cache, const uint16_t*
   if ((st = check_state(cfg, cache)) != KIVI_OK) return st;
   if (!aligned16(k_new_dev) || !aligned16(v_new_dev) || !cache_ptrs_ok(cache, false)) return KIVI_ERR_INVALID_ARG;
   if (cache->n_res == cfg->residual) return KIVI_ERR_RESIDUAL_FULL;
+  if (k_online(cfg, cache->n_quant)) {
+    if (cache->n_quant + cfg->residual > cfg->capacity) return KIVI_ERR_CAPACITY;
+    if (!cache_ptrs_ok(cache, true)) return KIVI_ERR_INVALID_ARG;
+    st = code_k_online(cfg, cache, k_new_dev, 1, 0, 1, cache->n_res, v_new_dev, static_cast<cudaStream_t>(stream));
+    if (st == KIVI_OK) cache->n_res += 1;
+    return st;
+  }
   kivi::AppendArgs a{};
   a.k_new = k_new_dev;
   a.v_new = v_new_dev;
@@ -250,6 +296,7 @@ int kivi_flush_residual(const kivi_config* cfg, kivi_cache* cache, void* stream)
   a.capacity = cfg->capacity;
   a.group_k = cfg->group_k;
   a.group_v = cfg->group_v;
+  a.v_only = k_online(cfg, cache->n_quant) ? 1 : 0;  // online K: the block's K codes are in place
   if (kivi::launch_quantize_blocks(a, cfg->bits, static_cast<cudaStream_t>(stream)) != cudaSuccess)
     return KIVI_ERR_CUDA;
   cache->n_quant += R;
@@ -271,7 +318,8 @@ size_t kivi_decode_workspace_bytes(const kivi_config* cfg, int32_t num_q_heads) 
 namespace {
 
 // Decode attention over `cache` (whose counters already include a fused append's token, which
-// k_new / v_new hold for residual slot new_slot; new_slot < 0: no append).
+// k_new / v_new hold for residual slot new_slot; new_slot < 0: no append; -2: check the
+// arguments only and enqueue nothing).
 int decode_impl(const kivi_config* cfg, const kivi_cache* cache, const uint16_t* q_dev, int32_t num_q_heads,
                 float scale, uint16_t* out_dev, void* workspace_dev, size_t workspace_bytes, int32_t* dev_status,
                 void* stream, const uint16_t* k_new_dev, const uint16_t* v_new_dev, int new_slot) {
@@ -285,6 +333,8 @@ int decode_impl(const kivi_config* cfg, const kivi_cache* cache, const uint16_t*
     return KIVI_ERR_INVALID_ARG;
   if (cache->n_quant + cache->n_res == 0) return KIVI_ERR_EMPTY;
   if (!cache_ptrs_ok(cache, cache->n_quant > 0)) return KIVI_ERR_INVALID_ARG;
+  const bool coded_res = k_online(cfg, cache->n_quant) && cache->n_res > 0;
+  if (coded_res && (cache->n_quant + cfg->residual > cfg->capacity || new_slot >= 0)) return KIVI_ERR_STATE;
   if (dev_status != nullptr && (reinterpret_cast<uintptr_t>(dev_status) & 3u) != 0) return KIVI_ERR_INVALID_ARG;
   DecodePlan plan{};
   if (get_plan(cfg->bits, gqa, &plan) != cudaSuccess) return KIVI_ERR_CUDA;
@@ -342,6 +392,9 @@ int decode_impl(const kivi_config* cfg, const kivi_cache* cache, const uint16_t*
   a.k_new = k_new_dev;
   a.v_new = v_new_dev;
   a.new_slot = new_slot;
+  a.k_res_coded = coded_res ? 1 : 0;
+  a.res_blk = cache->n_quant / cfg->residual;
+  if (new_slot == -2) return KIVI_OK;  // arguments checked, nothing enqueued
   if (kivi::launch_decode(a, cfg->bits, plan, static_cast<cudaStream_t>(stream)) != cudaSuccess)
     return KIVI_ERR_CUDA;
   return KIVI_OK;
@@ -365,6 +418,18 @@ int kivi_append_decode_attention(const kivi_config* cfg, kivi_cache* cache, cons
   if ((st = check_state(cfg, cache)) != KIVI_OK) return st;
   if (!aligned16(k_new_dev) || !aligned16(v_new_dev) || !cache_ptrs_ok(cache, false)) return KIVI_ERR_INVALID_ARG;
   if (cache->n_res == cfg->residual) return KIVI_ERR_RESIDUAL_FULL;
+  if (k_online(cfg, cache->n_quant)) {  // the K row is coded by its own launch before it is attended
+    if (cache->n_quant + cfg->residual > cfg->capacity) return KIVI_ERR_CAPACITY;
+    kivi_cache after = *cache;
+    after.n_res += 1;
+    // every argument check of the decode runs before anything is enqueued
+    st = decode_impl(cfg, &after, q_dev, num_q_heads, scale, out_dev, workspace_dev, workspace_bytes, dev_status,
+                     stream, nullptr, nullptr, -2);
+    if (st != KIVI_OK) return st;
+    if ((st = kivi_append_token(cfg, cache, k_new_dev, v_new_dev, stream)) != KIVI_OK) return st;
+    return decode_impl(cfg, cache, q_dev, num_q_heads, scale, out_dev, workspace_dev, workspace_bytes, dev_status,
+                       stream, nullptr, nullptr, -1);
+  }
   kivi_cache after = *cache;
   after.n_res += 1;
   st = decode_impl(cfg, &after, q_dev, num_q_heads, scale, out_dev, workspace_dev, workspace_bytes, dev_status,

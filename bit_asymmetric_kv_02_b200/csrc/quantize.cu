@@ -517,6 +517,7 @@ __global__ void __launch_bounds__(1024) quantize_tiles_kernel(QuantizeArgs a) {
   if (job < 2 * a.nblocks) {
     const int blk = job >> 1;
     const bool is_v = job & 1;
+    if (a.v_only && !is_v) return;
     const size_t src_tok = static_cast<size_t>(bh) * a.src_tokens + a.src_tok0 + static_cast<size_t>(blk) * R;
     const int dst_blk = a.dst_blk0 + blk;
     const size_t dst_tok = static_cast<size_t>(dst_blk) * R;
@@ -548,6 +549,7 @@ __global__ void __launch_bounds__(kThreads) quantize_blocks_kernel(QuantizeArgs 
   if (job < 2 * a.nblocks) {
     const int blk = job >> 1;
     const bool is_v = job & 1;
+    if (a.v_only && !is_v) return;
     const size_t src_tok = static_cast<size_t>(bh) * a.src_tokens + a.src_tok0 + static_cast<size_t>(blk) * R;
     const int dst_blk = a.dst_blk0 + blk;
     const size_t dst_tok = static_cast<size_t>(dst_blk) * R;
@@ -577,6 +579,36 @@ __global__ void __launch_bounds__(256) append_kernel(AppendArgs a) {
   const size_t dst = (static_cast<size_t>(bh) * a.residual + a.slot) * kChunks + c;
   reinterpret_cast<uint4*>(a.k_res)[dst] = __ldg(reinterpret_cast<const uint4*>(a.k_new) + i);
   reinterpret_cast<uint4*>(a.v_res)[dst] = __ldg(reinterpret_cast<const uint4*>(a.v_new) + i);
+}
+
+// Online K (section Per-Channel量子化: a new token's K is quantized at once with the existing scale
+// and zero point).  grid: x = batch * kv_heads, y = rows; 128 threads, one per channel.  The code
+// is clamp(rint((x - z) / s), 0, L) in fp64, which decides exactly: x - z of two fp16 values is
+// exact and the one rounding of the quotient cannot move it across a half-integer (s == 0: 0).
+// The P threads of one code word OR their shifted codes together.
+template <int BITS>
+__global__ void __launch_bounds__(kHeadDim) code_k_online_kernel(OnlineKArgs a) {
+  constexpr int P = 32 / BITS, L = (1 << BITS) - 1;
+  const int bh = blockIdx.x, row = blockIdx.y, c = threadIdx.x;
+  const int lg_gk = __ffs(a.group_k) - 1, ngk = kHeadDim >> lg_gk;
+  const size_t C = static_cast<size_t>(a.capacity), nblk = C / static_cast<size_t>(a.residual);
+  const size_t sb = (static_cast<size_t>(bh) * nblk + a.blk_src) * ngk;
+  const uint16_t xb = __ldg(a.k_src + (static_cast<size_t>(bh) * a.src_tokens + a.src_tok0 + row) * kHeadDim + c);
+  const double s = static_cast<double>(h2f(__ldg(a.k_scale + sb + (c >> lg_gk))));
+  const double z = static_cast<double>(h2f(__ldg(a.k_zero + sb + (c >> lg_gk))));
+  uint32_t code = 0u;
+  if (s > 0.0) code = static_cast<uint32_t>(fmin(fmax(rint((static_cast<double>(h2f(xb)) - z) / s), 0.0), double(L)));
+  const unsigned mask = (P == 32 ? 0xffffffffu : ((1u << P) - 1u)) << ((c & 31) & ~(P - 1));
+  const uint32_t word = __reduce_or_sync(mask, code << (BITS * (c & (P - 1))));
+  if ((c & (P - 1)) == 0)
+    a.k_codes[(static_cast<size_t>(bh) * C + a.dst_row0 + row) * (kHeadDim / P) + c / P] = word;
+  if (row == 0 && a.copy_scales && c < ngk) {
+    a.k_scale[sb + ngk + c] = a.k_scale[sb + c];
+    a.k_zero[sb + ngk + c] = a.k_zero[sb + c];
+  }
+  if (row == 0 && a.v_new != nullptr)
+    a.v_res[(static_cast<size_t>(bh) * a.residual + a.v_slot) * kHeadDim + c] =
+        __ldg(a.v_new + static_cast<size_t>(bh) * kHeadDim + c);
 }
 
 // K (s, z) of channel group blockIdx.y of head blockIdx.x over all nblocks * R source tokens
@@ -658,6 +690,16 @@ cudaError_t launch_k_prefix_extremes(const QuantizeArgs& args, int bits, cudaStr
     k_prefix_extremes_kernel<2><<<grid, kThreads, 0, stream>>>(a);
   else
     k_prefix_extremes_kernel<4><<<grid, kThreads, 0, stream>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_code_k_online(const OnlineKArgs& a, int bits, cudaStream_t stream) {
+  if (a.rows < 1) return cudaSuccess;
+  dim3 grid(a.bh, a.rows);
+  if (bits == 2)
+    code_k_online_kernel<2><<<grid, kHeadDim, 0, stream>>>(a);
+  else
+    code_k_online_kernel<4><<<grid, kHeadDim, 0, stream>>>(a);
   return cudaGetLastError();
 }
 

@@ -32,7 +32,8 @@ class KiviError(RuntimeError):
 
 class kivi_config(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in
-                ("batch", "num_kv_heads", "head_dim", "bits", "group_k", "group_v", "residual", "capacity")]
+                ("batch", "num_kv_heads", "head_dim", "bits", "group_k", "group_v", "residual", "capacity",
+                 "online_k")]
 
 
 class kivi_cache(ctypes.Structure):
@@ -166,11 +167,12 @@ class KiviCache:
 
     def __init__(self, batch: int, num_kv_heads: int, capacity: int, bits: int = 2, group_k: int = 32,
                  group_v: int = 32, residual: int = 128, head_dim: int = 128, num_q_heads: int | None = None,
-                 device=None):
+                 device=None, online_k: bool = False):
         import torch
         self.torch = torch
         self.device = torch.device(device or "cuda")
-        self.cfg = kivi_config(batch, num_kv_heads, head_dim, bits, group_k, group_v, residual, capacity)
+        self.cfg = kivi_config(batch, num_kv_heads, head_dim, bits, group_k, group_v, residual, capacity,
+                               1 if online_k else 0)
         st = kivi_check_config(self.cfg)
         if st != KIVI_OK:
             raise KiviError(st, "kivi_check_config")

@@ -55,7 +55,7 @@
 extern "C" {
 #endif
 
-#define KIVI_ABI_VERSION 1
+#define KIVI_ABI_VERSION 2
 
 /* Status codes. */
 #define KIVI_OK 0
@@ -76,8 +76,17 @@ extern "C" {
  * group_size_k, group_size_v, residual_length) plus the shape and capacity of the cache.
  * Rules: batch >= 1, num_kv_heads >= 1, capacity >= 0, capacity % residual == 0,
  * residual in {128, 256, 512, 1024}, group_k in {32, 64, 128}, group_v a power of two with
- * 32 <= group_v <= residual (KIVI_ERR_INVALID_ARG otherwise);
+ * 32 <= group_v <= residual, online_k in {0, 1} (KIVI_ERR_INVALID_ARG otherwise);
  * head_dim == 128, bits in {2, 4} (KIVI_ERR_UNSUPPORTED otherwise).
+ *
+ * online_k = 1 selects online K quantization (section Per-Channel量子化: a new token's K can be
+ * quantized at once with the existing scale and zero point).  Once a quantized block exists
+ * (n_quant > 0), the K row of every residual token is stored as codes, not fp16: token
+ * n_quant + i is code row n_quant + i of k_codes, coded with the (s, z) of block n_quant/R - 1,
+ * clamped to [0, 2^b-1], and block n_quant/R holds a copy of that (s, z).  V keeps its fp16
+ * residual and its flush.  Before the first block exists K stays fp16 as with online_k = 0.
+ * Such a cache needs n_quant + R <= capacity whenever it holds residual tokens (KIVI_ERR_CAPACITY
+ * from the prefill or append that would break it).
  */
 typedef struct kivi_config {
   int32_t batch;        /* B */
@@ -88,6 +97,7 @@ typedef struct kivi_config {
   int32_t group_v;      /* G_v: tokens per V group */
   int32_t residual;     /* R: residual (fp16) capacity in tokens, also the K block length */
   int32_t capacity;     /* C: maximum number of quantized tokens per head */
+  int32_t online_k;     /* 0: K residual in fp16; 1: online K quantization (see above) */
 } kivi_config;
 
 /* Device buffers of one cache (caller-owned) plus the two host-side counters the calls advance.
@@ -119,6 +129,7 @@ int kivi_check_config(const kivi_config* cfg);
  * k_dev, v_dev: fp16 [B][H][T][d].  Afterwards n_res = ((T-1) mod R) + 1 and
  * n_quant = T - n_res (so T <= R keeps everything in fp16); tokens [0, n_quant) are quantized
  * as n_quant/R blocks and tokens [n_quant, T) are copied into residual slots 0..n_res-1.
+ * With online_k and n_quant > 0 the tail's K rows are coded instead (a second launch).
  * Errors: T < 1 (INVALID_ARG), n_quant > capacity (CAPACITY).  One kernel launch.
  */
 int kivi_quantize_prefill(const kivi_config* cfg, kivi_cache* cache, const uint16_t* k_dev,
@@ -131,13 +142,17 @@ int kivi_quantize_prefill(const kivi_config* cfg, kivi_cache* cache, const uint1
  * attention, appends and later flushes (which quantize their own R-token blocks) are unchanged.
  * V groups, the residual split, arguments and errors are those of kivi_quantize_prefill.
  * Two kernel launches (the K group extremes over the prefix, then the quantization).
+ * online_k = 1 is not combined with this reading (KIVI_ERR_UNSUPPORTED).
  */
 int kivi_quantize_prefill_prefix_k(const kivi_config* cfg, kivi_cache* cache, const uint16_t* k_dev,
                                    const uint16_t* v_dev, int32_t num_tokens, void* stream);
 
 /*
  * Append: writes one new token's K and V (fp16 [B][H][d]) into residual slot n_res and
- * increments n_res.  Section 残差バッファ.  Errors: n_res == R (RESIDUAL_FULL).  One launch.
+ * increments n_res.  Section 残差バッファ.  With online_k and n_quant > 0 the K row is coded
+ * into code row n_quant + n_res instead (section Per-Channel量子化), and the first append after
+ * a flush copies block n_quant/R - 1's K (s, z) into block n_quant/R.
+ * Errors: n_res == R (RESIDUAL_FULL); online K with n_quant + R > capacity (CAPACITY).  One launch.
  */
 int kivi_append_token(const kivi_config* cfg, kivi_cache* cache, const uint16_t* k_new_dev,
                       const uint16_t* v_new_dev, void* stream);
@@ -145,6 +160,7 @@ int kivi_append_token(const kivi_config* cfg, kivi_cache* cache, const uint16_t*
 /*
  * Flush: quantizes the full residual (R tokens) as quantized block n_quant/R, then
  * n_quant += R, n_res = 0.  Sections Per-Token量子化 (flush once the group fills) and 残差バッファ.
+ * With online_k and n_quant > 0 only V is quantized: the block's K codes and (s, z) are in place.
  * Errors: n_res < R (RESIDUAL_NOT_FULL), n_quant + R > capacity (CAPACITY).  One launch.
  */
 int kivi_flush_residual(const kivi_config* cfg, kivi_cache* cache, void* stream);
@@ -163,6 +179,8 @@ size_t kivi_decode_workspace_bytes(const kivi_config* cfg, int32_t num_q_heads);
  * (after a device error, zero it again).  Calls sharing one workspace must not overlap.
  * dev_status: optional (may be NULL) device int32 that receives KIVI_ERR_DEVICE_TIMEOUT if a
  * bounded wait inside the kernel expires; the caller zeroes it and reads it with kivi_read_status.
+ * With online_k and n_quant > 0 the residual tokens' keys are their codes (dequantized with the
+ * block's copied (s, z)) and their values the fp16 residual rows.
  * Errors: empty cache (EMPTY), workspace too small (WORKSPACE).  One kernel launch.
  */
 int kivi_decode_attention(const kivi_config* cfg, const kivi_cache* cache, const uint16_t* q_dev,
@@ -178,7 +196,8 @@ int kivi_decode_attention(const kivi_config* cfg, const kivi_cache* cache, const
  * row into its shared-memory tile and into the cache.  On success n_res is incremented; on any
  * error the counters are unchanged (a device error may leave the slot written, as with a failed
  * append).  Arguments and errors are those of the two calls; RESIDUAL_FULL when n_res == R
- * (flush first).  One kernel launch.
+ * (flush first).  One kernel launch; with online_k and n_quant > 0 the K row must be coded before
+ * it is attended, and the call enqueues kivi_append_token and kivi_decode_attention (two launches).
  */
 int kivi_append_decode_attention(const kivi_config* cfg, kivi_cache* cache, const uint16_t* k_new_dev,
                                  const uint16_t* v_new_dev, const uint16_t* q_dev, int32_t num_q_heads,

@@ -305,6 +305,8 @@ class HeadCache:
         one R-token block.  The residual split, the V groups (g_v consecutive tokens, section
         Per-Token量子化) and the counters are those of prefill.  The shared K (s, z) is kept once per
         R-token block, so dequantization and later flushes use the same layout as prefill."""
+        if self.online_k:
+            raise OracleError("UNSUPPORTED", "online K is not combined with prefix K groups")
         k = np.asarray(k, np.float16)
         v = np.asarray(v, np.float16)
         T = k.shape[0]

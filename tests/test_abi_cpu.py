@@ -33,7 +33,7 @@ def test_every_declared_symbol_is_exported(kivi):
 
 
 def test_version_and_strerror(kivi):
-    assert kivi.kivi_abi_version() == 1
+    assert kivi.kivi_abi_version() == 2
     assert kivi.kivi_strerror(0) == "ok"
     assert "flush" in kivi.kivi_strerror(4)
     assert kivi.kivi_strerror(12345) == "unknown status"
@@ -125,6 +125,31 @@ def test_state_errors_before_any_device_work(kivi):
     with pytest.raises(kivi.KiviError) as e:
         kivi.kivi_quantize_prefill(cfg, cache, fake, fake, 1024 + 129, 0)
     assert e.value.code == "CAPACITY"
+
+
+def test_online_k_host_errors(kivi):
+    """Online K (section Per-Channel量子化): the flag's rule and the capacity its block slot needs,
+    checked on the host before anything is enqueued."""
+    assert kivi.kivi_check_config(_cfg(kivi, online_k=1)) == 0
+    assert kivi.kivi_check_config(_cfg(kivi, online_k=2)) == 1
+    cfg = _cfg(kivi, online_k=1)
+    fake = 1 << 20
+    cache = kivi.kivi_cache(*([fake] * 8), 1024, 3)     # every block slot used: no room for online rows
+    with pytest.raises(kivi.KiviError) as e:
+        kivi.kivi_append_token(cfg, cache, fake, fake, 0)
+    assert e.value.code == "CAPACITY" and cache.n_res == 3
+    with pytest.raises(kivi.KiviError) as e:
+        kivi.kivi_append_decode_attention(cfg, cache, fake, fake, fake, 3, 0.1, fake, fake, 1 << 30, None, 0)
+    assert e.value.code == "CAPACITY" and cache.n_res == 3
+    with pytest.raises(kivi.KiviError) as e:
+        kivi.kivi_decode_attention(cfg, cache, fake, 3, 0.1, fake, fake, 1 << 30, None, 0)
+    assert e.value.code == "STATE"
+    with pytest.raises(kivi.KiviError) as e:
+        kivi.kivi_quantize_prefill(cfg, cache, fake, fake, 1024 + 1, 0)
+    assert e.value.code == "CAPACITY" and (cache.n_quant, cache.n_res) == (1024, 3)
+    with pytest.raises(kivi.KiviError) as e:
+        kivi.kivi_quantize_prefill_prefix_k(cfg, cache, fake, fake, 300, 0)
+    assert e.value.code == "UNSUPPORTED"
 
 
 def test_binding_fails_loudly_without_library(tmp_path):
