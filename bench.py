@@ -40,6 +40,7 @@ WORKLOAD = synth.LARGE_BATCH
 FUSED = True   # append and decode in one launch (kivi_append_decode_attention); --separate-append: two
 STEP_NOTE = {True: "flush when full + append and decode attention in one launch",
              False: "flush when full + append + decode attention"}
+ONLINE_K = False   # --online-k: K rows coded at append with the newest block's (s, z) (config online_k)
 DECODE_SOURCES = ["decode.cu", "common.cuh", "kernels.h"]
 
 
@@ -79,7 +80,7 @@ def profiled_traffic(w: synth.Workload, alg_bytes_per_launch: float):
             rec = json.load(f)
     except Exception:
         return None
-    if rec.get("kernel_sha") != decode_kernel_sha() or rec.get("workload") != w.name:
+    if rec.get("kernel_sha") != decode_kernel_sha() or rec.get("workload") != w.name or ONLINE_K:
         return None
     return rec["dram_bytes"] / rec["alg_bytes"] * alg_bytes_per_launch
 
@@ -104,7 +105,9 @@ def decode_alg_bytes(w: synth.Workload, n_quant: int, n_res: int) -> int:
                 + (n_quant // w.group) * 4                               # V scale + zero
                 + n_res * w.head_dim * 4                                 # fp16 K and V residual rows
                 + 2 * w.gqa * w.head_dim * 2)                            # q in, out
-    return bh * per_head
+    if ONLINE_K and n_quant > 0 and n_res > 0:   # residual K rows are codes, plus the block's (s, z)
+        per_head += (w.head_dim // w.group) * 4 - n_res * w.head_dim * (2 - w.bits / 8)
+    return int(bh * per_head)
 
 
 class ClockSampler:
@@ -221,10 +224,10 @@ def weak_scaling_value(world: int, tokens_per_rank: int, batch: int, t_max_ms: f
 # ------------------------------------------------------------------------------------------------
 def make_state(w: synth.Workload, torch, kivi, device):
     n_quant0 = (w.tokens - 1) // w.residual * w.residual      # 8064: the prompt leaves a full residual
-    capacity = n_quant0 + w.residual
+    capacity = n_quant0 + (2 if ONLINE_K else 1) * w.residual   # online K: a slot for the block being filled
     k, v = synth.prompt_kv(w, w.tokens)
     cache = kivi.KiviCache(w.batch, w.kv_heads, capacity, bits=w.bits, group_k=w.group, group_v=w.group,
-                           residual=w.residual, num_q_heads=w.q_heads, device=device)
+                           residual=w.residual, num_q_heads=w.q_heads, device=device, online_k=ONLINE_K)
     kd = torch.from_numpy(k).to(device)
     vd = torch.from_numpy(v).to(device)
     cache.prefill(kd, vd)            # first run loads the module; the second one is timed
@@ -410,6 +413,7 @@ def run_gpu(args, rank, world, local_rank, w: synth.Workload):
                 "head_dim": w.head_dim, "bits": w.bits, "group_k": w.group, "group_v": w.group,
                 "residual": w.residual, "cached_tokens": f"{n_quant0 + 1}-{n_quant0 + 2 * R} (128-step cycles)",
                 "step": STEP_NOTE[FUSED],
+                "k_residual": "codes (online K, config online_k = 1)" if ONLINE_K else "fp16",
                 "l2": l2_note(w, n_quant0),
                 "parallelism": f"weak: one independent batch per GPU x {world}",
             },
@@ -531,11 +535,17 @@ def main():
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end loop (profiling runs)")
     ap.add_argument("--separate-append", action="store_true",
                     help="append and decode as two launches (kivi_append_token + kivi_decode_attention)")
+    ap.add_argument("--online-k", action="store_true",
+                    help="online K quantization (config online_k = 1); implies --separate-append and no "
+                         "cpu baseline")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
-    global FUSED
-    FUSED = not args.separate_append
+    global FUSED, ONLINE_K
+    ONLINE_K = args.online_k
+    FUSED = not (args.separate_append or args.online_k)
+    if ONLINE_K and args.impl == "reference":
+        ap.error("--online-k times the GPU arm only")
     w = synth.WORKLOADS[args.workload]
     if args.bits is not None:
         w = w.with_(bits=args.bits)
@@ -548,7 +558,7 @@ def main():
         res = run_reference(args, rank, world, w)
     else:
         res = run_gpu(args, rank, world, local_rank, w)
-        if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        if rank == 0 and world == 1 and not args.no_cpu_baseline and not ONLINE_K:
             log("cpu baseline (oracle)")
             value, cores, sample, dt, hs = oracle_sample(w, n_heads=min(64, 2 * (os.cpu_count() or 1)),
                                                          n_steps=16, budget_s=25.0)
