@@ -25,6 +25,10 @@ Readings taken where the page leaves a step open (each is pinned by tests/test_o
   * Decode attention follows the Attention equation of section 残差バッファ: logits over the
     dequantized quantized tokens followed by the fp16 residual tokens, softmax, weighted sum of
     the matching V rows.  No mask; the query-head -> KV-head map is contiguous (h // (Hq/H)).
+  * Fine-grained groups (an opt-in variant, section KVキャッシュの分布特性: K ranges are taken along
+    each channel, V ranges along each token): K has one (s, z) per channel per g_k consecutive tokens,
+    V one per token per g_v consecutive channels.  Blocks, residual and flushes are as in the base
+    scheme; only the group axes (and so the scale layouts) change.
   * Online K (an opt-in variant, section Per-Channel量子化: a new token's K can be quantized at
     once with the existing scale and zero point): once a quantized block exists, every new K row
     is coded at append time with the (s, z) of the newest quantized block, clamped to [0, 2^b-1];
@@ -44,6 +48,7 @@ __all__ = [
     "OracleError", "levels", "codes_per_word", "fp16_round", "scale_zero", "quantize_values",
     "quantize_k_block", "quantize_v_block", "pack_k", "pack_v", "unpack_k", "unpack_v",
     "dequantize_k", "dequantize_v", "attention", "HeadCache", "OracleCache",
+    "quantize_k_block_fine", "quantize_v_block_fine", "dequantize_k_fine", "dequantize_v_fine",
 ]
 
 
@@ -135,6 +140,42 @@ def quantize_v_block(block, group_v: int, bits: int):
     return codes, s, z
 
 
+def quantize_k_block_fine(block, group_k: int, bits: int):
+    """Fine-grained K groups (section KVキャッシュの分布特性: the range of each channel; section
+    Per-Channel量子化 for Q): one (s, z) per channel per g_k consecutive tokens.  block: fp16 [n][d]
+    with n a multiple of g_k.  Returns codes uint8 [n][d], s and z fp16 [n/g_k][d]."""
+    block = np.asarray(block, dtype=np.float16)
+    n, d = block.shape
+    ng = n // group_k
+    lo = np.empty((ng, d), dtype=np.float16)
+    hi = np.empty((ng, d), dtype=np.float16)
+    for u in range(ng):
+        rows = block[u * group_k:(u + 1) * group_k, :]
+        lo[u] = rows.min(axis=0)
+        hi[u] = rows.max(axis=0)
+    s, z = scale_zero(lo, hi, bits)
+    codes = quantize_values(block, np.repeat(s, group_k, axis=0), np.repeat(z, group_k, axis=0), bits)
+    return codes, s, z
+
+
+def quantize_v_block_fine(block, group_v: int, bits: int):
+    """Fine-grained V groups (section KVキャッシュの分布特性: the range of each token; section
+    Per-Token量子化 for Q): one (s, z) per token per g_v consecutive channels.  block: fp16 [n][d].
+    Returns codes uint8 [n][d], s and z fp16 [n][d/g_v]."""
+    block = np.asarray(block, dtype=np.float16)
+    n, d = block.shape
+    ng = d // group_v
+    lo = np.empty((n, ng), dtype=np.float16)
+    hi = np.empty((n, ng), dtype=np.float16)
+    for g in range(ng):
+        cols = block[:, g * group_v:(g + 1) * group_v]
+        lo[:, g] = cols.min(axis=1)
+        hi[:, g] = cols.max(axis=1)
+    s, z = scale_zero(lo, hi, bits)
+    codes = quantize_values(block, np.repeat(s, group_v, axis=1), np.repeat(z, group_v, axis=1), bits)
+    return codes, s, z
+
+
 def pack_k(codes, bits: int) -> np.ndarray:
     """Token-major K packing of the cache layout: word i of token t holds the codes of channels
     P*i + j at bits [b*j, b*j+b), P = 32/b.  codes: uint8 [n][d] -> uint32 [n][d/P]."""
@@ -205,6 +246,24 @@ def dequantize_v(codes, s, z, group_v: int) -> np.ndarray:
     return s64 * codes + z64
 
 
+def dequantize_k_fine(codes, s, z, group_k: int) -> np.ndarray:
+    """D(K^) = s*K^ + z in float64 with the (token group, channel) pair of each element (D equation).
+    codes uint8 [n][d]; s, z fp16 [n/g_k][d]."""
+    codes = np.asarray(codes, dtype=np.float64)
+    s64 = np.repeat(np.asarray(s, dtype=np.float16).astype(np.float64), group_k, axis=0)
+    z64 = np.repeat(np.asarray(z, dtype=np.float16).astype(np.float64), group_k, axis=0)
+    return s64 * codes + z64
+
+
+def dequantize_v_fine(codes, s, z, group_v: int) -> np.ndarray:
+    """D(V^) = s*V^ + z in float64 with the (token, channel group) pair of each element (D equation).
+    codes uint8 [n][d]; s, z fp16 [n][d/g_v]."""
+    codes = np.asarray(codes, dtype=np.float64)
+    s64 = np.repeat(np.asarray(s, dtype=np.float16).astype(np.float64), group_v, axis=1)
+    z64 = np.repeat(np.asarray(z, dtype=np.float16).astype(np.float64), group_v, axis=1)
+    return s64 * codes + z64
+
+
 def attention(q, keys, values, scale: float) -> np.ndarray:
     """softmax(scale * q K^T) V for each query row, in float64 (section 残差バッファ, Attention
     equation).  q: [G][d]; keys, values: [T][d] float64 (dequantized then residual rows).
@@ -222,19 +281,23 @@ class HeadCache:
 
     Mirrors the library's counters: n_quant (a multiple of R) and n_res in [0, R].  With online_k,
     k_codes also holds the n_res online-coded rows after the n_quant block rows and k_s / k_z
-    hold one row for the block being filled."""
+    hold one row for the block being filled.  With fine_groups, g_k counts tokens and g_v channels
+    (k_s / k_z [n_quant/g_k][d], v_s / v_z [n_quant][d/g_v])."""
 
     def __init__(self, head_dim: int, bits: int, group_k: int, group_v: int, residual: int,
-                 capacity: int, online_k: bool = False):
+                 capacity: int, online_k: bool = False, fine_groups: bool = False):
         self.d, self.bits, self.gk, self.gv = head_dim, bits, group_k, group_v
         self.R, self.capacity = residual, capacity
         self.online_k = bool(online_k)
+        self.fine = bool(fine_groups)
+        if self.fine and self.online_k:
+            raise OracleError("UNSUPPORTED", "online K is not combined with fine-grained groups")
         self.k_codes = np.zeros((0, head_dim), np.uint8)
         self.v_codes = np.zeros((0, head_dim), np.uint8)
-        self.k_s = np.zeros((0, head_dim // group_k), np.float16)
-        self.k_z = np.zeros((0, head_dim // group_k), np.float16)
-        self.v_s = np.zeros((0,), np.float16)
-        self.v_z = np.zeros((0,), np.float16)
+        self.k_s = np.zeros((0, head_dim if self.fine else head_dim // group_k), np.float16)
+        self.k_z = np.zeros((0, head_dim if self.fine else head_dim // group_k), np.float16)
+        self.v_s = np.zeros((0, head_dim // group_v) if self.fine else (0,), np.float16)
+        self.v_z = np.zeros((0, head_dim // group_v) if self.fine else (0,), np.float16)
         self.k_res = np.zeros((0, head_dim), np.float16)
         self.v_res = np.zeros((0, head_dim), np.float16)
 
@@ -265,6 +328,16 @@ class HeadCache:
         self.k_codes = np.concatenate([self.k_codes, codes])
 
     def _quantize_block(self, kblk, vblk):
+        if self.fine:
+            kc, ks, kz = quantize_k_block_fine(kblk, self.gk, self.bits)
+            vc, vs, vz = quantize_v_block_fine(vblk, self.gv, self.bits)
+            self.k_codes = np.concatenate([self.k_codes, kc])
+            self.v_codes = np.concatenate([self.v_codes, vc])
+            self.k_s = np.concatenate([self.k_s, ks])
+            self.k_z = np.concatenate([self.k_z, kz])
+            self.v_s = np.concatenate([self.v_s, vs])
+            self.v_z = np.concatenate([self.v_z, vz])
+            return
         kc, ks, kz = quantize_k_block(kblk, self.gk, self.bits)
         vc, vs, vz = quantize_v_block(vblk, self.gv, self.bits)
         self.k_codes = np.concatenate([self.k_codes, kc])
@@ -287,7 +360,7 @@ class HeadCache:
         n_quant = T - n_res
         if n_quant > self.capacity:
             raise OracleError("CAPACITY", f"{n_quant} > {self.capacity}")
-        self.__init__(self.d, self.bits, self.gk, self.gv, self.R, self.capacity, self.online_k)
+        self.__init__(self.d, self.bits, self.gk, self.gv, self.R, self.capacity, self.online_k, self.fine)
         for j in range(n_quant // self.R):
             sl = slice(j * self.R, (j + 1) * self.R)
             self._quantize_block(k[sl], v[sl])
@@ -305,8 +378,8 @@ class HeadCache:
         one R-token block.  The residual split, the V groups (g_v consecutive tokens, section
         Per-Token量子化) and the counters are those of prefill.  The shared K (s, z) is kept once per
         R-token block, so dequantization and later flushes use the same layout as prefill."""
-        if self.online_k:
-            raise OracleError("UNSUPPORTED", "online K is not combined with prefix K groups")
+        if self.online_k or self.fine:
+            raise OracleError("UNSUPPORTED", "prefix K groups are not combined with online K or fine groups")
         k = np.asarray(k, np.float16)
         v = np.asarray(v, np.float16)
         T = k.shape[0]
@@ -363,12 +436,18 @@ class HeadCache:
     def keys(self) -> np.ndarray:
         """[D(K_quant); K_res] as float64 [n_quant + n_res][d] (with online K every row is
         dequantized)."""
-        kd = dequantize_k(self.k_codes, self.k_s, self.k_z, self.R, self.gk)
+        if self.fine:
+            kd = dequantize_k_fine(self.k_codes, self.k_s, self.k_z, self.gk)
+        else:
+            kd = dequantize_k(self.k_codes, self.k_s, self.k_z, self.R, self.gk)
         return np.concatenate([kd, self.k_res.astype(np.float64)])
 
     def values(self) -> np.ndarray:
         """[D(V_quant); V_res] as float64 [n_quant + n_res][d]."""
-        vd = dequantize_v(self.v_codes, self.v_s, self.v_z, self.gv)
+        if self.fine:
+            vd = dequantize_v_fine(self.v_codes, self.v_s, self.v_z, self.gv)
+        else:
+            vd = dequantize_v(self.v_codes, self.v_s, self.v_z, self.gv)
         return np.concatenate([vd, self.v_res.astype(np.float64)])
 
     def attend(self, q, scale: float) -> np.ndarray:
@@ -393,11 +472,11 @@ class OracleCache:
 
     def __init__(self, batch: int, num_kv_heads: int, head_dim: int = 128, bits: int = 2,
                  group_k: int = 32, group_v: int = 32, residual: int = 128, capacity: int = 0,
-                 heads=None, online_k: bool = False):
+                 heads=None, online_k: bool = False, fine_groups: bool = False):
         self.B, self.H = batch, num_kv_heads
         self.heads = sorted(heads) if heads is not None else [
             (b, h) for b in range(batch) for h in range(num_kv_heads)]
-        self.cache = {bh: HeadCache(head_dim, bits, group_k, group_v, residual, capacity, online_k)
+        self.cache = {bh: HeadCache(head_dim, bits, group_k, group_v, residual, capacity, online_k, fine_groups)
                       for bh in self.heads}
 
     def _counters(self):

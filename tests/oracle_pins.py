@@ -394,6 +394,55 @@ def check_online_k(O, bits, group):
     assert list(e.k_codes[R]) == nearest_codes and e.k_res.shape[0] == 0
 
 
+def check_fine_groups(O, bits, gk, gv):
+    """Fine-grained groups (section KVキャッシュの分布特性: K ranges along each channel, V ranges along
+    each token): every K (s, z) is the range of one channel over g_k consecutive tokens and every V
+    (s, z) the range of one token over g_v consecutive channels, by brute force with exact rationals;
+    codes are the nearest grid points; prefill equals streaming; D is s * code + z exactly."""
+    rng = np.random.default_rng(171 + bits + gk + gv)
+    R, d, L = 128, 128, 2 ** bits - 1
+    T = 2 * R + 21
+    k = (rng.standard_normal((T, d)) * np.exp2(rng.integers(-2, 3, (1, d)))).astype(np.float16)
+    k[:, 5] *= np.float16(12)                       # an outlier channel
+    v = rng.standard_normal((T, d)).astype(np.float16)
+    v[0] *= np.float16(6)                           # a sink token
+    h = O.HeadCache(d, bits, gk, gv, R, 4 * R, fine_groups=True)
+    h.prefill(k, v)
+    n_q = 2 * R
+    assert (h.n_quant, h.n_res) == (n_q, 21)
+    assert h.k_s.shape == (n_q // gk, d) and h.v_s.shape == (n_q, d // gv)
+    for u in range(n_q // gk):
+        for c in list(range(0, d, 9)) + [5]:
+            vals = [_fr(k[t, c]) for t in range(u * gk, (u + 1) * gk)]
+            lo, hi = min(vals), max(vals)
+            sx = fp16_round_exact((hi - lo) / L)
+            assert Fraction(float(h.k_s[u, c])) == sx and Fraction(float(h.k_z[u, c])) == lo, (u, c)
+            for t in range(u * gk, (u + 1) * gk, 7):
+                assert h.k_codes[t, c] == code_nearest_grid(_fr(k[t, c]), sx, lo, bits), (t, c)
+    for t in list(range(0, n_q, 13)) + [0]:
+        for g in range(d // gv):
+            vals = [_fr(v[t, c]) for c in range(g * gv, (g + 1) * gv)]
+            lo, hi = min(vals), max(vals)
+            sx = fp16_round_exact((hi - lo) / L)
+            assert Fraction(float(h.v_s[t, g])) == sx and Fraction(float(h.v_z[t, g])) == lo, (t, g)
+            for c in range(g * gv, (g + 1) * gv, 5):
+                assert h.v_codes[t, c] == code_nearest_grid(_fr(v[t, c]), sx, lo, bits), (t, c)
+    keys, values = h.keys(), h.values()
+    for t, c in ((0, 5), (R + 3, 64), (n_q - 1, 127)):
+        assert Fraction(float(keys[t, c])) == _fr(h.k_s[t // gk, c]) * int(h.k_codes[t, c]) + _fr(h.k_z[t // gk, c])
+        g = c // gv
+        assert Fraction(float(values[t, c])) == _fr(h.v_s[t, g]) * int(h.v_codes[t, c]) + _fr(h.v_z[t, g])
+    assert np.array_equal(keys[n_q:], k[n_q:].astype(np.float64))
+    a = O.HeadCache(d, bits, gk, gv, R, 4 * R, fine_groups=True)
+    a.prefill(k[:40], v[:40])
+    for t in range(40, T):
+        if a.n_res == R:
+            a.flush()
+        a.append(k[t], v[t])
+    for key, want in h.packed().items():
+        assert np.array_equal(np.asarray(a.packed()[key]).view(np.uint8), np.asarray(want).view(np.uint8)), key
+
+
 def check_errors(O):
     h = _head(O, cap=128)
     k = np.zeros((128, 128), np.float16)

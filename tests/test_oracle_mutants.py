@@ -193,3 +193,31 @@ def test_online_pin_catches_mutant(mutant, monkeypatch):
     monkeypatch.setattr(O.HeadCache, "_code_online", mutant)
     with pytest.raises(AssertionError):
         pins.check_online_k(O, 2, 32)
+
+
+_real_fine_k, _real_fine_v = O.quantize_k_block_fine, O.quantize_v_block_fine
+
+
+def _fine_k_over_channels(block, group_k, bits):     # K ranges taken along channels, not tokens
+    codes, s, z = O.quantize_k_block(block[:group_k * (block.shape[0] // group_k)], 32, bits)
+    c2, s2, z2 = _real_fine_k(block, group_k, bits)
+    s2[:] = np.repeat(s, 32)[None, :]
+    z2[:] = np.repeat(z, 32)[None, :]
+    return codes, s2, z2
+
+
+def _fine_v_over_tokens(block, group_v, bits):       # V ranges taken along tokens, not channels
+    codes, s, z = O.quantize_v_block(block, 32, bits)
+    c2, s2, z2 = _real_fine_v(block, group_v, bits)
+    s2[:] = np.repeat(s, 32)[:, None]
+    z2[:] = np.repeat(z, 32)[:, None]
+    return codes, s2, z2
+
+
+@pytest.mark.parametrize("name,mutant", [("quantize_k_block_fine", _fine_k_over_channels),
+                                         ("quantize_v_block_fine", _fine_v_over_tokens)],
+                         ids=["k_over_channels", "v_over_tokens"])
+def test_fine_pin_catches_mutant(name, mutant, monkeypatch):
+    monkeypatch.setattr(O, name, mutant)
+    with pytest.raises(AssertionError):
+        pins.check_fine_groups(O, 2, 32, 32)

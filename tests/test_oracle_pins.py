@@ -76,3 +76,8 @@ def test_prefix_k_groups(bits, group):
 @pytest.mark.parametrize("bits,group", [(2, 32), (4, 64), (2, 128)])
 def test_online_k(bits, group):
     pins.check_online_k(O, bits, group)
+
+
+@pytest.mark.parametrize("bits,gk,gv", [(2, 32, 32), (4, 64, 32), (2, 128, 64), (2, 32, 128)])
+def test_fine_groups(bits, gk, gv):
+    pins.check_fine_groups(O, bits, gk, gv)
