@@ -83,11 +83,14 @@ constexpr float kQRangeBal = 8323072.f;
 // path, which keeps a fourth, all-zero limb slot (the B operand columns of no limb read it).
 constexpr int kLimbVecs = 32;
 
-template <int G>
+// FG (fine-grained groups): qw holds the Q limbs of each K token group of a unit and pw the P limbs
+// of each V channel group (up to 4 each); oscr turns the output into the residual layout.
+template <int G, bool FG = false>
 struct __align__(16) WarpSmem {
   uint8_t buf[ring_buffers<G>()][buf_bytes<G>()];
-  uint4 qw[G][kLimbVecs];  // Q limbs of each query
-  uint4 pw[G][kLimbVecs];  // P limbs of each query
+  uint4 qw[FG ? 4 : G][kLimbVecs];  // Q limbs of each query (FG: of each K token group)
+  uint4 pw[FG ? 4 : G][kLimbVecs];  // P limbs of each query (FG: of each V channel group)
+  float oscr[FG ? kHeadDim : 4];
   uint64_t bar[ring_buffers<G>()];
 };
 
@@ -182,8 +185,9 @@ __device__ __forceinline__ void dot_set(uint32_t m, uint32_t L, uint32_t M, uint
 }
 
 // KC: the residual tokens' K rows are codes (online K); a separate instantiation keeps that path
-// out of the register allocation of the others.
-template <int BITS, int G, bool KC>
+// out of the register allocation of the others.  FG: fine-grained groups (2 bits, one query per KV
+// head): K (s, z) per channel per g_k tokens, V (s, z) per token per g_v channels.
+template <int BITS, int G, bool KC, bool FG = false>
 struct Decoder {
   static constexpr int P = 32 / BITS;              // codes per word
   static constexpr int UT = BITS == 2 ? 128 : 64;  // tokens per quantized unit (8 KB of codes)
@@ -199,7 +203,7 @@ struct Decoder {
   static constexpr int NBLK = G / 2;  // several queries: n8 blocks of queries (2 p, 2 p + 1)
 
   const DecodeArgs& a;
-  WarpSmem<G>& S;
+  WarpSmem<G, FG>& S;
   const int lane;
   const long long worker, ub, ue;
   const int ngk;  // K groups per head (d / G_k)
@@ -218,11 +222,15 @@ struct Decoder {
   float alpha_[G], invv_[G], pres_[G];
   bool hasv_[G];
   bool omma_;  // o is in the tensor-core layout of several queries (see o_swap_layout)
+  // FG: per K token group of the unit, 1 / Q scale and the z constant; per V channel group, the
+  // lane's part of sum_t p_t z_(t, group); o in the FG layout while quantized units run
+  float invqf[4], cblkf[4], ZF[4];
+  bool ofg_;
   // bytes per head of the code arrays and of a residual array; this lane's scale role
   const size_t code_head_bytes, res_head_bytes;
   const bool k_lane, v_lane;
 
-  __device__ Decoder(const DecodeArgs& args, WarpSmem<G>& smem, int ln, long long w, long long b, long long e)
+  __device__ Decoder(const DecodeArgs& args, WarpSmem<G, FG>& smem, int ln, long long w, long long b, long long e)
       : a(args), S(smem), lane(ln), worker(w), ub(b), ue(e), ngk(kHeadDim >> args.lg_gk), qkey(-1),
         code_head_bytes(static_cast<size_t>(args.capacity) * (kHeadDim * BITS / 8)),
         res_head_bytes(static_cast<size_t>(args.residual) * kHeadDim * 2),
@@ -270,7 +278,7 @@ struct Decoder {
     const uint16_t* ps = k_lane ? a.k_scale + ik : a.v_scale + iv;
     const uint16_t* pz = k_lane ? a.k_zero + ik : a.v_zero + iv;
     uint32_t r = 0u;
-    if ((k_lane || v_lane) && local < a.units_q)
+    if (!FG && (k_lane || v_lane) && local < a.units_q)  // FG loads its own scales per unit
       r = static_cast<uint32_t>(__ldg(ps)) | (static_cast<uint32_t>(__ldg(pz)) << 16);
     return r;
   }
@@ -319,6 +327,9 @@ struct Decoder {
     qkey = -1;
     qhead = head;
     omma_ = kMmaG;  // o is zero: either layout
+    ofg_ = FG;
+#pragma unroll
+    for (int gc = 0; gc < 4; ++gc) ZF[gc] = 0.f;
     __syncwarp();
   }
 
@@ -328,6 +339,12 @@ struct Decoder {
       if (omma_) {
         o_swap_layout();
         omma_ = false;
+      }
+    }
+    if constexpr (FG) {
+      if (ofg_) {
+        fg_to_residual_layout();
+        ofg_ = false;
       }
     }
   }
@@ -589,6 +606,186 @@ struct Decoder {
         base[16] = static_cast<uint8_t>((Q >> 16) & 255);
       }
     }
+  }
+
+  // ---- fine-grained groups (FG: 2 bits, one query per KV head) ----------------------------------
+  // Section KVキャッシュの分布特性: the K range is taken along each channel (one (s, z) per channel per
+  // g_k tokens: k_scale [bh][C / g_k][128]) and the V range along each token (one (s, z) per token per
+  // g_v channels: v_scale [bh][C][128 / g_v]).  K: the Q limbs q_c s_(u, c) and the constant
+  // sum_c q_c z_(u, c) are formed for each token group u of the unit (tile pair j uses group
+  // 32 j / g_k).  V: P_(t, gc) = p_t s_(t, gc) per channel group gc, one limb array per group; tile pair
+  // v holds channels 32 v .. 32 v + 31 (group 32 v / g_v) with tile (v, b) row g' + 8 c on channel
+  // 32 v + 16 b + 2 g' + c, so after the exchange lane (g, t) holds channel 32 v + 16 (t / 2) + 2 g +
+  // t % 2 in o[0][v].  sum_t p_t z_(t, gc) stays per group (ZF) until fg_to_residual_layout() adds it.
+
+  static __device__ __forceinline__ float sel4(const float (&x)[4], int i) {
+    return i == 0 ? x[0] : (i == 1 ? x[1] : (i == 2 ? x[2] : x[3]));
+  }
+
+  __device__ void fg_k(const uint8_t* kt, long long head, int local) {
+    const int ngt = UT >> a.lg_gk;  // K token groups in the unit: 4, 2 or 1
+    const size_t row0 = (static_cast<size_t>(head) * (static_cast<size_t>(a.capacity) >> a.lg_gk) +
+                         ((static_cast<size_t>(local) * UT) >> a.lg_gk)) * kHeadDim;
+    const int i = lane >> 2, kk = lane & 3, sw = (i >> 1) & 3;
+    __syncwarp();  // the previous unit's limbs are no longer read
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      if (u < ngt) {
+        float qv[4], qz = 0.f;
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+          const size_t ci = row0 + static_cast<size_t>(u) * kHeadDim + 16 * i + 4 * m + kk;
+          const float sk = h2f(__ldg(a.k_scale + ci)), zk = h2f(__ldg(a.k_zero + ci));
+          qv[m] = q_of(0, m) * sk;
+          qz = fmaf(q_of(0, m), zk, qz);
+        }
+        const float mabs = warp_max(fmaxf(fmaxf(fabsf(qv[0]), fabsf(qv[1])), fmaxf(fabsf(qv[2]), fabsf(qv[3]))));
+        const float scq = mabs > 0.f ? kQRangeBal * fast_rcp(mabs) : 0.f;
+        invqf[u] = mabs * (1.0f / kQRangeBal);
+        cblkf[u] = warp_sum(qz);
+        const float f = scq * ((lane & 1) ? 0.25f : 1.f);
+        uint32_t Q[4];
+#pragma unroll
+        for (int m = 0; m < 4; ++m) Q[m] = static_cast<uint32_t>(__float2int_rn(qv[m] * f));
+        uint32_t* row = reinterpret_cast<uint32_t*>(S.qw[u]) + 16 * i + kk;
+        row[4 * (0 ^ sw)] = pick_bytes(Q[0] + 32896u, Q[1] + 32896u, Q[2] + 32896u, Q[3] + 32896u, 2);
+        row[4 * (1 ^ sw)] = pick_bytes(Q[0] + 128u, Q[1] + 128u, Q[2] + 128u, Q[3] + 128u, 1);
+        row[4 * (2 ^ sw)] = pick_bytes(Q[0], Q[1], Q[2], Q[3], 0);
+      }
+    }
+    __syncwarp();
+    const int g = lane >> 2, t = lane & 3;
+    const int se = g < 4 ? g : 3, so = g >= 4 ? g - 4 : 3;
+    const bool odd = t & 1;
+    float lg[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int u = (32 * j) >> a.lg_gk;
+      const uint4 be0 = S.qw[u][8 * t + (se ^ t)], be1 = S.qw[u][8 * t + 4 + (se ^ t)];
+      const uint4 bo0 = S.qw[u][8 * t + (so ^ t)], bo1 = S.qw[u][8 * t + 4 + (so ^ t)];
+      int c[4] = {0, 0, 0, 0};
+#pragma unroll
+      for (int b = 0; b < 2; ++b) {
+        const uint8_t* r0 = kt + (32 * j + 16 * b + g) * 32 + 8 * t;
+        const uint2 wg = *reinterpret_cast<const uint2*>(r0);
+        const uint2 wh = *reinterpret_cast<const uint2*>(r0 + 8 * 32);
+        const uint4& B0 = b ? bo0 : be0;
+        const uint4& B1 = b ? bo1 : be1;
+        uint32_t mg[4], mh[4];
+        masks2(wg.x, mg);
+        masks2(wh.x, mh);
+        mma_u8s8(c, mg[0], mh[0], mg[1], mh[1], B0.x, B0.y);
+        mma_u8s8(c, mg[2], mh[2], mg[3], mh[3], B0.z, B0.w);
+        masks2(wg.y, mg);
+        masks2(wh.y, mh);
+        mma_u8s8(c, mg[0], mh[0], mg[1], mh[1], B1.x, B1.y);
+        mma_u8s8(c, mg[2], mh[2], mg[3], mh[3], B1.z, B1.w);
+      }
+      lg[j] = fmaf(gather_limbs(c, odd), sel4(invqf, u), sel4(cblkf, u));
+    }
+    softmax_fg(head, local, lg);
+  }
+
+  // Online softmax of the unit and the P limbs of each V channel group.  The lane's token
+  // 32 j + 16 (t / 2) + 8 (t % 2) + g has one (s, z) per channel group.
+  __device__ void softmax_fg(long long head, int local, const float (&lg)[4]) {
+    const int g = lane >> 2, t = lane & 3;
+    const int ngv = kHeadDim >> a.lg_gv;
+    float sv[4][4], zv[4][4], smax_l = 0.f;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const size_t tok = static_cast<size_t>(head) * a.capacity + static_cast<size_t>(local) * UT + 32 * j +
+                         16 * (t >> 1) + 8 * (t & 1) + g;
+#pragma unroll
+      for (int gc = 0; gc < 4; ++gc) {
+        sv[j][gc] = gc < ngv ? h2f(__ldg(a.v_scale + tok * ngv + gc)) : 0.f;
+        zv[j][gc] = gc < ngv ? h2f(__ldg(a.v_zero + tok * ngv + gc)) : 0.f;
+        smax_l = fmaxf(smax_l, sv[j][gc]);
+      }
+    }
+    const float mu = warp_max(fmaxf(fmaxf(lg[0], lg[1]), fmaxf(lg[2], lg[3])));
+    const float smax = warp_max(smax_l);
+    const float m_new = fmaxf(m[0], mu);
+    const float alpha = fast_exp2(m[0] - m_new);
+    const float d = mu - m_new;
+    const bool hv = d > -64.f && smax > 0.f;
+    const float fb = hv ? (kPRange * fast_rcp(smax)) * fast_exp2(-d) * ((g & 1) ? 0.25f : 1.f) : 0.f;
+    float psum = 0.f, zl[4] = {0.f, 0.f, 0.f, 0.f};
+    const int boff = 64 * (t >> 1) + 4 * (g & 3) + 2 * (t & 1) + (g >> 2);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float p = fast_exp2(lg[j] - m_new);
+      psum += p;
+#pragma unroll
+      for (int gc = 0; gc < 4; ++gc) {
+        if (gc < ngv) {
+          zl[gc] = fmaf(p, zv[j][gc], zl[gc]);
+          const uint32_t P = __float2uint_rn(p * (sv[j][gc] * fb));
+          uint8_t* pb = reinterpret_cast<uint8_t*>(S.pw[gc]) + boff + 128 * j;
+          pb[16 * (0 ^ j)] = static_cast<uint8_t>(P >> 16);
+          pb[16 * (1 ^ j)] = static_cast<uint8_t>(P >> 8);
+          pb[16 * (2 ^ j)] = static_cast<uint8_t>(P);
+        }
+      }
+    }
+    m[0] = m_new;
+    l[0] = fmaf(l[0], alpha, psum);
+    Z[0] *= alpha;
+#pragma unroll
+    for (int gc = 0; gc < 4; ++gc) ZF[gc] = fmaf(ZF[gc], alpha, zl[gc]);
+    alpha_[0] = alpha;
+    hasv_[0] = hv;
+    invv_[0] = hv ? fast_exp2(d) * smax * (1.0f / kPRange) : 0.f;
+  }
+
+  __device__ void v_mma_fg(const uint8_t* vt) {
+    const int g = lane >> 2, t = lane & 3;
+    const int se = g < 4 ? g : 3, so = g >= 4 ? g - 4 : 3;
+    const bool odd = t & 1;
+#pragma unroll
+    for (int v = 0; v < 4; ++v) {
+      const int gc = (32 * v) >> a.lg_gv;
+      int cv[4] = {0, 0, 0, 0};
+#pragma unroll
+      for (int x = 0; x < 2; ++x) {
+        const uint4 be = S.pw[gc][8 * t + 4 * x + (se ^ t)], bo = S.pw[gc][8 * t + 4 * x + (so ^ t)];
+        const uint8_t* rowp = vt + t * kVPieceStride + x * 512 + 4 * (32 * v + 2 * g);
+        const uint2 w0 = *reinterpret_cast<const uint2*>(rowp);           // tile (v, 0): rows g, g + 8
+        const uint2 w1 = *reinterpret_cast<const uint2*>(rowp + 4 * 16);  // tile (v, 1)
+        uint32_t mg[4], mh[4];
+        masks2(w0.x, mg);
+        masks2(w0.y, mh);
+        mma_u8u8(cv, mg[0], mh[0], mg[1], mh[1], be.x, be.y);
+        mma_u8u8(cv, mg[2], mh[2], mg[3], mh[3], be.z, be.w);
+        masks2(w1.x, mg);
+        masks2(w1.y, mh);
+        mma_u8u8(cv, mg[0], mh[0], mg[1], mh[1], bo.x, bo.y);
+        mma_u8u8(cv, mg[2], mh[2], mg[3], mh[3], bo.z, bo.w);
+      }
+      o[0][v] = fmaf(o[0][v], alpha_[0], gather_limbs(cv, odd) * invv_[0]);
+    }
+  }
+
+  // o from the FG layout to the residual layout (lane l: channels 4 l .. 4 l + 3), with each V
+  // channel group's z term added to its channels.
+  __device__ void fg_to_residual_layout() {
+    const int g = lane >> 2, t = lane & 3;
+    float zs[4];
+#pragma unroll
+    for (int gc = 0; gc < 4; ++gc) zs[gc] = warp_sum(ZF[gc]);
+    __syncwarp();
+#pragma unroll
+    for (int v = 0; v < 4; ++v) S.oscr[32 * v + 16 * (t >> 1) + 2 * g + (t & 1)] = o[0][v];
+    __syncwarp();
+    const float4 ov = *reinterpret_cast<const float4*>(S.oscr + 4 * lane);
+    const float zc = sel4(zs, (4 * lane) >> a.lg_gv);
+    o[0][0] = ov.x + zc;
+    o[0][1] = ov.y + zc;
+    o[0][2] = ov.z + zc;
+    o[0][3] = ov.w + zc;
+#pragma unroll
+    for (int gc = 0; gc < 4; ++gc) ZF[gc] = 0.f;
+    __syncwarp();
   }
 
   // ---- tensor-core path, several queries per KV head ------------------------------------------
@@ -884,6 +1081,10 @@ struct Decoder {
 
   // ---- K half of a quantized unit: logits, online softmax, P limbs (A6, A8, A9 set-up) ---------
   __device__ void quantized_k(const uint8_t* kt, long long head, int local, uint32_t pairs) {
+    if constexpr (FG) {
+      fg_k(kt, head, local);
+      return;
+    }
     const long long key = head * a.blocks_per_head + (local >> a.lg_units_per_blk);
     if (key != qkey) {
       build_q(pairs);
@@ -970,6 +1171,8 @@ struct Decoder {
     if (G == 1 && !hasv_[0]) {  // every weight of the unit is zero: only rescale
 #pragma unroll
       for (int e = 0; e < 4; ++e) o[0][e] *= alpha_[0];
+    } else if constexpr (FG) {
+      v_mma_fg(vt);
     } else if constexpr (kMma1) {
       v_mma(vt);
     } else if constexpr (kMmaG) {
@@ -1309,7 +1512,7 @@ struct Decoder {
       asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     if constexpr (kMma) {  // slot 3 of every limb row stays zero; slots 0..2 are written before use
-      for (int i = lane; i < 4 * kLimbVecs * G; i += 32) {
+      for (int i = lane; i < static_cast<int>(sizeof(S.qw) / 4); i += 32) {
         reinterpret_cast<uint32_t*>(S.qw)[i] = 0u;
         reinterpret_cast<uint32_t*>(S.pw)[i] = 0u;
       }
@@ -1389,50 +1592,70 @@ struct Decoder {
   }
 };
 
-template <int BITS, int G, bool KC>
+template <int BITS, int G, bool KC, bool FG = false>
 __global__ void __launch_bounds__(warps_per_cta<G>() * 32, 1) decode_kernel(const __grid_constant__ DecodeArgs a) {
   extern __shared__ __align__(128) uint8_t smem_raw[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  WarpSmem<G>& S = reinterpret_cast<WarpSmem<G>*>(smem_raw)[warp];
+  WarpSmem<G, FG>& S = reinterpret_cast<WarpSmem<G, FG>*>(smem_raw)[warp];
   const long long W = a.workers, U = a.total_units;
   const long long worker = static_cast<long long>(blockIdx.x) * warps_per_cta<G>() + warp;
   if (worker >= W) return;  // the last CTA may hold fewer workers
   const long long ub = U * worker / W, ue = U * (worker + 1) / W;  // non-empty because W <= U
-  Decoder<BITS, G, KC> d(a, S, lane, worker, ub, ue);
+  Decoder<BITS, G, KC, FG> d(a, S, lane, worker, ub, ue);
   d.run();
 }
 
-template <int BITS, int G>
-cudaError_t plan_for(DecodePlan* plan) {
+template <int BITS, int G, bool FG>
+cudaError_t plan_for_kernels(DecodePlan* plan) {
   constexpr int kWarps = warps_per_cta<G>();
-  const int smem = kWarps * static_cast<int>(sizeof(WarpSmem<G>));
-  cudaError_t e = cudaFuncSetAttribute(decode_kernel<BITS, G, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  const int smem = kWarps * static_cast<int>(sizeof(WarpSmem<G, FG>));
+  cudaError_t e = cudaFuncSetAttribute(decode_kernel<BITS, G, false, FG>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(decode_kernel<BITS, G, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  if (e != cudaSuccess) return e;
+  if constexpr (!FG) {
+    e = cudaFuncSetAttribute(decode_kernel<BITS, G, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+  }
   int dev = 0, sms = 0, occ = 0;
   if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
   if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
-  if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, decode_kernel<BITS, G, false>, kWarps * 32, smem)) !=
+  if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, decode_kernel<BITS, G, false, FG>, kWarps * 32, smem)) !=
       cudaSuccess)
     return e;
   if (occ < 1) return cudaErrorInvalidConfiguration;
   plan->warps_per_cta = kWarps;
   plan->ctas = sms * occ;
   plan->smem_bytes = smem;
-  plan->unit_tokens = Decoder<BITS, G, false>::UT;
+  plan->unit_tokens = Decoder<BITS, G, false, FG>::UT;
   plan->res_unit_tokens = kResTokens;
   return cudaSuccess;
+}
+
+// Fine-grained groups are built for 2 bits and one query per KV head.
+template <int BITS, int G>
+cudaError_t plan_for(DecodePlan* plan, int fine) {
+  if (fine) {
+    if constexpr (BITS == 2 && G == 1)
+      return plan_for_kernels<BITS, G, true>(plan);
+    else
+      return cudaErrorInvalidValue;
+  }
+  return plan_for_kernels<BITS, G, false>(plan);
 }
 
 template <int BITS, int G>
 cudaError_t launch_for(const DecodeArgs& a, const DecodePlan& plan, cudaStream_t stream) {
   if (a.workers < 1 || a.workers > plan.workers() || a.total_units < a.workers) return cudaErrorInvalidValue;
   const int ctas = (a.workers + plan.warps_per_cta - 1) / plan.warps_per_cta;
-  if (a.k_res_coded)
+  if (a.fine) {
+    if constexpr (BITS == 2 && G == 1)
+      decode_kernel<BITS, G, false, true><<<ctas, plan.warps_per_cta * 32, plan.smem_bytes, stream>>>(a);
+    else
+      return cudaErrorInvalidValue;
+  } else if (a.k_res_coded) {
     decode_kernel<BITS, G, true><<<ctas, plan.warps_per_cta * 32, plan.smem_bytes, stream>>>(a);
-  else
+  } else {
     decode_kernel<BITS, G, false><<<ctas, plan.warps_per_cta * 32, plan.smem_bytes, stream>>>(a);
+  }
   return cudaGetLastError();
 }
 
@@ -1458,7 +1681,9 @@ cudaError_t launch_for(const DecodeArgs& a, const DecodePlan& plan, cudaStream_t
     return cudaErrorInvalidValue;                                        \
   } while (0)
 
-cudaError_t decode_plan(int bits, int gqa, DecodePlan* plan) { KIVI_DISPATCH(bits, gqa, plan_for, plan); }
+cudaError_t decode_plan(int bits, int gqa, int fine, DecodePlan* plan) {
+  KIVI_DISPATCH(bits, gqa, plan_for, plan, fine);
+}
 
 cudaError_t launch_decode(const DecodeArgs& a, int bits, const DecodePlan& plan, cudaStream_t stream) {
   KIVI_DISPATCH(bits, a.gqa, launch_for, a, plan, stream);

@@ -27,6 +27,8 @@ struct QuantizeArgs {
   int lg_gk, lg_gv;  // log2(group_k), log2(group_v): set by launch_quantize_blocks
   int k_given;       // 1: the K (s, z) of each block are already in k_scale / k_zero (prefix groups)
   int v_only;        // 1: quantize the V blocks only (online K: the K codes are in place)
+  int fine;          // 1: fine-grained groups: K (s, z) per channel per group_k tokens
+                     //    ([bh][C/group_k][128]), V (s, z) per token per group_v channels ([bh][C][128/group_v])
 };
 
 // Online K: codes `rows` K rows per head (fp16 source rows src_tok0 .. of a [bh][src_tokens][128]
@@ -82,6 +84,9 @@ struct DecodeArgs {
   // online K: the residual tokens' K rows are code rows n_quant .. of k_codes with the (s, z) of
   // block res_blk (= n_quant / residual); 0: fp16 rows of k_res
   int k_res_coded, res_blk;
+  // fine-grained groups (2 bits, one query per KV head): k_scale / k_zero [bh][C >> lg_gk][128]
+  // (lg_gk: tokens per K group), v_scale / v_zero [bh][C][128 >> lg_gv] (lg_gv: channels per V group)
+  int fine;
 };
 
 constexpr int kPartialStride = 132;  // m, l, Z, pad, o[128]
@@ -102,7 +107,7 @@ struct DecodePlan {
   int res_unit_tokens;  // tokens per residual unit
   int workers() const { return warps_per_cta * ctas; }
 };
-cudaError_t decode_plan(int bits, int gqa, DecodePlan* plan);
+cudaError_t decode_plan(int bits, int gqa, int fine, DecodePlan* plan);
 cudaError_t launch_decode(const DecodeArgs& a, int bits, const DecodePlan& plan, cudaStream_t stream);
 
 }  // namespace kivi

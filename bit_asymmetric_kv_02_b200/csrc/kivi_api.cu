@@ -46,8 +46,15 @@ int check_cfg(const kivi_config* c) {
   if (c->residual < 128 || c->residual > 1024 || !pow2(c->residual)) return KIVI_ERR_INVALID_ARG;
   if (c->capacity % c->residual != 0) return KIVI_ERR_INVALID_ARG;
   if (c->group_k != 32 && c->group_k != 64 && c->group_k != 128) return KIVI_ERR_INVALID_ARG;
-  if (c->group_v < 32 || !pow2(c->group_v) || c->group_v > c->residual) return KIVI_ERR_INVALID_ARG;
+  if (c->fine_groups != 0 && c->fine_groups != 1) return KIVI_ERR_INVALID_ARG;
+  if (c->fine_groups) {  // group_k: tokens (<= R), group_v: channels
+    if (c->group_k > c->residual) return KIVI_ERR_INVALID_ARG;
+    if (c->group_v != 32 && c->group_v != 64 && c->group_v != 128) return KIVI_ERR_INVALID_ARG;
+  } else if (c->group_v < 32 || !pow2(c->group_v) || c->group_v > c->residual) {
+    return KIVI_ERR_INVALID_ARG;
+  }
   if (c->online_k != 0 && c->online_k != 1) return KIVI_ERR_INVALID_ARG;
+  if (c->online_k && c->fine_groups) return KIVI_ERR_UNSUPPORTED;
   if (static_cast<long long>(c->batch) * c->num_kv_heads > (1ll << 30)) return KIVI_ERR_UNSUPPORTED;
   if (c->capacity / c->residual > 32767) return KIVI_ERR_UNSUPPORTED;  // grid.y limit of a prefill
   return KIVI_OK;
@@ -71,7 +78,7 @@ bool cache_ptrs_ok(const kivi_cache* k, bool need_codes) {
 struct PlanCache {
   std::mutex mu;
   struct Entry {
-    int dev, bits, gqa;
+    int dev, bits, gqa, fine;
     DecodePlan plan;
   };
   Entry entries[64];
@@ -82,21 +89,22 @@ PlanCache& plan_cache() {
   return c;
 }
 
-cudaError_t get_plan(int bits, int gqa, DecodePlan* out) {
+cudaError_t get_plan(int bits, int gqa, int fine, DecodePlan* out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   PlanCache& pc = plan_cache();
   std::lock_guard<std::mutex> lock(pc.mu);
   for (int i = 0; i < pc.n; ++i) {
-    if (pc.entries[i].dev == dev && pc.entries[i].bits == bits && pc.entries[i].gqa == gqa) {
+    if (pc.entries[i].dev == dev && pc.entries[i].bits == bits && pc.entries[i].gqa == gqa &&
+        pc.entries[i].fine == fine) {
       *out = pc.entries[i].plan;
       return cudaSuccess;
     }
   }
   DecodePlan p{};
-  if ((e = kivi::decode_plan(bits, gqa, &p)) != cudaSuccess) return e;
-  if (pc.n < 64) pc.entries[pc.n++] = {dev, bits, gqa, p};
+  if ((e = kivi::decode_plan(bits, gqa, fine, &p)) != cudaSuccess) return e;
+  if (pc.n < 64) pc.entries[pc.n++] = {dev, bits, gqa, fine, p};
   *out = p;
   return cudaSuccess;
 }
@@ -167,8 +175,13 @@ int kivi_cache_sizes(const kivi_config* cfg, size_t* out) {
   const size_t code_bytes = bh * C * d * cfg->bits / 8;
   out[KIVI_BUF_K_CODES] = code_bytes;
   out[KIVI_BUF_V_CODES] = code_bytes;
-  out[KIVI_BUF_K_SCALE] = out[KIVI_BUF_K_ZERO] = bh * (C / cfg->residual) * (d / cfg->group_k) * 2;
-  out[KIVI_BUF_V_SCALE] = out[KIVI_BUF_V_ZERO] = bh * (C / cfg->group_v) * 2;
+  if (cfg->fine_groups) {
+    out[KIVI_BUF_K_SCALE] = out[KIVI_BUF_K_ZERO] = bh * (C / cfg->group_k) * d * 2;
+    out[KIVI_BUF_V_SCALE] = out[KIVI_BUF_V_ZERO] = bh * C * (d / cfg->group_v) * 2;
+  } else {
+    out[KIVI_BUF_K_SCALE] = out[KIVI_BUF_K_ZERO] = bh * (C / cfg->residual) * (d / cfg->group_k) * 2;
+    out[KIVI_BUF_V_SCALE] = out[KIVI_BUF_V_ZERO] = bh * (C / cfg->group_v) * 2;
+  }
   out[KIVI_BUF_K_RES] = out[KIVI_BUF_V_RES] = bh * cfg->residual * d * 2;
   return KIVI_OK;
 }
@@ -184,7 +197,7 @@ int prefill_impl(const kivi_config* cfg, kivi_cache* cache, const uint16_t* k_de
   const int n_res = (num_tokens - 1) % R + 1;
   const int n_quant = num_tokens - n_res;
   if (n_quant > cfg->capacity) return KIVI_ERR_CAPACITY;
-  if (prefix_k && cfg->online_k) return KIVI_ERR_UNSUPPORTED;
+  if (prefix_k && (cfg->online_k || cfg->fine_groups)) return KIVI_ERR_UNSUPPORTED;
   if (k_online(cfg, n_quant) && n_quant + R > cfg->capacity) return KIVI_ERR_CAPACITY;
   if (!cache_ptrs_ok(cache, n_quant > 0)) return KIVI_ERR_INVALID_ARG;
   kivi::QuantizeArgs a{};
@@ -209,6 +222,7 @@ int prefill_impl(const kivi_config* cfg, kivi_cache* cache, const uint16_t* k_de
   a.capacity = cfg->capacity;
   a.group_k = cfg->group_k;
   a.group_v = cfg->group_v;
+  a.fine = cfg->fine_groups;
   if (prefix_k && a.nblocks > 0) {
     if (kivi::launch_k_prefix_extremes(a, cfg->bits, static_cast<cudaStream_t>(stream)) != cudaSuccess)
       return KIVI_ERR_CUDA;
@@ -297,6 +311,7 @@ int kivi_flush_residual(const kivi_config* cfg, kivi_cache* cache, void* stream)
   a.group_k = cfg->group_k;
   a.group_v = cfg->group_v;
   a.v_only = k_online(cfg, cache->n_quant) ? 1 : 0;  // online K: the block's K codes are in place
+  a.fine = cfg->fine_groups;
   if (kivi::launch_quantize_blocks(a, cfg->bits, static_cast<cudaStream_t>(stream)) != cudaSuccess)
     return KIVI_ERR_CUDA;
   cache->n_quant += R;
@@ -309,7 +324,7 @@ size_t kivi_decode_workspace_bytes(const kivi_config* cfg, int32_t num_q_heads) 
   const int gqa = num_q_heads / cfg->num_kv_heads;
   if (!gqa_supported(gqa)) return 0;
   DecodePlan p{};
-  if (get_plan(cfg->bits, gqa, &p) != cudaSuccess) return 0;
+  if (get_plan(cfg->bits, gqa, cfg->fine_groups && cfg->bits == 2 && gqa == 1, &p) != cudaSuccess) return 0;
   const size_t bh = static_cast<size_t>(cfg->batch) * cfg->num_kv_heads;
   return align256(static_cast<size_t>(p.workers()) * 2 * gqa * kivi::kPartialStride * sizeof(float)) +
          align256(bh * sizeof(int32_t));
@@ -329,6 +344,7 @@ int decode_impl(const kivi_config* cfg, const kivi_cache* cache, const uint16_t*
   if (num_q_heads < 1 || num_q_heads % cfg->num_kv_heads != 0) return KIVI_ERR_INVALID_ARG;
   const int gqa = num_q_heads / cfg->num_kv_heads;
   if (!gqa_supported(gqa)) return KIVI_ERR_UNSUPPORTED;
+  if (cfg->fine_groups && (cfg->bits != 2 || gqa != 1)) return KIVI_ERR_UNSUPPORTED;
   if (!aligned16(q_dev) || !aligned16(out_dev) || !(scale == scale) || scale > 3.0e38f || scale < -3.0e38f)
     return KIVI_ERR_INVALID_ARG;
   if (cache->n_quant + cache->n_res == 0) return KIVI_ERR_EMPTY;
@@ -337,7 +353,7 @@ int decode_impl(const kivi_config* cfg, const kivi_cache* cache, const uint16_t*
   if (coded_res && (cache->n_quant + cfg->residual > cfg->capacity || new_slot >= 0)) return KIVI_ERR_STATE;
   if (dev_status != nullptr && (reinterpret_cast<uintptr_t>(dev_status) & 3u) != 0) return KIVI_ERR_INVALID_ARG;
   DecodePlan plan{};
-  if (get_plan(cfg->bits, gqa, &plan) != cudaSuccess) return KIVI_ERR_CUDA;
+  if (get_plan(cfg->bits, gqa, cfg->fine_groups, &plan) != cudaSuccess) return KIVI_ERR_CUDA;
   const size_t bh = static_cast<size_t>(cfg->batch) * cfg->num_kv_heads;
   const size_t part_bytes = align256(static_cast<size_t>(plan.workers()) * 2 * gqa * kivi::kPartialStride * 4);
   if (workspace_dev == nullptr || (reinterpret_cast<uintptr_t>(workspace_dev) & 255u) != 0 ||
@@ -393,6 +409,7 @@ int decode_impl(const kivi_config* cfg, const kivi_cache* cache, const uint16_t*
   a.v_new = v_new_dev;
   a.new_slot = new_slot;
   a.k_res_coded = coded_res ? 1 : 0;
+  a.fine = cfg->fine_groups;
   a.res_blk = cache->n_quant / cfg->residual;
   if (new_slot == -2) return KIVI_OK;  // arguments checked, nothing enqueued
   if (kivi::launch_decode(a, cfg->bits, plan, static_cast<cudaStream_t>(stream)) != cudaSuccess)

@@ -581,6 +581,123 @@ __global__ void __launch_bounds__(256) append_kernel(AppendArgs a) {
   reinterpret_cast<uint4*>(a.v_res)[dst] = __ldg(reinterpret_cast<const uint4*>(a.v_new) + i);
 }
 
+// ---------------------------------------------------------------------------------------------
+// Fine-grained groups (section KVキャッシュの分布特性: the K range along each channel, the V range
+// along each token).  grid: x = batch * kv_heads, y = 2 * nblocks (+1 residual-copy job); 128
+// threads, thread c owns channel c.  K: per group of g_k tokens, thread c reduces its channel, forms
+// (s, z) and codes the group's tokens (the P threads of a code word OR their codes together).
+// V: per token, the g_v threads of a channel group reduce it (warp shuffles, then shared memory
+// across warps for g_v > 32), and thread c shifts its code into its channel's word of P tokens.
+// ---------------------------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t quantize_one(float x, const GroupParams& g, int levels) {
+  constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23: rounds r to the nearest integer, ties to even
+  const float r = __fmul_rn(__fadd_rn(x, -g.zf), g.inv_s);
+  const float t = __fadd_rn(r, kMagic);
+  const float dr = __fadd_rn(r, __fadd_rn(kMagic, -t));
+  uint32_t q = min(__float_as_uint(t) - 0x4B400000u, static_cast<uint32_t>(levels));
+  if (fabsf(dr) > 0.499755859375f) q = quantize_exact(x, g, levels);  // within 2^-12 of a tie
+  return g.inv_s == 0.f ? 0u : q;
+}
+
+template <int BITS>
+__global__ void __launch_bounds__(kHeadDim) quantize_fine_kernel(QuantizeArgs a) {
+  constexpr int P = 32 / BITS, L = (1 << BITS) - 1;
+  __shared__ float red_lo[8][kHeadDim / 32], red_hi[8][kHeadDim / 32];
+  const int bh = blockIdx.x, job = blockIdx.y, c = threadIdx.x, warp = c >> 5;
+  const int R = a.residual;
+  const size_t C = static_cast<size_t>(a.capacity);
+  if (job >= 2 * a.nblocks) {
+    copy_residual(a, bh);
+    return;
+  }
+  const int blk = job >> 1;
+  const bool is_v = job & 1;
+  if (a.v_only && !is_v) return;
+  const size_t src_tok = static_cast<size_t>(bh) * a.src_tokens + a.src_tok0 + static_cast<size_t>(blk) * R;
+  const size_t dst_tok = static_cast<size_t>(a.dst_blk0 + blk) * R;
+  const unsigned word_mask = (P == 32 ? 0xffffffffu : ((1u << P) - 1u)) << ((c & 31) & ~(P - 1));
+  if (!is_v) {
+    const uint16_t* src = a.k_src + src_tok * kHeadDim + c;
+    const int gk = a.group_k;
+    for (int u = 0; u < R / gk; ++u) {
+      float lo = INFINITY, hi = -INFINITY;
+      for (int t = 0; t < gk; ++t) {
+        const float x = h2f(__ldg(src + static_cast<size_t>(u * gk + t) * kHeadDim));
+        lo = fminf(lo, x);
+        hi = fmaxf(hi, x);
+      }
+      const GroupParams gp = make_group(lo, hi, L);
+      const size_t si = (static_cast<size_t>(bh) * (C / gk) + (dst_tok / gk) + u) * kHeadDim + c;
+      a.k_scale[si] = gp.s_bits;
+      a.k_zero[si] = gp.z_bits;
+      for (int t = 0; t < gk; ++t) {
+        const int tok = u * gk + t;
+        const uint32_t q = quantize_one(h2f(__ldg(src + static_cast<size_t>(tok) * kHeadDim)), gp, L);
+        const uint32_t word = __reduce_or_sync(word_mask, q << (BITS * (c & (P - 1))));
+        if ((c & (P - 1)) == 0)
+          a.k_codes[(static_cast<size_t>(bh) * C + dst_tok + tok) * (kHeadDim / P) + c / P] = word;
+      }
+    }
+  } else {
+    const uint16_t* src = a.v_src + src_tok * kHeadDim + c;
+    const int gv = a.group_v, wpg = gv >> 5;  // warps per channel group
+    const int ngv = kHeadDim / gv, g = c / gv;
+    uint32_t word = 0u;
+    for (int t0 = 0; t0 < R; t0 += 8) {
+      float x[8], lo[8], hi[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        x[i] = h2f(__ldg(src + static_cast<size_t>(t0 + i) * kHeadDim));
+        lo[i] = x[i];
+        hi[i] = x[i];
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+          lo[i] = fminf(lo[i], __shfl_xor_sync(0xffffffffu, lo[i], off));
+          hi[i] = fmaxf(hi[i], __shfl_xor_sync(0xffffffffu, hi[i], off));
+        }
+      }
+      if (wpg > 1) {
+        __syncthreads();  // the previous batch's partials are read
+        float mlo = lo[0], mhi = hi[0];  // lane i < 8 publishes token i's warp extremes
+#pragma unroll
+        for (int i = 1; i < 8; ++i) {
+          if ((c & 7) == i) {
+            mlo = lo[i];
+            mhi = hi[i];
+          }
+        }
+        if ((c & 31) < 8) {
+          red_lo[c & 31][warp] = mlo;
+          red_hi[c & 31][warp] = mhi;
+        }
+        __syncthreads();
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          for (int w = g * wpg; w < (g + 1) * wpg; ++w) {
+            lo[i] = fminf(lo[i], red_lo[i][w]);
+            hi[i] = fmaxf(hi[i], red_hi[i][w]);
+          }
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int tok = t0 + i;
+        const GroupParams gp = make_group(lo[i], hi[i], L);
+        if (c % gv == 0) {
+          const size_t si = (static_cast<size_t>(bh) * C + dst_tok + tok) * ngv + g;
+          a.v_scale[si] = gp.s_bits;
+          a.v_zero[si] = gp.z_bits;
+        }
+        word |= quantize_one(x[i], gp, L) << (BITS * (tok & (P - 1)));
+        if ((tok & (P - 1)) == P - 1) {
+          a.v_codes[(static_cast<size_t>(bh) * (C / P) + (dst_tok + tok) / P) * kHeadDim + c] = word;
+          word = 0u;
+        }
+      }
+    }
+  }
+}
+
 // Online K (section Per-Channel量子化: a new token's K is quantized at once with the existing scale
 // and zero point).  grid: x = batch * kv_heads, y = rows; 128 threads, one per channel.  The code
 // is clamp(rint((x - z) / s), 0, L) in fp64, which decides exactly: x - z of two fp16 values is
@@ -667,7 +784,12 @@ cudaError_t launch_quantize_blocks(const QuantizeArgs& args, int bits, cudaStrea
   a.lg_gk = __builtin_ctz(static_cast<unsigned>(a.group_k));
   a.lg_gv = __builtin_ctz(static_cast<unsigned>(a.group_v));
   dim3 grid(a.bh, jobs);
-  if (a.residual <= 512) {  // one thread per 8 tokens x 8 channels of a block
+  if (a.fine) {
+    if (bits == 2)
+      quantize_fine_kernel<2><<<grid, kHeadDim, 0, stream>>>(a);
+    else
+      quantize_fine_kernel<4><<<grid, kHeadDim, 0, stream>>>(a);
+  } else if (a.residual <= 512) {  // one thread per 8 tokens x 8 channels of a block
     if (bits == 2)
       quantize_tiles_kernel<2><<<grid, 2 * a.residual, 0, stream>>>(a);
     else

@@ -33,7 +33,7 @@ class KiviError(RuntimeError):
 class kivi_config(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in
                 ("batch", "num_kv_heads", "head_dim", "bits", "group_k", "group_v", "residual", "capacity",
-                 "online_k")]
+                 "online_k", "fine_groups")]
 
 
 class kivi_cache(ctypes.Structure):
@@ -167,12 +167,12 @@ class KiviCache:
 
     def __init__(self, batch: int, num_kv_heads: int, capacity: int, bits: int = 2, group_k: int = 32,
                  group_v: int = 32, residual: int = 128, head_dim: int = 128, num_q_heads: int | None = None,
-                 device=None, online_k: bool = False):
+                 device=None, online_k: bool = False, fine_groups: bool = False):
         import torch
         self.torch = torch
         self.device = torch.device(device or "cuda")
         self.cfg = kivi_config(batch, num_kv_heads, head_dim, bits, group_k, group_v, residual, capacity,
-                               1 if online_k else 0)
+                               1 if online_k else 0, 1 if fine_groups else 0)
         st = kivi_check_config(self.cfg)
         if st != KIVI_OK:
             raise KiviError(st, "kivi_check_config")
@@ -203,6 +203,10 @@ class KiviCache:
             "v_scale": (t.float16, (B, H, C // c.group_v)), "v_zero": (t.float16, (B, H, C // c.group_v)),
             "k_res": (t.float16, (B, H, R, d)), "v_res": (t.float16, (B, H, R, d)),
         }
+        if c.fine_groups:   # K: per channel per group_k tokens; V: per token per group_v channels
+            for n_, sh in (("k_scale", (B, H, C // c.group_k, d)), ("k_zero", (B, H, C // c.group_k, d)),
+                           ("v_scale", (B, H, C, d // c.group_v)), ("v_zero", (B, H, C, d // c.group_v))):
+                shapes[n_] = (t.float16, sh)
         dtype, shape = shapes[name]
         n = math.prod(shape) * (4 if dtype == t.int32 else 2)
         return self.buffers[name][:n].view(dtype).view(shape)

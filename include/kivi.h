@@ -36,8 +36,10 @@
  *                                     P*i + j (j = 0..P-1) at bits [b*j, b*j + b).
  *   v_codes  uint32 [B][H][C/P][d]   channel-major within P-token rows.  Word (r, c) holds the
  *                                     codes of tokens P*r + j of channel c at bits [b*j, b*j + b).
- *   k_scale, k_zero  fp16 [B][H][C/R][d/G_k]   one pair per (R-token block, channel group).
- *   v_scale, v_zero  fp16 [B][H][C/G_v]        one pair per G_v-token group.
+ *   k_scale, k_zero  fp16 [B][H][C/R][d/G_k]   one pair per (R-token block, channel group);
+ *                    fine_groups: [B][H][C/G_k][d], one pair per (G_k-token group, channel).
+ *   v_scale, v_zero  fp16 [B][H][C/G_v]        one pair per G_v-token group;
+ *                    fine_groups: [B][H][C][d/G_v], one pair per (token, G_v-channel group).
  *   k_res, v_res     fp16 [B][H][R][d]         residual slots 0..n_res-1 hold the newest tokens.
  *   Token order of a head: quantized tokens 0..n_quant-1, then residual slots 0..n_res-1.
  * Host inputs: k, v fp16 [B][H][T][d]; k_new, v_new fp16 [B][H][d]; q, out fp16 [B][Hq][d].
@@ -55,7 +57,7 @@
 extern "C" {
 #endif
 
-#define KIVI_ABI_VERSION 2
+#define KIVI_ABI_VERSION 3
 
 /* Status codes. */
 #define KIVI_OK 0
@@ -76,7 +78,7 @@ extern "C" {
  * group_size_k, group_size_v, residual_length) plus the shape and capacity of the cache.
  * Rules: batch >= 1, num_kv_heads >= 1, capacity >= 0, capacity % residual == 0,
  * residual in {128, 256, 512, 1024}, group_k in {32, 64, 128}, group_v a power of two with
- * 32 <= group_v <= residual, online_k in {0, 1} (KIVI_ERR_INVALID_ARG otherwise);
+ * 32 <= group_v <= residual, online_k in {0, 1}, fine_groups in {0, 1} (KIVI_ERR_INVALID_ARG otherwise);
  * head_dim == 128, bits in {2, 4} (KIVI_ERR_UNSUPPORTED otherwise).
  *
  * online_k = 1 selects online K quantization (section Per-Channel量子化: a new token's K can be
@@ -87,6 +89,15 @@ extern "C" {
  * residual and its flush.  Before the first block exists K stays fp16 as with online_k = 0.
  * Such a cache needs n_quant + R <= capacity whenever it holds residual tokens (KIVI_ERR_CAPACITY
  * from the prefill or append that would break it).
+ *
+ * fine_groups = 1 selects fine-grained groups (section KVキャッシュの分布特性: the K range along each
+ * channel, the V range along each token): group_k then counts TOKENS (one K (s, z) per channel per
+ * group_k consecutive tokens; group_k in {32, 64, 128}, group_k <= residual) and group_v counts
+ * CHANNELS (one V (s, z) per token per group_v consecutive channels; group_v in {32, 64, 128}).
+ * The scale layouts change (see DEVICE LAYOUT); codes, residual, blocks and flushes do not.
+ * Decode attention over such a cache is built for bits == 2 with one query head per KV head
+ * (KIVI_ERR_UNSUPPORTED otherwise); it is not combined with online_k or the prefix-K prefill
+ * (KIVI_ERR_UNSUPPORTED).
  */
 typedef struct kivi_config {
   int32_t batch;        /* B */
@@ -98,6 +109,7 @@ typedef struct kivi_config {
   int32_t residual;     /* R: residual (fp16) capacity in tokens, also the K block length */
   int32_t capacity;     /* C: maximum number of quantized tokens per head */
   int32_t online_k;     /* 0: K residual in fp16; 1: online K quantization (see above) */
+  int32_t fine_groups;  /* 0: block / token groups; 1: fine-grained groups (see above) */
 } kivi_config;
 
 /* Device buffers of one cache (caller-owned) plus the two host-side counters the calls advance.

@@ -33,7 +33,7 @@ def test_every_declared_symbol_is_exported(kivi):
 
 
 def test_version_and_strerror(kivi):
-    assert kivi.kivi_abi_version() == 2
+    assert kivi.kivi_abi_version() == 3
     assert kivi.kivi_strerror(0) == "ok"
     assert "flush" in kivi.kivi_strerror(4)
     assert kivi.kivi_strerror(12345) == "unknown status"
@@ -149,6 +149,29 @@ def test_online_k_host_errors(kivi):
     assert e.value.code == "CAPACITY" and (cache.n_quant, cache.n_res) == (1024, 3)
     with pytest.raises(kivi.KiviError) as e:
         kivi.kivi_quantize_prefill_prefix_k(cfg, cache, fake, fake, 300, 0)
+    assert e.value.code == "UNSUPPORTED"
+
+
+def test_fine_groups_host_rules(kivi):
+    """Fine-grained groups (section KVキャッシュの分布特性): group_k counts tokens (<= R), group_v counts
+    channels; the scale buffers change size; decode is built for 2 bits and one query per KV head."""
+    assert kivi.kivi_check_config(_cfg(kivi, fine_groups=1)) == 0
+    assert kivi.kivi_check_config(_cfg(kivi, fine_groups=2)) == 1
+    assert kivi.kivi_check_config(_cfg(kivi, fine_groups=1, group_v=256, residual=256, capacity=1024)) == 1
+    assert kivi.kivi_check_config(_cfg(kivi, fine_groups=1, group_k=128, group_v=64)) == 0
+    assert kivi.kivi_check_config(_cfg(kivi, fine_groups=1, online_k=1)) == 2
+    sizes = kivi.kivi_cache_sizes(_cfg(kivi, fine_groups=1, group_k=64, group_v=32))
+    bh = 2 * 3
+    assert sizes[2] == sizes[3] == bh * (1024 // 64) * 128 * 2      # K: [C/G_k][d]
+    assert sizes[4] == sizes[5] == bh * 1024 * (128 // 32) * 2      # V: [C][d/G_v]
+    fake = 1 << 20
+    cache = kivi.kivi_cache(*([fake] * 8), 128, 3)
+    for cfg, hq in ((_cfg(kivi, fine_groups=1, bits=4), 3), (_cfg(kivi, fine_groups=1), 6)):
+        with pytest.raises(kivi.KiviError) as e:
+            kivi.kivi_decode_attention(cfg, cache, fake, hq, 0.1, fake, fake, 1 << 30, None, 0)
+        assert e.value.code == "UNSUPPORTED"
+    with pytest.raises(kivi.KiviError) as e:
+        kivi.kivi_quantize_prefill_prefix_k(_cfg(kivi, fine_groups=1), cache, fake, fake, 300, 0)
     assert e.value.code == "UNSUPPORTED"
 
 
