@@ -41,6 +41,7 @@ FUSED = True   # append and decode in one launch (kivi_append_decode_attention);
 STEP_NOTE = {True: "flush when full + append and decode attention in one launch",
              False: "flush when full + append + decode attention"}
 ONLINE_K = False   # --online-k: K rows coded at append with the newest block's (s, z) (config online_k)
+FINE = False       # --fine-groups: K (s, z) per channel per G tokens, V per token per G channels
 DECODE_SOURCES = ["decode.cu", "common.cuh", "kernels.h"]
 
 
@@ -80,7 +81,7 @@ def profiled_traffic(w: synth.Workload, alg_bytes_per_launch: float):
             rec = json.load(f)
     except Exception:
         return None
-    if rec.get("kernel_sha") != decode_kernel_sha() or rec.get("workload") != w.name or ONLINE_K:
+    if rec.get("kernel_sha") != decode_kernel_sha() or rec.get("workload") != w.name or ONLINE_K or FINE:
         return None
     return rec["dram_bytes"] / rec["alg_bytes"] * alg_bytes_per_launch
 
@@ -100,9 +101,12 @@ def append_bytes(w: synth.Workload) -> int:
 def decode_alg_bytes(w: synth.Workload, n_quant: int, n_res: int) -> int:
     """Bytes decode attention must move at least once: codes, scales/zeros, residual rows, q, out."""
     bh = w.batch * w.kv_heads
+    if FINE:   # K: one pair per channel per G tokens; V: one pair per token per G channels
+        scales = (n_quant // w.group) * w.head_dim * 4 + n_quant * (w.head_dim // w.gv) * 4
+    else:
+        scales = (n_quant // w.residual) * (w.head_dim // w.group) * 4 + (n_quant // w.gv) * 4
     per_head = (2 * n_quant * w.head_dim * w.bits // 8                 # K and V codes
-                + (n_quant // w.residual) * (w.head_dim // w.group) * 4  # K scale + zero (fp16)
-                + (n_quant // w.group) * 4                               # V scale + zero
+                + scales                                                 # scales + zeros (fp16)
                 + n_res * w.head_dim * 4                                 # fp16 K and V residual rows
                 + 2 * w.gqa * w.head_dim * 2)                            # q in, out
     if ONLINE_K and n_quant > 0 and n_res > 0:   # residual K rows are codes, plus the block's (s, z)
@@ -227,7 +231,8 @@ def make_state(w: synth.Workload, torch, kivi, device):
     capacity = n_quant0 + (2 if ONLINE_K else 1) * w.residual   # online K: a slot for the block being filled
     k, v = synth.prompt_kv(w, w.tokens)
     cache = kivi.KiviCache(w.batch, w.kv_heads, capacity, bits=w.bits, group_k=w.group, group_v=w.group,
-                           residual=w.residual, num_q_heads=w.q_heads, device=device, online_k=ONLINE_K)
+                           residual=w.residual, num_q_heads=w.q_heads, device=device, online_k=ONLINE_K,
+                           fine_groups=FINE)
     kd = torch.from_numpy(k).to(device)
     vd = torch.from_numpy(v).to(device)
     cache.prefill(kd, vd)            # first run loads the module; the second one is timed
@@ -414,6 +419,8 @@ def run_gpu(args, rank, world, local_rank, w: synth.Workload):
                 "residual": w.residual, "cached_tokens": f"{n_quant0 + 1}-{n_quant0 + 2 * R} (128-step cycles)",
                 "step": STEP_NOTE[FUSED],
                 "k_residual": "codes (online K, config online_k = 1)" if ONLINE_K else "fp16",
+                "groups": ("fine: K per channel per G tokens, V per token per G channels (config fine_groups = 1)"
+                           if FINE else "K per R-token block x G channels, V per G tokens x all channels"),
                 "l2": l2_note(w, n_quant0),
                 "parallelism": f"weak: one independent batch per GPU x {world}",
             },
@@ -535,14 +542,20 @@ def main():
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end loop (profiling runs)")
     ap.add_argument("--separate-append", action="store_true",
                     help="append and decode as two launches (kivi_append_token + kivi_decode_attention)")
+    ap.add_argument("--fine-groups", action="store_true",
+                    help="fine-grained groups (config fine_groups = 1; 2 bits, one query per KV head); no cpu "
+                         "baseline")
     ap.add_argument("--online-k", action="store_true",
                     help="online K quantization (config online_k = 1); implies --separate-append and no "
                          "cpu baseline")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
-    global FUSED, ONLINE_K
+    global FUSED, ONLINE_K, FINE
     ONLINE_K = args.online_k
+    FINE = args.fine_groups
+    if FINE and args.impl == "reference":
+        ap.error("--fine-groups times the GPU arm only")
     FUSED = not (args.separate_append or args.online_k)
     if ONLINE_K and args.impl == "reference":
         ap.error("--online-k times the GPU arm only")
@@ -558,7 +571,7 @@ def main():
         res = run_reference(args, rank, world, w)
     else:
         res = run_gpu(args, rank, world, local_rank, w)
-        if rank == 0 and world == 1 and not args.no_cpu_baseline and not ONLINE_K:
+        if rank == 0 and world == 1 and not args.no_cpu_baseline and not ONLINE_K and not FINE:
             log("cpu baseline (oracle)")
             value, cores, sample, dt, hs = oracle_sample(w, n_heads=min(64, 2 * (os.cpu_count() or 1)),
                                                          n_steps=16, budget_s=25.0)
