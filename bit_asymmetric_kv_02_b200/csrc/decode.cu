@@ -193,6 +193,7 @@ struct Decoder {
   static constexpr int UT = BITS == 2 ? 128 : 64;  // tokens per quantized unit (8 KB of codes)
   static constexpr int TPL = UT / 32;              // tokens per lane (K side)
   static constexpr int ROWS = UT / P;              // V word rows per unit (8)
+  static_assert(P * BITS == 32 && ROWS * P == UT, "a unit is ROWS V word rows of P tokens");
   static constexpr int kBuffers = ring_buffers<G>();
   static constexpr int GP = G == 1 ? 1 : 2;        // queries per pass over a unit's codes
   // 2 bits: the byte dot products run on the tensor cores (mma.sync); one query per KV head pairs
@@ -359,56 +360,11 @@ struct Decoder {
     return h2f(__ldg(a.q + (static_cast<size_t>(qhead) * G + g) * kHeadDim + c)) * a.qscale;
   }
 
-  // Bytes 0, 1 and 2 of four integers as three words: word b holds byte b of x_m in byte m.
-  static __device__ __forceinline__ void limb_words(int x0, int x1, int x2, int x3, uint32_t& L, uint32_t& M,
-                                                   uint32_t& H) {
-    const uint32_t t01 = __byte_perm(x0, x1, 0x5140), t23 = __byte_perm(x2, x3, 0x5140);
-    L = __byte_perm(t01, t23, 0x5410);
-    M = __byte_perm(t01, t23, 0x7632);
-    H = __byte_perm(__byte_perm(x0, x1, 0x0062), __byte_perm(x2, x3, 0x0062), 0x5410);
-  }
-
-  // 2 bits: lane (i, k) owns byte m of set k of K word i for m = 0..3 (channels 16 i + 4 m + k), so
-  // it forms that set's three limb words itself.  Odd sets read as 4 * code: their limbs are / 4.
-  __device__ void build_q2(uint32_t pairs) {
-    const int gi = (16 * (lane >> 2)) >> a.lg_gk;  // the K group of all four channels
-    const float s = h2f(static_cast<uint16_t>(__shfl_sync(kFull, pairs, gi) & 0xFFFFu));
-    const float z_own = k_lane ? h2f(static_cast<uint16_t>(pairs >> 16)) : 0.f;
-    const float set_scale = (lane & 1) ? 0.25f : 1.f;
-    uint32_t* qw = reinterpret_cast<uint32_t*>(S.qw);
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-      float qv[4];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) qv[j] = q_of(g, j) * s;
-      const float mabs = warp_max(fmaxf(fmaxf(fabsf(qv[0]), fabsf(qv[1])), fmaxf(fabsf(qv[2]), fabsf(qv[3]))));
-      // |Q| <= 2^23 - 61: the margin keeps the rounded largest element below 2^23, where the
-      // signed top limb would wrap (rcp and the product add at most 3 * 2^-22 relative)
-      const float scq = mabs > 0.f ? kQRange * fast_rcp(mabs) : 0.f;
-      invq[g] = mabs * (1.0f / kQRange);
-      // sum over K groups of z_g * (sum of q over group g): lanes 0..3 hold one group each
-      float c = z_own * qsum[g][0];
-      c += __shfl_xor_sync(kFull, c, 1);
-      c += __shfl_xor_sync(kFull, c, 2);
-      cblk[g] = __shfl_sync(kFull, c, 0);
-      const float f = scq * set_scale;
-      uint32_t L, M, H;
-      limb_words(__float2int_rn(qv[0] * f), __float2int_rn(qv[1] * f), __float2int_rn(qv[2] * f),
-                 __float2int_rn(qv[3] * f), L, M, H);
-      uint32_t* row = qw + g * 96 + (lane >> 2) * 12 + (lane & 3);  // word i, limb b, set k
-      row[0] = L;
-      row[4] = M;
-      row[8] = H;
-    }
-  }
-
   // ---- A6 set-up for one K block: fixed-point limbs of q_c * s_g(c) -------------------------
   __device__ void build_q(uint32_t pairs) {
     __syncwarp();  // the previous block's limbs are no longer read
     if constexpr (kMma)
       build_q2_mma(pairs);
-    else if constexpr (BITS == 2)
-      build_q2(pairs);
     else
       build_q4(pairs);
     __syncwarp();
@@ -961,121 +917,35 @@ struct Decoder {
       }
   }
 
-  // ---- A6 over the K codes of a unit: integer dot products of TPL tokens per lane, for every
-  // query of the KV head (each code word is unpacked once) -----------------------------------------
+  // ---- A6 at 4 bits: integer dot products of TPL tokens per lane, for every query of the KV head
+  // (each code word is unpacked once) -----------------------------------------------------------------
   // Queries g0 .. g0 + GP - 1 (the accumulators of one pass).
   __device__ void k_dot(const uint8_t* kt, int g0, int (&al)[GP][TPL], int (&am)[GP][TPL], int (&ah)[GP][TPL]) const {
 #pragma unroll
     for (int g = 0; g < GP; ++g)
 #pragma unroll
       for (int j = 0; j < TPL; ++j) al[g][j] = am[g][j] = ah[g][j] = 0;
-    if (BITS == 2) {
-#pragma unroll  // both halves in one block: the second half's code words load during the first's dp4a
-      for (int h = 0; h < 2; ++h) {
-        const int hh = h ^ ((lane >> 2) & 1);  // bank-conflict-free order of the two 16-byte halves
-        uint4 kw[TPL];
-#pragma unroll
-        for (int j = 0; j < TPL; ++j)  // token 16 (lane / 4) + 4 j + lane % 4
-          kw[j] = *reinterpret_cast<const uint4*>(kt + (16 * (lane >> 2) + 4 * j + (lane & 3)) * 32 + 16 * hh);
-#pragma unroll
-        for (int ii = 0; ii < 4; ++ii) {
-          uint32_t mk[TPL][4];
-#pragma unroll
-          for (int j = 0; j < TPL; ++j) masks2(comp(kw[j], ii), mk[j]);
-#pragma unroll
-          for (int g = 0; g < GP; ++g) {
-            const uint4* qrow = S.qw[g0 + g] + 12 * hh + ii * 3;
-            const uint4 QL = qrow[0], QM = qrow[1], QH = qrow[2];
-#pragma unroll
-            for (int k = 0; k < 4; ++k)
-#pragma unroll
-              for (int j = 0; j < TPL; ++j)
-                dot_set(mk[j][k], comp(QL, k), comp(QM, k), comp(QH, k), al[g][j], am[g][j], ah[g][j], true);
-          }
-        }
-      }
-    } else {
 #pragma unroll 1
-      for (int qq = 0; qq < 4; ++qq) {
-        const int cq = (qq + (lane >> 1)) & 3;  // bank-conflict-free chunk order
-        uint4 kw[TPL];
+    for (int qq = 0; qq < 4; ++qq) {
+      const int cq = (qq + (lane >> 1)) & 3;  // bank-conflict-free chunk order
+      uint4 kw[TPL];
 #pragma unroll
-        for (int j = 0; j < TPL; ++j) kw[j] = *reinterpret_cast<const uint4*>(kt + (lane + 32 * j) * 64 + 16 * cq);
+      for (int j = 0; j < TPL; ++j) kw[j] = *reinterpret_cast<const uint4*>(kt + (lane + 32 * j) * 64 + 16 * cq);
 #pragma unroll
-        for (int ii = 0; ii < 4; ++ii) {
-          uint32_t mk[TPL][2];
+      for (int ii = 0; ii < 4; ++ii) {
+        uint32_t mk[TPL][2];
 #pragma unroll
-          for (int j = 0; j < TPL; ++j) masks4(comp(kw[j], ii), mk[j]);
+        for (int j = 0; j < TPL; ++j) masks4(comp(kw[j], ii), mk[j]);
 #pragma unroll
-          for (int g = 0; g < GP; ++g) {
-            const uint2* qrow = reinterpret_cast<const uint2*>(S.qw[g0 + g]) + 12 * cq + ii * 3;
-            const uint2 QL = qrow[0], QM = qrow[1], QH = qrow[2];
+        for (int g = 0; g < GP; ++g) {
+          const uint2* qrow = reinterpret_cast<const uint2*>(S.qw[g0 + g]) + 12 * cq + ii * 3;
+          const uint2 QL = qrow[0], QM = qrow[1], QH = qrow[2];
 #pragma unroll
-            for (int j = 0; j < TPL; ++j) dot_set(mk[j][0], QL.x, QM.x, QH.x, al[g][j], am[g][j], ah[g][j], true);
+          for (int j = 0; j < TPL; ++j) dot_set(mk[j][0], QL.x, QM.x, QH.x, al[g][j], am[g][j], ah[g][j], true);
 #pragma unroll
-            for (int j = 0; j < TPL; ++j) dot_set(mk[j][1], QL.y, QM.y, QH.y, al[g][j], am[g][j], ah[g][j], true);
-          }
+          for (int j = 0; j < TPL; ++j) dot_set(mk[j][1], QL.y, QM.y, QH.y, al[g][j], am[g][j], ah[g][j], true);
         }
       }
-    }
-  }
-
-  // V scale and zero of this lane's four tokens (one V group), and the unit's largest V scale.
-  struct VScales {
-    float sv, zv, smax, inv_smax;
-  };
-  __device__ __forceinline__ VScales v_scales2(uint32_t pairs) const {
-    VScales v;
-    const uint32_t vp = __shfl_sync(kFull, pairs, 8 + ((16 * (lane >> 2)) >> a.lg_gv));
-    v.sv = h2f(static_cast<uint16_t>(vp & 0xFFFFu));
-    v.zv = h2f(static_cast<uint16_t>(vp >> 16));
-    v.smax = warp_max(v_lane ? h2f(static_cast<uint16_t>(pairs & 0xFFFFu)) : 0.f);
-    v.inv_smax = v.smax > 0.f ? fast_rcp(v.smax) : 0.f;
-    return v;
-  }
-
-  // 2 bits: lane (r, k) holds tokens 16 r + 4 j + k (j = 0..3), i.e. byte j of set k of V word row
-  // r, so it forms that set's three P limb words itself; its four tokens share one V group.
-  // P is scaled by the bound (largest weight of the unit) x (largest V scale of the unit), which
-  // needs one warp reduction instead of two; the bound sums over the units to at most smax * l,
-  // the same error bound as the exact maximum.  A unit whose weights are all below 2^-64 of the
-  // running maximum contributes its z-terms only.
-  __device__ void softmax2(const VScales& vs, int g0, const int (&al)[GP][TPL], const int (&am)[GP][TPL],
-                           const int (&ah)[GP][TPL]) {
-    const float sv = vs.sv, zv = vs.zv;
-    const float set_scale = (lane & 1) ? 0.25f : 1.f;
-    uint32_t* pw = reinterpret_cast<uint32_t*>(S.pw);
-#pragma unroll
-    for (int gg = 0; gg < GP; ++gg) {
-      const int g = g0 + gg;
-      float lg[TPL];
-#pragma unroll
-      for (int j = 0; j < TPL; ++j) lg[j] = fmaf(combine_limbs(ah[gg][j], am[gg][j], al[gg][j]), invq[g], cblk[g]);
-      const float mu = warp_max(fmaxf(fmaxf(lg[0], lg[1]), fmaxf(lg[2], lg[3])));
-      const float m_new = fmaxf(m[g], mu);
-      const float alpha = fast_exp2(m[g] - m_new);
-      float p[TPL];
-#pragma unroll
-      for (int j = 0; j < TPL; ++j) p[j] = fast_exp2(lg[j] - m_new);
-      const float psum = (p[0] + p[1]) + (p[2] + p[3]);
-      const float d = mu - m_new;  // <= 0: the unit's largest weight is 2^d
-      const bool hv = d > -64.f && vs.smax > 0.f;
-      m[g] = m_new;
-      l[g] = fmaf(l[g], alpha, psum);
-      Z[g] = fmaf(Z[g], alpha, psum * zv);
-      alpha_[g] = alpha;
-      hasv_[g] = hv;
-      // P <= 2^24 - 128 (1 + 2^-20): the top token must not round to 2^24, where it would wrap to 0
-      invv_[g] = hv ? fast_exp2(d) * vs.smax * (1.0f / kPRange) : 0.f;
-      const float f = hv ? sv * (kPRange * vs.inv_smax) * fast_exp2(-d) * set_scale : 0.f;
-      uint32_t L, M, H;
-      limb_words(static_cast<int>(__float2uint_rn(p[0] * f)), static_cast<int>(__float2uint_rn(p[1] * f)),
-                 static_cast<int>(__float2uint_rn(p[2] * f)), static_cast<int>(__float2uint_rn(p[3] * f)),
-                 L, M, H);
-      uint32_t* row = pw + g * 96 + (lane >> 2) * 12 + (lane & 3);  // row r, limb b, set k
-      row[0] = L;
-      row[4] = M;
-      row[8] = H;
     }
   }
 
@@ -1098,14 +968,6 @@ struct Decoder {
       float lg[NBLK][8];
       k_mma_g(kt, lg);
       softmax_mma_g(pairs, lg);
-    } else if constexpr (BITS == 2) {
-      const VScales vs = v_scales2(pairs);  // independent of the dot products: issued first
-#pragma unroll
-      for (int g0 = 0; g0 < G; g0 += GP) {
-        int al[GP][TPL], am[GP][TPL], ah[GP][TPL];
-        k_dot(kt, g0, al, am, ah);
-        softmax2(vs, g0, al, am, ah);
-      }
     } else {
 #pragma unroll
       for (int g0 = 0; g0 < G; g0 += GP) {
@@ -1183,7 +1045,7 @@ struct Decoder {
     __syncwarp();  // P limbs are rewritten by the next unit
   }
 
-  // CUDA-core P . codes: dp4a on the three limbs of every query's P.
+  // CUDA-core P . codes at 4 bits: dp4a on the three limbs of every query's P.
   __device__ void dot_v(const uint8_t* vt) {
 #pragma unroll
     for (int g0 = 0; g0 < G; g0 += GP) {  // queries g0 .. g0 + GP - 1 per pass over the codes
@@ -1195,35 +1057,18 @@ struct Decoder {
 #pragma unroll 2
       for (int r = 0; r < ROWS; ++r) {
         const uint4 vw = *reinterpret_cast<const uint4*>(vt + r * 512 + 16 * lane);
-        if (BITS == 2) {
-          uint32_t mv4[4][4];
+        uint32_t mv4[4][2];
 #pragma unroll
-          for (int e = 0; e < 4; ++e) masks2(comp(vw, e), mv4[e]);
+        for (int e = 0; e < 4; ++e) masks4(comp(vw, e), mv4[e]);
 #pragma unroll
-          for (int g = 0; g < GP; ++g) {
-            if (G > 1 && !hasv_[g0 + g]) continue;
-            const uint4* pr = S.pw[g0 + g] + r * 3;
-            const uint4 PL = pr[0], PM = pr[1], PH = pr[2];
+        for (int g = 0; g < GP; ++g) {
+          if (G > 1 && !hasv_[g0 + g]) continue;
+          const uint2* pw2 = reinterpret_cast<const uint2*>(S.pw[g0 + g]);
+          const uint2 PL = pw2[r * 3 + 0], PM = pw2[r * 3 + 1], PH = pw2[r * 3 + 2];
 #pragma unroll
-            for (int k = 0; k < 4; ++k)  // set-major: 12 independent accumulators between reuses
+          for (int e = 0; e < 4; ++e) dot_set(mv4[e][0], PL.x, PM.x, PH.x, vl[g][e], vm[g][e], vh[g][e], false);
 #pragma unroll
-              for (int e = 0; e < 4; ++e)
-                dot_set(mv4[e][k], comp(PL, k), comp(PM, k), comp(PH, k), vl[g][e], vm[g][e], vh[g][e], false);
-          }
-        } else {
-          uint32_t mv4[4][2];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) masks4(comp(vw, e), mv4[e]);
-#pragma unroll
-          for (int g = 0; g < GP; ++g) {
-            if (G > 1 && !hasv_[g0 + g]) continue;
-            const uint2* pw2 = reinterpret_cast<const uint2*>(S.pw[g0 + g]);
-            const uint2 PL = pw2[r * 3 + 0], PM = pw2[r * 3 + 1], PH = pw2[r * 3 + 2];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) dot_set(mv4[e][0], PL.x, PM.x, PH.x, vl[g][e], vm[g][e], vh[g][e], false);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) dot_set(mv4[e][1], PL.y, PM.y, PH.y, vl[g][e], vm[g][e], vh[g][e], false);
-          }
+          for (int e = 0; e < 4; ++e) dot_set(mv4[e][1], PL.y, PM.y, PH.y, vl[g][e], vm[g][e], vh[g][e], false);
         }
       }
 #pragma unroll
