@@ -679,10 +679,27 @@ __global__ void __launch_bounds__(kHeadDim) quantize_fine_kernel(QuantizeArgs a)
           }
         }
       }
+      // every lane of a warp holds the same 8 group ranges: lane i % 8 forms token i's (s, z) once and
+      // the warp broadcasts it
+      float mlo = lo[0], mhi = hi[0];
+#pragma unroll
+      for (int i = 1; i < 8; ++i) {
+        if ((c & 7) == i) {
+          mlo = lo[i];
+          mhi = hi[i];
+        }
+      }
+      const GroupParams mine = make_group(mlo, mhi, L);
+      const uint32_t mine_sz = static_cast<uint32_t>(mine.s_bits) | (static_cast<uint32_t>(mine.z_bits) << 16);
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         const int tok = t0 + i;
-        const GroupParams gp = make_group(lo[i], hi[i], L);
+        GroupParams gp;
+        gp.inv_s = __shfl_sync(0xffffffffu, mine.inv_s, i);
+        gp.zf = __shfl_sync(0xffffffffu, mine.zf, i);
+        const uint32_t sz = __shfl_sync(0xffffffffu, mine_sz, i);
+        gp.s_bits = static_cast<uint16_t>(sz & 0xFFFFu);
+        gp.z_bits = static_cast<uint16_t>(sz >> 16);
         if (c % gv == 0) {
           const size_t si = (static_cast<size_t>(bh) * C + dst_tok + tok) * ngv + g;
           a.v_scale[si] = gp.s_bits;
