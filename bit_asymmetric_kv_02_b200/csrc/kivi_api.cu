@@ -444,8 +444,10 @@ int kivi_append_decode_attention(const kivi_config* cfg, kivi_cache* cache, cons
                      stream, nullptr, nullptr, -2);
     if (st != KIVI_OK) return st;
     if ((st = kivi_append_token(cfg, cache, k_new_dev, v_new_dev, stream)) != KIVI_OK) return st;
-    return decode_impl(cfg, cache, q_dev, num_q_heads, scale, out_dev, workspace_dev, workspace_bytes, dev_status,
-                       stream, nullptr, nullptr, -1);
+    st = decode_impl(cfg, cache, q_dev, num_q_heads, scale, out_dev, workspace_dev, workspace_bytes, dev_status,
+                     stream, nullptr, nullptr, -1);
+    if (st != KIVI_OK) cache->n_res -= 1;  // a failed launch: the counters are left as they were
+    return st;
   }
   kivi_cache after = *cache;
   after.n_res += 1;
