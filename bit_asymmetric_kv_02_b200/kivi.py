@@ -163,7 +163,12 @@ def kivi_debug_inject(mode: int, value: int = 0) -> None:
 
 # ---- torch-owned cache --------------------------------------------------------------------------
 class KiviCache:
-    """Caller-owned device buffers of one cache, allocated as torch tensors, plus the C struct."""
+    """Caller-owned device buffers of one cache, allocated as torch tensors, plus the C struct.
+
+    The arguments are the fields of kivi_config (include/kivi.h).  online_k: K rows are coded at
+    append with the newest block's (s, z) once a block exists.  fine_groups: group_k counts tokens
+    (one K pair per channel per group_k tokens) and group_v channels (one V pair per token per group_v
+    channels).  num_q_heads sizes the decode workspace (default: one query head per KV head)."""
 
     def __init__(self, batch: int, num_kv_heads: int, capacity: int, bits: int = 2, group_k: int = 32,
                  group_v: int = 32, residual: int = 128, head_dim: int = 128, num_q_heads: int | None = None,
