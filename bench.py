@@ -6,7 +6,8 @@ R=128): flush the residual when it is full (once every 128 steps), append one ne
 (batch, KV head), and run decode attention for every query head over the whole cache.  After each
 128-step cycle the host moves n_quant back by one block, so the cache cycles between 8193 and 8320
 cached tokens instead of growing; every step does its full work.  Inputs live in HBM (1.2 GB of codes
-and scales per step, ten times the 126 MB L2, so no L2 flush is needed).
+and scales per step, ten times the 126 MB L2, so no L2 flush is needed; a workload smaller than twice
+the L2 rotates several cache replicas, one per step, so that a step finds its cache evicted).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
 
@@ -23,6 +24,7 @@ import math
 import os
 import statistics
 import sys
+import threading
 import time
 
 import numpy as np
@@ -36,6 +38,7 @@ METRIC = "2-bit KV decode-attention cached tokens/s/head and HBM GB/s vs 8 TB/s 
 UNIT = "cached tokens/s/head"
 SPEC_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
+L2_BYTES = 126e6
 WORKLOAD = synth.LARGE_BATCH
 FUSED = True   # append and decode in one launch (kivi_append_decode_attention); --separate-append: two
 STEP_NOTE = {True: "flush when full + append and decode attention in one launch",
@@ -43,6 +46,15 @@ STEP_NOTE = {True: "flush when full + append and decode attention in one launch"
 ONLINE_K = False   # --online-k: K rows coded at append with the newest block's (s, z) (config online_k)
 FINE = False       # --fine-groups: K (s, z) per channel per G tokens, V per token per G channels
 DECODE_SOURCES = ["decode.cu", "common.cuh", "kernels.h"]
+CLOCK_WINDOW_S = 1.0   # the clock record spans at least this much wall time around the timed steps
+# The KIVI page's own end-to-end figures (section 実験結果, results table): context only, not a target.
+PUBLISHED = {
+    "source": "KIVI explainer page, results table (arXiv 2402.02750)",
+    "hardware": "not stated",
+    "peak_memory_reduction_vs_fp16": "2.6x (Llama-2-7B-chat, 2-bit KIVI)",
+    "throughput_vs_fp16": {"Llama-2-7B": "2.35x", "Llama-2-70B": "3.47x"},
+    "note": "model-level results with larger batches; no kernel-level figure is given",
+}
 
 
 # ------------------------------------------------------------------------------------------------
@@ -86,13 +98,6 @@ def profiled_traffic(w: synth.Workload, alg_bytes_per_launch: float):
     return rec["dram_bytes"] / rec["alg_bytes"] * alg_bytes_per_launch
 
 
-def l2_note(w: synth.Workload, n_quant: int) -> str:
-    gb = decode_alg_bytes(w, n_quant, w.residual) / 1e9
-    if gb * 1e3 > 2 * 126:
-        return f"not flushed: inputs ({gb:.2f} GB per step) exceed the 126 MB L2"
-    return f"WARNING: inputs ({gb * 1e3:.0f} MB per step) fit in the 126 MB L2; not flushed"
-
-
 def append_bytes(w: synth.Workload) -> int:
     """Bytes a fused append adds to the decode launch: the new K and V rows read and written once."""
     return w.batch * w.kv_heads * w.head_dim * 2 * 2 * 2
@@ -114,9 +119,30 @@ def decode_alg_bytes(w: synth.Workload, n_quant: int, n_res: int) -> int:
     return int(bh * per_head)
 
 
+def auto_replicas(w: synth.Workload, n_quant0: int) -> int:
+    """Cache replicas a step rotates through so that each step reads a cache the L2 has dropped:
+    one when a step moves more than twice the L2, else enough that the other replicas' steps move
+    at least twice the L2 between two uses of one replica (at most 64)."""
+    per_step = decode_alg_bytes(w, n_quant0 + w.residual, w.residual)
+    if per_step > 2 * L2_BYTES:
+        return 1
+    return int(min(64, math.ceil(2 * L2_BYTES / per_step) + 1))
+
+
+def l2_note(w: synth.Workload, n_quant: int, replicas: int) -> str:
+    gb = decode_alg_bytes(w, n_quant, w.residual) / 1e9
+    if replicas <= 1:
+        if gb * 1e9 > 2 * L2_BYTES:
+            return f"not flushed: inputs ({gb:.2f} GB per step) exceed the 126 MB L2"
+        return f"WARNING: inputs ({gb * 1e3:.0f} MB per step) fit in the 126 MB L2; not flushed"
+    return (f"{replicas} cache replicas, one per step in turn: {(replicas - 1) * gb * 1e3:.0f} MB move between two "
+            f"uses of a replica ({gb * 1e3:.1f} MB per step, 126 MB L2)")
+
+
 class ClockSampler:
-    """Samples SM clock, max clock and throttle reasons of one GPU with nvidia-smi every 50 ms while
-    the timed region runs (the clocks line of the profiling recipe)."""
+    """Samples SM clock, max clock and throttle reasons of one GPU with nvidia-smi every 50 ms (the
+    clocks line of the profiling recipe).  start() returns once the first sample has arrived, so a
+    window marked afterwards is covered; every line is time-stamped on arrival."""
 
     FIELDS = ("index,pci.bus_id,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -132,7 +158,9 @@ class ClockSampler:
         except Exception:
             pass
         self.proc = None
-        self.lines = []
+        self.lines = []      # (monotonic time, line)
+        self._thread = None
+        self._first = threading.Event()
 
     @staticmethod
     def _bus_of(field: str):
@@ -143,29 +171,41 @@ class ClockSampler:
         except (ValueError, IndexError):
             return None
 
-    def __enter__(self):
+    def _reader(self):
+        for ln in self.proc.stdout:
+            if ln.strip():
+                self.lines.append((time.monotonic(), ln))
+                self._first.set()
+
+    def start(self, wait_s: float = 10.0):
         import shutil
         import subprocess
         exe = shutil.which("nvidia-smi")
         if exe:
             self.proc = subprocess.Popen([exe, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
                                           "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
-                                         text=True)
+                                         text=True, bufsize=1)
+            self._thread = threading.Thread(target=self._reader, daemon=True)
+            self._thread.start()
+            self._first.wait(wait_s)
         return self
 
-    def __exit__(self, *exc):
+    def stop(self):
         if self.proc is not None:
             self.proc.terminate()
             try:
-                out, _ = self.proc.communicate(timeout=10)
+                self.proc.wait(timeout=10)
             except Exception:
                 self.proc.kill()
-                out, _ = self.proc.communicate()
-            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+            if self._thread is not None:
+                self._thread.join(timeout=10)
+            self.proc = None
 
-    def summary(self):
+    def summary(self, t0: float | None = None, t1: float | None = None):
         rows = []
-        for ln in self.lines:
+        for t, ln in self.lines:
+            if (t0 is not None and t < t0) or (t1 is not None and t > t1):
+                continue
             f = [x.strip() for x in ln.split(",")]
             if len(f) < 10:
                 continue
@@ -176,7 +216,8 @@ class ClockSampler:
             except ValueError:
                 continue
         if not rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0,
+                    "note": "no nvidia-smi sample in the window"}
         loaded = [r for r in rows if r[2] > 300.0] or rows   # power draw separates load from idle
         reasons = set()
         for r in loaded:
@@ -223,40 +264,53 @@ def weak_scaling_value(world: int, tokens_per_rank: int, batch: int, t_max_ms: f
     return world * tokens_per_rank * batch / (t_max_ms / 1e3)
 
 
+def first_prompt_split(w: synth.Workload):
+    """(n_quant, capacity) of the bench's cache: the prompt leaves a full residual; the cache holds
+    one more block (two under online K: the block being filled keeps its own scale row)."""
+    n_quant0 = (w.tokens - 1) // w.residual * w.residual
+    return n_quant0, n_quant0 + (2 if ONLINE_K else 1) * w.residual
+
+
+def workload_config(w: synth.Workload, world: int, replicas: int) -> dict:
+    """The `config` of the JSON line, the same for both arms."""
+    n_quant0, _ = first_prompt_split(w)
+    R = w.residual
+    return {
+        "workload": w.name, "batch": w.batch, "q_heads": w.q_heads, "kv_heads": w.kv_heads,
+        "head_dim": w.head_dim, "bits": w.bits, "group_k": w.group, "group_v": w.gv,
+        "residual": R, "cached_tokens": f"{n_quant0 + 1}-{n_quant0 + 2 * R} (128-step cycles)",
+        "step": STEP_NOTE[FUSED],
+        "k_residual": "codes (online K, config online_k = 1)" if ONLINE_K else "fp16",
+        "groups": ("fine: K per channel per G tokens, V per token per G channels (config fine_groups = 1)"
+                   if FINE else "K per R-token block x G channels, V per G tokens x all channels"),
+        "l2": l2_note(w, n_quant0, replicas),
+        "parallelism": f"weak: one independent batch per GPU x {world}",
+    }
+
+
 # ------------------------------------------------------------------------------------------------
 # the GPU arm
 # ------------------------------------------------------------------------------------------------
-def make_state(w: synth.Workload, torch, kivi, device):
-    n_quant0 = (w.tokens - 1) // w.residual * w.residual      # 8064: the prompt leaves a full residual
-    capacity = n_quant0 + (2 if ONLINE_K else 1) * w.residual   # online K: a slot for the block being filled
-    k, v = synth.prompt_kv(w, w.tokens)
-    cache = kivi.KiviCache(w.batch, w.kv_heads, capacity, bits=w.bits, group_k=w.group, group_v=w.group,
+def make_cache(w: synth.Workload, torch, kivi, device, kd, vd):
+    _, capacity = first_prompt_split(w)
+    cache = kivi.KiviCache(w.batch, w.kv_heads, capacity, bits=w.bits, group_k=w.group, group_v=w.gv,
                            residual=w.residual, num_q_heads=w.q_heads, device=device, online_k=ONLINE_K,
                            fine_groups=FINE)
-    kd = torch.from_numpy(k).to(device)
-    vd = torch.from_numpy(v).to(device)
-    cache.prefill(kd, vd)            # first run loads the module; the second one is timed
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
     cache.prefill(kd, vd)
-    e1.record()
-    torch.cuda.synchronize(device)
-    prefill_ms = e0.elapsed_time(e1)
-    del kd, vd, k, v
-    torch.cuda.empty_cache()   # hand the 8.6 GB of prompt back: the decode loop holds ~1.3 GB
-    # per-step inputs for a cycle of 128 steps (new K/V rows and queries), resident in HBM
-    steps_in = []
+    return cache
+
+
+def step_inputs(w: synth.Workload, torch, device):
+    """New K/V rows and queries of synthetic steps 1..R, resident in HBM (a cycle of R steps)."""
+    host = []
     for s in range(w.residual):
         kn, vn = synth.new_kv(w, s + 1)
-        q = synth.queries(w, s + 1)
-        steps_in.append((kn, vn, q))
-    dev_in = [tuple(torch.from_numpy(a).to(device) for a in x) for x in steps_in]
-    torch.cuda.synchronize(device)
-    assert (cache.n_quant, cache.n_res) == (n_quant0, w.residual)
-    return cache, n_quant0, steps_in, dev_in, prefill_ms
+        host.append((kn, vn, synth.queries(w, s + 1)))
+    dev = [tuple(torch.from_numpy(a).to(device) for a in x) for x in host]
+    return host, dev
 
 
-def gpu_step(cache, n_quant0, w, inputs, out, stream, decode_events=None, stage_events=None):
+def gpu_step(cache, n_quant0, w, inputs, out, stream, decode_events=None, stage_events=None, status=True):
     """One streaming decode step on device-resident inputs; returns (launches, cached tokens).
     stage_events (optional): {"flush": [...], "append": [...]} lists that receive event pairs."""
     import torch
@@ -276,7 +330,7 @@ def gpu_step(cache, n_quant0, w, inputs, out, stream, decode_events=None, stage_
     if FUSED:
         if decode_events is not None:
             decode_events[0].record(stream)
-        cache.append_attend(kn, vn, q, out=out, stream=stream, status=False)
+        cache.append_attend(kn, vn, q, out=out, stream=stream, status=status)
         if decode_events is not None:
             decode_events[1].record(stream)
         return launches + 1, cache.c.n_quant + cache.c.n_res
@@ -290,7 +344,7 @@ def gpu_step(cache, n_quant0, w, inputs, out, stream, decode_events=None, stage_
     launches += 1
     if decode_events is not None:
         decode_events[0].record(stream)
-    cache.attend(q, out=out, stream=stream, status=False)
+    cache.attend(q, out=out, stream=stream, status=status)
     if decode_events is not None:
         decode_events[1].record(stream)
     launches += 1
@@ -309,56 +363,121 @@ def run_gpu(args, rank, world, local_rank, w: synth.Workload):
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=device)
     ranks = Ranks(dist, device)
+    R = w.residual
+    n_quant0, _ = first_prompt_split(w)
+    replicas = args.replicas if args.replicas > 0 else auto_replicas(w, n_quant0)
 
-    log("generating inputs and prefilling the cache")
-    cache, n_quant0, host_in, dev_in, prefill_ms = make_state(w, torch, kivi, device)
+    log(f"generating inputs and prefilling {replicas} cache(s)")
+    k, v = synth.prompt_kv(w, w.tokens)
+    kd = torch.from_numpy(k).to(device)
+    vd = torch.from_numpy(v).to(device)
+    del k, v
+    caches = [make_cache(w, torch, kivi, device, kd, vd) for _ in range(replicas)]
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    caches[0].prefill(kd, vd)          # the first prefill loaded the module; this one is timed
+    e1.record()
+    torch.cuda.synchronize(device)
+    prefill_ms = e0.elapsed_time(e1)
+    del kd, vd
+    torch.cuda.empty_cache()   # hand the prompt back: the decode loop holds the caches only
+    host_in, dev_in = step_inputs(w, torch, device)
+    for c in caches:
+        assert (c.n_quant, c.n_res) == (n_quant0, R)
+        c.status.zero_()
     log("cache ready")
     stream = torch.cuda.Stream(device)
     out = torch.empty(w.batch, w.q_heads, w.head_dim, dtype=torch.float16, device=device)
-    R = w.residual
+    schedule = [[] for _ in caches]   # synthetic step id of every step each replica has run
+    counter = [0]
+
+    def step(inputs_index, decode_events=None, stage_events=None, outbuf=None, inputs=None):
+        i = counter[0]
+        counter[0] += 1
+        r = i % replicas
+        schedule[r].append(inputs_index + 1)
+        return gpu_step(caches[r], n_quant0, w, inputs if inputs is not None else dev_in[inputs_index],
+                        outbuf if outbuf is not None else out, stream, decode_events, stage_events)
 
     barrier = ranks.barrier
+    sampler = ClockSampler(local_rank).start()
 
     # ---- device-resident timing -------------------------------------------------------------
     def timed_loop(K, W):
         with torch.cuda.stream(stream):
             for i in range(W):
-                gpu_step(cache, n_quant0, w, dev_in[i % R], out, stream)
+                step(i % R)
         stream.synchronize()
         barrier()
         torch.cuda.synchronize(device)
         ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        launches, tokens = 0, 0
-        bytes_decode = 0
+        launches, tokens, bytes_decode = 0, 0, 0
         stage_ev = {"flush": [], "append": []}
-        with ClockSampler(local_rank) as clocks, torch.cuda.stream(stream):
+        t_wall0 = time.monotonic()
+        with torch.cuda.stream(stream):
             e0.record(stream)
             for i in range(K):
-                n_q, n_r = cache.c.n_quant, cache.c.n_res
-                lz, t = gpu_step(cache, n_quant0, w, dev_in[(W + i) % R], out, stream, ev[i], stage_ev)
+                lz, t = step((W + i) % R, ev[i], stage_ev)
+                c = caches[(counter[0] - 1) % replicas]
                 launches += lz
                 tokens += t
-                n_q2 = cache.c.n_quant
+                n_q2 = c.c.n_quant
                 bytes_decode += decode_alg_bytes(w, n_q2, t - n_q2) + (append_bytes(w) if FUSED else 0)
             e1.record(stream)
             stream.synchronize()
         torch.cuda.synchronize(device)
         barrier()
+        t_wall1 = time.monotonic()
+        last = {"out": out.clone(), "replica": (counter[0] - 1) % replicas,
+                "steps": len(schedule[(counter[0] - 1) % replicas])}
+        # the clock record spans at least CLOCK_WINDOW_S: the same steps continue, untimed
+        ext = 0
+        with torch.cuda.stream(stream):
+            while time.monotonic() - t_wall0 < CLOCK_WINDOW_S:
+                for _ in range(64):
+                    step((W + K + ext) % R)
+                    ext += 1
+                stream.synchronize()
+        t_wall2 = time.monotonic()
         ms = e0.elapsed_time(e1)
         dec_ms = sum(a.elapsed_time(b) for a, b in ev)
         stage_ms = {k: (sum(a.elapsed_time(b) for a, b in v) / len(v) if v else None) for k, v in stage_ev.items()}
-        clk = clocks.summary()
-        clk["stage_ms"] = stage_ms
-        return ms, dec_ms, launches, tokens, bytes_decode, clk
+        clk = sampler.summary(t_wall0, t_wall2)
+        clk["window_s"] = round(t_wall2 - t_wall0, 3)
+        clk["window"] = (f"the {K} timed steps ({(t_wall1 - t_wall0) * 1e3:.1f} ms wall) and {ext} more of the same "
+                         f"steps after them, untimed, so that nvidia-smi (50 ms period) samples the kernel")
+        return ms, dec_ms, launches, tokens, bytes_decode, clk, stage_ms, last
 
-    ms, dec_ms, launches, tokens, bytes_decode, clk = timed_loop(args.steps, args.warmup)
-    log(f"timed loop done: {ms:.3f} ms for {args.steps} steps")
+    ms, dec_ms, launches, tokens, bytes_decode, clk, stage_ms, last = timed_loop(args.steps, args.warmup)
+    log(f"timed loop done: {ms:.3f} ms for {args.steps} steps; clocks {clk.get('sm_mhz')} MHz "
+        f"({clk.get('samples')} samples)")
     if BAD_REASONS & set(clk["reasons"]):
-        ms, dec_ms, launches, tokens, bytes_decode, clk = timed_loop(args.steps, args.warmup)
+        ms, dec_ms, launches, tokens, bytes_decode, clk, stage_ms, last = timed_loop(args.steps, args.warmup)
         clk["remeasured"] = True
         log(f"re-measured (throttle reasons seen): {ms:.3f} ms")
+    sampler.stop()
     t_max, dec_ms = ranks.max(ms, dec_ms)
+    status = max(c.read_status(stream) for c in caches)
+    if status != 0:
+        log(f"device status {status} after the timed steps")
+
+    # ---- one flush, timed on its own (the timed window may hold none) -------------------------
+    flush_ms_sep = []
+    fl = [torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)]
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            c = caches[counter[0] % replicas]
+            while c.c.n_res < R:        # steps of this replica until its residual is full
+                for _r in range(replicas):
+                    step(counter[0] % R)
+            if c.c.n_quant == n_quant0 + R:
+                c.c.n_quant = n_quant0   # the cycle of gpu_step; the replica's next step finds n_res = 0
+            fl[0].record(stream)
+            c.flush(stream)
+            fl[1].record(stream)
+            stream.synchronize()
+            flush_ms_sep.append(fl[0].elapsed_time(fl[1]))
 
     # ---- end to end through the public API with host buffers ---------------------------------
     # Each step's new K, V rows and queries sit back to back in one pinned buffer and arrive with one
@@ -387,7 +506,7 @@ def run_gpu(args, rank, world, local_rank, w: synth.Workload):
             f0.record(stream)
             for i in range(K):
                 stage_buf.copy_(pinned[i % R], non_blocking=True)
-                _, t = gpu_step(cache, n_quant0, w, stage, out, stream)
+                _, t = step(i % R, inputs=stage)
                 toks += t
                 out_host.copy_(out, non_blocking=True)
                 stream.synchronize()      # the caller consumes the step's result
@@ -399,6 +518,7 @@ def run_gpu(args, rank, world, local_rank, w: synth.Workload):
     e2e_steps = 0 if args.no_e2e else min(args.steps, 4 * R)
     e2e_ms, e2e_tokens = e2e_loop(e2e_steps) if e2e_steps else (float("nan"), 0)
     e2e_ms = ranks.max(e2e_ms)
+    status = max(status, max(c.read_status(stream) for c in caches))
 
     result = None
     if rank == 0:
@@ -407,32 +527,28 @@ def run_gpu(args, rank, world, local_rank, w: synth.Workload):
         peak, peak_kind = hbm_peak()
         dec_avg_ms = dec_ms / K
         achieved = (bytes_decode / K) / (dec_avg_ms / 1e3) / 1e9
-        traffic = profiled_traffic(w, bytes_decode / K)
+        traffic = profiled_traffic(w, bytes_decode / K) if replicas == 1 else None
         e2e_value = weak_scaling_value(world, e2e_tokens, w.batch, e2e_ms)
+        flush_window = stage_ms["flush"]
         result = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
             "ms_per_step": t_max / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": f"u{w.bits} codes x i8 limbs ({dot_engine(w)}, i32 acc), f32 softmax", "data": "synthetic",
-            "config": {
-                "workload": w.name, "batch": w.batch, "q_heads": w.q_heads, "kv_heads": w.kv_heads,
-                "head_dim": w.head_dim, "bits": w.bits, "group_k": w.group, "group_v": w.group,
-                "residual": w.residual, "cached_tokens": f"{n_quant0 + 1}-{n_quant0 + 2 * R} (128-step cycles)",
-                "step": STEP_NOTE[FUSED],
-                "k_residual": "codes (online K, config online_k = 1)" if ONLINE_K else "fp16",
-                "groups": ("fine: K per channel per G tokens, V per token per G channels (config fine_groups = 1)"
-                           if FINE else "K per R-token block x G channels, V per G tokens x all channels"),
-                "l2": l2_note(w, n_quant0),
-                "parallelism": f"weak: one independent batch per GPU x {world}",
-            },
+            "config": workload_config(w, world, replicas),
             "hbm_gbs_decode": achieved, "hbm_frac_of_8tbs": achieved / SPEC_HBM_GBS,
             "decode_ms_avg": dec_avg_ms,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "peak_kind": peak_kind, "traffic": traffic,
                          "kernel": f"decode_kernel<{w.bits},{w.gqa}>", "alg_bytes_per_launch": bytes_decode / K},
-            "clocks": {k: v for k, v in clk.items() if k != "stage_ms"},
+            "clocks": clk,
+            "device_status": status,
             "stages": {
                 "decode_ms": dec_avg_ms,
-                "append_ms": clk["stage_ms"]["append"], "flush_ms": clk["stage_ms"]["flush"],
+                "append_ms": stage_ms["append"],
+                "flush_ms": flush_window if flush_window is not None else statistics.median(flush_ms_sep),
+                "flush_ms_source": ("flushes inside the timed window" if flush_window is not None else
+                                    "3 flushes timed on their own after the timed window"),
+                "flush_ms_separate": statistics.median(flush_ms_sep),
                 "prefill_ms": prefill_ms, "prefill_tokens": w.tokens,
                 "prefill_gbs": (w.batch * w.kv_heads * w.tokens * w.head_dim * 2 * 2
                                 + decode_alg_bytes(w, n_quant0, 0)) / (prefill_ms / 1e3) / 1e9,
@@ -440,7 +556,10 @@ def run_gpu(args, rank, world, local_rank, w: synth.Workload):
             "gpu_launches": launches,
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "steps": e2e_steps, "ms_per_step": e2e_ms / max(1, e2e_steps)},
+            "published": PUBLISHED,
         }
+        result["_parity_state"] = {"out": last["out"].cpu().numpy(), "schedule": schedule[last["replica"]][:last["steps"]],
+                                   "n_quant0": n_quant0}
     if dist is not None:
         ranks.barrier()
         dist.destroy_process_group()
@@ -450,38 +569,82 @@ def run_gpu(args, rank, world, local_rank, w: synth.Workload):
 # ------------------------------------------------------------------------------------------------
 # the CPU oracle (cpu_baseline leg and --impl reference)
 # ------------------------------------------------------------------------------------------------
+def _oracle_head(w: synth.Workload, b: int, h: int):
+    import oracle.kivi_oracle as O
+    n_quant0, cap = first_prompt_split(w)
+    hc = O.HeadCache(w.head_dim, w.bits, w.group, w.gv, w.residual, cap, online_k=ONLINE_K, fine_groups=FINE)
+    hc.prefill(synth.prompt_k(w, b, h, w.tokens), synth.prompt_v(w, b, h, w.tokens))
+    return hc, n_quant0
+
+
+def _oracle_cycle_flush(w: synth.Workload, hc, n_quant0: int):
+    """The flush of gpu_step: at the end of a 128-step cycle n_quant goes back by one block first."""
+    R = w.residual
+    if hc.n_quant == n_quant0 + R:
+        n = n_quant0
+        hc.k_codes, hc.v_codes = hc.k_codes[:n], hc.v_codes[:n]
+        if hc.fine:
+            hc.k_s, hc.k_z = hc.k_s[:n // w.group], hc.k_z[:n // w.group]
+            hc.v_s, hc.v_z = hc.v_s[:n], hc.v_z[:n]
+        else:
+            hc.k_s, hc.k_z = hc.k_s[:n // R], hc.k_z[:n // R]
+            hc.v_s, hc.v_z = hc.v_s[:n // w.gv], hc.v_z[:n // w.gv]
+    hc.flush()
+
+
+def oracle_parity(w: synth.Workload, state: dict, n_heads: int):
+    """The oracle replays the steps the GPU cache of the last timed step went through (prefill, then
+    every flush and append, with the same synthetic inputs) on a sample of KV heads and compares the
+    last timed step's output with its attention (max-abs 2e-3 and max-rel 1e-2, relative to
+    max(|o*|, 1e-2))."""
+    R = w.residual
+    rng = np.random.default_rng(w.seed)
+    heads = {(0, 0), (w.batch - 1, w.kv_heads - 1)}
+    while len(heads) < min(n_heads, w.batch * w.kv_heads):
+        heads.add((int(rng.integers(w.batch)), int(rng.integers(w.kv_heads))))
+    sched = state["schedule"]
+    got = state["out"].astype(np.float64)
+    scale = 1.0 / math.sqrt(w.head_dim)
+    ea = er = 0.0
+    t0 = time.perf_counter()
+    for (b, h) in sorted(heads):
+        hc, n_quant0 = _oracle_head(w, b, h)
+        for sid in sched:
+            if hc.n_res == R:
+                _oracle_cycle_flush(w, hc, n_quant0)
+            hc.append(synth.new_k(w, b, h, sid), synth.new_v(w, b, h, sid))
+        q = np.stack([synth.query(w, b, h * w.gqa + g, sched[-1]) for g in range(w.gqa)])
+        want = hc.attend(q, scale)
+        err = np.abs(got[b, h * w.gqa:(h + 1) * w.gqa] - want)
+        ea = max(ea, float(err.max()))
+        er = max(er, float((err / np.maximum(np.abs(want), 1e-2)).max()))
+    return {"heads": len(heads), "steps_replayed": len(sched), "max_abs": ea, "max_rel": er,
+            "ok": bool(ea <= 2e-3 and er <= 1e-2), "tolerance": "max-abs 2e-3 and max-rel 1e-2 vs the fp64 oracle",
+            "seconds": round(time.perf_counter() - t0, 1)}
+
+
 def oracle_sample(w: synth.Workload, n_heads: int, n_steps: int, budget_s: float):
     """Times the oracle as it stands on `n_heads` KV heads for up to `n_steps` decode steps each
-    (threads over heads).  Returns (value in tokens/s/head, cores, sample description, seconds)."""
-    import oracle.kivi_oracle as O
+    (threads over heads).  Returns (value in tokens/s/head, cores, sample description, seconds,
+    head-steps)."""
     from concurrent.futures import ThreadPoolExecutor
     R = w.residual
-    n_quant0 = (w.tokens - 1) // R * R
-    cap = n_quant0 + R
     heads = [(b, h) for b in range(w.batch) for h in range(w.kv_heads)][:: max(1, (w.batch * w.kv_heads) // n_heads)]
     heads = heads[:n_heads]
-    caches = {}
-    for (b, h) in heads:
-        hc = O.HeadCache(w.head_dim, w.bits, w.group, w.group, R, cap)
-        hc.prefill(synth.prompt_k(w, b, h, w.tokens), synth.prompt_v(w, b, h, w.tokens))
-        caches[(b, h)] = hc
+    caches = {bh: _oracle_head(w, *bh) for bh in heads}
     scale = 1.0 / math.sqrt(w.head_dim)
     cores = os.cpu_count() or 1
     deadline = time.perf_counter() + budget_s
 
     def run_head(bh):
         b, h = bh
-        hc = caches[bh]
+        hc, n_quant0 = caches[bh]
         done, toks = 0, 0
         for s in range(1, n_steps + 1):
             if time.perf_counter() > deadline and done > 0:
                 break
             if hc.n_res == R:
-                if hc.n_quant == n_quant0 + R:   # same 128-step cycle as the GPU arm
-                    hc.k_codes, hc.v_codes = hc.k_codes[:n_quant0], hc.v_codes[:n_quant0]
-                    hc.k_s, hc.k_z = hc.k_s[:n_quant0 // R], hc.k_z[:n_quant0 // R]
-                    hc.v_s, hc.v_z = hc.v_s[:n_quant0 // w.group], hc.v_z[:n_quant0 // w.group]
-                hc.flush()
+                _oracle_cycle_flush(w, hc, n_quant0)
             hc.append(synth.new_k(w, b, h, s), synth.new_v(w, b, h, s))
             q = np.stack([synth.query(w, b, h * w.gqa + g, s) for g in range(w.gqa)])
             hc.attend(q, scale)
@@ -509,16 +672,21 @@ def run_reference(args, rank, world, w: synth.Workload):
     budget = max(5.0, min(60.0, 0.6 * args.steps + 5.0))
     value, cores, sample, dt, hs = oracle_sample(w, n_heads=min(64, 2 * (os.cpu_count() or 1)),
                                                  n_steps=max(1, args.steps), budget_s=budget)
-    ms_full_step = dt * 1e3 * (w.batch * w.kv_heads) / max(1, hs)   # one step covers every KV head
+    ms_head_step = dt * 1e3 / max(1, hs)
+    ms_full_step = ms_head_step * (w.batch * w.kv_heads)   # one step covers every KV head
+    n_quant0, _ = first_prompt_split(w)
+    replicas = args.replicas if args.replicas > 0 else auto_replicas(w, n_quant0)
     return {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_full_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": w.name, "batch": w.batch, "q_heads": w.q_heads, "kv_heads": w.kv_heads,
-                   "head_dim": w.head_dim, "bits": w.bits, "group_k": w.group, "group_v": w.group,
-                   "residual": w.residual, "step": STEP_NOTE[FUSED]},
+        "config": workload_config(w, world, replicas),
+        "ms_per_step_kind": (f"extrapolated: {ms_head_step:.2f} ms measured per head-step on {hs} head-steps, "
+                             f"times {w.batch * w.kv_heads} KV heads per step"),
+        "ms_per_head_step_measured": ms_head_step,
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "published": PUBLISHED,
     }
 
 
@@ -538,16 +706,19 @@ def main():
                     help="workload to time (default: the large-batch workload the metric is quoted on)")
     ap.add_argument("--bits", type=int, choices=[2, 4], default=None, help="override the workload's bits")
     ap.add_argument("--group", type=int, choices=[32, 64, 128], default=None, help="override G_k = G_v")
-    ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing (profiling runs)")
+    ap.add_argument("--replicas", type=int, default=0,
+                    help="cache replicas rotated one per step (0: enough to defeat the L2 for small workloads)")
+    ap.add_argument("--parity-heads", type=int, default=16,
+                    help="KV heads the cpu_baseline leg replays to check the last timed step (0: none)")
+    ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle legs (profiling runs)")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end loop (profiling runs)")
     ap.add_argument("--separate-append", action="store_true",
                     help="append and decode as two launches (kivi_append_token + kivi_decode_attention)")
     ap.add_argument("--fine-groups", action="store_true",
-                    help="fine-grained groups (config fine_groups = 1; 2 bits, one query per KV head); no cpu "
-                         "baseline")
+                    help="fine-grained groups (config fine_groups = 1); no cpu baseline timing")
     ap.add_argument("--online-k", action="store_true",
                     help="online K quantization (config online_k = 1); implies --separate-append and no "
-                         "cpu baseline")
+                         "cpu baseline timing")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -571,12 +742,18 @@ def main():
         res = run_reference(args, rank, world, w)
     else:
         res = run_gpu(args, rank, world, local_rank, w)
-        if rank == 0 and world == 1 and not args.no_cpu_baseline and not ONLINE_K and not FINE:
-            log("cpu baseline (oracle)")
-            value, cores, sample, dt, hs = oracle_sample(w, n_heads=min(64, 2 * (os.cpu_count() or 1)),
-                                                         n_steps=16, budget_s=25.0)
-            res["cpu_baseline"] = {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
-                                   "sample": sample}
+        if res is not None:
+            state = res.pop("_parity_state")
+            if world == 1 and not args.no_cpu_baseline:
+                if args.parity_heads > 0:
+                    log("cpu baseline leg: oracle replay of the last timed step")
+                    res["parity"] = oracle_parity(w, state, args.parity_heads)
+                if not ONLINE_K and not FINE:
+                    log("cpu baseline leg: oracle timing")
+                    value, cores, sample, dt, hs = oracle_sample(w, n_heads=min(64, 2 * (os.cpu_count() or 1)),
+                                                                 n_steps=16, budget_s=25.0)
+                    res["cpu_baseline"] = {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                                           "sample": sample}
     if rank == 0 and res is not None:
         print(json.dumps(res), flush=True)
 

@@ -55,7 +55,8 @@ extern "C" int kivi_decode_attention_noalloc(const kivi_config* cfg, const kivi_
   int st = kivi_decode_attention(cfg, cache, q_dev, num_q_heads, scale, out_dev, nullptr, 0, dev_status, stream);
   if (st != KIVI_ERR_WORKSPACE) return st;
   const size_t need = kivi_decode_workspace_bytes(cfg, num_q_heads);
-  if (need == 0) return KIVI_ERR_CUDA;
+  // decode_impl accepted every argument, so a zero size means the two size rules disagree
+  if (need == 0) return KIVI_ERR_INTERNAL;
   if (need > static_cast<size_t>(KIVI_NOALLOC_SCRATCH_BYTES)) return KIVI_ERR_WORKSPACE;
   void* base = nullptr;
   if ((st = scratch_address(&base)) != KIVI_OK) return st;

@@ -9,6 +9,7 @@ import pytest
 
 import gpu_common as gc
 import oracle.kivi_oracle as O
+import oracle_workers as ow
 from bit_asymmetric_kv_02_b200 import synth
 
 pytestmark = pytest.mark.gpu
@@ -256,54 +257,146 @@ def test_device_timeout_is_reported_and_context_survives():
     assert torch.equal(again, ref)
 
 
-FULL = [synth.LLAMA2_7B, synth.LARGE_BATCH, synth.GQA_LLAMA3_8B]
+FULL = [synth.LLAMA2_7B, synth.GQA_LLAMA3_8B]
+
+
+def _gpu_head_digests(cache, heads, shapes):
+    """{(b, h): {buffer: digest}} of the GPU cache, each buffer cut to the oracle's row count."""
+    out = {bh: {} for bh in heads}
+    for key in shapes:
+        rows = shapes[key][0]
+        full = cache.view(key)[:, :, :rows].cpu().numpy()
+        if key in ("k_codes", "v_codes"):
+            full = full.view(np.uint32)
+        for (b, h) in heads:
+            out[(b, h)][key] = ow.digest(full[b, h])
+    return out
+
+
+def _compare(label, gpu_digests, gpu_out, oracle_runs, gqa, what):
+    """Checks one checkpoint of every head: buffers bit for bit (digests), outputs within tolerance."""
+    worst = (0.0, 0.0)
+    for (b, h), run in oracle_runs.items():
+        entries = {(lab, kind): payload for lab, kind, payload in run}
+        if gpu_digests is not None:
+            want = entries[(label, "buffers")]
+            got = gpu_digests[(b, h)]
+            bad = [k for k in want if got[k] != want[k]]
+            assert not bad, f"{what} {label} head {(b, h)}: buffers {bad} differ from the oracle"
+        if gpu_out is not None:
+            ea, er = gc.assert_attention_close(gpu_out[b, h * gqa:(h + 1) * gqa], entries[(label, "out")],
+                                               f"{what} {label} head {(b, h)}")
+            worst = (max(worst[0], ea), max(worst[1], er))
+    return worst
+
+
+def _shapes(oracle_runs, label):
+    """{buffer: shape} of the oracle's packed buffers at one checkpoint (the same for every head)."""
+    run = next(iter(oracle_runs.values()))
+    for lab, kind, payload in run:
+        if lab == label and kind == "buffers":
+            return {key: shape for key, (shape, _sha) in payload.items()}
+    raise KeyError(label)
 
 
 @pytest.mark.parametrize("w", FULL, ids=[w.name for w in FULL])
-def test_full_size_sampled_heads(w):
-    """Full-size workloads in the bench's launch configuration; the oracle checks 12 sampled KV
-    heads (codes bit-exact, outputs within tolerance)."""
-    gc_heads = gc.sample_heads(w, 12, seed=w.seed)
-    run_prefill_case(w, heads=gc_heads)
+def test_full_size_all_heads(w):
+    """Full-size workloads in the bench's launch configuration: every KV head's codes, scales,
+    zero points and residual rows bit for bit, every query head's output within tolerance."""
+    kivi = _kivi()
+    T = w.tokens
+    cap = ((T + w.residual - 1) // w.residual) * w.residual
+    heads = [(b, h) for b in range(w.batch) for h in range(w.kv_heads)]
+    specs = [ow.HeadStream(w, b, h, cap, T, attend_at=frozenset({0}), digest_at=frozenset({0})) for b, h in heads]
+    with ow.pool() as ex:
+        fut = ex.map(ow.run_head, specs, chunksize=4)
+        k, v = synth.prompt_kv(w, T)
+        cache = kivi.KiviCache(w.batch, w.kv_heads, cap, bits=w.bits, group_k=w.group, group_v=w.gv,
+                               residual=w.residual, num_q_heads=w.q_heads)
+        cache.status.zero_()
+        cache.prefill(torch.from_numpy(k).cuda(), torch.from_numpy(v).cuda())
+        del k, v
+        out = cache.attend(torch.from_numpy(synth.queries(w, 0)).cuda()).cpu().numpy()
+        assert cache.read_status() == 0
+        runs = dict(zip(heads, fut))
+    shapes = _shapes(runs, "step 0")
+    _compare("step 0", _gpu_head_digests(cache, heads, shapes), out, runs, w.gqa, w.name)
+
+
+def test_full_size_large_batch_fused_all_heads():
+    """The bench's workload and call (kivi_append_decode_attention) at full size on every head:
+    prefill, attention, a flush, then two fused append + decode steps; buffers bit for bit after
+    the prefill, after the flush and at the end, outputs within tolerance at every step."""
+    kivi = _kivi()
+    w = synth.LARGE_BATCH
+    T = w.tokens
+    cap = (T - 1) // w.residual * w.residual + w.residual
+    heads = [(b, h) for b in range(w.batch) for h in range(w.kv_heads)]
+    specs = [ow.HeadStream(w, b, h, cap, T, steps=2, attend_at=frozenset({0, 1, 2}), digest_at=frozenset({0, 2}))
+             for b, h in heads]
+    with ow.pool() as ex:
+        fut = ex.map(ow.run_head, specs, chunksize=8)
+        k, v = synth.prompt_kv(w, T)
+        cache = kivi.KiviCache(w.batch, w.kv_heads, cap, bits=w.bits, group_k=w.group, group_v=w.gv,
+                               residual=w.residual, num_q_heads=w.q_heads)
+        cache.status.zero_()
+        cache.prefill(torch.from_numpy(k).cuda(), torch.from_numpy(v).cuda())
+        del k, v
+        outs = {0: cache.attend(torch.from_numpy(synth.queries(w, 0)).cuda()).cpu().numpy()}
+        runs = dict(zip(heads, fut))
+        gpu = {"step 0": _gpu_head_digests(cache, heads, _shapes(runs, "step 0"))}
+        for s in (1, 2):
+            if cache.n_res == w.residual:
+                cache.flush()
+                gpu[f"flush before step {s}"] = _gpu_head_digests(cache, heads, _shapes(runs, f"flush before step {s}"))
+            kn, vn = synth.new_kv(w, s)
+            q = synth.queries(w, s)
+            outs[s] = cache.append_attend(*(torch.from_numpy(x).cuda() for x in (kn, vn, q))).cpu().numpy()
+        gpu["step 2"] = _gpu_head_digests(cache, heads, _shapes(runs, "step 2"))
+        assert cache.read_status() == 0
+    for label in ("step 0", "flush before step 1", "step 2"):
+        _compare(label, gpu[label], None, runs, w.gqa, w.name)
+    for s in (0, 1, 2):
+        _compare(f"step {s}", None, outs[s], runs, w.gqa, w.name)
 
 
 @pytest.mark.parametrize("bits,group", [(2, 32), (2, 128), (4, 32), (4, 128)])
 def test_full_size_streaming(bits, group):
-    """Prefill 32768 tokens, then 256 decode steps (append, flush when full, attend).  The oracle
-    follows 4 sampled heads through every step and checks steps around both flushes."""
+    """Prefill 32768 tokens, then 256 decode steps (flush when full, append, attend), every head:
+    buffers bit for bit after both flushes and at the checked steps, outputs within tolerance at
+    steps around the flushes."""
     kivi = _kivi()
     w = synth.STREAMING.with_(bits=bits, group=group)
     cap = 33024
-    k, v = _streaming_prompt()
-    heads = gc.sample_heads(w, 4, seed=bits * 1000 + group)
-    ref = {bh: O.HeadCache(128, bits, group, group, w.residual, cap) for bh in heads}
-    for (b, h), hc in ref.items():
-        hc.prefill(k[b, h], v[b, h])
-    cache = kivi.KiviCache(w.batch, w.kv_heads, cap, bits=bits, group_k=group, group_v=group,
-                           residual=w.residual, num_q_heads=w.q_heads)
-    cache.prefill(torch.from_numpy(k).cuda(), torch.from_numpy(v).cuda())
-    for (b, h), hc in ref.items():
-        gc.assert_head_bitexact(gc.gpu_buffers_of_head(cache, b, h, cache.n_quant, cache.n_res), hc.packed(),
-                                f"prefill head {(b, h)}")
-    check_at = {1, 2, 127, 128, 129, 256}
-    for s in range(1, w.steps + 1):
-        if cache.n_res == w.residual:
-            cache.flush()
-            for hc in ref.values():
-                hc.flush()
-        kn, vn = synth.new_kv(w, s)
-        cache.append(torch.from_numpy(kn).cuda(), torch.from_numpy(vn).cuda())
-        for (b, h), hc in ref.items():
-            hc.append(kn[b, h], vn[b, h])
-        q = synth.queries(w, s)
-        out = cache.attend(torch.from_numpy(q).cuda())
-        if s in check_at:
-            out = out.cpu().numpy()
-            for (b, h), hc in ref.items():
-                gc.assert_attention_close(out[b, h:h + 1], hc.attend(q[b, h:h + 1], gc.default_scale()),
-                                          f"step {s} head {(b, h)}")
-                gc.assert_head_bitexact(gc.gpu_buffers_of_head(cache, b, h, cache.n_quant, cache.n_res),
-                                        hc.packed(), f"step {s} head {(b, h)}")
+    check_at = frozenset({1, 2, 127, 128, 129, 256})
+    heads = [(b, h) for b in range(w.batch) for h in range(w.kv_heads)]
+    specs = [ow.HeadStream(w, b, h, cap, w.tokens, steps=w.steps, attend_at=check_at, digest_at=check_at | {0})
+             for b, h in heads]
+    with ow.pool() as ex:
+        fut = ex.map(ow.run_head, specs, chunksize=2)
+        k, v = _streaming_prompt()
+        cache = kivi.KiviCache(w.batch, w.kv_heads, cap, bits=bits, group_k=group, group_v=group,
+                               residual=w.residual, num_q_heads=w.q_heads)
+        cache.prefill(torch.from_numpy(k).cuda(), torch.from_numpy(v).cuda())
+        runs = dict(zip(heads, fut))
+        shapes_of = lambda label: _shapes(runs, label)  # noqa: E731
+        _compare("step 0", _gpu_head_digests(cache, heads, shapes_of("step 0")), None, runs, w.gqa, "prefill")
+        for s in range(1, w.steps + 1):
+            if cache.n_res == w.residual:
+                cache.flush()
+                label = f"flush before step {s}"
+                _compare(label, _gpu_head_digests(cache, heads, shapes_of(label)), None, runs, w.gqa, w.name)
+            kn, vn = synth.new_kv(w, s)
+            q = synth.queries(w, s)
+            if s % 2:     # the fused call and the separate calls alternate
+                out = cache.append_attend(*(torch.from_numpy(x).cuda() for x in (kn, vn, q)))
+            else:
+                cache.append(torch.from_numpy(kn).cuda(), torch.from_numpy(vn).cuda())
+                out = cache.attend(torch.from_numpy(q).cuda())
+            if s in check_at:
+                label = f"step {s}"
+                _compare(label, _gpu_head_digests(cache, heads, shapes_of(label)), out.cpu().numpy(), runs, w.gqa,
+                         f"{w.name} {bits}-bit G={group}")
     assert cache.read_status() == 0
     assert (cache.n_quant, cache.n_res) == (32896, 128)
 
