@@ -14,6 +14,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libkivi.so")
+LIB_DEBUG = os.path.join(PKG, "libkivi_debug.so")   # -DKIVI_DEBUG: device-side bounds checks
 SOURCES = ["kivi_api.cu", "quantize.cu", "decode.cu", "noalloc.cu"]
 HEADERS = ["common.cuh", "kernels.h"]
 
@@ -25,20 +26,24 @@ def nvcc() -> str:
     raise RuntimeError("nvcc not found: set NVCC or put CUDA's bin/ on PATH")
 
 
-def _stale() -> bool:
-    if not os.path.exists(LIB):
+def _stale(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     deps = [os.path.join(CSRC, f) for f in SOURCES + HEADERS] + [os.path.join(INCLUDE, "kivi.h")]
     return any(os.path.getmtime(p) > t for p in deps)
 
 
-def build(force: bool = False, verbose_ptxas: bool = False) -> str:
-    """Compiles libkivi.so next to this file (skipped when up to date) and returns its path."""
-    if not force and not verbose_ptxas and not _stale():
-        return LIB
+def build(force: bool = False, verbose_ptxas: bool = False, debug: bool = False) -> str:
+    """Compiles libkivi.so next to this file (skipped when up to date) and returns its path.
+    debug=True builds libkivi_debug.so instead, with -DKIVI_DEBUG (the kernels' bounds checks)."""
+    lib = LIB_DEBUG if debug else LIB
+    if not force and not verbose_ptxas and not _stale(lib):
+        return lib
     cmd = [nvcc(), "-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",
-           "-Xcompiler", "-fPIC", "-shared", "-I", INCLUDE, "-I", CSRC, "-o", LIB + ".tmp"]
+           "-Xcompiler", "-fPIC", "-shared", "-I", INCLUDE, "-I", CSRC, "-o", lib + ".tmp"]
+    if debug:
+        cmd += ["-DKIVI_DEBUG"]
     if verbose_ptxas:
         cmd += ["-Xptxas", "-v"]
     cmd += [os.path.join(CSRC, f) for f in SOURCES]
@@ -47,9 +52,9 @@ def build(force: bool = False, verbose_ptxas: bool = False) -> str:
         raise RuntimeError("nvcc failed:\n" + proc.stdout + proc.stderr)
     if verbose_ptxas:
         sys.stderr.write(proc.stderr)
-    os.replace(LIB + ".tmp", LIB)
-    return LIB
+    os.replace(lib + ".tmp", lib)
+    return lib
 
 
 if __name__ == "__main__":
-    print(build(force=True, verbose_ptxas="--verbose-ptxas" in sys.argv))
+    print(build(force=True, verbose_ptxas="--verbose-ptxas" in sys.argv, debug="--debug" in sys.argv))

@@ -3,6 +3,7 @@
 
 #include <cstdint>
 #include <cuda_fp16.h>
+#include <cuda_runtime.h>
 
 #include "kivi.h"
 
@@ -67,13 +68,26 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
   return t;
 }
 
-// Bounded wait on an mbarrier phase: gives up after `limit_ns` of wall time and returns false.
+// try_wait that may suspend the thread for up to `hint_ns` while the phase is incomplete (the
+// thread resumes as soon as it completes), so a waiting warp does not spin through issue slots.
+__device__ __forceinline__ bool mbar_try_wait_hint(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait on an mbarrier phase: gives up after `limit_ns` of wall time (checked every 16
+// tries, each suspending for at most 20 us) and returns false.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   for (uint32_t spin = 0;; ++spin) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((spin & 63u) == 63u && global_timer_ns() - t0 > limit_ns) return false;
+    if (mbar_try_wait_hint(bar, parity, 20000u)) return true;
+    if ((spin & 15u) == 15u && global_timer_ns() - t0 > limit_ns) return false;
   }
 }
 
@@ -94,6 +108,44 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 
 __device__ __forceinline__ void report_status(int32_t* status, int code) {
   if (status != nullptr) atomicCAS(status, 0, code);
+}
+
+// ---- debug build (nvcc -DKIVI_DEBUG): device-side bounds checks ------------------------------
+// dbg_check(cond, status) is true in a release build (the condition is not evaluated at run time).
+// In a debug build a false condition records KIVI_ERR_INTERNAL in `status` (if given) and in the
+// translation unit's own debug word (read and cleared by kivi_debug_status), without a trap; the
+// caller then skips the access it guards.
+#ifdef KIVI_DEBUG
+constexpr bool kDebugBuild = true;
+static __device__ int32_t g_debug_status = 0;  // one per translation unit
+#else
+constexpr bool kDebugBuild = false;
+#endif
+
+__device__ __forceinline__ bool dbg_check(bool cond, int32_t* status = nullptr) {
+#ifdef KIVI_DEBUG
+  if (!cond) {
+    report_status(status, KIVI_ERR_INTERNAL);
+    atomicCAS(&g_debug_status, 0, KIVI_ERR_INTERNAL);
+    return false;
+  }
+#endif
+  (void)cond;
+  (void)status;
+  return true;
+}
+
+// Host side: reads and clears this translation unit's debug word (0 in a release build).
+static inline cudaError_t take_debug_status_tu(int32_t* out) {
+#ifdef KIVI_DEBUG
+  cudaError_t e = cudaMemcpyFromSymbol(out, g_debug_status, sizeof(int32_t));
+  if (e != cudaSuccess) return e;
+  const int32_t zero = 0;
+  return cudaMemcpyToSymbol(g_debug_status, &zero, sizeof(int32_t));
+#else
+  *out = 0;
+  return cudaSuccess;
+#endif
 }
 
 }  // namespace kivi

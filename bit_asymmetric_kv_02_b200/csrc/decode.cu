@@ -20,24 +20,27 @@
 // the residual unit holding its slot; that warp patches its shared-memory copy and the cache.
 //
 // Arithmetic.  The byte dot products are exact int32 sums.  At 2 bits they run on the tensor cores
-// (mma.sync m16n8k32, codes x limbs): dp4a would need 768 issues of the half-rate FMA-heavy pipe per
-// 8 KB and query, more than the HBM time of those bytes.  At 4 bits dp4a on the CUDA cores forms
-// them (half the dp4a per byte).
+// (mma.sync m16n8k32, code bytes x operand digits): dp4a would need 768 issues of the half-rate
+// FMA-heavy pipe per 8 KB and query, more than the HBM time of those bytes.  At 4 bits dp4a on the
+// CUDA cores forms them (half the dp4a per byte).
 //   A6  logit_t = sum_c q_c (s_g code + z_g) = sum_c (q_c s_g) code_tc + sum_g z_g sum_{c in g} q_c.
-//       (q_c s_g) for one R-token block is turned into a 24-bit signed fixed-point integer split in
-//       three byte limbs (kept while the warp stays in the same block); the codes are unpacked to
-//       bytes with one shift and masks and multiplied with the limbs exactly in int32.
-//       The block constant sum_g z_g q_g is added in fp32.
+//       (q_c s_g) for one R-token block is turned into a 24-bit signed fixed-point integer Q (kept
+//       while the warp stays in the same block).  At 2 bits a code word enters the tensor core as
+//       itself plus three masked copies (raw bytes: see variants2) against operand values built
+//       from the Q of each byte's four channels, four balanced signed byte digits each; at 4 bits
+//       the codes are unpacked to bytes and multiplied with three byte limbs of Q.  Both are exact
+//       in int32.  The block constant sum_g z_g q_g is added in fp32.
 //   A8  online softmax in base 2 (q pre-scaled by scale*log2 e), redux.sync warp maxima, lane-local
 //       sums.
 //   A9  o_c = sum_t (p_t s_g(t)) code_tc + sum_t p_t z_g(t): (p_t s_g(t)) is turned into 24-bit
 //       unsigned fixed point relative to a bound of the unit's largest value (at 2 bits: the
 //       unit's largest weight times its largest V scale; at 4 bits: the exact maximum) and dotted
-//       with the V codes; the z term is the same for every channel and is one scalar.
+//       with the V codes (raw bytes and operand digits at 2 bits, as for A6); the z term is the
+//       same for every channel and is one scalar.
 //   A7/A9 residual rows: fp32 FMAs on the fp16 values.
 //   A10 merge of (m, l, Z, o) states: o / l with o += Z.
-// 24-bit limbs keep every product relative error below 2^-21, the integer sums are exact, and the
-// remaining error is fp32 rounding.
+// 24-bit fixed point keeps every product relative error below 2^-21, the integer sums are exact, and
+// the remaining error is fp32 rounding.
 #include <cstdint>
 
 #include "common.cuh"
@@ -78,6 +81,9 @@ constexpr float kPRange = 16777088.f;  // 2^24 - 128: largest P before rounding 
 // Largest |Q| before rounding for balanced signed limbs (every digit in [-128, 127], so the top
 // digit (Q + 32896) >> 16 must stay below 128): 2^23 - 2^16.
 constexpr float kQRangeBal = 8323072.f;
+// Raw-byte operands (2 bits, base scheme): |Q| <= 2^23 keeps every operand value X below 2^30 in
+// magnitude (|X| <= 80 |Q|), inside the range of four balanced signed byte digits.
+constexpr float kQRangeRaw = 8388544.f;  // 2^23 - 64
 
 // Limb words per query: 96 (three limbs) for the CUDA-core dot products, 128 for the tensor-core
 // path, which keeps a fourth, all-zero limb slot (the B operand columns of no limb read it).
@@ -88,8 +94,9 @@ constexpr int kLimbVecs = 32;
 template <int G, bool FG = false>
 struct __align__(16) WarpSmem {
   uint8_t buf[ring_buffers<G>()][buf_bytes<G>()];
-  uint4 qw[FG ? 4 : G][kLimbVecs];  // Q limbs of each query (FG: of each K token group)
-  uint4 pw[FG ? 4 : G][kLimbVecs];  // P limbs of each query (FG: of each V channel group)
+  uint4 qw[FG ? 4 : G][kLimbVecs];  // Q operand digits of each query (FG: limbs of each K token group)
+  uint4 pw[FG ? 4 : G][kLimbVecs];  // P operand digits of each query (FG: limbs of each V channel group)
+  uint4 zero4;                      // the all-zero B operand of the other tile of a pair
   float oscr[FG ? kHeadDim : 4];
   uint64_t bar[ring_buffers<G>()];
 };
@@ -156,6 +163,56 @@ __device__ __forceinline__ float gather_limbs(const int (&c)[4], bool odd) {
   const int r2 = __shfl_xor_sync(0xffffffffu, c[3], 1);
   const int hi = odd ? r1 : c[0], mid = odd ? r2 : c[1], lo = odd ? c[2] : r1;
   return fmaf(static_cast<float>(hi), 65536.f, static_cast<float>((mid << 8) + lo));
+}
+
+// ---- raw-byte operands of the 2-bit tensor-core path ------------------------------------------
+// A byte of a 2-bit code word holds four codes c0 + 4 c1 + 16 c2 + 64 c3 (bits 0, 2, 4, 6).  The A
+// operand takes the word and three masked copies of it, whose bytes are
+//   V0 = c0 + 4 c1 + 16 c2 + 64 c3,  V1 = 4 c1 + 16 c2 + 64 c3,  V2 = 16 c2 + 64 c3,  V3 = 64 c3,
+// against B operand values X0 = 64 Q0, X1 = 16 Q1 - 64 Q0, X2 = 4 Q2 - 16 Q1, X3 = Q3 - 4 Q2 built
+// from the fixed-point values Q0..Q3 of the byte's four elements, so that
+//   V0 X0 + V1 X1 + V2 X2 + V3 X3 = 64 (c0 Q0 + c1 Q1 + c2 Q2 + c3 Q3)
+// exactly: three LOP3 per word instead of a shift and four masks.  Each X (|X| < 2^30) enters the
+// tensor core as four balanced signed byte digits, one B column per digit.
+__device__ __forceinline__ void variants2(uint32_t w, uint32_t (&v)[4]) {
+  v[0] = w;
+  v[1] = w & 0xFCFCFCFCu;
+  v[2] = w & 0xF0F0F0F0u;
+  v[3] = w & 0xC0C0C0C0u;
+}
+// Balanced signed digits of four operand values: word d holds digit d (weight 256^d) of x[m] in
+// byte m.  The digits are the bytes of x + 0x80808080, each minus 128 (= xor 0x80 as an s8), and a
+// 4 x 4 byte transpose gathers one digit of the four values into one word.
+__device__ __forceinline__ void digit_words(const int (&x)[4], uint32_t (&wd)[4]) {
+  uint32_t u[4];
+#pragma unroll
+  for (int m = 0; m < 4; ++m) u[m] = static_cast<uint32_t>(x[m]) + 0x80808080u;
+  const uint32_t t0 = __byte_perm(u[0], u[1], 0x5140), t1 = __byte_perm(u[0], u[1], 0x7362);
+  const uint32_t t2 = __byte_perm(u[2], u[3], 0x5140), t3 = __byte_perm(u[2], u[3], 0x7362);
+  wd[0] = __byte_perm(t0, t2, 0x5410) ^ 0x80808080u;
+  wd[1] = __byte_perm(t0, t2, 0x7632) ^ 0x80808080u;
+  wd[2] = __byte_perm(t1, t3, 0x5410) ^ 0x80808080u;
+  wd[3] = __byte_perm(t1, t3, 0x7632) ^ 0x80808080u;
+}
+// Stores the digit words of element variant `var` of operand row `row`: digit d goes to slot 3 - d
+// (B column 3 - d of its query or tile), word 16 row + 4 (slot ^ (row / 2 % 4)) + var.
+__device__ __forceinline__ void store_digits(uint4* rows, int row, int var, const uint32_t (&wd)[4]) {
+  uint32_t* base = reinterpret_cast<uint32_t*>(rows) + 16 * row + var;
+  const int sw = (row >> 1) & 3;
+  base[4 * (3 ^ sw)] = wd[0];
+  base[4 * (2 ^ sw)] = wd[1];
+  base[4 * (1 ^ sw)] = wd[2];
+  base[4 * (0 ^ sw)] = wd[3];
+}
+// Digit columns 3 and 2 of a tile (or query) land in even lanes t, columns 1 and 0 in odd lanes:
+// each lane forms c0 * 256 + c1 for rows g and g + 8 (exact in int32: every digit sum is below
+// 2^22), scales by 2^16 if even, and one exchange with lane ^ 1 leaves row g (even lane) or g + 8
+// (odd lane) whole.  sc = 65536 in even lanes, 1 in odd lanes.
+__device__ __forceinline__ float gather4(const int (&c)[4], bool odd, float sc) {
+  const float fg = static_cast<float>(c[0] * 256 + c[1]) * sc;
+  const float fh = static_cast<float>(c[2] * 256 + c[3]) * sc;
+  const float r = __shfl_xor_sync(0xffffffffu, odd ? fg : fh, 1);
+  return (odd ? fh : fg) + r;
 }
 
 // Largest worker whose range starts at or before unit u: start(x) = floor(U x / W).
@@ -250,6 +307,19 @@ struct Decoder {
                              : reinterpret_cast<const char*>(is_v ? a.v_res : a.k_res);
     const size_t stride = quant ? code_head_bytes : res_head_bytes;
     const int unit = quant ? local : local - a.units_q;
+    if constexpr (kDebugBuild) {  // the copy stays inside the head's arrays and the filled tokens
+      bool ok = head >= 0 && head < a.bh && local >= 0 && local < a.units;
+      if (KC && !quant && !is_v)
+        ok = ok && a.n_quant + (unit + 1) * kResTokens <= a.capacity;
+      else if (quant)
+        ok = ok && (unit + 1) * UT <= a.n_quant && static_cast<size_t>(unit + 1) * kHalfBytes <= code_head_bytes;
+      else
+        ok = ok && unit * kResTokens < a.n_res && (unit + 1) * kResTokens <= a.residual;
+      if (!dbg_check(ok, a.status)) {  // no copy: the phase completes at once on stale data
+        mbar_arrive_expect_tx(&S.bar[b], 0);
+        return;
+      }
+    }
     const char* src = base + static_cast<size_t>(head) * stride + static_cast<size_t>(unit) * kHalfBytes;
     if (KC && !quant && !is_v) {  // online K: 16 code rows from token n_quant + 16 unit
       constexpr uint32_t kRowBytes = kHeadDim * BITS / 8;
@@ -279,7 +349,9 @@ struct Decoder {
     const uint16_t* ps = k_lane ? a.k_scale + ik : a.v_scale + iv;
     const uint16_t* pz = k_lane ? a.k_zero + ik : a.v_zero + iv;
     uint32_t r = 0u;
-    if (!FG && (k_lane || v_lane) && local < a.units_q)  // FG loads its own scales per unit
+    if (!FG && (k_lane || v_lane) && local < a.units_q &&  // FG loads its own scales per unit
+        dbg_check(k_lane ? ik < static_cast<size_t>(a.bh) * a.blocks_per_head * ngk
+                         : iv < static_cast<size_t>(a.bh) * a.vgroups_per_head, a.status))
       r = static_cast<uint32_t>(__ldg(ps)) | (static_cast<uint32_t>(__ldg(pz)) << 16);
     return r;
   }
@@ -370,134 +442,140 @@ struct Decoder {
     __syncwarp();
   }
 
-  // ---- tensor-core path (2 bits, one query per KV head) ---------------------------------------
-  // Limb layout in shared memory, Q and P alike: word (i, slot, set) at 16 i + 4 (slot ^ (i / 2 % 4))
-  // + set for i = K code word (Q) or V word row (P); slots 0, 1, 2 hold the high, middle and low
-  // limbs and slot 3 stays zero.  The XOR spreads the four lanes t that read rows 2 t + x of one
-  // slot over four bank groups.  Byte m of (i, slot, set) belongs to channel 16 i + 4 m + set (Q) or token
-  // 16 i + 4 m + set (P), the element that byte m of set `set` of a code word multiplies.
+  // ---- tensor-core path (2 bits), raw-byte operands ------------------------------------------
+  // Operand layout in shared memory, Q and P alike: word (row, slot, var) at 16 row + 4 (slot ^
+  // (row / 2 % 4)) + var, for row = K code word (Q) or V word row (P) and var = the element variant
+  // 0..3 of a byte.  Slot s holds digit 3 - s of the operand values; byte m of the word belongs to
+  // byte m of the code words (channels 16 row + 4 m + var of Q, tokens 16 row + 4 m + var of P).  The
+  // XOR spreads the four lanes t that read rows 2 t + x of one slot over four bank groups.
   //
-  // An m16n8k32 tile contracts 32 channels (K) or 32 tokens (V) of 16 rows (tokens or channels)
-  // against the three limbs in B columns 0..2.  Two tiles share one accumulator: the second's limbs
-  // sit in columns 4..6, so lane (n, t) with n = lane / 4 reads B from slot n (n < 3) for the first
-  // tile and slot n - 4 (4 <= n < 7) for the second, slot 3 otherwise.
+  // An m16n8k32 tile contracts 8 code bytes (32 elements) of 16 rows (tokens or channels) against
+  // the four digit columns.  With one query per KV head two tiles share one accumulator: the first
+  // tile's digits sit in B columns 0..3 and the second's in 4..7, so lane (n, t) with n = lane / 4
+  // reads slot n of the first tile's operand (n < 4) or of the second's (n >= 4) and the all-zero
+  // operand for the other tile.  With several queries, n8 block p holds queries 2 p (columns 0..3)
+  // and 2 p + 1 (columns 4..7).
 
-  // Q limbs as balanced signed digits, Q = H 2^16 + M 2^8 + L with every digit in [-128, 127]
-  // (an s8 B operand): L = byte 0 of Q, M = byte 1 of Q + 128, H = byte 2 of Q + 32896.
-  // Lane (i, k) forms the words (i, slot, k) of channels 16 i + 4 m + k; odd sets read 4 * code.
+  // Q operands of one K block: lane (i, k) forms variant k of K word i for bytes m = 0..3 (channels
+  // 16 i + 4 m + k); the previous channel's Q is lane - 1's (variant k - 1 of the same word).
   __device__ void build_q2_mma(uint32_t pairs) {
     const int gi = (16 * (lane >> 2)) >> a.lg_gk;  // the K group of all four channels
     const float s = h2f(static_cast<uint16_t>(__shfl_sync(kFull, pairs, gi) & 0xFFFFu));
     const float z_own = k_lane ? h2f(static_cast<uint16_t>(pairs >> 16)) : 0.f;
-    const int i = lane >> 2, sw = (i >> 1) & 3;
+    const int i = lane >> 2, k = lane & 3;
+    const int xa = 64 >> (2 * k), xb = k ? (256 >> (2 * k)) : 0;
 #pragma unroll
     for (int g = 0; g < G; ++g) {
       float qv[4];
 #pragma unroll
       for (int j = 0; j < 4; ++j) qv[j] = q_of(g, j) * s;
       const float mabs = warp_max(fmaxf(fmaxf(fabsf(qv[0]), fabsf(qv[1])), fmaxf(fabsf(qv[2]), fabsf(qv[3]))));
-      const float scq = mabs > 0.f ? kQRangeBal * fast_rcp(mabs) : 0.f;
-      invq[g] = mabs * (1.0f / kQRangeBal);
+      const float scq = mabs > 0.f ? kQRangeRaw * fast_rcp(mabs) : 0.f;
+      invq[g] = mabs * (1.0f / (64.f * kQRangeRaw));  // the operands carry 64 Q
       float c = z_own * qsum[g][0];
       c += __shfl_xor_sync(kFull, c, 1);
       c += __shfl_xor_sync(kFull, c, 2);
       cblk[g] = __shfl_sync(kFull, c, 0);
-      const float f = scq * ((lane & 1) ? 0.25f : 1.f);
-      uint32_t Q[4];
+      int x[4];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) Q[j] = static_cast<uint32_t>(__float2int_rn(qv[j] * f));
-      uint32_t* row = reinterpret_cast<uint32_t*>(S.qw[g]) + 16 * i + (lane & 3);
-      row[4 * (0 ^ sw)] = pick_bytes(Q[0] + 32896u, Q[1] + 32896u, Q[2] + 32896u, Q[3] + 32896u, 2);
-      row[4 * (1 ^ sw)] = pick_bytes(Q[0] + 128u, Q[1] + 128u, Q[2] + 128u, Q[3] + 128u, 1);
-      row[4 * (2 ^ sw)] = pick_bytes(Q[0], Q[1], Q[2], Q[3], 0);
+      for (int j = 0; j < 4; ++j) {
+        const int Q = __float2int_rn(qv[j] * scq);
+        const int Qp = __shfl_up_sync(kFull, Q, 1);
+        x[j] = Q * xa - Qp * xb;
+      }
+      uint32_t wd[4];
+      digit_words(x, wd);
+      store_digits(S.qw[g], i, k, wd);
     }
   }
 
-  // Logits of the unit's 128 tokens.  Tile 2 j + b holds tokens 32 j + 16 b + (0..15) as rows;
-  // lane (g, t) unpacks code words 2 t and 2 t + 1 of tokens 32 j + 16 b + g and + 8.  After the
-  // exchange, lg[j] is the logit of token 32 j + 16 (t / 2) + 8 (t % 2) + g.
+  // Logits of the unit's 128 tokens.  Tile b of pair j holds on row g + 8 c the token
+  // 16 (g / 4 + 2 c + 4 b) + 4 j + g % 4, so that after the exchange lane (g, t) holds in lg[j] the
+  // logit of token 16 r + 4 j + v with r = g / 4 + 2 (t % 2) + 4 (t / 2) and v = g % 4: the four
+  // tokens whose P operands variant v of word row r needs (see softmax_mma).
   __device__ void k_mma(const uint8_t* kt, float (&lg)[4]) const {
     const int g = lane >> 2, t = lane & 3;
-    const int se = g < 4 ? g : 3, so = g >= 4 ? g - 4 : 3;
-    const uint4 be0 = S.qw[0][8 * t + (se ^ t)], be1 = S.qw[0][8 * t + 4 + (se ^ t)];
-    const uint4 bo0 = S.qw[0][8 * t + (so ^ t)], bo1 = S.qw[0][8 * t + 4 + (so ^ t)];
+    const int si = 8 * t + ((g & 3) ^ t);
+    const uint4* pe = g < 4 ? &S.qw[0][si] : &S.zero4;   // tile 0's operand, or zero
+    const uint4* po = g >= 4 ? &S.qw[0][si] : &S.zero4;  // tile 1's
+    const uint4 be0 = pe[0], be1 = pe[g < 4 ? 4 : 0], bo0 = po[0], bo1 = po[g >= 4 ? 4 : 0];
     const bool odd = t & 1;
+    const float sc = odd ? 1.f : 65536.f;
+    const uint8_t* base = kt + (16 * (g >> 2) + (g & 3)) * 32 + 8 * t;
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       int c[4] = {0, 0, 0, 0};
 #pragma unroll
       for (int b = 0; b < 2; ++b) {
-        const uint8_t* r0 = kt + (32 * j + 16 * b + g) * 32 + 8 * t;
+        const uint8_t* r0 = base + (4 * j + 64 * b) * 32;
         const uint2 wg = *reinterpret_cast<const uint2*>(r0);
-        const uint2 wh = *reinterpret_cast<const uint2*>(r0 + 8 * 32);
+        const uint2 wh = *reinterpret_cast<const uint2*>(r0 + 32 * 32);  // row g + 8: 32 tokens on
         const uint4& B0 = b ? bo0 : be0;
         const uint4& B1 = b ? bo1 : be1;
-        uint32_t mg[4], mh[4];
-        masks2(wg.x, mg);
-        masks2(wh.x, mh);
-        mma_u8s8(c, mg[0], mh[0], mg[1], mh[1], B0.x, B0.y);
-        mma_u8s8(c, mg[2], mh[2], mg[3], mh[3], B0.z, B0.w);
-        masks2(wg.y, mg);
-        masks2(wh.y, mh);
-        mma_u8s8(c, mg[0], mh[0], mg[1], mh[1], B1.x, B1.y);
-        mma_u8s8(c, mg[2], mh[2], mg[3], mh[3], B1.z, B1.w);
+        uint32_t vg[4], vh[4];
+        variants2(wg.x, vg);
+        variants2(wh.x, vh);
+        mma_u8s8(c, vg[0], vh[0], vg[1], vh[1], B0.x, B0.y);
+        mma_u8s8(c, vg[2], vh[2], vg[3], vh[3], B0.z, B0.w);
+        variants2(wg.y, vg);
+        variants2(wh.y, vh);
+        mma_u8s8(c, vg[0], vh[0], vg[1], vh[1], B1.x, B1.y);
+        mma_u8s8(c, vg[2], vh[2], vg[3], vh[3], B1.z, B1.w);
       }
-      lg[j] = fmaf(gather_limbs(c, odd), invq[0], cblk[0]);
+      lg[j] = fmaf(gather4(c, odd, sc), invq[0], cblk[0]);
     }
   }
 
-  // Online softmax of the unit and its P limbs (unsigned bytes), scaled by the bound 2^(mu - m) *
-  // s_max as on the CUDA-core path.  Token 32 j + ... lies in V group (32 j) >> lg_gv of the unit
-  // (V groups span at least 32 tokens); its P goes to byte 2 (t % 2) + g / 4 of word
-  // (2 j + t / 2, slot, g % 4), whose slot position is slot ^ j.
+  // Online softmax of the unit and its P operands, P = p s scaled by the bound 2^(mu - m) s_max
+  // (reading R16).  Lane (g, t) holds tokens 16 r + 4 m + v (m = 0..3) of word row r, which lie in
+  // one V group (V groups span at least 32 tokens); the previous token's P is lane - 4's.
   __device__ void softmax_mma(uint32_t pairs, const float (&lg)[4]) {
     const int g = lane >> 2, t = lane & 3;
+    const int r = (g >> 2) + 2 * (t & 1) + 4 * (t >> 1), v = g & 3;
     const float mu = warp_max(fmaxf(fmaxf(lg[0], lg[1]), fmaxf(lg[2], lg[3])));
     const float smax = warp_max(v_lane ? h2f(static_cast<uint16_t>(pairs & 0xFFFFu)) : 0.f);
     const float m_new = fmaxf(m[0], mu);
     const float alpha = fast_exp2(m[0] - m_new);
     const float d = mu - m_new;  // <= 0: the unit's largest weight is 2^d
     const bool hv = d > -64.f && smax > 0.f;
-    const float fb = hv ? (kPRange * fast_rcp(smax)) * fast_exp2(-d) * ((g & 1) ? 0.25f : 1.f) : 0.f;
-    float p[4], sv[4], psum = 0.f, zsum = 0.f;
+    const uint32_t vp = __shfl_sync(kFull, pairs, 8 + ((16 * r) >> a.lg_gv));
+    const float sv = h2f(static_cast<uint16_t>(vp & 0xFFFFu)), zv = h2f(static_cast<uint16_t>(vp >> 16));
+    const float f = hv ? (kPRange * fast_rcp(smax)) * fast_exp2(-d) * sv : 0.f;
+    const int xa = 64 >> (2 * v), xb = v ? (256 >> (2 * v)) : 0;
+    float psum = 0.f;
+    int x[4];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      const uint32_t vp = __shfl_sync(kFull, pairs, 8 + ((32 * j) >> a.lg_gv));
-      sv[j] = h2f(static_cast<uint16_t>(vp & 0xFFFFu));
-      p[j] = fast_exp2(lg[j] - m_new);
-      psum += p[j];
-      zsum = fmaf(p[j], h2f(static_cast<uint16_t>(vp >> 16)), zsum);
+      const float p = fast_exp2(lg[j] - m_new);
+      psum += p;
+      const int P = static_cast<int>(__float2uint_rn(p * f));
+      const int Pp = __shfl_up_sync(kFull, P, 4);
+      x[j] = P * xa - Pp * xb;
     }
     m[0] = m_new;
     l[0] = fmaf(l[0], alpha, psum);
-    Z[0] = fmaf(Z[0], alpha, zsum);
+    Z[0] = fmaf(Z[0], alpha, psum * zv);
     alpha_[0] = alpha;
     hasv_[0] = hv;
-    invv_[0] = hv ? fast_exp2(d) * smax * (1.0f / kPRange) : 0.f;
-    uint8_t* pb = reinterpret_cast<uint8_t*>(S.pw[0]) + 64 * (t >> 1) + 4 * (g & 3) + 2 * (t & 1) + (g >> 2);
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const uint32_t P = __float2uint_rn(p[j] * (sv[j] * fb));
-      pb[128 * j + 16 * (0 ^ j)] = static_cast<uint8_t>(P >> 16);
-      pb[128 * j + 16 * (1 ^ j)] = static_cast<uint8_t>(P >> 8);
-      pb[128 * j + 16 * (2 ^ j)] = static_cast<uint8_t>(P);
-    }
+    invv_[0] = hv ? fast_exp2(d) * smax * (1.0f / (64.f * kPRange)) : 0.f;
+    uint32_t wd[4];
+    digit_words(x, wd);
+    store_digits(S.pw[0], r, v, wd);
   }
 
   // P . codes of the unit.  Tile pair v holds channels 16 g' + 8 b + 4 c + v (tile 2 v + b, row
-  // g' + 8 c) as rows; lane (g, t) unpacks V word rows 2 t and 2 t + 1 of channels 16 g .. 16 g + 15
+  // g' + 8 c) as rows; lane (g, t) reads V word rows 2 t and 2 t + 1 of channels 16 g .. 16 g + 15
   // (four 16-byte loads per row).  After the exchange the lane holds channel 4 lane + v of tile
   // pair v, the channel it accumulates in o[0][v].  Rows 2 t and 2 t + 1 are piece t of the buffer.
   __device__ void v_mma(const uint8_t* vt) {
     static_assert(P == 16 && ROWS == 8, "2-bit units: 8 V word rows of 16 tokens");
     const int g = lane >> 2, t = lane & 3;
-    const int se = g < 4 ? g : 3, so = g >= 4 ? g - 4 : 3;
-    uint4 be[2], bo[2];
-#pragma unroll
-    for (int x = 0; x < 2; ++x) {
-      be[x] = S.pw[0][8 * t + 4 * x + (se ^ t)];
-      bo[x] = S.pw[0][8 * t + 4 * x + (so ^ t)];
-    }
+    const int si = 8 * t + ((g & 3) ^ t);
+    const uint4* pe = g < 4 ? &S.pw[0][si] : &S.zero4;
+    const uint4* po = g >= 4 ? &S.pw[0][si] : &S.zero4;
+    const uint4 be[2] = {pe[0], pe[g < 4 ? 4 : 0]}, bo[2] = {po[0], po[g >= 4 ? 4 : 0]};
+    const bool odd = t & 1;
+    const float sc = odd ? 1.f : 65536.f;
     int cv[4][4];
 #pragma unroll
     for (int v = 0; v < 4; ++v) cv[v][0] = cv[v][1] = cv[v][2] = cv[v][3] = 0;
@@ -511,17 +589,16 @@ struct Decoder {
         const uint4& B = b ? bo[x] : be[x];
 #pragma unroll
         for (int v = 0; v < 4; ++v) {
-          uint32_t mg[4], mh[4];
-          masks2(comp(wlo, v), mg);
-          masks2(comp(whi, v), mh);
-          mma_u8u8(cv[v], mg[0], mh[0], mg[1], mh[1], B.x, B.y);
-          mma_u8u8(cv[v], mg[2], mh[2], mg[3], mh[3], B.z, B.w);
+          uint32_t vg[4], vh[4];
+          variants2(comp(wlo, v), vg);
+          variants2(comp(whi, v), vh);
+          mma_u8s8(cv[v], vg[0], vh[0], vg[1], vh[1], B.x, B.y);
+          mma_u8s8(cv[v], vg[2], vh[2], vg[3], vh[3], B.z, B.w);
         }
       }
     }
-    const bool odd = t & 1;
 #pragma unroll
-    for (int v = 0; v < 4; ++v) o[0][v] = fmaf(o[0][v], alpha_[0], gather_limbs(cv[v], odd) * invv_[0]);
+    for (int v = 0; v < 4; ++v) o[0][v] = fmaf(o[0][v], alpha_[0], gather4(cv[v], odd, sc) * invv_[0]);
   }
 
   // 4 bits: lane holds channels lane + 32 j; each byte of a limb word is stored on its own.
@@ -590,7 +667,10 @@ struct Decoder {
         float qv[4], qz = 0.f;
 #pragma unroll
         for (int m = 0; m < 4; ++m) {
-          const size_t ci = row0 + static_cast<size_t>(u) * kHeadDim + 16 * i + 4 * m + kk;
+          size_t ci = row0 + static_cast<size_t>(u) * kHeadDim + 16 * i + 4 * m + kk;
+          if (!dbg_check(ci < static_cast<size_t>(a.bh) * (static_cast<size_t>(a.capacity) >> a.lg_gk) * kHeadDim,
+                         a.status))
+            ci = 0;
           const float sk = h2f(__ldg(a.k_scale + ci)), zk = h2f(__ldg(a.k_zero + ci));
           qv[m] = q_of(0, m) * sk;
           qz = fmaf(q_of(0, m), zk, qz);
@@ -653,9 +733,10 @@ struct Decoder {
       const size_t tok = static_cast<size_t>(head) * a.capacity + static_cast<size_t>(local) * UT + 32 * j +
                          16 * (t >> 1) + 8 * (t & 1) + g;
 #pragma unroll
+      const bool in = dbg_check(tok < static_cast<size_t>(a.bh) * a.capacity, a.status);
       for (int gc = 0; gc < 4; ++gc) {
-        sv[j][gc] = gc < ngv ? h2f(__ldg(a.v_scale + tok * ngv + gc)) : 0.f;
-        zv[j][gc] = gc < ngv ? h2f(__ldg(a.v_zero + tok * ngv + gc)) : 0.f;
+        sv[j][gc] = gc < ngv && in ? h2f(__ldg(a.v_scale + tok * ngv + gc)) : 0.f;
+        zv[j][gc] = gc < ngv && in ? h2f(__ldg(a.v_zero + tok * ngv + gc)) : 0.f;
         smax_l = fmaxf(smax_l, sv[j][gc]);
       }
     }
@@ -746,18 +827,20 @@ struct Decoder {
 
   // ---- tensor-core path, several queries per KV head ------------------------------------------
   // B column n of n8 block p reads slot n % 4 of query 2 p + n / 4, so one accumulator holds the
-  // three limbs of queries 2 p (columns 0..2) and 2 p + 1 (columns 4..6) for one 16-row tile.  After
-  // the exchange a lane holds query 2 p + t / 2 of row g + 8 (t % 2).
+  // four digit columns of queries 2 p (columns 0..3) and 2 p + 1 (columns 4..7) for one 16-row tile.
+  // After the exchange a lane holds query 2 p + t / 2 of row g + 8 (t % 2).
   //
   // Output layout while quantized units run: o[2 p + b][v] of lane (g, t) holds query 2 p + t / 2,
   // channel 16 g + 8 b + 4 (t % 2) + v.  o_swap_layout() turns it into the layout of the residual
   // path and the merge (o[q][e]: query q, channel 4 lane + e) and back: it is an involution.
 
-  // Logits of the unit's 128 tokens for every query: tile tau holds tokens 16 tau + (0..15) as
-  // rows; lg[p][tau] is the logit of query 2 p + t / 2 for token 16 tau + 8 (t % 2) + g.
+  // Logits of the unit's 128 tokens for every query.  Tile tau holds on row g + 8 c the token
+  // 16 (g / 4 + 2 c + 4 (tau / 4)) + 4 (tau % 4) + g % 4; lg[p][tau] is the logit of query
+  // 2 p + t / 2 for token 16 (r0 + 4 (tau / 4)) + 4 (tau % 4) + v, r0 = g / 4 + 2 (t % 2), v = g % 4.
   __device__ void k_mma_g(const uint8_t* kt, float (&lg)[NBLK][8]) const {
     const int g = lane >> 2, t = lane & 3, qh = g >> 2, sl = (g & 3) ^ t;
     const bool odd = t & 1;
+    const float sc = odd ? 1.f : 65536.f;
     uint4 B[NBLK][2];
 #pragma unroll
     for (int p = 0; p < NBLK; ++p) {
@@ -770,44 +853,47 @@ struct Decoder {
       iq[p] = (t >> 1) ? invq[2 * p + 1] : invq[2 * p];
       cb[p] = (t >> 1) ? cblk[2 * p + 1] : cblk[2 * p];
     }
+    const uint8_t* base = kt + (16 * (g >> 2) + (g & 3)) * 32 + 8 * t;
 #pragma unroll
     for (int tau = 0; tau < 8; ++tau) {
-      const uint8_t* r0 = kt + (16 * tau + g) * 32 + 8 * t;
+      const uint8_t* r0 = base + (64 * (tau >> 2) + 4 * (tau & 3)) * 32;
       const uint2 wg = *reinterpret_cast<const uint2*>(r0);
-      const uint2 wh = *reinterpret_cast<const uint2*>(r0 + 8 * 32);
+      const uint2 wh = *reinterpret_cast<const uint2*>(r0 + 32 * 32);  // row g + 8: 32 tokens on
       int c[NBLK][4];
 #pragma unroll
       for (int p = 0; p < NBLK; ++p) c[p][0] = c[p][1] = c[p][2] = c[p][3] = 0;
 #pragma unroll
       for (int w = 0; w < 2; ++w) {
-        uint32_t mg[4], mh[4];
-        masks2(w ? wg.y : wg.x, mg);
-        masks2(w ? wh.y : wh.x, mh);
+        uint32_t vg[4], vh[4];
+        variants2(w ? wg.y : wg.x, vg);
+        variants2(w ? wh.y : wh.x, vh);
 #pragma unroll
         for (int p = 0; p < NBLK; ++p) {
-          mma_u8s8(c[p], mg[0], mh[0], mg[1], mh[1], B[p][w].x, B[p][w].y);
-          mma_u8s8(c[p], mg[2], mh[2], mg[3], mh[3], B[p][w].z, B[p][w].w);
+          mma_u8s8(c[p], vg[0], vh[0], vg[1], vh[1], B[p][w].x, B[p][w].y);
+          mma_u8s8(c[p], vg[2], vh[2], vg[3], vh[3], B[p][w].z, B[p][w].w);
         }
       }
 #pragma unroll
-      for (int p = 0; p < NBLK; ++p) lg[p][tau] = fmaf(gather_limbs(c[p], odd), iq[p], cb[p]);
+      for (int p = 0; p < NBLK; ++p) lg[p][tau] = fmaf(gather4(c[p], odd, sc), iq[p], cb[p]);
     }
   }
 
-  // Online softmax of every query over the unit and the P limbs of each query (bound scaling as on
-  // the other paths).  Token 16 tau + ... lies in V group (16 tau) >> lg_gv of the unit; its P goes
-  // to byte (g / 4) + 2 (t % 2) of word (tau, slot, g % 4) of its query.
+  // Online softmax of every query over the unit and the P operands of each query (bound scaling as
+  // on the other paths).  Lane (g, t) holds, for query 2 p + t / 2, tokens 16 r + 4 m + v of word
+  // rows r = r0 and r0 + 4 (tiles tau = 4 h + m): each row lies in one V group; the previous token's
+  // P is lane - 4's.
   __device__ void softmax_mma_g(uint32_t pairs, const float (&lg)[NBLK][8]) {
     const int g = lane >> 2, t = lane & 3, h = t >> 1;
+    const int r0 = (g >> 2) + 2 * (t & 1), v = g & 3;
+    const int xa = 64 >> (2 * v), xb = v ? (256 >> (2 * v)) : 0;
     const float smax = warp_max(v_lane ? h2f(static_cast<uint16_t>(pairs & 0xFFFFu)) : 0.f);
     const float kinv = smax > 0.f ? kPRange * fast_rcp(smax) : 0.f;
-    const float set_scale = (g & 1) ? 0.25f : 1.f;
-    float sv[8], zv[8];
+    float sv[2], zv[2];
 #pragma unroll
-    for (int tau = 0; tau < 8; ++tau) {
-      const uint32_t vp = __shfl_sync(kFull, pairs, 8 + ((16 * tau) >> a.lg_gv));
-      sv[tau] = h2f(static_cast<uint16_t>(vp & 0xFFFFu));
-      zv[tau] = h2f(static_cast<uint16_t>(vp >> 16));
+    for (int hh = 0; hh < 2; ++hh) {
+      const uint32_t vp = __shfl_sync(kFull, pairs, 8 + ((16 * (r0 + 4 * hh)) >> a.lg_gv));
+      sv[hh] = h2f(static_cast<uint16_t>(vp & 0xFFFFu));
+      zv[hh] = h2f(static_cast<uint16_t>(vp >> 16));
     }
 #pragma unroll
     for (int p = 0; p < NBLK; ++p) {
@@ -824,25 +910,32 @@ struct Decoder {
         const bool hv = d > -64.f && smax > 0.f;
         alpha_[q] = fast_exp2(m[q] - m_new);
         hasv_[q] = hv;
-        invv_[q] = hv ? fast_exp2(d) * smax * (1.0f / kPRange) : 0.f;
+        invv_[q] = hv ? fast_exp2(d) * smax * (1.0f / (64.f * kPRange)) : 0.f;
         m[q] = m_new;
         if (h == e) {
           mn_l = m_new;
-          fb = hv ? kinv * fast_exp2(-d) * set_scale : 0.f;
+          fb = hv ? kinv * fast_exp2(-d) : 0.f;
         }
       }
-      uint8_t* pb = reinterpret_cast<uint8_t*>(S.pw[2 * p + h]) + 4 * (g & 3) + (g >> 2) + 2 * (t & 1);
       float psum = 0.f, zsum = 0.f;
 #pragma unroll
-      for (int tau = 0; tau < 8; ++tau) {
-        const float pv = fast_exp2(lg[p][tau] - mn_l);
-        psum += pv;
-        zsum = fmaf(pv, zv[tau], zsum);
-        const uint32_t P = __float2uint_rn(pv * (sv[tau] * fb));
-        const int sw = (tau >> 1) & 3;
-        pb[64 * tau + 16 * (0 ^ sw)] = static_cast<uint8_t>(P >> 16);
-        pb[64 * tau + 16 * (1 ^ sw)] = static_cast<uint8_t>(P >> 8);
-        pb[64 * tau + 16 * (2 ^ sw)] = static_cast<uint8_t>(P);
+      for (int hh = 0; hh < 2; ++hh) {
+        const float f = sv[hh] * fb;
+        float ph = 0.f;
+        int x[4];
+#pragma unroll
+        for (int mm = 0; mm < 4; ++mm) {
+          const float pv = fast_exp2(lg[p][4 * hh + mm] - mn_l);
+          ph += pv;
+          const int P = static_cast<int>(__float2uint_rn(pv * f));
+          const int Pp = __shfl_up_sync(kFull, P, 4);
+          x[mm] = P * xa - Pp * xb;
+        }
+        psum += ph;
+        zsum = fmaf(ph, zv[hh], zsum);
+        uint32_t wd[4];
+        digit_words(x, wd);
+        store_digits(S.pw[2 * p + h], r0 + 4 * hh, v, wd);
       }
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
@@ -854,10 +947,11 @@ struct Decoder {
   }
 
   // P . codes of the unit for every query.  Tile (v, b) holds channels 16 g' + 8 b + 4 c + v (row
-  // g' + 8 c); lane (g, t) unpacks V word rows 2 t + x of channels 16 g .. 16 g + 15.
+  // g' + 8 c); lane (g, t) reads V word rows 2 t + x of channels 16 g .. 16 g + 15.
   __device__ void v_mma_g(const uint8_t* vt) {
     const int g = lane >> 2, t = lane & 3, qh = g >> 2, sl = (g & 3) ^ t;
     const bool odd = t & 1;
+    const float sc = odd ? 1.f : 65536.f;
     uint4 B[NBLK][2];
 #pragma unroll
     for (int p = 0; p < NBLK; ++p) {
@@ -884,13 +978,13 @@ struct Decoder {
         const uint4 whi = *reinterpret_cast<const uint4*>(rowp + 32 * b + 16);
 #pragma unroll
         for (int v = 0; v < 4; ++v) {
-          uint32_t mg[4], mh[4];
-          masks2(comp(wlo, v), mg);
-          masks2(comp(whi, v), mh);
+          uint32_t vg[4], vh[4];
+          variants2(comp(wlo, v), vg);
+          variants2(comp(whi, v), vh);
 #pragma unroll
           for (int p = 0; p < NBLK; ++p) {
-            mma_u8u8(acc[v][p], mg[0], mh[0], mg[1], mh[1], B[p][x].x, B[p][x].y);
-            mma_u8u8(acc[v][p], mg[2], mh[2], mg[3], mh[3], B[p][x].z, B[p][x].w);
+            mma_u8s8(acc[v][p], vg[0], vh[0], vg[1], vh[1], B[p][x].x, B[p][x].y);
+            mma_u8s8(acc[v][p], vg[2], vh[2], vg[3], vh[3], B[p][x].z, B[p][x].w);
           }
         }
       }
@@ -898,7 +992,7 @@ struct Decoder {
       for (int v = 0; v < 4; ++v)
 #pragma unroll
         for (int p = 0; p < NBLK; ++p)
-          o[2 * p + b][v] = fmaf(o[2 * p + b][v], al[p], gather_limbs(acc[v][p], odd) * iv[p]);
+          o[2 * p + b][v] = fmaf(o[2 * p + b][v], al[p], gather4(acc[v][p], odd, sc) * iv[p]);
     }
   }
 
@@ -1097,6 +1191,7 @@ struct Decoder {
   __device__ void insert_new_row(uint8_t* buf, int r, long long head, const uint16_t* src, uint16_t* res, bool v_half) {
     const int row = a.new_slot - r * kResTokens;
     if (a.new_slot < 0 || row < 0 || row >= kResTokens) return;
+    if (!dbg_check(a.new_slot < a.residual && head < a.bh, a.status)) return;
     const uint2 v = __ldg(reinterpret_cast<const uint2*>(src + static_cast<size_t>(head) * kHeadDim) + lane);
     *reinterpret_cast<uint2*>(buf + (v_half ? vrow(row) : row * 256) + 8 * lane) = v;
     uint16_t* dst = res + (static_cast<size_t>(head) * a.residual + a.new_slot) * kHeadDim;
@@ -1111,7 +1206,8 @@ struct Decoder {
     constexpr int kRowBytes = kHeadDim * BITS / 8, WPL = 64 / P;
     constexpr uint32_t L = (1u << BITS) - 1u;
     const int t = lane >> 1, hf = lane & 1;
-    const size_t sb = (static_cast<size_t>(head) * a.blocks_per_head + a.res_blk) * ngk;
+    size_t sb = (static_cast<size_t>(head) * a.blocks_per_head + a.res_blk) * ngk;
+    if (!dbg_check(a.res_blk < a.blocks_per_head && head < a.bh, a.status)) sb = 0;
     uint32_t w[WPL];
 #pragma unroll
     for (int i = 0; i < WPL; i += 4) {
@@ -1237,6 +1333,7 @@ struct Decoder {
       return;
     }
     const int slot = seg_a == ub ? 0 : 1;
+    if (!dbg_check(worker < a.workers && head < a.bh, a.status)) return;
     float* mine = a.partials + ((worker * 2 + slot) * G) * kPartialStride;
 #pragma unroll
     for (int g = 0; g < G; ++g) {
@@ -1266,6 +1363,7 @@ struct Decoder {
     // before the head (its partial is then in its slot 1); every later one starts inside it.
     const int nparts = static_cast<int>(wlast - wfirst + 1);
     const int first_slot = (U * wfirst / W) >= h0 ? 0 : 1;
+    if (!dbg_check(wfirst >= 0 && wlast < W, a.status)) return;
 #pragma unroll 1
     for (int g = 0; g < G; ++g) {
       auto part = [&](int k) -> const float* {
@@ -1335,11 +1433,13 @@ struct Decoder {
     return __all_sync(kFull, ok);
   }
 
-  // After a timeout: wait (bounded by max(timeout, 1 s)) until the halves in flight have landed.
+  // After a timeout: wait, each for at most the same limit, until the halves in flight have landed,
+  // so that the warp does not exit with bulk copies still writing its shared memory.  A copy that
+  // truly never lands outlives the wait; the warp's buffers are then undefined, and so is the
+  // output (the status word holds KIVI_ERR_DEVICE_TIMEOUT).
   __device__ void drain_from(int h, int nhalves) {
-    const unsigned long long lim = a.timeout_ns > 1000000000ull ? a.timeout_ns : 1000000000ull;
     for (int x = h; x < h + kBuffers && x < nhalves; ++x)
-      (void)mbar_wait_bounded(&S.bar[x % kBuffers], (x / kBuffers) & 1, lim);
+      (void)mbar_wait_bounded(&S.bar[x % kBuffers], (x / kBuffers) & 1, a.timeout_ns);
     __syncwarp();
   }
 
@@ -1356,11 +1456,12 @@ struct Decoder {
       for (int b = 0; b < kBuffers; ++b) mbar_init(&S.bar[b], 1);
       asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
-    if constexpr (kMma) {  // slot 3 of every limb row stays zero; slots 0..2 are written before use
+    if constexpr (kMma) {  // FG: slot 3 of every limb row stays zero; the other paths write every word
       for (int i = lane; i < static_cast<int>(sizeof(S.qw) / 4); i += 32) {
         reinterpret_cast<uint32_t*>(S.qw)[i] = 0u;
         reinterpret_cast<uint32_t*>(S.pw)[i] = 0u;
       }
+      if (lane == 0) S.zero4 = make_uint4(0u, 0u, 0u, 0u);
     }
     __syncwarp();
     const int nhalves = static_cast<int>(2 * (ue - ub));
@@ -1525,6 +1626,8 @@ cudaError_t launch_for(const DecodeArgs& a, const DecodePlan& plan, cudaStream_t
     }                                                                    \
     return cudaErrorInvalidValue;                                        \
   } while (0)
+
+cudaError_t debug_status_decode(int32_t* out) { return take_debug_status_tu(out); }
 
 cudaError_t decode_plan(int bits, int gqa, int fine, DecodePlan* plan) {
   KIVI_DISPATCH(bits, gqa, plan_for, plan, fine);

@@ -110,4 +110,9 @@ struct DecodePlan {
 cudaError_t decode_plan(int bits, int gqa, int fine, DecodePlan* plan);
 cudaError_t launch_decode(const DecodeArgs& a, int bits, const DecodePlan& plan, cudaStream_t stream);
 
+// Debug build: read and clear the device-side check word of the quantize and the decode kernels
+// (always 0 in a release build).
+cudaError_t debug_status_quantize(int32_t* out);
+cudaError_t debug_status_decode(int32_t* out);
+
 }  // namespace kivi

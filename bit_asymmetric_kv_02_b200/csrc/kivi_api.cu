@@ -22,6 +22,7 @@ struct DebugState {
   int mode = 0;
   unsigned long long timeout_ns = kDefaultTimeoutNs;
   long long max_workers = 0;  // 0: no cap
+  int units_q_skew = 0;       // debug build: decode sees this many quantized units more than n_quant holds
 };
 DebugState& debug_state() {
   static DebugState s;
@@ -404,6 +405,17 @@ int decode_impl(const kivi_config* cfg, const kivi_cache* cache, const uint16_t*
     std::lock_guard<std::mutex> lock(d.mu);
     a.timeout_ns = d.timeout_ns;
     a.debug_extra_tx = d.mode == 1 ? 16u : 0u;
+#ifdef KIVI_DEBUG
+    // test hook of the debug build: units the kernel's bounds checks must refuse.  The extra units
+    // lie inside the capacity (checked here), so even an unguarded copy would stay in bounds.
+    if (d.units_q_skew > 0 && !coded_res && !cfg->fine_groups &&
+        static_cast<long long>(a.units_q + d.units_q_skew) * plan.unit_tokens <= cfg->capacity) {
+      a.units_q += d.units_q_skew;
+      a.units += d.units_q_skew;
+      a.total_units = static_cast<long long>(bh) * a.units;
+      if (a.workers > a.total_units) a.workers = static_cast<int>(a.total_units);
+    }
+#endif
   }
   a.k_new = k_new_dev;
   a.v_new = v_new_dev;
@@ -474,6 +486,7 @@ int kivi_debug_inject(int32_t mode, uint64_t value) {
       d.mode = 0;
       d.timeout_ns = kDefaultTimeoutNs;
       d.max_workers = 0;
+      d.units_q_skew = 0;
       return KIVI_OK;
     case 1:
       d.mode = 1;
@@ -482,9 +495,28 @@ int kivi_debug_inject(int32_t mode, uint64_t value) {
     case 2:
       d.max_workers = static_cast<long long>(value);
       return KIVI_OK;
+    case 3:
+#ifdef KIVI_DEBUG
+      d.units_q_skew = static_cast<int>(value > 8 ? 8 : value);
+      return KIVI_OK;
+#else
+      return KIVI_ERR_UNSUPPORTED;
+#endif
     default:
       return KIVI_ERR_INVALID_ARG;
   }
+}
+
+int kivi_debug_status(void) {
+#ifdef KIVI_DEBUG
+  if (cudaDeviceSynchronize() != cudaSuccess) return KIVI_ERR_CUDA;
+  int32_t q = 0, d = 0;
+  if (kivi::debug_status_quantize(&q) != cudaSuccess || kivi::debug_status_decode(&d) != cudaSuccess)
+    return KIVI_ERR_CUDA;
+  return q != 0 ? q : d;
+#else
+  return KIVI_ERR_UNSUPPORTED;
+#endif
 }
 
 }  // extern "C"

@@ -238,8 +238,15 @@ __device__ void quantize_v_block(const uint16_t* __restrict__ src, int R, int gv
   }
 }
 
+// Debug build: the job's source tokens and destination block lie inside their arrays.
+__device__ __forceinline__ bool job_in_bounds(const QuantizeArgs& a, int blk) {
+  return dbg_check(blk >= 0 && a.dst_blk0 + blk < a.capacity / a.residual &&
+                   a.src_tok0 + static_cast<long long>(blk + 1) * a.residual <= a.src_tokens);
+}
+
 // Residual copy: tokens [res_tok0, res_tok0 + res_tokens) of the source -> residual slots 0..
 __device__ void copy_residual(const QuantizeArgs& a, int bh) {
+  if (!dbg_check(a.res_tok0 + a.res_tokens <= a.src_tokens && a.res_tokens <= a.residual)) return;
   const size_t src_tok = static_cast<size_t>(bh) * a.src_tokens + a.res_tok0;
   const uint4* ks = reinterpret_cast<const uint4*>(a.k_src + src_tok * kHeadDim);
   const uint4* vs = reinterpret_cast<const uint4*>(a.v_src + src_tok * kHeadDim);
@@ -518,6 +525,7 @@ __global__ void __launch_bounds__(1024) quantize_tiles_kernel(QuantizeArgs a) {
     const int blk = job >> 1;
     const bool is_v = job & 1;
     if (a.v_only && !is_v) return;
+    if (!job_in_bounds(a, blk)) return;
     const size_t src_tok = static_cast<size_t>(bh) * a.src_tokens + a.src_tok0 + static_cast<size_t>(blk) * R;
     const int dst_blk = a.dst_blk0 + blk;
     const size_t dst_tok = static_cast<size_t>(dst_blk) * R;
@@ -550,6 +558,7 @@ __global__ void __launch_bounds__(kThreads) quantize_blocks_kernel(QuantizeArgs 
     const int blk = job >> 1;
     const bool is_v = job & 1;
     if (a.v_only && !is_v) return;
+    if (!job_in_bounds(a, blk)) return;
     const size_t src_tok = static_cast<size_t>(bh) * a.src_tokens + a.src_tok0 + static_cast<size_t>(blk) * R;
     const int dst_blk = a.dst_blk0 + blk;
     const size_t dst_tok = static_cast<size_t>(dst_blk) * R;
@@ -575,6 +584,7 @@ __global__ void __launch_bounds__(256) append_kernel(AppendArgs a) {
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   const int n = a.bh * kChunks;
   if (i >= n) return;
+  if (!dbg_check(a.slot >= 0 && a.slot < a.residual)) return;
   const int bh = i / kChunks, c = i % kChunks;
   const size_t dst = (static_cast<size_t>(bh) * a.residual + a.slot) * kChunks + c;
   reinterpret_cast<uint4*>(a.k_res)[dst] = __ldg(reinterpret_cast<const uint4*>(a.k_new) + i);
@@ -613,6 +623,7 @@ __global__ void __launch_bounds__(kHeadDim) quantize_fine_kernel(QuantizeArgs a)
   const int blk = job >> 1;
   const bool is_v = job & 1;
   if (a.v_only && !is_v) return;
+  if (!job_in_bounds(a, blk)) return;
   const size_t src_tok = static_cast<size_t>(bh) * a.src_tokens + a.src_tok0 + static_cast<size_t>(blk) * R;
   const size_t dst_tok = static_cast<size_t>(a.dst_blk0 + blk) * R;
   const unsigned word_mask = (P == 32 ? 0xffffffffu : ((1u << P) - 1u)) << ((c & 31) & ~(P - 1));
@@ -727,6 +738,10 @@ __global__ void __launch_bounds__(kHeadDim) code_k_online_kernel(OnlineKArgs a) 
   const int lg_gk = __ffs(a.group_k) - 1, ngk = kHeadDim >> lg_gk;
   const size_t C = static_cast<size_t>(a.capacity), nblk = C / static_cast<size_t>(a.residual);
   const size_t sb = (static_cast<size_t>(bh) * nblk + a.blk_src) * ngk;
+  if (!dbg_check(a.blk_src >= 0 && a.blk_src + (a.copy_scales ? 1 : 0) < static_cast<long long>(nblk) &&
+                 a.dst_row0 + row < a.capacity && a.src_tok0 + row < a.src_tokens &&
+                 (a.v_new == nullptr || (a.v_slot >= 0 && a.v_slot < a.residual))))
+    return;
   const uint16_t xb = __ldg(a.k_src + (static_cast<size_t>(bh) * a.src_tokens + a.src_tok0 + row) * kHeadDim + c);
   const double s = static_cast<double>(h2f(__ldg(a.k_scale + sb + (c >> lg_gk))));
   const double z = static_cast<double>(h2f(__ldg(a.k_zero + sb + (c >> lg_gk))));
@@ -756,6 +771,9 @@ __global__ void __launch_bounds__(kThreads) k_prefix_extremes_kernel(QuantizeArg
   __shared__ uint32_t sz;
   const int bh = blockIdx.x, g = blockIdx.y, tid = threadIdx.x;
   const int lg_cpg = a.lg_gk - 3, cpg = 1 << lg_cpg;  // 16-byte chunks per group
+  if (!dbg_check(a.dst_blk0 + a.nblocks <= a.capacity / a.residual &&
+                 a.src_tok0 + static_cast<long long>(a.nblocks) * a.residual <= a.src_tokens))
+    return;
   const long long ntok = static_cast<long long>(a.nblocks) * a.residual;
   const uint4* src = reinterpret_cast<const uint4*>(a.k_src + (static_cast<size_t>(bh) * a.src_tokens + a.src_tok0) *
                                                                   kHeadDim) + g * cpg;
@@ -793,6 +811,8 @@ __global__ void __launch_bounds__(kThreads) k_prefix_extremes_kernel(QuantizeArg
 }
 
 }  // namespace
+
+cudaError_t debug_status_quantize(int32_t* out) { return take_debug_status_tu(out); }
 
 cudaError_t launch_quantize_blocks(const QuantizeArgs& args, int bits, cudaStream_t stream) {
   const int jobs = 2 * args.nblocks + (args.res_tokens > 0 ? 1 : 0);

@@ -12,7 +12,10 @@ import math
 import os
 
 PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(PKG, "libkivi.so")
+# KIVI_LIB=debug selects the debug build (libkivi_debug.so: device-side bounds checks); any other
+# value is taken as the path of the library to load.
+LIB_PATH = {"": os.path.join(PKG, "libkivi.so"), "debug": os.path.join(PKG, "libkivi_debug.so")}.get(
+    os.environ.get("KIVI_LIB", ""), os.environ.get("KIVI_LIB", ""))
 
 KIVI_OK = 0
 STATUS_NAMES = {
@@ -72,6 +75,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "kivi_decode_attention_noalloc": (I32, [cfgp, cachep, P, I32, ctypes.c_float, P, P, P]),
         "kivi_read_status": (I32, [P, P]),
         "kivi_debug_inject": (I32, [I32, U64]),
+        "kivi_debug_status": (I32, []),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -159,6 +163,11 @@ def kivi_read_status(status_ptr: int, stream: int) -> int:
 
 def kivi_debug_inject(mode: int, value: int = 0) -> None:
     _check(load_library().kivi_debug_inject(mode, value), "kivi_debug_inject")
+
+
+def kivi_debug_status() -> int:
+    """The first device-side check failure of the debug build since the last call (0: none)."""
+    return load_library().kivi_debug_status()
 
 
 # ---- torch-owned cache --------------------------------------------------------------------------

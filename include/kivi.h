@@ -254,6 +254,18 @@ const char* kivi_strerror(int status);
 int kivi_abi_version(void);
 
 /*
+ * Debug build (nvcc -DKIVI_DEBUG, e.g. python -m bit_asymmetric_kv_02_b200.build --debug, which
+ * writes libkivi_debug.so; no counterpart on the page).  Every kernel checks the index ranges of its
+ * global-memory accesses (copy sources inside the head's arrays and filled tokens, scale indices,
+ * destination blocks, residual slots, partial and ticket slots) and, instead of making an access
+ * that fails its check, records KIVI_ERR_INTERNAL (in dev_status too, when given) and skips it; no
+ * kernel traps.  kivi_debug_status() synchronizes the device and returns the first such status
+ * since the previous call (KIVI_OK if none), then clears it.  A release build returns
+ * KIVI_ERR_UNSUPPORTED.
+ */
+int kivi_debug_status(void);
+
+/*
  * Test hooks (no counterpart on the page); process-wide, not for production use.
  *   mode 0: restore normal operation.
  *   mode 1: every later kivi_decode_attention makes its bulk-copy barriers expect 16 bytes more
@@ -262,6 +274,9 @@ int kivi_abi_version(void);
  *           output is then undefined).
  *   mode 2: cap the number of decode workers (warps) at `value` (0: no cap), to exercise the
  *           split-and-merge path with chosen splits.
+ *   mode 3: debug build only (KIVI_ERR_UNSUPPORTED otherwise): later decode launches see `value`
+ *           (at most 8) quantized units more than n_quant holds, when they still fit the capacity,
+ *           so that the kernel's bounds checks refuse those units and report KIVI_ERR_INTERNAL.
  */
 int kivi_debug_inject(int32_t mode, uint64_t value);
 

@@ -184,3 +184,19 @@ def test_binding_fails_loudly_without_library(tmp_path):
             k.load_library(str(tmp_path / "missing.so"))
     finally:
         k._lib = saved
+
+
+def test_debug_entry_points_of_the_release_build(kivi):
+    """kivi_debug_status and test hook 3 belong to the debug build; the release build refuses them
+    on the host (no device call)."""
+    assert kivi.load_library().kivi_debug_status() == 2          # KIVI_ERR_UNSUPPORTED
+    assert kivi.load_library().kivi_debug_inject(3, 1) == 2
+    assert kivi.load_library().kivi_debug_inject(0, 0) == 0
+
+
+def test_debug_build_exports_the_same_symbols():
+    from bit_asymmetric_kv_02_b200 import build
+    path = build.build(debug=True)
+    lib = ctypes.CDLL(path)
+    for n in declared_functions():
+        assert hasattr(lib, n), n
