@@ -47,9 +47,10 @@ ONLINE_K = False   # --online-k: K rows coded at append with the newest block's 
 FINE = False       # --fine-groups: K (s, z) per channel per G tokens, V per token per G channels
 DECODE_SOURCES = ["decode.cu", "common.cuh", "kernels.h"]
 CLOCK_WINDOW_S = 1.0   # the clock record spans at least this much wall time around the timed steps
-# The KIVI page's own end-to-end figures (section 実験結果, results table): context only, not a target.
+# The KIVI page's own end-to-end figures (section 実験結果（Results）: its Table 1 and throughput figures):
+# context only, not a target.
 PUBLISHED = {
-    "source": "KIVI explainer page, results table (arXiv 2402.02750)",
+    "source": "KIVI explainer page, section 実験結果（Results） (arXiv 2402.02750)",
     "hardware": "not stated",
     "peak_memory_reduction_vs_fp16": "2.6x (Llama-2-7B-chat, 2-bit KIVI)",
     "throughput_vs_fp16": {"Llama-2-7B": "2.35x", "Llama-2-70B": "3.47x"},
@@ -605,7 +606,7 @@ def oracle_parity(w: synth.Workload, state: dict, n_heads: int):
     sched = state["schedule"]
     got = state["out"].astype(np.float64)
     scale = 1.0 / math.sqrt(w.head_dim)
-    ea = er = 0.0
+    ea = er = raw = 0.0
     t0 = time.perf_counter()
     for (b, h) in sorted(heads):
         hc, n_quant0 = _oracle_head(w, b, h)
@@ -616,10 +617,15 @@ def oracle_parity(w: synth.Workload, state: dict, n_heads: int):
         q = np.stack([synth.query(w, b, h * w.gqa + g, sched[-1]) for g in range(w.gqa)])
         want = hc.attend(q, scale)
         err = np.abs(got[b, h * w.gqa:(h + 1) * w.gqa] - want)
-        ea = max(ea, float(err.max()))
+        # half the fp16 spacing at |o*|: what a correctly rounded fp16 output may differ by
+        half_ulp = np.exp2(np.floor(np.log2(np.maximum(np.abs(want), 2.0 ** -14))) - 11)
+        raw = max(raw, float(err.max()))
+        ea = max(ea, float(np.maximum(err - half_ulp, 0.0).max()))
         er = max(er, float((err / np.maximum(np.abs(want), 1e-2)).max()))
-    return {"heads": len(heads), "steps_replayed": len(sched), "max_abs": ea, "max_rel": er,
-            "ok": bool(ea <= 2e-3 and er <= 1e-2), "tolerance": "max-abs 2e-3 and max-rel 1e-2 vs the fp64 oracle",
+    return {"heads": len(heads), "steps_replayed": len(sched), "max_abs": ea, "max_rel": er, "max_abs_raw": raw,
+            "ok": bool(ea <= 2e-3 and er <= 1e-2),
+            "tolerance": ("vs the fp64 oracle: max-abs 2e-3 beyond the fp16 output's own rounding (half an fp16 ulp "
+                          "of o*) and max-rel 1e-2 (floor 1e-2)"),
             "seconds": round(time.perf_counter() - t0, 1)}
 
 
