@@ -55,9 +55,10 @@ namespace {
 // pipe idle more often).  The warps of one CTA are scheduled fairly;
 // warps of separate CTAs on one SM are not (the oldest CTA's warps take precedence and finish
 // early, leaving the SM with fewer warps for the rest of the launch).
-template <int G>
+template <int G, bool FG = false>
 __host__ __device__ constexpr int warps_per_cta() {
-  return G == 1 ? 16 : (G <= 4 ? 12 : 8);  // 128, 168 and 255 registers
+  // fine-grained groups keep P operands per (query, V channel group) and more per-query state
+  return FG ? (G == 1 ? 16 : (G == 2 ? 12 : (G == 4 ? 8 : 6))) : (G == 1 ? 16 : (G <= 4 ? 12 : 8));
 }
 constexpr int kHalfBytes = 4096;    // one half unit: the K part or the V part of a unit
 // The tensor-core path lands a V half as four 1 KB pieces (two V word rows each) 1040 bytes apart,
@@ -89,13 +90,14 @@ constexpr float kQRangeRaw = 8388544.f;  // 2^23 - 64
 // path, which keeps a fourth, all-zero limb slot (the B operand columns of no limb read it).
 constexpr int kLimbVecs = 32;
 
-// FG (fine-grained groups): qw holds the Q limbs of each K token group of a unit and pw the P limbs
-// of each V channel group (up to 4 each); oscr turns the output into the residual layout.
+// FG (fine-grained groups): qw holds the Q limbs of each K token group of a unit (for the query in
+// hand) and pw the P limbs of each (query, V channel group) (4 groups per query); oscr turns the
+// output into the residual layout.
 template <int G, bool FG = false>
 struct __align__(16) WarpSmem {
   uint8_t buf[ring_buffers<G>()][buf_bytes<G>()];
-  uint4 qw[FG ? 4 : G][kLimbVecs];  // Q operand digits of each query (FG: limbs of each K token group)
-  uint4 pw[FG ? 4 : G][kLimbVecs];  // P operand digits of each query (FG: limbs of each V channel group)
+  uint4 qw[FG ? 4 : G][kLimbVecs];      // Q operand digits of each query (FG: limbs of each K token group)
+  uint4 pw[FG ? 4 * G : G][kLimbVecs];  // P operand digits of each query (FG: limbs per query and V channel group)
   uint4 zero4;                      // the all-zero B operand of the other tile of a pair
   float oscr[FG ? kHeadDim : 4];
   uint64_t bar[ring_buffers<G>()];
@@ -257,7 +259,7 @@ struct Decoder {
   // two token (channel) tiles per accumulator, several queries pair two queries per accumulator
   static constexpr bool kMma = BITS == 2;
   static constexpr bool kMma1 = kMma && G == 1;
-  static constexpr bool kMmaG = kMma && G > 1;
+  static constexpr bool kMmaG = kMma && G > 1 && !FG;
   static constexpr int NBLK = G / 2;  // several queries: n8 blocks of queries (2 p, 2 p + 1)
 
   const DecodeArgs& a;
@@ -280,9 +282,10 @@ struct Decoder {
   float alpha_[G], invv_[G], pres_[G];
   bool hasv_[G];
   bool omma_;  // o is in the tensor-core layout of several queries (see o_swap_layout)
-  // FG: per K token group of the unit, 1 / Q scale and the z constant; per V channel group, the
-  // lane's part of sum_t p_t z_(t, group); o in the FG layout while quantized units run
-  float invqf[4], cblkf[4], ZF[4];
+  // FG: per K token group of the unit, 1 / Q scale and the z constant (of the query in hand); per
+  // query and V channel group, the lane's part of sum_t p_t z_(t, group) and (4 bits) 1 / P scale;
+  // at 2 bits o is in the FG layout while quantized units run
+  float invqf[4], cblkf[4], ZF[FG ? G : 1][4], invvf[FG && BITS == 4 ? G : 1][4];
   bool ofg_;
   // bytes per head of the code arrays and of a residual array; this lane's scale role
   const size_t code_head_bytes, res_head_bytes;
@@ -402,7 +405,9 @@ struct Decoder {
     omma_ = kMmaG;  // o is zero: either layout
     ofg_ = FG;
 #pragma unroll
-    for (int gc = 0; gc < 4; ++gc) ZF[gc] = 0.f;
+    for (int g = 0; g < (FG ? G : 1); ++g)
+#pragma unroll
+      for (int gc = 0; gc < 4; ++gc) ZF[g][gc] = 0.f;
     __syncwarp();
   }
 
@@ -641,39 +646,49 @@ struct Decoder {
     }
   }
 
-  // ---- fine-grained groups (FG: 2 bits, one query per KV head) ----------------------------------
+  // ---- fine-grained groups (FG) -----------------------------------------------------------------
   // Section KVキャッシュの分布特性: the K range is taken along each channel (one (s, z) per channel per
   // g_k tokens: k_scale [bh][C / g_k][128]) and the V range along each token (one (s, z) per token per
   // g_v channels: v_scale [bh][C][128 / g_v]).  K: the Q limbs q_c s_(u, c) and the constant
-  // sum_c q_c z_(u, c) are formed for each token group u of the unit (tile pair j uses group
-  // 32 j / g_k).  V: P_(t, gc) = p_t s_(t, gc) per channel group gc, one limb array per group; tile pair
-  // v holds channels 32 v .. 32 v + 31 (group 32 v / g_v) with tile (v, b) row g' + 8 c on channel
-  // 32 v + 16 b + 2 g' + c, so after the exchange lane (g, t) holds channel 32 v + 16 (t / 2) + 2 g +
-  // t % 2 in o[0][v].  sum_t p_t z_(t, gc) stays per group (ZF) until fg_to_residual_layout() adds it.
+  // sum_c q_c z_(u, c) are formed for each token group u of the unit.  V: P_(t, gc) = p_t s_(t, gc)
+  // per channel group gc, one limb array per (query, group); sum_t p_t z_(t, gc) stays per group (ZF)
+  // until fg_to_residual_layout() adds it to the group's channels.  Queries are taken one at a time:
+  // each pass over a unit's codes serves one query.
+  //
+  // 2 bits (tensor cores, three limbs): tile pair j of the K side holds tokens 32 j .. 32 j + 31 (one
+  // token group, g_k >= 32).  On the V side tile pair v holds channels 32 v .. 32 v + 31 (group
+  // 32 v / g_v) with tile (v, b) row g' + 8 c on channel 32 v + 16 b + 2 g' + c, so after the exchange
+  // lane (g, t) holds channel 32 v + 16 (t / 2) + 2 g + t % 2 in o[q][v].
+  // 4 bits (dp4a): lane holds tokens lane + 32 j (j = 0, 1: token groups j when g_k = 32, else one)
+  // and channels 4 lane .. 4 lane + 3 (one channel group) of the output.
 
   static __device__ __forceinline__ float sel4(const float (&x)[4], int i) {
     return i == 0 ? x[0] : (i == 1 ? x[1] : (i == 2 ? x[2] : x[3]));
   }
 
-  __device__ void fg_k(const uint8_t* kt, long long head, int local) {
+  // K (s, z) index of channel c in token group u of the head (FG layout), bounds-checked in a debug build.
+  __device__ __forceinline__ size_t fg_kidx(long long head, size_t u, int c) const {
+    const size_t rows = static_cast<size_t>(a.capacity) >> a.lg_gk;
+    const size_t i = (static_cast<size_t>(head) * rows + u) * kHeadDim + c;
+    return dbg_check(i < static_cast<size_t>(a.bh) * rows * kHeadDim, a.status) ? i : 0;
+  }
+
+  __device__ void fg_k(int gq, const uint8_t* kt, long long head, int local) {
     const int ngt = UT >> a.lg_gk;  // K token groups in the unit: 4, 2 or 1
-    const size_t row0 = (static_cast<size_t>(head) * (static_cast<size_t>(a.capacity) >> a.lg_gk) +
-                         ((static_cast<size_t>(local) * UT) >> a.lg_gk)) * kHeadDim;
+    const size_t u0 = (static_cast<size_t>(local) * UT) >> a.lg_gk;
     const int i = lane >> 2, kk = lane & 3, sw = (i >> 1) & 3;
-    __syncwarp();  // the previous unit's limbs are no longer read
+    __syncwarp();  // the previous pass's limbs are no longer read
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
       if (u < ngt) {
         float qv[4], qz = 0.f;
 #pragma unroll
         for (int m = 0; m < 4; ++m) {
-          size_t ci = row0 + static_cast<size_t>(u) * kHeadDim + 16 * i + 4 * m + kk;
-          if (!dbg_check(ci < static_cast<size_t>(a.bh) * (static_cast<size_t>(a.capacity) >> a.lg_gk) * kHeadDim,
-                         a.status))
-            ci = 0;
+          const size_t ci = fg_kidx(head, u0 + u, 16 * i + 4 * m + kk);
           const float sk = h2f(__ldg(a.k_scale + ci)), zk = h2f(__ldg(a.k_zero + ci));
-          qv[m] = q_of(0, m) * sk;
-          qz = fmaf(q_of(0, m), zk, qz);
+          const float qm = q_of(gq, m);
+          qv[m] = qm * sk;
+          qz = fmaf(qm, zk, qz);
         }
         const float mabs = warp_max(fmaxf(fmaxf(fabsf(qv[0]), fabsf(qv[1])), fmaxf(fabsf(qv[2]), fabsf(qv[3]))));
         const float scq = mabs > 0.f ? kQRangeBal * fast_rcp(mabs) : 0.f;
@@ -719,12 +734,12 @@ struct Decoder {
       }
       lg[j] = fmaf(gather_limbs(c, odd), sel4(invqf, u), sel4(cblkf, u));
     }
-    softmax_fg(head, local, lg);
+    softmax_fg(gq, head, local, lg);
   }
 
-  // Online softmax of the unit and the P limbs of each V channel group.  The lane's token
-  // 32 j + 16 (t / 2) + 8 (t % 2) + g has one (s, z) per channel group.
-  __device__ void softmax_fg(long long head, int local, const float (&lg)[4]) {
+  // Online softmax of query gq over the unit and its P limbs for each V channel group.  The lane's
+  // token 32 j + 16 (t / 2) + 8 (t % 2) + g has one (s, z) per channel group.
+  __device__ void softmax_fg(int gq, long long head, int local, const float (&lg)[4]) {
     const int g = lane >> 2, t = lane & 3;
     const int ngv = kHeadDim >> a.lg_gv;
     float sv[4][4], zv[4][4], smax_l = 0.f;
@@ -732,8 +747,8 @@ struct Decoder {
     for (int j = 0; j < 4; ++j) {
       const size_t tok = static_cast<size_t>(head) * a.capacity + static_cast<size_t>(local) * UT + 32 * j +
                          16 * (t >> 1) + 8 * (t & 1) + g;
-#pragma unroll
       const bool in = dbg_check(tok < static_cast<size_t>(a.bh) * a.capacity, a.status);
+#pragma unroll
       for (int gc = 0; gc < 4; ++gc) {
         sv[j][gc] = gc < ngv && in ? h2f(__ldg(a.v_scale + tok * ngv + gc)) : 0.f;
         zv[j][gc] = gc < ngv && in ? h2f(__ldg(a.v_zero + tok * ngv + gc)) : 0.f;
@@ -742,8 +757,8 @@ struct Decoder {
     }
     const float mu = warp_max(fmaxf(fmaxf(lg[0], lg[1]), fmaxf(lg[2], lg[3])));
     const float smax = warp_max(smax_l);
-    const float m_new = fmaxf(m[0], mu);
-    const float alpha = fast_exp2(m[0] - m_new);
+    const float m_new = fmaxf(m[gq], mu);
+    const float alpha = fast_exp2(m[gq] - m_new);
     const float d = mu - m_new;
     const bool hv = d > -64.f && smax > 0.f;
     const float fb = hv ? (kPRange * fast_rcp(smax)) * fast_exp2(-d) * ((g & 1) ? 0.25f : 1.f) : 0.f;
@@ -758,24 +773,24 @@ struct Decoder {
         if (gc < ngv) {
           zl[gc] = fmaf(p, zv[j][gc], zl[gc]);
           const uint32_t P = __float2uint_rn(p * (sv[j][gc] * fb));
-          uint8_t* pb = reinterpret_cast<uint8_t*>(S.pw[gc]) + boff + 128 * j;
+          uint8_t* pb = reinterpret_cast<uint8_t*>(S.pw[4 * gq + gc]) + boff + 128 * j;
           pb[16 * (0 ^ j)] = static_cast<uint8_t>(P >> 16);
           pb[16 * (1 ^ j)] = static_cast<uint8_t>(P >> 8);
           pb[16 * (2 ^ j)] = static_cast<uint8_t>(P);
         }
       }
     }
-    m[0] = m_new;
-    l[0] = fmaf(l[0], alpha, psum);
-    Z[0] *= alpha;
+    m[gq] = m_new;
+    l[gq] = fmaf(l[gq], alpha, psum);
+    Z[gq] *= alpha;
 #pragma unroll
-    for (int gc = 0; gc < 4; ++gc) ZF[gc] = fmaf(ZF[gc], alpha, zl[gc]);
-    alpha_[0] = alpha;
-    hasv_[0] = hv;
-    invv_[0] = hv ? fast_exp2(d) * smax * (1.0f / kPRange) : 0.f;
+    for (int gc = 0; gc < 4; ++gc) ZF[gq][gc] = fmaf(ZF[gq][gc], alpha, zl[gc]);
+    alpha_[gq] = alpha;
+    hasv_[gq] = hv;
+    invv_[gq] = hv ? fast_exp2(d) * smax * (1.0f / kPRange) : 0.f;
   }
 
-  __device__ void v_mma_fg(const uint8_t* vt) {
+  __device__ void v_mma_fg(int gq, const uint8_t* vt) {
     const int g = lane >> 2, t = lane & 3;
     const int se = g < 4 ? g : 3, so = g >= 4 ? g - 4 : 3;
     const bool odd = t & 1;
@@ -785,7 +800,7 @@ struct Decoder {
       int cv[4] = {0, 0, 0, 0};
 #pragma unroll
       for (int x = 0; x < 2; ++x) {
-        const uint4 be = S.pw[gc][8 * t + 4 * x + (se ^ t)], bo = S.pw[gc][8 * t + 4 * x + (so ^ t)];
+        const uint4 be = S.pw[4 * gq + gc][8 * t + 4 * x + (se ^ t)], bo = S.pw[4 * gq + gc][8 * t + 4 * x + (so ^ t)];
         const uint8_t* rowp = vt + t * kVPieceStride + x * 512 + 4 * (32 * v + 2 * g);
         const uint2 w0 = *reinterpret_cast<const uint2*>(rowp);           // tile (v, 0): rows g, g + 8
         const uint2 w1 = *reinterpret_cast<const uint2*>(rowp + 4 * 16);  // tile (v, 1)
@@ -799,29 +814,182 @@ struct Decoder {
         mma_u8u8(cv, mg[0], mh[0], mg[1], mh[1], bo.x, bo.y);
         mma_u8u8(cv, mg[2], mh[2], mg[3], mh[3], bo.z, bo.w);
       }
-      o[0][v] = fmaf(o[0][v], alpha_[0], gather_limbs(cv, odd) * invv_[0]);
+      o[gq][v] = fmaf(o[gq][v], alpha_[gq], gather_limbs(cv, odd) * invv_[gq]);
     }
   }
 
-  // o from the FG layout to the residual layout (lane l: channels 4 l .. 4 l + 3), with each V
-  // channel group's z term added to its channels.
+  // 4 bits: the Q limbs of query gq for the unit's token groups (S.qw[jg], layout of build_q4),
+  // then the dot products of the lane's tokens lane + 32 j against their group's limbs.
+  __device__ void fg4_k(int gq, const uint8_t* kt, long long head, int local) {
+    const int ngt = (UT >> a.lg_gk) > 0 ? (UT >> a.lg_gk) : 1;  // 2 when g_k = 32, else 1
+    const size_t u0 = (static_cast<size_t>(local) * UT) >> a.lg_gk;
+    __syncwarp();  // the previous pass's limbs are no longer read
+#pragma unroll
+    for (int jg = 0; jg < 2; ++jg) {
+      if (jg < ngt) {
+        float qv[4], qz = 0.f, mabs = 0.f;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const size_t ci = fg_kidx(head, u0 + jg, lane + 32 * j);
+          const float qj = q_of(gq, j);
+          qv[j] = qj * h2f(__ldg(a.k_scale + ci));
+          qz = fmaf(qj, h2f(__ldg(a.k_zero + ci)), qz);
+          mabs = fmaxf(mabs, fabsf(qv[j]));
+        }
+        mabs = warp_max(mabs);
+        const float scq = mabs > 0.f ? kQRange * fast_rcp(mabs) : 0.f;
+        invqf[jg] = mabs * (1.0f / kQRange);
+        cblkf[jg] = warp_sum(qz);
+        uint8_t* qwb = reinterpret_cast<uint8_t*>(S.qw[jg]);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int ch = lane + 32 * j;
+          const int word = ch >> 3, k = ch & 1, mb = (ch >> 1) & 3;
+          const int Q = __float2int_rn(qv[j] * scq);
+          uint8_t* base = qwb + ((word * 3) * 2 + k) * 4 + mb;
+          base[0] = static_cast<uint8_t>(Q & 255);
+          base[8] = static_cast<uint8_t>((Q >> 8) & 255);
+          base[16] = static_cast<uint8_t>((Q >> 16) & 255);
+        }
+      }
+    }
+    __syncwarp();
+    int al[TPL], am[TPL], ah[TPL];
+#pragma unroll
+    for (int j = 0; j < TPL; ++j) al[j] = am[j] = ah[j] = 0;
+#pragma unroll 1
+    for (int qq = 0; qq < 4; ++qq) {
+      const int cq = (qq + (lane >> 1)) & 3;  // bank-conflict-free chunk order
+      uint4 kw[TPL];
+#pragma unroll
+      for (int j = 0; j < TPL; ++j) kw[j] = *reinterpret_cast<const uint4*>(kt + (lane + 32 * j) * 64 + 16 * cq);
+#pragma unroll
+      for (int ii = 0; ii < 4; ++ii) {
+#pragma unroll
+        for (int j = 0; j < TPL; ++j) {
+          uint32_t mk[2];
+          masks4(comp(kw[j], ii), mk);
+          const uint2* qrow = reinterpret_cast<const uint2*>(S.qw[ngt == 2 ? j : 0]) + 12 * cq + ii * 3;
+          const uint2 QL = qrow[0], QM = qrow[1], QH = qrow[2];
+          dot_set(mk[0], QL.x, QM.x, QH.x, al[j], am[j], ah[j], true);
+          dot_set(mk[1], QL.y, QM.y, QH.y, al[j], am[j], ah[j], true);
+        }
+      }
+    }
+    float lg[TPL];
+#pragma unroll
+    for (int j = 0; j < TPL; ++j) {
+      const int jg = ngt == 2 ? j : 0;
+      lg[j] = fmaf(combine_limbs(ah[j], am[j], al[j]), invqf[jg], cblkf[jg]);
+    }
+    softmax4_fg(gq, head, local, lg);
+  }
+
+  // 4 bits: online softmax of query gq and its P limbs per V channel group (layout of softmax4),
+  // each group scaled by its exact maximum.
+  __device__ void softmax4_fg(int gq, long long head, int local, const float (&lg)[TPL]) {
+    const int ngv = kHeadDim >> a.lg_gv;
+    float mu = lg[0];
+#pragma unroll
+    for (int j = 1; j < TPL; ++j) mu = fmaxf(mu, lg[j]);
+    mu = warp_max(mu);
+    const float m_new = fmaxf(m[gq], mu);
+    const float alpha = fast_exp2(m[gq] - m_new);
+    float p[TPL], psum = 0.f;
+#pragma unroll
+    for (int j = 0; j < TPL; ++j) {
+      p[j] = fast_exp2(lg[j] - m_new);
+      psum += p[j];
+    }
+#pragma unroll
+    for (int gc = 0; gc < 4; ++gc) {
+      float zl = 0.f, mv = 0.f, pp[TPL];
+      if (gc < ngv) {
+#pragma unroll
+        for (int j = 0; j < TPL; ++j) {
+          const size_t tok = static_cast<size_t>(head) * a.capacity + static_cast<size_t>(local) * UT + lane + 32 * j;
+          const bool in = dbg_check(tok < static_cast<size_t>(a.bh) * a.capacity, a.status);
+          const float sv = in ? h2f(__ldg(a.v_scale + tok * ngv + gc)) : 0.f;
+          const float zv = in ? h2f(__ldg(a.v_zero + tok * ngv + gc)) : 0.f;
+          zl = fmaf(p[j], zv, zl);
+          pp[j] = p[j] * sv;
+          mv = fmaxf(mv, pp[j]);
+        }
+      }
+      mv = warp_max(mv);  // every lane joins: the group count is warp-uniform
+      if (gc < ngv) {
+        const float scv = mv > 0.f ? kPRange * fast_rcp(mv) : 0.f;
+        invvf[gq][gc] = mv * (1.0f / kPRange);
+        uint8_t* pwb = reinterpret_cast<uint8_t*>(S.pw[4 * gq + gc]);
+#pragma unroll
+        for (int j = 0; j < TPL; ++j) {
+          const int t = lane + 32 * j;
+          const int row = t >> 3, k = t & 1, mb = (t >> 1) & 3;
+          const uint32_t Pq = __float2uint_rn(pp[j] * scv);
+          uint8_t* base = pwb + ((row * 3) * 2 + k) * 4 + mb;
+          base[0] = static_cast<uint8_t>(Pq & 255u);
+          base[8] = static_cast<uint8_t>((Pq >> 8) & 255u);
+          base[16] = static_cast<uint8_t>((Pq >> 16) & 255u);
+        }
+        ZF[gq][gc] = fmaf(ZF[gq][gc], alpha, zl);
+      }
+    }
+    m[gq] = m_new;
+    l[gq] = fmaf(l[gq], alpha, psum);
+    Z[gq] *= alpha;
+    alpha_[gq] = alpha;
+  }
+
+  // 4 bits: P . codes of query gq; the lane's channels 4 lane .. 4 lane + 3 lie in one V channel group.
+  __device__ void fg4_v(int gq, const uint8_t* vt) {
+    const int gcl = (4 * lane) >> a.lg_gv;
+    const uint2* pw2 = reinterpret_cast<const uint2*>(S.pw[4 * gq + gcl]);
+    int vl[4], vm[4], vh[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) vl[e] = vm[e] = vh[e] = 0;
+#pragma unroll 2
+    for (int r = 0; r < ROWS; ++r) {
+      const uint4 vw = *reinterpret_cast<const uint4*>(vt + r * 512 + 16 * lane);
+      const uint2 PL = pw2[r * 3 + 0], PM = pw2[r * 3 + 1], PH = pw2[r * 3 + 2];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        uint32_t mv4[2];
+        masks4(comp(vw, e), mv4);
+        dot_set(mv4[0], PL.x, PM.x, PH.x, vl[e], vm[e], vh[e], false);
+        dot_set(mv4[1], PL.y, PM.y, PH.y, vl[e], vm[e], vh[e], false);
+      }
+    }
+    const float iv = sel4(invvf[gq], gcl);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) o[gq][e] = fmaf(o[gq][e], alpha_[gq], combine_limbs(vh[e], vm[e], vl[e]) * iv);
+  }
+
+  // o to the residual layout (lane l: channels 4 l .. 4 l + 3; at 4 bits it is already there), with
+  // each V channel group's z term added to its channels.
   __device__ void fg_to_residual_layout() {
     const int g = lane >> 2, t = lane & 3;
-    float zs[4];
 #pragma unroll
-    for (int gc = 0; gc < 4; ++gc) zs[gc] = warp_sum(ZF[gc]);
-    __syncwarp();
+    for (int gq = 0; gq < G; ++gq) {
+      float zs[4];
 #pragma unroll
-    for (int v = 0; v < 4; ++v) S.oscr[32 * v + 16 * (t >> 1) + 2 * g + (t & 1)] = o[0][v];
-    __syncwarp();
-    const float4 ov = *reinterpret_cast<const float4*>(S.oscr + 4 * lane);
-    const float zc = sel4(zs, (4 * lane) >> a.lg_gv);
-    o[0][0] = ov.x + zc;
-    o[0][1] = ov.y + zc;
-    o[0][2] = ov.z + zc;
-    o[0][3] = ov.w + zc;
+      for (int gc = 0; gc < 4; ++gc) zs[gc] = warp_sum(ZF[gq][gc]);
+      const float zc = sel4(zs, (4 * lane) >> a.lg_gv);
+      if constexpr (BITS == 2) {
+        __syncwarp();
 #pragma unroll
-    for (int gc = 0; gc < 4; ++gc) ZF[gc] = 0.f;
+        for (int v = 0; v < 4; ++v) S.oscr[32 * v + 16 * (t >> 1) + 2 * g + (t & 1)] = o[gq][v];
+        __syncwarp();
+        const float4 ov = *reinterpret_cast<const float4*>(S.oscr + 4 * lane);
+        o[gq][0] = ov.x;
+        o[gq][1] = ov.y;
+        o[gq][2] = ov.z;
+        o[gq][3] = ov.w;
+      }
+#pragma unroll
+      for (int e = 0; e < 4; ++e) o[gq][e] += zc;
+#pragma unroll
+      for (int gc = 0; gc < 4; ++gc) ZF[gq][gc] = 0.f;
+    }
     __syncwarp();
   }
 
@@ -1046,7 +1214,13 @@ struct Decoder {
   // ---- K half of a quantized unit: logits, online softmax, P limbs (A6, A8, A9 set-up) ---------
   __device__ void quantized_k(const uint8_t* kt, long long head, int local, uint32_t pairs) {
     if constexpr (FG) {
-      fg_k(kt, head, local);
+#pragma unroll 1
+      for (int gq = 0; gq < G; ++gq) {
+        if constexpr (BITS == 2)
+          fg_k(gq, kt, head, local);
+        else
+          fg4_k(gq, kt, head, local);
+      }
       return;
     }
     const long long key = head * a.blocks_per_head + (local >> a.lg_units_per_blk);
@@ -1124,11 +1298,23 @@ struct Decoder {
   // ---- V half of a quantized unit: P . codes for every query (A9) ------------------------------
   __device__ void quantized_v(const uint8_t* vt) {
     __syncwarp();  // P limbs of every query are in shared memory
-    if (G == 1 && !hasv_[0]) {  // every weight of the unit is zero: only rescale
+    if constexpr (FG) {
+#pragma unroll 1
+      for (int gq = 0; gq < G; ++gq) {
+        if constexpr (BITS == 2) {
+          if (hasv_[gq]) {
+            v_mma_fg(gq, vt);
+          } else {  // every weight of the unit is zero for this query: only rescale
+#pragma unroll
+            for (int e = 0; e < 4; ++e) o[gq][e] *= alpha_[gq];
+          }
+        } else {
+          fg4_v(gq, vt);
+        }
+      }
+    } else if (G == 1 && !hasv_[0]) {  // every weight of the unit is zero: only rescale
 #pragma unroll
       for (int e = 0; e < 4; ++e) o[0][e] *= alpha_[0];
-    } else if constexpr (FG) {
-      v_mma_fg(vt);
     } else if constexpr (kMma1) {
       v_mma(vt);
     } else if constexpr (kMmaG) {
@@ -1457,10 +1643,8 @@ struct Decoder {
       asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     if constexpr (kMma) {  // FG: slot 3 of every limb row stays zero; the other paths write every word
-      for (int i = lane; i < static_cast<int>(sizeof(S.qw) / 4); i += 32) {
-        reinterpret_cast<uint32_t*>(S.qw)[i] = 0u;
-        reinterpret_cast<uint32_t*>(S.pw)[i] = 0u;
-      }
+      for (int i = lane; i < static_cast<int>(sizeof(S.qw) / 4); i += 32) reinterpret_cast<uint32_t*>(S.qw)[i] = 0u;
+      for (int i = lane; i < static_cast<int>(sizeof(S.pw) / 4); i += 32) reinterpret_cast<uint32_t*>(S.pw)[i] = 0u;
       if (lane == 0) S.zero4 = make_uint4(0u, 0u, 0u, 0u);
     }
     __syncwarp();
@@ -1539,12 +1723,12 @@ struct Decoder {
 };
 
 template <int BITS, int G, bool KC, bool FG = false>
-__global__ void __launch_bounds__(warps_per_cta<G>() * 32, 1) decode_kernel(const __grid_constant__ DecodeArgs a) {
+__global__ void __launch_bounds__(warps_per_cta<G, FG>() * 32, 1) decode_kernel(const __grid_constant__ DecodeArgs a) {
   extern __shared__ __align__(128) uint8_t smem_raw[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   WarpSmem<G, FG>& S = reinterpret_cast<WarpSmem<G, FG>*>(smem_raw)[warp];
   const long long W = a.workers, U = a.total_units;
-  const long long worker = static_cast<long long>(blockIdx.x) * warps_per_cta<G>() + warp;
+  const long long worker = static_cast<long long>(blockIdx.x) * warps_per_cta<G, FG>() + warp;
   if (worker >= W) return;  // the last CTA may hold fewer workers
   const long long ub = U * worker / W, ue = U * (worker + 1) / W;  // non-empty because W <= U
   Decoder<BITS, G, KC, FG> d(a, S, lane, worker, ub, ue);
@@ -1553,7 +1737,7 @@ __global__ void __launch_bounds__(warps_per_cta<G>() * 32, 1) decode_kernel(cons
 
 template <int BITS, int G, bool FG>
 cudaError_t plan_for_kernels(DecodePlan* plan) {
-  constexpr int kWarps = warps_per_cta<G>();
+  constexpr int kWarps = warps_per_cta<G, FG>();
   const int smem = kWarps * static_cast<int>(sizeof(WarpSmem<G, FG>));
   cudaError_t e = cudaFuncSetAttribute(decode_kernel<BITS, G, false, FG>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
@@ -1576,15 +1760,9 @@ cudaError_t plan_for_kernels(DecodePlan* plan) {
   return cudaSuccess;
 }
 
-// Fine-grained groups are built for 2 bits and one query per KV head.
 template <int BITS, int G>
 cudaError_t plan_for(DecodePlan* plan, int fine) {
-  if (fine) {
-    if constexpr (BITS == 2 && G == 1)
-      return plan_for_kernels<BITS, G, true>(plan);
-    else
-      return cudaErrorInvalidValue;
-  }
+  if (fine) return plan_for_kernels<BITS, G, true>(plan);
   return plan_for_kernels<BITS, G, false>(plan);
 }
 
@@ -1593,10 +1771,7 @@ cudaError_t launch_for(const DecodeArgs& a, const DecodePlan& plan, cudaStream_t
   if (a.workers < 1 || a.workers > plan.workers() || a.total_units < a.workers) return cudaErrorInvalidValue;
   const int ctas = (a.workers + plan.warps_per_cta - 1) / plan.warps_per_cta;
   if (a.fine) {
-    if constexpr (BITS == 2 && G == 1)
-      decode_kernel<BITS, G, false, true><<<ctas, plan.warps_per_cta * 32, plan.smem_bytes, stream>>>(a);
-    else
-      return cudaErrorInvalidValue;
+    decode_kernel<BITS, G, false, true><<<ctas, plan.warps_per_cta * 32, plan.smem_bytes, stream>>>(a);
   } else if (a.k_res_coded) {
     decode_kernel<BITS, G, true><<<ctas, plan.warps_per_cta * 32, plan.smem_bytes, stream>>>(a);
   } else {

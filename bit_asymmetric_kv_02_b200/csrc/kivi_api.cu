@@ -325,7 +325,7 @@ size_t kivi_decode_workspace_bytes(const kivi_config* cfg, int32_t num_q_heads) 
   const int gqa = num_q_heads / cfg->num_kv_heads;
   if (!gqa_supported(gqa)) return 0;
   DecodePlan p{};
-  if (get_plan(cfg->bits, gqa, cfg->fine_groups && cfg->bits == 2 && gqa == 1, &p) != cudaSuccess) return 0;
+  if (get_plan(cfg->bits, gqa, cfg->fine_groups, &p) != cudaSuccess) return 0;
   const size_t bh = static_cast<size_t>(cfg->batch) * cfg->num_kv_heads;
   return align256(static_cast<size_t>(p.workers()) * 2 * gqa * kivi::kPartialStride * sizeof(float)) +
          align256(bh * sizeof(int32_t));
@@ -345,7 +345,6 @@ int decode_impl(const kivi_config* cfg, const kivi_cache* cache, const uint16_t*
   if (num_q_heads < 1 || num_q_heads % cfg->num_kv_heads != 0) return KIVI_ERR_INVALID_ARG;
   const int gqa = num_q_heads / cfg->num_kv_heads;
   if (!gqa_supported(gqa)) return KIVI_ERR_UNSUPPORTED;
-  if (cfg->fine_groups && (cfg->bits != 2 || gqa != 1)) return KIVI_ERR_UNSUPPORTED;
   if (!aligned16(q_dev) || !aligned16(out_dev) || !(scale == scale) || scale > 3.0e38f || scale < -3.0e38f)
     return KIVI_ERR_INVALID_ARG;
   if (cache->n_quant + cache->n_res == 0) return KIVI_ERR_EMPTY;

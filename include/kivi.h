@@ -95,9 +95,8 @@ extern "C" {
  * group_k consecutive tokens; group_k in {32, 64, 128}, group_k <= residual) and group_v counts
  * CHANNELS (one V (s, z) per token per group_v consecutive channels; group_v in {32, 64, 128}).
  * The scale layouts change (see DEVICE LAYOUT); codes, residual, blocks and flushes do not.
- * Decode attention over such a cache is built for bits == 2 with one query head per KV head
- * (KIVI_ERR_UNSUPPORTED otherwise); it is not combined with online_k or the prefix-K prefill
- * (KIVI_ERR_UNSUPPORTED).
+ * Decode attention over such a cache works at both bit widths and every query-head ratio; it is
+ * not combined with online_k or the prefix-K prefill (KIVI_ERR_UNSUPPORTED).
  */
 typedef struct kivi_config {
   int32_t batch;        /* B */

@@ -166,10 +166,6 @@ def test_fine_groups_host_rules(kivi):
     assert sizes[4] == sizes[5] == bh * 1024 * (128 // 32) * 2      # V: [C][d/G_v]
     fake = 1 << 20
     cache = kivi.kivi_cache(*([fake] * 8), 128, 3)
-    for cfg, hq in ((_cfg(kivi, fine_groups=1, bits=4), 3), (_cfg(kivi, fine_groups=1), 6)):
-        with pytest.raises(kivi.KiviError) as e:
-            kivi.kivi_decode_attention(cfg, cache, fake, hq, 0.1, fake, fake, 1 << 30, None, 0)
-        assert e.value.code == "UNSUPPORTED"
     with pytest.raises(kivi.KiviError) as e:
         kivi.kivi_quantize_prefill_prefix_k(_cfg(kivi, fine_groups=1), cache, fake, fake, 300, 0)
     assert e.value.code == "UNSUPPORTED"

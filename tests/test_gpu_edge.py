@@ -124,7 +124,7 @@ CASES = [
 
 
 def _fine_attention_supported(bits, gqa):
-    return bits == 2 and gqa == 1
+    return True
 
 
 @pytest.mark.parametrize("family", ["full_range", "moderate"])

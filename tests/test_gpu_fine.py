@@ -3,8 +3,8 @@ each token) on the GPU, against the oracle's fine_groups mode.
 
 K codes, K (s, z) per channel per g_k tokens, V codes, V (s, z) per token per g_v channels and the
 residual must equal the oracle's bit for bit after the prefill, the appends and the flush; decode
-attention (2 bits, one query per KV head) must be within tolerance.  At 4 bits the quantization is
-checked and decode reports UNSUPPORTED.
+attention must be within tolerance at 2 and 4 bits with one to eight queries per KV head, also with
+each head split over several warps.
 """
 import numpy as np
 import pytest
@@ -37,6 +37,21 @@ CASES = [
     synth.TINY.with_(name="fine_2bit_gk32_gv128_R1024", batch=1, q_heads=1, kv_heads=1, tokens=1024 + 70,
                      group_v=128, residual=1024, seed=74),
     synth.TINY.with_(name="fine_fits_residual", batch=1, q_heads=2, kv_heads=2, tokens=90, seed=75),
+    # several queries per KV head and 4 bits
+    synth.TINY.with_(name="fine_2bit_gqa2_gk32_gv64", batch=2, q_heads=4, kv_heads=2, tokens=3 * 128 + 11, group_v=64,
+                     seed=76),
+    synth.TINY.with_(name="fine_2bit_gqa4_gk64_gv32", batch=1, q_heads=8, kv_heads=2, tokens=2 * 128 + 77, group=64,
+                     seed=77),
+    synth.TINY.with_(name="fine_2bit_gqa8_gk128", batch=1, q_heads=8, kv_heads=1, tokens=3 * 128 + 5, group=128,
+                     seed=78),
+    synth.TINY.with_(name="fine_4bit_gk32_gv32", batch=2, q_heads=2, kv_heads=2, tokens=3 * 128 + 37, bits=4, seed=79),
+    synth.TINY.with_(name="fine_4bit_gk64_gv128", batch=1, q_heads=2, kv_heads=2, tokens=2 * 128 + 9, bits=4, group=64,
+                     group_v=128, seed=80),
+    synth.TINY.with_(name="fine_4bit_gk128_gv64_gqa2", batch=1, q_heads=4, kv_heads=2, tokens=3 * 128 + 100, bits=4,
+                     group=128, group_v=64, seed=81),
+    synth.TINY.with_(name="fine_4bit_gqa4_gk32", batch=1, q_heads=8, kv_heads=2, tokens=2 * 128 + 50, bits=4, seed=82),
+    synth.TINY.with_(name="fine_4bit_gqa8_R512", batch=1, q_heads=8, kv_heads=1, tokens=512 + 300, bits=4,
+                     group_v=64, residual=512, seed=83),
 ]
 
 
@@ -106,22 +121,27 @@ def test_fine_groups_match_oracle(w):
     assert cache.read_status() == 0
 
 
-def test_fine_groups_4bit_quantize_and_unsupported_decode():
+def test_fine_groups_with_forced_splits():
+    """Fine-grained heads split over many warps (partials merged), 4 bits and 2 bits with GQA."""
     kivi = _kivi()
-    w = synth.TINY.with_(name="fine_4bit", batch=1, q_heads=1, kv_heads=2, tokens=2 * 128 + 5, bits=4, group=64,
-                         group_v=32, seed=76)
-    cap = 4 * w.residual
-    k, v = synth.prompt_kv(w, w.tokens)
-    cache = kivi.KiviCache(w.batch, w.kv_heads, cap, bits=4, group_k=64, group_v=32, residual=128,
-                           num_q_heads=w.kv_heads, fine_groups=True)
-    cache.prefill(torch.from_numpy(k).cuda(), torch.from_numpy(v).cuda())
-    ref = {}
-    for h in range(w.kv_heads):
-        hc = O.HeadCache(128, 4, 64, 32, 128, cap, fine_groups=True)
-        hc.prefill(k[0, h], v[0, h])
-        ref[(0, h)] = hc
-    _check(cache, ref, "fine 4-bit prefill")
-    q = torch.from_numpy(synth.queries(w.with_(q_heads=w.kv_heads), 0)).cuda()
-    with pytest.raises(kivi.KiviError) as e:
-        cache.attend(q)
-    assert e.value.code == "UNSUPPORTED"
+    for bits, gqa in ((4, 2), (2, 4)):
+        w = synth.TINY.with_(name=f"fine_split_{bits}_{gqa}", batch=1, q_heads=2 * gqa, kv_heads=2,
+                             tokens=5 * 128 + 31, bits=bits, seed=84 + bits)
+        cap = 6 * 128
+        k, v = synth.prompt_kv(w, w.tokens)
+        q = synth.queries(w, 0)
+        cache = kivi.KiviCache(1, 2, cap, bits=bits, num_q_heads=2 * gqa, fine_groups=True)
+        cache.prefill(torch.from_numpy(k).cuda(), torch.from_numpy(v).cuda())
+        try:
+            kivi.kivi_debug_inject(2, 7)
+            cache.status.zero_()
+            out = cache.attend(torch.from_numpy(q).cuda()).cpu().numpy()
+            assert cache.read_status() == 0
+        finally:
+            kivi.kivi_debug_inject(0, 0)
+        for h in range(2):
+            hc = O.HeadCache(128, bits, 32, 32, 128, cap, fine_groups=True)
+            hc.prefill(k[0, h], v[0, h])
+            gc.assert_attention_close(out[0, h * gqa:(h + 1) * gqa], hc.attend(q[0, h * gqa:(h + 1) * gqa],
+                                                                              gc.default_scale()),
+                                      f"fine split {bits}-bit gqa {gqa} head {h}")
