@@ -1115,7 +1115,8 @@ struct Decoder {
   }
 
   // P . codes of the unit for every query.  Tile (v, b) holds channels 16 g' + 8 b + 4 c + v (row
-  // g' + 8 c); lane (g, t) reads V word rows 2 t + x of channels 16 g .. 16 g + 15.
+  // g' + 8 c); lane (g, t) reads V word rows 2 t + x of channels 16 g .. 16 g + 15.  Per tile column b
+  // the lane's eight V words are read once and the accumulators live for one v at a time.
   __device__ void v_mma_g(const uint8_t* vt) {
     const int g = lane >> 2, t = lane & 3, qh = g >> 2, sl = (g & 3) ^ t;
     const bool odd = t & 1;
@@ -1134,33 +1135,33 @@ struct Decoder {
     }
 #pragma unroll
     for (int b = 0; b < 2; ++b) {
-      int acc[4][NBLK][4];
-#pragma unroll
-      for (int v = 0; v < 4; ++v)
-#pragma unroll
-        for (int p = 0; p < NBLK; ++p) acc[v][p][0] = acc[v][p][1] = acc[v][p][2] = acc[v][p][3] = 0;
+      uint4 wlo[2], whi[2];
 #pragma unroll
       for (int x = 0; x < 2; ++x) {
         const uint8_t* rowp = vt + t * kVPieceStride + x * 512 + 64 * g;
-        const uint4 wlo = *reinterpret_cast<const uint4*>(rowp + 32 * b);
-        const uint4 whi = *reinterpret_cast<const uint4*>(rowp + 32 * b + 16);
-#pragma unroll
-        for (int v = 0; v < 4; ++v) {
-          uint32_t vg[4], vh[4];
-          variants2(comp(wlo, v), vg);
-          variants2(comp(whi, v), vh);
-#pragma unroll
-          for (int p = 0; p < NBLK; ++p) {
-            mma_u8s8(acc[v][p], vg[0], vh[0], vg[1], vh[1], B[p][x].x, B[p][x].y);
-            mma_u8s8(acc[v][p], vg[2], vh[2], vg[3], vh[3], B[p][x].z, B[p][x].w);
-          }
-        }
+        wlo[x] = *reinterpret_cast<const uint4*>(rowp + 32 * b);
+        whi[x] = *reinterpret_cast<const uint4*>(rowp + 32 * b + 16);
       }
 #pragma unroll
-      for (int v = 0; v < 4; ++v)
+      for (int v = 0; v < 4; ++v) {
+        int acc[NBLK][4];
+#pragma unroll
+        for (int p = 0; p < NBLK; ++p) acc[p][0] = acc[p][1] = acc[p][2] = acc[p][3] = 0;
+#pragma unroll
+        for (int x = 0; x < 2; ++x) {
+          uint32_t vg[4], vh[4];
+          variants2(comp(wlo[x], v), vg);
+          variants2(comp(whi[x], v), vh);
+#pragma unroll
+          for (int p = 0; p < NBLK; ++p) {
+            mma_u8s8(acc[p], vg[0], vh[0], vg[1], vh[1], B[p][x].x, B[p][x].y);
+            mma_u8s8(acc[p], vg[2], vh[2], vg[3], vh[3], B[p][x].z, B[p][x].w);
+          }
+        }
 #pragma unroll
         for (int p = 0; p < NBLK; ++p)
-          o[2 * p + b][v] = fmaf(o[2 * p + b][v], al[p], gather4(acc[v][p], odd, sc) * iv[p]);
+          o[2 * p + b][v] = fmaf(o[2 * p + b][v], al[p], gather4(acc[p], odd, sc) * iv[p]);
+      }
     }
   }
 
