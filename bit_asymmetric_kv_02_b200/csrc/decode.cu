@@ -55,10 +55,13 @@ namespace {
 // pipe idle more often).  The warps of one CTA are scheduled fairly;
 // warps of separate CTAs on one SM are not (the oldest CTA's warps take precedence and finish
 // early, leaving the SM with fewer warps for the rest of the launch).
+#ifndef KIVI_GQA_WARPS
+#define KIVI_GQA_WARPS 12  // warps per CTA for 2 and 4 queries per KV head (base groups)
+#endif
 template <int G, bool FG = false>
 __host__ __device__ constexpr int warps_per_cta() {
   // fine-grained groups keep P operands per (query, V channel group) and more per-query state
-  return FG ? (G == 1 ? 16 : (G == 2 ? 12 : (G == 4 ? 8 : 6))) : (G == 1 ? 16 : (G <= 4 ? 12 : 8));
+  return FG ? (G == 1 ? 16 : (G == 2 ? 12 : (G == 4 ? 8 : 6))) : (G == 1 ? 16 : (G <= 4 ? KIVI_GQA_WARPS : 8));
 }
 constexpr int kHalfBytes = 4096;    // one half unit: the K part or the V part of a unit
 // The tensor-core path lands a V half as four 1 KB pieces (two V word rows each) 1040 bytes apart,
@@ -1454,7 +1457,9 @@ struct Decoder {
     for (int g = 0; g < G; ++g) {
       const uint4* qp = reinterpret_cast<const uint4*>(a.q + (static_cast<size_t>(head) * G + g) * kHeadDim);
       float dot = 0.f;
-#pragma unroll
+      // several queries: one chunk at a time, so that the loads of all queries are not in flight at
+      // once (they would hold more registers than the kernel has)
+#pragma unroll(G == 1 ? 8 : 1)
       for (int k = 0; k < 8; ++k) {
         const int cc = (k + lane) & 7;  // bank-conflict-free chunk order
         const int c0 = 64 * hf + 8 * cc;

@@ -513,6 +513,258 @@ __device__ void quantize_v_tiles(const uint16_t* __restrict__ src, int R, int lg
   }
 }
 
+// ---------------------------------------------------------------------------------------------
+// Fine-grained groups with register tiles (R <= 256; section KVキャッシュの分布特性): the tiles of
+// quantize_tiles_kernel, with one (s, z) per channel per g_k tokens for K and one per token per g_v
+// channels for V.  K: a thread reduces each of its 8 channels over its 8 tokens, the warp's two token
+// groups and then the g_k / 16 warps of the K group combine them (shared memory), and every thread
+// forms the 8 pairs of its channels.  V: a thread reduces each of its 8 tokens over its 8 channels,
+// then the g_v / 8 chunks of the channel group combine them by shuffles within the half warp.
+// Codes follow the same exact rules (2 bits: thresholds per channel or per token; 4 bits:
+// arithmetic with the fp64 re-decision near ties).
+// ---------------------------------------------------------------------------------------------
+__device__ __forceinline__ __half2 half2_of(const uint4& v, int i) {
+  const uint32_t w = comp4(v, i);
+  return *reinterpret_cast<const __half2*>(&w);
+}
+__device__ __forceinline__ uint32_t u32_of(__half2 h) { return *reinterpret_cast<const uint32_t*>(&h); }
+__device__ __forceinline__ __half2 h2_from(uint32_t u) { return *reinterpret_cast<const __half2*>(&u); }
+
+// Thresholds of two groups side by side: the low half from ga, the high half from gb.
+__device__ __forceinline__ Thresh2 thresh_pair(const GroupParams& ga, const GroupParams& gb) {
+  const Thresh2 ta = make_thresh2(ga), tb = make_thresh2(gb);
+  Thresh2 t;
+#pragma unroll
+  for (int k = 0; k < 3; ++k) t.t[k] = (ta.t[k] & 0xFFFFu) | (tb.t[k] & 0xFFFF0000u);
+  return t;
+}
+
+// Q of two elements with their own (s, z) (ga for the low half, gb for the high half).
+__device__ __forceinline__ void quantize_pair2(uint32_t hx2, const GroupParams& ga, const GroupParams& gb, int levels,
+                                               uint32_t& qa, uint32_t& qb) {
+  constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
+  const float2 x = __half22float2(*reinterpret_cast<const __half2*>(&hx2));
+  const float2 r = __fmul2_rn(__fadd2_rn(x, make_float2(-ga.zf, -gb.zf)), make_float2(ga.inv_s, gb.inv_s));
+  const float2 t = __fadd2_rn(r, make_float2(kMagic, kMagic));
+  const float2 d = __fadd2_rn(r, __fadd2_rn(make_float2(kMagic, kMagic), make_float2(-t.x, -t.y)));
+  qa = min(__float_as_uint(t.x) - 0x4B400000u, static_cast<uint32_t>(levels));
+  qb = min(__float_as_uint(t.y) - 0x4B400000u, static_cast<uint32_t>(levels));
+  if (fabsf(d.x) > 0.499755859375f) qa = quantize_exact(x.x, ga, levels);  // within 2^-12 of a tie
+  if (fabsf(d.y) > 0.499755859375f) qb = quantize_exact(x.y, gb, levels);
+  if (ga.inv_s == 0.f) qa = 0u;
+  if (gb.inv_s == 0.f) qb = 0u;
+}
+
+template <int BITS>
+__device__ void quantize_k_fine_tiles(const uint16_t* __restrict__ src, int lg_gk, uint32_t* __restrict__ codes,
+                                      uint16_t* __restrict__ scale, uint16_t* __restrict__ zero) {
+  constexpr int L = (1 << BITS) - 1;
+  __shared__ uint4 red_lo[1024 / 32][16], red_hi[1024 / 32][16];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int c = tid & 15, tg = tid >> 4;
+  const uint4* s4 = reinterpret_cast<const uint4*>(src) + (tg * kTileTokens) * kChunks + c;
+  uint4 x[kTileTokens];
+#pragma unroll
+  for (int k = 0; k < kTileTokens; ++k) x[k] = __ldg(s4 + k * kChunks);
+  // per-channel extremes over the tile's tokens, then over the warp's other token group
+  __half2 lo[4], hi[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    lo[i] = hi[i] = half2_of(x[0], i);
+#pragma unroll
+    for (int k = 1; k < kTileTokens; ++k) {
+      lo[i] = __hmin2(lo[i], half2_of(x[k], i));
+      hi[i] = __hmax2(hi[i], half2_of(x[k], i));
+    }
+    lo[i] = __hmin2(lo[i], shfl_xor_h2(lo[i], 16));
+    hi[i] = __hmax2(hi[i], shfl_xor_h2(hi[i], 16));
+  }
+  if (lane < 16) {
+    red_lo[warp][c] = make_uint4(u32_of(lo[0]), u32_of(lo[1]), u32_of(lo[2]), u32_of(lo[3]));
+    red_hi[warp][c] = make_uint4(u32_of(hi[0]), u32_of(hi[1]), u32_of(hi[2]), u32_of(hi[3]));
+  }
+  __syncthreads();
+  const int wpg = 1 << (lg_gk - 4);  // warps of one K group (g_k / 16)
+  const int w0 = warp & ~(wpg - 1);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    lo[i] = h2_from(comp4(red_lo[w0][c], i));
+    hi[i] = h2_from(comp4(red_hi[w0][c], i));
+  }
+  for (int w = 1; w < wpg; ++w) {
+    const uint4 l4 = red_lo[w0 + w][c], h4 = red_hi[w0 + w][c];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      lo[i] = __hmin2(lo[i], h2_from(comp4(l4, i)));
+      hi[i] = __hmax2(hi[i], h2_from(comp4(h4, i)));
+    }
+  }
+  GroupParams gp[8];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    gp[2 * i] = make_group(__low2float(lo[i]), __low2float(hi[i]), L);
+    gp[2 * i + 1] = make_group(__high2float(lo[i]), __high2float(hi[i]), L);
+  }
+  const int tpg = 1 << (lg_gk - 3);  // token groups (tiles) of one K group
+  if ((tg & (tpg - 1)) == 0) {       // the K group's first tile stores the pairs of its 8 channels
+    const size_t row = static_cast<size_t>(tg >> (lg_gk - 3)) * kHeadDim + 8 * c;
+    uint32_t sw[4], zw[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      sw[i] = static_cast<uint32_t>(gp[2 * i].s_bits) | (static_cast<uint32_t>(gp[2 * i + 1].s_bits) << 16);
+      zw[i] = static_cast<uint32_t>(gp[2 * i].z_bits) | (static_cast<uint32_t>(gp[2 * i + 1].z_bits) << 16);
+    }
+    *reinterpret_cast<uint4*>(scale + row) = make_uint4(sw[0], sw[1], sw[2], sw[3]);
+    *reinterpret_cast<uint4*>(zero + row) = make_uint4(zw[0], zw[1], zw[2], zw[3]);
+  }
+  const int tok0 = tg * kTileTokens;
+  if constexpr (BITS == 4) {  // K word c of a token is exactly the tile's 8 channels
+#pragma unroll
+    for (int k = 0; k < kTileTokens; ++k) {
+      const uint32_t w[4] = {x[k].x, x[k].y, x[k].z, x[k].w};
+      uint32_t r = 0;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        uint32_t qa, qb;
+        quantize_pair2(w[e], gp[2 * e], gp[2 * e + 1], L, qa, qb);
+        r += (qa << (BITS * 2 * e)) + (qb << (BITS * (2 * e + 1)));
+      }
+      codes[(tok0 + k) * (kHeadDim / 8) + c] = r;
+    }
+  } else {  // K word c / 2 of a token: chunk 2i in bits 0..15, chunk 2i + 1 in bits 16..31
+    Thresh2 tp[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) tp[i] = thresh_pair(gp[2 * i], gp[2 * i + 1]);
+    uint32_t h[kTileTokens];
+#pragma unroll
+    for (int k = 0; k < kTileTokens; ++k) {
+      const uint32_t h0 = codes2_h2(x[k].x, tp[0]), h1 = codes2_h2(x[k].y, tp[1]);
+      const uint32_t h2 = codes2_h2(x[k].z, tp[2]), h3 = codes2_h2(x[k].w, tp[3]);
+      h[k] = gather4x2(__byte_perm(h0, h1, 0x6420)) | (gather4x2(__byte_perm(h2, h3, 0x6420)) << 8);
+    }
+    const bool odd = c & 1;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {  // the even chunk stores tokens 0..3 of the tile, the odd one 4..7
+      const uint32_t other = __shfl_xor_sync(0xffffffffu, odd ? h[j] : h[4 + j], 1);
+      const int k = odd ? 4 + j : j;
+      const uint32_t word = odd ? (other | (h[4 + j] << 16)) : (h[j] | (other << 16));
+      codes[(tok0 + k) * (kHeadDim / 16) + (c >> 1)] = word;
+    }
+  }
+}
+
+template <int BITS>
+__device__ void quantize_v_fine_tiles(const uint16_t* __restrict__ src, int lg_gv, uint32_t* __restrict__ codes,
+                                      uint16_t* __restrict__ scale, uint16_t* __restrict__ zero) {
+  constexpr int L = (1 << BITS) - 1;
+  const int tid = threadIdx.x;
+  const int c = tid & 15, tg = tid >> 4;
+  const uint4* s4 = reinterpret_cast<const uint4*>(src) + (tg * kTileTokens) * kChunks + c;
+  uint4 x[kTileTokens];
+#pragma unroll
+  for (int k = 0; k < kTileTokens; ++k) x[k] = __ldg(s4 + k * kChunks);
+  // per-token extremes over the chunk's 8 channels, then over the g_v / 8 chunks of the channel
+  // group (lanes c of one half warp)
+  const int cpg = 1 << (lg_gv - 3);
+  GroupParams gp[kTileTokens];
+#pragma unroll
+  for (int k = 0; k < kTileTokens; ++k) {
+    __half2 lo = half2_of(x[k], 0), hi = lo;
+#pragma unroll
+    for (int i = 1; i < 4; ++i) {
+      lo = __hmin2(lo, half2_of(x[k], i));
+      hi = __hmax2(hi, half2_of(x[k], i));
+    }
+    __half2 m = __halves2half2(__hmin(__low2half(lo), __high2half(lo)), __hneg(__hmax(__low2half(hi), __high2half(hi))));
+    for (int off = 1; off < cpg; off <<= 1) m = __hmin2(m, shfl_xor_h2(m, off));
+    gp[k] = group_from_pair(m, L);
+  }
+  const int ngv = kHeadDim >> lg_gv, g = c >> (lg_gv - 3);
+  const int tok0 = tg * kTileTokens;
+  if ((c & (cpg - 1)) == 0) {  // the group's first chunk stores the pairs of its 8 tokens
+#pragma unroll
+    for (int k = 0; k < kTileTokens; ++k) {
+      scale[(tok0 + k) * ngv + g] = gp[k].s_bits;
+      zero[(tok0 + k) * ngv + g] = gp[k].z_bits;
+    }
+  }
+  // codes of channel 8 c + e for the tile's 8 tokens, token k at bits BITS * k
+  uint32_t col[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  if constexpr (BITS == 4) {
+#pragma unroll
+    for (int k = 0; k < kTileTokens; ++k) {
+      const uint32_t w[4] = {x[k].x, x[k].y, x[k].z, x[k].w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        uint32_t qa, qb;
+        quantize_pair(w[e], gp[k], L, qa, qb);
+        col[2 * e] += qa << (BITS * k);
+        col[2 * e + 1] += qb << (BITS * k);
+      }
+    }
+    uint4* dst = reinterpret_cast<uint4*>(codes + tg * kHeadDim + 8 * c);
+    dst[0] = make_uint4(col[0], col[1], col[2], col[3]);
+    dst[1] = make_uint4(col[4], col[5], col[6], col[7]);
+  } else {
+    Thresh2 t[kTileTokens];
+#pragma unroll
+    for (int k = 0; k < kTileTokens; ++k) t[k] = make_thresh2(gp[k]);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      uint32_t A[4];
+#pragma unroll
+      for (int a2 = 0; a2 < 4; ++a2) {
+        const uint32_t w0 = comp4(x[2 * a2], e), w1 = comp4(x[2 * a2 + 1], e);
+        A[a2] = __byte_perm(codes2_h2(w0, t[2 * a2]), codes2_h2(w1, t[2 * a2 + 1]), 0x6240);
+      }
+      col[2 * e] = gather4x2(__byte_perm(A[0], A[1], 0x5410)) | (gather4x2(__byte_perm(A[2], A[3], 0x5410)) << 8);
+      col[2 * e + 1] = gather4x2(__byte_perm(A[0], A[1], 0x7632)) | (gather4x2(__byte_perm(A[2], A[3], 0x7632)) << 8);
+    }
+    const bool odd = tg & 1;
+    uint32_t word[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {  // the even token group stores channels 0..3, the odd one 4..7
+      const uint32_t other = __shfl_xor_sync(0xffffffffu, odd ? col[e] : col[4 + e], 16);
+      word[e] = odd ? (other | (col[4 + e] << 16)) : (col[e] | (other << 16));
+    }
+    *reinterpret_cast<uint4*>(codes + (tg >> 1) * kHeadDim + 8 * c + (odd ? 4 : 0)) =
+        make_uint4(word[0], word[1], word[2], word[3]);
+  }
+}
+
+// grid: x = batch * kv_heads, y = 2 * nblocks (+1 residual-copy job); block = 2R threads (R <= 256:
+// the per-channel and per-token parameters need more than the 64 registers of a 1024-thread block)
+template <int BITS>
+__global__ void __launch_bounds__(512) quantize_fine_tiles_kernel(QuantizeArgs a) {
+  constexpr int P = 32 / BITS;
+  const int bh = blockIdx.x;
+  const int job = blockIdx.y;
+  const int R = a.residual;
+  const size_t C = static_cast<size_t>(a.capacity);
+  if (job >= 2 * a.nblocks) {
+    copy_residual(a, bh);
+    return;
+  }
+  const int blk = job >> 1;
+  const bool is_v = job & 1;
+  if (a.v_only && !is_v) return;
+  if (!job_in_bounds(a, blk)) return;
+  const size_t src_tok = static_cast<size_t>(bh) * a.src_tokens + a.src_tok0 + static_cast<size_t>(blk) * R;
+  const size_t dst_tok = static_cast<size_t>(a.dst_blk0 + blk) * R;
+  if (!is_v) {
+    const size_t srow = (static_cast<size_t>(bh) * (C >> a.lg_gk) + (dst_tok >> a.lg_gk)) * kHeadDim;
+    quantize_k_fine_tiles<BITS>(a.k_src + src_tok * kHeadDim, a.lg_gk,
+                                a.k_codes + (static_cast<size_t>(bh) * C + dst_tok) * (kHeadDim / P), a.k_scale + srow,
+                                a.k_zero + srow);
+  } else {
+    const size_t ngv = kHeadDim >> a.lg_gv;
+    const size_t srow = (static_cast<size_t>(bh) * C + dst_tok) * ngv;
+    quantize_v_fine_tiles<BITS>(a.v_src + src_tok * kHeadDim, a.lg_gv,
+                                a.v_codes + (static_cast<size_t>(bh) * (C / P) + dst_tok / P) * kHeadDim, a.v_scale + srow,
+                                a.v_zero + srow);
+  }
+}
+
 // grid: x = batch * kv_heads, y = 2 * nblocks (+1 residual-copy job); block = 2R threads (R <= 512)
 template <int BITS>
 __global__ void __launch_bounds__(1024) quantize_tiles_kernel(QuantizeArgs a) {
@@ -821,7 +1073,12 @@ cudaError_t launch_quantize_blocks(const QuantizeArgs& args, int bits, cudaStrea
   a.lg_gk = __builtin_ctz(static_cast<unsigned>(a.group_k));
   a.lg_gv = __builtin_ctz(static_cast<unsigned>(a.group_v));
   dim3 grid(a.bh, jobs);
-  if (a.fine) {
+  if (a.fine && a.residual <= 256) {  // one thread per 8 tokens x 8 channels of a block
+    if (bits == 2)
+      quantize_fine_tiles_kernel<2><<<grid, 2 * a.residual, 0, stream>>>(a);
+    else
+      quantize_fine_tiles_kernel<4><<<grid, 2 * a.residual, 0, stream>>>(a);
+  } else if (a.fine) {
     if (bits == 2)
       quantize_fine_kernel<2><<<grid, kHeadDim, 0, stream>>>(a);
     else
