@@ -80,13 +80,17 @@ __device__ __forceinline__ bool mbar_try_wait_hint(uint64_t* bar, uint32_t parit
   return ok != 0;
 }
 
+#ifndef KIVI_WAIT_HINT_NS
+#define KIVI_WAIT_HINT_NS 20000u  // longest suspension of one try of a bounded wait
+#endif
+
 // Bounded wait on an mbarrier phase: gives up after `limit_ns` of wall time (checked every 16
-// tries, each suspending for at most 20 us) and returns false.
+// tries, each suspending for at most KIVI_WAIT_HINT_NS) and returns false.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   for (uint32_t spin = 0;; ++spin) {
-    if (mbar_try_wait_hint(bar, parity, 20000u)) return true;
+    if (mbar_try_wait_hint(bar, parity, KIVI_WAIT_HINT_NS)) return true;
     if ((spin & 15u) == 15u && global_timer_ns() - t0 > limit_ns) return false;
   }
 }
