@@ -103,6 +103,7 @@ struct __align__(16) WarpSmem {
   uint4 pw[FG ? 4 * G : G][kLimbVecs];  // P operand digits of each query (FG: limbs per query and V channel group)
   uint4 zero4;                      // the all-zero B operand of the other tile of a pair
   float oscr[FG ? kHeadDim : 4];
+  float qs[G > 1 ? G : 1][G > 1 ? kHeadDim : 1];  // several queries: q * scale * log2 e of the head
   uint64_t bar[ring_buffers<G>()];
 };
 
@@ -374,7 +375,10 @@ struct Decoder {
         for (int j = 0; j < 4; ++j) {
           const int c = 16 * (lane >> 2) + 4 * j + (lane & 3);
           const float v = h2f(__ldg(qp + c)) * a.qscale;
-          if (G == 1) qreg[j] = v;
+          if (G == 1)
+            qreg[j] = v;
+          else
+            S.qs[g][c] = v;
           part += v;
         }
         // the 2^(lg_gk - 2) consecutive lanes of a K group reduce its sum; lane j takes group j's
@@ -386,7 +390,10 @@ struct Decoder {
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         qv[j] = h2f(__ldg(qp + lane + 32 * j)) * a.qscale;
-        if (G == 1) qreg[j] = qv[j];
+        if (G == 1)
+          qreg[j] = qv[j];
+        else
+          S.qs[g][lane + 32 * j] = qv[j];
       }
 #pragma unroll
       for (int gi = 0; gi < 4; ++gi) {
@@ -431,13 +438,12 @@ struct Decoder {
   }
 
   // This lane's q channel j of query g (scaled by scale * log2 e): channel 16 (lane / 4) + 4 j +
-  // lane % 4 at 2 bits, lane + 32 j at 4 bits.  Several queries per KV head read it from L1 (the
-  // block set-up runs once per 128 tokens) to keep registers for a second resident warp per
-  // sub-partition.
+  // lane % 4 at 2 bits, lane + 32 j at 4 bits.  Several queries per KV head keep it in shared memory
+  // (written by start_head) rather than in registers.
   __device__ __forceinline__ float q_of(int g, int j) const {
     if (G == 1) return qreg[j];
     const int c = BITS == 2 ? 16 * (lane >> 2) + 4 * j + (lane & 3) : lane + 32 * j;
-    return h2f(__ldg(a.q + (static_cast<size_t>(qhead) * G + g) * kHeadDim + c)) * a.qscale;
+    return S.qs[G > 1 ? g : 0][G > 1 ? c : 0];
   }
 
   // ---- A6 set-up for one K block: fixed-point limbs of q_c * s_g(c) -------------------------
@@ -881,9 +887,9 @@ struct Decoder {
     }
     float lg[TPL];
 #pragma unroll
-    for (int j = 0; j < TPL; ++j) {
-      const int jg = ngt == 2 ? j : 0;
-      lg[j] = fmaf(combine_limbs(ah[j], am[j], al[j]), invqf[jg], cblkf[jg]);
+    for (int j = 0; j < TPL; ++j) {  // token group of token j: j when g_k = 32, else 0 (no runtime index)
+      const bool own = ngt == 2 && j == 1;
+      lg[j] = fmaf(combine_limbs(ah[j], am[j], al[j]), own ? invqf[1] : invqf[0], own ? cblkf[1] : cblkf[0]);
     }
     softmax4_fg(gq, head, local, lg);
   }
@@ -1218,7 +1224,7 @@ struct Decoder {
   // ---- K half of a quantized unit: logits, online softmax, P limbs (A6, A8, A9 set-up) ---------
   __device__ void quantized_k(const uint8_t* kt, long long head, int local, uint32_t pairs) {
     if constexpr (FG) {
-#pragma unroll 1
+#pragma unroll  // the per-query state stays in registers
       for (int gq = 0; gq < G; ++gq) {
         if constexpr (BITS == 2)
           fg_k(gq, kt, head, local);
@@ -1303,7 +1309,7 @@ struct Decoder {
   __device__ void quantized_v(const uint8_t* vt) {
     __syncwarp();  // P limbs of every query are in shared memory
     if constexpr (FG) {
-#pragma unroll 1
+#pragma unroll  // the per-query state stays in registers
       for (int gq = 0; gq < G; ++gq) {
         if constexpr (BITS == 2) {
           if (hasv_[gq]) {
@@ -1457,25 +1463,38 @@ struct Decoder {
     for (int g = 0; g < G; ++g) {
       const uint4* qp = reinterpret_cast<const uint4*>(a.q + (static_cast<size_t>(head) * G + g) * kHeadDim);
       float dot = 0.f;
-      // several queries: one chunk at a time, so that the loads of all queries are not in flight at
-      // once (they would hold more registers than the kernel has)
-#pragma unroll(G == 1 ? 8 : 1)
+      // several queries read the scaled q from shared memory (start_head), two chunks at a time so
+      // that the loads of all queries are not in flight at once
+#pragma unroll(G == 1 ? 8 : 2)
       for (int k = 0; k < 8; ++k) {
         const int cc = (k + lane) & 7;  // bank-conflict-free chunk order
         const int c0 = 64 * hf + 8 * cc;
         const uint4 kv = *reinterpret_cast<const uint4*>(kt + t * 256 + 2 * c0);
-        const uint4 qv = __ldg(qp + (c0 >> 3));
-        const uint32_t kw[4] = {kv.x, kv.y, kv.z, kv.w}, qw[4] = {qv.x, qv.y, qv.z, qv.w};
+        const uint32_t kw[4] = {kv.x, kv.y, kv.z, kv.w};
+        if constexpr (G > 1) {
+          const float4 qa = *reinterpret_cast<const float4*>(&S.qs[G > 1 ? g : 0][G > 1 ? c0 : 0]);
+          const float4 qb = *reinterpret_cast<const float4*>(&S.qs[G > 1 ? g : 0][G > 1 ? c0 + 4 : 0]);
+          const float qf[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float2 kf = __half22float2(*reinterpret_cast<const __half2*>(&kw[e]));
-          const float2 qf = __half22float2(*reinterpret_cast<const __half2*>(&qw[e]));
-          dot = fmaf(qf.x, kf.x, dot);
-          dot = fmaf(qf.y, kf.y, dot);
+          for (int e = 0; e < 4; ++e) {
+            const float2 kf = __half22float2(*reinterpret_cast<const __half2*>(&kw[e]));
+            dot = fmaf(qf[2 * e], kf.x, dot);
+            dot = fmaf(qf[2 * e + 1], kf.y, dot);
+          }
+        } else {
+          const uint4 qv = __ldg(qp + (c0 >> 3));
+          const uint32_t qw[4] = {qv.x, qv.y, qv.z, qv.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 kf = __half22float2(*reinterpret_cast<const __half2*>(&kw[e]));
+            const float2 qf = __half22float2(*reinterpret_cast<const __half2*>(&qw[e]));
+            dot = fmaf(qf.x, kf.x, dot);
+            dot = fmaf(qf.y, kf.y, dot);
+          }
         }
       }
       dot += __shfl_xor_sync(kFull, dot, 1);
-      dot *= a.qscale;
+      if (G == 1) dot *= a.qscale;  // several queries: q in shared memory is scaled already
       const bool valid = t < nvalid;
       const float lg = valid ? dot : -INFINITY;
       const float m_new = fmaxf(m[g], warp_max(lg));
