@@ -16,7 +16,7 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libkivi.so")
 LIB_DEBUG = os.path.join(PKG, "libkivi_debug.so")   # -DKIVI_DEBUG: device-side bounds checks
 SOURCES = ["kivi_api.cu", "quantize.cu", "decode.cu", "noalloc.cu"]
-HEADERS = ["common.cuh", "kernels.h"]
+HEADERS = ["common.cuh", "kernels.h", "quant_rules.cuh"]
 
 
 def nvcc() -> str:
