@@ -40,9 +40,17 @@ SPEC_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
 L2_BYTES = 126e6
 WORKLOAD = synth.LARGE_BATCH
-FUSED = True   # append and decode in one launch (kivi_append_decode_attention); --separate-append: two
-STEP_NOTE = {True: "flush when full + append and decode attention in one launch",
-             False: "flush when full + append + decode attention"}
+# How a step reaches the library:
+#   "step"     (default): kivi_decode_step, one launch per step: append, decode attention and, at the
+#              step whose token fills the residual, its flush (eager);
+#   "fused"    (--lazy-flush): kivi_flush_residual when the residual is full, then
+#              kivi_append_decode_attention (two launches on flush steps);
+#   "separate" (--separate-append, --online-k): flush when full + kivi_append_token +
+#              kivi_decode_attention.
+MODE = "step"
+STEP_NOTE = {"step": "append, decode attention and (when the token fills the residual) its flush in one launch",
+             "fused": "flush when full + append and decode attention in one launch",
+             "separate": "flush when full + append + decode attention"}
 ONLINE_K = False   # --online-k: K rows coded at append with the newest block's (s, z) (config online_k)
 FINE = False       # --fine-groups: K (s, z) per channel per G tokens, V per token per G channels
 DECODE_SOURCES = ["decode.cu", "common.cuh", "kernels.h"]
@@ -102,6 +110,16 @@ def profiled_traffic(w: synth.Workload, alg_bytes_per_launch: float):
 def append_bytes(w: synth.Workload) -> int:
     """Bytes a fused append adds to the decode launch: the new K and V rows read and written once."""
     return w.batch * w.kv_heads * w.head_dim * 2 * 2 * 2
+
+
+def flush_bytes(w: synth.Workload) -> int:
+    """Bytes a flush moves at least once: the R fp16 K and V residual rows read, their codes and the
+    block's scales and zero points written (base groups)."""
+    R = w.residual
+    per_head = (2 * R * w.head_dim * 2                       # fp16 K and V rows
+                + 2 * R * w.head_dim * w.bits // 8           # K and V codes
+                + ((w.head_dim // w.group) + R // w.gv) * 4)  # K and V (s, z) pairs, fp16
+    return w.batch * w.kv_heads * per_head
 
 
 def decode_alg_bytes(w: synth.Workload, n_quant: int, n_res: int) -> int:
@@ -267,9 +285,10 @@ def weak_scaling_value(world: int, tokens_per_rank: int, batch: int, t_max_ms: f
 
 def first_prompt_split(w: synth.Workload):
     """(n_quant, capacity) of the bench's cache: the prompt leaves a full residual; the cache holds
-    one more block (two under online K: the block being filled keeps its own scale row)."""
+    one more block, two when the block being filled needs its own room (online K keeps its scale
+    row there; the decode step flushes a full residual into it before the cycle drops it)."""
     n_quant0 = (w.tokens - 1) // w.residual * w.residual
-    return n_quant0, n_quant0 + (2 if ONLINE_K else 1) * w.residual
+    return n_quant0, n_quant0 + (2 if (ONLINE_K or MODE == "step") else 1) * w.residual
 
 
 def workload_config(w: synth.Workload, world: int, replicas: int) -> dict:
@@ -279,8 +298,8 @@ def workload_config(w: synth.Workload, world: int, replicas: int) -> dict:
     return {
         "workload": w.name, "batch": w.batch, "q_heads": w.q_heads, "kv_heads": w.kv_heads,
         "head_dim": w.head_dim, "bits": w.bits, "group_k": w.group, "group_v": w.gv,
-        "residual": R, "cached_tokens": f"{n_quant0 + 1}-{n_quant0 + 2 * R} (128-step cycles)",
-        "step": STEP_NOTE[FUSED],
+        "residual": R, "cached_tokens": f"{n_quant0 + R + 1}-{n_quant0 + 2 * R} ({R}-step cycles)",
+        "step": STEP_NOTE[MODE],
         "k_residual": "codes (online K, config online_k = 1)" if ONLINE_K else "fp16",
         "groups": ("fine: K per channel per G tokens, V per token per G channels (config fine_groups = 1)"
                    if FINE else "K per R-token block x G channels, V per G tokens x all channels"),
@@ -312,13 +331,35 @@ def step_inputs(w: synth.Workload, torch, device):
 
 
 def gpu_step(cache, n_quant0, w, inputs, out, stream, decode_events=None, stage_events=None, status=True):
-    """One streaming decode step on device-resident inputs; returns (launches, cached tokens).
-    stage_events (optional): {"flush": [...], "append": [...]} lists that receive event pairs."""
+    """One streaming decode step on device-resident inputs.  Returns (launches, cached tokens
+    attended, quantized tokens attended, whether the step's own launch flushed the residual).
+    stage_events (optional): {"flush": [...], "append": [...]} lists that receive event pairs.
+
+    The cache cycles through R steps: every step attends n_quant0 + R quantized tokens and 1..R
+    residual tokens.  The decode step flushes the residual at the step that fills it, into the
+    block after those, which the next step drops again; the lazy modes flush a full residual at the
+    next step, after moving n_quant back to n_quant0 (the cycle's block is rewritten)."""
     import torch
+    R = w.residual
+    kn, vn, q = inputs
+    if MODE == "step":
+        if cache.c.n_quant == n_quant0 + 2 * R:
+            cache.c.n_quant = n_quant0 + R     # end of a cycle: drop the block the filling step wrote
+        full = cache.c.n_res == R              # only after the prefill: flushed first, by its own launch
+        nq = cache.c.n_quant + (R if full else 0)
+        nr = (0 if full else cache.c.n_res) + 1
+        if decode_events is not None:
+            decode_events[0].record(stream)
+        cache.step(kn, vn, q, out=out, stream=stream, status=status)
+        if decode_events is not None:
+            decode_events[1].record(stream)
+        flushed = nr == R and nq + R <= cache.cfg.capacity
+        assert (cache.c.n_quant, cache.c.n_res) == ((nq + R, 0) if flushed else (nq, nr))
+        return (2 if full else 1), nq + nr, nq, flushed
     launches = 0
-    if cache.c.n_res == w.residual:
-        if cache.c.n_quant == n_quant0 + w.residual:
-            cache.c.n_quant = n_quant0     # end of a 128-step cycle: drop the newest block again
+    if cache.c.n_res == R:
+        if cache.c.n_quant == n_quant0 + R:
+            cache.c.n_quant = n_quant0     # end of a cycle: drop the newest block again
         if stage_events is not None:
             ev = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
             ev[0].record(stream)
@@ -327,14 +368,13 @@ def gpu_step(cache, n_quant0, w, inputs, out, stream, decode_events=None, stage_
             ev[1].record(stream)
             stage_events["flush"].append(ev)
         launches += 1
-    kn, vn, q = inputs
-    if FUSED:
+    if MODE == "fused":
         if decode_events is not None:
             decode_events[0].record(stream)
         cache.append_attend(kn, vn, q, out=out, stream=stream, status=status)
         if decode_events is not None:
             decode_events[1].record(stream)
-        return launches + 1, cache.c.n_quant + cache.c.n_res
+        return launches + 1, cache.c.n_quant + cache.c.n_res, cache.c.n_quant, False
     if stage_events is not None:
         ev = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
         ev[0].record(stream)
@@ -349,7 +389,7 @@ def gpu_step(cache, n_quant0, w, inputs, out, stream, decode_events=None, stage_
     if decode_events is not None:
         decode_events[1].record(stream)
     launches += 1
-    return launches, cache.c.n_quant + cache.c.n_res
+    return launches, cache.c.n_quant + cache.c.n_res, cache.c.n_quant, False
 
 
 def run_gpu(args, rank, world, local_rank, w: synth.Workload):
@@ -415,16 +455,17 @@ def run_gpu(args, rank, world, local_rank, w: synth.Workload):
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         launches, tokens, bytes_decode = 0, 0, 0
         stage_ev = {"flush": [], "append": []}
+        flush_steps = []   # whether each timed step's own launch flushed the residual
         t_wall0 = time.monotonic()
         with torch.cuda.stream(stream):
             e0.record(stream)
             for i in range(K):
-                lz, t = step((W + i) % R, ev[i], stage_ev)
-                c = caches[(counter[0] - 1) % replicas]
+                lz, t, nq, fl = step((W + i) % R, ev[i], stage_ev)
                 launches += lz
                 tokens += t
-                n_q2 = c.c.n_quant
-                bytes_decode += decode_alg_bytes(w, n_q2, t - n_q2) + (append_bytes(w) if FUSED else 0)
+                flush_steps.append(fl)
+                bytes_decode += (decode_alg_bytes(w, nq, t - nq) + (append_bytes(w) if MODE != "separate" else 0)
+                                 + (flush_bytes(w) if fl else 0))
             e1.record(stream)
             stream.synchronize()
         torch.cuda.synchronize(device)
@@ -442,8 +483,14 @@ def run_gpu(args, rank, world, local_rank, w: synth.Workload):
                 stream.synchronize()
         t_wall2 = time.monotonic()
         ms = e0.elapsed_time(e1)
-        dec_ms = sum(a.elapsed_time(b) for a, b in ev)
+        step_ms = [a.elapsed_time(b) for a, b in ev]
+        dec_ms = sum(step_ms)
         stage_ms = {k: (sum(a.elapsed_time(b) for a, b in v) / len(v) if v else None) for k, v in stage_ev.items()}
+        fl_ms = [x for x, f in zip(step_ms, flush_steps) if f]
+        plain_ms = [x for x, f in zip(step_ms, flush_steps) if not f]
+        if fl_ms and plain_ms:   # the decode step: what its flush adds to the launch
+            stage_ms["flush_in_launch"] = statistics.mean(fl_ms) - statistics.mean(plain_ms)
+            stage_ms["flush_steps"] = len(fl_ms)
         clk = sampler.summary(t_wall0, t_wall2)
         clk["window_s"] = round(t_wall2 - t_wall0, 3)
         clk["window"] = (f"the {K} timed steps ({(t_wall1 - t_wall0) * 1e3:.1f} ms wall) and {ext} more of the same "
@@ -469,11 +516,17 @@ def run_gpu(args, rank, world, local_rank, w: synth.Workload):
     with torch.cuda.stream(stream):
         for _ in range(3):
             c = caches[counter[0] % replicas]
-            while c.c.n_res < R:        # steps of this replica until its residual is full
-                for _r in range(replicas):
-                    step(counter[0] % R)
-            if c.c.n_quant == n_quant0 + R:
-                c.c.n_quant = n_quant0   # the cycle of gpu_step; the replica's next step finds n_res = 0
+            if MODE == "step":          # the decode step never leaves a full residual: append to one
+                if c.c.n_quant == n_quant0 + 2 * R:
+                    c.c.n_quant = n_quant0 + R
+                while c.c.n_res < R:
+                    c.append(dev_in[0][0], dev_in[0][1], stream)
+            else:
+                while c.c.n_res < R:        # steps of this replica until its residual is full
+                    for _r in range(replicas):
+                        step(counter[0] % R)
+                if c.c.n_quant == n_quant0 + R:
+                    c.c.n_quant = n_quant0   # the cycle of gpu_step; the replica's next step finds n_res = 0
             fl[0].record(stream)
             c.flush(stream)
             fl[1].record(stream)
@@ -507,8 +560,7 @@ def run_gpu(args, rank, world, local_rank, w: synth.Workload):
             f0.record(stream)
             for i in range(K):
                 stage_buf.copy_(pinned[i % R], non_blocking=True)
-                _, t = step(i % R, inputs=stage)
-                toks += t
+                toks += step(i % R, inputs=stage)[1]
                 out_host.copy_(out, non_blocking=True)
                 stream.synchronize()      # the caller consumes the step's result
             f1.record(stream)
@@ -531,6 +583,11 @@ def run_gpu(args, rank, world, local_rank, w: synth.Workload):
         traffic = profiled_traffic(w, bytes_decode / K) if replicas == 1 else None
         e2e_value = weak_scaling_value(world, e2e_tokens, w.batch, e2e_ms)
         flush_window = stage_ms["flush"]
+        flush_source = "flushes inside the timed window"
+        if stage_ms.get("flush_in_launch") is not None:
+            flush_window = stage_ms["flush_in_launch"]
+            flush_source = (f"in-launch: the {stage_ms['flush_steps']} timed steps that flushed, minus the "
+                            f"average of the others")
         result = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
             "ms_per_step": t_max / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
@@ -547,7 +604,7 @@ def run_gpu(args, rank, world, local_rank, w: synth.Workload):
                 "decode_ms": dec_avg_ms,
                 "append_ms": stage_ms["append"],
                 "flush_ms": flush_window if flush_window is not None else statistics.median(flush_ms_sep),
-                "flush_ms_source": ("flushes inside the timed window" if flush_window is not None else
+                "flush_ms_source": (flush_source if flush_window is not None else
                                     "3 flushes timed on their own after the timed window"),
                 "flush_ms_separate": statistics.median(flush_ms_sep),
                 "prefill_ms": prefill_ms, "prefill_tokens": w.tokens,
@@ -578,18 +635,31 @@ def _oracle_head(w: synth.Workload, b: int, h: int):
     return hc, n_quant0
 
 
-def _oracle_cycle_flush(w: synth.Workload, hc, n_quant0: int):
-    """The flush of gpu_step: at the end of a 128-step cycle n_quant goes back by one block first."""
+def _oracle_truncate(w: synth.Workload, hc, n: int):
+    """Drops the quantized tokens from n on (whole blocks), as the bench's cycle does on the GPU."""
     R = w.residual
+    hc.k_codes, hc.v_codes = hc.k_codes[:n], hc.v_codes[:n]
+    if hc.fine:
+        hc.k_s, hc.k_z = hc.k_s[:n // w.group], hc.k_z[:n // w.group]
+        hc.v_s, hc.v_z = hc.v_s[:n], hc.v_z[:n]
+    else:
+        hc.k_s, hc.k_z = hc.k_s[:n // R], hc.k_z[:n // R]
+        hc.v_s, hc.v_z = hc.v_s[:n // w.gv], hc.v_z[:n // w.gv]
+
+
+def _oracle_cycle_flush(w: synth.Workload, hc, n_quant0: int):
+    """The flush of gpu_step's cycle, applied to a full residual before the next append.  The decode
+    step flushes into the block after n_quant0 + R and drops it; the lazy modes move n_quant back to
+    n_quant0 first (the cycle's block is rewritten).  Flushing eagerly or at the next append gives
+    the same attention, so the oracle flushes at the next append in every mode."""
+    R = w.residual
+    if MODE == "step":
+        hc.flush()
+        if hc.n_quant == n_quant0 + 2 * R:
+            _oracle_truncate(w, hc, n_quant0 + R)
+        return
     if hc.n_quant == n_quant0 + R:
-        n = n_quant0
-        hc.k_codes, hc.v_codes = hc.k_codes[:n], hc.v_codes[:n]
-        if hc.fine:
-            hc.k_s, hc.k_z = hc.k_s[:n // w.group], hc.k_z[:n // w.group]
-            hc.v_s, hc.v_z = hc.v_s[:n], hc.v_z[:n]
-        else:
-            hc.k_s, hc.k_z = hc.k_s[:n // R], hc.k_z[:n // R]
-            hc.v_s, hc.v_z = hc.v_s[:n // w.gv], hc.v_z[:n // w.gv]
+        _oracle_truncate(w, hc, n_quant0)
     hc.flush()
 
 
@@ -720,6 +790,9 @@ def main():
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end loop (profiling runs)")
     ap.add_argument("--separate-append", action="store_true",
                     help="append and decode as two launches (kivi_append_token + kivi_decode_attention)")
+    ap.add_argument("--lazy-flush", action="store_true",
+                    help="flush a full residual with its own launch at the next step, then append and decode in "
+                         "one launch (kivi_flush_residual + kivi_append_decode_attention)")
     ap.add_argument("--fine-groups", action="store_true",
                     help="fine-grained groups (config fine_groups = 1); no cpu baseline timing")
     ap.add_argument("--online-k", action="store_true",
@@ -728,12 +801,12 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
-    global FUSED, ONLINE_K, FINE
+    global MODE, ONLINE_K, FINE
     ONLINE_K = args.online_k
     FINE = args.fine_groups
     if FINE and args.impl == "reference":
         ap.error("--fine-groups times the GPU arm only")
-    FUSED = not (args.separate_append or args.online_k)
+    MODE = "separate" if (args.separate_append or args.online_k) else ("fused" if args.lazy_flush else "step")
     if ONLINE_K and args.impl == "reference":
         ap.error("--online-k times the GPU arm only")
     w = synth.WORKLOADS[args.workload]

@@ -45,6 +45,7 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "quant_rules.cuh"
 
 namespace kivi {
 
@@ -61,7 +62,7 @@ namespace {
 template <int G, bool FG = false>
 __host__ __device__ constexpr int warps_per_cta() {
   // fine-grained groups keep P operands per (query, V channel group) and more per-query state
-  return FG ? (G == 1 ? 16 : (G == 2 ? 12 : (G == 4 ? 8 : 6))) : (G == 1 ? 16 : (G <= 4 ? KIVI_GQA_WARPS : 8));
+  return FG ? (G == 1 ? 16 : (G == 2 ? 12 : (G == 4 ? 8 : 5))) : (G == 1 ? 16 : (G <= 4 ? KIVI_GQA_WARPS : 8));
 }
 constexpr int kHalfBytes = 4096;    // one half unit: the K part or the V part of a unit
 // The tensor-core path lands a V half as four 1 KB pieces (two V word rows each) 1040 bytes apart,
@@ -77,6 +78,14 @@ __host__ __device__ constexpr int buf_bytes() {
 template <int G>
 __host__ __device__ constexpr int ring_buffers() {
   return G <= 4 ? 2 : 3;
+}
+// Slots for the fp16 queries that land with a head's first K half.  With a ring of 2 the next
+// unit's K half is issued only after this unit's K half (the last reader of the raw queries) is
+// done, so one slot is enough; with a ring of 3 the K half two units ahead can start a head while
+// the next unit's head has yet to read its queries: two slots, taken by head parity.
+template <int G>
+__host__ __device__ constexpr int q_slots() {
+  return ring_buffers<G>() == 2 ? 1 : 2;
 }
 constexpr int kResTokens = 16;      // tokens per residual unit
 constexpr unsigned kFull = 0xffffffffu;
@@ -99,6 +108,7 @@ constexpr int kLimbVecs = 32;
 template <int G, bool FG = false>
 struct __align__(16) WarpSmem {
   uint8_t buf[ring_buffers<G>()][buf_bytes<G>()];
+  uint16_t qraw[q_slots<G>()][G][kHeadDim];  // fp16 queries of a head (see q_slots)
   uint4 qw[FG ? 4 : G][kLimbVecs];      // Q operand digits of each query (FG: limbs of each K token group)
   uint4 pw[FG ? 4 * G : G][kLimbVecs];  // P operand digits of each query (FG: limbs per query and V channel group)
   uint4 zero4;                      // the all-zero B operand of the other tile of a pair
@@ -247,10 +257,174 @@ __device__ __forceinline__ void dot_set(uint32_t m, uint32_t L, uint32_t M, uint
   ah = signed_hi ? dp4a_us(m, H, ah) : dp4a_uu(m, H, ah);
 }
 
+// ---- in-launch flush of a full residual (the decode step) ----------------------------------
+// A step whose appended token fills the residual also quantizes it, in the same launch, as block
+// flush_blk of the quantized arrays (section 残差バッファ: the full residual becomes one quantized
+// block; section 量子化アルゴリズム: Q, s and z, by the rule of quant_rules.cuh, so the codes equal
+// those of the flush kernel bit for bit).  Jobs: per KV head each K group (g_k channels over the R
+// tokens) and each V group (g_v tokens over all channels); worker w takes jobs w, w + W, ... after
+// its decode range.  A job moves its group through the warp's free ring buffers 8 KB at a time
+// (16 cp.async of 16 bytes per lane, no registers held while they fly): a pass over the stage
+// forms the extremes, a second one the codes; a group larger than 8 KB (R > 128 with g_k = 32,
+// g_k > 32, g_v > 32) is staged twice, the second time from L2.  Residual slot new_slot is read
+// from k_new / v_new: the warp that attends that slot writes it into the cache in this same launch.
+__device__ __forceinline__ float warp_min(float v) {
+  float r;
+  asm volatile("redux.sync.min.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(v));
+  return r;
+}
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.commit_group;\n cp.async.wait_group 0;" ::: "memory");
+}
+
+template <int BITS>
+struct Flusher {
+  static constexpr int L = (1 << BITS) - 1;  // largest code
+  static constexpr int P = 32 / BITS;        // codes per word
+  static constexpr int kStage = 16;          // 16-byte chunks per lane per stage (8 KB per warp)
+  const DecodeArgs& a;
+  uint4* stage;  // the warp's ring buffers: slot [k][lane]
+  const int lane;
+
+  // Address of 16-byte chunk `chunk` of residual token t of KV head `head` (K or V)
+  __device__ __forceinline__ const uint4* res_chunk(bool v, long long head, int t, int chunk) const {
+    const uint16_t* row = t == a.new_slot ? (v ? a.v_new : a.k_new) + static_cast<size_t>(head) * kHeadDim
+                                          : (v ? a.v_res : a.k_res) +
+                                                (static_cast<size_t>(head) * a.residual + t) * kHeadDim;
+    return reinterpret_cast<const uint4*>(row) + chunk;
+  }
+  // stage[k][lane] = chunk `chunk` of token tok(k), k < kStage
+  template <typename Tok>
+  __device__ __forceinline__ void fill(bool v, long long head, int chunk, Tok tok) const {
+    __syncwarp();  // the previous stage is no longer read
+#pragma unroll
+    for (int k = 0; k < kStage; ++k) cp_async16(stage + k * 32 + lane, res_chunk(v, head, tok(k), chunk));
+    cp_async_wait_all();
+    __syncwarp();
+  }
+
+  // K group gi of `head`: channels [gi g_k, (gi + 1) g_k) over the R tokens.  Lane (s, c) holds
+  // chunk c (8 channels) of tokens s, s + slots, ...; a 2-bit code word (16 channels) is the OR of
+  // two lanes' halves.
+  __device__ void k_group(long long head, int gi) const {
+    const int R = a.residual, cpr = (1 << a.lg_gk) >> 3, slots = 32 / cpr;
+    const int c = lane % cpr, s = lane / cpr, nt = R / slots;  // nt: the lane's tokens, a multiple of 16
+    const int chunk = (gi << (a.lg_gk - 3)) + c;  // chunk of the row (8 channels each)
+    float lo = INFINITY, hi = -INFINITY;
+    for (int k0 = 0; k0 < nt; k0 += kStage) {
+      fill(false, head, chunk, [&](int k) { return s + slots * (k0 + k); });
+#pragma unroll
+      for (int k = 0; k < kStage; ++k) minmax8(stage[k * 32 + lane], lo, hi);
+    }
+    const GroupParams g = make_group(warp_min(lo), warp_max(hi), L);
+    const size_t C = static_cast<size_t>(a.capacity);
+    const int ngk = kHeadDim >> a.lg_gk;
+    if (lane == 0) {
+      const size_t si = (static_cast<size_t>(head) * (C / R) + a.flush_blk) * ngk + gi;
+      a.fk_scale[si] = g.s_bits;
+      a.fk_zero[si] = g.z_bits;
+    }
+    uint32_t* dst = a.fk_codes + (static_cast<size_t>(head) * C + static_cast<size_t>(a.flush_blk) * R) * (kHeadDim / P);
+    for (int k0 = 0; k0 < nt; k0 += kStage) {
+      if (nt > kStage) fill(false, head, chunk, [&](int k) { return s + slots * (k0 + k); });
+#pragma unroll 4
+      for (int k = 0; k < kStage; ++k) {
+        const int t = s + slots * (k0 + k);
+        const uint4 v = stage[k * 32 + lane];
+        uint32_t part = 0u;  // the chunk's 8 codes at their bits of the word
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          uint32_t qa, qb;
+          quantize_pair(comp(v, e), g, L, qa, qb);
+          part |= (qa << (BITS * 2 * e)) | (qb << (BITS * (2 * e + 1)));
+        }
+        if constexpr (BITS == 2) {  // word = chunks 2 w and 2 w + 1
+          part <<= 16 * (c & 1);
+          part |= __shfl_xor_sync(kFull, part, 1);
+          if ((c & 1) == 0) dst[static_cast<size_t>(t) * (kHeadDim / P) + (chunk >> 1)] = part;
+        } else {  // word = one chunk
+          dst[static_cast<size_t>(t) * (kHeadDim / P) + chunk] = part;
+        }
+      }
+    }
+  }
+
+  // V group vg of `head`: tokens [vg g_v, (vg + 1) g_v) over all channels, in slabs of 32 tokens.
+  // Lane (h, c) holds chunk c of the slab's tokens 16 h .. 16 h + 15, i.e. whole code words (one
+  // word row at 2 bits, two at 4 bits) of its 8 channels.
+  __device__ void v_group(long long head, int vg) const {
+    const int R = a.residual, gv = 1 << a.lg_gv, nslab = gv >> 5;
+    const int c = lane & 15, h = lane >> 4;
+    const int t0 = vg * gv + 16 * h;
+    float lo = INFINITY, hi = -INFINITY;
+    for (int sl = 0; sl < nslab; ++sl) {
+      fill(true, head, c, [&](int k) { return t0 + 32 * sl + k; });
+#pragma unroll
+      for (int k = 0; k < kStage; ++k) minmax8(stage[k * 32 + lane], lo, hi);
+    }
+    const GroupParams g = make_group(warp_min(lo), warp_max(hi), L);
+    const size_t C = static_cast<size_t>(a.capacity);
+    const size_t T0 = static_cast<size_t>(a.flush_blk) * R;  // first token of the block
+    if (lane == 0) {
+      const size_t si = static_cast<size_t>(head) * (C >> a.lg_gv) + ((T0 + vg * gv) >> a.lg_gv);
+      a.fv_scale[si] = g.s_bits;
+      a.fv_zero[si] = g.z_bits;
+    }
+    for (int sl = 0; sl < nslab; ++sl) {
+      if (nslab > 1) fill(true, head, c, [&](int k) { return t0 + 32 * sl + k; });
+      uint32_t w[16 / P][8];
+#pragma unroll
+      for (int r = 0; r < 16 / P; ++r)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) w[r][e] = 0u;
+#pragma unroll
+      for (int k = 0; k < kStage; ++k) {
+        const uint4 v = stage[k * 32 + lane];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          uint32_t qa, qb;
+          quantize_pair(comp(v, e), g, L, qa, qb);
+          w[k / P][2 * e] |= qa << (BITS * (k % P));
+          w[k / P][2 * e + 1] |= qb << (BITS * (k % P));
+        }
+      }
+#pragma unroll
+      for (int r = 0; r < 16 / P; ++r) {
+        const size_t row = (T0 + vg * gv + 32 * sl + 16 * h) / P + r;  // word row of the head
+        uint4* dst = reinterpret_cast<uint4*>(a.fv_codes + (static_cast<size_t>(head) * (C / P) + row) * kHeadDim + 8 * c);
+        dst[0] = make_uint4(w[r][0], w[r][1], w[r][2], w[r][3]);
+        dst[1] = make_uint4(w[r][4], w[r][5], w[r][6], w[r][7]);
+      }
+    }
+  }
+
+  // Not inlined: the flush's registers get their own allocation instead of pushing the decode
+  // loop's values into local memory.
+  __device__ __noinline__ void run(long long worker) const {
+    const int ngk = kHeadDim >> a.lg_gk, nvg = a.residual >> a.lg_gv, per_head = ngk + nvg;
+    const long long jobs = static_cast<long long>(a.bh) * per_head;
+    if (!dbg_check(a.flush_blk >= 0 && static_cast<long long>(a.flush_blk + 1) * a.residual <= a.capacity &&
+                       a.new_slot == a.residual - 1 && a.residual % 128 == 0 && a.lg_gv >= 5,
+                   a.status))
+      return;
+    for (long long j = worker; j < jobs; j += a.workers) {
+      const long long head = j / per_head;
+      const int r = static_cast<int>(j - head * per_head);
+      if (r < ngk)
+        k_group(head, r);
+      else
+        v_group(head, r - ngk);
+    }
+  }
+};
+
 // KC: the residual tokens' K rows are codes (online K); a separate instantiation keeps that path
 // out of the register allocation of the others.  FG: fine-grained groups (2 bits, one query per KV
 // head): K (s, z) per channel per g_k tokens, V (s, z) per token per g_v channels.
-template <int BITS, int G, bool KC, bool FG = false>
+template <int BITS, int G, bool KC, bool FG = false, bool FL = false>
 struct Decoder {
   static constexpr int P = 32 / BITS;              // codes per word
   static constexpr int UT = BITS == 2 ? 128 : 64;  // tokens per quantized unit (8 KB of codes)
@@ -275,9 +449,8 @@ struct Decoder {
   // per-head state.  At 2 bits lane (i, k) = (lane / 4, lane % 4) holds channels 16 i + 4 m + k
   // (m = 0..3: byte m of set k of K word i) and lane j < d / G_k holds the q sum of K group j in
   // qsum[g][0]; at 4 bits lane holds channels lane + 32 j and every lane holds all group sums.
-  float qreg[4];        // one query per KV head: its channels of q; several: read from L1 (q_of)
+  float qreg[4];        // one query per KV head: its channels of q; several: in shared memory (q_of)
   float qsum[G][4];
-  long long qhead;      // the KV head whose q is loaded
   float m[G], l[G], Z[G], o[G][4];
   // per-block state: the Q limbs in S.qw belong to (head, block) == qkey
   long long qkey;
@@ -291,6 +464,8 @@ struct Decoder {
   // at 2 bits o is in the FG layout while quantized units run
   float invqf[4], cblkf[4], ZF[FG ? G : 1][4], invvf[FG && BITS == 4 ? G : 1][4];
   bool ofg_;
+  // heads whose partials this worker wrote (at most two: the first and the last segment)
+  int pend0_, pend1_, npend_;
   // bytes per head of the code arrays and of a residual array; this lane's scale role
   const size_t code_head_bytes, res_head_bytes;
   const bool k_lane, v_lane;
@@ -300,7 +475,8 @@ struct Decoder {
         code_head_bytes(static_cast<size_t>(args.capacity) * (kHeadDim * BITS / 8)),
         res_head_bytes(static_cast<size_t>(args.residual) * kHeadDim * 2),
         k_lane(ln < (kHeadDim >> args.lg_gk)),
-        v_lane(ln >= 8 && ln < 8 + ((UT >> args.lg_gv) > 0 ? (UT >> args.lg_gv) : 1)) {}
+        v_lane(ln >= 8 && ln < 8 + ((UT >> args.lg_gv) > 0 ? (UT >> args.lg_gv) : 1)),
+        pend0_(-1), pend1_(-1), npend_(0) {}
 
   // ---- half-unit addressing: half h of the warp's range is the K (h even) or V (h odd) part -----
   // A unit's K half and V half are each 4 KB and contiguous: quantized unit `local` of a head
@@ -310,6 +486,9 @@ struct Decoder {
     const int b = h % kBuffers;
     const bool is_v = h & 1;
     const bool quant = local < a.units_q;
+    // the first K half of every head the warp starts also brings the head's queries
+    const bool with_q = !is_v && (h == 0 || local == 0);
+    const uint32_t qbytes = with_q ? G * kHeadDim * 2 : 0u;
     const char* base = quant ? reinterpret_cast<const char*>(is_v ? a.v_codes : a.k_codes)
                              : reinterpret_cast<const char*>(is_v ? a.v_res : a.k_res);
     const size_t stride = quant ? code_head_bytes : res_head_bytes;
@@ -332,11 +511,13 @@ struct Decoder {
       constexpr uint32_t kRowBytes = kHeadDim * BITS / 8;
       src = reinterpret_cast<const char*>(a.k_codes) + static_cast<size_t>(head) * code_head_bytes +
             (static_cast<size_t>(a.n_quant) + static_cast<size_t>(unit) * kResTokens) * kRowBytes;
-      mbar_arrive_expect_tx(&S.bar[b], kResTokens * kRowBytes + a.debug_extra_tx);
+      mbar_arrive_expect_tx(&S.bar[b], kResTokens * kRowBytes + qbytes + a.debug_extra_tx);
+      if (with_q) issue_q(head, b);
       bulk_g2s(S.buf[b], src, kResTokens * kRowBytes, &S.bar[b]);
       return;
     }
-    mbar_arrive_expect_tx(&S.bar[b], kHalfBytes + a.debug_extra_tx);
+    mbar_arrive_expect_tx(&S.bar[b], kHalfBytes + qbytes + a.debug_extra_tx);
+    if (with_q) issue_q(head, b);
     if (kMma && is_v) {
 #pragma unroll
       for (int c = 0; c < kHalfBytes / kVPiece; ++c)
@@ -345,6 +526,12 @@ struct Decoder {
       bulk_g2s(S.buf[b], src, kHalfBytes, &S.bar[b]);
     }
   }
+
+  // The G queries of KV head `head` (contiguous fp16 rows, 16-byte aligned) into its q slot.
+  __device__ void issue_q(long long head, int b) {
+    bulk_g2s(S.qraw[qslot(head)], a.q + static_cast<size_t>(head) * G * kHeadDim, G * kHeadDim * 2, &S.bar[b]);
+  }
+  static __device__ __forceinline__ int qslot(long long head) { return q_slots<G>() == 1 ? 0 : static_cast<int>(head & 1); }
 
   // (s, z) pairs of a quantized unit: lanes [0, ngk) hold K groups, lanes [8, 8 + nvg) V groups.
   // Branch-free: every lane forms both candidate indices and at most one lane group loads.
@@ -368,13 +555,13 @@ struct Decoder {
     __syncwarp();
 #pragma unroll
     for (int g = 0; g < G; ++g) {
-      const uint16_t* qp = a.q + (static_cast<size_t>(head) * G + g) * kHeadDim;
+      const uint16_t* qp = S.qraw[qslot(head)][g];  // landed with the head's first K half
       if constexpr (BITS == 2) {
         float part = 0.f;
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           const int c = 16 * (lane >> 2) + 4 * j + (lane & 3);
-          const float v = h2f(__ldg(qp + c)) * a.qscale;
+          const float v = h2f(qp[c]) * a.qscale;
           if (G == 1)
             qreg[j] = v;
           else
@@ -389,7 +576,7 @@ struct Decoder {
       float qv[4];
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        qv[j] = h2f(__ldg(qp + lane + 32 * j)) * a.qscale;
+        qv[j] = h2f(qp[lane + 32 * j]) * a.qscale;
         if (G == 1)
           qreg[j] = qv[j];
         else
@@ -411,7 +598,6 @@ struct Decoder {
       for (int e = 0; e < 4; ++e) o[g][e] = 0.f;
     }
     qkey = -1;
-    qhead = head;
     omma_ = kMmaG;  // o is zero: either layout
     ofg_ = FG;
 #pragma unroll
@@ -1415,7 +1601,7 @@ struct Decoder {
     }
 #pragma unroll  // the per-query state must stay in registers: no runtime index into it
     for (int g = 0; g < G; ++g) {
-      const uint4* qp = reinterpret_cast<const uint4*>(a.q + (static_cast<size_t>(head) * G + g) * kHeadDim + 64 * hf);
+      const uint4* qp = reinterpret_cast<const uint4*>(S.qraw[qslot(head)][g] + 64 * hf);
       float dot = 0.f;
 #pragma unroll
       for (int i = 0; i < WPL; ++i) {
@@ -1424,7 +1610,7 @@ struct Decoder {
         float acc = 0.f, qs = 0.f;
 #pragma unroll
         for (int k8 = 0; k8 < P / 8; ++k8) {
-          const uint4 qv = __ldg(qp + (P * i) / 8 + k8);
+          const uint4 qv = qp[(P * i) / 8 + k8];
           const uint32_t qw4[4] = {qv.x, qv.y, qv.z, qv.w};
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
@@ -1461,7 +1647,7 @@ struct Decoder {
     const int t = lane >> 1, hf = lane & 1;  // 2 lanes per token, 64 channels each
 #pragma unroll
     for (int g = 0; g < G; ++g) {
-      const uint4* qp = reinterpret_cast<const uint4*>(a.q + (static_cast<size_t>(head) * G + g) * kHeadDim);
+      const uint4* qp = reinterpret_cast<const uint4*>(S.qraw[qslot(head)][g]);
       float dot = 0.f;
       // several queries read the scaled q from shared memory (start_head), two chunks at a time so
       // that the loads of all queries are not in flight at once
@@ -1482,7 +1668,7 @@ struct Decoder {
             dot = fmaf(qf[2 * e + 1], kf.y, dot);
           }
         } else {
-          const uint4 qv = __ldg(qp + (c0 >> 3));
+          const uint4 qv = qp[c0 >> 3];
           const uint32_t qw[4] = {qv.x, qv.y, qv.z, qv.w};
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
@@ -1528,7 +1714,12 @@ struct Decoder {
     }
   }
 
-  // ---- end of a head segment: write the output, or a partial and maybe merge ----------------
+  // ---- end of a head segment: the output, or a partial ----------------------------------------
+  // A segment that covers its head whole writes the output.  Otherwise the segment's partial
+  // (m, l, Z, o) goes with plain stores to this worker's slot 0 (the first segment of its range)
+  // or slot 1 (the last one); the tickets that choose the worker that merges the head are taken at
+  // the end of the range (publish), after one fence that covers both partials, so that no fence or
+  // atomic round trip stalls the warp in the middle of its range.
   __device__ void finish_segment(long long head, long long seg_a, long long seg_b) {
     residual_layout();
     const long long h0 = head * a.units, h1 = h0 + a.units;
@@ -1556,76 +1747,126 @@ struct Decoder {
       }
       *reinterpret_cast<float4*>(p + 4 + 4 * lane) = make_float4(o[g][0], o[g][1], o[g][2], o[g][3]);
     }
-    __threadfence();  // every lane publishes its own slice of the partial before the ticket
+    // only the first and the last segment of a range can be partial
+    if (npend_ == 0)
+      pend0_ = static_cast<int>(head);
+    else
+      pend1_ = static_cast<int>(head);
+    ++npend_;
+  }
+
+  // Workers that hold a part of a head (a contiguous run of them: ranges are contiguous in units).
+  __device__ __forceinline__ void head_workers(long long head, long long& wfirst, long long& wlast) const {
+    const long long h0 = head * a.units, W = a.workers, U = a.total_units;
+    wfirst = worker_of(h0, U, W);
+    wlast = worker_of(h0 + a.units - 1, U, W);
+  }
+
+  // End of the range: one fence publishes this worker's partials, then one ticket per partial head
+  // (both atomics in flight together); the last of a head's workers to arrive merges the head.
+  __device__ void publish() {
+    if (npend_ == 0) return;
+    __threadfence();  // every lane publishes its own slices of the partials before the tickets
     __syncwarp();
-    const long long W = a.workers, U = a.total_units;
-    const long long wfirst = worker_of(h0, U, W), wlast = worker_of(h1 - 1, U, W);
     int last = 0;
     if (lane == 0) {
-      const int ticket = atomicAdd(a.tickets + head, 1);
-      last = ticket == static_cast<int>(wlast - wfirst);
-      __threadfence();  // acquire side: the partials published before the other tickets
+      const int t0 = atomicAdd(a.tickets + pend0_, 1);
+      const int t1 = npend_ > 1 ? atomicAdd(a.tickets + pend1_, 1) : -1;
+      long long wf, wl;
+      head_workers(pend0_, wf, wl);
+      if (t0 == static_cast<int>(wl - wf)) last |= 1;
+      if (npend_ > 1) {
+        head_workers(pend1_, wf, wl);
+        if (t1 == static_cast<int>(wl - wf)) last |= 2;
+      }
+      if (last) __threadfence();  // acquire side: the partials published before the other tickets
     }
-    __syncwarp();
     last = __shfl_sync(kFull, last, 0);
     if (!last) return;
     __threadfence();
-    // Workers wfirst..wlast each left one partial of this head.  Only wfirst can have started
-    // before the head (its partial is then in its slot 1); every later one starts inside it.
-    const int nparts = static_cast<int>(wlast - wfirst + 1);
-    const int first_slot = (U * wfirst / W) >= h0 ? 0 : 1;
-    if (!dbg_check(wfirst >= 0 && wlast < W, a.status)) return;
 #pragma unroll 1
+    for (int i = 0; i < 2; ++i)
+      if ((last >> i) & 1) merge(i ? pend1_ : pend0_);
+  }
+
+  // Merge of a head's partials: workers wfirst..wlast each left one.  Only wfirst can have started
+  // before the head (its partial is then in its slot 1); every later one starts inside it (slot 0).
+  // Lane k reads (m, l, Z) of part k; the o rows follow CH parts at a time, the loads of every query
+  // in flight together.
+  __device__ void merge(long long head) {
+    long long wfirst, wlast;
+    head_workers(head, wfirst, wlast);
+    const long long W = a.workers, U = a.total_units;
+    const int nparts = static_cast<int>(wlast - wfirst + 1);
+    const int first_slot = (U * wfirst / W) >= head * a.units ? 0 : 1;
+    if (!dbg_check(wfirst >= 0 && wlast < W, a.status)) return;
+    auto part = [&](int k, int g) -> const float* {
+      const long long x = wfirst + k;
+      return a.partials + ((x * 2 + (k == 0 ? first_slot : 0)) * G + g) * kPartialStride;
+    };
+    constexpr int CH = 8 / G > 0 ? 8 / G : 1;  // o rows of CH parts per query in flight
+    float mm[G], ls[G], zs[G], acc[G][4];
+#pragma unroll
     for (int g = 0; g < G; ++g) {
-      auto part = [&](int k) -> const float* {
-        const long long x = wfirst + k;
-        return a.partials + ((x * 2 + (k == 0 ? first_slot : 0)) * G + g) * kPartialStride;
-      };
-      // (m, l, Z) of up to 32 partials per pass, one per lane
-      float mm = -INFINITY;
-      for (int base = 0; base < nparts; base += 32) {
-        const int k = base + lane;
-        if (k < nparts) mm = fmaxf(mm, __ldcg(part(k)));
-      }
-      mm = warp_max(mm);
-      float ls = 0.f, zs = 0.f, acc[4] = {0.f, 0.f, 0.f, 0.f};
-      for (int base = 0; base < nparts; base += 32) {
-        const int k = base + lane;
-        float wk = 0.f;
-        if (k < nparts) {
-          const float* p = part(k);
-          const float lx = __ldcg(p + 1);
-          if (!(lx > 0.f)) report_status(a.status, KIVI_ERR_INTERNAL);  // never written
-          wk = fast_exp2(__ldcg(p) - mm);
-          ls = fmaf(wk, lx, ls);
-          zs = fmaf(wk, __ldcg(p + 2), zs);
-        }
-        const int n = min(32, nparts - base);
-        int i = 0;
-        for (; i + 4 <= n; i += 4) {  // four partial rows in flight
-          float4 ov[4];
+      mm[g] = -INFINITY;
+      ls[g] = 0.f;
+      zs[g] = 0.f;
 #pragma unroll
-          for (int u = 0; u < 4; ++u) ov[u] = __ldcg(reinterpret_cast<const float4*>(part(base + i + u) + 4) + lane);
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const float w = __shfl_sync(kFull, wk, i + u);
-            acc[0] = fmaf(w, ov[u].x, acc[0]);
-            acc[1] = fmaf(w, ov[u].y, acc[1]);
-            acc[2] = fmaf(w, ov[u].z, acc[2]);
-            acc[3] = fmaf(w, ov[u].w, acc[3]);
-          }
-        }
-        for (; i < n; ++i) {
-          const float4 ov = __ldcg(reinterpret_cast<const float4*>(part(base + i) + 4) + lane);
-          const float w = __shfl_sync(kFull, wk, i);
-          acc[0] = fmaf(w, ov.x, acc[0]);
-          acc[1] = fmaf(w, ov.y, acc[1]);
-          acc[2] = fmaf(w, ov.z, acc[2]);
-          acc[3] = fmaf(w, ov.w, acc[3]);
-        }
-      }
-      store_out(head, g, acc, warp_sum(zs), 1.f / warp_sum(ls));
+      for (int e = 0; e < 4; ++e) acc[g][e] = 0.f;
     }
+    if (nparts > 32) {  // the largest m first; up to 32 parts take it from the pass below
+      for (int k = lane; k < nparts; k += 32)
+#pragma unroll
+        for (int g = 0; g < G; ++g) mm[g] = fmaxf(mm[g], __ldcg(part(k, g)));
+#pragma unroll
+      for (int g = 0; g < G; ++g) mm[g] = warp_max(mm[g]);
+    }
+    for (int base = 0; base < nparts; base += 32) {
+      const int k = base + lane;
+      float mk[G], lk[G], zk[G], wk[G];
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        mk[g] = -INFINITY;
+        lk[g] = 0.f;
+        zk[g] = 0.f;
+        if (k < nparts) {
+          const float* p = part(k, g);
+          mk[g] = __ldcg(p);
+          lk[g] = __ldcg(p + 1);
+          zk[g] = __ldcg(p + 2);
+        }
+      }
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        if (k < nparts && !(lk[g] > 0.f)) report_status(a.status, KIVI_ERR_INTERNAL);  // never written
+        if (nparts <= 32) mm[g] = warp_max(mk[g]);
+        wk[g] = k < nparts ? fast_exp2(mk[g] - mm[g]) : 0.f;
+        ls[g] = fmaf(wk[g], lk[g], ls[g]);
+        zs[g] = fmaf(wk[g], zk[g], zs[g]);
+      }
+      const int n = min(32, nparts - base);
+      for (int i = 0; i < n; i += CH) {
+        float4 ov[CH][G];
+#pragma unroll
+        for (int u = 0; u < CH; ++u)
+#pragma unroll
+          for (int g = 0; g < G; ++g)
+            ov[u][g] = i + u < n ? __ldcg(reinterpret_cast<const float4*>(part(base + i + u, g) + 4) + lane)
+                                 : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int u = 0; u < CH; ++u)
+#pragma unroll
+          for (int g = 0; g < G; ++g) {
+            const float w = __shfl_sync(kFull, wk[g], (i + u) & 31);
+            acc[g][0] = fmaf(w, ov[u][g].x, acc[g][0]);
+            acc[g][1] = fmaf(w, ov[u][g].y, acc[g][1]);
+            acc[g][2] = fmaf(w, ov[u][g].z, acc[g][2]);
+            acc[g][3] = fmaf(w, ov[u][g].w, acc[g][3]);
+          }
+      }
+    }
+#pragma unroll
+    for (int g = 0; g < G; ++g) store_out(head, g, acc[g], warp_sum(zs[g]), 1.f / warp_sum(ls[g]));
     if (lane == 0) a.tickets[head] = 0;
   }
 
@@ -1692,9 +1933,9 @@ struct Decoder {
     long long cur_head = -1, seg_a = ub;
     int hk = 0;
     for (long long u = ub; u < ue; ++u, hk += 2) {
-      if (head != cur_head) {
+      const bool new_head = head != cur_head;
+      if (new_head) {
         if (cur_head >= 0) finish_segment(cur_head, seg_a, u);
-        start_head(head);
         cur_head = head;
         seg_a = u;
       }
@@ -1707,6 +1948,7 @@ struct Decoder {
         drain_from(hk, nhalves);
         return;
       }
+      if (new_head) start_head(head);  // the head's queries landed with this K half
       if (quant) {
         quantized_k(S.buf[hk % kBuffers], head, local, pairs);
       } else {
@@ -1714,7 +1956,10 @@ struct Decoder {
         residual_k(S.buf[hk % kBuffers], nvalid, head, local - a.units_q);
       }
       __syncwarp();
-      fence_proxy_async_smem();
+      // The bulk copy issued next overwrites the buffer just read.  The reads are complete (their
+      // values were consumed before the __syncwarp); a residual unit also wrote the new token's row
+      // into it, and that generic-proxy write is ordered before the async-proxy copy by a fence.
+      if (!quant) fence_proxy_async_smem();
       // half hk + kBuffers reuses the buffer just consumed: the next unit's V (ring of 3) or K (2)
       if (lane == 0 && hk + kBuffers < nhalves) issue_half(hk + kBuffers, h1, l1);
       // V half
@@ -1728,7 +1973,7 @@ struct Decoder {
       else
         residual_v(S.buf[(hk + 1) % kBuffers], nvalid, head, local - a.units_q);
       __syncwarp();
-      fence_proxy_async_smem();
+      if (!quant) fence_proxy_async_smem();
       // the unit after next's K half (ring of 3) or the next unit's V half (2)
       if (lane == 0 && hk + 1 + kBuffers < nhalves) {
         if (kBuffers == 3)
@@ -1744,10 +1989,17 @@ struct Decoder {
       advance(h2, l2);
     }
     finish_segment(cur_head, seg_a, ue);
+    publish();
+    if constexpr (FL) {  // the ring buffers are free: every copy the warp issued has landed and been read
+      static_assert(sizeof(S.buf) >= 32 * Flusher<BITS>::kStage * sizeof(uint4), "a flush stage is 8 KB");
+      Flusher<BITS>{a, reinterpret_cast<uint4*>(S.buf), lane}.run(worker);
+    }
   }
 };
 
-template <int BITS, int G, bool KC, bool FG = false>
+// FL: the step whose appended token fills the residual also flushes it (its own instantiation: the
+// flush's registers stay out of the allocation of the plain decode).
+template <int BITS, int G, bool KC, bool FG = false, bool FL = false>
 __global__ void __launch_bounds__(warps_per_cta<G, FG>() * 32, 1) decode_kernel(const __grid_constant__ DecodeArgs a) {
   extern __shared__ __align__(128) uint8_t smem_raw[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -1756,18 +2008,23 @@ __global__ void __launch_bounds__(warps_per_cta<G, FG>() * 32, 1) decode_kernel(
   const long long worker = static_cast<long long>(blockIdx.x) * warps_per_cta<G, FG>() + warp;
   if (worker >= W) return;  // the last CTA may hold fewer workers
   const long long ub = U * worker / W, ue = U * (worker + 1) / W;  // non-empty because W <= U
-  Decoder<BITS, G, KC, FG> d(a, S, lane, worker, ub, ue);
+  static_assert(!FL || (!KC && !FG), "the in-launch flush is for the base groups with fp16 residual keys");
+  Decoder<BITS, G, KC, FG, FL> d(a, S, lane, worker, ub, ue);
   d.run();
 }
 
 template <int BITS, int G, bool FG>
 cudaError_t plan_for_kernels(DecodePlan* plan) {
   constexpr int kWarps = warps_per_cta<G, FG>();
+  static_assert(kWarps * sizeof(WarpSmem<G, FG>) <= 232448, "a CTA's warps exceed 227 KB of shared memory");
   const int smem = kWarps * static_cast<int>(sizeof(WarpSmem<G, FG>));
   cudaError_t e = cudaFuncSetAttribute(decode_kernel<BITS, G, false, FG>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   if constexpr (!FG) {
     e = cudaFuncSetAttribute(decode_kernel<BITS, G, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(decode_kernel<BITS, G, false, false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             smem);
     if (e != cudaSuccess) return e;
   }
   int dev = 0, sms = 0, occ = 0;
@@ -1794,11 +2051,14 @@ cudaError_t plan_for(DecodePlan* plan, int fine) {
 template <int BITS, int G>
 cudaError_t launch_for(const DecodeArgs& a, const DecodePlan& plan, cudaStream_t stream) {
   if (a.workers < 1 || a.workers > plan.workers() || a.total_units < a.workers) return cudaErrorInvalidValue;
+  if (a.flush_blk >= 0 && (a.fine || a.k_res_coded)) return cudaErrorInvalidValue;
   const int ctas = (a.workers + plan.warps_per_cta - 1) / plan.warps_per_cta;
   if (a.fine) {
     decode_kernel<BITS, G, false, true><<<ctas, plan.warps_per_cta * 32, plan.smem_bytes, stream>>>(a);
   } else if (a.k_res_coded) {
     decode_kernel<BITS, G, true><<<ctas, plan.warps_per_cta * 32, plan.smem_bytes, stream>>>(a);
+  } else if (a.flush_blk >= 0) {
+    decode_kernel<BITS, G, false, false, true><<<ctas, plan.warps_per_cta * 32, plan.smem_bytes, stream>>>(a);
   } else {
     decode_kernel<BITS, G, false><<<ctas, plan.warps_per_cta * 32, plan.smem_bytes, stream>>>(a);
   }

@@ -87,6 +87,12 @@ struct DecodeArgs {
   // fine-grained groups (2 bits, one query per KV head): k_scale / k_zero [bh][C >> lg_gk][128]
   // (lg_gk: tokens per K group), v_scale / v_zero [bh][C][128 >> lg_gv] (lg_gv: channels per V group)
   int fine;
+  // in-launch flush (decode step whose appended token fills the residual, base groups only): the R
+  // residual tokens become quantized block flush_blk (< 0: no flush), written through these
+  // pointers to the arrays above.  No unit of the launch reads that block.
+  int flush_blk;
+  uint32_t *fk_codes, *fv_codes;
+  uint16_t *fk_scale, *fk_zero, *fv_scale, *fv_zero;
 };
 
 constexpr int kPartialStride = 132;  // m, l, Z, pad, o[128]

@@ -335,10 +335,12 @@ namespace {
 
 // Decode attention over `cache` (whose counters already include a fused append's token, which
 // k_new / v_new hold for residual slot new_slot; new_slot < 0: no append; -2: check the
-// arguments only and enqueue nothing).
+// arguments only and enqueue nothing).  flush: the appended token fills the residual, and the same
+// launch quantizes the residual as block n_quant / R (the caller updates the counters).
 int decode_impl(const kivi_config* cfg, const kivi_cache* cache, const uint16_t* q_dev, int32_t num_q_heads,
                 float scale, uint16_t* out_dev, void* workspace_dev, size_t workspace_bytes, int32_t* dev_status,
-                void* stream, const uint16_t* k_new_dev, const uint16_t* v_new_dev, int new_slot) {
+                void* stream, const uint16_t* k_new_dev, const uint16_t* v_new_dev, int new_slot,
+                bool flush = false) {
   int st = check_cfg(cfg);
   if (st != KIVI_OK) return st;
   if ((st = check_state(cfg, cache)) != KIVI_OK) return st;
@@ -422,6 +424,20 @@ int decode_impl(const kivi_config* cfg, const kivi_cache* cache, const uint16_t*
   a.k_res_coded = coded_res ? 1 : 0;
   a.fine = cfg->fine_groups;
   a.res_blk = cache->n_quant / cfg->residual;
+  a.flush_blk = -1;
+  if (flush) {  // the caller passes only full residuals of the base groups with fp16 residual keys
+    if ((new_slot != -2 && new_slot != cfg->residual - 1) || cache->n_res != cfg->residual || coded_res || cfg->fine_groups ||
+        cache->n_quant + cfg->residual > cfg->capacity)
+      return KIVI_ERR_INTERNAL;
+    if (!cache_ptrs_ok(cache, true)) return KIVI_ERR_INVALID_ARG;
+    a.flush_blk = cache->n_quant / cfg->residual;
+    a.fk_codes = cache->k_codes;
+    a.fv_codes = cache->v_codes;
+    a.fk_scale = cache->k_scale;
+    a.fk_zero = cache->k_zero;
+    a.fv_scale = cache->v_scale;
+    a.fv_zero = cache->v_zero;
+  }
   if (new_slot == -2) return KIVI_OK;  // arguments checked, nothing enqueued
   if (kivi::launch_decode(a, cfg->bits, plan, static_cast<cudaStream_t>(stream)) != cudaSuccess)
     return KIVI_ERR_CUDA;
@@ -465,6 +481,52 @@ int kivi_append_decode_attention(const kivi_config* cfg, kivi_cache* cache, cons
   st = decode_impl(cfg, &after, q_dev, num_q_heads, scale, out_dev, workspace_dev, workspace_bytes, dev_status,
                    stream, k_new_dev, v_new_dev, cache->n_res);
   if (st == KIVI_OK) cache->n_res += 1;
+  return st;
+}
+
+int kivi_decode_step(const kivi_config* cfg, kivi_cache* cache, const uint16_t* k_new_dev, const uint16_t* v_new_dev,
+                     const uint16_t* q_dev, int32_t num_q_heads, float scale, uint16_t* out_dev, void* workspace_dev,
+                     size_t workspace_bytes, int32_t* dev_status, void* stream) {
+  int st = check_cfg(cfg);
+  if (st != KIVI_OK) return st;
+  if ((st = check_state(cfg, cache)) != KIVI_OK) return st;
+  if (!aligned16(k_new_dev) || !aligned16(v_new_dev) || !cache_ptrs_ok(cache, false)) return KIVI_ERR_INVALID_ARG;
+  const int R = cfg->residual;
+  // the state the append sees: a residual left full by an earlier call is flushed first
+  kivi_cache cur = *cache;
+  const bool pre_flush = cur.n_res == R;
+  if (pre_flush) {
+    if (cur.n_quant + R > cfg->capacity) return KIVI_ERR_CAPACITY;
+    if (!cache_ptrs_ok(cache, true)) return KIVI_ERR_INVALID_ARG;
+    cur.n_quant += R;
+    cur.n_res = 0;
+  }
+  const bool online = k_online(cfg, cur.n_quant);
+  if (online && cur.n_quant + R > cfg->capacity) return KIVI_ERR_CAPACITY;
+  const bool flush = cur.n_res + 1 == R && cur.n_quant + R <= cfg->capacity;
+  // online K past the first block, and fine-grained groups, flush with their own launch
+  const bool fused_flush = flush && !online && !cfg->fine_groups;
+  // every argument check of the attention, on the state it will see, before anything is enqueued
+  kivi_cache after = cur;
+  after.n_res += 1;
+  st = decode_impl(cfg, &after, q_dev, num_q_heads, scale, out_dev, workspace_dev, workspace_bytes, dev_status, stream,
+                   nullptr, nullptr, -2, fused_flush);
+  if (st != KIVI_OK) return st;
+  if (pre_flush && (st = kivi_flush_residual(cfg, cache, stream)) != KIVI_OK) return st;
+  if (!fused_flush) {
+    st = kivi_append_decode_attention(cfg, cache, k_new_dev, v_new_dev, q_dev, num_q_heads, scale, out_dev,
+                                      workspace_dev, workspace_bytes, dev_status, stream);
+    if (st == KIVI_OK && flush) st = kivi_flush_residual(cfg, cache, stream);
+    return st;
+  }
+  after = *cache;
+  after.n_res += 1;
+  st = decode_impl(cfg, &after, q_dev, num_q_heads, scale, out_dev, workspace_dev, workspace_bytes, dev_status, stream,
+                   k_new_dev, v_new_dev, cache->n_res, true);
+  if (st == KIVI_OK) {
+    cache->n_quant += R;
+    cache->n_res = 0;
+  }
   return st;
 }
 

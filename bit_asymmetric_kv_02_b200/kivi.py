@@ -72,6 +72,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "kivi_decode_workspace_bytes": (SZ, [cfgp, I32]),
         "kivi_decode_attention": (I32, [cfgp, cachep, P, I32, ctypes.c_float, P, P, SZ, P, P]),
         "kivi_append_decode_attention": (I32, [cfgp, cachep, P, P, P, I32, ctypes.c_float, P, P, SZ, P, P]),
+        "kivi_decode_step": (I32, [cfgp, cachep, P, P, P, I32, ctypes.c_float, P, P, SZ, P, P]),
         "kivi_decode_attention_noalloc": (I32, [cfgp, cachep, P, I32, ctypes.c_float, P, P, P]),
         "kivi_read_status": (I32, [P, P]),
         "kivi_debug_inject": (I32, [I32, U64]),
@@ -146,6 +147,13 @@ def kivi_append_decode_attention(cfg, cache, k_new_ptr: int, v_new_ptr: int, q_p
                                                        q_ptr, num_q_heads, scale, out_ptr, ws_ptr, ws_bytes,
                                                        status_ptr, stream),
            "kivi_append_decode_attention")
+
+
+def kivi_decode_step(cfg, cache, k_new_ptr: int, v_new_ptr: int, q_ptr: int, num_q_heads: int, scale: float,
+                     out_ptr: int, ws_ptr: int, ws_bytes: int, status_ptr: int | None, stream: int) -> None:
+    _check(load_library().kivi_decode_step(ctypes.byref(cfg), ctypes.byref(cache), k_new_ptr, v_new_ptr, q_ptr,
+                                           num_q_heads, scale, out_ptr, ws_ptr, ws_bytes, status_ptr, stream),
+           "kivi_decode_step")
 
 
 def kivi_decode_attention_noalloc(cfg, cache, q_ptr: int, num_q_heads: int, scale: float, out_ptr: int,
@@ -272,6 +280,17 @@ class KiviCache:
         kivi_append_decode_attention(self.cfg, self.c, k_new.data_ptr(), v_new.data_ptr(), q.data_ptr(), q.shape[1],
                                      scale, out.data_ptr(), self.ws_ptr, self.ws_bytes,
                                      self.status.data_ptr() if status else None, self._stream(stream))
+        return out
+
+    def step(self, k_new, v_new, q, out=None, scale: float | None = None, stream=None, status: bool = True):
+        """One streaming decode step: append(k_new, v_new), attend(q), and quantize the residual in
+        the same launch when this token fills it (kivi_decode_step)."""
+        if out is None:
+            out = self.torch.empty_like(q)
+        scale = 1.0 / math.sqrt(self.cfg.head_dim) if scale is None else scale
+        kivi_decode_step(self.cfg, self.c, k_new.data_ptr(), v_new.data_ptr(), q.data_ptr(), q.shape[1], scale,
+                         out.data_ptr(), self.ws_ptr, self.ws_bytes, self.status.data_ptr() if status else None,
+                         self._stream(stream))
         return out
 
     def read_status(self, stream=None) -> int:

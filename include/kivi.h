@@ -57,7 +57,7 @@
 extern "C" {
 #endif
 
-#define KIVI_ABI_VERSION 3
+#define KIVI_ABI_VERSION 4
 
 /* Status codes. */
 #define KIVI_OK 0
@@ -214,6 +214,30 @@ int kivi_append_decode_attention(const kivi_config* cfg, kivi_cache* cache, cons
                                  const uint16_t* v_new_dev, const uint16_t* q_dev, int32_t num_q_heads,
                                  float scale, uint16_t* out_dev, void* workspace_dev, size_t workspace_bytes,
                                  int32_t* dev_status, void* stream);
+
+/*
+ * One streaming decode step: append one token, attend, and quantize the residual as soon as it is
+ * full.  Section 残差バッファ: the newest tokens stay fp16 and R of them become one quantized block
+ * (the quantization of sections 量子化アルゴリズム, Per-Channel量子化 and Per-Token量子化).  The
+ * attention output is that of kivi_append_decode_attention(k_new, v_new, q); in addition, when
+ * the appended token fills the residual (n_res becomes R) and n_quant + R <= capacity, the same
+ * launch quantizes the R residual tokens as block n_quant / R, bit-exactly as kivi_flush_residual
+ * would, and on success the counters become n_quant + R and n_res = 0.  The flush is eager (at the
+ * step that fills the residual) rather than lazy (at the next step): the outputs of every step are
+ * the same either way, since the step that fills the residual attends its tokens in fp16 and the
+ * next one attends the new block.
+ * Launches: one per step, flush steps included, for the base groups while the residual keys are
+ * fp16.  With online_k and n_quant > 0 (and with fine_groups) the step enqueues
+ * kivi_append_decode_attention and, on a filling step, kivi_flush_residual.  A residual that is
+ * already full when the call starts (left by other calls) is flushed first, by its own launch.
+ * Arguments: those of kivi_append_decode_attention.  Errors: those of the calls it stands for,
+ * checked before anything is enqueued; CAPACITY when the residual is full at entry and cannot be
+ * flushed.  When the residual fills and no block is left (n_quant + R > capacity) the step attends
+ * and leaves n_res = R; the next step then returns CAPACITY.
+ */
+int kivi_decode_step(const kivi_config* cfg, kivi_cache* cache, const uint16_t* k_new_dev, const uint16_t* v_new_dev,
+                     const uint16_t* q_dev, int32_t num_q_heads, float scale, uint16_t* out_dev, void* workspace_dev,
+                     size_t workspace_bytes, int32_t* dev_status, void* stream);
 
 /*
  * Largest scratch kivi_decode_attention_noalloc can use, in bytes (see below).

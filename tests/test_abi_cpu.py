@@ -33,7 +33,7 @@ def test_every_declared_symbol_is_exported(kivi):
 
 
 def test_version_and_strerror(kivi):
-    assert kivi.kivi_abi_version() == 3
+    assert kivi.kivi_abi_version() == 4
     assert kivi.kivi_strerror(0) == "ok"
     assert "flush" in kivi.kivi_strerror(4)
     assert kivi.kivi_strerror(12345) == "unknown status"

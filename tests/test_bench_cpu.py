@@ -2,6 +2,8 @@
 valid JSON line with the contract's keys."""
 import json
 import os
+
+import pytest
 import py_compile
 import subprocess
 import sys
@@ -60,36 +62,55 @@ def test_algorithmic_bytes_match_the_buffer_layout():
         bench.ONLINE_K, bench.FINE = saved
 
 
-def test_parity_replay_follows_the_bench_cycle():
-    """bench.oracle_parity replays prefill, flushes (with the n_quant cycle) and appends of a step
-    schedule; it accepts the oracle's own output for that schedule and rejects a perturbed one."""
+@pytest.mark.parametrize("mode", ["step", "fused"])
+def test_parity_replay_follows_the_bench_cycle(mode):
+    """bench.oracle_parity replays prefill, flushes (with the n_quant cycle of the mode) and appends
+    of a step schedule; it accepts the oracle's own output for that schedule and rejects a
+    perturbed one.  The decode step ("step") flushes the residual into the block after
+    n_quant0 + R and drops that block; the lazy mode moves n_quant back to n_quant0 and rewrites
+    the cycle's block."""
     sys.path.insert(0, ROOT)
     import numpy as np
 
     import bench
     import oracle.kivi_oracle as O
     from bit_asymmetric_kv_02_b200 import synth
-    w = synth.TINY.with_(batch=2, q_heads=4, kv_heads=2, tokens=300)
-    n_quant0, cap = bench.first_prompt_split(w)
-    sched = [(i % 128) + 1 for i in range(3 * 128 + 5)]
-    out = np.zeros((w.batch, w.q_heads, w.head_dim), np.float16)
-    for b in range(w.batch):
-        for h in range(w.kv_heads):
-            hc = O.HeadCache(128, 2, 32, 32, 128, cap)
-            hc.prefill(synth.prompt_k(w, b, h, w.tokens), synth.prompt_v(w, b, h, w.tokens))
-            for sid in sched:
-                if hc.n_res == 128:
-                    if hc.n_quant == n_quant0 + 128:     # the bench's cycle, written out here
-                        hc.k_codes, hc.v_codes = hc.k_codes[:n_quant0], hc.v_codes[:n_quant0]
-                        hc.k_s, hc.k_z = hc.k_s[:n_quant0 // 128], hc.k_z[:n_quant0 // 128]
-                        hc.v_s, hc.v_z = hc.v_s[:n_quant0 // 32], hc.v_z[:n_quant0 // 32]
-                    hc.flush()
-                hc.append(synth.new_k(w, b, h, sid), synth.new_v(w, b, h, sid))
-            assert hc.n_quant <= cap
-            q = np.stack([synth.query(w, b, 2 * h + g, sched[-1]) for g in range(2)])
-            out[b, 2 * h:2 * h + 2] = hc.attend(q, 1 / np.sqrt(128)).astype(np.float16)
-    state = {"out": out, "schedule": sched, "n_quant0": n_quant0}
-    rep = bench.oracle_parity(w, state, n_heads=4)
-    assert rep["ok"] and rep["heads"] == 4 and rep["steps_replayed"] == len(sched), rep
-    bad = dict(state, out=out + np.float16(0.01))
-    assert not bench.oracle_parity(w, bad, n_heads=4)["ok"]
+    saved = bench.MODE
+    bench.MODE = mode
+    try:
+        w = synth.TINY.with_(batch=2, q_heads=4, kv_heads=2, tokens=300)
+        n_quant0, cap = bench.first_prompt_split(w)
+        assert cap == n_quant0 + (2 if mode == "step" else 1) * 128
+        sched = [(i % 128) + 1 for i in range(3 * 128 + 5)]
+        out = np.zeros((w.batch, w.q_heads, w.head_dim), np.float16)
+
+        def keep(hc, n):     # the bench's cycle, written out here
+            hc.k_codes, hc.v_codes = hc.k_codes[:n], hc.v_codes[:n]
+            hc.k_s, hc.k_z = hc.k_s[:n // 128], hc.k_z[:n // 128]
+            hc.v_s, hc.v_z = hc.v_s[:n // 32], hc.v_z[:n // 32]
+
+        for b in range(w.batch):
+            for h in range(w.kv_heads):
+                hc = O.HeadCache(128, 2, 32, 32, 128, cap)
+                hc.prefill(synth.prompt_k(w, b, h, w.tokens), synth.prompt_v(w, b, h, w.tokens))
+                for sid in sched:
+                    if hc.n_res == 128:
+                        if mode == "step":
+                            hc.flush()
+                            if hc.n_quant == n_quant0 + 256:
+                                keep(hc, n_quant0 + 128)
+                        else:
+                            if hc.n_quant == n_quant0 + 128:
+                                keep(hc, n_quant0)
+                            hc.flush()
+                    hc.append(synth.new_k(w, b, h, sid), synth.new_v(w, b, h, sid))
+                    assert hc.n_quant in (n_quant0, n_quant0 + 128)
+                q = np.stack([synth.query(w, b, 2 * h + g, sched[-1]) for g in range(2)])
+                out[b, 2 * h:2 * h + 2] = hc.attend(q, 1 / np.sqrt(128)).astype(np.float16)
+        state = {"out": out, "schedule": sched, "n_quant0": n_quant0}
+        rep = bench.oracle_parity(w, state, n_heads=4)
+        assert rep["ok"] and rep["heads"] == 4 and rep["steps_replayed"] == len(sched), rep
+        bad = dict(state, out=out + np.float16(0.01))
+        assert not bench.oracle_parity(w, bad, n_heads=4)["ok"]
+    finally:
+        bench.MODE = saved
