@@ -280,6 +280,17 @@ __device__ __forceinline__ void cp_async_wait_all() {
   asm volatile("cp.async.commit_group;\n cp.async.wait_group 0;" ::: "memory");
 }
 
+// fp16 extremes of 8 values, both halves of a half2 (exact: min and max of fp16 values)
+__device__ __forceinline__ void minmax_h2(const uint4& v, __half2& lo, __half2& hi) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const __half2 x = *reinterpret_cast<const __half2*>(&w[i]);
+    lo = __hmin2(lo, x);
+    hi = __hmax2(hi, x);
+  }
+}
+
 template <int BITS>
 struct Flusher {
   static constexpr int L = (1 << BITS) - 1;  // largest code
@@ -295,6 +306,12 @@ struct Flusher {
                                           : (v ? a.v_res : a.k_res) +
                                                 (static_cast<size_t>(head) * a.residual + t) * kHeadDim;
     return reinterpret_cast<const uint4*>(row) + chunk;
+  }
+  // (s, z) of a group from the lanes' fp16 extremes
+  __device__ __forceinline__ GroupParams group_of(__half2 lo, __half2 hi) const {
+    const float l = warp_min(fminf(__low2float(lo), __high2float(lo)));
+    const float h = warp_max(fmaxf(__low2float(hi), __high2float(hi)));
+    return make_group(l, h, L);
   }
   // stage[k][lane] = chunk `chunk` of token tok(k), k < kStage
   template <typename Tok>
@@ -313,13 +330,13 @@ struct Flusher {
     const int R = a.residual, cpr = (1 << a.lg_gk) >> 3, slots = 32 / cpr;
     const int c = lane % cpr, s = lane / cpr, nt = R / slots;  // nt: the lane's tokens, a multiple of 16
     const int chunk = (gi << (a.lg_gk - 3)) + c;  // chunk of the row (8 channels each)
-    float lo = INFINITY, hi = -INFINITY;
+    __half2 lo = __float2half2_rn(INFINITY), hi = __float2half2_rn(-INFINITY);
     for (int k0 = 0; k0 < nt; k0 += kStage) {
       fill(false, head, chunk, [&](int k) { return s + slots * (k0 + k); });
 #pragma unroll
-      for (int k = 0; k < kStage; ++k) minmax8(stage[k * 32 + lane], lo, hi);
+      for (int k = 0; k < kStage; ++k) minmax_h2(stage[k * 32 + lane], lo, hi);
     }
-    const GroupParams g = make_group(warp_min(lo), warp_max(hi), L);
+    const GroupParams g = group_of(lo, hi);
     const size_t C = static_cast<size_t>(a.capacity);
     const int ngk = kHeadDim >> a.lg_gk;
     if (lane == 0) {
@@ -328,19 +345,16 @@ struct Flusher {
       a.fk_zero[si] = g.z_bits;
     }
     uint32_t* dst = a.fk_codes + (static_cast<size_t>(head) * C + static_cast<size_t>(a.flush_blk) * R) * (kHeadDim / P);
+    Thresh2 th;
+    if constexpr (BITS == 2) th = make_thresh2(g);
     for (int k0 = 0; k0 < nt; k0 += kStage) {
       if (nt > kStage) fill(false, head, chunk, [&](int k) { return s + slots * (k0 + k); });
 #pragma unroll 4
       for (int k = 0; k < kStage; ++k) {
         const int t = s + slots * (k0 + k);
         const uint4 v = stage[k * 32 + lane];
-        uint32_t part = 0u;  // the chunk's 8 codes at their bits of the word
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          uint32_t qa, qb;
-          quantize_pair(comp(v, e), g, L, qa, qb);
-          part |= (qa << (BITS * 2 * e)) | (qb << (BITS * (2 * e + 1)));
-        }
+        // the chunk's 8 codes at their bits of the word
+        uint32_t part = BITS == 2 ? row_codes2(v, th) : quantize_row8<BITS>(v, g);
         if constexpr (BITS == 2) {  // word = chunks 2 w and 2 w + 1
           part <<= 16 * (c & 1);
           part |= __shfl_xor_sync(kFull, part, 1);
@@ -359,13 +373,13 @@ struct Flusher {
     const int R = a.residual, gv = 1 << a.lg_gv, nslab = gv >> 5;
     const int c = lane & 15, h = lane >> 4;
     const int t0 = vg * gv + 16 * h;
-    float lo = INFINITY, hi = -INFINITY;
+    __half2 lo = __float2half2_rn(INFINITY), hi = __float2half2_rn(-INFINITY);
     for (int sl = 0; sl < nslab; ++sl) {
       fill(true, head, c, [&](int k) { return t0 + 32 * sl + k; });
 #pragma unroll
-      for (int k = 0; k < kStage; ++k) minmax8(stage[k * 32 + lane], lo, hi);
+      for (int k = 0; k < kStage; ++k) minmax_h2(stage[k * 32 + lane], lo, hi);
     }
-    const GroupParams g = make_group(warp_min(lo), warp_max(hi), L);
+    const GroupParams g = group_of(lo, hi);
     const size_t C = static_cast<size_t>(a.capacity);
     const size_t T0 = static_cast<size_t>(a.flush_blk) * R;  // first token of the block
     if (lane == 0) {
@@ -373,6 +387,8 @@ struct Flusher {
       a.fv_scale[si] = g.s_bits;
       a.fv_zero[si] = g.z_bits;
     }
+    Thresh2 th;
+    if constexpr (BITS == 2) th = make_thresh2(g);
     for (int sl = 0; sl < nslab; ++sl) {
       if (nslab > 1) fill(true, head, c, [&](int k) { return t0 + 32 * sl + k; });
       uint32_t w[16 / P][8];
@@ -380,15 +396,33 @@ struct Flusher {
       for (int r = 0; r < 16 / P; ++r)
 #pragma unroll
         for (int e = 0; e < 8; ++e) w[r][e] = 0u;
+      if constexpr (BITS == 2) {
+        // tokens 2 a, 2 a + 1 of channels 2 e, 2 e + 1 -> one word of four byte codes; then per
+        // channel the bytes of four tokens -> one 8-bit field (token k at bits 2 k)
 #pragma unroll
-      for (int k = 0; k < kStage; ++k) {
-        const uint4 v = stage[k * 32 + lane];
+        for (int q4 = 0; q4 < 4; ++q4) {  // tokens 4 q4 .. 4 q4 + 3
+          uint4 v[4];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          uint32_t qa, qb;
-          quantize_pair(comp(v, e), g, L, qa, qb);
-          w[k / P][2 * e] |= qa << (BITS * (k % P));
-          w[k / P][2 * e + 1] |= qb << (BITS * (k % P));
+          for (int i = 0; i < 4; ++i) v[i] = stage[(4 * q4 + i) * 32 + lane];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const uint32_t A0 = __byte_perm(codes2_h2(comp(v[0], e), th), codes2_h2(comp(v[1], e), th), 0x6240);
+            const uint32_t A1 = __byte_perm(codes2_h2(comp(v[2], e), th), codes2_h2(comp(v[3], e), th), 0x6240);
+            w[0][2 * e] |= gather4x2(__byte_perm(A0, A1, 0x5410)) << (8 * q4);
+            w[0][2 * e + 1] |= gather4x2(__byte_perm(A0, A1, 0x7632)) << (8 * q4);
+          }
+        }
+      } else {
+#pragma unroll
+        for (int k = 0; k < kStage; ++k) {
+          const uint4 v = stage[k * 32 + lane];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            uint32_t qa, qb;
+            quantize_pair(comp(v, e), g, L, qa, qb);
+            w[k / P][2 * e] |= qa << (BITS * (k % P));
+            w[k / P][2 * e + 1] |= qb << (BITS * (k % P));
+          }
         }
       }
 #pragma unroll

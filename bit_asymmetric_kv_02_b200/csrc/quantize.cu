@@ -219,10 +219,6 @@ __device__ __forceinline__ __half2 tile_min_negmax(const uint4 (&x)[kTileTokens]
   return __halves2half2(__hmin(__low2half(lo), __high2half(lo)), __hneg(__hmax(__low2half(hi), __high2half(hi))));
 }
 
-__device__ __forceinline__ uint32_t comp4(const uint4& v, int i) {
-  return i == 0 ? v.x : (i == 1 ? v.y : (i == 2 ? v.z : v.w));
-}
-
 __device__ __forceinline__ __half2 shfl_xor_h2(__half2 v, int off) {
   const uint32_t u = __shfl_xor_sync(0xffffffffu, *reinterpret_cast<uint32_t*>(&v), off);
   return *reinterpret_cast<const __half2*>(&u);
@@ -230,79 +226,6 @@ __device__ __forceinline__ __half2 shfl_xor_h2(__half2 v, int off) {
 
 __device__ __forceinline__ GroupParams group_from_pair(__half2 m, int levels) {
   return make_group(__low2float(m), -__high2float(m), levels);
-}
-
-// ---- 2 bits: the code as a count of thresholds ----------------------------------------------
-// For s > 0, Q(x) = clamp(rint((x - z)/s), 0, 3) with ties to even is [r > 1/2] + [r >= 3/2] +
-// [r > 5/2], r = (x - z)/s, i.e. [x > T0] + [x >= T1] + [x > T2] with T_k = z + (k + 1/2) s.  T_k is
-// exact in fp64.  Over fp16 x, x > T equals x > (largest fp16 <= T) and x >= T equals
-// x > (largest fp16 < T), so three strict fp16 comparisons decide the code exactly; s = 0 (all
-// codes 0) uses +inf.
-struct Thresh2 {
-  uint32_t t[3];  // each threshold in both halves of a half2
-};
-
-__device__ __forceinline__ uint16_t f64_to_h_rd(double x) {
-  uint16_t r;
-  asm("cvt.rm.f16.f64 %0, %1;" : "=h"(r) : "d"(x));
-  return r;
-}
-// The largest fp16 below the finite fp16 h.
-__device__ __forceinline__ uint16_t h_below(uint16_t h) {
-  if ((h & 0x7FFFu) == 0) return 0x8001u;  // below +-0: the negative subnormal closest to 0
-  return (h & 0x8000u) ? static_cast<uint16_t>(h + 1) : static_cast<uint16_t>(h - 1);
-}
-
-__device__ Thresh2 make_thresh2(const GroupParams& g) {
-  Thresh2 t;
-  const double s = static_cast<double>(h2f(g.s_bits)), z = static_cast<double>(g.zf);
-#pragma unroll
-  for (int k = 0; k < 3; ++k) {
-    uint16_t h = 0x7C00u;  // +inf
-    if (s > 0.0) {
-      const double T = z + (k + 0.5) * s;  // exact
-      h = f64_to_h_rd(T);
-      if (k == 1 && static_cast<double>(h2f(h)) == T) h = h_below(h);
-    }
-    t.t[k] = static_cast<uint32_t>(h) * 0x00010001u;
-  }
-  return t;
-}
-
-// Codes of one half2 as the half2 (1024 + c0, 1024 + c1): byte 0 holds c0 and byte 2 holds c1.
-__device__ __forceinline__ uint32_t codes2_h2(uint32_t x2, const Thresh2& t) {
-  const __half2 x = *reinterpret_cast<const __half2*>(&x2);
-  const __half2 t0 = *reinterpret_cast<const __half2*>(&t.t[0]);
-  const __half2 t1 = *reinterpret_cast<const __half2*>(&t.t[1]);
-  const __half2 t2 = *reinterpret_cast<const __half2*>(&t.t[2]);
-  const __half2 c = __hadd2(__hadd2(__hgt2(x, t0), __hgt2(x, t1)), __hadd2(__hgt2(x, t2), __float2half2_rn(1024.f)));
-  return *reinterpret_cast<const uint32_t*>(&c);
-}
-
-// Four 2-bit codes held one per byte -> an 8-bit field (byte i at bits 2 i).  The product with
-// 2^24 + 2^18 + 2^12 + 2^6 moves byte i to bit 24 + 2 i; every other partial product lands below
-// bit 24 (their sum stays below 2^24) or above bit 31.
-__device__ __forceinline__ uint32_t gather4x2(uint32_t bytes) { return (bytes * 0x01041040u) >> 24; }
-
-// 16-bit codes of the 8 channels of one token row, channel 8 c + j at bits 2 j.
-__device__ __forceinline__ uint32_t row_codes2(const uint4& v, const Thresh2& t) {
-  const uint32_t h0 = codes2_h2(v.x, t), h1 = codes2_h2(v.y, t), h2 = codes2_h2(v.z, t), h3 = codes2_h2(v.w, t);
-  return gather4x2(__byte_perm(h0, h1, 0x6420)) | (gather4x2(__byte_perm(h2, h3, 0x6420)) << 8);
-}
-
-// Codes of the 8 channels of one token row of a tile (bits BITS * j for channel 8 c + j).
-template <int BITS>
-__device__ __forceinline__ uint32_t quantize_row8(const uint4& v, const GroupParams& g) {
-  constexpr int L = (1 << BITS) - 1;
-  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-  uint32_t r = 0;
-#pragma unroll
-  for (int e = 0; e < 4; ++e) {
-    uint32_t qa, qb;
-    quantize_pair(w[e], g, L, qa, qb);
-    r += (qa << (BITS * 2 * e)) + (qb << (BITS * (2 * e + 1)));
-  }
-  return r;
 }
 
 template <int BITS>
@@ -466,15 +389,6 @@ __device__ __forceinline__ __half2 half2_of(const uint4& v, int i) {
 __device__ __forceinline__ uint32_t u32_of(__half2 h) { return *reinterpret_cast<const uint32_t*>(&h); }
 __device__ __forceinline__ __half2 h2_from(uint32_t u) { return *reinterpret_cast<const __half2*>(&u); }
 
-// Thresholds of two groups side by side: the low half from ga, the high half from gb.
-__device__ __forceinline__ Thresh2 thresh_pair(const GroupParams& ga, const GroupParams& gb) {
-  const Thresh2 ta = make_thresh2(ga), tb = make_thresh2(gb);
-  Thresh2 t;
-#pragma unroll
-  for (int k = 0; k < 3; ++k) t.t[k] = (ta.t[k] & 0xFFFFu) | (tb.t[k] & 0xFFFF0000u);
-  return t;
-}
-
 // Q of two elements with their own (s, z) (ga for the low half, gb for the high half).
 __device__ __forceinline__ void quantize_pair2(uint32_t hx2, const GroupParams& ga, const GroupParams& gb, int levels,
                                                uint32_t& qa, uint32_t& qb) {
@@ -491,11 +405,18 @@ __device__ __forceinline__ void quantize_pair2(uint32_t hx2, const GroupParams& 
   if (gb.inv_s == 0.f) qb = 0u;
 }
 
+// The code rule of one channel (fine K) or token (fine V) group: (s, z) and the 2-bit thresholds.
+struct ChanRule {
+  GroupParams g;
+  uint16_t t[3];
+};
+
 template <int BITS>
 __device__ void quantize_k_fine_tiles(const uint16_t* __restrict__ src, int lg_gk, uint32_t* __restrict__ codes,
                                       uint16_t* __restrict__ scale, uint16_t* __restrict__ zero) {
   constexpr int L = (1 << BITS) - 1;
   __shared__ uint4 red_lo[1024 / 32][16], red_hi[1024 / 32][16];
+  __shared__ ChanRule k_rule[256 / 32][kHeadDim];  // [K token group of the block][channel]
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int c = tid & 15, tg = tid >> 4;
   const uint4* s4 = reinterpret_cast<const uint4*>(src) + (tg * kTileTokens) * kChunks + c;
@@ -535,13 +456,34 @@ __device__ void quantize_k_fine_tiles(const uint16_t* __restrict__ src, int lg_g
       hi[i] = __hmax2(hi[i], h2_from(comp4(h4, i)));
     }
   }
+  // Every thread of the K group's tpg tiles that hold chunk c has the same extremes.  Thread `sub`
+  // forms (s, z) and the 2-bit thresholds of channels sub, sub + tpg (< 8) once and shares them.
+  const int tpg = 1 << (lg_gk - 3);  // token groups (tiles) of one K group
+  const int kg = tg >> (lg_gk - 3), sub = tg & (tpg - 1);
+  {
+    const uint4 l4 = make_uint4(u32_of(lo[0]), u32_of(lo[1]), u32_of(lo[2]), u32_of(lo[3]));
+    const uint4 h4 = make_uint4(u32_of(hi[0]), u32_of(hi[1]), u32_of(hi[2]), u32_of(hi[3]));
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const int j = sub + tpg * i;
+      if (j < 8) {
+        const __half2 lj = h2_from(comp4(l4, j >> 1)), hj = h2_from(comp4(h4, j >> 1));
+        const float lf = (j & 1) ? __high2float(lj) : __low2float(lj);
+        const float hf = (j & 1) ? __high2float(hj) : __low2float(hj);
+        ChanRule& cr = k_rule[kg][8 * c + j];
+        cr.g = make_group(lf, hf, L);
+        if constexpr (BITS == 2) {
+          const Thresh2 t = make_thresh2(cr.g);
+#pragma unroll
+          for (int k = 0; k < 3; ++k) cr.t[k] = static_cast<uint16_t>(t.t[k]);
+        }
+      }
+    }
+  }
+  __syncthreads();
   GroupParams gp[8];
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    gp[2 * i] = make_group(__low2float(lo[i]), __low2float(hi[i]), L);
-    gp[2 * i + 1] = make_group(__high2float(lo[i]), __high2float(hi[i]), L);
-  }
-  const int tpg = 1 << (lg_gk - 3);  // token groups (tiles) of one K group
+  for (int j = 0; j < 8; ++j) gp[j] = k_rule[kg][8 * c + j].g;
   if ((tg & (tpg - 1)) == 0) {       // the K group's first tile stores the pairs of its 8 channels
     const size_t row = static_cast<size_t>(tg >> (lg_gk - 3)) * kHeadDim + 8 * c;
     uint32_t sw[4], zw[4];
@@ -568,9 +510,13 @@ __device__ void quantize_k_fine_tiles(const uint16_t* __restrict__ src, int lg_g
       codes[(tok0 + k) * (kHeadDim / 8) + c] = r;
     }
   } else {  // K word c / 2 of a token: chunk 2i in bits 0..15, chunk 2i + 1 in bits 16..31
-    Thresh2 tp[4];
+    Thresh2 tp[4];  // thresholds of channels 2 i (low half) and 2 i + 1 (high half)
 #pragma unroll
-    for (int i = 0; i < 4; ++i) tp[i] = thresh_pair(gp[2 * i], gp[2 * i + 1]);
+    for (int i = 0; i < 4; ++i) {
+      const ChanRule &ra = k_rule[kg][8 * c + 2 * i], &rb = k_rule[kg][8 * c + 2 * i + 1];
+#pragma unroll
+      for (int k = 0; k < 3; ++k) tp[i].t[k] = static_cast<uint32_t>(ra.t[k]) | (static_cast<uint32_t>(rb.t[k]) << 16);
+    }
     uint32_t h[kTileTokens];
 #pragma unroll
     for (int k = 0; k < kTileTokens; ++k) {
@@ -602,7 +548,7 @@ __device__ void quantize_v_fine_tiles(const uint16_t* __restrict__ src, int lg_g
   // per-token extremes over the chunk's 8 channels, then over the g_v / 8 chunks of the channel
   // group (lanes c of one half warp)
   const int cpg = 1 << (lg_gv - 3);
-  GroupParams gp[kTileTokens];
+  uint32_t mw[kTileTokens];  // (min, -max) of each token's group, the same in all cpg lanes
 #pragma unroll
   for (int k = 0; k < kTileTokens; ++k) {
     __half2 lo = half2_of(x[k], 0), hi = lo;
@@ -613,15 +559,53 @@ __device__ void quantize_v_fine_tiles(const uint16_t* __restrict__ src, int lg_g
     }
     __half2 m = __halves2half2(__hmin(__low2half(lo), __high2half(lo)), __hneg(__hmax(__low2half(hi), __high2half(hi))));
     for (int off = 1; off < cpg; off <<= 1) m = __hmin2(m, shfl_xor_h2(m, off));
-    gp[k] = group_from_pair(m, L);
+    mw[k] = u32_of(m);
   }
   const int ngv = kHeadDim >> lg_gv, g = c >> (lg_gv - 3);
   const int tok0 = tg * kTileTokens;
-  if ((c & (cpg - 1)) == 0) {  // the group's first chunk stores the pairs of its 8 tokens
+  // Lane ci of the group's cpg lanes forms the rule of tokens ci, ci + cpg (< 8) once, stores their
+  // (s, z), and hands the rule to the other lanes by shuffles: 2 bits the three thresholds, 4 bits
+  // 1/s, z and the stored (s, z) bits.
+  const int ci = c & (cpg - 1);
+  const int lane = tid & 31;
+  uint32_t pa[2] = {0u, 0u}, pb[2] = {0u, 0u}, pc[2] = {0u, 0u};
 #pragma unroll
-    for (int k = 0; k < kTileTokens; ++k) {
-      scale[(tok0 + k) * ngv + g] = gp[k].s_bits;
-      zero[(tok0 + k) * ngv + g] = gp[k].z_bits;
+  for (int i = 0; i < 2; ++i) {
+    const int k = ci + cpg * i;
+    if (k < kTileTokens) {
+      const uint4 m4 = k < 4 ? make_uint4(mw[0], mw[1], mw[2], mw[3]) : make_uint4(mw[4], mw[5], mw[6], mw[7]);
+      const GroupParams gk = group_from_pair(h2_from(comp4(m4, k & 3)), L);
+      scale[(tok0 + k) * ngv + g] = gk.s_bits;
+      zero[(tok0 + k) * ngv + g] = gk.z_bits;
+      if constexpr (BITS == 2) {
+        const Thresh2 t = make_thresh2(gk);
+        pa[i] = (t.t[0] & 0xFFFFu) | (t.t[1] << 16);
+        pb[i] = t.t[2] & 0xFFFFu;
+      } else {
+        pa[i] = __float_as_uint(gk.inv_s);
+        pb[i] = __float_as_uint(gk.zf);
+        pc[i] = static_cast<uint32_t>(gk.s_bits) | (static_cast<uint32_t>(gk.z_bits) << 16);
+      }
+    }
+  }
+  GroupParams gp[kTileTokens];
+  Thresh2 t[kTileTokens];
+#pragma unroll
+  for (int k = 0; k < kTileTokens; ++k) {
+    const int src_lane = (lane & ~(cpg - 1)) | (k & (cpg - 1));
+    const bool second = k >= cpg;
+    const uint32_t a = __shfl_sync(0xffffffffu, second ? pa[1] : pa[0], src_lane);
+    const uint32_t b = __shfl_sync(0xffffffffu, second ? pb[1] : pb[0], src_lane);
+    if constexpr (BITS == 2) {
+      t[k].t[0] = (a & 0xFFFFu) * 0x00010001u;
+      t[k].t[1] = (a >> 16) * 0x00010001u;
+      t[k].t[2] = (b & 0xFFFFu) * 0x00010001u;
+    } else {
+      const uint32_t sz = __shfl_sync(0xffffffffu, second ? pc[1] : pc[0], src_lane);
+      gp[k].inv_s = __uint_as_float(a);
+      gp[k].zf = __uint_as_float(b);
+      gp[k].s_bits = static_cast<uint16_t>(sz & 0xFFFFu);
+      gp[k].z_bits = static_cast<uint16_t>(sz >> 16);
     }
   }
   // codes of channel 8 c + e for the tile's 8 tokens, token k at bits BITS * k
@@ -642,9 +626,6 @@ __device__ void quantize_v_fine_tiles(const uint16_t* __restrict__ src, int lg_g
     dst[0] = make_uint4(col[0], col[1], col[2], col[3]);
     dst[1] = make_uint4(col[4], col[5], col[6], col[7]);
   } else {
-    Thresh2 t[kTileTokens];
-#pragma unroll
-    for (int k = 0; k < kTileTokens; ++k) t[k] = make_thresh2(gp[k]);
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
       uint32_t A[4];

@@ -91,10 +91,12 @@ def _run_steps(kivi, w, steps, cap, check_every=None, **kw):
         assert (step.n_quant, step.n_res) == (ref[heads[0]].n_quant, ref[heads[0]].n_res), f"step {s}"
         if check:
             for (b, h), hc in ref.items():
-                if kw.get("fine_groups") or kw.get("online_k"):
+                if kw.get("fine_groups") or kw.get("online_k"):   # rows as the oracle's buffers have them
                     want_buf = hc.packed()
-                    full = gc.gpu_buffers_of_head(step, b, h, step.cfg.capacity, step.cfg.residual)
-                    got = {key: full[key][:np.asarray(x).shape[0]] for key, x in want_buf.items()}
+                    got = {}
+                    for key, x in want_buf.items():
+                        rows = step.view(key)[b, h, :np.asarray(x).shape[0]].cpu().numpy()
+                        got[key] = rows.view(np.uint32) if key in ("k_codes", "v_codes") else rows
                     gc.assert_head_bitexact(got, want_buf, f"{w.name} step {s} head {(b, h)}")
                 else:
                     gc.assert_head_bitexact(gc.gpu_buffers_of_head(step, b, h, step.n_quant, step.n_res),
