@@ -481,22 +481,23 @@ __device__ void quantize_k_fine_tiles(const uint16_t* __restrict__ src, int lg_g
     }
   }
   __syncthreads();
-  GroupParams gp[8];
-#pragma unroll
-  for (int j = 0; j < 8; ++j) gp[j] = k_rule[kg][8 * c + j].g;
   if ((tg & (tpg - 1)) == 0) {       // the K group's first tile stores the pairs of its 8 channels
     const size_t row = static_cast<size_t>(tg >> (lg_gk - 3)) * kHeadDim + 8 * c;
     uint32_t sw[4], zw[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      sw[i] = static_cast<uint32_t>(gp[2 * i].s_bits) | (static_cast<uint32_t>(gp[2 * i + 1].s_bits) << 16);
-      zw[i] = static_cast<uint32_t>(gp[2 * i].z_bits) | (static_cast<uint32_t>(gp[2 * i + 1].z_bits) << 16);
+      const GroupParams &ga = k_rule[kg][8 * c + 2 * i].g, &gb = k_rule[kg][8 * c + 2 * i + 1].g;
+      sw[i] = static_cast<uint32_t>(ga.s_bits) | (static_cast<uint32_t>(gb.s_bits) << 16);
+      zw[i] = static_cast<uint32_t>(ga.z_bits) | (static_cast<uint32_t>(gb.z_bits) << 16);
     }
     *reinterpret_cast<uint4*>(scale + row) = make_uint4(sw[0], sw[1], sw[2], sw[3]);
     *reinterpret_cast<uint4*>(zero + row) = make_uint4(zw[0], zw[1], zw[2], zw[3]);
   }
   const int tok0 = tg * kTileTokens;
   if constexpr (BITS == 4) {  // K word c of a token is exactly the tile's 8 channels
+    GroupParams gp[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) gp[j] = k_rule[kg][8 * c + j].g;
 #pragma unroll
     for (int k = 0; k < kTileTokens; ++k) {
       const uint32_t w[4] = {x[k].x, x[k].y, x[k].z, x[k].w};
@@ -651,8 +652,9 @@ __device__ void quantize_v_fine_tiles(const uint16_t* __restrict__ src, int lg_g
 
 // grid: x = batch * kv_heads, y = 2 * nblocks (+1 residual-copy job); block = 2R threads (R <= 256:
 // the per-channel and per-token parameters need more than the 64 registers of a 1024-thread block)
-template <int BITS>
-__global__ void __launch_bounds__(512) quantize_fine_tiles_kernel(QuantizeArgs a) {
+// NT = 2R threads: 256 threads (R = 128) are held to 80 registers, so that three CTAs share an SM.
+template <int BITS, int NT>
+__global__ void __launch_bounds__(NT, NT == 256 ? 3 : 1) quantize_fine_tiles_kernel(QuantizeArgs a) {
   constexpr int P = 32 / BITS;
   const int bh = blockIdx.x;
   const int job = blockIdx.y;
@@ -991,10 +993,17 @@ cudaError_t launch_quantize_blocks(const QuantizeArgs& args, int bits, cudaStrea
   a.lg_gv = __builtin_ctz(static_cast<unsigned>(a.group_v));
   dim3 grid(a.bh, jobs);
   if (a.fine && a.residual <= 256) {  // one thread per 8 tokens x 8 channels of a block
-    if (bits == 2)
-      quantize_fine_tiles_kernel<2><<<grid, 2 * a.residual, 0, stream>>>(a);
-    else
-      quantize_fine_tiles_kernel<4><<<grid, 2 * a.residual, 0, stream>>>(a);
+    if (a.residual == 128) {
+      if (bits == 2)
+        quantize_fine_tiles_kernel<2, 256><<<grid, 256, 0, stream>>>(a);
+      else
+        quantize_fine_tiles_kernel<4, 256><<<grid, 256, 0, stream>>>(a);
+    } else {
+      if (bits == 2)
+        quantize_fine_tiles_kernel<2, 512><<<grid, 512, 0, stream>>>(a);
+      else
+        quantize_fine_tiles_kernel<4, 512><<<grid, 512, 0, stream>>>(a);
+    }
   } else if (a.fine) {
     if (bits == 2)
       quantize_fine_kernel<2><<<grid, kHeadDim, 0, stream>>>(a);

@@ -362,9 +362,9 @@ def test_full_size_large_batch_fused_all_heads():
 
 @pytest.mark.parametrize("bits,group", [(2, 32), (2, 128), (4, 32), (4, 128)])
 def test_full_size_streaming(bits, group):
-    """Prefill 32768 tokens, then 256 decode steps (flush when full, append, attend), every head:
-    buffers bit for bit after both flushes and at the checked steps, outputs within tolerance at
-    steps around the flushes."""
+    """Prefill 32768 tokens, then 256 decode steps (flush when full, append, attend; the second
+    flush inside kivi_decode_step's launch), every head: buffers bit for bit after both flushes and
+    at the checked steps, outputs within tolerance at steps around the flushes."""
     kivi = _kivi()
     w = synth.STREAMING.with_(bits=bits, group=group)
     cap = 33024
@@ -388,15 +388,24 @@ def test_full_size_streaming(bits, group):
                 _compare(label, _gpu_head_digests(cache, heads, shapes_of(label)), None, runs, w.gqa, w.name)
             kn, vn = synth.new_kv(w, s)
             q = synth.queries(w, s)
-            if s % 2:     # the fused call and the separate calls alternate
+            # the decode step (every third step, and step 128, whose token fills the residual and is
+            # flushed in the same launch), the fused call and the separate calls take turns
+            use_step = s % 3 == 0 or s == 128
+            if use_step:
+                out = cache.step(*(torch.from_numpy(x).cuda() for x in (kn, vn, q)))
+            elif s % 2:
                 out = cache.append_attend(*(torch.from_numpy(x).cuda() for x in (kn, vn, q)))
             else:
                 cache.append(torch.from_numpy(kn).cuda(), torch.from_numpy(vn).cuda())
                 out = cache.attend(torch.from_numpy(q).cuda())
+            flushed = use_step and cache.n_res == 0   # eager: the oracle's flush of the next step
+            if flushed:
+                label = f"flush before step {s + 1}"
+                _compare(label, _gpu_head_digests(cache, heads, shapes_of(label)), None, runs, w.gqa, w.name)
             if s in check_at:
                 label = f"step {s}"
-                _compare(label, _gpu_head_digests(cache, heads, shapes_of(label)), out.cpu().numpy(), runs, w.gqa,
-                         f"{w.name} {bits}-bit G={group}")
+                gpu = None if flushed else _gpu_head_digests(cache, heads, shapes_of(label))
+                _compare(label, gpu, out.cpu().numpy(), runs, w.gqa, f"{w.name} {bits}-bit G={group}")
     assert cache.read_status() == 0
     assert (cache.n_quant, cache.n_res) == (32896, 128)
 
