@@ -1679,44 +1679,59 @@ struct Decoder {
     }
     insert_new_row(kt, r, head, a.k_new, a.k_res, false);
     const int t = lane >> 1, hf = lane & 1;  // 2 lanes per token, 64 channels each
+    float dot[G];
 #pragma unroll
-    for (int g = 0; g < G; ++g) {
-      const uint4* qp = reinterpret_cast<const uint4*>(S.qraw[qslot(head)][g]);
-      float dot = 0.f;
-      // several queries read the scaled q from shared memory (start_head), two chunks at a time so
-      // that the loads of all queries are not in flight at once
-#pragma unroll(G == 1 ? 8 : 2)
+    for (int g = 0; g < G; ++g) dot[g] = 0.f;
+    if constexpr (G > 1) {
+      // several queries: each K chunk is read and converted once for all of them; q (scaled) comes
+      // from shared memory (start_head)
+#pragma unroll 2
       for (int k = 0; k < 8; ++k) {
         const int cc = (k + lane) & 7;  // bank-conflict-free chunk order
         const int c0 = 64 * hf + 8 * cc;
         const uint4 kv = *reinterpret_cast<const uint4*>(kt + t * 256 + 2 * c0);
         const uint32_t kw[4] = {kv.x, kv.y, kv.z, kv.w};
-        if constexpr (G > 1) {
+        float kf[8];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&kw[e]));
+          kf[2 * e] = f.x;
+          kf[2 * e + 1] = f.y;
+        }
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
           const float4 qa = *reinterpret_cast<const float4*>(&S.qs[G > 1 ? g : 0][G > 1 ? c0 : 0]);
           const float4 qb = *reinterpret_cast<const float4*>(&S.qs[G > 1 ? g : 0][G > 1 ? c0 + 4 : 0]);
           const float qf[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float2 kf = __half22float2(*reinterpret_cast<const __half2*>(&kw[e]));
-            dot = fmaf(qf[2 * e], kf.x, dot);
-            dot = fmaf(qf[2 * e + 1], kf.y, dot);
-          }
-        } else {
-          const uint4 qv = qp[c0 >> 3];
-          const uint32_t qw[4] = {qv.x, qv.y, qv.z, qv.w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float2 kf = __half22float2(*reinterpret_cast<const __half2*>(&kw[e]));
-            const float2 qf = __half22float2(*reinterpret_cast<const __half2*>(&qw[e]));
-            dot = fmaf(qf.x, kf.x, dot);
-            dot = fmaf(qf.y, kf.y, dot);
-          }
+          for (int e = 0; e < 8; ++e) dot[g] = fmaf(qf[e], kf[e], dot[g]);
         }
       }
-      dot += __shfl_xor_sync(kFull, dot, 1);
-      if (G == 1) dot *= a.qscale;  // several queries: q in shared memory is scaled already
+    } else {
+      const uint4* qp = reinterpret_cast<const uint4*>(S.qraw[qslot(head)][0]);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const int cc = (k + lane) & 7;  // bank-conflict-free chunk order
+        const int c0 = 64 * hf + 8 * cc;
+        const uint4 kv = *reinterpret_cast<const uint4*>(kt + t * 256 + 2 * c0);
+        const uint32_t kw[4] = {kv.x, kv.y, kv.z, kv.w};
+        const uint4 qv = qp[c0 >> 3];
+        const uint32_t qw[4] = {qv.x, qv.y, qv.z, qv.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 kf = __half22float2(*reinterpret_cast<const __half2*>(&kw[e]));
+          const float2 qf = __half22float2(*reinterpret_cast<const __half2*>(&qw[e]));
+          dot[0] = fmaf(qf.x, kf.x, dot[0]);
+          dot[0] = fmaf(qf.y, kf.y, dot[0]);
+        }
+      }
+    }
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      float d = dot[g] + __shfl_xor_sync(kFull, dot[g], 1);
+      if (G == 1) d *= a.qscale;  // several queries: q in shared memory is scaled already
       const bool valid = t < nvalid;
-      const float lg = valid ? dot : -INFINITY;
+      const float lg = valid ? d : -INFINITY;
       const float m_new = fmaxf(m[g], warp_max(lg));
       const float alpha = fast_exp2(m[g] - m_new);
       const float p = valid ? fast_exp2(lg - m_new) : 0.f;
@@ -1732,14 +1747,16 @@ struct Decoder {
   __device__ void residual_v(uint8_t* vt, int nvalid, long long head, int r) {
     insert_new_row(vt, r, head, a.v_new, a.v_res, true);
 #pragma unroll
-    for (int g = 0; g < G; ++g) {
+    for (int g = 0; g < G; ++g)
 #pragma unroll
       for (int e = 0; e < 4; ++e) o[g][e] *= alpha_[g];
-      for (int tt = 0; tt < nvalid; ++tt) {
+    for (int tt = 0; tt < nvalid; ++tt) {  // each row is read and converted once for every query
+      const uint2 vv = *reinterpret_cast<const uint2*>(vt + vrow(tt) + 8 * lane);
+      const float2 v0 = __half22float2(*reinterpret_cast<const __half2*>(&vv.x));
+      const float2 v1 = __half22float2(*reinterpret_cast<const __half2*>(&vv.y));
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
         const float pt = __shfl_sync(kFull, pres_[g], 2 * tt);
-        const uint2 vv = *reinterpret_cast<const uint2*>(vt + vrow(tt) + 8 * lane);
-        const float2 v0 = __half22float2(*reinterpret_cast<const __half2*>(&vv.x));
-        const float2 v1 = __half22float2(*reinterpret_cast<const __half2*>(&vv.y));
         o[g][0] = fmaf(pt, v0.x, o[g][0]);
         o[g][1] = fmaf(pt, v0.y, o[g][1]);
         o[g][2] = fmaf(pt, v1.x, o[g][2]);
