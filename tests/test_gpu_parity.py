@@ -231,6 +231,31 @@ def test_errors_through_the_abi():
     assert e.value.code == "WORKSPACE"
 
 
+@pytest.mark.parametrize("bits,kv_heads,q_heads,fine", [(2, 4, 4, False), (2, 2, 8, False), (4, 1, 8, False),
+                                                      (2, 3, 3, True), (4, 2, 4, True)])
+def test_workspace_size_rule_matches_the_decode(bits, kv_heads, q_heads, fine):
+    """kivi_decode_workspace_bytes is exactly what kivi_decode_attention (and the no-alloc entry's
+    ticket offset) requires: one byte less is refused with WORKSPACE, the size itself decodes."""
+    kivi = _kivi()
+    w = synth.TINY.with_(batch=2, q_heads=q_heads, kv_heads=kv_heads, tokens=300, bits=bits, seed=77)
+    k, v = synth.prompt_kv(w, w.tokens)
+    cache = kivi.KiviCache(w.batch, w.kv_heads, 384, bits=bits, num_q_heads=w.q_heads, fine_groups=fine)
+    cache.prefill(torch.from_numpy(k).cuda(), torch.from_numpy(v).cuda())
+    need = kivi.kivi_decode_workspace_bytes(cache.cfg, w.q_heads)
+    assert 0 < need <= cache.ws_bytes
+    q = torch.from_numpy(synth.queries(w)).cuda()
+    out = torch.empty_like(q)
+    stream = torch.cuda.current_stream().cuda_stream
+    with pytest.raises(kivi.KiviError) as e:
+        kivi.kivi_decode_attention(cache.cfg, cache.c, q.data_ptr(), w.q_heads, 0.1, out.data_ptr(), cache.ws_ptr,
+                                   need - 1, None, stream)
+    assert e.value.code == "WORKSPACE"
+    kivi.kivi_decode_attention(cache.cfg, cache.c, q.data_ptr(), w.q_heads, 0.1, out.data_ptr(), cache.ws_ptr, need,
+                               None, stream)
+    torch.cuda.synchronize()
+    assert torch.isfinite(out.float()).all()
+
+
 def test_device_timeout_is_reported_and_context_survives():
     """A barrier that can never complete (the test hook asks for 16 bytes more than are copied)
     makes every bounded wait run out: the kernel reports DEVICE_TIMEOUT and returns; afterwards
