@@ -2,10 +2,10 @@
 """Benchmark: 2-bit KIVI decode over a quantized KV cache on B200, one JSON line on stdout.
 
 A step is one streaming decode step of the large-batch workload (B=64, H=32, d=128, 2-bit, G=32,
-R=128): flush the residual when it is full (once every 128 steps), append one new K/V token per
-(batch, KV head), and run decode attention for every query head over the whole cache.  After each
-128-step cycle the host moves n_quant back by one block, so the cache cycles between 8193 and 8320
-cached tokens instead of growing; every step does its full work.  Inputs live in HBM (1.2 GB of codes
+R=128): append one new K/V token per (batch, KV head), run decode attention for every query head over
+the whole cache, and flush the residual once it is full (once every 128 steps; by default inside the
+same launch, kivi_decode_step).  After each 128-step cycle the host drops one block again, so the
+cache cycles between 8193 and 8320 cached tokens instead of growing; every step does its full work.  Inputs live in HBM (1.2 GB of codes
 and scales per step, ten times the 126 MB L2, so no L2 flush is needed; a workload smaller than twice
 the L2 rotates several cache replicas, one per step, so that a step finds its cache evicted).
 
@@ -545,11 +545,20 @@ def run_gpu(args, rank, world, local_rank, w: synth.Workload):
         for a, o0, o1 in zip(x, offs[:-1], offs[1:]):
             buf[o0:o1].copy_(torch.from_numpy(np.ascontiguousarray(a)).reshape(-1))
         pinned.append(buf)
-    stage_buf = torch.empty(int(offs[-1]), dtype=torch.float16, device=device)
-    stage = [stage_buf[o0:o1].view(sh) for o0, o1, sh in zip(offs[:-1], offs[1:], shapes)]
+    # two staging buffers: step i + 1's inputs cross PCIe on a copy stream while step i computes
+    stage_bufs = [torch.empty(int(offs[-1]), dtype=torch.float16, device=device) for _ in range(2)]
+    stages = [[sb[o0:o1].view(sh) for o0, o1, sh in zip(offs[:-1], offs[1:], shapes)] for sb in stage_bufs]
+    copy_stream = torch.cuda.Stream(device)
+    landed = [torch.cuda.Event(), torch.cuda.Event()]
     out_host = torch.empty(w.batch, w.q_heads, w.head_dim, dtype=torch.float16).pin_memory()
     h2d = int(offs[-1]) * 2
     d2h = out_host.numel() * out_host.element_size()
+
+    def copy_inputs(i):
+        """Step i's inputs into staging buffer i % 2, on the copy stream."""
+        with torch.cuda.stream(copy_stream):
+            stage_bufs[i % 2].copy_(pinned[i % R], non_blocking=True)
+            landed[i % 2].record(copy_stream)
 
     def e2e_loop(K):
         barrier()
@@ -558,9 +567,13 @@ def run_gpu(args, rank, world, local_rank, w: synth.Workload):
         toks = 0
         with torch.cuda.stream(stream):
             f0.record(stream)
+            copy_stream.wait_stream(stream)   # the first copy starts inside the timed region
+            copy_inputs(0)
             for i in range(K):
-                stage_buf.copy_(pinned[i % R], non_blocking=True)
-                toks += step(i % R, inputs=stage)[1]
+                stream.wait_event(landed[i % 2])
+                if i + 1 < K:   # buffer (i + 1) % 2 was read by step i - 1, which the last synchronize ended
+                    copy_inputs(i + 1)
+                toks += step(i % R, inputs=stages[i % 2])[1]
                 out_host.copy_(out, non_blocking=True)
                 stream.synchronize()      # the caller consumes the step's result
             f1.record(stream)

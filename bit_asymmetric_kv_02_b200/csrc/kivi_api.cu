@@ -504,6 +504,7 @@ int kivi_decode_step(const kivi_config* cfg, kivi_cache* cache, const uint16_t* 
   const bool online = k_online(cfg, cur.n_quant);
   if (online && cur.n_quant + R > cfg->capacity) return KIVI_ERR_CAPACITY;
   const bool flush = cur.n_res + 1 == R && cur.n_quant + R <= cfg->capacity;
+  if (flush && !cache_ptrs_ok(cache, true)) return KIVI_ERR_INVALID_ARG;  // the flush writes the block arrays
   // online K past the first block, and fine-grained groups, flush with their own launch
   const bool fused_flush = flush && !online && !cfg->fine_groups;
   // every argument check of the attention, on the state it will see, before anything is enqueued

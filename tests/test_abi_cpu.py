@@ -127,6 +127,33 @@ def test_state_errors_before_any_device_work(kivi):
     assert e.value.code == "CAPACITY"
 
 
+def test_decode_step_host_errors(kivi):
+    """kivi_decode_step checks everything on the host before it enqueues anything, and leaves the
+    counters unchanged on an error: misaligned rows, a full residual with no block left, a state
+    the configuration cannot hold, and (after those pass) the attention's own checks."""
+    cfg = _cfg(kivi)
+    fake = 1 << 20
+    cache = kivi.kivi_cache(*([fake] * 8), 0, 5)
+    with pytest.raises(kivi.KiviError) as e:
+        kivi.kivi_decode_step(cfg, cache, fake + 8, fake, fake, 3, 0.1, fake, fake, 1 << 30, None, 0)
+    assert e.value.code == "INVALID_ARG" and (cache.n_quant, cache.n_res) == (0, 5)
+    cache.n_quant, cache.n_res = 1024, 128       # full residual, every block used: no flush possible
+    with pytest.raises(kivi.KiviError) as e:
+        kivi.kivi_decode_step(cfg, cache, fake, fake, fake, 3, 0.1, fake, fake, 1 << 30, None, 0)
+    assert e.value.code == "CAPACITY" and (cache.n_quant, cache.n_res) == (1024, 128)
+    cache.n_quant, cache.n_res = 100, 5
+    with pytest.raises(kivi.KiviError) as e:
+        kivi.kivi_decode_step(cfg, cache, fake, fake, fake, 3, 0.1, fake, fake, 1 << 30, None, 0)
+    assert e.value.code == "STATE" and (cache.n_quant, cache.n_res) == (100, 5)
+    cache.n_quant = 0
+    with pytest.raises(kivi.KiviError) as e:      # 4 query heads over 3 KV heads
+        kivi.kivi_decode_step(cfg, cache, fake, fake, fake, 4, 0.1, fake, fake, 1 << 30, None, 0)
+    assert e.value.code == "INVALID_ARG" and (cache.n_quant, cache.n_res) == (0, 5)
+    with pytest.raises(kivi.KiviError) as e:      # a misaligned output
+        kivi.kivi_decode_step(cfg, cache, fake, fake, fake, 3, 0.1, fake + 2, fake, 1 << 30, None, 0)
+    assert e.value.code == "INVALID_ARG" and (cache.n_quant, cache.n_res) == (0, 5)
+
+
 def test_online_k_host_errors(kivi):
     """Online K (section Per-Channel量子化): the flag's rule and the capacity its block slot needs,
     checked on the host before anything is enqueued."""
