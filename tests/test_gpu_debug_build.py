@@ -2,8 +2,9 @@
 
 Its kernels check the index ranges of their global-memory accesses and report KIVI_ERR_INTERNAL
 instead of making an access that fails a check.  In a child process that loads the debug library:
-prefill, appends, flushes and decode attention (2 and 4 bits, one and four queries per KV head)
-leave every check quiet and match the oracle; then test hook 3 makes the decode see one quantized
+prefill, appends, flushes and decode attention, with every other step a decode step whose flush runs
+in its launch (2 and 4 bits, one and four queries per KV head), leave every check quiet and match the
+oracle; then test hook 3 makes the decode see one quantized
 unit more than the cache holds (inside the capacity, so the unguarded copy would stay in bounds
 too), and the kernel's check refuses it and reports KIVI_ERR_INTERNAL through the status word and
 kivi_debug_status, after which normal calls give the earlier results again.
@@ -48,12 +49,16 @@ for bits, gqa in ((2, 1), (4, 1), (2, 4)):
                 hc.flush()
         kn, vn = synth.new_kv(w, s)
         q = synth.queries(w, s)
-        out = c.append_attend(*(torch.from_numpy(x).cuda() for x in (kn, vn, q))).cpu().numpy()
+        call = c.step if s % 2 == 0 else c.append_attend   # step 40 fills the residual: flushed in the launch
+        out = call(*(torch.from_numpy(x).cuda() for x in (kn, vn, q))).cpu().numpy()
         for (b, h), hc in ref.items():
             hc.append(kn[b, h], vn[b, h])
-        if s in (1, 40, 139):
+        if s in (1, 40, 41, 139):
             for (b, h), hc in ref.items():
                 gc.assert_attention_close(out[b, h * gqa:(h + 1) * gqa], hc.attend(q[b, h * gqa:(h + 1) * gqa], gc.default_scale()), f"debug build {bits}-bit gqa {gqa} step {s}")
+        if s % 2 == 0 and c.n_res == 0:
+            for hc in ref.values():
+                hc.flush()
     assert c.read_status() == 0
     assert kivi.kivi_debug_status() == 0, "a check fired on valid calls"
     q = torch.from_numpy(synth.queries(w, 0)).cuda()

@@ -114,6 +114,17 @@ def test_step_equals_lazy_calls_and_oracle(w):
     assert _run_steps(kivi, w, steps, cap, check_every=41) == 2
 
 
+@pytest.mark.parametrize("bits", [2, 4])
+def test_step_largest_residual(bits):
+    """R = 1024: a K group job spans 128 tokens per lane slot and is staged eight times per pass."""
+    kivi = _kivi()
+    w = synth.TINY.with_(name=f"step_R1024_{bits}bit", batch=1, q_heads=2, kv_heads=2, tokens=1100, bits=bits,
+                         residual=1024, group_v=64, seed=141)
+    steps = 1024 + 3
+    cap = ((w.tokens + steps) // w.residual + 1) * w.residual
+    assert _run_steps(kivi, w, steps, cap, check_every=257) == 1
+
+
 def test_step_with_forced_splits():
     """Every head split over 5 warps, so one head's residual and its flush jobs land on different
     warps."""
