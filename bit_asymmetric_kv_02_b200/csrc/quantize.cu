@@ -405,10 +405,15 @@ __device__ __forceinline__ void quantize_pair2(uint32_t hx2, const GroupParams& 
   if (gb.inv_s == 0.f) qb = 0u;
 }
 
-// The code rule of one channel (fine K) or token (fine V) group: (s, z) and the 2-bit thresholds.
-struct ChanRule {
-  GroupParams g;
-  uint16_t t[3];
+// The code rules of the channels of the block's K token groups, one array per field ([K token
+// group][channel]), so that a thread reads its 8 channels' field with one 16-byte load: (s, z) bits,
+// and the 2-bit thresholds (bits = 2) or 1/s and z (bits = 4).  Two channels' 16-bit fields in one
+// word are exactly the (channel 2 i, 2 i + 1) pairs the codes and the scale rows use.
+template <int BITS>
+struct KRules {
+  uint16_t s[256 / 32][kHeadDim], z[256 / 32][kHeadDim];
+  uint16_t t[BITS == 2 ? 3 : 1][256 / 32][BITS == 2 ? kHeadDim : 1];
+  float inv_s[BITS == 4 ? 256 / 32 : 1][BITS == 4 ? kHeadDim : 1], zf[BITS == 4 ? 256 / 32 : 1][BITS == 4 ? kHeadDim : 1];
 };
 
 template <int BITS>
@@ -416,7 +421,7 @@ __device__ void quantize_k_fine_tiles(const uint16_t* __restrict__ src, int lg_g
                                       uint16_t* __restrict__ scale, uint16_t* __restrict__ zero) {
   constexpr int L = (1 << BITS) - 1;
   __shared__ uint4 red_lo[1024 / 32][16], red_hi[1024 / 32][16];
-  __shared__ ChanRule k_rule[256 / 32][kHeadDim];  // [K token group of the block][channel]
+  __shared__ __align__(16) KRules<BITS> kr;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int c = tid & 15, tg = tid >> 4;
   const uint4* s4 = reinterpret_cast<const uint4*>(src) + (tg * kTileTokens) * kChunks + c;
@@ -470,12 +475,17 @@ __device__ void quantize_k_fine_tiles(const uint16_t* __restrict__ src, int lg_g
         const __half2 lj = h2_from(comp4(l4, j >> 1)), hj = h2_from(comp4(h4, j >> 1));
         const float lf = (j & 1) ? __high2float(lj) : __low2float(lj);
         const float hf = (j & 1) ? __high2float(hj) : __low2float(hj);
-        ChanRule& cr = k_rule[kg][8 * c + j];
-        cr.g = make_group(lf, hf, L);
+        const int ch = 8 * c + j;
+        const GroupParams g = make_group(lf, hf, L);
+        kr.s[kg][ch] = g.s_bits;
+        kr.z[kg][ch] = g.z_bits;
         if constexpr (BITS == 2) {
-          const Thresh2 t = make_thresh2(cr.g);
+          const Thresh2 t = make_thresh2(g);
 #pragma unroll
-          for (int k = 0; k < 3; ++k) cr.t[k] = static_cast<uint16_t>(t.t[k]);
+          for (int k = 0; k < 3; ++k) kr.t[k][kg][ch] = static_cast<uint16_t>(t.t[k]);
+        } else {
+          kr.inv_s[kg][ch] = g.inv_s;
+          kr.zf[kg][ch] = g.zf;
         }
       }
     }
@@ -483,21 +493,29 @@ __device__ void quantize_k_fine_tiles(const uint16_t* __restrict__ src, int lg_g
   __syncthreads();
   if ((tg & (tpg - 1)) == 0) {       // the K group's first tile stores the pairs of its 8 channels
     const size_t row = static_cast<size_t>(tg >> (lg_gk - 3)) * kHeadDim + 8 * c;
-    uint32_t sw[4], zw[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const GroupParams &ga = k_rule[kg][8 * c + 2 * i].g, &gb = k_rule[kg][8 * c + 2 * i + 1].g;
-      sw[i] = static_cast<uint32_t>(ga.s_bits) | (static_cast<uint32_t>(gb.s_bits) << 16);
-      zw[i] = static_cast<uint32_t>(ga.z_bits) | (static_cast<uint32_t>(gb.z_bits) << 16);
-    }
-    *reinterpret_cast<uint4*>(scale + row) = make_uint4(sw[0], sw[1], sw[2], sw[3]);
-    *reinterpret_cast<uint4*>(zero + row) = make_uint4(zw[0], zw[1], zw[2], zw[3]);
+    *reinterpret_cast<uint4*>(scale + row) = *reinterpret_cast<const uint4*>(&kr.s[kg][8 * c]);
+    *reinterpret_cast<uint4*>(zero + row) = *reinterpret_cast<const uint4*>(&kr.z[kg][8 * c]);
   }
   const int tok0 = tg * kTileTokens;
   if constexpr (BITS == 4) {  // K word c of a token is exactly the tile's 8 channels
     GroupParams gp[8];
+    {
+      const uint4 sb = *reinterpret_cast<const uint4*>(&kr.s[kg][8 * c]);
+      const uint4 zb = *reinterpret_cast<const uint4*>(&kr.z[kg][8 * c]);
+      const float4 i0 = *reinterpret_cast<const float4*>(&kr.inv_s[BITS == 4 ? kg : 0][BITS == 4 ? 8 * c : 0]);
+      const float4 i1 = *reinterpret_cast<const float4*>(&kr.inv_s[BITS == 4 ? kg : 0][BITS == 4 ? 8 * c + 4 : 0]);
+      const float4 z0 = *reinterpret_cast<const float4*>(&kr.zf[BITS == 4 ? kg : 0][BITS == 4 ? 8 * c : 0]);
+      const float4 z1 = *reinterpret_cast<const float4*>(&kr.zf[BITS == 4 ? kg : 0][BITS == 4 ? 8 * c + 4 : 0]);
+      const float inv[8] = {i0.x, i0.y, i0.z, i0.w, i1.x, i1.y, i1.z, i1.w};
+      const float zfs[8] = {z0.x, z0.y, z0.z, z0.w, z1.x, z1.y, z1.z, z1.w};
 #pragma unroll
-    for (int j = 0; j < 8; ++j) gp[j] = k_rule[kg][8 * c + j].g;
+      for (int j = 0; j < 8; ++j) {
+        gp[j].inv_s = inv[j];
+        gp[j].zf = zfs[j];
+        gp[j].s_bits = static_cast<uint16_t>(comp4(sb, j >> 1) >> (16 * (j & 1)));
+        gp[j].z_bits = static_cast<uint16_t>(comp4(zb, j >> 1) >> (16 * (j & 1)));
+      }
+    }
 #pragma unroll
     for (int k = 0; k < kTileTokens; ++k) {
       const uint32_t w[4] = {x[k].x, x[k].y, x[k].z, x[k].w};
@@ -513,10 +531,10 @@ __device__ void quantize_k_fine_tiles(const uint16_t* __restrict__ src, int lg_g
   } else {  // K word c / 2 of a token: chunk 2i in bits 0..15, chunk 2i + 1 in bits 16..31
     Thresh2 tp[4];  // thresholds of channels 2 i (low half) and 2 i + 1 (high half)
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const ChanRule &ra = k_rule[kg][8 * c + 2 * i], &rb = k_rule[kg][8 * c + 2 * i + 1];
+    for (int k = 0; k < 3; ++k) {
+      const uint4 tw = *reinterpret_cast<const uint4*>(&kr.t[BITS == 2 ? k : 0][kg][BITS == 2 ? 8 * c : 0]);
 #pragma unroll
-      for (int k = 0; k < 3; ++k) tp[i].t[k] = static_cast<uint32_t>(ra.t[k]) | (static_cast<uint32_t>(rb.t[k]) << 16);
+      for (int i = 0; i < 4; ++i) tp[i].t[k] = comp4(tw, i);
     }
     uint32_t h[kTileTokens];
 #pragma unroll
