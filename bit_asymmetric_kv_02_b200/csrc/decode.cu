@@ -456,8 +456,9 @@ struct Flusher {
 };
 
 // KC: the residual tokens' K rows are codes (online K); a separate instantiation keeps that path
-// out of the register allocation of the others.  FG: fine-grained groups (2 bits, one query per KV
-// head): K (s, z) per channel per g_k tokens, V (s, z) per token per g_v channels.
+// out of the register allocation of the others.  FG: fine-grained groups (2 or 4 bits, one to
+// eight queries per KV head): K (s, z) per channel per g_k tokens, V (s, z) per token per g_v channels.
+// FL: the decode step's in-launch flush of a full residual (base groups only).
 template <int BITS, int G, bool KC, bool FG = false, bool FL = false>
 struct Decoder {
   static constexpr int P = 32 / BITS;              // codes per word

@@ -84,7 +84,7 @@ struct DecodeArgs {
   // online K: the residual tokens' K rows are code rows n_quant .. of k_codes with the (s, z) of
   // block res_blk (= n_quant / residual); 0: fp16 rows of k_res
   int k_res_coded, res_blk;
-  // fine-grained groups (2 bits, one query per KV head): k_scale / k_zero [bh][C >> lg_gk][128]
+  // fine-grained groups (2 or 4 bits, 1-8 queries per KV head): k_scale / k_zero [bh][C >> lg_gk][128]
   // (lg_gk: tokens per K group), v_scale / v_zero [bh][C][128 >> lg_gv] (lg_gv: channels per V group)
   int fine;
   // in-launch flush (decode step whose appended token fills the residual, base groups only): the R
