@@ -5,9 +5,6 @@ import math
 
 import numpy as np
 
-import oracle.kivi_oracle as O
-from bit_asymmetric_kv_02_b200 import synth
-
 ATOL = 2e-3        # max-abs bound on decode outputs, beyond the fp16 output's own rounding
 RTOL = 1e-2        # max-rel bound, relative to max(|o*|, REL_FLOOR)
 REL_FLOOR = 1e-2
@@ -37,22 +34,6 @@ def assert_attention_close(got, want, what=""):
     assert ea <= ATOL and er <= RTOL, (f"{what}: max abs beyond fp16 rounding {ea:.3e} (bar {ATOL}; raw {raw:.3e}), "
                                        f"max rel {er:.3e} (bar {RTOL})")
     return ea, er
-
-
-def oracle_head(w: synth.Workload, b: int, h: int, capacity: int, prompt_tokens: int):
-    """HeadCache of KV head (b, h) after prefill of `prompt_tokens` synthetic tokens."""
-    hc = O.HeadCache(w.head_dim, w.bits, w.group, w.gv, w.residual, capacity)
-    hc.prefill(synth.prompt_k(w, b, h, prompt_tokens), synth.prompt_v(w, b, h, prompt_tokens))
-    return hc
-
-
-def sample_heads(w: synth.Workload, n: int, seed: int = 0):
-    """First, last and n-2 seeded random (b, h) KV heads."""
-    rng = np.random.default_rng(seed)
-    heads = {(0, 0), (w.batch - 1, w.kv_heads - 1)}
-    while len(heads) < min(n, w.batch * w.kv_heads):
-        heads.add((int(rng.integers(w.batch)), int(rng.integers(w.kv_heads))))
-    return sorted(heads)
 
 
 def gpu_buffers_of_head(cache, b: int, h: int, n_quant: int, n_res: int):

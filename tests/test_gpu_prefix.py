@@ -6,7 +6,6 @@ follow the oracle (the flushed block takes its own block-local K groups).  Cases
 kernels (register tiles for R <= 512, two passes for R = 1024), 2 and 4 bits, G_k != G_v, GQA and a
 prompt that fits the residual.
 """
-import numpy as np
 import pytest
 
 import gpu_common as gc
