@@ -348,16 +348,21 @@ def test_full_size_all_heads(w):
     _compare("step 0", _gpu_head_digests(cache, heads, shapes), out, runs, w.gqa, w.name)
 
 
-def test_full_size_large_batch_fused_all_heads():
-    """The bench's workload and call (kivi_append_decode_attention) at full size on every head:
-    prefill, attention, a flush, then two fused append + decode steps; buffers bit for bit after
-    the prefill, after the flush and at the end, outputs within tolerance at every step."""
+def test_full_size_large_batch_step_all_heads():
+    """The bench's workload and call (kivi_decode_step) at full size on every head: prefill,
+    attention, then R decode steps.  Step 1 meets the prompt's full residual and flushes it in a
+    launch of its own; step 2 takes the fused append + decode call instead; the token of step R fills
+    the residual, and the step's one launch also quantizes it.  Buffers bit for bit after the
+    prefill, after step 1 and after the in-launch flush; outputs within tolerance at steps 0, 1, 2,
+    R - 1 and R."""
     kivi = _kivi()
     w = synth.LARGE_BATCH
-    T = w.tokens
-    cap = (T - 1) // w.residual * w.residual + w.residual
+    T, R = w.tokens, w.residual
+    cap = (T - 1) // R * R + 2 * R  # room for the prompt's residual block and one more
+    attend_at = frozenset({0, 1, 2, R - 1, R})
     heads = [(b, h) for b in range(w.batch) for h in range(w.kv_heads)]
-    specs = [ow.HeadStream(w, b, h, cap, T, steps=2, attend_at=frozenset({0, 1, 2}), digest_at=frozenset({0, 2}))
+    # the oracle runs one step further: its flush before step R + 1 is the GPU's flush inside step R
+    specs = [ow.HeadStream(w, b, h, cap, T, steps=R + 1, attend_at=attend_at, digest_at=frozenset({0, 1}))
              for b, h in heads]
     with ow.pool() as ex:
         fut = ex.map(ow.run_head, specs, chunksize=8)
@@ -367,21 +372,25 @@ def test_full_size_large_batch_fused_all_heads():
         cache.status.zero_()
         cache.prefill(torch.from_numpy(k).cuda(), torch.from_numpy(v).cuda())
         del k, v
+        assert cache.n_res == R
         outs = {0: cache.attend(torch.from_numpy(synth.queries(w, 0)).cuda()).cpu().numpy()}
         runs = dict(zip(heads, fut))
         gpu = {"step 0": _gpu_head_digests(cache, heads, _shapes(runs, "step 0"))}
-        for s in (1, 2):
-            if cache.n_res == w.residual:
-                cache.flush()
-                gpu[f"flush before step {s}"] = _gpu_head_digests(cache, heads, _shapes(runs, f"flush before step {s}"))
+        for s in range(1, R + 1):
             kn, vn = synth.new_kv(w, s)
-            q = synth.queries(w, s)
-            outs[s] = cache.append_attend(*(torch.from_numpy(x).cuda() for x in (kn, vn, q))).cpu().numpy()
-        gpu["step 2"] = _gpu_head_digests(cache, heads, _shapes(runs, "step 2"))
+            x = [torch.from_numpy(a).cuda() for a in (kn, vn, synth.queries(w, s))]
+            out = cache.append_attend(*x) if s == 2 else cache.step(*x)
+            if s in attend_at:
+                outs[s] = out.cpu().numpy()
+            if s == 1:
+                gpu["step 1"] = _gpu_head_digests(cache, heads, _shapes(runs, "step 1"))
+        assert (cache.n_quant, cache.n_res) == (cap, 0)
+        label = f"flush before step {R + 1}"
+        gpu[label] = _gpu_head_digests(cache, heads, _shapes(runs, label))
         assert cache.read_status() == 0
-    for label in ("step 0", "flush before step 1", "step 2"):
-        _compare(label, gpu[label], None, runs, w.gqa, w.name)
-    for s in (0, 1, 2):
+    for lab in ("step 0", "step 1", label):
+        _compare(lab, gpu[lab], None, runs, w.gqa, w.name)
+    for s in sorted(attend_at):
         _compare(f"step {s}", None, outs[s], runs, w.gqa, w.name)
 
 
