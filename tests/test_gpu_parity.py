@@ -324,39 +324,14 @@ def _shapes(oracle_runs, label):
     raise KeyError(label)
 
 
-@pytest.mark.parametrize("w", FULL, ids=[w.name for w in FULL])
-def test_full_size_all_heads(w):
-    """Full-size workloads in the bench's launch configuration: every KV head's codes, scales,
-    zero points and residual rows bit for bit, every query head's output within tolerance."""
-    kivi = _kivi()
-    T = w.tokens
-    cap = ((T + w.residual - 1) // w.residual) * w.residual
-    heads = [(b, h) for b in range(w.batch) for h in range(w.kv_heads)]
-    specs = [ow.HeadStream(w, b, h, cap, T, attend_at=frozenset({0}), digest_at=frozenset({0})) for b, h in heads]
-    with ow.pool() as ex:
-        fut = ex.map(ow.run_head, specs, chunksize=4)
-        k, v = synth.prompt_kv(w, T)
-        cache = kivi.KiviCache(w.batch, w.kv_heads, cap, bits=w.bits, group_k=w.group, group_v=w.gv,
-                               residual=w.residual, num_q_heads=w.q_heads)
-        cache.status.zero_()
-        cache.prefill(torch.from_numpy(k).cuda(), torch.from_numpy(v).cuda())
-        del k, v
-        out = cache.attend(torch.from_numpy(synth.queries(w, 0)).cuda()).cpu().numpy()
-        assert cache.read_status() == 0
-        runs = dict(zip(heads, fut))
-    shapes = _shapes(runs, "step 0")
-    _compare("step 0", _gpu_head_digests(cache, heads, shapes), out, runs, w.gqa, w.name)
-
-
-def test_full_size_large_batch_step_all_heads():
-    """The bench's workload and call (kivi_decode_step) at full size on every head: prefill,
+def _full_size_steps(w, chunksize):
+    """A full-size workload through the bench's call (kivi_decode_step) on every head: prefill,
     attention, then R decode steps.  Step 1 meets the prompt's full residual and flushes it in a
     launch of its own; step 2 takes the fused append + decode call instead; the token of step R fills
     the residual, and the step's one launch also quantizes it.  Buffers bit for bit after the
     prefill, after step 1 and after the in-launch flush; outputs within tolerance at steps 0, 1, 2,
     R - 1 and R."""
     kivi = _kivi()
-    w = synth.LARGE_BATCH
     T, R = w.tokens, w.residual
     cap = (T - 1) // R * R + 2 * R  # room for the prompt's residual block and one more
     attend_at = frozenset({0, 1, 2, R - 1, R})
@@ -365,7 +340,7 @@ def test_full_size_large_batch_step_all_heads():
     specs = [ow.HeadStream(w, b, h, cap, T, steps=R + 1, attend_at=attend_at, digest_at=frozenset({0, 1}))
              for b, h in heads]
     with ow.pool() as ex:
-        fut = ex.map(ow.run_head, specs, chunksize=8)
+        fut = ex.map(ow.run_head, specs, chunksize=chunksize)
         k, v = synth.prompt_kv(w, T)
         cache = kivi.KiviCache(w.batch, w.kv_heads, cap, bits=w.bits, group_k=w.group, group_v=w.gv,
                                residual=w.residual, num_q_heads=w.q_heads)
@@ -392,6 +367,18 @@ def test_full_size_large_batch_step_all_heads():
         _compare(lab, gpu[lab], None, runs, w.gqa, w.name)
     for s in sorted(attend_at):
         _compare(f"step {s}", None, outs[s], runs, w.gqa, w.name)
+
+
+@pytest.mark.parametrize("w", FULL, ids=[w.name for w in FULL])
+def test_full_size_all_heads(w):
+    """The Llama-2 layer and the GQA workload at full size through the decode step (see
+    _full_size_steps)."""
+    _full_size_steps(w, chunksize=4)
+
+
+def test_full_size_large_batch_step_all_heads():
+    """The large batch (2048 KV heads) at full size through the decode step (see _full_size_steps)."""
+    _full_size_steps(synth.LARGE_BATCH, chunksize=8)
 
 
 @pytest.mark.parametrize("bits,group", [(2, 32), (2, 128), (4, 32), (4, 128)])
