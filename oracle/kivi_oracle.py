@@ -327,25 +327,26 @@ class HeadCache:
         codes = quantize_values(rows, np.repeat(s, self.gk)[None, :], np.repeat(z, self.gk)[None, :], self.bits)
         self.k_codes = np.concatenate([self.k_codes, codes])
 
-    def _quantize_block(self, kblk, vblk):
+    def _block_parts(self, kblk, vblk):
+        """Codes, scales and zero points of one R-token block, rows ready to append."""
         if self.fine:
             kc, ks, kz = quantize_k_block_fine(kblk, self.gk, self.bits)
             vc, vs, vz = quantize_v_block_fine(vblk, self.gv, self.bits)
-            self.k_codes = np.concatenate([self.k_codes, kc])
-            self.v_codes = np.concatenate([self.v_codes, vc])
-            self.k_s = np.concatenate([self.k_s, ks])
-            self.k_z = np.concatenate([self.k_z, kz])
-            self.v_s = np.concatenate([self.v_s, vs])
-            self.v_z = np.concatenate([self.v_z, vz])
-            return
+            return kc, vc, ks, kz, vs, vz
         kc, ks, kz = quantize_k_block(kblk, self.gk, self.bits)
         vc, vs, vz = quantize_v_block(vblk, self.gv, self.bits)
-        self.k_codes = np.concatenate([self.k_codes, kc])
-        self.v_codes = np.concatenate([self.v_codes, vc])
-        self.k_s = np.concatenate([self.k_s, ks[None, :]])
-        self.k_z = np.concatenate([self.k_z, kz[None, :]])
-        self.v_s = np.concatenate([self.v_s, vs])
-        self.v_z = np.concatenate([self.v_z, vz])
+        return kc, vc, ks[None, :], kz[None, :], vs, vz
+
+    def _append_blocks(self, parts):
+        """Appends the blocks' rows to the quantized part (one concatenation per array)."""
+        if not parts:
+            return
+        names = ("k_codes", "v_codes", "k_s", "k_z", "v_s", "v_z")
+        for i, name in enumerate(names):
+            setattr(self, name, np.concatenate([getattr(self, name)] + [p[i] for p in parts]))
+
+    def _quantize_block(self, kblk, vblk):
+        self._append_blocks([self._block_parts(kblk, vblk)])
 
     def prefill(self, k, v):
         """Resets the head and caches a prompt: the newest ((T-1) mod R)+1 tokens stay fp16, the
@@ -361,9 +362,8 @@ class HeadCache:
         if n_quant > self.capacity:
             raise OracleError("CAPACITY", f"{n_quant} > {self.capacity}")
         self.__init__(self.d, self.bits, self.gk, self.gv, self.R, self.capacity, self.online_k, self.fine)
-        for j in range(n_quant // self.R):
-            sl = slice(j * self.R, (j + 1) * self.R)
-            self._quantize_block(k[sl], v[sl])
+        self._append_blocks([self._block_parts(k[j * self.R:(j + 1) * self.R], v[j * self.R:(j + 1) * self.R])
+                             for j in range(n_quant // self.R)])
         self.v_res = v[n_quant:].copy()
         if self.k_online:
             if n_quant + self.R > self.capacity:
