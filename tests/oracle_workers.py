@@ -93,10 +93,20 @@ def run_head(spec: HeadStream) -> list:
     return out
 
 
+def _one_thread_per_worker():
+    """The pool runs one process per core: each keeps its numpy linear algebra to one thread, so the
+    processes do not share the cores with each other's thread pools."""
+    try:
+        from threadpoolctl import threadpool_limits
+    except ImportError:
+        return
+    threadpool_limits(limits=1)
+
+
 def pool(workers: int | None = None) -> ProcessPoolExecutor:
     import multiprocessing as mp
     n = workers or max(1, min(32, os.cpu_count() or 1))
-    return ProcessPoolExecutor(n, mp_context=mp.get_context("spawn"))
+    return ProcessPoolExecutor(n, mp_context=mp.get_context("spawn"), initializer=_one_thread_per_worker)
 
 
 def run_heads(specs, workers: int | None = None) -> dict:
