@@ -95,12 +95,13 @@ def run_head(spec: HeadStream) -> list:
 
 def _one_thread_per_worker():
     """The pool runs one process per core: each keeps its numpy linear algebra to one thread, so the
-    processes do not share the cores with each other's thread pools."""
+    processes do not share the cores with each other's thread pools.  Only the speed depends on it:
+    where the limit cannot be set, the worker runs with the default threads."""
     try:
         from threadpoolctl import threadpool_limits
-    except ImportError:
-        return
-    threadpool_limits(limits=1)
+        threadpool_limits(limits=1)
+    except Exception:
+        pass
 
 
 def pool(workers: int | None = None) -> ProcessPoolExecutor:
