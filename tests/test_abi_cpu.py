@@ -72,6 +72,18 @@ def test_cache_sizes(kivi):
     assert s4[0] == bh * C * d // 2 and s4[2] == bh * (C // 128) * 2 and s4[4] == bh * (C // 128) * 2
 
 
+def test_cache_sizes_past_32_bits(kivi):
+    """Sizes are size_t all the way: 512 KV heads with room for 2^20 tokens need 2^32 code words (16 GiB)
+    per code array, and the largest capacity the prefill grid allows (32767 blocks) as well."""
+    sizes = kivi.kivi_cache_sizes(_cfg(kivi, batch=8, num_kv_heads=64, capacity=1 << 20))
+    assert sizes[0] == sizes[1] == (1 << 32) * 4
+    assert sizes[6] == 512 * 128 * 128 * 2
+    big = _cfg(kivi, batch=1024, num_kv_heads=64, capacity=32767 * 128)
+    assert kivi.kivi_check_config(big) == 0
+    assert kivi.kivi_cache_sizes(big)[0] == 1024 * 64 * 32767 * 128 * 32
+    assert kivi.kivi_check_config(_cfg(kivi, capacity=32768 * 128)) == 2  # the prefill grid's limit
+
+
 def test_state_errors_before_any_device_work(kivi):
     """Errors detected on the host return before anything is enqueued; fake (aligned, never
     dereferenced) pointers are enough to reach them."""
